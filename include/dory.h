@@ -1,0 +1,215 @@
+/*
+ * dory.h -- C ABI of the B200 (sm_100a) looped nGPT forward-pass library.
+ *
+ * What it computes.  The forward pass of a looped normalized-GPT stack as the
+ * Dory1.0-4B pages describe it:
+ *   - "Dory1.0-4B: A Looped Normalized-GPT" (ai.info AI summary), Key
+ *     Contributions item 1: an input block, a shared recurrent block applied k
+ *     times, an output block (effective depth 32 + 40k sublayers);
+ *     Methodology in Plain English: nGPT hypersphere residual updates
+ *     h <- Norm(h + alpha * (Norm(f(h)) - h)) with learned per-channel alpha,
+ *     GQA attention with sigmoid output gates interleaving sliding-window and
+ *     full layers (RoPE per layer type), L2 norm of the gated attention output
+ *     before the output projection and of the SwiGLU activations before the
+ *     down-projection, and re-injection of the input block's output before
+ *     every pass of the recurrent block;
+ *   - "Dory 1.0 4B Benchmarks: How Do 1, 2 and 4 Loops Compare?" (goremy.ai),
+ *     How does looping work at inference time?: k is chosen per request on the
+ *     same weights; per-loop KV caching keeps one cache per loop, last-loop
+ *     caching keeps one cache per recurrent attention layer that every loop
+ *     overwrites, so its footprint is the one-loop size for any k.
+ *
+ * Conventions.
+ *   - Every function returning int returns DORY_OK (0) or a negative
+ *     dory_status.  Nothing aborts the process.
+ *   - Memory is owned by the caller: the library never allocates device
+ *     memory.  It keeps host-side metadata (handles, CUDA graphs, tensor-map
+ *     descriptors) which dory_kv_free / dory_destroy release.
+ *   - `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *     legacy default stream).  Calls are asynchronous on that stream; outputs
+ *     are valid once it has been synchronised.
+ *   - Hidden states are bf16, row-major [rows, d_model].  Input rows are
+ *     expected to have unit L2 norm and are not re-normalised.
+ *   - Pointers named h_in / h_out may be device pointers or host pointers
+ *     (pinned host memory gives overlapped copies); host buffers are staged
+ *     through the workspace with cudaMemcpyAsync on `stream`.
+ *   - Device pointers passed in must be 256-byte aligned (DORY_ERR_MISALIGNED).
+ */
+#ifndef DORY_H
+#define DORY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DORY_API __attribute__((visibility("default")))
+#else
+#define DORY_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dory_status {
+  DORY_OK = 0,
+  DORY_ERR_INVALID_ARG = -1,      /* null pointer, negative size, bad index      */
+  DORY_ERR_BAD_CONFIG = -2,       /* unsupported shapes in dory_config            */
+  DORY_ERR_K_RANGE = -3,          /* k outside 1..4 (1..8 with allow_extrapolated_k) */
+  DORY_ERR_K_EXCEEDS_KMAX = -4,   /* per-loop cache allocated for fewer loops     */
+  DORY_ERR_CTX_OVERFLOW = -5,     /* positions beyond the cache's max_ctx         */
+  DORY_ERR_BUFFER_TOO_SMALL = -6, /* weight / kv / workspace buffer too small     */
+  DORY_ERR_MISALIGNED = -7,       /* a device buffer is not 256-byte aligned      */
+  DORY_ERR_CUDA = -8,             /* a CUDA runtime/driver call failed            */
+  DORY_ERR_DEVICE_TIMEOUT = -9,   /* a kernel's bounded wait expired (device word) */
+  DORY_ERR_UNSUPPORTED_ARCH = -10,/* device is not sm_100                         */
+  DORY_ERR_DEVICE_BOUNDS = -11    /* a kernel's bounds check fired (device word)   */
+} dory_status;
+
+typedef enum dory_kv_mode {
+  DORY_KV_PER_LOOP = 0,   /* recurrent layers keep one cache per loop (k_max of them) */
+  DORY_KV_LAST_LOOP = 1   /* one cache per layer; each loop overwrites the last        */
+} dory_kv_mode;
+
+/* Model shape.  Global block b (0-based over in+rec+out blocks) uses full
+ * attention iff b % full_period == full_period - 1, otherwise a sliding window
+ * of `window` keys ending at (and including) the query position.
+ * Supported: head_dim 64 or 128; d_model == n_q_heads * head_dim;
+ * n_q_heads % n_kv_heads == 0 with a group of at most 4; d_model and d_ff
+ * multiples of 128; window >= 1. */
+typedef struct dory_config {
+  int32_t d_model;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t d_ff;
+  int32_t n_in_blocks;
+  int32_t n_rec_blocks;
+  int32_t n_out_blocks;
+  int32_t window;
+  int32_t full_period;
+  double rope_base_swa;     /* RoPE base of sliding-window layers          */
+  double rope_base_full;    /* RoPE base of full-attention layers          */
+  float softmax_scale;      /* logit = softmax_scale * q_hat . k_hat       */
+  float gate_scale;         /* SwiGLU: SiLU(gate_scale * h Wg^T) * (h Wu^T) */
+  float norm_eps;           /* Norm(x) = x / sqrt(max(sum x^2, norm_eps))  */
+  int32_t allow_extrapolated_k; /* nonzero: accept k up to 8               */
+} dory_config;
+
+/* Source tensors of one block, row-major [out, in] bf16 matrices (as
+ * uint16_t bit patterns) and fp32 vectors.  Host or device pointers. */
+typedef struct dory_block_src {
+  const uint16_t* wq;      /* [n_q_heads*head_dim, d_model]  */
+  const uint16_t* wk;      /* [n_kv_heads*head_dim, d_model] */
+  const uint16_t* wv;      /* [n_kv_heads*head_dim, d_model] */
+  const uint16_t* wg;      /* [n_q_heads, d_model]  attention output gates */
+  const uint16_t* wo;      /* [d_model, n_q_heads*head_dim] */
+  const uint16_t* w_gate;  /* [d_ff, d_model]  */
+  const uint16_t* w_up;    /* [d_ff, d_model]  */
+  const uint16_t* w_down;  /* [d_model, d_ff]  */
+  const float* alpha_attn; /* [d_model] */
+  const float* alpha_mlp;  /* [d_model] */
+  const float* s_qk;       /* [head_dim] */
+} dory_block_src;
+
+typedef struct dory_model dory_model;
+typedef struct dory_kv dory_kv;
+
+/* Bytes of the device buffer dory_create packs the weights into
+ * (weights in the kernels' layout plus a small device status area). */
+DORY_API size_t dory_weight_bytes(const dory_config* cfg);
+
+/* Validate `cfg`, check that the current device is sm_100, and pack the
+ * weights of all blocks (`src[b]` for global block b) into `weight_buf`
+ * (device, caller-owned, at least dory_weight_bytes, 256-byte aligned).
+ * The copies are ordered on `stream`.  On success *out is a new handle. */
+DORY_API int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
+                const dory_block_src* src, int n_src, void* stream, dory_model** out);
+
+/* Bytes of a KV cache: pure arithmetic, no allocation.  Per attention layer
+ * (and per loop for recurrent layers under DORY_KV_PER_LOOP with `k_max`
+ * loops) and per sequence: K and V, n_kv_heads * head_dim bf16 each, for
+ * min(window, max_ctx) positions (sliding-window layers) or max_ctx
+ * positions (full layers).  Under DORY_KV_LAST_LOOP the result does not
+ * depend on k_max.  Returns 0 for invalid arguments. */
+DORY_API size_t dory_kv_bytes(const dory_config* cfg, int mode, int max_seqs, int max_ctx, int k_max);
+
+/* Bind a KV cache of `mode` to `kv_buf` (device, caller-owned,
+ * >= dory_kv_bytes).  The contents are not touched. */
+DORY_API int dory_kv_alloc(dory_model* m, int mode, int max_seqs, int max_ctx, int k_max,
+                  void* kv_buf, size_t kv_bytes, dory_kv** out);
+
+/* Byte offsets from kv_buf of the K and V entries of (global block `layer`,
+ * loop `loop` (1-based; ignored unless the layer is recurrent and the mode is
+ * per-loop), sequence `seq`, position `pos`, KV head `head`).  Each entry is
+ * head_dim contiguous bf16.  Sliding-window layers are rings of
+ * min(window, max_ctx) slots (slot = pos % capacity); full layers use slot = pos.
+ * Within one (layer, loop, seq, head) the slots are contiguous (stride
+ * head_dim * 2 bytes). */
+DORY_API int dory_kv_layout(const dory_kv* kv, int layer, int loop, int seq, int pos, int head,
+                   size_t* k_off, size_t* v_off);
+
+/* Workspace bytes for calls of up to `max_tokens` rows (prefill tokens or
+ * decode batch), 256-byte aligned base required. */
+DORY_API size_t dory_workspace_bytes(const dory_model* m, int max_tokens);
+
+/* Prefill `n_tokens` tokens of sequence `seq` at positions pos0 .. pos0+n-1
+ * with k recurrent loops.  Chunked prefill is repeated calls with increasing
+ * pos0; positions before pos0 must already be in the cache.  Under last-loop
+ * caching the call's tokens at loop j attend to earlier positions' cached
+ * entries and to this call's own loop-j keys; after the call the cache holds
+ * loop k's entries.  h_in, h_out: [n_tokens, d_model] bf16 (host or device). */
+DORY_API int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens,
+                 const void* h_in, void* h_out, int k,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step for `batch` sequences: row i is sequence d_seq[i] at
+ * position d_pos[i] (int32 device arrays, so a captured step replays across
+ * steps).  Every row's positions before d_pos[i] must be cached.  h_in,
+ * h_out: [batch, d_model] bf16 (host or device).  `max_pos_hint` is an upper
+ * bound on every d_pos[i] (it sizes the split-KV grid; positions above it are
+ * reported as DORY_ERR_DEVICE_BOUNDS by dory_device_status). */
+DORY_API int dory_decode_step(dory_model* m, dory_kv* kv, int batch,
+                     const int32_t* d_seq, const int32_t* d_pos, int max_pos_hint,
+                     const void* h_in, void* h_out, int k,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the model's device status word:
+ * DORY_OK, DORY_ERR_DEVICE_TIMEOUT or DORY_ERR_DEVICE_BOUNDS. */
+DORY_API int dory_device_status(dory_model* m, void* stream);
+
+/* Kernel launches of the most recent dory_prefill / dory_decode_step, and how
+ * many nGPT sublayer updates it applied (32 + 40k for the Dory shape). */
+DORY_API int dory_last_call_stats(const dory_model* m, int* kernel_launches, int* sublayer_updates);
+
+DORY_API const char* dory_error_string(int status);
+
+DORY_API void dory_kv_free(dory_kv* kv);
+DORY_API void dory_destroy(dory_model* m);
+
+/* ---------------------------------------------------------------------
+ * Single-sublayer entry points (diagnostics and per-sublayer parity).
+ * They run exactly the kernels the full pass runs for one sublayer of
+ * global block `layer` at loop `loop`, on `n_rows` rows.
+ * --------------------------------------------------------------------- */
+
+/* Attention sublayer on rows h [n_rows, d_model] (fp32, device, updated in
+ * place) of sequence `seq` at positions pos0.. (prefill semantics, the
+ * call's keys committed to the cache after attention). */
+DORY_API int dory_attention_sublayer(dory_model* m, dory_kv* kv, int layer, int loop, int seq,
+                            int pos0, int n_rows, float* h, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* SwiGLU sublayer on rows h [n_rows, d_model] (fp32, device, in place). */
+DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* The tensor-core GEMM alone: C[M,N] (fp32) = A[M,K] (bf16) * B[N,K]^T (bf16),
+ * all row-major device buffers, K a multiple of 64, N a multiple of 128. */
+DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DORY_H */

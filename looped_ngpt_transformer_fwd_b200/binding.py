@@ -1,0 +1,199 @@
+"""ctypes binding of libdory.so (the C ABI in include/dory.h).
+
+Argument marshalling only: every step of the forward pass runs in the
+library's sm_100a kernels.  PyTorch supplies device memory and streams.  If the
+shared library has not been built, importing `lib()` raises ImportError; there
+is no fallback implementation.
+"""
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libdory.so")
+
+DORY_OK = 0
+DORY_KV_PER_LOOP = 0
+DORY_KV_LAST_LOOP = 1
+MODES = {"per_loop": DORY_KV_PER_LOOP, "last_loop": DORY_KV_LAST_LOOP}
+
+STATUS = {
+    0: "DORY_OK", -1: "DORY_ERR_INVALID_ARG", -2: "DORY_ERR_BAD_CONFIG", -3: "DORY_ERR_K_RANGE",
+    -4: "DORY_ERR_K_EXCEEDS_KMAX", -5: "DORY_ERR_CTX_OVERFLOW", -6: "DORY_ERR_BUFFER_TOO_SMALL",
+    -7: "DORY_ERR_MISALIGNED", -8: "DORY_ERR_CUDA", -9: "DORY_ERR_DEVICE_TIMEOUT",
+    -10: "DORY_ERR_UNSUPPORTED_ARCH", -11: "DORY_ERR_DEVICE_BOUNDS",
+}
+
+# every entry point declared in include/dory.h
+EXPORTS = (
+    "dory_weight_bytes", "dory_create", "dory_kv_bytes", "dory_kv_alloc", "dory_kv_layout",
+    "dory_workspace_bytes", "dory_prefill", "dory_decode_step", "dory_device_status",
+    "dory_last_call_stats", "dory_error_string", "dory_kv_free", "dory_destroy",
+    "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
+)
+
+
+class DoryError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_errstr(status)})")
+
+
+class DoryConfig(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("d_ff", ctypes.c_int32), ("n_in_blocks", ctypes.c_int32),
+        ("n_rec_blocks", ctypes.c_int32), ("n_out_blocks", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("full_period", ctypes.c_int32),
+        ("rope_base_swa", ctypes.c_double), ("rope_base_full", ctypes.c_double),
+        ("softmax_scale", ctypes.c_float), ("gate_scale", ctypes.c_float),
+        ("norm_eps", ctypes.c_float), ("allow_extrapolated_k", ctypes.c_int32),
+    ]
+
+
+class DoryBlockSrc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down",
+        "alpha_attn", "alpha_mlp", "s_qk")]
+
+
+_LIB = None
+P = ctypes.c_void_p
+I = ctypes.c_int
+SZ = ctypes.c_size_t
+
+
+def lib():
+    """The loaded libdory.so (ImportError when it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "looped_ngpt_transformer_fwd_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "dory_weight_bytes": (SZ, [P]),
+            "dory_create": (I, [P, P, SZ, P, I, P, P]),
+            "dory_kv_bytes": (SZ, [P, I, I, I, I]),
+            "dory_kv_alloc": (I, [P, I, I, I, I, P, SZ, P]),
+            "dory_kv_layout": (I, [P, I, I, I, I, I, P, P]),
+            "dory_workspace_bytes": (SZ, [P, I]),
+            "dory_prefill": (I, [P, P, I, I, I, P, P, I, P, SZ, P]),
+            "dory_decode_step": (I, [P, P, I, P, P, I, P, P, I, P, SZ, P]),
+            "dory_device_status": (I, [P, P]),
+            "dory_last_call_stats": (I, [P, P, P]),
+            "dory_error_string": (ctypes.c_char_p, [I]),
+            "dory_kv_free": (None, [P]),
+            "dory_destroy": (None, [P]),
+            "dory_attention_sublayer": (I, [P, P, I, I, I, I, I, P, P, SZ, P]),
+            "dory_mlp_sublayer": (I, [P, I, I, P, P, SZ, P]),
+            "dory_gemm_bf16": (I, [P, P, P, I, I, I, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _errstr(status):
+    try:
+        return lib().dory_error_string(status).decode()
+    except ImportError:
+        return "?"
+
+
+def check(status, where):
+    if status != DORY_OK:
+        raise DoryError(status, where)
+    return status
+
+
+def make_config(cfg, allow_extrapolated_k=False):
+    """dory_config from a config dict (configs/*.json)."""
+    return DoryConfig(
+        cfg["d_model"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"], cfg["d_ff"],
+        cfg["n_in_blocks"], cfg["n_rec_blocks"], cfg["n_out_blocks"], cfg["window"],
+        cfg["full_period"], float(cfg["rope_base_swa"]), float(cfg["rope_base_full"]),
+        float(cfg["softmax_scale"]), float(cfg["gate_scale"]), float(cfg["norm_eps"]),
+        1 if allow_extrapolated_k else 0)
+
+
+# ----------------------------------------------------------------- thin wrappers
+def dory_weight_bytes(cfg_struct):
+    return lib().dory_weight_bytes(ctypes.byref(cfg_struct))
+
+
+def dory_kv_bytes(cfg_struct, mode, max_seqs, max_ctx, k_max):
+    return lib().dory_kv_bytes(ctypes.byref(cfg_struct), MODES.get(mode, mode), max_seqs, max_ctx, k_max)
+
+
+def dory_create(cfg_struct, weight_ptr, weight_bytes, srcs, stream):
+    arr = (DoryBlockSrc * len(srcs))(*srcs)
+    out = ctypes.c_void_p()
+    check(lib().dory_create(ctypes.byref(cfg_struct), weight_ptr, weight_bytes, arr, len(srcs),
+                            stream, ctypes.byref(out)), "dory_create")
+    return out.value
+
+
+def dory_kv_alloc(model, mode, max_seqs, max_ctx, k_max, kv_ptr, kv_bytes):
+    out = ctypes.c_void_p()
+    check(lib().dory_kv_alloc(model, MODES.get(mode, mode), max_seqs, max_ctx, k_max, kv_ptr,
+                              kv_bytes, ctypes.byref(out)), "dory_kv_alloc")
+    return out.value
+
+
+def dory_kv_layout(kv, layer, loop, seq, pos, head):
+    k_off, v_off = ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().dory_kv_layout(kv, layer, loop, seq, pos, head, ctypes.byref(k_off),
+                               ctypes.byref(v_off)), "dory_kv_layout")
+    return k_off.value, v_off.value
+
+
+def dory_workspace_bytes(model, max_tokens):
+    return lib().dory_workspace_bytes(model, max_tokens)
+
+
+def dory_prefill(model, kv, seq, pos0, n_tokens, h_in, h_out, k, ws, ws_bytes, stream):
+    return check(lib().dory_prefill(model, kv, seq, pos0, n_tokens, h_in, h_out, k, ws, ws_bytes,
+                                    stream), "dory_prefill")
+
+
+def dory_decode_step(model, kv, batch, d_seq, d_pos, max_pos_hint, h_in, h_out, k, ws, ws_bytes,
+                     stream):
+    return check(lib().dory_decode_step(model, kv, batch, d_seq, d_pos, max_pos_hint, h_in, h_out,
+                                        k, ws, ws_bytes, stream), "dory_decode_step")
+
+
+def dory_device_status(model, stream):
+    return lib().dory_device_status(model, stream)
+
+
+def dory_last_call_stats(model):
+    a, b = ctypes.c_int(), ctypes.c_int()
+    check(lib().dory_last_call_stats(model, ctypes.byref(a), ctypes.byref(b)), "dory_last_call_stats")
+    return a.value, b.value
+
+
+def dory_attention_sublayer(model, kv, layer, loop, seq, pos0, n_rows, h, ws, ws_bytes, stream):
+    return check(lib().dory_attention_sublayer(model, kv, layer, loop, seq, pos0, n_rows, h, ws,
+                                               ws_bytes, stream), "dory_attention_sublayer")
+
+
+def dory_mlp_sublayer(model, layer, n_rows, h, ws, ws_bytes, stream):
+    return check(lib().dory_mlp_sublayer(model, layer, n_rows, h, ws, ws_bytes, stream),
+                 "dory_mlp_sublayer")
+
+
+def dory_gemm_bf16(A, B, C, M, N, K, stream):
+    return check(lib().dory_gemm_bf16(A, B, C, M, N, K, stream), "dory_gemm_bf16")
+
+
+def dory_kv_free(kv):
+    lib().dory_kv_free(kv)
+
+
+def dory_destroy(model):
+    lib().dory_destroy(model)

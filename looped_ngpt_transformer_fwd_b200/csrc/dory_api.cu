@@ -1,0 +1,798 @@
+// C ABI of the looped nGPT forward-pass library: model and KV-cache handles,
+// weight packing, workspace layout, and the loop controller that runs
+//   input block (once) -> recurrent block (k times, re-injecting the input
+//   block's output before every pass) -> output block (once)
+// ("Dory1.0-4B: A Looped Normalized-GPT", Key Contributions item 1 and
+// Methodology in Plain English; "Dory 1.0 4B Benchmarks: How Do 1, 2 and 4
+// Loops Compare?", How does looping work at inference time?) as one CUDA graph
+// per call shape.  The recurrent blocks' weights are the same device pointers
+// in every loop: re-read, never copied.  KV caches follow the per-loop (one
+// cache per loop of a recurrent layer) or last-loop (one cache per layer,
+// overwritten by every loop) mode of the same passages.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <memory>
+#include <new>
+#include <tuple>
+#include <vector>
+
+#include "../../include/dory.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace dory;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDecodeRows = 256;     // decode batch limit of a workspace
+constexpr int kMaxDecodeSplits = 64;    // split-KV slices per (sequence, head)
+constexpr int kMaxKSplits = 8;
+
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+bool is_aligned(const void* p, size_t a = kAlign) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+struct BlockW {
+  __nv_bfloat16* wqkvg = nullptr;   // [n_qkvg, d]: q | k | v | gate rows
+  __nv_bfloat16* wo = nullptr;      // [d, Hq*hd]
+  __nv_bfloat16* wgu = nullptr;     // [2*ff, d]: 128 gate rows, 128 up rows, ...
+  __nv_bfloat16* wd = nullptr;      // [d, ff]
+  float* alpha_attn = nullptr;
+  float* alpha_mlp = nullptr;
+  float* s_qk = nullptr;
+  bool full = false;
+  bool recurrent = false;
+  // B-operand tensor maps, box rows 128 and 256
+  CUtensorMap tm_qkvg[2], tm_o[2], tm_gu, tm_d[2];
+};
+
+struct GraphKey {
+  int phase, k, n, seq, pos0, max_pos;
+  const void *src, *dst, *ws, *kv, *dseq, *dpos;
+  bool operator<(const GraphKey& o) const {
+    return std::tie(phase, k, n, seq, pos0, max_pos, src, dst, ws, kv, dseq, dpos) <
+           std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.src, o.dst, o.ws, o.kv, o.dseq,
+                    o.dpos);
+  }
+};
+
+struct GraphEntry {
+  cudaGraphExec_t exec = nullptr;
+  int launches = 0, sublayers = 0;
+  uint64_t last_use = 0;
+};
+
+}  // namespace
+
+struct dory_model {
+  dory_config cfg;
+  int d, hq, hkv, hd, ff, d_attn, n_qkvg, nb;
+  int device = 0, num_sms = 148;
+  uint8_t* wbuf = nullptr;
+  size_t wbytes = 0;
+  uint32_t* status = nullptr;
+  double* inv_freq_swa = nullptr;
+  double* inv_freq_full = nullptr;
+  std::vector<BlockW> blocks;
+  cudaStream_t cap_stream = nullptr;
+  std::map<GraphKey, GraphEntry> graphs;
+  uint64_t tick = 0;
+  int last_launches = 0, last_sublayers = 0;
+  // counters of the call being enqueued
+  int cur_launches = 0, cur_sublayers = 0;
+};
+
+struct dory_kv {
+  dory_model* m = nullptr;
+  int mode = 0, max_seqs = 0, max_ctx = 0, k_max = 1;
+  uint8_t* buf = nullptr;
+  size_t bytes = 0;
+  // per block: first slot's byte offset, capacity, number of loop slots
+  std::vector<size_t> base;
+  std::vector<int> cap, loops;
+  std::vector<int> seq_k;   // per sequence: k of its last prefill (per-loop mode checks)
+};
+
+namespace {
+
+// ------------------------------------------------------------------ layouts
+int n_blocks(const dory_config* c) { return c->n_in_blocks + c->n_rec_blocks + c->n_out_blocks; }
+
+bool is_full(const dory_config* c, int b) { return (b % c->full_period) == c->full_period - 1; }
+
+bool is_recurrent(const dory_config* c, int b) {
+  return b >= c->n_in_blocks && b < c->n_in_blocks + c->n_rec_blocks;
+}
+
+int validate_config(const dory_config* c) {
+  if (!c) return DORY_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return DORY_ERR_BAD_CONFIG;
+  if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads) return DORY_ERR_BAD_CONFIG;
+  if (c->n_q_heads / c->n_kv_heads > 4) return DORY_ERR_BAD_CONFIG;
+  if (c->d_model != c->n_q_heads * c->head_dim) return DORY_ERR_BAD_CONFIG;
+  if (c->d_model % 128 || c->d_ff % 128 || c->d_model > 4096 || c->d_model < 128) return DORY_ERR_BAD_CONFIG;
+  if (c->n_in_blocks < 1 || c->n_rec_blocks < 1 || c->n_out_blocks < 1) return DORY_ERR_BAD_CONFIG;
+  if (c->window < 1 || c->full_period < 1) return DORY_ERR_BAD_CONFIG;
+  if (!(c->rope_base_swa > 1.0) || !(c->rope_base_full > 1.0)) return DORY_ERR_BAD_CONFIG;
+  if (!(c->softmax_scale > 0.f) || !(c->norm_eps > 0.f)) return DORY_ERR_BAD_CONFIG;
+  return DORY_OK;
+}
+
+struct WeightLayout {
+  size_t header = 0;                 // status word + RoPE tables
+  size_t per_block = 0;
+  size_t off_qkvg = 0, off_o = 0, off_gu = 0, off_d = 0, off_aa = 0, off_am = 0, off_sqk = 0;
+  size_t total = 0;
+};
+
+WeightLayout weight_layout(const dory_config* c) {
+  WeightLayout L;
+  const size_t d = c->d_model, hd = c->head_dim, da = size_t(c->n_q_heads) * hd, ff = c->d_ff;
+  const size_t nq = da + 2 * size_t(c->n_kv_heads) * hd + c->n_q_heads;
+  L.header = align_up(64) + 2 * align_up(hd / 2 * sizeof(double));
+  size_t o = 0;
+  L.off_qkvg = o; o = align_up(o + nq * d * 2);
+  L.off_o = o;    o = align_up(o + d * da * 2);
+  L.off_gu = o;   o = align_up(o + 2 * ff * d * 2);
+  L.off_d = o;    o = align_up(o + d * ff * 2);
+  L.off_aa = o;   o = align_up(o + d * 4);
+  L.off_am = o;   o = align_up(o + d * 4);
+  L.off_sqk = o;  o = align_up(o + hd * 4);
+  L.per_block = o;
+  L.total = L.header + L.per_block * n_blocks(c);
+  return L;
+}
+
+struct WsLayout {
+  size_t h32, e32, hb, st_in, st_out, q, kf, vf, gate, o, y, a, dacc, dml, total;
+  int y_rows;
+};
+
+WsLayout ws_layout(const dory_model* m, int T) {
+  WsLayout L;
+  const size_t d = m->d, da = m->d_attn, kvw = size_t(m->hkv) * m->hd, ff = m->ff;
+  const int dec_rows = std::min(T, kMaxDecodeRows);
+  L.y_rows = std::max(T, kMaxKSplits * dec_rows);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.h32 = take(size_t(T) * d * 4);
+  L.e32 = take(size_t(T) * d * 4);
+  L.hb = take(size_t(T) * d * 2);
+  L.st_in = take(size_t(T) * d * 2);
+  L.st_out = take(size_t(T) * d * 2);
+  L.q = take(size_t(T) * da * 2);
+  L.kf = take(size_t(T) * kvw * 2);
+  L.vf = take(size_t(T) * kvw * 2);
+  L.gate = take(size_t(T) * m->hq * 4);
+  L.o = take(size_t(T) * da * 2);
+  L.y = take(size_t(L.y_rows) * d * 4);
+  L.a = take(size_t(T) * ff * 2);
+  L.dacc = take(size_t(dec_rows) * m->hq * kMaxDecodeSplits * m->hd * 4);
+  L.dml = take(size_t(dec_rows) * m->hq * kMaxDecodeSplits * 2 * 4);
+  L.total = o;
+  return L;
+}
+
+struct Ws {
+  float *h32, *e32, *y, *gate, *dacc, *dml;
+  __nv_bfloat16 *hb, *st_in, *st_out, *q, *kf, *vf, *o, *a;
+};
+
+Ws ws_bind(const dory_model* m, void* base, int T) {
+  const WsLayout L = ws_layout(m, T);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Ws w;
+  w.h32 = reinterpret_cast<float*>(b + L.h32);
+  w.e32 = reinterpret_cast<float*>(b + L.e32);
+  w.hb = reinterpret_cast<__nv_bfloat16*>(b + L.hb);
+  w.st_in = reinterpret_cast<__nv_bfloat16*>(b + L.st_in);
+  w.st_out = reinterpret_cast<__nv_bfloat16*>(b + L.st_out);
+  w.q = reinterpret_cast<__nv_bfloat16*>(b + L.q);
+  w.kf = reinterpret_cast<__nv_bfloat16*>(b + L.kf);
+  w.vf = reinterpret_cast<__nv_bfloat16*>(b + L.vf);
+  w.gate = reinterpret_cast<float*>(b + L.gate);
+  w.o = reinterpret_cast<__nv_bfloat16*>(b + L.o);
+  w.y = reinterpret_cast<float*>(b + L.y);
+  w.a = reinterpret_cast<__nv_bfloat16*>(b + L.a);
+  w.dacc = reinterpret_cast<float*>(b + L.dacc);
+  w.dml = reinterpret_cast<float*>(b + L.dml);
+  return w;
+}
+
+KvLayerView kv_view(const dory_kv* kv, int b, int loop) {
+  const dory_model* m = kv->m;
+  KvLayerView v;
+  const int slot = (kv->loops[b] > 1) ? (loop - 1) : 0;
+  const size_t cap = kv->cap[b];
+  const size_t seq_elems = 2 * size_t(m->hkv) * cap * m->hd;
+  uint8_t* base = kv->buf + kv->base[b] + size_t(slot) * kv->max_seqs * seq_elems * 2;
+  v.k_base = reinterpret_cast<__nv_bfloat16*>(base);
+  v.v_base = v.k_base + size_t(m->hkv) * cap * m->hd;
+  v.seq_stride = seq_elems;
+  v.cap = kv->cap[b];
+  v.n_kv = m->hkv;
+  v.hd = m->hd;
+  v.max_seqs = kv->max_seqs;
+  v.max_ctx = kv->max_ctx;
+  return v;
+}
+
+// ------------------------------------------------------------------ kernels of one block
+struct CallCtx {
+  dory_model* m;
+  dory_kv* kv;
+  Ws w;
+  int n;                 // rows
+  bool decode;
+  int seq, pos0;         // prefill
+  const int32_t *dseq, *dpos;
+  int max_pos;
+  int k;
+  cudaStream_t s;
+};
+
+#define DORY_TRY(expr)                         \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return _e;          \
+  } while (0)
+
+int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
+  const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
+  if (tiles >= m->num_sms / 2) return 1;
+  int s = std::max(1, m->num_sms / tiles);
+  s = std::min(s, kMaxKSplits);
+  s = std::min(s, std::max(1, (K / 64) / 4));
+  // the kernel gives each split ceil(kb / s) k-blocks: drop splits left empty
+  const int kb = K / 64, per = (kb + s - 1) / s;
+  return (kb + per - 1) / per;
+}
+
+cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloat16* hb,
+                               bool commit_after) {
+  dory_model* m = c.m;
+  const BlockW& W = m->blocks[b];
+  const int bn_q = c.decode ? 128 : 256;
+  CUtensorMap tmA;
+  if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
+  GemmParams g;
+  g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
+  g.epi = kEpiQKVG;
+  g.q_out = c.w.q; g.k_out = c.w.kf; g.v_out = c.w.vf; g.gate_out = c.w.gate;
+  g.n_q_heads = m->hq; g.n_kv_heads = m->hkv;
+  g.s_qk = W.s_qk;
+  g.inv_freq = W.full ? m->inv_freq_full : m->inv_freq_swa;
+  g.norm_eps = m->cfg.norm_eps;
+  g.pos0 = c.decode ? 0 : c.pos0;
+  g.d_pos = c.decode ? c.dpos : nullptr;
+  g.status = m->status;
+  DORY_TRY(launch_gemm(tmA, W.tm_qkvg[bn_q == 256], g, bn_q, m->hd, m->num_sms, c.s));
+  ++c.m->cur_launches;
+
+  const KvLayerView view = kv_view(c.kv, b, loop);
+  const int window = W.full ? 0 : m->cfg.window;
+  const float scale_log2 = m->cfg.softmax_scale * 1.4426950408889634f;
+  if (c.decode) {
+    DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s));
+    DecodeAttnParams a;
+    a.q = c.w.q; a.gate = c.w.gate; a.out = c.w.o; a.kv = view;
+    a.d_seq = c.dseq; a.d_pos = c.dpos;
+    a.batch = c.n; a.n_q_heads = m->hq; a.window = window; a.max_pos = c.max_pos;
+    const int max_keys = window > 0 ? std::min(c.max_pos + 1, window) : c.max_pos + 1;
+    int sk = (max_keys + kMaxDecodeSplits - 1) / kMaxDecodeSplits;
+    sk = std::max(512, (sk + 63) / 64 * 64);
+    a.split_keys = sk;
+    a.scale_log2 = scale_log2;
+    a.part_acc = c.w.dacc; a.part_ml = c.w.dml;
+    a.status = m->status;
+    DORY_TRY(launch_decode_attention(a, c.s));
+    c.m->cur_launches += 3;
+  } else {
+    PrefillAttnParams a;
+    a.q = c.w.q; a.k_new = c.w.kf; a.v_new = c.w.vf; a.gate = c.w.gate; a.out = c.w.o;
+    a.kv = view; a.seq = c.seq; a.pos0 = c.pos0; a.n = c.n; a.n_q_heads = m->hq;
+    a.window = window; a.scale_log2 = scale_log2; a.status = m->status;
+    DORY_TRY(launch_prefill_attention(a, c.s));
+    ++c.m->cur_launches;
+    if (commit_after) {
+      const int first = W.full ? 0 : std::max(0, c.n - view.cap);
+      DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, first, c.seq, c.pos0, nullptr, nullptr,
+                                m->status, c.s));
+      ++c.m->cur_launches;
+    }
+  }
+
+  // output projection, then the nGPT update of the stream
+  CUtensorMap tmO;
+  if (!make_tmap_bf16(&tmO, c.w.o, c.n, m->d_attn, 128)) return cudaErrorInvalidValue;
+  const int bn_o = c.decode ? 128 : 256;
+  GemmParams go;
+  go.M = c.n; go.N = m->d; go.K = m->d_attn;
+  go.epi = kEpiStoreF32;
+  go.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_o, m->d_attn) : 1;
+  go.out_f32 = c.w.y; go.ld_out = m->d; go.split_stride = size_t(c.n) * m->d;
+  go.status = m->status;
+  DORY_TRY(launch_gemm(tmO, W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms, c.s));
+  ++c.m->cur_launches;
+
+  RowUpdateParams r;
+  r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = go.k_splits; r.split_stride = go.split_stride;
+  r.h = h; r.hb = hb; r.alpha = W.alpha_attn; r.norm_eps = m->cfg.norm_eps;
+  DORY_TRY(launch_row_update(r, c.s));
+  ++c.m->cur_launches;
+  ++c.m->cur_sublayers;
+  return cudaSuccess;
+}
+
+// `reinject`: after the update, x <- Norm(x + e); `save_e`: store the update
+// result as e first; `out`: also write the result as bf16 there.
+cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool save_e,
+                         bool reinject, __nv_bfloat16* out) {
+  dory_model* m = c.m;
+  const BlockW& W = m->blocks[b];
+  CUtensorMap tmA;
+  if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
+  GemmParams g;
+  g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
+  g.epi = kEpiSwiGLU;
+  g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
+  g.status = m->status;
+  DORY_TRY(launch_gemm(tmA, W.tm_gu, g, 256, m->hd, m->num_sms, c.s));
+  ++c.m->cur_launches;
+
+  CUtensorMap tmAct;
+  if (!make_tmap_bf16(&tmAct, c.w.a, c.n, m->ff, 128)) return cudaErrorInvalidValue;
+  const int bn_d = c.decode ? 128 : 256;
+  GemmParams gd;
+  gd.M = c.n; gd.N = m->d; gd.K = m->ff;
+  gd.epi = kEpiStoreF32;
+  gd.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_d, m->ff) : 1;
+  gd.out_f32 = c.w.y; gd.ld_out = m->d; gd.split_stride = size_t(c.n) * m->d;
+  gd.status = m->status;
+  DORY_TRY(launch_gemm(tmAct, W.tm_d[bn_d == 256], gd, bn_d, m->hd, m->num_sms, c.s));
+  ++c.m->cur_launches;
+
+  RowUpdateParams r;
+  r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = gd.k_splits; r.split_stride = gd.split_stride;
+  r.h = h; r.hb = hb; r.alpha = W.alpha_mlp; r.norm_eps = m->cfg.norm_eps;
+  r.e_save = save_e ? c.w.e32 : nullptr;
+  r.e = reinject ? c.w.e32 : nullptr;
+  r.out = out;
+  DORY_TRY(launch_row_update(r, c.s));
+  ++c.m->cur_launches;
+  ++c.m->cur_sublayers;
+  return cudaSuccess;
+}
+
+// The whole stack for one call, enqueued on c.s.
+cudaError_t enqueue_stack(CallCtx& c, const __nv_bfloat16* src, __nv_bfloat16* dst) {
+  dory_model* m = c.m;
+  const dory_config* cfg = &m->cfg;
+  const int n_in = cfg->n_in_blocks, n_rec = cfg->n_rec_blocks, nb = m->nb;
+  DORY_TRY(launch_load_rows(src, c.w.h32, c.w.hb, c.n, m->d, c.s));
+  ++m->cur_launches;
+  const bool last_loop = c.kv->mode == DORY_KV_LAST_LOOP;
+  for (int b = 0; b < n_in; ++b) {
+    DORY_TRY(attention_sublayer(c, b, 1, c.w.h32, c.w.hb, true));
+    const bool last = b == n_in - 1;
+    // the input block's output e is saved and re-injected before loop 1
+    DORY_TRY(mlp_sublayer(c, b, c.w.h32, c.w.hb, last, last, nullptr));
+  }
+  for (int j = 1; j <= c.k; ++j) {
+    for (int b = n_in; b < n_in + n_rec; ++b) {
+      // last-loop caching: this call's keys reach the cache after the final loop only
+      const bool commit = !last_loop || j == c.k;
+      DORY_TRY(attention_sublayer(c, b, j, c.w.h32, c.w.hb, commit));
+      const bool reinject = (b == n_in + n_rec - 1) && j < c.k;
+      DORY_TRY(mlp_sublayer(c, b, c.w.h32, c.w.hb, false, reinject, nullptr));
+    }
+  }
+  for (int b = n_in + n_rec; b < nb; ++b) {
+    DORY_TRY(attention_sublayer(c, b, 1, c.w.h32, c.w.hb, true));
+    DORY_TRY(mlp_sublayer(c, b, c.w.h32, c.w.hb, false, false, b == nb - 1 ? dst : nullptr));
+  }
+  return cudaSuccess;
+}
+
+// Capture (or reuse) the graph for this call and launch it on `stream`.
+int run_graph(dory_model* m, const GraphKey& key, CallCtx& c, const __nv_bfloat16* src,
+              __nv_bfloat16* dst, cudaStream_t stream) {
+  auto it = m->graphs.find(key);
+  if (it == m->graphs.end()) {
+    if (m->graphs.size() >= 16) {   // evict the least recently used graph
+      auto lru = m->graphs.begin();
+      for (auto g = m->graphs.begin(); g != m->graphs.end(); ++g)
+        if (g->second.last_use < lru->second.last_use) lru = g;
+      cudaGraphExecDestroy(lru->second.exec);
+      m->graphs.erase(lru);
+    }
+    m->cur_launches = 0;
+    m->cur_sublayers = 0;
+    c.s = m->cap_stream;
+    if (cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+      return DORY_ERR_CUDA;
+    cudaError_t e = enqueue_stack(c, src, dst);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &graph);
+    if (e != cudaSuccess || e2 != cudaSuccess || !graph) {
+      if (graph) cudaGraphDestroy(graph);
+      cudaGetLastError();
+      return DORY_ERR_CUDA;
+    }
+    GraphEntry ent;
+    e = cudaGraphInstantiate(&ent.exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return DORY_ERR_CUDA;
+    ent.launches = m->cur_launches;
+    ent.sublayers = m->cur_sublayers;
+    it = m->graphs.emplace(key, ent).first;
+  }
+  it->second.last_use = ++m->tick;
+  if (cudaGraphLaunch(it->second.exec, stream) != cudaSuccess) return DORY_ERR_CUDA;
+  m->last_launches = it->second.launches;
+  m->last_sublayers = it->second.sublayers;
+  return DORY_OK;
+}
+
+int check_k(const dory_model* m, const dory_kv* kv, int k) {
+  const int kmax = m->cfg.allow_extrapolated_k ? 8 : 4;
+  if (k < 1 || k > kmax) return DORY_ERR_K_RANGE;
+  if (kv->mode == DORY_KV_PER_LOOP && k > kv->k_max) return DORY_ERR_K_EXCEEDS_KMAX;
+  return DORY_OK;
+}
+
+void fill_inv_freq(std::vector<double>& v, double base, int hd) {
+  v.resize(hd / 2);
+  for (int i = 0; i < hd / 2; ++i) v[i] = pow(base, -2.0 * i / hd);
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+extern "C" {
+
+const char* dory_error_string(int status) {
+  switch (status) {
+    case DORY_OK: return "ok";
+    case DORY_ERR_INVALID_ARG: return "invalid argument";
+    case DORY_ERR_BAD_CONFIG: return "unsupported model configuration";
+    case DORY_ERR_K_RANGE: return "loop count k out of range";
+    case DORY_ERR_K_EXCEEDS_KMAX: return "k exceeds the per-loop cache's k_max";
+    case DORY_ERR_CTX_OVERFLOW: return "positions exceed the cache's max_ctx";
+    case DORY_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    case DORY_ERR_MISALIGNED: return "device buffer not 256-byte aligned";
+    case DORY_ERR_CUDA: return "CUDA call failed";
+    case DORY_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    case DORY_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
+    case DORY_ERR_DEVICE_BOUNDS: return "a kernel's bounds check fired";
+    default: return "unknown status";
+  }
+}
+
+size_t dory_weight_bytes(const dory_config* cfg) {
+  if (validate_config(cfg) != DORY_OK) return 0;
+  return weight_layout(cfg).total;
+}
+
+int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
+                const dory_block_src* src, int n_src, void* stream, dory_model** out) {
+  if (!out || !weight_buf || !src) return DORY_ERR_INVALID_ARG;
+  *out = nullptr;
+  int st = validate_config(cfg);
+  if (st != DORY_OK) return st;
+  if (n_src != n_blocks(cfg)) return DORY_ERR_INVALID_ARG;
+  const WeightLayout L = weight_layout(cfg);
+  if (weight_bytes < L.total) return DORY_ERR_BUFFER_TOO_SMALL;
+  if (!is_aligned(weight_buf)) return DORY_ERR_MISALIGNED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DORY_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DORY_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return DORY_ERR_UNSUPPORTED_ARCH;
+  for (int b = 0; b < n_src; ++b) {
+    const dory_block_src& s = src[b];
+    if (!s.wq || !s.wk || !s.wv || !s.wg || !s.wo || !s.w_gate || !s.w_up || !s.w_down ||
+        !s.alpha_attn || !s.alpha_mlp || !s.s_qk)
+      return DORY_ERR_INVALID_ARG;
+  }
+
+  std::unique_ptr<dory_model> m(new (std::nothrow) dory_model());
+  if (!m) return DORY_ERR_INVALID_ARG;
+  m->cfg = *cfg;
+  m->d = cfg->d_model; m->hq = cfg->n_q_heads; m->hkv = cfg->n_kv_heads; m->hd = cfg->head_dim;
+  m->ff = cfg->d_ff; m->d_attn = m->hq * m->hd;
+  m->n_qkvg = m->d_attn + 2 * m->hkv * m->hd + m->hq;
+  m->nb = n_blocks(cfg);
+  m->device = dev;
+  m->num_sms = prop.multiProcessorCount;
+  m->wbuf = static_cast<uint8_t*>(weight_buf);
+  m->wbytes = weight_bytes;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  uint8_t* hdr = m->wbuf;
+  m->status = reinterpret_cast<uint32_t*>(hdr);
+  m->inv_freq_swa = reinterpret_cast<double*>(hdr + align_up(64));
+  m->inv_freq_full = reinterpret_cast<double*>(hdr + align_up(64) + align_up(m->hd / 2 * sizeof(double)));
+  static thread_local std::vector<double> fs, ff;
+  fill_inv_freq(fs, cfg->rope_base_swa, m->hd);
+  fill_inv_freq(ff, cfg->rope_base_full, m->hd);
+  if (cudaMemsetAsync(m->status, 0, 64, s) != cudaSuccess ||
+      cudaMemcpyAsync(m->inv_freq_swa, fs.data(), fs.size() * sizeof(double), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(m->inv_freq_full, ff.data(), ff.size() * sizeof(double), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+
+  const size_t d = m->d, hd = m->hd, da = m->d_attn, F = m->ff;
+  m->blocks.resize(m->nb);
+  for (int b = 0; b < m->nb; ++b) {
+    BlockW& W = m->blocks[b];
+    uint8_t* base = m->wbuf + L.header + L.per_block * b;
+    W.wqkvg = reinterpret_cast<__nv_bfloat16*>(base + L.off_qkvg);
+    W.wo = reinterpret_cast<__nv_bfloat16*>(base + L.off_o);
+    W.wgu = reinterpret_cast<__nv_bfloat16*>(base + L.off_gu);
+    W.wd = reinterpret_cast<__nv_bfloat16*>(base + L.off_d);
+    W.alpha_attn = reinterpret_cast<float*>(base + L.off_aa);
+    W.alpha_mlp = reinterpret_cast<float*>(base + L.off_am);
+    W.s_qk = reinterpret_cast<float*>(base + L.off_sqk);
+    W.full = is_full(cfg, b);
+    W.recurrent = is_recurrent(cfg, b);
+    const dory_block_src& S = src[b];
+    const size_t kvr = size_t(m->hkv) * hd;
+    cudaError_t e = cudaSuccess;
+    uint8_t* q = reinterpret_cast<uint8_t*>(W.wqkvg);
+    e = e ? e : cudaMemcpyAsync(q, S.wq, da * d * 2, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(q + da * d * 2, S.wk, kvr * d * 2, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(q + (da + kvr) * d * 2, S.wv, kvr * d * 2, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(q + (da + 2 * kvr) * d * 2, S.wg, size_t(m->hq) * d * 2, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(W.wo, S.wo, d * da * 2, cudaMemcpyDefault, s);
+    // gate/up interleaved in groups of 128 rows (the SwiGLU epilogue's tile halves)
+    for (size_t t = 0; t < F / 128 && e == cudaSuccess; ++t) {
+      uint8_t* g = reinterpret_cast<uint8_t*>(W.wgu) + (2 * t) * 128 * d * 2;
+      e = cudaMemcpyAsync(g, reinterpret_cast<const uint8_t*>(S.w_gate) + t * 128 * d * 2,
+                          128 * d * 2, cudaMemcpyDefault, s);
+      e = e ? e : cudaMemcpyAsync(g + 128 * d * 2, reinterpret_cast<const uint8_t*>(S.w_up) + t * 128 * d * 2,
+                                  128 * d * 2, cudaMemcpyDefault, s);
+    }
+    e = e ? e : cudaMemcpyAsync(W.wd, S.w_down, d * F * 2, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(W.alpha_attn, S.alpha_attn, d * 4, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(W.alpha_mlp, S.alpha_mlp, d * 4, cudaMemcpyDefault, s);
+    e = e ? e : cudaMemcpyAsync(W.s_qk, S.s_qk, hd * 4, cudaMemcpyDefault, s);
+    if (e != cudaSuccess) return DORY_ERR_CUDA;
+    bool ok = true;
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t box = i ? 256 : 128;
+      ok &= make_tmap_bf16(&W.tm_qkvg[i], W.wqkvg, m->n_qkvg, d, box);
+      ok &= make_tmap_bf16(&W.tm_o[i], W.wo, d, da, box);
+      ok &= make_tmap_bf16(&W.tm_d[i], W.wd, d, F, box);
+    }
+    ok &= make_tmap_bf16(&W.tm_gu, W.wgu, 2 * F, d, 256);
+    if (!ok) return DORY_ERR_CUDA;
+  }
+  if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  *out = m.release();
+  return DORY_OK;
+}
+
+size_t dory_kv_bytes(const dory_config* cfg, int mode, int max_seqs, int max_ctx, int k_max) {
+  if (validate_config(cfg) != DORY_OK || max_seqs <= 0 || max_ctx <= 0 || k_max < 1) return 0;
+  if (mode != DORY_KV_PER_LOOP && mode != DORY_KV_LAST_LOOP) return 0;
+  const size_t per_pos = 2 * size_t(cfg->n_kv_heads) * cfg->head_dim * 2;
+  size_t total = 0;
+  for (int b = 0; b < n_blocks(cfg); ++b) {
+    const size_t loops = (mode == DORY_KV_PER_LOOP && is_recurrent(cfg, b)) ? k_max : 1;
+    const size_t cap = is_full(cfg, b) ? size_t(max_ctx) : std::min<size_t>(cfg->window, max_ctx);
+    total += loops * size_t(max_seqs) * cap * per_pos;
+  }
+  return total;
+}
+
+int dory_kv_alloc(dory_model* m, int mode, int max_seqs, int max_ctx, int k_max, void* kv_buf,
+                  size_t kv_bytes, dory_kv** out) {
+  if (!m || !kv_buf || !out || max_seqs <= 0 || max_ctx <= 0 || k_max < 1) return DORY_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (mode != DORY_KV_PER_LOOP && mode != DORY_KV_LAST_LOOP) return DORY_ERR_INVALID_ARG;
+  if (k_max > (m->cfg.allow_extrapolated_k ? 8 : 4)) return DORY_ERR_K_RANGE;
+  if (!is_aligned(kv_buf)) return DORY_ERR_MISALIGNED;
+  const size_t need = dory_kv_bytes(&m->cfg, mode, max_seqs, max_ctx, k_max);
+  if (kv_bytes < need) return DORY_ERR_BUFFER_TOO_SMALL;
+  std::unique_ptr<dory_kv> kv(new (std::nothrow) dory_kv());
+  if (!kv) return DORY_ERR_INVALID_ARG;
+  kv->m = m; kv->mode = mode; kv->max_seqs = max_seqs; kv->max_ctx = max_ctx; kv->k_max = k_max;
+  kv->buf = static_cast<uint8_t*>(kv_buf); kv->bytes = kv_bytes;
+  size_t off = 0;
+  const size_t per_pos = 2 * size_t(m->hkv) * m->hd * 2;
+  for (int b = 0; b < m->nb; ++b) {
+    const int loops = (mode == DORY_KV_PER_LOOP && m->blocks[b].recurrent) ? k_max : 1;
+    const int cap = m->blocks[b].full ? max_ctx : std::min(m->cfg.window, max_ctx);
+    kv->base.push_back(off);
+    kv->cap.push_back(cap);
+    kv->loops.push_back(loops);
+    off += size_t(loops) * max_seqs * cap * per_pos;
+  }
+  kv->seq_k.assign(max_seqs, 0);
+  *out = kv.release();
+  return DORY_OK;
+}
+
+int dory_kv_layout(const dory_kv* kv, int layer, int loop, int seq, int pos, int head,
+                   size_t* k_off, size_t* v_off) {
+  if (!kv || !k_off || !v_off) return DORY_ERR_INVALID_ARG;
+  const dory_model* m = kv->m;
+  if (layer < 0 || layer >= m->nb || seq < 0 || seq >= kv->max_seqs || head < 0 || head >= m->hkv)
+    return DORY_ERR_INVALID_ARG;
+  if (pos < 0 || pos >= kv->max_ctx) return DORY_ERR_CTX_OVERFLOW;
+  if (kv->loops[layer] > 1 && (loop < 1 || loop > kv->loops[layer])) return DORY_ERR_INVALID_ARG;
+  const KvLayerView v = kv_view(kv, layer, kv->loops[layer] > 1 ? loop : 1);
+  const size_t elem = (size_t(seq) * v.seq_stride + (size_t(head) * v.cap + pos % v.cap) * v.hd);
+  *k_off = reinterpret_cast<const uint8_t*>(v.k_base + elem) - kv->buf;
+  *v_off = reinterpret_cast<const uint8_t*>(v.v_base + elem) - kv->buf;
+  return DORY_OK;
+}
+
+size_t dory_workspace_bytes(const dory_model* m, int max_tokens) {
+  if (!m || max_tokens <= 0) return 0;
+  return ws_layout(m, max_tokens).total;
+}
+
+int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, const void* h_in,
+                 void* h_out, int k, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !kv || kv->m != m || !h_in || !h_out || !ws || n_tokens <= 0 || pos0 < 0)
+    return DORY_ERR_INVALID_ARG;
+  if (seq < 0 || seq >= kv->max_seqs) return DORY_ERR_INVALID_ARG;
+  int st = check_k(m, kv, k);
+  if (st != DORY_OK) return st;
+  if (size_t(pos0) + n_tokens > size_t(kv->max_ctx)) return DORY_ERR_CTX_OVERFLOW;
+  if (!is_aligned(ws)) return DORY_ERR_MISALIGNED;
+  if (ws_bytes < ws_layout(m, n_tokens).total) return DORY_ERR_BUFFER_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool in_dev = is_device_ptr(h_in), out_dev = is_device_ptr(h_out);
+  if ((in_dev && !is_aligned(h_in, 16)) || (out_dev && !is_aligned(h_out, 16))) return DORY_ERR_MISALIGNED;
+  CallCtx c;
+  c.m = m; c.kv = kv; c.w = ws_bind(m, ws, n_tokens); c.n = n_tokens; c.decode = false;
+  c.seq = seq; c.pos0 = pos0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = pos0 + n_tokens - 1;
+  c.k = k; c.s = s;
+  const size_t bytes = size_t(n_tokens) * m->d * 2;
+  const __nv_bfloat16* src = in_dev ? static_cast<const __nv_bfloat16*>(h_in) : c.w.st_in;
+  __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
+  if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  GraphKey key{0, k, n_tokens, seq, pos0, 0, src, dst, ws, kv, nullptr, nullptr};
+  st = run_graph(m, key, c, src, dst, s);
+  if (st != DORY_OK) return st;
+  if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  kv->seq_k[seq] = k;
+  return DORY_OK;
+}
+
+int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq,
+                     const int32_t* d_pos, int max_pos_hint, const void* h_in, void* h_out, int k,
+                     void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !kv || kv->m != m || !d_seq || !d_pos || !h_in || !h_out || !ws || batch <= 0)
+    return DORY_ERR_INVALID_ARG;
+  if (batch > kMaxDecodeRows) return DORY_ERR_INVALID_ARG;
+  int st = check_k(m, kv, k);
+  if (st != DORY_OK) return st;
+  if (max_pos_hint < 0) return DORY_ERR_INVALID_ARG;
+  if (max_pos_hint >= kv->max_ctx) return DORY_ERR_CTX_OVERFLOW;
+  if (!is_aligned(ws)) return DORY_ERR_MISALIGNED;
+  if (ws_bytes < ws_layout(m, batch).total) return DORY_ERR_BUFFER_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool in_dev = is_device_ptr(h_in), out_dev = is_device_ptr(h_out);
+  CallCtx c;
+  c.m = m; c.kv = kv; c.w = ws_bind(m, ws, batch); c.n = batch; c.decode = true;
+  c.seq = 0; c.pos0 = 0; c.dseq = d_seq; c.dpos = d_pos; c.max_pos = max_pos_hint;
+  c.k = k; c.s = s;
+  const size_t bytes = size_t(batch) * m->d * 2;
+  const __nv_bfloat16* src = in_dev ? static_cast<const __nv_bfloat16*>(h_in) : c.w.st_in;
+  __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
+  if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  GraphKey key{1, k, batch, 0, 0, max_pos_hint, src, dst, ws, kv, d_seq, d_pos};
+  st = run_graph(m, key, c, src, dst, s);
+  if (st != DORY_OK) return st;
+  if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_device_status(dory_model* m, void* stream) {
+  if (!m) return DORY_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, m->status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  if (word) {
+    if (cudaMemsetAsync(m->status, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+      return DORY_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) return DORY_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusBounds) return DORY_ERR_DEVICE_BOUNDS;
+  return DORY_OK;
+}
+
+int dory_last_call_stats(const dory_model* m, int* kernel_launches, int* sublayer_updates) {
+  if (!m) return DORY_ERR_INVALID_ARG;
+  if (kernel_launches) *kernel_launches = m->last_launches;
+  if (sublayer_updates) *sublayer_updates = m->last_sublayers;
+  return DORY_OK;
+}
+
+void dory_kv_free(dory_kv* kv) { delete kv; }
+
+void dory_destroy(dory_model* m) {
+  if (!m) return;
+  for (auto& g : m->graphs) cudaGraphExecDestroy(g.second.exec);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  delete m;
+}
+
+int dory_attention_sublayer(dory_model* m, dory_kv* kv, int layer, int loop, int seq, int pos0,
+                            int n_rows, float* h, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !kv || kv->m != m || !h || !ws || n_rows <= 0 || pos0 < 0) return DORY_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= m->nb || seq < 0 || seq >= kv->max_seqs) return DORY_ERR_INVALID_ARG;
+  if (kv->loops[layer] > 1 && (loop < 1 || loop > kv->loops[layer])) return DORY_ERR_INVALID_ARG;
+  if (size_t(pos0) + n_rows > size_t(kv->max_ctx)) return DORY_ERR_CTX_OVERFLOW;
+  if (!is_aligned(ws) || !is_aligned(h, 16)) return DORY_ERR_MISALIGNED;
+  if (ws_bytes < ws_layout(m, n_rows).total) return DORY_ERR_BUFFER_TOO_SMALL;
+  CallCtx c;
+  c.m = m; c.kv = kv; c.w = ws_bind(m, ws, n_rows); c.n = n_rows; c.decode = false;
+  c.seq = seq; c.pos0 = pos0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = pos0 + n_rows - 1;
+  c.k = 1; c.s = static_cast<cudaStream_t>(stream);
+  m->cur_launches = m->cur_sublayers = 0;
+  if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
+  if (attention_sublayer(c, layer, kv->loops[layer] > 1 ? loop : 1, h, c.w.hb, true) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h, void* ws, size_t ws_bytes,
+                      void* stream) {
+  if (!m || !h || !ws || n_rows <= 0 || layer < 0 || layer >= m->nb) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(ws) || !is_aligned(h, 16)) return DORY_ERR_MISALIGNED;
+  if (ws_bytes < ws_layout(m, n_rows).total) return DORY_ERR_BUFFER_TOO_SMALL;
+  CallCtx c;
+  c.m = m; c.kv = nullptr; c.w = ws_bind(m, ws, n_rows); c.n = n_rows; c.decode = false;
+  c.seq = 0; c.pos0 = 0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = 0; c.k = 1;
+  c.s = static_cast<cudaStream_t>(stream);
+  m->cur_launches = m->cur_sublayers = 0;
+  if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
+  if (mlp_sublayer(c, layer, h, c.w.hb, false, false, nullptr) != cudaSuccess) return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || K % 64 || N % 128) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return DORY_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, A, M, K, 128) || !make_tmap_bf16(&tb, B, N, K, BN)) return DORY_ERR_CUDA;
+  GemmParams p;
+  p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  if (launch_gemm(ta, tb, p, BN, 128, sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+}  // extern "C"

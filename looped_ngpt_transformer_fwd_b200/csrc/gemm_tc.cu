@@ -1,0 +1,428 @@
+// Persistent tcgen05 GEMM for sm_100a: C = A * B^T with bf16 operands fed by
+// TMA (128-byte swizzle), fp32 accumulators in TMEM (double-buffered so the
+// epilogue of one tile overlaps the main loop of the next), and fused
+// epilogues for the projections of a looped nGPT block:
+//   - kEpiQKVG: the fused QKV + gate projection of the attention sublayer
+//     ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain English:
+//     GQA with sigmoid output gates, RoPE per layer type), with the nGPT
+//     query/key normalisation q_hat = s_qk * Norm(RoPE(q)) per head;
+//   - kEpiSwiGLU: the gate/up projection with SiLU(gate) * up (same section);
+//   - kEpiStoreF32: plain fp32 output (output and down projections, whose
+//     nGPT update needs whole-row norms and runs in the row kernel).
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues the MMAs, warps 2..5 run the epilogue (one TMEM lane = one output row
+// per thread).  Every wait is bounded (see common.cuh); on expiry the kernel
+// records kStatusTimeout, drains its outstanding copies and MMAs, frees TMEM
+// and returns.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dory {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+};
+
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+// --------------------------------------------------------------- epilogues
+__device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32], int valid) {
+  if (valid >= 32) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    for (int i = 0; i < valid; ++i) dst[i] = v[i];
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t taddr, int row, int nt,
+                                              int ks) {
+  float* out = p.out_f32 + static_cast<size_t>(ks) * p.split_stride;
+  const bool row_ok = row < p.M;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float v[32];
+    tmem_ld32(taddr + c, v);
+    const int col = nt * BN + c;
+    if (row_ok && col < p.N)
+      store_f32_chunk(out + static_cast<size_t>(row) * p.ld_out + col, v, p.N - col);
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, int row, int nt) {
+  constexpr int H = BN / 2;
+  const bool row_ok = row < p.M;
+  __nv_bfloat16* out = p.out_act + static_cast<size_t>(row) * p.ld_act + nt * H;
+#pragma unroll 1
+  for (int c = 0; c < H; c += 32) {
+    float g[32], u[32];
+    tmem_ld32(taddr + c, g);
+    tmem_ld32(taddr + H + c, u);
+    if (!row_ok) continue;
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float g0 = p.gate_scale * g[2 * i], g1 = p.gate_scale * g[2 * i + 1];
+      const float a0 = g0 * sigmoidf_(g0) * u[2 * i];
+      const float a1 = g1 * sigmoidf_(g1) * u[2 * i + 1];
+      packed[i] = pack_bf16x2(a0, a1);
+    }
+    uint4* d4 = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  }
+}
+
+// One head-sized column group (HD columns starting at global column col0).
+template <int HD>
+__device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t taddr, int row,
+                                               int col0) {
+  const int hq = p.n_q_heads, hkv = p.n_kv_heads;
+  const int q_end = hq * HD, k_end = q_end + hkv * HD, v_end = k_end + hkv * HD;
+  float x[HD];
+#pragma unroll
+  for (int c = 0; c < HD; c += 32) {
+    float t[32];
+    tmem_ld32(taddr + c, t);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[c + i] = t[i];
+  }
+  if (row >= p.M) return;
+  if (col0 >= v_end) {
+    // attention output gate logits, one per query head
+    float* g = p.gate_out + static_cast<size_t>(row) * hq;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) {
+      const int j = col0 - v_end + i;
+      if (j < hq) g[j] = sigmoidf_(x[i]);
+    }
+    return;
+  }
+  __nv_bfloat16* dst;
+  if (col0 < k_end) {
+    // RoPE (pairs i, i + HD/2) at this row's absolute position, then the
+    // per-head L2 norm and the learned per-dimension scale s_qk.
+    const int pos = p.d_pos ? p.d_pos[row] : p.pos0 + row;
+    const double dpos = static_cast<double>(pos);
+#pragma unroll
+    for (int i = 0; i < HD / 2; ++i) {
+      const double ang = dpos * p.inv_freq[i];
+      const double turns = rint(ang * (1.0 / kTwoPi));
+      const float r = static_cast<float>(fma(-turns, kTwoPi, ang));
+      float sn, cs;
+      sincosf(r, &sn, &cs);
+      const float a = x[i], b = x[i + HD / 2];
+      x[i] = a * cs - b * sn;
+      x[i + HD / 2] = b * cs + a * sn;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) ss = fmaf(x[i], x[i], ss);
+    const float inv = rsqrtf(fmaxf(ss, p.norm_eps));
+#pragma unroll
+    for (int i = 0; i < HD; ++i) x[i] *= inv * p.s_qk[i];
+    dst = (col0 < q_end)
+              ? p.q_out + (static_cast<size_t>(row) * hq + col0 / HD) * HD
+              : p.k_out + (static_cast<size_t>(row) * hkv + (col0 - q_end) / HD) * HD;
+  } else {
+    dst = p.v_out + (static_cast<size_t>(row) * hkv + (col0 - k_end) / HD) * HD;
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) {
+    d4[i] = make_uint4(pack_bf16x2(x[8 * i], x[8 * i + 1]), pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
+                       pack_bf16x2(x[8 * i + 4], x[8 * i + 5]),
+                       pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
+  }
+}
+
+// A wait used only while cleaning up after an abort: short, ignores the flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) return;   // 0.2 s
+  }
+}
+
+template <int BN, int HD, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+  using C = GemmCfg<BN>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (p.M + kBM - 1) / kBM;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int kb_total = p.K / kBK;
+  const int kb_per_split = (kb_total + p.k_splits - 1) / p.k_splits;
+  const int total = m_tiles * n_tiles * p.k_splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int mt = t % m_tiles;
+        const int rest = t / m_tiles;
+        const int nt = rest % n_tiles;
+        const int ks = rest / n_tiles;
+        const int kb0 = ks * kb_per_split;
+        const int kb1 = min(kb_total, kb0 + kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = tiles + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * kBK, mt * kBM);
+          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * kBK, nt * BN);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy this thread started land before the CTA exits
+        for (int s = 0; s < S; ++s)
+          if (issued_mask & (1u << s)) drain_wait(&full[s], (issued_parity >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const int rest = t / m_tiles;
+        const int ks = rest / n_tiles;
+        const int kb0 = ks * kb_per_split;
+        const int kb1 = min(kb_total, kb0 + kb_per_split);
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
+                      idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      if (!ok && issued) {
+        umma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else {
+    // ---------------------------------------------------- epilogue warps
+    const int quad = warp & 3;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const int mt = t % m_tiles;
+      const int rest = t / m_tiles;
+      const int nt = rest % n_tiles;
+      const int ks = rest / n_tiles;
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int row = mt * kBM + quad * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      if constexpr (EPI == kEpiStoreF32) {
+        epi_store_f32<BN>(p, taddr, row, nt, ks);
+      } else if constexpr (EPI == kEpiSwiGLU) {
+        epi_swiglu<BN>(p, taddr, row, nt);
+      } else {
+#pragma unroll 1
+        for (int g = 0; g < BN / HD; ++g) epi_qkvg_group<HD>(p, taddr + g * HD, row, nt * BN + g * HD);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int BN, int HD, int EPI>
+cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                        int num_sms, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, HD, EPI>;
+  static uint32_t attr_done = 0;   // one bit per device ordinal < 32
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 32 || !(attr_done & (1u << dev))) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 32) attr_done |= 1u << dev;
+  }
+  const int m_tiles = (p.M + kBM - 1) / kBM;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int total = m_tiles * n_tiles * p.k_splits;
+  const int grid = total < num_sms ? total : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<EncodeFn>(fn);
+  }
+  if ((cols * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                        int BN, int head_dim, int num_sms, cudaStream_t s) {
+  if (p.K % kBK != 0 || p.K <= 0 || p.k_splits < 1) return cudaErrorInvalidValue;
+  {
+    // every K split must own at least one k-block
+    const int kb = p.K / kBK, per = (kb + p.k_splits - 1) / p.k_splits;
+    if ((p.k_splits - 1) * per >= kb) return cudaErrorInvalidValue;
+  }
+  if (BN == 256) {
+    switch (p.epi) {
+      case kEpiStoreF32: return launch_impl<256, 128, kEpiStoreF32>(tmA, tmB, p, num_sms, s);
+      case kEpiSwiGLU: return launch_impl<256, 128, kEpiSwiGLU>(tmA, tmB, p, num_sms, s);
+      case kEpiQKVG:
+        if (p.k_splits != 1) return cudaErrorInvalidValue;
+        if (head_dim == 128) return launch_impl<256, 128, kEpiQKVG>(tmA, tmB, p, num_sms, s);
+        if (head_dim == 64) return launch_impl<256, 64, kEpiQKVG>(tmA, tmB, p, num_sms, s);
+        return cudaErrorInvalidValue;
+    }
+  } else if (BN == 128) {
+    switch (p.epi) {
+      case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32>(tmA, tmB, p, num_sms, s);
+      case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU>(tmA, tmB, p, num_sms, s);
+      case kEpiQKVG:
+        if (p.k_splits != 1) return cudaErrorInvalidValue;
+        if (head_dim == 128) return launch_impl<128, 128, kEpiQKVG>(tmA, tmB, p, num_sms, s);
+        if (head_dim == 64) return launch_impl<128, 64, kEpiQKVG>(tmA, tmB, p, num_sms, s);
+        return cudaErrorInvalidValue;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dory

@@ -1,0 +1,132 @@
+// Host-side launch interfaces of the sm_100a kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dory {
+
+// ----------------------------------------------------------------- GEMM
+enum GemmEpilogue : int {
+  kEpiStoreF32 = 0,   // C (fp32), optionally one slice per K split
+  kEpiSwiGLU = 1,     // a = SiLU(gate_scale * C[:, gate cols]) * C[:, up cols] -> bf16
+  kEpiQKVG = 2,       // RoPE + per-head L2 norm + s_qk on q/k heads, v copy, sigmoid gates
+};
+
+struct GemmParams {
+  int M = 0, N = 0, K = 0;
+  int k_splits = 1;
+  int epi = kEpiStoreF32;
+  // kEpiStoreF32
+  float* out_f32 = nullptr;
+  int ld_out = 0;
+  size_t split_stride = 0;   // elements between K-split slices
+  // kEpiSwiGLU: tile of BN columns = [BN/2 gate cols | BN/2 up cols]
+  __nv_bfloat16* out_act = nullptr;
+  int ld_act = 0;
+  float gate_scale = 1.f;
+  // kEpiQKVG: columns [q heads | k heads | v heads | Hq gate logits | pad]
+  __nv_bfloat16* q_out = nullptr;   // [M, Hq, hd]
+  __nv_bfloat16* k_out = nullptr;   // [M, Hkv, hd]
+  __nv_bfloat16* v_out = nullptr;   // [M, Hkv, hd]
+  float* gate_out = nullptr;        // [M, Hq]
+  int n_q_heads = 0, n_kv_heads = 0;
+  const float* s_qk = nullptr;       // [hd]
+  const double* inv_freq = nullptr;  // [hd/2] RoPE inverse frequencies of this layer
+  float norm_eps = 1e-20f;
+  int pos0 = 0;                      // row r sits at position pos0 + r ...
+  const int32_t* d_pos = nullptr;    // ... or at d_pos[r] when given
+  uint32_t* status = nullptr;
+};
+
+// Encode a 2D tensor map for a row-major bf16 matrix [rows, cols] with a
+// (64 x box_rows) box and the 128-byte swizzle.  Returns false on failure.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+
+// C[M, N] = A[M, K] * B[N, K]^T with the chosen epilogue.  BN is 128 or 256;
+// head_dim (64 or 128) selects the QKVG epilogue instantiation.
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                        int BN, int head_dim, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------- rows
+struct RowUpdateParams {
+  int rows = 0, d = 0;
+  const float* y = nullptr;   // [splits, rows, d] sublayer output before normalisation
+  int splits = 1;
+  size_t split_stride = 0;    // elements
+  float* h = nullptr;         // [rows, d] fp32 stream, updated in place
+  __nv_bfloat16* hb = nullptr;  // [rows, d] bf16 copy for the next GEMM (may be null)
+  const float* alpha = nullptr;  // [d]
+  float norm_eps = 1e-20f;
+  // optional re-injection: after the update, save the result to e_save (if
+  // set) and then replace it by Norm(h + e) when e is set
+  float* e_save = nullptr;
+  const float* e = nullptr;
+  __nv_bfloat16* out = nullptr;  // optional final output [rows, d] bf16
+};
+cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s);
+
+// bf16 [rows, d] -> fp32 stream + bf16 copy
+cudaError_t launch_load_rows(const __nv_bfloat16* src, float* h, __nv_bfloat16* hb, int rows,
+                             int d, cudaStream_t s);
+// fp32 -> bf16 copy
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
+
+// ----------------------------------------------------------------- KV cache
+// Where one layer's cache lives: sequence s, KV head h, slot t:
+//   K at k_base + s*seq_stride + (h*cap + t)*hd, V at v_base + same (elements)
+struct KvLayerView {
+  __nv_bfloat16* k_base = nullptr;
+  __nv_bfloat16* v_base = nullptr;
+  size_t seq_stride = 0;   // elements
+  int cap = 0;             // slots per (seq, head)
+  int n_kv = 0, hd = 0;
+  int max_seqs = 0, max_ctx = 0;
+};
+
+// Copy fresh K/V rows [rows, Hkv, hd] into cache slots.  Row r goes to
+// sequence seq (or d_seq[r]) at position pos0 + r (or d_pos[r]); rows below
+// `first_row` are skipped.
+cudaError_t launch_kv_commit(const KvLayerView& kv, const __nv_bfloat16* k_new,
+                             const __nv_bfloat16* v_new, int rows, int first_row, int seq,
+                             int pos0, const int32_t* d_seq, const int32_t* d_pos,
+                             uint32_t* status, cudaStream_t s);
+
+// ----------------------------------------------------------------- attention
+struct PrefillAttnParams {
+  const __nv_bfloat16* q = nullptr;     // [n, Hq, hd]
+  const __nv_bfloat16* k_new = nullptr; // [n, Hkv, hd]  this call's keys (positions >= pos0)
+  const __nv_bfloat16* v_new = nullptr;
+  const float* gate = nullptr;          // [n, Hq]
+  __nv_bfloat16* out = nullptr;         // [n, Hq*hd]
+  KvLayerView kv;                       // earlier positions (< pos0)
+  int seq = 0, pos0 = 0, n = 0;
+  int n_q_heads = 0;
+  int window = 0;                       // 0 = full attention
+  float scale_log2 = 0.f;               // softmax_scale * log2(e)
+  uint32_t* status = nullptr;
+};
+cudaError_t launch_prefill_attention(const PrefillAttnParams& p, cudaStream_t s);
+
+struct DecodeAttnParams {
+  const __nv_bfloat16* q = nullptr;     // [B, Hq, hd]
+  const float* gate = nullptr;          // [B, Hq]
+  __nv_bfloat16* out = nullptr;         // [B, Hq*hd]
+  KvLayerView kv;
+  const int32_t* d_seq = nullptr;
+  const int32_t* d_pos = nullptr;
+  int batch = 0, n_q_heads = 0, window = 0;
+  int max_pos = 0;                      // upper bound of d_pos (grid sizing)
+  int split_keys = 0;                   // keys per split
+  float scale_log2 = 0.f;
+  float* part_acc = nullptr;            // [B, Hq, n_splits, hd]
+  float* part_ml = nullptr;             // [B, Hq, n_splits, 2]
+  uint32_t* status = nullptr;
+};
+int decode_attention_splits(int max_pos, int window, int split_keys);
+cudaError_t launch_decode_attention(const DecodeAttnParams& p, cudaStream_t s);
+
+}  // namespace dory

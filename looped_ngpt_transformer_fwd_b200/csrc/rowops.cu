@@ -1,0 +1,187 @@
+// Row-wise kernels of the looped nGPT pass (HBM-bound; one CTA per row):
+//   - the nGPT hypersphere update h <- Norm(h + alpha * (Norm(y) - h)) that
+//     closes every sublayer ("Dory1.0-4B: A Looped Normalized-GPT",
+//     Methodology in Plain English), summing K-split partial products of the
+//     projection first, and optionally saving the input block's output e and
+//     re-injecting it, x <- Norm(x + e), before a pass of the recurrent block
+//     (same page, Methodology);
+//   - input staging (bf16 -> fp32 stream + bf16 GEMM operand);
+//   - KV-cache commits of fresh keys/values into their slots (ring slots
+//     pos % window for sliding-window layers, pos for full layers).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dory {
+
+namespace {
+
+constexpr int kRowMaxChunks = 4;   // float4 chunks per thread
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();   // red may still be read from a previous reduction
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  const int nw = (blockDim.x + 31) >> 5;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+__device__ __forceinline__ float dot4(const float4& a, const float4& b) {
+  return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+}
+
+__global__ void row_update_kernel(const RowUpdateParams p) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const int nch = p.d >> 2;
+  const size_t row_off = static_cast<size_t>(r) * p.d;
+  float4 y[kRowMaxChunks], h[kRowMaxChunks];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    y[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    h[j] = y[j];
+    if (c < nch) {
+      for (int s = 0; s < p.splits; ++s) {
+        const float4 t = reinterpret_cast<const float4*>(p.y + s * p.split_stride + row_off)[c];
+        y[j].x += t.x; y[j].y += t.y; y[j].z += t.z; y[j].w += t.w;
+      }
+      h[j] = reinterpret_cast<const float4*>(p.h + row_off)[c];
+      ss += dot4(y[j], y[j]);
+    }
+  }
+  const float inv_y = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+  ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    if (c < nch) {
+      const float4 a = reinterpret_cast<const float4*>(p.alpha)[c];
+      h[j].x += a.x * (y[j].x * inv_y - h[j].x);
+      h[j].y += a.y * (y[j].y * inv_y - h[j].y);
+      h[j].z += a.z * (y[j].z * inv_y - h[j].z);
+      h[j].w += a.w * (y[j].w * inv_y - h[j].w);
+      ss += dot4(h[j], h[j]);
+    }
+  }
+  const float inv_h = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+  ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    if (c < nch) {
+      h[j].x *= inv_h; h[j].y *= inv_h; h[j].z *= inv_h; h[j].w *= inv_h;
+      if (p.e_save) reinterpret_cast<float4*>(p.e_save + row_off)[c] = h[j];
+      if (p.e) {
+        const float4 e = reinterpret_cast<const float4*>(p.e + row_off)[c];
+        h[j].x += e.x; h[j].y += e.y; h[j].z += e.z; h[j].w += e.w;
+        ss += dot4(h[j], h[j]);
+      }
+    }
+  }
+  if (p.e) {
+    // block_sum is reached by every thread (p.e is uniform)
+    const float inv_x = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+#pragma unroll
+    for (int j = 0; j < kRowMaxChunks; ++j) {
+      h[j].x *= inv_x; h[j].y *= inv_x; h[j].z *= inv_x; h[j].w *= inv_x;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    if (c < nch) {
+      reinterpret_cast<float4*>(p.h + row_off)[c] = h[j];
+      const uint2 b = make_uint2(pack_bf16x2(h[j].x, h[j].y), pack_bf16x2(h[j].z, h[j].w));
+      if (p.hb) reinterpret_cast<uint2*>(p.hb + row_off)[c] = b;
+      if (p.out) reinterpret_cast<uint2*>(p.out + row_off)[c] = b;
+    }
+  }
+}
+
+__global__ void load_rows_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ h,
+                                 __nv_bfloat16* __restrict__ hb, size_t n4) {
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (i >= n4) return;
+  const uint2 v = reinterpret_cast<const uint2*>(src)[i];
+  reinterpret_cast<float4*>(h)[i] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+  reinterpret_cast<uint2*>(hb)[i] = v;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                   size_t n4) {
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(src)[i];
+  reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+
+__global__ void kv_commit_kernel(const KvLayerView kv, const __nv_bfloat16* __restrict__ k_new,
+                                 const __nv_bfloat16* __restrict__ v_new, int rows, int first_row,
+                                 int seq, int pos0, const int32_t* __restrict__ d_seq,
+                                 const int32_t* __restrict__ d_pos, uint32_t* status) {
+  const int per_row = kv.n_kv * (kv.hd / 8);
+  const size_t id = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  const size_t total = static_cast<size_t>(rows - first_row) * per_row;
+  if (id >= total) return;
+  const int r = first_row + static_cast<int>(id / per_row);
+  const int rem = static_cast<int>(id % per_row);
+  const int head = rem / (kv.hd / 8);
+  const int c8 = rem % (kv.hd / 8);
+  const int s = d_seq ? d_seq[r] : seq;
+  const int pos = d_pos ? d_pos[r] : pos0 + r;
+  if (s < 0 || s >= kv.max_seqs || pos < 0 || pos >= kv.max_ctx) {
+    report_status(status, kStatusBounds);
+    return;
+  }
+  const int slot = pos % kv.cap;
+  const size_t src = (static_cast<size_t>(r) * kv.n_kv + head) * kv.hd + c8 * 8;
+  const size_t dst = s * kv.seq_stride + (static_cast<size_t>(head) * kv.cap + slot) * kv.hd + c8 * 8;
+  reinterpret_cast<uint4*>(kv.k_base + dst)[0] = reinterpret_cast<const uint4*>(k_new + src)[0];
+  reinterpret_cast<uint4*>(kv.v_base + dst)[0] = reinterpret_cast<const uint4*>(v_new + src)[0];
+}
+
+}  // namespace
+
+cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s) {
+  if (p.d % 4 != 0 || p.rows < 0) return cudaErrorInvalidValue;
+  if (p.rows == 0) return cudaSuccess;
+  int threads = (p.d / 4 + kRowMaxChunks - 1) / kRowMaxChunks;
+  threads = ((threads + 31) / 32) * 32;
+  if (threads > 1024) return cudaErrorInvalidValue;
+  if (threads < 32) threads = 32;
+  row_update_kernel<<<p.rows, threads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_load_rows(const __nv_bfloat16* src, float* h, __nv_bfloat16* hb, int rows,
+                             int d, cudaStream_t s) {
+  const size_t n4 = static_cast<size_t>(rows) * d / 4;
+  if (n4 == 0) return cudaSuccess;
+  load_rows_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(src, h, hb, n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
+  const size_t n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  f32_to_bf16_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(src, dst, n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_commit(const KvLayerView& kv, const __nv_bfloat16* k_new,
+                             const __nv_bfloat16* v_new, int rows, int first_row, int seq,
+                             int pos0, const int32_t* d_seq, const int32_t* d_pos,
+                             uint32_t* status, cudaStream_t s) {
+  if (first_row >= rows) return cudaSuccess;
+  const size_t total = static_cast<size_t>(rows - first_row) * kv.n_kv * (kv.hd / 8);
+  kv_commit_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
+      kv, k_new, v_new, rows, first_row, seq, pos0, d_seq, d_pos, status);
+  return cudaGetLastError();
+}
+
+}  // namespace dory

@@ -1,0 +1,171 @@
+"""Torch-side plumbing around the C ABI: device buffers, streams and handles.
+
+`DoryModel` owns the caller-side memory the library asks for (packed weights,
+KV caches, workspaces) as torch tensors and forwards every call to the C ABI
+(`binding`).  No arithmetic of the forward pass happens here.
+"""
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class KVCache:
+    """A KV cache bound to a torch byte buffer."""
+
+    def __init__(self, model, mode, max_seqs, max_ctx, k_max=1):
+        self.model = model
+        self.mode = mode
+        self.max_seqs, self.max_ctx, self.k_max = max_seqs, max_ctx, k_max
+        self.nbytes = B.dory_kv_bytes(model.cfg_struct, mode, max_seqs, max_ctx, k_max)
+        if self.nbytes == 0:
+            raise ValueError("invalid KV cache arguments")
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=model.device)
+        self.handle = B.dory_kv_alloc(model.handle, mode, max_seqs, max_ctx, k_max,
+                                      _ptr(self.buf), self.nbytes)
+
+    def layout(self, layer, loop, seq, pos, head):
+        return B.dory_kv_layout(self.handle, layer, loop, seq, pos, head)
+
+    def entry_view(self, layer, loop, seq, head, which="k"):
+        """bf16 view [capacity, head_dim] of one (layer, loop, seq, head) slot ring."""
+        cfg = self.model.cfg
+        k_off, v_off = self.layout(layer, loop, seq, 0, head)
+        off = k_off if which == "k" else v_off
+        full = (layer % cfg["full_period"]) == cfg["full_period"] - 1
+        cap = self.max_ctx if full else min(cfg["window"], self.max_ctx)
+        n = cap * cfg["head_dim"]
+        return self.buf[off:off + 2 * n].view(torch.bfloat16).view(cap, cfg["head_dim"])
+
+    def free(self):
+        if self.handle:
+            B.dory_kv_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+class DoryModel:
+    """Packed weights on the device plus a library handle.
+
+    weights: callable b -> dict in the synthetic generator's format (bf16
+    matrices as uint16 arrays [out, in], float32 vectors).
+    """
+
+    def __init__(self, cfg, weights, device="cuda:0", allow_extrapolated_k=False, stream=None):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.cfg_struct = B.make_config(cfg, allow_extrapolated_k)
+        nb = cfg["n_in_blocks"] + cfg["n_rec_blocks"] + cfg["n_out_blocks"]
+        self.n_blocks = nb
+        self.wbytes = B.dory_weight_bytes(self.cfg_struct)
+        if self.wbytes == 0:
+            raise ValueError("configuration rejected by dory_weight_bytes")
+        self.wbuf = torch.empty(self.wbytes, dtype=torch.uint8, device=self.device)
+        torch.cuda.set_device(self.device)
+        staged = []
+        srcs = []
+        for b in range(nb):
+            w = weights(b)
+            dev = {}
+            for name, arr in w.items():
+                a = np.ascontiguousarray(arr)
+                t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+                dev[name] = t.to(self.device, non_blocking=False)
+            staged.append(dev)
+            srcs.append(B.DoryBlockSrc(*[dev[n].data_ptr() for n in (
+                "wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down",
+                "alpha_attn", "alpha_mlp", "s_qk")]))
+        self.handle = B.dory_create(self.cfg_struct, _ptr(self.wbuf), self.wbytes, srcs,
+                                    _stream(stream))
+        torch.cuda.synchronize(self.device)
+        del staged
+        self._ws = None
+        self._ws_tokens = 0
+
+    # ---------------------------------------------------------------- buffers
+    def kv_cache(self, mode, max_seqs, max_ctx, k_max=1):
+        return KVCache(self, mode, max_seqs, max_ctx, k_max)
+
+    def workspace(self, max_tokens):
+        if self._ws is None or self._ws_tokens < max_tokens:
+            n = B.dory_workspace_bytes(self.handle, max_tokens)
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._ws_tokens = max_tokens
+        return self._ws
+
+    # ---------------------------------------------------------------- calls
+    def prefill(self, kv, h_in, k, seq=0, pos0=0, h_out=None, stream=None):
+        """h_in: [n, d] bf16 tensor on the device or in (pinned) host memory."""
+        n = h_in.shape[0]
+        if h_out is None:
+            h_out = torch.empty_like(h_in)
+        ws = self.workspace(n)
+        B.dory_prefill(self.handle, kv.handle, seq, pos0, n, _ptr(h_in), _ptr(h_out), k,
+                       _ptr(ws), ws.numel(), _stream(stream))
+        return h_out
+
+    def decode(self, kv, h_in, d_seq, d_pos, max_pos, k, h_out=None, stream=None):
+        """One decode step; d_seq / d_pos: int32 device tensors [batch]."""
+        n = h_in.shape[0]
+        if h_out is None:
+            h_out = torch.empty_like(h_in)
+        ws = self.workspace(n)
+        B.dory_decode_step(self.handle, kv.handle, n, _ptr(d_seq), _ptr(d_pos), max_pos,
+                           _ptr(h_in), _ptr(h_out), k, _ptr(ws), ws.numel(), _stream(stream))
+        return h_out
+
+    def attention_sublayer(self, kv, layer, h, loop=1, seq=0, pos0=0, stream=None):
+        """In place on h: [n, d] float32 device tensor."""
+        ws = self.workspace(h.shape[0])
+        B.dory_attention_sublayer(self.handle, kv.handle, layer, loop, seq, pos0, h.shape[0],
+                                  _ptr(h), _ptr(ws), ws.numel(), _stream(stream))
+        return h
+
+    def mlp_sublayer(self, layer, h, stream=None):
+        ws = self.workspace(h.shape[0])
+        B.dory_mlp_sublayer(self.handle, layer, h.shape[0], _ptr(h), _ptr(ws), ws.numel(),
+                            _stream(stream))
+        return h
+
+    def device_status(self, stream=None):
+        return B.dory_device_status(self.handle, _stream(stream))
+
+    def last_call_stats(self):
+        return B.dory_last_call_stats(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            B.dory_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def gemm_bf16(A, Bm, stream=None):
+    """C = A @ Bm^T through the library's tcgen05 GEMM (bf16 in, fp32 out)."""
+    M, K = A.shape
+    N = Bm.shape[0]
+    C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    B.dory_gemm_bf16(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, _stream(stream))
+    return C

@@ -1,0 +1,226 @@
+"""GPU parity: the sm_100a library (through its C ABI) against the float64 oracle
+on the same seeded inputs (tiny config: several tiles, ragged tails, ring wraps)."""
+
+import numpy as np
+import pytest
+import torch
+
+from tests.gpu_util import (build, inputs, to_np, assert_parity, oracle, oracle_cache, metrics)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return build("tiny", seed=0, variant="random")
+
+
+# ------------------------------------------------------------------ GEMM
+@pytest.mark.parametrize("M,N,K", [(300, 512, 384), (64, 384, 3072), (1, 128, 64), (1000, 768, 256),
+                                   (129, 256, 128)])
+def test_gemm_matches_fp64(M, N, K):
+    from looped_ngpt_transformer_fwd_b200 import build as libbuild
+    from looped_ngpt_transformer_fwd_b200.model import gemm_bf16
+    libbuild.build()
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    Bm = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    C = gemm_bf16(A, Bm)
+    torch.cuda.synchronize()
+    ref = (A.double() @ Bm.double().T)
+    err = (C.double() - ref).abs().max().item()
+    assert err <= 1e-4 * ref.abs().max().item() + 1e-4, err
+
+
+# ------------------------------------------------------------------ sublayers
+def test_mlp_sublayer_matches_oracle(tiny):
+    cfg, prov, model = tiny
+    _, h = inputs(cfg, 11, 200)
+    for layer in (0, 5):
+        ht = torch.from_numpy(h.astype(np.float32)).cuda()
+        model.mlp_sublayer(layer, ht)
+        torch.cuda.synchronize()
+        ref = oracle(cfg, prov).mlp_sublayer(layer, h)
+        assert_parity(to_np(ht), ref, tol_abs=5e-3, tol_cos=0.9999, what=f"mlp layer {layer}")
+
+
+@pytest.mark.parametrize("layer", [0, 1])     # SWA, full
+def test_attention_sublayer_matches_oracle(tiny, layer):
+    cfg, prov, model = tiny
+    _, h = inputs(cfg, 12, 150)
+    kv = model.kv_cache("last_loop", 2, 256)
+    ocache = oracle_cache(cfg, "last_loop")
+    orc = oracle(cfg, prov)
+    # two calls: the second reads the first's committed keys (ring for SWA)
+    for pos0, n in ((0, 90), (90, 60)):
+        ht = torch.from_numpy(h[pos0:pos0 + n].astype(np.float32)).cuda()
+        model.attention_sublayer(kv, layer, ht, loop=1, seq=1, pos0=pos0)
+        torch.cuda.synchronize()
+        ref = orc.attention_sublayer(layer, h[pos0:pos0 + n], pos0, 1, 1, ocache)
+        assert_parity(to_np(ht), ref, tol_abs=5e-3, tol_cos=0.9999, what=f"attn {layer} @{pos0}")
+
+
+# ------------------------------------------------------------------ whole stack
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_prefill_matches_oracle(tiny, mode, k):
+    cfg, prov, model = tiny
+    x, h = inputs(cfg, 13, 128)
+    kv = model.kv_cache(mode, 1, 256, k_max=3)
+    out = model.prefill(kv, x, k)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=3))
+    assert_parity(to_np(out), ref, what=f"prefill {mode} k={k}")
+    launches, sub = model.last_call_stats()
+    assert sub == 2 * (cfg["n_in_blocks"] + k * cfg["n_rec_blocks"] + cfg["n_out_blocks"])
+    assert launches > sub
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_chunked_prefill_then_decode_matches_oracle(tiny, mode):
+    """Chunks that straddle the 32-slot SWA ring several times, then decode steps."""
+    cfg, prov, model = tiny
+    k = 2
+    x, h = inputs(cfg, 14, 110)
+    kv = model.kv_cache(mode, 3, 160, k_max=2)
+    ocache = oracle_cache(cfg, mode, k_max=2)
+    orc = oracle(cfg, prov)
+    seq = 2
+    for a, b in ((0, 45), (45, 46), (46, 100)):
+        out = model.prefill(kv, x[a:b], k, seq=seq, pos0=a)
+        torch.cuda.synchronize()
+        ref = orc.forward(h[a:b], a, k, ocache, seq=seq)
+        assert_parity(to_np(out), ref, what=f"chunk {a}:{b} {mode}")
+    for step, p in enumerate(range(100, 110)):
+        d_seq = torch.tensor([seq], dtype=torch.int32, device="cuda")
+        d_pos = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d_seq, d_pos, 159, k)
+        torch.cuda.synchronize()
+        ref = orc.decode(h[p:p + 1], [seq], [p], k, ocache)
+        assert_parity(to_np(out), ref, what=f"decode step {step} {mode}")
+    assert model.device_status() == 0
+
+
+def test_decode_batch_of_sequences_matches_oracle(tiny):
+    """A batch of sequences at different positions (ragged contexts) in one step."""
+    cfg, prov, model = tiny
+    k = 2
+    mode = "last_loop"
+    kv = model.kv_cache(mode, 5, 200, k_max=2)
+    ocache = oracle_cache(cfg, mode, k_max=2)
+    orc = oracle(cfg, prov)
+    lens = [3, 40, 77, 1, 64]
+    xs = [inputs(cfg, 20 + s, lens[s] + 2) for s in range(5)]
+    for s, L in enumerate(lens):
+        model.prefill(kv, xs[s][0][:L], k, seq=s, pos0=0)
+        orc.forward(xs[s][1][:L], 0, k, ocache, seq=s)
+    order = [3, 0, 4, 1, 2]          # rows in a different order than the sequences
+    for step in range(2):
+        rows_t = torch.cat([xs[s][0][lens[s] + step:lens[s] + step + 1] for s in order])
+        rows_h = np.concatenate([xs[s][1][lens[s] + step:lens[s] + step + 1] for s in order])
+        d_seq = torch.tensor(order, dtype=torch.int32, device="cuda")
+        d_pos = torch.tensor([lens[s] + step for s in order], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, rows_t, d_seq, d_pos, 199, k)
+        torch.cuda.synchronize()
+        ref = orc.decode(rows_h, order, [lens[s] + step for s in order], k, ocache)
+        assert_parity(to_np(out), ref, what=f"batched decode step {step}")
+
+
+def test_window_mask_is_exact():
+    """W = 4: an off-by-one in the sliding window or causal mask moves a fifth of the
+    softmax mass and fails the bar."""
+    cfg, prov, model = build("tiny", seed=3, variant="random", window=4)
+    x, h = inputs(cfg, 15, 70)
+    kv = model.kv_cache("last_loop", 1, 128)
+    out = model.prefill(kv, x[:60], 2)
+    ocache = oracle_cache(cfg, "last_loop")
+    orc = oracle(cfg, prov)
+    ref = orc.forward(h[:60], 0, 2, ocache)
+    assert_parity(to_np(out), ref, tol_cos=0.9995, what="W=4 prefill")
+    for p in range(60, 66):
+        d = torch.tensor([0], dtype=torch.int32, device="cuda")
+        pp = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d, pp, 127, 2)
+        ref = orc.decode(h[p:p + 1], [0], [p], 2, ocache)
+        assert_parity(to_np(out), ref, tol_cos=0.9995, what=f"W=4 decode {p}")
+
+
+def test_modes_identical_at_k1(tiny):
+    """Per-loop and last-loop caching run the same kernels on the same slots at k = 1."""
+    cfg, prov, model = tiny
+    x, _ = inputs(cfg, 16, 96)
+    outs, caches = [], []
+    for mode in ("per_loop", "last_loop"):
+        kv = model.kv_cache(mode, 1, 128, k_max=1)
+        kv.buf.zero_()
+        outs.append(model.prefill(kv, x[:80], 1).clone())
+        torch.cuda.synchronize()
+        caches.append(kv.buf.clone())
+    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(caches[0], caches[1])
+
+
+def test_kv_cache_slots_and_contents(tiny):
+    """Cache indexing is exact: full layers fill slots 0..T-1 and leave the rest
+    untouched (bit-exact sentinel); SWA rings hold positions T-W..T-1 at pos % W;
+    the stored k_hat / v match the oracle's entries for those positions."""
+    cfg, prov, model = tiny
+    T, ctx = 100, 128
+    x, h = inputs(cfg, 17, T)
+    kv = model.kv_cache("last_loop", 2, ctx, k_max=1)
+    kv.buf.view(torch.int16).fill_(0x7F7F)
+    model.prefill(kv, x, 2, seq=1)
+    torch.cuda.synchronize()
+    ocache = oracle_cache(cfg, "last_loop")
+    oracle(cfg, prov).forward(h, 0, 2, ocache, seq=1)
+    sentinel = torch.tensor(0x7F7F, dtype=torch.int16)
+    for layer in range(8):
+        full = layer % cfg["full_period"] == cfg["full_period"] - 1
+        for head in range(cfg["n_kv_heads"]):
+            kview = kv.entry_view(layer, 1, 1, head, "k")
+            vview = kv.entry_view(layer, 1, 1, head, "v")
+            other = kv.entry_view(layer, 1, 0, head, "k")     # sequence 0: never written
+            assert bool((other.view(torch.int16).cpu() == sentinel).all())
+            if full:
+                assert bool((kview[T:].view(torch.int16).cpu() == sentinel).all())
+                positions = list(range(T))
+                slots = positions
+            else:
+                positions = list(range(T - cfg["window"], T))
+                slots = [p % cfg["window"] for p in positions]
+            K, V = ocache.read(layer, 1, 1, positions[0], positions[-1] + 1)
+            gk = to_np(kview[slots])
+            gv = to_np(vview[slots])
+            assert np.abs(gk - K[:, head]).max() < 3e-2, (layer, head)
+            assert np.abs(gv - V[:, head]).max() < 3e-2, (layer, head)
+
+
+def test_host_buffers_give_the_same_result(tiny):
+    """dory_prefill with pinned host h_in / h_out equals the device-buffer call."""
+    cfg, prov, model = tiny
+    x, _ = inputs(cfg, 18, 64)
+    kv = model.kv_cache("last_loop", 1, 64)
+    dev = model.prefill(kv, x, 2).cpu()
+    hin = x.cpu().pin_memory()
+    hout = torch.empty_like(hin).pin_memory()
+    model.prefill(kv, hin, 2, h_out=hout)
+    torch.cuda.synchronize()
+    assert torch.equal(dev, hout)
+
+
+def test_argument_errors(tiny):
+    from looped_ngpt_transformer_fwd_b200.binding import DoryError
+    cfg, prov, model = tiny
+    x, _ = inputs(cfg, 19, 16)
+    kv = model.kv_cache("per_loop", 1, 32, k_max=2)
+    with pytest.raises(DoryError) as e:
+        model.prefill(kv, x, 3)
+    assert e.value.status == -4
+    with pytest.raises(DoryError) as e:
+        model.prefill(kv, x, 0)
+    assert e.value.status == -3
+    with pytest.raises(DoryError) as e:
+        model.prefill(kv, x, 1, pos0=20)
+    assert e.value.status == -5
+    assert model.device_status() == 0
