@@ -188,6 +188,28 @@ DORY_API void dory_kv_free(dory_kv* kv);
 DORY_API void dory_destroy(dory_model* m);
 
 /* ---------------------------------------------------------------------
+ * Per-kernel timing (diagnostics).  While enabled, calls whose CUDA graph is
+ * captured afterwards record a CUDA event before and after every kernel they
+ * launch (graphs captured without it are kept separately and stay
+ * uninstrumented).  dory_profile_read synchronises on the most recent
+ * instrumented call and returns, for one kernel kind, the summed device time
+ * in milliseconds and the number of launches of that call.
+ * --------------------------------------------------------------------- */
+typedef enum dory_kernel_kind {
+  DORY_KK_QKVG = 0,      /* QKV + gate projection with RoPE / QK-norm epilogue   */
+  DORY_KK_ATTN = 1,      /* prefill attention, or decode split-KV + combine      */
+  DORY_KK_OPROJ = 2,     /* output projection                                    */
+  DORY_KK_GATEUP = 3,    /* gate/up projection with SwiGLU epilogue              */
+  DORY_KK_DOWN = 4,      /* down projection                                      */
+  DORY_KK_ROW = 5,       /* nGPT update / re-injection row kernels, input load   */
+  DORY_KK_KVCOMMIT = 6,  /* KV-cache slot commits                                */
+  DORY_KK_COUNT = 7
+} dory_kernel_kind;
+
+DORY_API int dory_profile_enable(dory_model* m, int enable);
+DORY_API int dory_profile_read(dory_model* m, int kind, float* total_ms, int* launches);
+
+/* ---------------------------------------------------------------------
  * Single-sublayer entry points (diagnostics and per-sublayer parity).
  * They run exactly the kernels the full pass runs for one sublayer of
  * global block `layer` at loop `loop`, on `n_rows` rows.

@@ -30,7 +30,10 @@ EXPORTS = (
     "dory_workspace_bytes", "dory_prefill", "dory_decode_step", "dory_device_status",
     "dory_last_call_stats", "dory_error_string", "dory_kv_free", "dory_destroy",
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
+    "dory_profile_enable", "dory_profile_read",
 )
+
+KERNEL_KINDS = ("qkvg", "attn", "oproj", "gateup", "down", "row", "kvcommit")
 
 
 class DoryError(RuntimeError):
@@ -89,6 +92,8 @@ def lib():
             "dory_attention_sublayer": (I, [P, P, I, I, I, I, I, P, P, SZ, P]),
             "dory_mlp_sublayer": (I, [P, I, I, P, P, SZ, P]),
             "dory_gemm_bf16": (I, [P, P, P, I, I, I, P]),
+            "dory_profile_enable": (I, [P, I]),
+            "dory_profile_read": (I, [P, I, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -189,6 +194,19 @@ def dory_mlp_sublayer(model, layer, n_rows, h, ws, ws_bytes, stream):
 
 def dory_gemm_bf16(A, B, C, M, N, K, stream):
     return check(lib().dory_gemm_bf16(A, B, C, M, N, K, stream), "dory_gemm_bf16")
+
+
+def dory_profile_enable(model, enable):
+    return check(lib().dory_profile_enable(model, 1 if enable else 0), "dory_profile_enable")
+
+
+def dory_profile_read(model, kind):
+    """(total ms, launches) of one kernel kind in the last instrumented call."""
+    ms, n = ctypes.c_float(), ctypes.c_int()
+    kind = KERNEL_KINDS.index(kind) if isinstance(kind, str) else kind
+    check(lib().dory_profile_read(model, kind, ctypes.byref(ms), ctypes.byref(n)),
+          "dory_profile_read")
+    return ms.value, n.value
 
 
 def dory_kv_free(kv):

@@ -63,20 +63,37 @@ struct BlockW {
 };
 
 struct GraphKey {
-  int phase, k, n, seq, pos0, max_pos;
+  int phase, k, n, seq, pos0, max_pos, prof;
   const void *src, *dst, *ws, *kv, *dseq, *dpos;
   bool operator<(const GraphKey& o) const {
-    return std::tie(phase, k, n, seq, pos0, max_pos, src, dst, ws, kv, dseq, dpos) <
-           std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.src, o.dst, o.ws, o.kv, o.dseq,
-                    o.dpos);
+    return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos) <
+           std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.prof, o.src, o.dst, o.ws, o.kv,
+                    o.dseq, o.dpos);
   }
+};
+
+// events around one kernel launch of an instrumented graph
+struct Mark {
+  int kind;
+  cudaEvent_t start, end;
 };
 
 struct GraphEntry {
   cudaGraphExec_t exec = nullptr;
   int launches = 0, sublayers = 0;
   uint64_t last_use = 0;
+  std::vector<Mark> marks;
 };
+
+void destroy_entry(GraphEntry& g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  for (auto& mk : g.marks) {
+    cudaEventDestroy(mk.start);
+    cudaEventDestroy(mk.end);
+  }
+  g.marks.clear();
+  g.exec = nullptr;
+}
 
 }  // namespace
 
@@ -96,6 +113,10 @@ struct dory_model {
   int last_launches = 0, last_sublayers = 0;
   // counters of the call being enqueued
   int cur_launches = 0, cur_sublayers = 0;
+  // per-kernel timing
+  bool profile = false;
+  std::vector<Mark>* cur_marks = nullptr;      // marks of the graph being captured
+  const std::vector<Mark>* last_marks = nullptr;
 };
 
 struct dory_kv {
@@ -253,6 +274,36 @@ struct CallCtx {
     if (_e != cudaSuccess) return _e;          \
   } while (0)
 
+// Bracket one kernel launch with events when the graph being captured is
+// instrumented; counts the launch either way.
+struct Launch {
+  dory_model* m;
+  cudaStream_t s;
+  Mark mk{};
+  bool on = false;
+  Launch(dory_model* m_, cudaStream_t s_, int kind) : m(m_), s(s_) {
+    ++m->cur_launches;
+    if (m->cur_marks && cudaEventCreate(&mk.start) == cudaSuccess) {
+      if (cudaEventCreate(&mk.end) == cudaSuccess) {
+        mk.kind = kind;
+        on = cudaEventRecord(mk.start, s) == cudaSuccess;
+        if (!on) {
+          cudaEventDestroy(mk.start);
+          cudaEventDestroy(mk.end);
+        }
+      } else {
+        cudaEventDestroy(mk.start);
+      }
+    }
+  }
+  ~Launch() {
+    if (on) {
+      cudaEventRecord(mk.end, s);
+      m->cur_marks->push_back(mk);
+    }
+  }
+};
+
 int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   if (tiles >= m->num_sms / 2) return 1;
@@ -282,14 +333,19 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   g.pos0 = c.decode ? 0 : c.pos0;
   g.d_pos = c.decode ? c.dpos : nullptr;
   g.status = m->status;
-  DORY_TRY(launch_gemm(tmA, W.tm_qkvg[bn_q == 256], g, bn_q, m->hd, m->num_sms, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_QKVG);
+    DORY_TRY(launch_gemm(tmA, W.tm_qkvg[bn_q == 256], g, bn_q, m->hd, m->num_sms, c.s));
+  }
 
   const KvLayerView view = kv_view(c.kv, b, loop);
   const int window = W.full ? 0 : m->cfg.window;
   const float scale_log2 = m->cfg.softmax_scale * 1.4426950408889634f;
   if (c.decode) {
-    DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s));
+    {
+      Launch L(m, c.s, DORY_KK_KVCOMMIT);
+      DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s));
+    }
     DecodeAttnParams a;
     a.q = c.w.q; a.gate = c.w.gate; a.out = c.w.o; a.kv = view;
     a.d_seq = c.dseq; a.d_pos = c.dpos;
@@ -301,20 +357,25 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     a.scale_log2 = scale_log2;
     a.part_acc = c.w.dacc; a.part_ml = c.w.dml;
     a.status = m->status;
-    DORY_TRY(launch_decode_attention(a, c.s));
-    c.m->cur_launches += 3;
+    {
+      Launch L(m, c.s, DORY_KK_ATTN);
+      ++m->cur_launches;   // split-KV kernel + combine kernel
+      DORY_TRY(launch_decode_attention(a, c.s));
+    }
   } else {
     PrefillAttnParams a;
     a.q = c.w.q; a.k_new = c.w.kf; a.v_new = c.w.vf; a.gate = c.w.gate; a.out = c.w.o;
     a.kv = view; a.seq = c.seq; a.pos0 = c.pos0; a.n = c.n; a.n_q_heads = m->hq;
     a.window = window; a.scale_log2 = scale_log2; a.status = m->status;
-    DORY_TRY(launch_prefill_attention(a, c.s));
-    ++c.m->cur_launches;
+    {
+      Launch L(m, c.s, DORY_KK_ATTN);
+      DORY_TRY(launch_prefill_attention(a, c.s));
+    }
     if (commit_after) {
       const int first = W.full ? 0 : std::max(0, c.n - view.cap);
+      Launch L(m, c.s, DORY_KK_KVCOMMIT);
       DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, first, c.seq, c.pos0, nullptr, nullptr,
                                 m->status, c.s));
-      ++c.m->cur_launches;
     }
   }
 
@@ -328,14 +389,18 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   go.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_o, m->d_attn) : 1;
   go.out_f32 = c.w.y; go.ld_out = m->d; go.split_stride = size_t(c.n) * m->d;
   go.status = m->status;
-  DORY_TRY(launch_gemm(tmO, W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_OPROJ);
+    DORY_TRY(launch_gemm(tmO, W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms, c.s));
+  }
 
   RowUpdateParams r;
   r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = go.k_splits; r.split_stride = go.split_stride;
   r.h = h; r.hb = hb; r.alpha = W.alpha_attn; r.norm_eps = m->cfg.norm_eps;
-  DORY_TRY(launch_row_update(r, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_ROW);
+    DORY_TRY(launch_row_update(r, c.s));
+  }
   ++c.m->cur_sublayers;
   return cudaSuccess;
 }
@@ -353,8 +418,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   g.epi = kEpiSwiGLU;
   g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
   g.status = m->status;
-  DORY_TRY(launch_gemm(tmA, W.tm_gu, g, 256, m->hd, m->num_sms, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_GATEUP);
+    DORY_TRY(launch_gemm(tmA, W.tm_gu, g, 256, m->hd, m->num_sms, c.s));
+  }
 
   CUtensorMap tmAct;
   if (!make_tmap_bf16(&tmAct, c.w.a, c.n, m->ff, 128)) return cudaErrorInvalidValue;
@@ -365,8 +432,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   gd.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_d, m->ff) : 1;
   gd.out_f32 = c.w.y; gd.ld_out = m->d; gd.split_stride = size_t(c.n) * m->d;
   gd.status = m->status;
-  DORY_TRY(launch_gemm(tmAct, W.tm_d[bn_d == 256], gd, bn_d, m->hd, m->num_sms, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_DOWN);
+    DORY_TRY(launch_gemm(tmAct, W.tm_d[bn_d == 256], gd, bn_d, m->hd, m->num_sms, c.s));
+  }
 
   RowUpdateParams r;
   r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = gd.k_splits; r.split_stride = gd.split_stride;
@@ -374,8 +443,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   r.e_save = save_e ? c.w.e32 : nullptr;
   r.e = reinject ? c.w.e32 : nullptr;
   r.out = out;
-  DORY_TRY(launch_row_update(r, c.s));
-  ++c.m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_ROW);
+    DORY_TRY(launch_row_update(r, c.s));
+  }
   ++c.m->cur_sublayers;
   return cudaSuccess;
 }
@@ -385,8 +456,10 @@ cudaError_t enqueue_stack(CallCtx& c, const __nv_bfloat16* src, __nv_bfloat16* d
   dory_model* m = c.m;
   const dory_config* cfg = &m->cfg;
   const int n_in = cfg->n_in_blocks, n_rec = cfg->n_rec_blocks, nb = m->nb;
-  DORY_TRY(launch_load_rows(src, c.w.h32, c.w.hb, c.n, m->d, c.s));
-  ++m->cur_launches;
+  {
+    Launch L(m, c.s, DORY_KK_ROW);
+    DORY_TRY(launch_load_rows(src, c.w.h32, c.w.hb, c.n, m->d, c.s));
+  }
   const bool last_loop = c.kv->mode == DORY_KV_LAST_LOOP;
   for (int b = 0; b < n_in; ++b) {
     DORY_TRY(attention_sublayer(c, b, 1, c.w.h32, c.w.hb, true));
@@ -419,26 +492,33 @@ int run_graph(dory_model* m, const GraphKey& key, CallCtx& c, const __nv_bfloat1
       auto lru = m->graphs.begin();
       for (auto g = m->graphs.begin(); g != m->graphs.end(); ++g)
         if (g->second.last_use < lru->second.last_use) lru = g;
-      cudaGraphExecDestroy(lru->second.exec);
+      if (m->last_marks == &lru->second.marks) m->last_marks = nullptr;
+      destroy_entry(lru->second);
       m->graphs.erase(lru);
     }
     m->cur_launches = 0;
     m->cur_sublayers = 0;
+    GraphEntry ent;
+    m->cur_marks = key.prof ? &ent.marks : nullptr;
     c.s = m->cap_stream;
     if (cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
       return DORY_ERR_CUDA;
     cudaError_t e = enqueue_stack(c, src, dst);
+    m->cur_marks = nullptr;
     cudaGraph_t graph = nullptr;
     cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &graph);
     if (e != cudaSuccess || e2 != cudaSuccess || !graph) {
       if (graph) cudaGraphDestroy(graph);
+      destroy_entry(ent);
       cudaGetLastError();
       return DORY_ERR_CUDA;
     }
-    GraphEntry ent;
     e = cudaGraphInstantiate(&ent.exec, graph, 0);
     cudaGraphDestroy(graph);
-    if (e != cudaSuccess) return DORY_ERR_CUDA;
+    if (e != cudaSuccess) {
+      destroy_entry(ent);
+      return DORY_ERR_CUDA;
+    }
     ent.launches = m->cur_launches;
     ent.sublayers = m->cur_sublayers;
     it = m->graphs.emplace(key, ent).first;
@@ -447,6 +527,7 @@ int run_graph(dory_model* m, const GraphKey& key, CallCtx& c, const __nv_bfloat1
   if (cudaGraphLaunch(it->second.exec, stream) != cudaSuccess) return DORY_ERR_CUDA;
   m->last_launches = it->second.launches;
   m->last_sublayers = it->second.sublayers;
+  if (key.prof) m->last_marks = &it->second.marks;
   return DORY_OK;
 }
 
@@ -672,7 +753,7 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{0, k, n_tokens, seq, pos0, 0, src, dst, ws, kv, nullptr, nullptr};
+  GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv, nullptr, nullptr};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -704,7 +785,7 @@ int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{1, k, batch, 0, 0, max_pos_hint, src, dst, ws, kv, d_seq, d_pos};
+  GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv, d_seq, d_pos};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -735,11 +816,35 @@ int dory_last_call_stats(const dory_model* m, int* kernel_launches, int* sublaye
   return DORY_OK;
 }
 
+int dory_profile_enable(dory_model* m, int enable) {
+  if (!m) return DORY_ERR_INVALID_ARG;
+  m->profile = enable != 0;
+  return DORY_OK;
+}
+
+int dory_profile_read(dory_model* m, int kind, float* total_ms, int* launches) {
+  if (!m || !total_ms || kind < 0 || kind >= DORY_KK_COUNT) return DORY_ERR_INVALID_ARG;
+  if (!m->last_marks) return DORY_ERR_INVALID_ARG;
+  float tot = 0.f;
+  int cnt = 0;
+  for (const Mark& mk : *m->last_marks) {
+    if (mk.kind != kind) continue;
+    if (cudaEventSynchronize(mk.end) != cudaSuccess) return DORY_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, mk.start, mk.end) != cudaSuccess) return DORY_ERR_CUDA;
+    tot += ms;
+    ++cnt;
+  }
+  *total_ms = tot;
+  if (launches) *launches = cnt;
+  return DORY_OK;
+}
+
 void dory_kv_free(dory_kv* kv) { delete kv; }
 
 void dory_destroy(dory_model* m) {
   if (!m) return;
-  for (auto& g : m->graphs) cudaGraphExecDestroy(g.second.exec);
+  for (auto& g : m->graphs) destroy_entry(g.second);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;
 }

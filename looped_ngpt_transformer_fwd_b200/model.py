@@ -150,6 +150,13 @@ class DoryModel:
     def last_call_stats(self):
         return B.dory_last_call_stats(self.handle)
 
+    def profile(self, enable=True):
+        B.dory_profile_enable(self.handle, enable)
+
+    def profile_read(self):
+        """{kind: (total ms, launches)} of the last instrumented call."""
+        return {k: B.dory_profile_read(self.handle, k) for k in B.KERNEL_KINDS}
+
     def close(self):
         if getattr(self, "handle", None):
             B.dory_destroy(self.handle)

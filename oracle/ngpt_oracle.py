@@ -263,9 +263,9 @@ class Oracle:
         self.q_block = 128                # queries per softmax batch (memory only)
 
     # -- helpers ---------------------------------------------------------
-    def _w(self, b):
+    def _w(self, b, names):
         raw = self.weights(b)
-        return {name: _as_float(val, self.dt) for name, val in raw.items()}
+        return {name: _as_float(raw[name], self.dt) for name in names}
 
     def _norm(self, x, axis=-1):
         return l2norm(x, self.cfg["norm_eps"], axis)
@@ -287,7 +287,7 @@ class Oracle:
         L2 norm of the concatenated gated output before the output projection.
         """
         cfg = self.cfg
-        W = self._w(b)
+        W = self._w(b, ("wq", "wk", "wv", "wg", "wo", "alpha_attn", "s_qk"))
         n, d = h.shape
         hq, hkv, hd = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
         full = is_full_layer(cfg, b)
@@ -331,7 +331,7 @@ class Oracle:
     def mlp_sublayer(self, b, h):
         """SwiGLU sublayer with L2-normalised activations before the down-projection
         ([P1] Methodology in Plain English)."""
-        W = self._w(b)
+        W = self._w(b, ("w_gate", "w_up", "w_down", "alpha_mlp"))
         a = silu(self.cfg["gate_scale"] * (h @ W["w_gate"].T)) * (h @ W["w_up"].T)
         y = self._norm(a) @ W["w_down"].T
         return self._ngpt_update(h, y, W["alpha_mlp"])
