@@ -286,7 +286,8 @@ struct Launch {
     if (m->cur_marks && cudaEventCreate(&mk.start) == cudaSuccess) {
       if (cudaEventCreate(&mk.end) == cudaSuccess) {
         mk.kind = kind;
-        on = cudaEventRecord(mk.start, s) == cudaSuccess;
+        // external records become event nodes of the captured graph
+        on = cudaEventRecordWithFlags(mk.start, s, cudaEventRecordExternal) == cudaSuccess;
         if (!on) {
           cudaEventDestroy(mk.start);
           cudaEventDestroy(mk.end);
@@ -298,8 +299,12 @@ struct Launch {
   }
   ~Launch() {
     if (on) {
-      cudaEventRecord(mk.end, s);
-      m->cur_marks->push_back(mk);
+      if (cudaEventRecordWithFlags(mk.end, s, cudaEventRecordExternal) == cudaSuccess) {
+        m->cur_marks->push_back(mk);
+      } else {
+        cudaEventDestroy(mk.start);
+        cudaEventDestroy(mk.end);
+      }
     }
   }
 };

@@ -224,3 +224,23 @@ def test_argument_errors(tiny):
         model.prefill(kv, x, 1, pos0=20)
     assert e.value.status == -5
     assert model.device_status() == 0
+
+
+def test_kernel_profiling_counts_every_launch(tiny):
+    """Instrumented graphs time every kernel; counts add up to the call's launches."""
+    cfg, prov, model = tiny
+    x, _ = inputs(cfg, 21, 64)
+    kv = model.kv_cache("last_loop", 1, 64, k_max=2)
+    model.profile(True)
+    try:
+        out_p = model.prefill(kv, x, 2).clone()
+        prof = model.profile_read()
+    finally:
+        model.profile(False)
+    out = model.prefill(kv, x, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_p)
+    launches, sub = model.last_call_stats()
+    assert sum(n for _, n in prof.values()) == launches
+    assert prof["gateup"][1] == prof["down"][1] == sub // 2
+    assert all(t > 0 for t, n in prof.values() if n)
