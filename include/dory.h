@@ -63,7 +63,8 @@ typedef enum dory_status {
   DORY_ERR_CUDA = -8,             /* a CUDA runtime/driver call failed            */
   DORY_ERR_DEVICE_TIMEOUT = -9,   /* a kernel's bounded wait expired (device word) */
   DORY_ERR_UNSUPPORTED_ARCH = -10,/* device is not sm_100                         */
-  DORY_ERR_DEVICE_BOUNDS = -11    /* a kernel's bounds check fired (device word)   */
+  DORY_ERR_DEVICE_BOUNDS = -11,   /* a kernel's bounds check fired (device word)   */
+  DORY_ERR_SCRATCH_LIMIT = -12    /* rows exceed the library's built-in scratch    */
 } dory_status;
 
 typedef enum dory_kv_mode {
@@ -229,6 +230,39 @@ DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
 /* The tensor-core GEMM alone: C[M,N] (fp32) = A[M,K] (bf16) * B[N,K]^T (bf16),
  * all row-major device buffers, K a multiple of 64, N a multiple of 128. */
 DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Allocation-free variant (no counterpart in the paper: a deployment aid).
+ *
+ * Some callers cannot allocate device memory at all: code running where
+ * cudaMalloc is forbidden or unavailable (inside another allocator's hooks,
+ * in a process whose memory pool is fixed up front, or in a plugin that
+ * receives only its input and output buffers).  They cannot provide the
+ * workspace that dory_mlp_sublayer needs.  dory_mlp_sublayer_noalloc runs
+ * the same SwiGLU sublayer (same kernels, same results) with its scratch --
+ * the bf16 copy of h, the SwiGLU activations and the fp32 projection output
+ * -- in a fixed array of DORY_NOALLOC_SCRATCH_BYTES that is part of the
+ * library itself: every GPU that loads the library holds this array until the
+ * process exits.  The caller passes only the rows h [n_rows, d_model] (fp32,
+ * device, updated in place).
+ *
+ * Limit: with A(x) = x rounded up to 256, the call needs
+ *   A(2*n_rows*d_model) + A(2*n_rows*d_ff) + A(4*n_rows*d_model)
+ * bytes; larger n_rows return DORY_ERR_SCRATCH_LIMIT without launching
+ * anything (about 227 rows for d_model 3072, d_ff 9216).
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  The call itself allocates nothing.  All calls
+ * share the one array and it keeps the last call's contents; each call writes
+ * every scratch byte before reading it, so nothing needs clearing.  Calls
+ * that may overlap on the GPU (different streams, or graphs replayed
+ * concurrently) race on the array: serialise them.
+ * --------------------------------------------------------------------- */
+#define DORY_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+DORY_API int dory_mlp_sublayer_noalloc(dory_model* m, int layer, int n_rows, float* h,
+                                       void* stream);
 
 #ifdef __cplusplus
 }

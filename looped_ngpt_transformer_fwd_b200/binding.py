@@ -21,7 +21,7 @@ STATUS = {
     0: "DORY_OK", -1: "DORY_ERR_INVALID_ARG", -2: "DORY_ERR_BAD_CONFIG", -3: "DORY_ERR_K_RANGE",
     -4: "DORY_ERR_K_EXCEEDS_KMAX", -5: "DORY_ERR_CTX_OVERFLOW", -6: "DORY_ERR_BUFFER_TOO_SMALL",
     -7: "DORY_ERR_MISALIGNED", -8: "DORY_ERR_CUDA", -9: "DORY_ERR_DEVICE_TIMEOUT",
-    -10: "DORY_ERR_UNSUPPORTED_ARCH", -11: "DORY_ERR_DEVICE_BOUNDS",
+    -10: "DORY_ERR_UNSUPPORTED_ARCH", -11: "DORY_ERR_DEVICE_BOUNDS", -12: "DORY_ERR_SCRATCH_LIMIT",
 }
 
 # every entry point declared in include/dory.h
@@ -30,8 +30,11 @@ EXPORTS = (
     "dory_workspace_bytes", "dory_prefill", "dory_decode_step", "dory_device_status",
     "dory_last_call_stats", "dory_error_string", "dory_kv_free", "dory_destroy",
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
-    "dory_profile_enable", "dory_profile_read",
+    "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
 )
+
+# size of the library's built-in scratch array (DORY_NOALLOC_SCRATCH_BYTES)
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 KERNEL_KINDS = ("qkvg", "attn", "oproj", "gateup", "down", "row", "kvcommit")
 
@@ -94,6 +97,7 @@ def lib():
             "dory_gemm_bf16": (I, [P, P, P, I, I, I, P]),
             "dory_profile_enable": (I, [P, I]),
             "dory_profile_read": (I, [P, I, P, P]),
+            "dory_mlp_sublayer_noalloc": (I, [P, I, I, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -190,6 +194,23 @@ def dory_attention_sublayer(model, kv, layer, loop, seq, pos0, n_rows, h, ws, ws
 def dory_mlp_sublayer(model, layer, n_rows, h, ws, ws_bytes, stream):
     return check(lib().dory_mlp_sublayer(model, layer, n_rows, h, ws, ws_bytes, stream),
                  "dory_mlp_sublayer")
+
+
+def dory_mlp_sublayer_noalloc(model, layer, n_rows, h, stream):
+    """dory_mlp_sublayer without a workspace: scratch is the library's static array."""
+    return check(lib().dory_mlp_sublayer_noalloc(model, layer, n_rows, h, stream),
+                 "dory_mlp_sublayer_noalloc")
+
+
+def noalloc_max_rows(d_model, d_ff):
+    """Largest n_rows dory_mlp_sublayer_noalloc accepts for this shape."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    n = 0
+    while a256(2 * (n + 1) * d_model) + a256(2 * (n + 1) * d_ff) + a256(4 * (n + 1) * d_model) \
+            <= NOALLOC_SCRATCH_BYTES:
+        n += 1
+    return n
 
 
 def dory_gemm_bf16(A, B, C, M, N, K, stream):

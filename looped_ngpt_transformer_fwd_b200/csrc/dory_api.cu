@@ -15,6 +15,7 @@
 
 #include <algorithm>
 #include <map>
+#include <mutex>
 #include <memory>
 #include <new>
 #include <tuple>
@@ -567,6 +568,7 @@ const char* dory_error_string(int status) {
     case DORY_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
     case DORY_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
     case DORY_ERR_DEVICE_BOUNDS: return "a kernel's bounds check fired";
+    case DORY_ERR_SCRATCH_LIMIT: return "too many rows for the built-in scratch array";
     default: return "unknown status";
   }
 }
@@ -906,3 +908,59 @@ int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, 
 }
 
 }  // extern "C"
+
+// ========================================================== allocation-free MLP
+// Scratch of dory_mlp_sublayer_noalloc, part of the library image: no call
+// ever allocates it.  Host code must not hand the symbol itself to a kernel;
+// it looks up the device address per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[DORY_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device, with that device current).
+void* noalloc_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int dory_mlp_sublayer_noalloc(dory_model* m, int layer, int n_rows, float* h,
+                                         void* stream) {
+  if (!m || !h || n_rows <= 0 || layer < 0 || layer >= m->nb) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(h, 16)) return DORY_ERR_MISALIGNED;
+  const size_t hb_bytes = align_up(size_t(n_rows) * m->d * 2);
+  const size_t a_bytes = align_up(size_t(n_rows) * m->ff * 2);
+  const size_t y_bytes = align_up(size_t(n_rows) * m->d * 4);
+  if (hb_bytes + a_bytes + y_bytes > DORY_NOALLOC_SCRATCH_BYTES) return DORY_ERR_SCRATCH_LIMIT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DORY_ERR_CUDA;
+  if (dev != m->device || dev >= kNoallocMaxDevices) return DORY_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(noalloc_scratch(dev));
+  if (!base) return DORY_ERR_CUDA;
+  CallCtx c;
+  c.m = m; c.kv = nullptr; c.n = n_rows; c.decode = false;
+  c.seq = 0; c.pos0 = 0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = 0; c.k = 1;
+  c.s = static_cast<cudaStream_t>(stream);
+  memset(&c.w, 0, sizeof(c.w));
+  c.w.hb = reinterpret_cast<__nv_bfloat16*>(base);
+  c.w.a = reinterpret_cast<__nv_bfloat16*>(base + hb_bytes);
+  c.w.y = reinterpret_cast<float*>(base + hb_bytes + a_bytes);
+  m->cur_launches = m->cur_sublayers = 0;
+  if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
+  if (mlp_sublayer(c, layer, h, c.w.hb, false, false, nullptr) != cudaSuccess) return DORY_ERR_CUDA;
+  return DORY_OK;
+}

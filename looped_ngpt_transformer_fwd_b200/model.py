@@ -144,6 +144,11 @@ class DoryModel:
                             _stream(stream))
         return h
 
+    def mlp_sublayer_noalloc(self, layer, h, stream=None):
+        """As mlp_sublayer, but the library supplies the scratch (no workspace)."""
+        B.dory_mlp_sublayer_noalloc(self.handle, layer, h.shape[0], _ptr(h), _stream(stream))
+        return h
+
     def device_status(self, stream=None):
         return B.dory_device_status(self.handle, _stream(stream))
 
