@@ -455,10 +455,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--blocks", default=None,
                     help="profiling aid: IN,REC,OUT block counts (same kernel shapes, smaller model)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="profiling aid: decode batch override (same per-sequence work)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    if args.batch and wl["kind"] == "decode":
+        wl["batch"] = args.batch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -506,7 +510,7 @@ def main():
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline and not args.blocks:
+    if rank == 0 and not args.no_cpu_baseline and not args.blocks and not args.batch:
         v, u, sample = oracle_sample(wl, res["prov"])
         cpu = {"value": v, "unit": u, "cores": blas_threads(), "kind": "oracle", "sample": sample}
     if rank == 0:

@@ -59,8 +59,9 @@ struct BlockW {
   float* s_qk = nullptr;
   bool full = false;
   bool recurrent = false;
+  float m_log2 = 0.f;   // static softmax maximum: softmax_scale * log2(e) * max s_qk^2
   // B-operand tensor maps, box rows 128 and 256
-  CUtensorMap tm_qkvg[2], tm_o[2], tm_gu, tm_d[2];
+  CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
 };
 
 struct GraphKey {
@@ -182,7 +183,8 @@ WeightLayout weight_layout(const dory_config* c) {
 }
 
 struct WsLayout {
-  size_t h32, e32, hb, st_in, st_out, q, kf, vf, gate, o, y, a, dacc, dml, total;
+  size_t h32, e32, hb, st_in, st_out, q, kf, vf, gate, o, y, a, dacc, dml, rope_swa, rope_full,
+      part, total;
   int y_rows;
 };
 
@@ -207,13 +209,18 @@ WsLayout ws_layout(const dory_model* m, int T) {
   L.a = take(size_t(T) * ff * 2);
   L.dacc = take(size_t(dec_rows) * m->hq * kMaxDecodeSplits * m->hd * 4);
   L.dml = take(size_t(dec_rows) * m->hq * kMaxDecodeSplits * 2 * 4);
+  L.rope_swa = take(size_t(T) * (m->hd / 2) * 8);
+  L.rope_full = take(size_t(T) * (m->hd / 2) * 8);
+  // K-split partial products of the decode QKVG and gate/up projections
+  L.part = take(size_t(dec_rows) * kMaxKSplits * std::max<size_t>(m->n_qkvg, 2 * ff) * 4);
   L.total = o;
   return L;
 }
 
 struct Ws {
-  float *h32, *e32, *y, *gate, *dacc, *dml;
+  float *h32, *e32, *y, *gate, *dacc, *dml, *part;
   __nv_bfloat16 *hb, *st_in, *st_out, *q, *kf, *vf, *o, *a;
+  float2 *rope_swa, *rope_full;
 };
 
 Ws ws_bind(const dory_model* m, void* base, int T) {
@@ -234,6 +241,9 @@ Ws ws_bind(const dory_model* m, void* base, int T) {
   w.a = reinterpret_cast<__nv_bfloat16*>(b + L.a);
   w.dacc = reinterpret_cast<float*>(b + L.dacc);
   w.dml = reinterpret_cast<float*>(b + L.dml);
+  w.rope_swa = reinterpret_cast<float2*>(b + L.rope_swa);
+  w.rope_full = reinterpret_cast<float2*>(b + L.rope_full);
+  w.part = reinterpret_cast<float*>(b + L.part);
   return w;
 }
 
@@ -325,23 +335,43 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
                                bool commit_after) {
   dory_model* m = c.m;
   const BlockW& W = m->blocks[b];
-  const int bn_q = c.decode ? 128 : 256;
   CUtensorMap tmA;
   if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
-  GemmParams g;
-  g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
-  g.epi = kEpiQKVG;
-  g.q_out = c.w.q; g.k_out = c.w.kf; g.v_out = c.w.vf; g.gate_out = c.w.gate;
-  g.n_q_heads = m->hq; g.n_kv_heads = m->hkv;
-  g.s_qk = W.s_qk;
-  g.inv_freq = W.full ? m->inv_freq_full : m->inv_freq_swa;
-  g.norm_eps = m->cfg.norm_eps;
-  g.pos0 = c.decode ? 0 : c.pos0;
-  g.d_pos = c.decode ? c.dpos : nullptr;
-  g.status = m->status;
-  {
+  const float2* rope = W.full ? c.w.rope_full : c.w.rope_swa;
+  if (c.decode) {
+    // few rows: spread the weight stream over the SMs with K splits, then a
+    // row kernel applies RoPE / QK-norm / gates to the summed partials
+    GemmParams g;
+    g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
+    g.epi = kEpiStoreF32;
+    g.k_splits = pick_k_splits(m, c.n, m->n_qkvg, 128, m->d);
+    g.out_f32 = c.w.part; g.ld_out = m->n_qkvg; g.split_stride = size_t(c.n) * m->n_qkvg;
+    g.status = m->status;
+    {
+      Launch L(m, c.s, DORY_KK_QKVG);
+      DORY_TRY(launch_gemm(tmA, W.tm_qkvg[0], g, 128, m->hd, m->num_sms, c.s));
+    }
+    QkvgPostParams pp;
+    pp.part = c.w.part; pp.splits = g.k_splits; pp.split_stride = g.split_stride;
+    pp.rows = c.n; pp.n_q_heads = m->hq; pp.n_kv_heads = m->hkv; pp.hd = m->hd;
+    pp.s_qk = W.s_qk; pp.rope = rope; pp.norm_eps = m->cfg.norm_eps;
+    pp.q_out = c.w.q; pp.k_out = c.w.kf; pp.v_out = c.w.vf; pp.gate_out = c.w.gate;
+    {
+      Launch L(m, c.s, DORY_KK_QKVG);
+      DORY_TRY(launch_qkvg_post(pp, c.s));
+    }
+  } else {
+    GemmParams g;
+    g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
+    g.epi = kEpiQKVG;
+    g.q_out = c.w.q; g.k_out = c.w.kf; g.v_out = c.w.vf; g.gate_out = c.w.gate;
+    g.n_q_heads = m->hq; g.n_kv_heads = m->hkv;
+    g.s_qk = W.s_qk;
+    g.rope = rope;
+    g.norm_eps = m->cfg.norm_eps;
+    g.status = m->status;
     Launch L(m, c.s, DORY_KK_QKVG);
-    DORY_TRY(launch_gemm(tmA, W.tm_qkvg[bn_q == 256], g, bn_q, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_gemm(tmA, W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   const KvLayerView view = kv_view(c.kv, b, loop);
@@ -369,11 +399,19 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
       DORY_TRY(launch_decode_attention(a, c.s));
     }
   } else {
-    PrefillAttnParams a;
-    a.q = c.w.q; a.k_new = c.w.kf; a.v_new = c.w.vf; a.gate = c.w.gate; a.out = c.w.o;
-    a.kv = view; a.seq = c.seq; a.pos0 = c.pos0; a.n = c.n; a.n_q_heads = m->hq;
-    a.window = window; a.scale_log2 = scale_log2; a.status = m->status;
-    {
+    if (prefill_attention_tc_supported(m->hd, c.pos0, window, W.m_log2)) {
+      PrefillAttnTcParams a;
+      a.gate = c.w.gate; a.out = c.w.o; a.n = c.n; a.pos0 = c.pos0; a.seq = c.seq;
+      a.n_q_heads = m->hq; a.n_kv = m->hkv; a.cap = view.cap; a.window = window;
+      a.last_pos = c.pos0 + c.n - 1; a.scale_log2 = scale_log2; a.m_log2 = W.m_log2;
+      a.status = m->status;
+      Launch L(m, c.s, DORY_KK_ATTN);
+      DORY_TRY(launch_prefill_attention_tc(a, c.w.q, c.w.kf, c.w.vf, view, c.s));
+    } else {
+      PrefillAttnParams a;
+      a.q = c.w.q; a.k_new = c.w.kf; a.v_new = c.w.vf; a.gate = c.w.gate; a.out = c.w.o;
+      a.kv = view; a.seq = c.seq; a.pos0 = c.pos0; a.n = c.n; a.n_q_heads = m->hq;
+      a.window = window; a.scale_log2 = scale_log2; a.status = m->status;
       Launch L(m, c.s, DORY_KK_ATTN);
       DORY_TRY(launch_prefill_attention(a, c.s));
     }
@@ -419,14 +457,28 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   const BlockW& W = m->blocks[b];
   CUtensorMap tmA;
   if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
-  GemmParams g;
-  g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
-  g.epi = kEpiSwiGLU;
-  g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
-  g.status = m->status;
-  {
+  if (c.decode) {
+    GemmParams g;
+    g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
+    g.epi = kEpiStoreF32;
+    g.k_splits = pick_k_splits(m, c.n, 2 * m->ff, 128, m->d);
+    g.out_f32 = c.w.part; g.ld_out = 2 * m->ff; g.split_stride = size_t(c.n) * 2 * m->ff;
+    g.status = m->status;
+    {
+      Launch L(m, c.s, DORY_KK_GATEUP);
+      DORY_TRY(launch_gemm(tmA, W.tm_gu[0], g, 128, m->hd, m->num_sms, c.s));
+    }
     Launch L(m, c.s, DORY_KK_GATEUP);
-    DORY_TRY(launch_gemm(tmA, W.tm_gu, g, 256, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_swiglu_post(c.w.part, g.k_splits, g.split_stride, c.n, m->ff,
+                                m->cfg.gate_scale, c.w.a, c.s));
+  } else {
+    GemmParams g;
+    g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
+    g.epi = kEpiSwiGLU;
+    g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
+    g.status = m->status;
+    Launch L(m, c.s, DORY_KK_GATEUP);
+    DORY_TRY(launch_gemm(tmA, W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   CUtensorMap tmAct;
@@ -457,6 +509,20 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   return cudaSuccess;
 }
 
+// (cos, sin) tables of this call's positions for both RoPE bases
+cudaError_t enqueue_rope_tables(CallCtx& c) {
+  dory_model* m = c.m;
+  const int pos0 = c.decode ? 0 : c.pos0;
+  const int32_t* dpos = c.decode ? c.dpos : nullptr;
+  {
+    Launch L(m, c.s, DORY_KK_ROW);
+    DORY_TRY(launch_rope_table(m->inv_freq_swa, m->hd, c.n, pos0, dpos, c.w.rope_swa, c.s));
+  }
+  Launch L(m, c.s, DORY_KK_ROW);
+  DORY_TRY(launch_rope_table(m->inv_freq_full, m->hd, c.n, pos0, dpos, c.w.rope_full, c.s));
+  return cudaSuccess;
+}
+
 // The whole stack for one call, enqueued on c.s.
 cudaError_t enqueue_stack(CallCtx& c, const __nv_bfloat16* src, __nv_bfloat16* dst) {
   dory_model* m = c.m;
@@ -466,6 +532,7 @@ cudaError_t enqueue_stack(CallCtx& c, const __nv_bfloat16* src, __nv_bfloat16* d
     Launch L(m, c.s, DORY_KK_ROW);
     DORY_TRY(launch_load_rows(src, c.w.h32, c.w.hb, c.n, m->d, c.s));
   }
+  DORY_TRY(enqueue_rope_tables(c));
   const bool last_loop = c.kv->mode == DORY_KV_LAST_LOOP;
   for (int b = 0; b < n_in; ++b) {
     DORY_TRY(attention_sublayer(c, b, 1, c.w.h32, c.w.hb, true));
@@ -668,8 +735,23 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
       ok &= make_tmap_bf16(&W.tm_o[i], W.wo, d, da, box);
       ok &= make_tmap_bf16(&W.tm_d[i], W.wd, d, F, box);
     }
-    ok &= make_tmap_bf16(&W.tm_gu, W.wgu, 2 * F, d, 256);
+    ok &= make_tmap_bf16(&W.tm_gu[0], W.wgu, 2 * F, d, 128);
+    ok &= make_tmap_bf16(&W.tm_gu[1], W.wgu, 2 * F, d, 256);
     if (!ok) return DORY_ERR_CUDA;
+  }
+  // static softmax maxima from the packed s_qk vectors (one-time host read)
+  {
+    std::vector<float> sq(size_t(m->nb) * hd);
+    for (int b = 0; b < m->nb; ++b)
+      if (cudaMemcpyAsync(sq.data() + size_t(b) * hd, m->blocks[b].s_qk, hd * 4,
+                          cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return DORY_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DORY_ERR_CUDA;
+    for (int b = 0; b < m->nb; ++b) {
+      float mx = 0.f;
+      for (size_t i = 0; i < hd; ++i) mx = std::max(mx, sq[size_t(b) * hd + i] * sq[size_t(b) * hd + i]);
+      m->blocks[b].m_log2 = cfg->softmax_scale * 1.4426950408889634f * mx;
+    }
   }
   if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
     return DORY_ERR_CUDA;
@@ -870,6 +952,7 @@ int dory_attention_sublayer(dory_model* m, dory_kv* kv, int layer, int loop, int
   c.k = 1; c.s = static_cast<cudaStream_t>(stream);
   m->cur_launches = m->cur_sublayers = 0;
   if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
+  if (enqueue_rope_tables(c) != cudaSuccess) return DORY_ERR_CUDA;
   if (attention_sublayer(c, layer, kv->loops[layer] > 1 ? loop : 1, h, c.w.hb, true) != cudaSuccess)
     return DORY_ERR_CUDA;
   return DORY_OK;

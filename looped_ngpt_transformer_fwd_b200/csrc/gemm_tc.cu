@@ -39,8 +39,6 @@ struct GemmCfg {
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
 };
 
-constexpr double kTwoPi = 6.283185307179586476925286766559;
-
 // --------------------------------------------------------------- epilogues
 __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32], int valid) {
   if (valid >= 32) {
@@ -120,20 +118,18 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t tad
   }
   __nv_bfloat16* dst;
   if (col0 < k_end) {
-    // RoPE (pairs i, i + HD/2) at this row's absolute position, then the
+    // RoPE (pairs i, i + HD/2) with this row's (cos, sin) table, then the
     // per-head L2 norm and the learned per-dimension scale s_qk.
-    const int pos = p.d_pos ? p.d_pos[row] : p.pos0 + row;
-    const double dpos = static_cast<double>(pos);
+    const float4* rt = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(row) * (HD / 2));
 #pragma unroll
-    for (int i = 0; i < HD / 2; ++i) {
-      const double ang = dpos * p.inv_freq[i];
-      const double turns = rint(ang * (1.0 / kTwoPi));
-      const float r = static_cast<float>(fma(-turns, kTwoPi, ang));
-      float sn, cs;
-      sincosf(r, &sn, &cs);
-      const float a = x[i], b = x[i + HD / 2];
-      x[i] = a * cs - b * sn;
-      x[i + HD / 2] = b * cs + a * sn;
+    for (int i = 0; i < HD / 2; i += 2) {
+      const float4 cs = rt[i / 2];   // cos_i, sin_i, cos_{i+1}, sin_{i+1}
+      const float a0 = x[i], b0 = x[i + HD / 2];
+      const float a1 = x[i + 1], b1 = x[i + 1 + HD / 2];
+      x[i] = a0 * cs.x - b0 * cs.y;
+      x[i + HD / 2] = b0 * cs.x + a0 * cs.y;
+      x[i + 1] = a1 * cs.z - b1 * cs.w;
+      x[i + 1 + HD / 2] = b1 * cs.z + a1 * cs.w;
     }
     float ss = 0.f;
 #pragma unroll
@@ -315,7 +311,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int ks = rest / n_tiles;
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
+      // warp-uniform: the TMEM loads below are warp-collective
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status))) break;
       tc_fence_after();
       const int row = mt * kBM + quad * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;

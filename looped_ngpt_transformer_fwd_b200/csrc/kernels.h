@@ -34,10 +34,8 @@ struct GemmParams {
   float* gate_out = nullptr;        // [M, Hq]
   int n_q_heads = 0, n_kv_heads = 0;
   const float* s_qk = nullptr;       // [hd]
-  const double* inv_freq = nullptr;  // [hd/2] RoPE inverse frequencies of this layer
+  const float2* rope = nullptr;      // [M][hd/2] (cos, sin) of each row's angles, this layer's base
   float norm_eps = 1e-20f;
-  int pos0 = 0;                      // row r sits at position pos0 + r ...
-  const int32_t* d_pos = nullptr;    // ... or at d_pos[r] when given
   uint32_t* status = nullptr;
 };
 
@@ -50,6 +48,33 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 // head_dim (64 or 128) selects the QKVG epilogue instantiation.
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int BN, int head_dim, int num_sms, cudaStream_t s);
+
+// RoPE (cos, sin) table [rows][hd/2] for row r at position pos0 + r (or
+// d_pos[r]): angle = pos * inv_freq[i] in float64, reduced mod 2*pi, then
+// sincosf.
+cudaError_t launch_rope_table(const double* inv_freq, int hd, int rows, int pos0,
+                              const int32_t* d_pos, float2* out, cudaStream_t s);
+
+// K-split QKVG post-processing (decode): sum the split partial products
+// [splits][rows][n_qkvg], then the same per-head RoPE / L2 norm / s_qk / gate
+// steps as the fused kEpiQKVG epilogue.
+struct QkvgPostParams {
+  const float* part = nullptr;
+  int splits = 1;
+  size_t split_stride = 0;   // elements
+  int rows = 0, n_q_heads = 0, n_kv_heads = 0, hd = 0;
+  const float* s_qk = nullptr;
+  const float2* rope = nullptr;
+  float norm_eps = 1e-20f;
+  __nv_bfloat16 *q_out = nullptr, *k_out = nullptr, *v_out = nullptr;
+  float* gate_out = nullptr;
+};
+cudaError_t launch_qkvg_post(const QkvgPostParams& p, cudaStream_t s);
+
+// K-split gate/up post-processing (decode): columns are the interleaved
+// weight rows (128 gate, 128 up, ...); a = SiLU(gate_scale * g) * u.
+cudaError_t launch_swiglu_post(const float* part, int splits, size_t split_stride, int rows,
+                               int d_ff, float gate_scale, __nv_bfloat16* out, cudaStream_t s);
 
 // ----------------------------------------------------------------- rows
 struct RowUpdateParams {
@@ -110,6 +135,24 @@ struct PrefillAttnParams {
   uint32_t* status = nullptr;
 };
 cudaError_t launch_prefill_attention(const PrefillAttnParams& p, cudaStream_t s);
+
+// Tensor-core (tcgen05) prefill attention for head_dim 128 with a static
+// softmax maximum m_log2 = softmax_scale * log2(e) * max_i s_qk[i]^2.
+struct PrefillAttnTcParams {
+  const float* gate = nullptr;          // [n, Hq]
+  __nv_bfloat16* out = nullptr;         // [n, Hq*hd]
+  int n = 0, pos0 = 0, seq = 0;
+  int n_q_heads = 0, n_kv = 0;
+  int cap = 0;                          // cache slots per (seq, head)
+  int window = 0;                       // 0 = full attention
+  int last_pos = 0;                     // pos0 + n - 1
+  float scale_log2 = 0.f, m_log2 = 0.f;
+  uint32_t* status = nullptr;
+};
+bool prefill_attention_tc_supported(int head_dim, int pos0, int window, float m_log2);
+cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv_bfloat16* q,
+                                        const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                        const KvLayerView& kv, cudaStream_t s);
 
 struct DecodeAttnParams {
   const __nv_bfloat16* q = nullptr;     // [B, Hq, hd]

@@ -145,7 +145,107 @@ __global__ void kv_commit_kernel(const KvLayerView kv, const __nv_bfloat16* __re
   reinterpret_cast<uint4*>(kv.v_base + dst)[0] = reinterpret_cast<const uint4*>(v_new + src)[0];
 }
 
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+__global__ void rope_table_kernel(const double* __restrict__ inv_freq, int half, int rows,
+                                  int pos0, const int32_t* __restrict__ d_pos,
+                                  float2* __restrict__ out) {
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= rows * half) return;
+  const int r = id / half, i = id % half;
+  const int pos = d_pos ? d_pos[r] : pos0 + r;
+  const double ang = static_cast<double>(pos) * inv_freq[i];
+  const double turns = rint(ang * (1.0 / kTwoPi));
+  const float red = static_cast<float>(fma(-turns, kTwoPi, ang));
+  float sn, cs;
+  sincosf(red, &sn, &cs);
+  out[id] = make_float2(cs, sn);
+}
+
+// one CTA per (row, head group); thread i owns dimensions i and i + hd/2
+__global__ void qkvg_post_kernel(const QkvgPostParams p) {
+  __shared__ float red[32];
+  const int r = blockIdx.x, g = blockIdx.y, i = threadIdx.x;
+  const int hd = p.hd, half = hd / 2;
+  const int n_qkvg = (p.n_q_heads + 2 * p.n_kv_heads) * hd + p.n_q_heads;
+  const float* row = p.part + static_cast<size_t>(r) * n_qkvg;
+  const int n_heads = p.n_q_heads + 2 * p.n_kv_heads;
+  if (g == n_heads) {
+    // gate logits
+    for (int j = i; j < p.n_q_heads; j += blockDim.x) {
+      float v = 0.f;
+      for (int s = 0; s < p.splits; ++s) v += row[s * p.split_stride + n_heads * hd + j];
+      p.gate_out[static_cast<size_t>(r) * p.n_q_heads + j] = sigmoidf_(v);
+    }
+    return;
+  }
+  float a = 0.f, b = 0.f;
+  for (int s = 0; s < p.splits; ++s) {
+    a += row[s * p.split_stride + g * hd + i];
+    b += row[s * p.split_stride + g * hd + i + half];
+  }
+  const bool is_v = g >= p.n_q_heads + p.n_kv_heads;
+  if (!is_v) {
+    const float2 cs = p.rope[static_cast<size_t>(r) * half + i];
+    const float a2 = a * cs.x - b * cs.y;
+    const float b2 = b * cs.x + a * cs.y;
+    const float inv = rsqrtf(fmaxf(block_sum(a2 * a2 + b2 * b2, red), p.norm_eps));
+    a = a2 * inv * p.s_qk[i];
+    b = b2 * inv * p.s_qk[i + half];
+  }
+  __nv_bfloat16* dst;
+  if (g < p.n_q_heads)
+    dst = p.q_out + (static_cast<size_t>(r) * p.n_q_heads + g) * hd;
+  else if (!is_v)
+    dst = p.k_out + (static_cast<size_t>(r) * p.n_kv_heads + (g - p.n_q_heads)) * hd;
+  else
+    dst = p.v_out + (static_cast<size_t>(r) * p.n_kv_heads + (g - p.n_q_heads - p.n_kv_heads)) * hd;
+  dst[i] = __float2bfloat16_rn(a);
+  dst[i + half] = __float2bfloat16_rn(b);
+}
+
+__global__ void swiglu_post_kernel(const float* __restrict__ part, int splits, size_t split_stride,
+                                   int rows, int d_ff, float gate_scale,
+                                   __nv_bfloat16* __restrict__ out) {
+  const size_t id = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (id >= static_cast<size_t>(rows) * d_ff) return;
+  const int r = static_cast<int>(id / d_ff), c = static_cast<int>(id % d_ff);
+  const size_t gcol = static_cast<size_t>(c / 128) * 256 + (c % 128);
+  const float* row = part + static_cast<size_t>(r) * 2 * d_ff;
+  float g = 0.f, u = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    g += row[s * split_stride + gcol];
+    u += row[s * split_stride + gcol + 128];
+  }
+  g *= gate_scale;
+  out[id] = __float2bfloat16_rn(g * sigmoidf_(g) * u);
+}
+
 }  // namespace
+
+cudaError_t launch_rope_table(const double* inv_freq, int hd, int rows, int pos0,
+                              const int32_t* d_pos, float2* out, cudaStream_t s) {
+  const int n = rows * (hd / 2);
+  if (n <= 0) return cudaSuccess;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(inv_freq, hd / 2, rows, pos0, d_pos, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qkvg_post(const QkvgPostParams& p, cudaStream_t s) {
+  if (p.rows <= 0) return cudaSuccess;
+  dim3 grid(p.rows, p.n_q_heads + 2 * p.n_kv_heads + 1);
+  qkvg_post_kernel<<<grid, p.hd / 2, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_post(const float* part, int splits, size_t split_stride, int rows,
+                               int d_ff, float gate_scale, __nv_bfloat16* out, cudaStream_t s) {
+  const size_t n = static_cast<size_t>(rows) * d_ff;
+  if (n == 0) return cudaSuccess;
+  swiglu_post_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      part, splits, split_stride, rows, d_ff, gate_scale, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s) {
   if (p.d % 4 != 0 || p.rows < 0) return cudaErrorInvalidValue;

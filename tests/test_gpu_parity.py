@@ -244,3 +244,94 @@ def test_kernel_profiling_counts_every_launch(tiny):
     assert sum(n for _, n in prof.values()) == launches
     assert prof["gateup"][1] == prof["down"][1] == sub // 2
     assert all(t > 0 for t, n in prof.values() if n)
+
+
+# ------------------------------------------------------------------ head_dim 128
+# (d 512, 4/2 heads of 128, window 64): prefill attention runs on the tcgen05
+# kernel whenever pos0 and the window are multiples of 64, else on the
+# mma.sync kernel; both must match the oracle.
+HD128 = dict(d_model=512, n_q_heads=4, n_kv_heads=2, head_dim=128, d_ff=1024, window=64,
+             softmax_scale=float(np.sqrt(128.0)))
+
+
+@pytest.fixture(scope="module")
+def hd128():
+    return build("tiny", seed=7, variant="random", **HD128)
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_hd128_prefill_matches_oracle(hd128, mode):
+    cfg, prov, model = hd128
+    x, h = inputs(cfg, 51, 300)
+    kv = model.kv_cache(mode, 1, 400, k_max=2)
+    out = model.prefill(kv, x, 2)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, mode, k_max=2))
+    assert_parity(to_np(out), ref, what=f"hd128 prefill {mode}")
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_hd128_chunked_prefill_and_decode(hd128, mode):
+    """Chunks at multiples of 64 (tensor-core attention reading cached tiles and
+    ring slots), one unaligned chunk (mma.sync kernel), then decode steps."""
+    cfg, prov, model = hd128
+    k = 2
+    x, h = inputs(cfg, 52, 420)
+    kv = model.kv_cache(mode, 2, 480, k_max=2)
+    ocache = oracle_cache(cfg, mode, k_max=2)
+    orc = oracle(cfg, prov)
+    seq = 1
+    for a, b in ((0, 128), (128, 192), (192, 330), (330, 405), (405, 416)):
+        out = model.prefill(kv, x[a:b], k, seq=seq, pos0=a)
+        torch.cuda.synchronize()
+        ref = orc.forward(h[a:b], a, k, ocache, seq=seq)
+        assert_parity(to_np(out), ref, what=f"hd128 chunk {a}:{b} {mode}")
+    for p in range(416, 420):
+        d_seq = torch.tensor([seq], dtype=torch.int32, device="cuda")
+        d_pos = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d_seq, d_pos, 479, k)
+        ref = orc.decode(h[p:p + 1], [seq], [p], k, ocache)
+        assert_parity(to_np(out), ref, what=f"hd128 decode {p} {mode}")
+    assert model.device_status() == 0
+
+
+@pytest.mark.parametrize("layer", [0, 1])      # SWA (W = 64), full
+def test_hd128_attention_sublayer_alpha_one_is_tight(layer):
+    """alpha = 1 makes the sublayer output Norm(o W_o^T) itself, so the attention
+    output is compared almost undiluted: a key added or dropped at a mask edge
+    (one of ~64) would move it by ~1.5 %, far above the bf16 error."""
+    from tests.oracle_util import modified
+    from oracle import weights_from_generator
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from synthetic import load_config
+    cfg = load_config("tiny", **HD128)
+    base = weights_from_generator(cfg, 8, "random")
+
+    def alpha_one(b, w):
+        w["alpha_attn"][:] = 1.0
+    prov = modified(base, alpha_one)
+
+    def as_generator_format(b):
+        w = prov(b)
+        from synthetic import f32_to_bf16_bits
+        out = {}
+        for k_, v in w.items():
+            if k_ in ("alpha_attn", "alpha_mlp", "s_qk"):
+                out[k_] = v.astype(np.float32)
+            else:
+                out[k_] = f32_to_bf16_bits(v.astype(np.float32))
+        return out
+    model = DoryModel(cfg, as_generator_format)
+    _, h = inputs(cfg, 53, 320)
+    kv = model.kv_cache("last_loop", 1, 384)
+    ocache = oracle_cache(cfg, "last_loop")
+    orc = oracle(cfg, as_generator_format)
+    for pos0, n in ((0, 192), (192, 128)):
+        ht = torch.from_numpy(h[pos0:pos0 + n].astype(np.float32)).cuda()
+        model.attention_sublayer(kv, layer, ht, loop=1, seq=0, pos0=pos0)
+        torch.cuda.synchronize()
+        ref = orc.attention_sublayer(layer, h[pos0:pos0 + n], pos0, 0, 1, ocache)
+        assert_parity(to_np(ht), ref, tol_abs=1e-2, tol_cos=0.99995,
+                      what=f"alpha=1 attention layer {layer} @{pos0}")
+    model.close()
