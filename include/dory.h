@@ -185,6 +185,9 @@ DORY_API int dory_last_call_stats(const dory_model* m, int* kernel_launches, int
 
 DORY_API const char* dory_error_string(int status);
 
+/* dory_kv_free releases the cache handle (not its buffer) and the captured
+ * graphs that refer to it.  dory_destroy releases the model handle and its
+ * graphs; caches still bound to it become unusable but may still be freed. */
 DORY_API void dory_kv_free(dory_kv* kv);
 DORY_API void dory_destroy(dory_model* m);
 

@@ -268,11 +268,20 @@ cudaError_t launch_decode_impl(const DecodeAttnParams& p, cudaStream_t s) {
   kern<<<grid, kDecThreads, smem, s>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<HD><<<dim3(p.n_q_heads, p.batch), HD, 0, s>>>(p, n_splits);
-  return cudaGetLastError();
+  return launch_decode_combine(p, n_splits, s);
 }
 
 }  // namespace
+
+cudaError_t launch_decode_combine(const DecodeAttnParams& p, int n_splits, cudaStream_t s) {
+  if (p.kv.hd == 128)
+    decode_combine_kernel<128><<<dim3(p.n_q_heads, p.batch), 128, 0, s>>>(p, n_splits);
+  else if (p.kv.hd == 64)
+    decode_combine_kernel<64><<<dim3(p.n_q_heads, p.batch), 64, 0, s>>>(p, n_splits);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
 
 int decode_attention_splits(int max_pos, int window, int split_keys) {
   const int max_keys = window > 0 ? (max_pos + 1 < window ? max_pos + 1 : window) : max_pos + 1;

@@ -14,8 +14,10 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
+#include <set>
 #include <memory>
 #include <new>
 #include <tuple>
@@ -66,7 +68,9 @@ struct BlockW {
 
 struct GraphKey {
   int phase, k, n, seq, pos0, max_pos, prof;
-  const void *src, *dst, *ws, *kv, *dseq, *dpos;
+  const void *src, *dst, *ws;
+  uint64_t kv;              // unique id of the KV cache (handles may be recycled)
+  const void *dseq, *dpos;
   bool operator<(const GraphKey& o) const {
     return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos) <
            std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.prof, o.src, o.dst, o.ws, o.kv,
@@ -119,10 +123,12 @@ struct dory_model {
   bool profile = false;
   std::vector<Mark>* cur_marks = nullptr;      // marks of the graph being captured
   const std::vector<Mark>* last_marks = nullptr;
+  std::set<dory_kv*> caches;                   // live KV caches bound to this model
 };
 
 struct dory_kv {
   dory_model* m = nullptr;
+  uint64_t uid = 0;
   int mode = 0, max_seqs = 0, max_ctx = 0, k_max = 1;
   uint8_t* buf = nullptr;
   size_t bytes = 0;
@@ -396,7 +402,10 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     {
       Launch L(m, c.s, DORY_KK_ATTN);
       ++m->cur_launches;   // split-KV kernel + combine kernel
-      DORY_TRY(launch_decode_attention(a, c.s));
+      if (decode_attention_tma_supported(m->hd, window, m->hq / m->hkv) && 2.f * W.m_log2 < 120.f)
+        DORY_TRY(launch_decode_attention_tma(a, W.m_log2, c.s));
+      else
+        DORY_TRY(launch_decode_attention(a, c.s));
     }
   } else {
     if (prefill_attention_tc_supported(m->hd, c.pos0, window, W.m_log2)) {
@@ -796,6 +805,9 @@ int dory_kv_alloc(dory_model* m, int mode, int max_seqs, int max_ctx, int k_max,
     off += size_t(loops) * max_seqs * cap * per_pos;
   }
   kv->seq_k.assign(max_seqs, 0);
+  static std::atomic<uint64_t> next_uid{0};
+  kv->uid = ++next_uid;
+  m->caches.insert(kv.get());
   *out = kv.release();
   return DORY_OK;
 }
@@ -842,7 +854,7 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv, nullptr, nullptr};
+  GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv->uid, nullptr, nullptr};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -874,7 +886,7 @@ int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv, d_seq, d_pos};
+  GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv->uid, d_seq, d_pos};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -929,11 +941,28 @@ int dory_profile_read(dory_model* m, int kind, float* total_ms, int* launches) {
   return DORY_OK;
 }
 
-void dory_kv_free(dory_kv* kv) { delete kv; }
+void dory_kv_free(dory_kv* kv) {
+  if (!kv) return;
+  if (dory_model* m = kv->m) {
+    // graphs captured for this cache bake its addresses: drop them
+    for (auto it = m->graphs.begin(); it != m->graphs.end();) {
+      if (it->first.kv == kv->uid) {
+        if (m->last_marks == &it->second.marks) m->last_marks = nullptr;
+        destroy_entry(it->second);
+        it = m->graphs.erase(it);
+      } else {
+        ++it;
+      }
+    }
+    m->caches.erase(kv);
+  }
+  delete kv;
+}
 
 void dory_destroy(dory_model* m) {
   if (!m) return;
   for (auto& g : m->graphs) destroy_entry(g.second);
+  for (dory_kv* kv : m->caches) kv->m = nullptr;   // caches outliving the model stay freeable
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;
 }

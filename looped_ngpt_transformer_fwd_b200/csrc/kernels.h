@@ -171,5 +171,11 @@ struct DecodeAttnParams {
 };
 int decode_attention_splits(int max_pos, int window, int split_keys);
 cudaError_t launch_decode_attention(const DecodeAttnParams& p, cudaStream_t s);
+// merge the split partials (acc, (m, l)) of every (sequence, head), gate, store
+cudaError_t launch_decode_combine(const DecodeAttnParams& p, int n_splits, cudaStream_t s);
+// TMA-fed decode attention with a static softmax maximum (head_dim 128)
+bool decode_attention_tma_supported(int head_dim, int window, int group);
+int decode_attention_tma_splits(int max_pos, int window, int* split_tiles);
+cudaError_t launch_decode_attention_tma(const DecodeAttnParams& p, float m_log2, cudaStream_t s);
 
 }  // namespace dory

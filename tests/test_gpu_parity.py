@@ -335,3 +335,22 @@ def test_hd128_attention_sublayer_alpha_one_is_tight(layer):
         assert_parity(to_np(ht), ref, tol_abs=1e-2, tol_cos=0.99995,
                       what=f"alpha=1 attention layer {layer} @{pos0}")
     model.close()
+
+
+def test_recycled_cache_handles_do_not_reuse_stale_graphs(tiny):
+    """Caches freed and re-created with another mode may land on the same handle
+    and buffer addresses; every call must still run the graph of its own cache."""
+    import gc
+    cfg, prov, model = tiny
+    x, h = inputs(cfg, 22, 80)
+    for mode in ("per_loop", "last_loop", "per_loop", "last_loop"):
+        kv = model.kv_cache(mode, 1, 96, k_max=2)
+        ocache = oracle_cache(cfg, mode, k_max=2)
+        orc = oracle(cfg, prov)
+        for a, b in ((0, 40), (40, 80)):
+            out = model.prefill(kv, x[a:b], 2, pos0=a)
+            torch.cuda.synchronize()
+            assert_parity(to_np(out), orc.forward(h[a:b], a, 2, ocache), what=f"{mode} {a}:{b}")
+        kv.free()
+        del kv
+        gc.collect()
