@@ -14,16 +14,17 @@
 // underflow of the smallest weight in fp32/bf16); otherwise it keeps the
 // online-softmax kernel.
 //
-// One CTA = two adjacent 128-query tiles of one query head, sharing every K/V
-// tile.  Warp 0 issues TMA loads (both Q tiles once, then 64-key K/V tiles
-// through a 3-stage ring, from the layer's cache for positions below pos0 and
-// from this call's fresh K/V otherwise), warp 1 owns TMEM and issues the MMAs
-// (per query tile: S = Q K^T into one of two 64-column TMEM buffers, O += P V
-// into 128 columns), and two softmax warpgroups (warps 2-5 and 6-9, one per
-// query tile, so two warps share each SM sub-partition and hide each other's
-// latency) turn S into P (one query row per thread: mask, exp2, row sum, bf16
-// store to shared memory) and finally write gate * O / l.  Every wait is
-// bounded.
+// One CTA = 128 queries of one query head; 128-key K/V tiles.  Warp 0 issues
+// TMA loads of K/V tiles through a 3-stage ring (from the layer's cache for
+// positions below pos0, from this call's fresh K/V otherwise).  Q is staged
+// once into TMEM by the softmax warps.  Warp 1 owns TMEM and issues the MMAs,
+// both with the A operand read from TMEM: S = Q K^T (N = 128 keys) into one of
+// two 128-column buffers, and O += P V with P written over S.  Each MMA then
+// reads a single operand (K or V, 4 KB) from shared memory, which keeps the
+// tensor core's operand traffic within its shared-memory bandwidth.  Sixteen
+// softmax warps (row quadrant x key quarter) turn S into P = exp2(...) in
+// place (mask, exp2 on the MUFU and FMA pipes, row sums) and finally write
+// gate * O / l.  Every wait is bounded.
 #include <math.h>
 
 #include "common.cuh"
@@ -33,21 +34,22 @@ namespace dory {
 
 namespace {
 
-constexpr int kQ = 128;           // queries per query tile
-constexpr int kKT = 64;           // keys per tile
+constexpr int kQ = 128;           // queries per CTA (one TMEM lane each)
+constexpr int kKT = 128;          // keys per tile
 constexpr int kHD = 128;
 constexpr int kStages = 3;
-constexpr int kGroups = 2;        // query tiles (and softmax warpgroups) per CTA
-constexpr int kThreads = 64 + kGroups * 128;
-constexpr int kQBytes = kQ * kHD * 2;                 // 32 KB per query tile
-constexpr int kSubKV = kKT * 64 * 2;                  // 8 KB: 64 keys x 64 dims
-constexpr int kStageBytes = 4 * kSubKV;               // K (2 sub-tiles) + V (2 sub-tiles)
-constexpr int kPBytes = kQ * kKT * 2;                 // 16 KB
-constexpr int kOffKV = kGroups * kQBytes;
-constexpr int kOffP = kOffKV + kStages * kStageBytes;
-constexpr int kOffBar = kOffP + kGroups * 2 * kPBytes;
+constexpr int kSoftmaxWarps = 16; // 4 row quadrants x 4 column quarters of 32 keys
+constexpr int kSoftThreads = 32 * kSoftmaxWarps;
+constexpr int kThreads = 64 + kSoftThreads;
+constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 keys x 64 dims (one TMA box)
+constexpr int kStageBytes = 4 * kSub;                 // K (2 sub-tiles) + V (2 sub-tiles)
+constexpr int kOffKV = 0;
+constexpr int kOffBar = kOffKV + kStages * kStageBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
-constexpr uint32_t kTmemCols = 512;                   // per group: S0 | S1 | O (256 columns)
+constexpr int kSBufs = 2;                             // S/P buffers in TMEM
+constexpr uint32_t kTmemCols = 512;                   // S0 | S1 | O (128 columns each) | Q (64)
+constexpr uint32_t kColO = kSBufs * kKT;
+constexpr uint32_t kColQ = kColO + kHD;
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
@@ -71,10 +73,55 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint3
   return d;
 }
 
+// tcgen05.mma with the A operand in TMEM (K-major rows = TMEM lanes, two bf16
+// per 32-bit column) and B from shared memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for -126 < x <= 0 on the FMA pipe, to share the exponential work with the
+// MUFU unit: Cody-Waite style reduction x = n + f with n = round(x) (the
+// 1.5 * 2^23 shifter), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients were fitted here to minimise the relative error on that
+// interval (max 7.5e-5, far below the bf16 rounding of P); 2^n added to the
+// exponent field.
+__device__ __forceinline__ float ex2_poly(float x) {
+  const float shifter = 12582912.0f;
+  const float t = x + shifter;
+  const float f = x - (t - shifter);
+  float p = fmaf(0.05517113f, f, 0.24261008f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.9999281f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -84,28 +131,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Query-tile geometry shared by every role of the CTA.
-struct QTile {
-  int m0, rows, q_lo, q_hi, kb, ke;   // key tiles kb..ke (inclusive)
-  bool active;
-};
-
-__device__ __forceinline__ QTile make_qtile(const PrefillAttnTcParams& p, int qblock) {
-  QTile t;
-  t.m0 = qblock * kQ;
-  t.rows = min(kQ, p.n - t.m0);
-  t.active = t.rows > 0;
-  t.q_lo = p.pos0 + t.m0;
-  t.q_hi = t.q_lo + max(t.rows, 1) - 1;
-  const int key_lo = p.window > 0 ? max(0, t.q_lo - p.window + 1) : 0;
-  t.kb = key_lo / kKT;
-  t.ke = t.q_hi / kKT;
-  return t;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                           const __grid_constant__ CUtensorMap tmKnew,
+    prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmKnew,
                            const __grid_constant__ CUtensorMap tmVnew,
                            const __grid_constant__ CUtensorMap tmCache,
                            const PrefillAttnTcParams p) {
@@ -113,15 +140,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bars;
+  uint64_t* q_full = bars;                      // Q staged in TMEM by the softmax warps
   uint64_t* kv_full = bars + 1;                 // [kStages]
   uint64_t* kv_empty = kv_full + kStages;       // [kStages]
-  uint64_t* s_full = kv_empty + kStages;        // [group][2]
-  uint64_t* s_empty = s_full + 2 * kGroups;     // [group][2]
-  uint64_t* p_full = s_empty + 2 * kGroups;     // [group][2]
-  uint64_t* p_empty = p_full + 2 * kGroups;     // [group][2]
-  uint64_t* o_full = p_empty + 2 * kGroups;     // [group]
-  uint64_t* drain = o_full + kGroups;
+  uint64_t* s_full = kv_empty + kStages;        // [kSBufs] S tile in TMEM buffer b is ready
+  uint64_t* p_full = s_full + kSBufs;           // [kSBufs] P tile written over buffer b
+  uint64_t* pv_done = p_full + kSBufs;          // [kSBufs] the PV MMAs reading buffer b completed
+  uint64_t* o_full = pv_done + kSBufs;
+  uint64_t* drain = o_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -129,38 +155,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int head = blockIdx.y;
   const int group_size = p.n_q_heads / p.n_kv;
   const int kvh = head / group_size;
-  const int pair = gridDim.x - 1 - blockIdx.x;        // heaviest query tiles first
-  QTile qt[kGroups];
-#pragma unroll
-  for (int g = 0; g < kGroups; ++g) qt[g] = make_qtile(p, pair * kGroups + g);
-  // key tiles of the CTA: the union of the tiles' ranges (later tiles reach further)
-  const int kt_first = qt[0].kb;
-  int kt_last = qt[0].ke;
-#pragma unroll
-  for (int g = 1; g < kGroups; ++g)
-    if (qt[g].active) kt_last = max(kt_last, qt[g].ke);
-  const int n_tiles = kt_last - kt_first + 1;
+  const int qblk = gridDim.x - 1 - blockIdx.x;        // heaviest query tiles first
+  const int m0 = qblk * kQ;
+  const int rows = min(kQ, p.n - m0);
+  const int q_lo = p.pos0 + m0, q_hi = q_lo + rows - 1;
+  const int key_lo = p.window > 0 ? max(0, q_lo - p.window + 1) : 0;
+  const int kt_begin = key_lo / kKT, kt_end = q_hi / kKT;
+  const int n_tiles = kt_end - kt_begin + 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, kSoftThreads);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int b = 0; b < 2 * kGroups; ++b) {
+    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);
-      mbar_init(&p_full[b], 128);
-      mbar_init(&p_empty[b], 1);
+      mbar_init(&p_full[b], kSoftThreads);
+      mbar_init(&pv_done[b], 1);
     }
-    for (int g = 0; g < kGroups; ++g) mbar_init(&o_full[g], 1);
+    mbar_init(o_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmQ);
     prefetch_tmap(&tmKnew);
     prefetch_tmap(&tmVnew);
     prefetch_tmap(&tmCache);
@@ -178,16 +198,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------- TMA producer
       bool ok = true;
-      int q_bytes = 0;
-#pragma unroll
-      for (int g = 0; g < kGroups; ++g) q_bytes += qt[g].active ? kQBytes : 0;
-      mbar_arrive_expect_tx(q_full, q_bytes);
-#pragma unroll
-      for (int g = 0; g < kGroups; ++g) {
-        if (!qt[g].active) continue;
-        tma_load_3d(smem + g * kQBytes, &tmQ, q_full, 0, head, qt[g].m0);
-        tma_load_3d(smem + g * kQBytes + kQBytes / 2, &tmQ, q_full, 64, head, qt[g].m0);
-      }
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity_bits = 0;
       for (int j = 0; j < n_tiles; ++j) {
@@ -196,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* st = smem + kOffKV + stage * kStageBytes;
-        const int kp0 = (kt_first + j) * kKT;
+        const int kp0 = (kt_begin + j) * kKT;
         mbar_arrive_expect_tx(&kv_full[stage], kStageBytes);
         if (kp0 < p.pos0) {
           // cached positions: slot rows of this sequence's K and V planes
@@ -204,15 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + slot;
           const int vrow = krow + p.n_kv * p.cap;
           tma_load_2d(st, &tmCache, &kv_full[stage], 0, krow);
-          tma_load_2d(st + kSubKV, &tmCache, &kv_full[stage], 64, krow);
-          tma_load_2d(st + 2 * kSubKV, &tmCache, &kv_full[stage], 0, vrow);
-          tma_load_2d(st + 3 * kSubKV, &tmCache, &kv_full[stage], 64, vrow);
+          tma_load_2d(st + kSub, &tmCache, &kv_full[stage], 64, krow);
+          tma_load_2d(st + 2 * kSub, &tmCache, &kv_full[stage], 0, vrow);
+          tma_load_2d(st + 3 * kSub, &tmCache, &kv_full[stage], 64, vrow);
         } else {
           const int t0 = kp0 - p.pos0;
           tma_load_3d(st, &tmKnew, &kv_full[stage], 0, kvh, t0);
-          tma_load_3d(st + kSubKV, &tmKnew, &kv_full[stage], 64, kvh, t0);
-          tma_load_3d(st + 2 * kSubKV, &tmVnew, &kv_full[stage], 0, kvh, t0);
-          tma_load_3d(st + 3 * kSubKV, &tmVnew, &kv_full[stage], 64, kvh, t0);
+          tma_load_3d(st + kSub, &tmKnew, &kv_full[stage], 64, kvh, t0);
+          tma_load_3d(st + 2 * kSub, &tmVnew, &kv_full[stage], 0, kvh, t0);
+          tma_load_3d(st + 3 * kSub, &tmVnew, &kv_full[stage], 64, kvh, t0);
         }
         issued |= 1u << stage;
         parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
@@ -222,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        drain_wait(q_full, 0);
         for (int s = 0; s < kStages; ++s)
           if (issued & (1u << s)) drain_wait(&kv_full[s], (parity_bits >> s) & 1u);
       }
@@ -232,68 +241,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16(kQ, kKT);
       constexpr uint32_t idesc_o = umma_idesc_bf16(kQ, kHD) | (1u << 16);   // B (V) MN-major
+      const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffKV));
+      const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffKV + 2 * kSub), kSub);
       bool ok = mbar_wait_bounded(q_full, 0, abort_flag, p.status);
       bool issued = false;
       int stage = 0, prev_stage = 0;
       uint32_t phase = 0;
       for (int j = 0; ok && j <= n_tiles; ++j) {
-        const int t = kt_first + j;
         if (j < n_tiles) {
-          if (!mbar_wait_bounded(&kv_full[stage], phase, abort_flag, p.status)) {
+          const int buf = j % kSBufs;
+          // S(j) overwrites the buffer whose P fed PV(j-3): wait for that PV
+          // (three buffers keep the tensor core fed while PV(j-1) drains)
+          if (!mbar_wait_bounded(&kv_full[stage], phase, abort_flag, p.status) ||
+              !mbar_wait_bounded(&pv_done[buf], ((j / kSBufs) & 1u) ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          const uint32_t k_addr = smem_u32(smem + kOffKV + stage * kStageBytes);
+          tc_fence_after();
+          const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((stage * kStageBytes) >> 4);
+          const uint32_t d_s = tmem + buf * kKT;
 #pragma unroll
-          for (int g = 0; g < kGroups; ++g) {
-            if (!qt[g].active || t < qt[g].kb || t > qt[g].ke) continue;
-            const int i = t - qt[g].kb;                 // the group's own tile index
-            const int buf = i & 1;
-            if (!mbar_wait_bounded(&s_empty[2 * g + buf], ((i >> 1) & 1u) ^ 1u, abort_flag,
-                                   p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t q_addr = smem_u32(smem + g * kQBytes);
-#pragma unroll
-            for (int kk = 0; kk < kHD / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32;
-              const uint32_t koff = (kk >> 2) * kSubKV + (kk & 3) * 32;
-              umma_bf16(tmem + g * 256 + buf * kKT, umma_desc_sw128(q_addr + off),
-                        umma_desc_sw128(k_addr + koff), idesc_s, kk > 0 ? 1u : 0u);
-            }
-            issued = true;
-            umma_commit(&s_full[2 * g + buf]);
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            // A = Q from TMEM (dims 16kk.. in columns 8kk..), B = K from shared memory
+            const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+            umma_bf16_ts(d_s, tmem + kColQ + 8 * kk, k_desc + (koff >> 4), idesc_s,
+                         kk > 0 ? 1u : 0u);
           }
-          if (!ok) break;
+          issued = true;
+          umma_commit(&s_full[buf]);
         }
         if (j > 0) {
-          // O_g += P_g V for the previous key tile
-          const int tp = t - 1;
-          const uint32_t v_addr = smem_u32(smem + kOffKV + prev_stage * kStageBytes) + 2 * kSubKV;
-#pragma unroll
-          for (int g = 0; g < kGroups; ++g) {
-            if (!qt[g].active || tp < qt[g].kb || tp > qt[g].ke) continue;
-            const int i = tp - qt[g].kb;
-            const int buf = i & 1;
-            if (!mbar_wait_bounded(&p_full[2 * g + buf], (i >> 1) & 1u, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t p_addr = smem_u32(smem + kOffP + (2 * g + buf) * kPBytes);
-#pragma unroll
-            for (int kk = 0; kk < kKT / 16; ++kk) {
-              umma_bf16(tmem + g * 256 + 2 * kKT, umma_desc_sw128(p_addr + kk * 32),
-                        umma_desc_sw128_mn(v_addr + kk * 2048, kSubKV), idesc_o,
-                        (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(&p_empty[2 * g + buf]);
-            if (tp == qt[g].ke) umma_commit(&o_full[g]);
+          // O += P(j-1) V(j-1), P read from TMEM
+          const int i = j - 1;
+          const int buf = i % kSBufs;
+          if (!mbar_wait_bounded(&p_full[buf], (i / kSBufs) & 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
+          tc_fence_after();
+          const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((prev_stage * kStageBytes) >> 4);
+          const uint32_t p_col = tmem + buf * kKT;
+#pragma unroll
+          for (int kk = 0; kk < kKT / 16; ++kk) {
+            // keys 16kk..16kk+15 sit in columns 32*(kk/2) + 8*(kk%2) .. +7 of the buffer
+            const uint32_t a = p_col + 32 * (kk >> 1) + 8 * (kk & 1);
+            umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
+                         (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&pv_done[buf]);
           umma_commit(&kv_empty[prev_stage]);
+          if (i == n_tiles - 1) umma_commit(o_full);
         }
         prev_stage = stage;
         if (j < n_tiles && ++stage == kStages) {
@@ -308,98 +305,103 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ----------------------------------------------------- softmax / output
-    const int g = (warp - 2) >> 2;                 // softmax warpgroup = query tile
-    const QTile q = qt[g];
+    // warp w reads TMEM lanes 32*(w%4).. (its row quadrant) and one quarter
+    // (32 keys) of every S tile; it writes that quarter's P as bf16 pairs into
+    // the first 16 columns of the quarter, which only it has read.
+    const int quarter = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                // query row of this thread
-    const int qp = q.q_lo + r;
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + g * 256;
-    uint8_t* prow = smem + kOffP + (2 * g) * kPBytes + r * 128;
+    const int qp = q_lo + r;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float scale = p.scale_log2, moff = p.m_log2;
-    float l = 0.f;
-    bool ok = q.active;
-    const int n_mine = q.active ? q.ke - q.kb + 1 : 0;
-    for (int i = 0; ok && i < n_mine; ++i) {
-      const int buf = i & 1;
-      const uint32_t use = i >> 1;
-      // warp-uniform: the TMEM loads below are warp-collective
-      if (!__all_sync(0xFFFFFFFFu,
-                      mbar_wait_bounded(&s_full[2 * g + buf], use & 1u, abort_flag, p.status))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[kKT];
-      {
-        float t[32];
-        tmem_ld32(tbase + buf * kKT, t);
+    const int window = p.window;
+    {
+      // stage this thread's quarter of its Q row (32 dims) into TMEM
+      // columns kColQ + 16*quarter.. as bf16 pairs: the A operand of S = Q K^T
+      uint32_t qv[16];
+      if (r < rows) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.q + (static_cast<size_t>(m0 + r) * p.n_q_heads + head) * kHD + quarter * 32);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) s[c] = t[c];
-        tmem_ld32(tbase + buf * kKT + 32, t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[32 + c] = t[c];
-      }
-      tc_fence_before();
-      mbar_arrive(&s_empty[2 * g + buf]);
-      const int kp0 = (q.kb + i) * kKT;
-      const int key_lo = p.window > 0 ? max(0, q.q_lo - p.window + 1) : 0;
-      const bool need_mask = (kp0 < key_lo) || (kp0 + kKT - 1 > q.q_lo) ||
-                             (p.window > 0 && q.q_hi - kp0 >= p.window);
-      uint32_t packed[kKT / 2];
-      if (!need_mask) {
-#pragma unroll
-        for (int c = 0; c < kKT; c += 2) {
-          const float e0 = ex2(fmaf(s[c], scale, -moff));
-          const float e1 = ex2(fmaf(s[c + 1], scale, -moff));
-          l += e0 + e1;
-          packed[c / 2] = pack_bf16x2(e0, e1);
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v = src[k];
+          qv[4 * k] = v.x; qv[4 * k + 1] = v.y; qv[4 * k + 2] = v.z; qv[4 * k + 3] = v.w;
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < kKT; c += 2) {
-          const int k0 = kp0 + c, k1 = k0 + 1;
-          const bool ok0 = k0 <= qp && (p.window <= 0 || qp - k0 < p.window);
-          const bool ok1 = k1 <= qp && (p.window <= 0 || qp - k1 < p.window);
-          const float e0 = ok0 ? ex2(fmaf(s[c], scale, -moff)) : 0.f;
-          const float e1 = ok1 ? ex2(fmaf(s[c + 1], scale, -moff)) : 0.f;
-          l += e0 + e1;
-          packed[c / 2] = pack_bf16x2(e0, e1);
-        }
+        for (int k = 0; k < 16; ++k) qv[k] = 0u;
       }
-      if (i >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&p_empty[2 * g + buf],
-                                                               (use & 1u) ^ 1u, abort_flag,
-                                                               p.status))) {
+      tmem_st16(lane_addr + kColQ + quarter * 16, qv);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(q_full);
+    }
+    float l = 0.f;
+    bool ok = true;
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int buf = i % kSBufs;
+      // warp-uniform: TMEM loads and stores are warp-collective
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait_bounded(&s_full[buf], (i / kSBufs) & 1u, abort_flag, p.status))) {
         ok = false;
         break;
       }
-      uint8_t* pb = prow + buf * kPBytes;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        *reinterpret_cast<uint4*>(pb + ((c ^ (r & 7)) << 4)) =
-            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&p_full[2 * g + buf]);
-    }
-    if (ok && __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&o_full[g], 0, abort_flag, p.status))) {
       tc_fence_after();
-      const bool row_ok = r < q.rows;
-      const int t = q.m0 + r;
-      const float f = row_ok ? p.gate[static_cast<size_t>(t) * p.n_q_heads + head] / l : 0.f;
-      __nv_bfloat16* dst = p.out + (static_cast<size_t>(t) * p.n_q_heads + head) * kHD;
-#pragma unroll 1
-      for (int c = 0; c < kHD; c += 32) {
-        float o[32];
-        tmem_ld32(tbase + 2 * kKT + c, o);
-        if (row_ok) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+      float sv[32];
+      tmem_ld32(lane_addr + buf * kKT + quarter * 32, sv);
+      const int kp0 = (kt_begin + i) * kKT + quarter * 32;
+      const bool need_mask = (kp0 < key_lo) || (kp0 + 31 > q_lo) ||
+                             (window > 0 && q_hi - kp0 >= window);
+      uint32_t packed[16];
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            d4[k] = make_uint4(pack_bf16x2(o[8 * k] * f, o[8 * k + 1] * f),
-                               pack_bf16x2(o[8 * k + 2] * f, o[8 * k + 3] * f),
-                               pack_bf16x2(o[8 * k + 4] * f, o[8 * k + 5] * f),
-                               pack_bf16x2(o[8 * k + 6] * f, o[8 * k + 7] * f));
+      for (int c = 0; c < 32; c += 4) {
+        float e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x = fmaf(sv[c + u], scale, -moff);
+          e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
         }
+        if (need_mask) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int kp = kp0 + c + u;
+            const bool keep = kp <= qp && (window <= 0 || qp - kp < window);
+            e[u] = keep ? e[u] : 0.f;
+          }
+        }
+        l += (e[0] + e[1]) + (e[2] + e[3]);
+        packed[c / 2] = pack_bf16x2(e[0], e[1]);
+        packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
+      }
+      tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[buf]);
+    }
+    const bool done = __all_sync(0xFFFFFFFFu, ok) &&
+                      __all_sync(0xFFFFFFFFu, mbar_wait_bounded(o_full, 0, abort_flag, p.status));
+    // the four quarters of a row add their row sums (the K/V ring is free
+    // once every MMA has completed)
+    float* lsum = reinterpret_cast<float*>(smem + kOffKV);
+    if (done) lsum[r * 4 + quarter] = l;
+    named_bar_sync(1, kSoftThreads);
+    if (done) {
+      tc_fence_after();
+      const float l_row = (lsum[r * 4] + lsum[r * 4 + 1]) + (lsum[r * 4 + 2] + lsum[r * 4 + 3]);
+      const bool row_ok = r < rows;
+      const int t = m0 + r;
+      const float f = row_ok ? p.gate[static_cast<size_t>(t) * p.n_q_heads + head] / l_row : 0.f;
+      __nv_bfloat16* dst = p.out + (static_cast<size_t>(t) * p.n_q_heads + head) * kHD + quarter * 32;
+      float o[32];
+      tmem_ld32(lane_addr + kColO + quarter * 32, o);
+      if (row_ok) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          d4[k] = make_uint4(pack_bf16x2(o[8 * k] * f, o[8 * k + 1] * f),
+                             pack_bf16x2(o[8 * k + 2] * f, o[8 * k + 3] * f),
+                             pack_bf16x2(o[8 * k + 4] * f, o[8 * k + 5] * f),
+                             pack_bf16x2(o[8 * k + 6] * f, o[8 * k + 7] * f));
       }
     }
   }
@@ -451,9 +453,8 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
                                         const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                         const KvLayerView& kv, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
-  CUtensorMap tq, tk, tv, tc;
-  if (!make_tmap_3d(&tq, q, kHD, p.n_q_heads, p.n, 64, 1, kQ) ||
-      !make_tmap_3d(&tk, k_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
+  CUtensorMap tk, tv, tc;
+  if (!make_tmap_3d(&tk, k_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
       !make_tmap_3d(&tv, v_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
       !make_tmap_bf16(&tc, kv.k_base, static_cast<uint64_t>(kv.max_seqs) * 2 * kv.n_kv * kv.cap,
                       kHD, kKT))
@@ -468,8 +469,10 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
     if (e != cudaSuccess) return e;
     if (dev < 32) attr_done |= 1u << dev;
   }
-  dim3 grid((p.n + kGroups * kQ - 1) / (kGroups * kQ), p.n_q_heads);
-  prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, p);
+  dim3 grid((p.n + kQ - 1) / kQ, p.n_q_heads);
+  PrefillAttnTcParams pq = p;
+  pq.q = q;
+  prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tk, tv, tc, pq);
   return cudaGetLastError();
 }
 

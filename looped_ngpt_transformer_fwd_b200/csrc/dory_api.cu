@@ -23,7 +23,7 @@
 #include <tuple>
 #include <vector>
 
-#include "../../include/dory.h"
+#include "dory.h"
 #include "common.cuh"
 #include "kernels.h"
 

@@ -254,6 +254,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      // descriptors built once; a stage or k-step adds (byte offset >> 4)
+      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(tiles));
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(tiles + C::kABytes));
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -278,12 +281,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kABytes;
+          const uint64_t soff = static_cast<uint64_t>((stage * C::kStageBytes) >> 4);
+          const uint64_t a_desc = a_desc0 + soff, b_desc = b_desc0 + soff;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
-                      idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            umma_bf16(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4), idesc,
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           issued = true;
           umma_commit(&empty[stage]);

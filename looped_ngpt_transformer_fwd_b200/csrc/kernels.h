@@ -139,6 +139,7 @@ cudaError_t launch_prefill_attention(const PrefillAttnParams& p, cudaStream_t s)
 // Tensor-core (tcgen05) prefill attention for head_dim 128 with a static
 // softmax maximum m_log2 = softmax_scale * log2(e) * max_i s_qk[i]^2.
 struct PrefillAttnTcParams {
+  const __nv_bfloat16* q = nullptr;     // [n, Hq, hd] (set by the launcher)
   const float* gate = nullptr;          // [n, Hq]
   __nv_bfloat16* out = nullptr;         // [n, Hq*hd]
   int n = 0, pos0 = 0, seq = 0;

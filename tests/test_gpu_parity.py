@@ -247,10 +247,10 @@ def test_kernel_profiling_counts_every_launch(tiny):
 
 
 # ------------------------------------------------------------------ head_dim 128
-# (d 512, 4/2 heads of 128, window 64): prefill attention runs on the tcgen05
-# kernel whenever pos0 and the window are multiples of 64, else on the
+# (d 512, 4/2 heads of 128, window 128): prefill attention runs on the tcgen05
+# kernel whenever pos0 and the window are multiples of 128, else on the
 # mma.sync kernel; both must match the oracle.
-HD128 = dict(d_model=512, n_q_heads=4, n_kv_heads=2, head_dim=128, d_ff=1024, window=64,
+HD128 = dict(d_model=512, n_q_heads=4, n_kv_heads=2, head_dim=128, d_ff=1024, window=128,
              softmax_scale=float(np.sqrt(128.0)))
 
 
@@ -273,8 +273,8 @@ def test_hd128_prefill_matches_oracle(hd128, mode):
 
 @pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
 def test_hd128_chunked_prefill_and_decode(hd128, mode):
-    """Chunks at multiples of 64 (tensor-core attention reading cached tiles and
-    ring slots), one unaligned chunk (mma.sync kernel), then decode steps."""
+    """Chunks at multiples of 128 (tensor-core attention reading cached tiles and
+    ring slots), unaligned chunks (mma.sync kernel), then decode steps."""
     cfg, prov, model = hd128
     k = 2
     x, h = inputs(cfg, 52, 420)
@@ -282,7 +282,7 @@ def test_hd128_chunked_prefill_and_decode(hd128, mode):
     ocache = oracle_cache(cfg, mode, k_max=2)
     orc = oracle(cfg, prov)
     seq = 1
-    for a, b in ((0, 128), (128, 192), (192, 330), (330, 405), (405, 416)):
+    for a, b in ((0, 128), (128, 256), (256, 384), (384, 405), (405, 416)):
         out = model.prefill(kv, x[a:b], k, seq=seq, pos0=a)
         torch.cuda.synchronize()
         ref = orc.forward(h[a:b], a, k, ocache, seq=seq)
@@ -296,11 +296,11 @@ def test_hd128_chunked_prefill_and_decode(hd128, mode):
     assert model.device_status() == 0
 
 
-@pytest.mark.parametrize("layer", [0, 1])      # SWA (W = 64), full
+@pytest.mark.parametrize("layer", [0, 1])      # SWA (W = 128), full
 def test_hd128_attention_sublayer_alpha_one_is_tight(layer):
     """alpha = 1 makes the sublayer output Norm(o W_o^T) itself, so the attention
     output is compared almost undiluted: a key added or dropped at a mask edge
-    (one of ~64) would move it by ~1.5 %, far above the bf16 error."""
+    (one of ~128) would move it by ~0.8 %, far above the bf16 error."""
     from tests.oracle_util import modified
     from oracle import weights_from_generator
     from looped_ngpt_transformer_fwd_b200.model import DoryModel
@@ -323,11 +323,11 @@ def test_hd128_attention_sublayer_alpha_one_is_tight(layer):
                 out[k_] = f32_to_bf16_bits(v.astype(np.float32))
         return out
     model = DoryModel(cfg, as_generator_format)
-    _, h = inputs(cfg, 53, 320)
-    kv = model.kv_cache("last_loop", 1, 384)
+    _, h = inputs(cfg, 53, 448)
+    kv = model.kv_cache("last_loop", 1, 512)
     ocache = oracle_cache(cfg, "last_loop")
     orc = oracle(cfg, as_generator_format)
-    for pos0, n in ((0, 192), (192, 128)):
+    for pos0, n in ((0, 256), (256, 192)):
         ht = torch.from_numpy(h[pos0:pos0 + n].astype(np.float32)).cuda()
         model.attention_sublayer(kv, layer, ht, loop=1, seq=0, pos0=pos0)
         torch.cuda.synchronize()
