@@ -53,10 +53,16 @@ PROFILED = {
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
                           "2b5abcda8b52a241f9abeba8de52b778b1f4b967"),
                "profile": "profiles/gemm_tc_4b_prefill_full.md"},
+    # decode attention: measured (read + write) / algorithmic bytes, applied to
+    # the step's total KV bytes
+    "attn": {"ratio": (1075908000 + 8675840) / 1073758208,
+             "source": ("looped_ngpt_transformer_fwd_b200/csrc/attn_decode_tma.cu",
+                        "364d8cd720bac77c12c3080afcf6ee162dea4681"),
+             "profile": "profiles/attn_decode_tma_b8_ctx32768_full.md"},
 }
 
 
-def profiled_traffic(kernel):
+def profiled_traffic(kernel, work=None):
     import hashlib
     ent = PROFILED.get(kernel)
     if not ent:
@@ -68,6 +74,8 @@ def profiled_traffic(kernel):
                 return None
     except OSError:
         return None
+    if "ratio" in ent:
+        return ent["ratio"] * work if work is not None else None
     return ent["traffic"]
 
 
@@ -200,13 +208,13 @@ def fill_decode_cache(model, kv, cfg, seed, ctx, mode, k_max, batch):
             slots = positions % cap
         for loop in loops:
             for s in range(batch):
-                kk, vv = kv_values_torch(seed, b * 16 + (loop - 1), s, positions, hkv, hd, s_qk,
-                                         "cuda")
-                for h in range(hkv):
-                    kview = kv.entry_view(b, loop, s, h, "k")
-                    vview = kv.entry_view(b, loop, s, h, "v")
-                    kview[slots] = kk[:, h]
-                    vview[slots] = vv[:, h]
+                for c0 in range(0, positions.numel(), 16384):   # bounded temporaries
+                    pc, sc = positions[c0:c0 + 16384], slots[c0:c0 + 16384]
+                    kk, vv = kv_values_torch(seed, b * 16 + (loop - 1), s, pc, hkv, hd, s_qk,
+                                             "cuda")
+                    for h in range(hkv):
+                        kv.entry_view(b, loop, s, h, "k")[sc] = kk[:, h]
+                        kv.entry_view(b, loop, s, h, "v")[sc] = vv[:, h]
     torch.cuda.synchronize()
 
 
@@ -335,13 +343,24 @@ def run_ours(args, wl, rank, world, device_index):
     step()
     torch.cuda.synchronize()
     tot = {kk: [0.0, 0] for kk in ("qkvg", "attn", "oproj", "gateup", "down", "row", "kvcommit")}
-    reps = max(1, min(args.steps, 5)) if wl["kind"] != "prefill_chunked" else 1
-    for _ in range(reps):
-        step()
-        torch.cuda.synchronize()
-        for kk, (t, n) in model.profile_read().items():
-            tot[kk][0] += t
-            tot[kk][1] += n
+    if wl["kind"] == "prefill_chunked":
+        # one replay of the whole step, reading every chunk's kernels
+        reps = 1
+        T, C = wl["tokens"], wl["chunk"]
+        for c0 in range(0, T, C):
+            model.prefill(kv, xs[c0:c0 + C], k, pos0=c0, h_out=out)
+            torch.cuda.synchronize()
+            for kk, (t, n) in model.profile_read().items():
+                tot[kk][0] += t
+                tot[kk][1] += n
+    else:
+        reps = max(1, min(args.steps, 5))
+        for _ in range(reps):
+            step()
+            torch.cuda.synchronize()
+            for kk, (t, n) in model.profile_read().items():
+                tot[kk][0] += t
+                tot[kk][1] += n
     model.profile(False)
     kernel_ms = {kk: (v[0] / reps, v[1] // reps) for kk, v in tot.items()}
     dom_name, dom_work, bound = dom
@@ -504,7 +523,7 @@ def main():
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit = "TFLOP/s"
         if wl["kind"] == "prefill_chunked":
-            achieved = dom_work / (dom_ms / 1e3) / 1e12
+            achieved = dom_work / (dom_ms / 1e3) / 1e12   # all chunks' attention FLOPs / time
     else:
         achieved = dom_work / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
         peak = peaks["hbm_gbs"]
@@ -528,7 +547,8 @@ def main():
             "roofline": {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
                          "unit": unit, "frac": (achieved / peak) if achieved else None,
                          "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
-                         "traffic": profiled_traffic(dom_name),
+                         "traffic": (profiled_traffic(dom_name, dom_work) if bound == "hbm"
+                                     else profiled_traffic(dom_name)),
                          "work_per_step": dom_work, "launches_per_step": dom_n,
                          "device_ms_per_step": dom_ms},
             "kernel_ms_per_step": {kk: round(v[0], 4) for kk, v in res["kernel_ms"].items()},
