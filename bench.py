@@ -388,13 +388,22 @@ def barrier(world):
 
 
 def reduce_max(x, world):
+    """Max of x over the ranks (the slowest replica sets the step time)."""
     if world <= 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(units_per_step, ms_per_step_local, world):
+    """Whole-job throughput of `world` replicas: every rank's units over the
+    slowest rank's step time.  Returns (ms_per_step, units per second)."""
+    ms = reduce_max(ms_per_step_local, world)
+    return ms, units_per_step * world / ms * 1e3
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -533,7 +542,7 @@ def main():
         v, u, sample = oracle_sample(wl, res["prov"])
         cpu = {"value": v, "unit": u, "cores": blas_threads(), "kind": "oracle", "sample": sample}
     if rank == 0:
-        value = res["units"] * world / res["ms"] * 1e3
+        value = res["units"] * world / res["ms"] * 1e3   # res["ms"] is already the max over ranks
         line = {
             "metric": f"{'prefill' if 'prefill' in wl['kind'] else 'decode'} tokens/s",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
