@@ -14,7 +14,8 @@
 // underflow of the smallest weight in fp32/bf16); otherwise it keeps the
 // online-softmax kernel.
 //
-// One CTA = 128 queries of one query head; 128-key K/V tiles.  Warp 0 issues
+// Persistent: one CTA per SM works through (128-query tile, head) items dealt
+// longest first in snake order; 128-key K/V tiles.  Warp 0 issues
 // TMA loads of K/V tiles through a 3-stage ring (from the layer's cache for
 // positions below pos0, from this call's fresh K/V otherwise).  Q is staged
 // once into TMEM by the softmax warps.  Warp 1 owns TMEM and issues the MMAs,
@@ -44,7 +45,8 @@ constexpr int kThreads = 64 + kSoftThreads;
 constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 keys x 64 dims (one TMA box)
 constexpr int kStageBytes = 4 * kSub;                 // K (2 sub-tiles) + V (2 sub-tiles)
 constexpr int kOffKV = 0;
-constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+constexpr int kOffL = kOffKV + kStages * kStageBytes;     // row-sum exchange, 128 x 4 floats
+constexpr int kOffBar = kOffL + kQ * 4 * 4;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 constexpr int kSBufs = 2;                             // S/P buffers in TMEM
 constexpr uint32_t kTmemCols = 512;                   // S0 | S1 | O (128 columns each) | Q (64)
@@ -111,6 +113,20 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier over nthreads that also returns whether any of them passed true.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -131,6 +147,31 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Work item k of this CTA: query tiles sorted longest first (the causal or
+// windowed key range grows with the query tile), dealt out round by round in
+// alternating direction ("snake"), so every CTA gets a similar total.
+struct Item {
+  int qblk, head, m0, rows, q_lo, q_hi, key_lo, kt_begin, n_tiles;
+};
+
+__device__ __forceinline__ bool get_item(const PrefillAttnTcParams& p, int k, Item& it) {
+  const int n_qblk = (p.n + kQ - 1) / kQ;
+  const int total = n_qblk * p.n_q_heads;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int idx = k * G + ((k & 1) ? (G - 1 - c) : c);
+  if (idx >= total) return false;
+  it.qblk = n_qblk - 1 - idx / p.n_q_heads;
+  it.head = idx % p.n_q_heads;
+  it.m0 = it.qblk * kQ;
+  it.rows = min(kQ, p.n - it.m0);
+  it.q_lo = p.pos0 + it.m0;
+  it.q_hi = it.q_lo + it.rows - 1;
+  it.key_lo = p.window > 0 ? max(0, it.q_lo - p.window + 1) : 0;
+  it.kt_begin = it.key_lo / kKT;
+  it.n_tiles = it.q_hi / kKT - it.kt_begin + 1;
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmKnew,
                            const __grid_constant__ CUtensorMap tmVnew,
@@ -146,22 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = kv_empty + kStages;        // [kSBufs] S tile in TMEM buffer b is ready
   uint64_t* p_full = s_full + kSBufs;           // [kSBufs] P tile written over buffer b
   uint64_t* pv_done = p_full + kSBufs;          // [kSBufs] the PV MMAs reading buffer b completed
-  uint64_t* o_full = pv_done + kSBufs;
-  uint64_t* drain = o_full + 1;
+  uint64_t* o_full = pv_done + kSBufs;           // all MMAs of the current item completed
+  uint64_t* o_empty = o_full + 1;               // its output was read from TMEM
+  uint64_t* drain = o_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.y;
   const int group_size = p.n_q_heads / p.n_kv;
-  const int kvh = head / group_size;
-  const int qblk = gridDim.x - 1 - blockIdx.x;        // heaviest query tiles first
-  const int m0 = qblk * kQ;
-  const int rows = min(kQ, p.n - m0);
-  const int q_lo = p.pos0 + m0, q_hi = q_lo + rows - 1;
-  const int key_lo = p.window > 0 ? max(0, q_lo - p.window + 1) : 0;
-  const int kt_begin = key_lo / kKT, kt_end = q_hi / kKT;
-  const int n_tiles = kt_end - kt_begin + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, kSoftThreads);
@@ -175,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(o_full, 1);
+    mbar_init(o_empty, kSoftThreads);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -200,35 +234,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity_bits = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        if (!mbar_wait_bounded(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + kOffKV + stage * kStageBytes;
-        const int kp0 = (kt_begin + j) * kKT;
-        mbar_arrive_expect_tx(&kv_full[stage], kStageBytes);
-        if (kp0 < p.pos0) {
-          // cached positions: slot rows of this sequence's K and V planes
-          const int slot = kp0 % p.cap;
-          const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + slot;
-          const int vrow = krow + p.n_kv * p.cap;
-          tma_load_2d(st, &tmCache, &kv_full[stage], 0, krow);
-          tma_load_2d(st + kSub, &tmCache, &kv_full[stage], 64, krow);
-          tma_load_2d(st + 2 * kSub, &tmCache, &kv_full[stage], 0, vrow);
-          tma_load_2d(st + 3 * kSub, &tmCache, &kv_full[stage], 64, vrow);
-        } else {
-          const int t0 = kp0 - p.pos0;
-          tma_load_3d(st, &tmKnew, &kv_full[stage], 0, kvh, t0);
-          tma_load_3d(st + kSub, &tmKnew, &kv_full[stage], 64, kvh, t0);
-          tma_load_3d(st + 2 * kSub, &tmVnew, &kv_full[stage], 0, kvh, t0);
-          tma_load_3d(st + 3 * kSub, &tmVnew, &kv_full[stage], 64, kvh, t0);
-        }
-        issued |= 1u << stage;
-        parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+      Item it;
+      for (int k = 0; ok && get_item(p, k, it); ++k) {
+        const int kvh = it.head / group_size;
+        for (int j = 0; j < it.n_tiles; ++j) {
+          if (!mbar_wait_bounded(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + kOffKV + stage * kStageBytes;
+          const int kp0 = (it.kt_begin + j) * kKT;
+          mbar_arrive_expect_tx(&kv_full[stage], kStageBytes);
+          if (kp0 < p.pos0) {
+            // cached positions: slot rows of this sequence's K and V planes
+            const int slot = kp0 % p.cap;
+            const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + slot;
+            const int vrow = krow + p.n_kv * p.cap;
+            tma_load_2d(st, &tmCache, &kv_full[stage], 0, krow);
+            tma_load_2d(st + kSub, &tmCache, &kv_full[stage], 64, krow);
+            tma_load_2d(st + 2 * kSub, &tmCache, &kv_full[stage], 0, vrow);
+            tma_load_2d(st + 3 * kSub, &tmCache, &kv_full[stage], 64, vrow);
+          } else {
+            const int t0 = kp0 - p.pos0;
+            tma_load_3d(st, &tmKnew, &kv_full[stage], 0, kvh, t0);
+            tma_load_3d(st + kSub, &tmKnew, &kv_full[stage], 64, kvh, t0);
+            tma_load_3d(st + 2 * kSub, &tmVnew, &kv_full[stage], 0, kvh, t0);
+            tma_load_3d(st + 3 * kSub, &tmVnew, &kv_full[stage], 64, kvh, t0);
+          }
+          issued |= 1u << stage;
+          parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok) {
@@ -243,60 +281,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = umma_idesc_bf16(kQ, kHD) | (1u << 16);   // B (V) MN-major
       const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffKV));
       const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffKV + 2 * kSub), kSub);
-      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, p.status);
+      bool ok = true;
       bool issued = false;
       int stage = 0, prev_stage = 0;
       uint32_t phase = 0;
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int buf = j % kSBufs;
-          // S(j) overwrites the buffer whose P fed PV(j-3): wait for that PV
-          // (three buffers keep the tensor core fed while PV(j-1) drains)
-          if (!mbar_wait_bounded(&kv_full[stage], phase, abort_flag, p.status) ||
-              !mbar_wait_bounded(&pv_done[buf], ((j / kSBufs) & 1u) ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((stage * kStageBytes) >> 4);
-          const uint32_t d_s = tmem + buf * kKT;
+      int g = 0;                      // tile counter over all items (S/P buffer rotation)
+      Item it;
+      for (int k = 0; ok && get_item(p, k, it); ++k) {
+        // Q of this item staged in TMEM; the previous item's output read out
+        if (!mbar_wait_bounded(q_full, k & 1u, abort_flag, p.status) ||
+            (k > 0 && !mbar_wait_bounded(o_empty, (k - 1) & 1u, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        for (int j = 0; ok && j <= it.n_tiles; ++j) {
+          if (j < it.n_tiles) {
+            const int t = g + j;
+            const int buf = t % kSBufs;
+            // S(t) overwrites the buffer whose P fed PV(t - kSBufs): wait for that PV
+            if (!mbar_wait_bounded(&kv_full[stage], phase, abort_flag, p.status) ||
+                !mbar_wait_bounded(&pv_done[buf], ((t / kSBufs) & 1u) ^ 1u, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((stage * kStageBytes) >> 4);
+            const uint32_t d_s = tmem + buf * kKT;
 #pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk) {
-            // A = Q from TMEM (dims 16kk.. in columns 8kk..), B = K from shared memory
-            const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-            umma_bf16_ts(d_s, tmem + kColQ + 8 * kk, k_desc + (koff >> 4), idesc_s,
-                         kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kHD / 16; ++kk) {
+              // A = Q from TMEM (dims 16kk.. in columns 8kk..), B = K from shared memory
+              const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+              umma_bf16_ts(d_s, tmem + kColQ + 8 * kk, k_desc + (koff >> 4), idesc_s,
+                           kk > 0 ? 1u : 0u);
+            }
+            issued = true;
+            umma_commit(&s_full[buf]);
           }
-          issued = true;
-          umma_commit(&s_full[buf]);
-        }
-        if (j > 0) {
-          // O += P(j-1) V(j-1), P read from TMEM
-          const int i = j - 1;
-          const int buf = i % kSBufs;
-          if (!mbar_wait_bounded(&p_full[buf], (i / kSBufs) & 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((prev_stage * kStageBytes) >> 4);
-          const uint32_t p_col = tmem + buf * kKT;
+          if (j > 0) {
+            // O += P(i) V(i), P read from TMEM
+            const int i = j - 1;
+            const int t = g + i;
+            const int buf = t % kSBufs;
+            if (!mbar_wait_bounded(&p_full[buf], (t / kSBufs) & 1u, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((prev_stage * kStageBytes) >> 4);
+            const uint32_t p_col = tmem + buf * kKT;
 #pragma unroll
-          for (int kk = 0; kk < kKT / 16; ++kk) {
-            // keys 16kk..16kk+15 sit in columns 32*(kk/2) + 8*(kk%2) .. +7 of the buffer
-            const uint32_t a = p_col + 32 * (kk >> 1) + 8 * (kk & 1);
-            umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
-                         (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kKT / 16; ++kk) {
+              // keys 16kk..16kk+15 sit in columns 32*(kk/2) + 8*(kk%2) .. +7 of the buffer
+              const uint32_t a = p_col + 32 * (kk >> 1) + 8 * (kk & 1);
+              umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&pv_done[buf]);
+            umma_commit(&kv_empty[prev_stage]);
+            if (i == it.n_tiles - 1) umma_commit(o_full);
           }
-          umma_commit(&pv_done[buf]);
-          umma_commit(&kv_empty[prev_stage]);
-          if (i == n_tiles - 1) umma_commit(o_full);
+          prev_stage = stage;
+          if (j < it.n_tiles && ++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        prev_stage = stage;
-        if (j < n_tiles && ++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        g += it.n_tiles;
       }
       if (!ok && issued) {
         umma_commit(drain);
@@ -311,98 +361,113 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                // query row of this thread
-    const int qp = q_lo + r;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float scale = p.scale_log2, moff = p.m_log2;
     const int window = p.window;
-    {
-      // stage this thread's quarter of its Q row (32 dims) into TMEM
-      // columns kColQ + 16*quarter.. as bf16 pairs: the A operand of S = Q K^T
-      uint32_t qv[16];
-      if (r < rows) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.q + (static_cast<size_t>(m0 + r) * p.n_q_heads + head) * kHD + quarter * 32);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 v = src[k];
-          qv[4 * k] = v.x; qv[4 * k + 1] = v.y; qv[4 * k + 2] = v.z; qv[4 * k + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) qv[k] = 0u;
-      }
-      tmem_st16(lane_addr + kColQ + quarter * 16, qv);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(q_full);
-    }
-    float l = 0.f;
+    float* lsum = reinterpret_cast<float*>(smem + kOffL);
     bool ok = true;
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int buf = i % kSBufs;
-      // warp-uniform: TMEM loads and stores are warp-collective
-      if (!__all_sync(0xFFFFFFFFu,
-                      mbar_wait_bounded(&s_full[buf], (i / kSBufs) & 1u, abort_flag, p.status))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float sv[32];
-      tmem_ld32(lane_addr + buf * kKT + quarter * 32, sv);
-      const int kp0 = (kt_begin + i) * kKT + quarter * 32;
-      const bool need_mask = (kp0 < key_lo) || (kp0 + 31 > q_lo) ||
-                             (window > 0 && q_hi - kp0 >= window);
-      uint32_t packed[16];
+    int g = 0;
+    Item it;
+    for (int k = 0; ok && get_item(p, k, it); ++k) {
+      {
+        // stage this thread's quarter of its Q row (32 dims) into TMEM
+        // columns kColQ + 16*quarter.. as bf16 pairs: the A operand of S = Q K^T.
+        // The previous item's MMAs have all completed (its o_full was awaited).
+        uint32_t qv[16];
+        if (r < it.rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.q + (static_cast<size_t>(it.m0 + r) * p.n_q_heads + it.head) * kHD + quarter * 32);
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        float e[4];
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = src[c];
+            qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
+          }
+        } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float x = fmaf(sv[c + u], scale, -moff);
-          e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
+          for (int c = 0; c < 16; ++c) qv[c] = 0u;
         }
-        if (need_mask) {
+        tmem_st16(lane_addr + kColQ + quarter * 16, qv);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_full);
+      }
+      const int qp = it.q_lo + r;
+      float l = 0.f;
+      for (int i = 0; i < it.n_tiles; ++i) {
+        const int t = g + i;
+        const int buf = t % kSBufs;
+        // warp-uniform: TMEM loads and stores are warp-collective
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait_bounded(&s_full[buf], (t / kSBufs) & 1u, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float sv[32];
+        tmem_ld32(lane_addr + buf * kKT + quarter * 32, sv);
+        const int kp0 = (it.kt_begin + i) * kKT + quarter * 32;
+        const bool need_mask = (kp0 < it.key_lo) || (kp0 + 31 > it.q_lo) ||
+                               (window > 0 && it.q_hi - kp0 >= window);
+        uint32_t packed[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          float e[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int kp = kp0 + c + u;
-            const bool keep = kp <= qp && (window <= 0 || qp - kp < window);
-            e[u] = keep ? e[u] : 0.f;
+            const float x = fmaf(sv[c + u], scale, -moff);
+            e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
           }
-        }
-        l += (e[0] + e[1]) + (e[2] + e[3]);
-        packed[c / 2] = pack_bf16x2(e[0], e[1]);
-        packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
-      }
-      tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[buf]);
-    }
-    const bool done = __all_sync(0xFFFFFFFFu, ok) &&
-                      __all_sync(0xFFFFFFFFu, mbar_wait_bounded(o_full, 0, abort_flag, p.status));
-    // the four quarters of a row add their row sums (the K/V ring is free
-    // once every MMA has completed)
-    float* lsum = reinterpret_cast<float*>(smem + kOffKV);
-    if (done) lsum[r * 4 + quarter] = l;
-    named_bar_sync(1, kSoftThreads);
-    if (done) {
-      tc_fence_after();
-      const float l_row = (lsum[r * 4] + lsum[r * 4 + 1]) + (lsum[r * 4 + 2] + lsum[r * 4 + 3]);
-      const bool row_ok = r < rows;
-      const int t = m0 + r;
-      const float f = row_ok ? p.gate[static_cast<size_t>(t) * p.n_q_heads + head] / l_row : 0.f;
-      __nv_bfloat16* dst = p.out + (static_cast<size_t>(t) * p.n_q_heads + head) * kHD + quarter * 32;
-      float o[32];
-      tmem_ld32(lane_addr + kColO + quarter * 32, o);
-      if (row_ok) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+          if (need_mask) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          d4[k] = make_uint4(pack_bf16x2(o[8 * k] * f, o[8 * k + 1] * f),
-                             pack_bf16x2(o[8 * k + 2] * f, o[8 * k + 3] * f),
-                             pack_bf16x2(o[8 * k + 4] * f, o[8 * k + 5] * f),
-                             pack_bf16x2(o[8 * k + 6] * f, o[8 * k + 7] * f));
+            for (int u = 0; u < 4; ++u) {
+              const int kp = kp0 + c + u;
+              const bool keep = kp <= qp && (window <= 0 || qp - kp < window);
+              e[u] = keep ? e[u] : 0.f;
+            }
+          }
+          l += (e[0] + e[1]) + (e[2] + e[3]);
+          packed[c / 2] = pack_bf16x2(e[0], e[1]);
+          packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
+        }
+        tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[buf]);
       }
+      g += it.n_tiles;
+      const bool done = __all_sync(0xFFFFFFFFu, ok) &&
+                        __all_sync(0xFFFFFFFFu,
+                                   mbar_wait_bounded(o_full, k & 1u, abort_flag, p.status));
+      // the four quarters of a row add their row sums
+      if (done) lsum[r * 4 + quarter] = l;
+      named_bar_sync(1, kSoftThreads);
+      if (done) {
+        tc_fence_after();
+        const float l_row = (lsum[r * 4] + lsum[r * 4 + 1]) + (lsum[r * 4 + 2] + lsum[r * 4 + 3]);
+        const bool row_ok = r < it.rows;
+        const int tok = it.m0 + r;
+        const float f =
+            row_ok ? p.gate[static_cast<size_t>(tok) * p.n_q_heads + it.head] / l_row : 0.f;
+        __nv_bfloat16* dst =
+            p.out + (static_cast<size_t>(tok) * p.n_q_heads + it.head) * kHD + quarter * 32;
+        float o[32];
+        tmem_ld32(lane_addr + kColO + quarter * 32, o);
+        tc_fence_before();
+        mbar_arrive(o_empty);      // O may be overwritten by the next item
+        if (row_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            d4[c] = make_uint4(pack_bf16x2(o[8 * c] * f, o[8 * c + 1] * f),
+                               pack_bf16x2(o[8 * c + 2] * f, o[8 * c + 3] * f),
+                               pack_bf16x2(o[8 * c + 4] * f, o[8 * c + 5] * f),
+                               pack_bf16x2(o[8 * c + 6] * f, o[8 * c + 7] * f));
+        }
+      } else {
+        ok = false;
+      }
+      // lsum is reused by the next item; all softmax warps leave the loop together
+      if (named_bar_any(1, kSoftThreads, !ok)) ok = false;
     }
   }
 
@@ -469,7 +534,11 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
     if (e != cudaSuccess) return e;
     if (dev < 32) attr_done |= 1u << dev;
   }
-  dim3 grid((p.n + kQ - 1) / kQ, p.n_q_heads);
+  int dev_sms = 0;
+  e = cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int items = ((p.n + kQ - 1) / kQ) * p.n_q_heads;
+  dim3 grid(items < dev_sms ? items : dev_sms);
   PrefillAttnTcParams pq = p;
   pq.q = q;
   prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tk, tv, tc, pq);
