@@ -15,17 +15,17 @@
 // online-softmax kernel.
 //
 // Persistent: one CTA per SM works through (128-query tile, head) items dealt
-// longest first in snake order; 128-key K/V tiles.  Warp 0 issues
-// TMA loads of K/V tiles through a 3-stage ring (from the layer's cache for
-// positions below pos0, from this call's fresh K/V otherwise).  Q is staged
-// once into TMEM by the softmax warps.  Warp 1 owns TMEM and issues the MMAs,
-// both with the A operand read from TMEM: S = Q K^T (N = 128 keys) into one of
-// two 128-column buffers, and O += P V with P written over S.  Each MMA then
-// reads a single operand (K or V, 4 KB) from shared memory, which keeps the
-// tensor core's operand traffic within its shared-memory bandwidth.  Sixteen
-// softmax warps (row quadrant x key quarter) turn S into P = exp2(...) in
-// place (mask, exp2 on the MUFU and FMA pipes, row sums) and finally write
-// gate * O / l.  Every wait is bounded.
+// longest first in snake order; 128-key K/V tiles.  Warp 0 issues TMA loads:
+// the item's Q tile, and K and V tiles through two separate 3-slot rings (from
+// the layer's cache for positions below pos0, from this call's fresh K/V
+// otherwise).  Warp 1 owns TMEM and issues the MMAs: S = Q K^T (N = 128 keys)
+// into one of three 128-column buffers, and O += P V with the A operand (P)
+// read from TMEM, where the softmax warps wrote it over S.  Three S buffers let
+// S run two key tiles ahead of P V, so the tensor core always has the next
+// S = Q K^T queued behind each P V and never waits out a completion round trip.
+// Sixteen softmax warps (row quadrant x key quarter) turn S into P =
+// exp2(...) in place (mask, exp2 on the MUFU and FMA pipes, row sums) and
+// finally write gate * O / l.  Every wait is bounded.
 #include <math.h>
 
 #include "common.cuh"
@@ -35,23 +35,27 @@ namespace dory {
 
 namespace {
 
-constexpr int kQ = 128;           // queries per CTA (one TMEM lane each)
+constexpr int kQ = 128;           // queries per item (one TMEM lane each)
 constexpr int kKT = 128;          // keys per tile
 constexpr int kHD = 128;
-constexpr int kStages = 3;
+constexpr int kSlots = 3;         // K ring and V ring depth
 constexpr int kSoftmaxWarps = 16; // 4 row quadrants x 4 column quarters of 32 keys
 constexpr int kSoftThreads = 32 * kSoftmaxWarps;
 constexpr int kThreads = 64 + kSoftThreads;
-constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 keys x 64 dims (one TMA box)
-constexpr int kStageBytes = 4 * kSub;                 // K (2 sub-tiles) + V (2 sub-tiles)
-constexpr int kOffKV = 0;
-constexpr int kOffL = kOffKV + kStages * kStageBytes;     // row-sum exchange, 128 x 4 floats
+constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 rows x 64 dims (one TMA box)
+constexpr int kSlotBytes = 2 * kSub;                  // one K or V tile, or the Q tile
+// shared memory (base 1024-aligned): K ring | V ring | Q | row sums | barriers
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kSlots * kSlotBytes;
+constexpr int kOffQ = kOffV + kSlots * kSlotBytes;
+constexpr int kOffL = kOffQ + kSlotBytes;             // row-sum exchange, 128 x 4 floats
 constexpr int kOffBar = kOffL + kQ * 4 * 4;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;
-constexpr int kSBufs = 2;                             // S/P buffers in TMEM
-constexpr uint32_t kTmemCols = 512;                   // S0 | S1 | O (128 columns each) | Q (64)
+constexpr int kSmemBytes = kOffBar + 256;
+constexpr int kSBufs = 3;                             // S/P buffers in TMEM
+constexpr uint32_t kTmemCols = 512;                   // S0 | S1 | S2 | O (128 columns each)
 constexpr uint32_t kColO = kSBufs * kKT;
-constexpr uint32_t kColQ = kColO + kHD;
+static_assert(kColO + kHD <= kTmemCols, "TMEM columns");
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
@@ -173,21 +177,29 @@ __device__ __forceinline__ bool get_item(const PrefillAttnTcParams& p, int k, It
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmKnew,
+    prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                           const __grid_constant__ CUtensorMap tmKnew,
                            const __grid_constant__ CUtensorMap tmVnew,
                            const __grid_constant__ CUtensorMap tmCache,
                            const PrefillAttnTcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // the SW128 operand layouts need a 1024-byte aligned base; the launch
+  // reserves no slack for rounding, so refuse (uniformly, before any barrier)
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report_status(p.status, kStatusBounds);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bars;                      // Q staged in TMEM by the softmax warps
-  uint64_t* kv_full = bars + 1;                 // [kStages]
-  uint64_t* kv_empty = kv_full + kStages;       // [kStages]
-  uint64_t* s_full = kv_empty + kStages;        // [kSBufs] S tile in TMEM buffer b is ready
-  uint64_t* p_full = s_full + kSBufs;           // [kSBufs] P tile written over buffer b
+  uint64_t* q_full = bars;                      // Q tile of the current item landed
+  uint64_t* q_empty = q_full + 1;               // all S MMAs of the previous item completed
+  uint64_t* k_full = q_empty + 1;               // [kSlots]
+  uint64_t* k_empty = k_full + kSlots;          // [kSlots]
+  uint64_t* v_full = k_empty + kSlots;          // [kSlots]
+  uint64_t* v_empty = v_full + kSlots;          // [kSlots]
+  uint64_t* s_full = v_empty + kSlots;          // [kSBufs] S tile in TMEM buffer b is ready
+  uint64_t* p_full = s_full + kSBufs;           // [kSBufs] P tile written over buffer b (one arrival per softmax warp)
   uint64_t* pv_done = p_full + kSBufs;          // [kSBufs] the PV MMAs reading buffer b completed
-  uint64_t* o_full = pv_done + kSBufs;           // all MMAs of the current item completed
+  uint64_t* o_full = pv_done + kSBufs;          // all MMAs of the current item completed
   uint64_t* o_empty = o_full + 1;               // its output was read from TMEM
   uint64_t* drain = o_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -197,24 +209,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int group_size = p.n_q_heads / p.n_kv;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, kSoftThreads);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], kSoftThreads);
+      mbar_init(&p_full[b], kSoftmaxWarps);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_empty, kSoftThreads);
+    mbar_init(o_empty, kSoftmaxWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
     prefetch_tmap(&tmKnew);
     prefetch_tmap(&tmVnew);
     prefetch_tmap(&tmCache);
@@ -232,46 +248,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------- TMA producer
       bool ok = true;
-      int stage = 0;
-      uint32_t phase = 0, issued = 0, parity_bits = 0;
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0;
+      // parity of the last copy into each slot, for draining after an error
+      uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
+      bool q_issued = false;
+      uint32_t q_par = 0;
       Item it;
       for (int k = 0; ok && get_item(p, k, it); ++k) {
         const int kvh = it.head / group_size;
+        // the Q slot is free once every S MMA of the previous item has completed
+        if (!mbar_wait_bounded(q_empty, (k & 1u) ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full, kSlotBytes);
+        tma_load_3d(smem + kOffQ, &tmQ, q_full, 0, it.head, it.m0);
+        tma_load_3d(smem + kOffQ + kSub, &tmQ, q_full, 64, it.head, it.m0);
+        q_issued = true;
+        q_par = k & 1u;
         for (int j = 0; j < it.n_tiles; ++j) {
-          if (!mbar_wait_bounded(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+          const int kp0 = (it.kt_begin + j) * kKT;
+          // cached positions: slot rows of this sequence's K and V planes
+          const bool cached = kp0 < p.pos0;
+          const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + (cached ? kp0 % p.cap : 0);
+          const int vrow = krow + p.n_kv * p.cap;
+          const int t0 = kp0 - p.pos0;
+          if (!mbar_wait_bounded(&k_empty[ks], kph ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + kOffKV + stage * kStageBytes;
-          const int kp0 = (it.kt_begin + j) * kKT;
-          mbar_arrive_expect_tx(&kv_full[stage], kStageBytes);
-          if (kp0 < p.pos0) {
-            // cached positions: slot rows of this sequence's K and V planes
-            const int slot = kp0 % p.cap;
-            const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + slot;
-            const int vrow = krow + p.n_kv * p.cap;
-            tma_load_2d(st, &tmCache, &kv_full[stage], 0, krow);
-            tma_load_2d(st + kSub, &tmCache, &kv_full[stage], 64, krow);
-            tma_load_2d(st + 2 * kSub, &tmCache, &kv_full[stage], 0, vrow);
-            tma_load_2d(st + 3 * kSub, &tmCache, &kv_full[stage], 64, vrow);
+          uint8_t* kd = smem + kOffK + ks * kSlotBytes;
+          mbar_arrive_expect_tx(&k_full[ks], kSlotBytes);
+          if (cached) {
+            tma_load_2d(kd, &tmCache, &k_full[ks], 0, krow);
+            tma_load_2d(kd + kSub, &tmCache, &k_full[ks], 64, krow);
           } else {
-            const int t0 = kp0 - p.pos0;
-            tma_load_3d(st, &tmKnew, &kv_full[stage], 0, kvh, t0);
-            tma_load_3d(st + kSub, &tmKnew, &kv_full[stage], 64, kvh, t0);
-            tma_load_3d(st + 2 * kSub, &tmVnew, &kv_full[stage], 0, kvh, t0);
-            tma_load_3d(st + 3 * kSub, &tmVnew, &kv_full[stage], 64, kvh, t0);
+            tma_load_3d(kd, &tmKnew, &k_full[ks], 0, kvh, t0);
+            tma_load_3d(kd + kSub, &tmKnew, &k_full[ks], 64, kvh, t0);
           }
-          issued |= 1u << stage;
-          parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          k_issued |= 1u << ks;
+          k_par = (k_par & ~(1u << ks)) | (kph << ks);
+          if (++ks == kSlots) {
+            ks = 0;
+            kph ^= 1u;
+          }
+          if (!mbar_wait_bounded(&v_empty[vs], vph ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* vd = smem + kOffV + vs * kSlotBytes;
+          mbar_arrive_expect_tx(&v_full[vs], kSlotBytes);
+          if (cached) {
+            tma_load_2d(vd, &tmCache, &v_full[vs], 0, vrow);
+            tma_load_2d(vd + kSub, &tmCache, &v_full[vs], 64, vrow);
+          } else {
+            tma_load_3d(vd, &tmVnew, &v_full[vs], 0, kvh, t0);
+            tma_load_3d(vd + kSub, &tmVnew, &v_full[vs], 64, kvh, t0);
+          }
+          v_issued |= 1u << vs;
+          v_par = (v_par & ~(1u << vs)) | (vph << vs);
+          if (++vs == kSlots) {
+            vs = 0;
+            vph ^= 1u;
           }
         }
       }
       if (!ok) {
-        for (int s = 0; s < kStages; ++s)
-          if (issued & (1u << s)) drain_wait(&kv_full[s], (parity_bits >> s) & 1u);
+        // let the copies already in flight land before the CTA exits
+        if (q_issued) drain_wait(q_full, q_par);
+        for (int s = 0; s < kSlots; ++s) {
+          if (k_issued & (1u << s)) drain_wait(&k_full[s], (k_par >> s) & 1u);
+          if (v_issued & (1u << s)) drain_wait(&v_full[s], (v_par >> s) & 1u);
+        }
       }
     }
   } else if (warp == 1) {
@@ -279,74 +328,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16(kQ, kKT);
       constexpr uint32_t idesc_o = umma_idesc_bf16(kQ, kHD) | (1u << 16);   // B (V) MN-major
-      const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffKV));
-      const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffKV + 2 * kSub), kSub);
+      const uint64_t q_desc = umma_desc_sw128(smem_u32(smem + kOffQ));
+      const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffK));
+      const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffV), kSub);
       bool ok = true;
       bool issued = false;
-      int stage = 0, prev_stage = 0;
-      uint32_t phase = 0;
-      int g = 0;                      // tile counter over all items (S/P buffer rotation)
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0;
+      // S(t) = Q K(t)^T into buffer t % kSBufs, t counting key tiles over all items;
+      // the buffer is free once PV(t - kSBufs), which read its P, has completed
+      auto issue_s = [&](int t) -> bool {
+        const int buf = t % kSBufs;
+        if (!mbar_wait_bounded(&k_full[ks], kph, abort_flag, p.status) ||
+            !mbar_wait_bounded(&pv_done[buf], ((t / kSBufs) & 1u) ^ 1u, abort_flag, p.status))
+          return false;
+        tc_fence_after();
+        const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((ks * kSlotBytes) >> 4);
+        const uint32_t d_s = tmem + buf * kKT;
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          // dims 16kk..16kk+15: 32-byte step inside a 64-dim sub-tile
+          const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+          umma_bf16(d_s, q_desc + (koff >> 4), k_desc + (koff >> 4), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        umma_commit(&s_full[buf]);
+        umma_commit(&k_empty[ks]);
+        if (++ks == kSlots) {
+          ks = 0;
+          kph ^= 1u;
+        }
+        return true;
+      };
+      int g = 0;
       Item it;
       for (int k = 0; ok && get_item(p, k, it); ++k) {
-        // Q of this item staged in TMEM; the previous item's output read out
-        if (!mbar_wait_bounded(q_full, k & 1u, abort_flag, p.status) ||
-            (k > 0 && !mbar_wait_bounded(o_empty, (k - 1) & 1u, abort_flag, p.status))) {
+        const int n = it.n_tiles;
+        if (!mbar_wait_bounded(q_full, k & 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        for (int j = 0; ok && j <= it.n_tiles; ++j) {
-          if (j < it.n_tiles) {
-            const int t = g + j;
-            const int buf = t % kSBufs;
-            // S(t) overwrites the buffer whose P fed PV(t - kSBufs): wait for that PV
-            if (!mbar_wait_bounded(&kv_full[stage], phase, abort_flag, p.status) ||
-                !mbar_wait_bounded(&pv_done[buf], ((t / kSBufs) & 1u) ^ 1u, abort_flag, p.status)) {
+        // S runs two key tiles ahead of PV
+        for (int i = 0; ok && i < 2 && i < n; ++i) ok = issue_s(g + i);
+        if (!ok) break;
+        if (n <= 2) umma_commit(q_empty);
+        for (int i = 0; i < n; ++i) {
+          const int t = g + i;
+          const int buf = t % kSBufs;
+          // O += P(i) V(i); the first PV of an item overwrites O, which the
+          // softmax warps must have read out for the previous item
+          if (!mbar_wait_bounded(&p_full[buf], (t / kSBufs) & 1u, abort_flag, p.status) ||
+              (i == 0 && k > 0 &&
+               !mbar_wait_bounded(o_empty, (k - 1) & 1u, abort_flag, p.status)) ||
+              !mbar_wait_bounded(&v_full[vs], vph, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((vs * kSlotBytes) >> 4);
+          const uint32_t p_col = tmem + buf * kKT;
+#pragma unroll
+          for (int kk = 0; kk < kKT / 16; ++kk) {
+            // keys 16kk..16kk+15 sit in columns 32*(kk/2) + 8*(kk%2) .. +7 of the buffer
+            const uint32_t a = p_col + 32 * (kk >> 1) + 8 * (kk & 1);
+            umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
+                         (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&pv_done[buf]);
+          umma_commit(&v_empty[vs]);
+          if (++vs == kSlots) {
+            vs = 0;
+            vph ^= 1u;
+          }
+          if (i == n - 1) umma_commit(o_full);
+          if (i + 2 < n) {
+            if (!issue_s(t + 2)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((stage * kStageBytes) >> 4);
-            const uint32_t d_s = tmem + buf * kKT;
-#pragma unroll
-            for (int kk = 0; kk < kHD / 16; ++kk) {
-              // A = Q from TMEM (dims 16kk.. in columns 8kk..), B = K from shared memory
-              const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-              umma_bf16_ts(d_s, tmem + kColQ + 8 * kk, k_desc + (koff >> 4), idesc_s,
-                           kk > 0 ? 1u : 0u);
-            }
-            issued = true;
-            umma_commit(&s_full[buf]);
-          }
-          if (j > 0) {
-            // O += P(i) V(i), P read from TMEM
-            const int i = j - 1;
-            const int t = g + i;
-            const int buf = t % kSBufs;
-            if (!mbar_wait_bounded(&p_full[buf], (t / kSBufs) & 1u, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((prev_stage * kStageBytes) >> 4);
-            const uint32_t p_col = tmem + buf * kKT;
-#pragma unroll
-            for (int kk = 0; kk < kKT / 16; ++kk) {
-              // keys 16kk..16kk+15 sit in columns 32*(kk/2) + 8*(kk%2) .. +7 of the buffer
-              const uint32_t a = p_col + 32 * (kk >> 1) + 8 * (kk & 1);
-              umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
-                           (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(&pv_done[buf]);
-            umma_commit(&kv_empty[prev_stage]);
-            if (i == it.n_tiles - 1) umma_commit(o_full);
-          }
-          prev_stage = stage;
-          if (j < it.n_tiles && ++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+            if (i + 2 == n - 1) umma_commit(q_empty);   // last S of the item
           }
         }
-        g += it.n_tiles;
+        g += n;
       }
       if (!ok && issued) {
         umma_commit(drain);
@@ -369,28 +432,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     Item it;
     for (int k = 0; ok && get_item(p, k, it); ++k) {
-      {
-        // stage this thread's quarter of its Q row (32 dims) into TMEM
-        // columns kColQ + 16*quarter.. as bf16 pairs: the A operand of S = Q K^T.
-        // The previous item's MMAs have all completed (its o_full was awaited).
-        uint32_t qv[16];
-        if (r < it.rows) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.q + (static_cast<size_t>(it.m0 + r) * p.n_q_heads + it.head) * kHD + quarter * 32);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 v = src[c];
-            qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) qv[c] = 0u;
-        }
-        tmem_st16(lane_addr + kColQ + quarter * 16, qv);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(q_full);
-      }
       const int qp = it.q_lo + r;
       float l = 0.f;
       for (int i = 0; i < it.n_tiles; ++i) {
@@ -432,7 +473,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[buf]);
+        // one arrival per warp: 512 arrivals on one mbarrier serialise for
+        // thousands of cycles
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[buf]);
       }
       g += it.n_tiles;
       const bool done = __all_sync(0xFFFFFFFFu, ok) &&
@@ -453,7 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float o[32];
         tmem_ld32(lane_addr + kColO + quarter * 32, o);
         tc_fence_before();
-        mbar_arrive(o_empty);      // O may be overwritten by the next item
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_empty);      // O may be overwritten by the next item
         if (row_ok) {
           uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -518,8 +563,9 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
                                         const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                         const KvLayerView& kv, cudaStream_t s) {
   if (p.n <= 0) return cudaSuccess;
-  CUtensorMap tk, tv, tc;
-  if (!make_tmap_3d(&tk, k_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
+  CUtensorMap tq, tk, tv, tc;
+  if (!make_tmap_3d(&tq, q, kHD, p.n_q_heads, p.n, 64, 1, kQ) ||
+      !make_tmap_3d(&tk, k_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
       !make_tmap_3d(&tv, v_new, kHD, p.n_kv, p.n, 64, 1, kKT) ||
       !make_tmap_bf16(&tc, kv.k_base, static_cast<uint64_t>(kv.max_seqs) * 2 * kv.n_kv * kv.cap,
                       kHD, kKT))
@@ -541,7 +587,7 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
   dim3 grid(items < dev_sms ? items : dev_sms);
   PrefillAttnTcParams pq = p;
   pq.q = q;
-  prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tk, tv, tc, pq);
+  prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, pq);
   return cudaGetLastError();
 }
 

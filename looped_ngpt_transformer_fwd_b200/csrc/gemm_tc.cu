@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 4);   // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -328,7 +328,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int g = 0; g < BN / HD; ++g) epi_qkvg_group<HD>(p, taddr + g * HD, row, nt * BN + g * HD);
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      // one arrival per warp: many arrivals on one mbarrier are serialised
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
   }
 
