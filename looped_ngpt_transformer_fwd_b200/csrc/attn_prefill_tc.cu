@@ -18,11 +18,12 @@
 // longest first in snake order; 128-key K/V tiles.  Warp 0 issues TMA loads:
 // the item's Q tile, and K and V tiles through two separate 3-slot rings (from
 // the layer's cache for positions below pos0, from this call's fresh K/V
-// otherwise).  Warp 1 owns TMEM and issues the MMAs: S = Q K^T (N = 128 keys)
-// into one of three 128-column buffers, and O += P V with the A operand (P)
-// read from TMEM, where the softmax warps wrote it over S.  Three S buffers let
-// S run two key tiles ahead of P V, so the tensor core always has the next
-// S = Q K^T queued behind each P V and never waits out a completion round trip.
+// otherwise).  Warp 1 owns TMEM and issues S = Q K^T (N = 128 keys) into one of
+// three 128-column buffers; warp 18 issues O += P V with the A operand (P)
+// read from TMEM, where the softmax warps wrote it over S.  Two issuing
+// threads keep the two dependency chains apart: a wait in one (for P, or for
+// a free S buffer) never holds back MMAs of the other, and with three S
+// buffers S runs up to two key tiles ahead of P V.
 // Sixteen softmax warps (row quadrant x key quarter) turn S into P =
 // exp2(...) in place (mask, exp2 on the MUFU and FMA pipes, row sums) and
 // finally write gate * O / l.  Every wait is bounded.
@@ -41,7 +42,8 @@ constexpr int kHD = 128;
 constexpr int kSlots = 3;         // K ring and V ring depth
 constexpr int kSoftmaxWarps = 16; // 4 row quadrants x 4 column quarters of 32 keys
 constexpr int kSoftThreads = 32 * kSoftmaxWarps;
-constexpr int kThreads = 64 + kSoftThreads;
+constexpr int kPvWarp = 2 + kSoftmaxWarps;        // issues the O += P V MMAs
+constexpr int kThreads = 64 + kSoftThreads + 32;
 constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 rows x 64 dims (one TMA box)
 constexpr int kSlotBytes = 2 * kSub;                  // one K or V tile, or the Q tile
 // shared memory (base 1024-aligned): K ring | V ring | Q | row sums | barriers
@@ -201,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pv_done = p_full + kSBufs;          // [kSBufs] the PV MMAs reading buffer b completed
   uint64_t* o_full = pv_done + kSBufs;          // all MMAs of the current item completed
   uint64_t* o_empty = o_full + 1;               // its output was read from TMEM
-  uint64_t* drain = o_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = o_empty + 1;                // [2]: S issuer, PV issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(o_full, 1);
     mbar_init(o_empty, kSoftmaxWarps);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     fence_proxy_async_smem();
@@ -325,42 +328,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ------------------------------------------------------- MMA issuer
+      // ------------------------------------------------------- S = Q K^T issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16(kQ, kKT);
-      constexpr uint32_t idesc_o = umma_idesc_bf16(kQ, kHD) | (1u << 16);   // B (V) MN-major
       const uint64_t q_desc = umma_desc_sw128(smem_u32(smem + kOffQ));
       const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffK));
-      const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffV), kSub);
       bool ok = true;
       bool issued = false;
-      int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0;
-      // S(t) = Q K(t)^T into buffer t % kSBufs, t counting key tiles over all items;
-      // the buffer is free once PV(t - kSBufs), which read its P, has completed
-      auto issue_s = [&](int t) -> bool {
-        const int buf = t % kSBufs;
-        if (!mbar_wait_bounded(&k_full[ks], kph, abort_flag, p.status) ||
-            !mbar_wait_bounded(&pv_done[buf], ((t / kSBufs) & 1u) ^ 1u, abort_flag, p.status))
-          return false;
-        tc_fence_after();
-        const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((ks * kSlotBytes) >> 4);
-        const uint32_t d_s = tmem + buf * kKT;
-#pragma unroll
-        for (int kk = 0; kk < kHD / 16; ++kk) {
-          // dims 16kk..16kk+15: 32-byte step inside a 64-dim sub-tile
-          const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
-          umma_bf16(d_s, q_desc + (koff >> 4), k_desc + (koff >> 4), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        issued = true;
-        umma_commit(&s_full[buf]);
-        umma_commit(&k_empty[ks]);
-        if (++ks == kSlots) {
-          ks = 0;
-          kph ^= 1u;
-        }
-        return true;
-      };
-      int g = 0;
+      int ks = 0;
+      uint32_t kph = 0;
+      int g = 0;                      // key tiles of earlier items (S/P buffer rotation)
       Item it;
       for (int k = 0; ok && get_item(p, k, it); ++k) {
         const int n = it.n_tiles;
@@ -368,15 +344,59 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // S runs two key tiles ahead of PV
-        for (int i = 0; ok && i < 2 && i < n; ++i) ok = issue_s(g + i);
-        if (!ok) break;
-        if (n <= 2) umma_commit(q_empty);
+        for (int i = 0; i < n; ++i) {
+          // S(t) goes to buffer t % kSBufs, free once PV(t - kSBufs), which
+          // read the P written there, has completed
+          const int t = g + i;
+          const int buf = t % kSBufs;
+          if (!mbar_wait_bounded(&k_full[ks], kph, abort_flag, p.status) ||
+              !mbar_wait_bounded(&pv_done[buf], ((t / kSBufs) & 1u) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((ks * kSlotBytes) >> 4);
+          const uint32_t d_s = tmem + buf * kKT;
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            // dims 16kk..16kk+15: 32-byte step inside a 64-dim sub-tile
+            const uint32_t koff = (kk >> 2) * kSub + (kk & 3) * 32;
+            umma_bf16(d_s, q_desc + (koff >> 4), k_desc + (koff >> 4), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(&s_full[buf]);
+          umma_commit(&k_empty[ks]);
+          if (++ks == kSlots) {
+            ks = 0;
+            kph ^= 1u;
+          }
+          if (i == n - 1) umma_commit(q_empty);   // the Q slot may take the next item's tile
+        }
+        g += n;
+      }
+      if (!ok && issued) {
+        umma_commit(&drain[0]);
+        drain_wait(&drain[0], 0);
+      }
+    }
+  } else if (warp == kPvWarp) {
+    if (lane == 0) {
+      // ------------------------------------------------------- O += P V issuer
+      constexpr uint32_t idesc_o = umma_idesc_bf16(kQ, kHD) | (1u << 16);   // B (V) MN-major
+      const uint64_t v_desc0 = umma_desc_sw128_mn(smem_u32(smem + kOffV), kSub);
+      bool ok = true;
+      bool issued = false;
+      int vs = 0;
+      uint32_t vph = 0;
+      int g = 0;
+      Item it;
+      for (int k = 0; ok && get_item(p, k, it); ++k) {
+        const int n = it.n_tiles;
         for (int i = 0; i < n; ++i) {
           const int t = g + i;
           const int buf = t % kSBufs;
-          // O += P(i) V(i); the first PV of an item overwrites O, which the
-          // softmax warps must have read out for the previous item
+          // the first PV of an item overwrites O, which the softmax warps
+          // must have read out for the previous item
           if (!mbar_wait_bounded(&p_full[buf], (t / kSBufs) & 1u, abort_flag, p.status) ||
               (i == 0 && k > 0 &&
                !mbar_wait_bounded(o_empty, (k - 1) & 1u, abort_flag, p.status)) ||
@@ -394,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16_ts(tmem + kColO, a, v_desc + ((kk * 2048) >> 4), idesc_o,
                          (i > 0 || kk > 0) ? 1u : 0u);
           }
+          issued = true;
           umma_commit(&pv_done[buf]);
           umma_commit(&v_empty[vs]);
           if (++vs == kSlots) {
@@ -401,23 +422,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             vph ^= 1u;
           }
           if (i == n - 1) umma_commit(o_full);
-          if (i + 2 < n) {
-            if (!issue_s(t + 2)) {
-              ok = false;
-              break;
-            }
-            if (i + 2 == n - 1) umma_commit(q_empty);   // last S of the item
-          }
         }
         g += n;
       }
       if (!ok && issued) {
-        umma_commit(drain);
-        drain_wait(drain, 0);
+        umma_commit(&drain[1]);
+        drain_wait(&drain[1], 0);
       }
     }
   } else {
-    // ----------------------------------------------------- softmax / output
+    // ----------------------------------------------------- softmax / output (warps 2..17)
     // warp w reads TMEM lanes 32*(w%4).. (its row quadrant) and one quarter
     // (32 keys) of every S tile; it writes that quarter's P as bf16 pairs into
     // the first 16 columns of the quarter, which only it has read.
