@@ -16,8 +16,9 @@
 //
 // Persistent: one CTA per SM works through (128-query tile, head) items dealt
 // longest first in snake order; 128-key K/V tiles.  Warp 0 issues TMA loads:
-// the item's Q tile, and K and V tiles through two separate 3-slot rings (from
-// the layer's cache for positions below pos0, from this call's fresh K/V
+// Q tiles into two slots (the next item's Q lands while this one runs), K
+// tiles through a 2-slot ring and V tiles through a 3-slot ring (from the
+// layer's cache for positions below pos0, from this call's fresh K/V
 // otherwise).  Warp 1 owns TMEM and issues S = Q K^T (N = 128 keys) into one of
 // three 128-column buffers; warp 18 issues O += P V with the A operand (P)
 // read from TMEM, where the softmax warps wrote it over S.  Two issuing
@@ -39,18 +40,20 @@ namespace {
 constexpr int kQ = 128;           // queries per item (one TMEM lane each)
 constexpr int kKT = 128;          // keys per tile
 constexpr int kHD = 128;
-constexpr int kSlots = 3;         // K ring and V ring depth
+constexpr int kKSlots = 2;        // K ring depth (a K tile is free once its S completes)
+constexpr int kVSlots = 3;        // V ring depth
+constexpr int kQSlots = 2;        // Q tiles: the next item's loads during this one
 constexpr int kSoftmaxWarps = 16; // 4 row quadrants x 4 column quarters of 32 keys
 constexpr int kSoftThreads = 32 * kSoftmaxWarps;
 constexpr int kPvWarp = 2 + kSoftmaxWarps;        // issues the O += P V MMAs
 constexpr int kThreads = 64 + kSoftThreads + 32;
 constexpr int kSub = kKT * 64 * 2;                    // 16 KB: 128 rows x 64 dims (one TMA box)
 constexpr int kSlotBytes = 2 * kSub;                  // one K or V tile, or the Q tile
-// shared memory (base 1024-aligned): K ring | V ring | Q | row sums | barriers
+// shared memory (base 1024-aligned): K ring | V ring | Q slots | row sums | barriers
 constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + kSlots * kSlotBytes;
-constexpr int kOffQ = kOffV + kSlots * kSlotBytes;
-constexpr int kOffL = kOffQ + kSlotBytes;             // row-sum exchange, 128 x 4 floats
+constexpr int kOffV = kOffK + kKSlots * kSlotBytes;
+constexpr int kOffQ = kOffV + kVSlots * kSlotBytes;
+constexpr int kOffL = kOffQ + kQSlots * kSlotBytes;   // row-sum exchange, 128 x 4 floats
 constexpr int kOffBar = kOffL + kQ * 4 * 4;
 constexpr int kSmemBytes = kOffBar + 256;
 constexpr int kSBufs = 3;                             // S/P buffers in TMEM
@@ -192,13 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bars;                      // Q tile of the current item landed
-  uint64_t* q_empty = q_full + 1;               // all S MMAs of the previous item completed
-  uint64_t* k_full = q_empty + 1;               // [kSlots]
-  uint64_t* k_empty = k_full + kSlots;          // [kSlots]
-  uint64_t* v_full = k_empty + kSlots;          // [kSlots]
-  uint64_t* v_empty = v_full + kSlots;          // [kSlots]
-  uint64_t* s_full = v_empty + kSlots;          // [kSBufs] S tile in TMEM buffer b is ready
+  uint64_t* q_full = bars;                      // [kQSlots] Q tile landed (item k uses slot k % 2)
+  uint64_t* q_empty = q_full + kQSlots;         // [kQSlots] all S MMAs reading the slot completed
+  uint64_t* k_full = q_empty + kQSlots;         // [kKSlots]
+  uint64_t* k_empty = k_full + kKSlots;         // [kKSlots]
+  uint64_t* v_full = k_empty + kKSlots;         // [kVSlots]
+  uint64_t* v_empty = v_full + kVSlots;         // [kVSlots]
+  uint64_t* s_full = v_empty + kVSlots;         // [kSBufs] S tile in TMEM buffer b is ready
   uint64_t* p_full = s_full + kSBufs;           // [kSBufs] P tile written over buffer b (one arrival per softmax warp)
   uint64_t* pv_done = p_full + kSBufs;          // [kSBufs] the PV MMAs reading buffer b completed
   uint64_t* o_full = pv_done + kSBufs;          // all MMAs of the current item completed
@@ -211,11 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int group_size = p.n_q_heads / p.n_kv;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < kQSlots; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -255,21 +262,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kph = 0, vph = 0;
       // parity of the last copy into each slot, for draining after an error
       uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
-      bool q_issued = false;
-      uint32_t q_par = 0;
+      uint32_t q_issued = 0, q_par = 0;
       Item it;
       for (int k = 0; ok && get_item(p, k, it); ++k) {
         const int kvh = it.head / group_size;
-        // the Q slot is free once every S MMA of the previous item has completed
-        if (!mbar_wait_bounded(q_empty, (k & 1u) ^ 1u, abort_flag, p.status)) {
+        // Q slot k % 2 is free once every S MMA of item k - 2 has completed
+        const int qs = k & 1;
+        const uint32_t qph = (k >> 1) & 1u;
+        if (!mbar_wait_bounded(&q_empty[qs], qph ^ 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(q_full, kSlotBytes);
-        tma_load_3d(smem + kOffQ, &tmQ, q_full, 0, it.head, it.m0);
-        tma_load_3d(smem + kOffQ + kSub, &tmQ, q_full, 64, it.head, it.m0);
-        q_issued = true;
-        q_par = k & 1u;
+        uint8_t* qd = smem + kOffQ + qs * kSlotBytes;
+        mbar_arrive_expect_tx(&q_full[qs], kSlotBytes);
+        tma_load_3d(qd, &tmQ, &q_full[qs], 0, it.head, it.m0);
+        tma_load_3d(qd + kSub, &tmQ, &q_full[qs], 64, it.head, it.m0);
+        q_issued |= 1u << qs;
+        q_par = (q_par & ~(1u << qs)) | (qph << qs);
         for (int j = 0; j < it.n_tiles; ++j) {
           const int kp0 = (it.kt_begin + j) * kKT;
           // cached positions: slot rows of this sequence's K and V planes
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           k_issued |= 1u << ks;
           k_par = (k_par & ~(1u << ks)) | (kph << ks);
-          if (++ks == kSlots) {
+          if (++ks == kKSlots) {
             ks = 0;
             kph ^= 1u;
           }
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           v_issued |= 1u << vs;
           v_par = (v_par & ~(1u << vs)) | (vph << vs);
-          if (++vs == kSlots) {
+          if (++vs == kVSlots) {
             vs = 0;
             vph ^= 1u;
           }
@@ -319,18 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // let the copies already in flight land before the CTA exits
-        if (q_issued) drain_wait(q_full, q_par);
-        for (int s = 0; s < kSlots; ++s) {
+        for (int s = 0; s < kQSlots; ++s)
+          if (q_issued & (1u << s)) drain_wait(&q_full[s], (q_par >> s) & 1u);
+        for (int s = 0; s < kKSlots; ++s)
           if (k_issued & (1u << s)) drain_wait(&k_full[s], (k_par >> s) & 1u);
+        for (int s = 0; s < kVSlots; ++s)
           if (v_issued & (1u << s)) drain_wait(&v_full[s], (v_par >> s) & 1u);
-        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- S = Q K^T issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16(kQ, kKT);
-      const uint64_t q_desc = umma_desc_sw128(smem_u32(smem + kOffQ));
+      const uint64_t q_desc0 = umma_desc_sw128(smem_u32(smem + kOffQ));
       const uint64_t k_desc0 = umma_desc_sw128(smem_u32(smem + kOffK));
       bool ok = true;
       bool issued = false;
@@ -340,10 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       for (int k = 0; ok && get_item(p, k, it); ++k) {
         const int n = it.n_tiles;
-        if (!mbar_wait_bounded(q_full, k & 1u, abort_flag, p.status)) {
+        const int qs = k & 1;
+        if (!mbar_wait_bounded(&q_full[qs], (k >> 1) & 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
+        const uint64_t q_desc = q_desc0 + static_cast<uint64_t>((qs * kSlotBytes) >> 4);
         for (int i = 0; i < n; ++i) {
           // S(t) goes to buffer t % kSBufs, free once PV(t - kSBufs), which
           // read the P written there, has completed
@@ -366,11 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued = true;
           umma_commit(&s_full[buf]);
           umma_commit(&k_empty[ks]);
-          if (++ks == kSlots) {
+          if (++ks == kKSlots) {
             ks = 0;
             kph ^= 1u;
           }
-          if (i == n - 1) umma_commit(q_empty);   // the Q slot may take the next item's tile
+          if (i == n - 1) umma_commit(&q_empty[qs]);   // the slot may take item k + 2's Q
         }
         g += n;
       }
@@ -417,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued = true;
           umma_commit(&pv_done[buf]);
           umma_commit(&v_empty[vs]);
-          if (++vs == kSlots) {
+          if (++vs == kVSlots) {
             vs = 0;
             vph ^= 1u;
           }
