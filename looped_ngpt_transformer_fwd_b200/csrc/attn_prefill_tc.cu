@@ -446,7 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------- softmax / output (warps 2..17)
     // warp w reads TMEM lanes 32*(w%4).. (its row quadrant) and one quarter
     // (32 keys) of every S tile; it writes that quarter's P as bf16 pairs into
-    // the first 16 columns of the quarter, which only it has read.
+    // the first 16 columns of the quarter, which only it has read.  The output
+    // gate * O / l of item k is written after the first tile of item k + 1,
+    // when the last PV of item k has long completed, so the softmax warps do
+    // not wait for it.
     const int quarter = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                // query row of this thread
@@ -454,60 +457,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale = p.scale_log2, moff = p.m_log2;
     const int window = p.window;
     float* lsum = reinterpret_cast<float*>(smem + kOffL);
-    bool ok = true;
-    int g = 0;
-    Item it;
-    for (int k = 0; ok && get_item(p, k, it); ++k) {
+    int g = 0;                                     // key tiles of earlier items
+
+    // S -> P for key tile i of item `it`, adding to the row sum l; false when
+    // a wait gave up (warp-uniform: TMEM loads and stores are warp-collective)
+    auto softmax_tile = [&](const Item& it, int i, float& l) -> bool {
+      const int t = g + i;
+      const int buf = t % kSBufs;
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait_bounded(&s_full[buf], (t / kSBufs) & 1u, abort_flag, p.status)))
+        return false;
+      tc_fence_after();
+      float sv[32];
+      tmem_ld32(lane_addr + buf * kKT + quarter * 32, sv);
       const int qp = it.q_lo + r;
-      float l = 0.f;
-      for (int i = 0; i < it.n_tiles; ++i) {
-        const int t = g + i;
-        const int buf = t % kSBufs;
-        // warp-uniform: TMEM loads and stores are warp-collective
-        if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait_bounded(&s_full[buf], (t / kSBufs) & 1u, abort_flag, p.status))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float sv[32];
-        tmem_ld32(lane_addr + buf * kKT + quarter * 32, sv);
-        const int kp0 = (it.kt_begin + i) * kKT + quarter * 32;
-        const bool need_mask = (kp0 < it.key_lo) || (kp0 + 31 > it.q_lo) ||
-                               (window > 0 && it.q_hi - kp0 >= window);
-        uint32_t packed[16];
+      const int kp0 = (it.kt_begin + i) * kKT + quarter * 32;
+      const bool need_mask = (kp0 < it.key_lo) || (kp0 + 31 > it.q_lo) ||
+                             (window > 0 && it.q_hi - kp0 >= window);
+      uint32_t packed[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          float e[4];
+      for (int c = 0; c < 32; c += 4) {
+        float e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x = fmaf(sv[c + u], scale, -moff);
+          e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
+        }
+        if (need_mask) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float x = fmaf(sv[c + u], scale, -moff);
-            e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
+            const int kp = kp0 + c + u;
+            const bool keep = kp <= qp && (window <= 0 || qp - kp < window);
+            e[u] = keep ? e[u] : 0.f;
           }
-          if (need_mask) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int kp = kp0 + c + u;
-              const bool keep = kp <= qp && (window <= 0 || qp - kp < window);
-              e[u] = keep ? e[u] : 0.f;
-            }
-          }
-          l += (e[0] + e[1]) + (e[2] + e[3]);
-          packed[c / 2] = pack_bf16x2(e[0], e[1]);
-          packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
         }
-        tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
-        tmem_wait_st();
-        tc_fence_before();
-        // one arrival per warp: 512 arrivals on one mbarrier serialise for
-        // thousands of cycles
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
+        l += (e[0] + e[1]) + (e[2] + e[3]);
+        packed[c / 2] = pack_bf16x2(e[0], e[1]);
+        packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
       }
-      g += it.n_tiles;
-      const bool done = __all_sync(0xFFFFFFFFu, ok) &&
+      tmem_st16(lane_addr + buf * kKT + quarter * 32, packed);
+      tmem_wait_st();
+      tc_fence_before();
+      // one arrival per warp: 512 arrivals on one mbarrier serialise for
+      // thousands of cycles
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[buf]);
+      return true;
+    };
+
+    // gate * O / l of item number kk to the output.  Every softmax thread
+    // calls it at the same point of its loop, failed or not; all get the same
+    // verdict (true = carry on).
+    auto epilogue = [&](const Item& it, int kk, float l, float gate_v, bool good) -> bool {
+      const bool done = __all_sync(0xFFFFFFFFu, good) &&
                         __all_sync(0xFFFFFFFFu,
-                                   mbar_wait_bounded(o_full, k & 1u, abort_flag, p.status));
+                                   mbar_wait_bounded(o_full, kk & 1u, abort_flag, p.status));
       // the four quarters of a row add their row sums
       if (done) lsum[r * 4 + quarter] = l;
       named_bar_sync(1, kSoftThreads);
@@ -516,17 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l_row = (lsum[r * 4] + lsum[r * 4 + 1]) + (lsum[r * 4 + 2] + lsum[r * 4 + 3]);
         const bool row_ok = r < it.rows;
         const int tok = it.m0 + r;
-        const float f =
-            row_ok ? p.gate[static_cast<size_t>(tok) * p.n_q_heads + it.head] / l_row : 0.f;
-        __nv_bfloat16* dst =
-            p.out + (static_cast<size_t>(tok) * p.n_q_heads + it.head) * kHD + quarter * 32;
+        const float f = row_ok ? gate_v / l_row : 0.f;
         float o[32];
         tmem_ld32(lane_addr + kColO + quarter * 32, o);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_empty);      // O may be overwritten by the next item
         if (row_ok) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          uint4* d4 = reinterpret_cast<uint4*>(
+              p.out + (static_cast<size_t>(tok) * p.n_q_heads + it.head) * kHD + quarter * 32);
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             d4[c] = make_uint4(pack_bf16x2(o[8 * c] * f, o[8 * c + 1] * f),
@@ -534,12 +536,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                                pack_bf16x2(o[8 * c + 4] * f, o[8 * c + 5] * f),
                                pack_bf16x2(o[8 * c + 6] * f, o[8 * c + 7] * f));
         }
-      } else {
-        ok = false;
       }
       // lsum is reused by the next item; all softmax warps leave the loop together
-      if (named_bar_any(1, kSoftThreads, !ok)) ok = false;
+      return !named_bar_any(1, kSoftThreads, !done);
+    };
+
+    bool ok = true;
+    bool pending = false;                          // an item's output is still to be written
+    Item it, prev;
+    float l_prev = 0.f, gate_prev = 0.f;
+    int k = 0;
+    for (; get_item(p, k, it); ++k) {
+      // this thread's gate value, loaded now so its latency is hidden
+      const float gate_v =
+          r < it.rows ? p.gate[static_cast<size_t>(it.m0 + r) * p.n_q_heads + it.head] : 0.f;
+      float l = 0.f;
+      if (ok) ok = softmax_tile(it, 0, l);
+      if (pending) {
+        pending = false;
+        ok = epilogue(prev, k - 1, l_prev, gate_prev, ok);
+        if (!ok) break;
+      }
+      for (int i = 1; ok && i < it.n_tiles; ++i) ok = softmax_tile(it, i, l);
+      g += it.n_tiles;
+      prev = it;
+      l_prev = l;
+      gate_prev = gate_v;
+      pending = true;
     }
+    if (pending) epilogue(prev, k - 1, l_prev, gate_prev, ok);
   }
 
   tc_fence_before();
