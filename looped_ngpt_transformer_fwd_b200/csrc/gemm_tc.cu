@@ -16,6 +16,7 @@
 // records kStatusTimeout, drains its outstanding copies and MMAs, frees TMEM
 // and returns.
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -35,9 +36,35 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
+  // fp32 output staging for bulk tensor stores: 4 epilogue warps x 2 buffers
+  // of 32 rows x 32 columns
+  static constexpr int kOutBufBytes = 32 * 32 * 4;
+  static constexpr int kOutStageBytes = 4 * 2 * kOutBufBytes;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + kBarBytes + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
+
+// Bulk tensor store of one staged box (shared -> global, no multicast) and
+// the bulk-group bookkeeping around it.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t c0,
+                                             int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// at most one bulk group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 // --------------------------------------------------------------- epilogues
 __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32], int valid) {
@@ -62,6 +89,38 @@ __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t tadd
     const int col = nt * BN + c;
     if (row_ok && col < p.N)
       store_f32_chunk(out + static_cast<size_t>(row) * p.ld_out + col, v, p.N - col);
+  }
+}
+
+// fp32 output through shared memory and bulk tensor stores: each warp stages
+// its 32 rows x 32 columns with the 128-byte swizzle (16-byte chunk j of row r
+// at chunk j ^ (r % 8), conflict-free) and one lane stores the box; the tensor
+// map [splits][M][N] clips rows past M and columns past N.  Two buffers per
+// warp alternate so staging overlaps the previous store.
+template <int BN>
+__device__ __forceinline__ void epi_store_f32_tma(const GemmParams& p, const CUtensorMap* tmC,
+                                                  uint32_t taddr, uint8_t* stage, int lane,
+                                                  int row0, int nt, int ks, uint32_t& nbuf) {
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float v[32];
+    tmem_ld32(taddr + c, v);
+    const int col = nt * BN + c;
+    if (col >= p.N) continue;                   // warp-uniform
+    uint8_t* buf = stage + (nbuf & 1u) * (32 * 32 * 4);
+    if (lane == 0) bulk_wait_read_1();          // the store that last read `buf` is done
+    __syncwarp();
+    float4* rowp = reinterpret_cast<float4*>(buf + lane * 128);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      rowp[j ^ (lane & 7)] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    fence_proxy_async_smem();                   // generic-proxy writes -> bulk copy
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(tmC, buf, col, row0, ks);
+      bulk_commit();
+    }
+    ++nbuf;
   }
 }
 
@@ -163,14 +222,15 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 template <int BN, int HD, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using C = GemmCfg<BN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint8_t* out_stage = smem + S * C::kStageBytes;   // 1024-aligned: stage bytes are multiples of 1 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + C::kOutStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
@@ -306,6 +366,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---------------------------------------------------- epilogue warps
     const int quad = warp & 3;
+    uint8_t* my_stage = out_stage + (warp - 2) * 2 * C::kOutBufBytes;
+    uint32_t nbuf = 0;                 // staged boxes so far (buffer rotation)
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const int mt = t % m_tiles;
@@ -320,7 +382,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int row = mt * kBM + quad * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       if constexpr (EPI == kEpiStoreF32) {
-        epi_store_f32<BN>(p, taddr, row, nt, ks);
+        if (p.c_tma)
+          epi_store_f32_tma<BN>(p, &tmC, taddr, my_stage, lane, mt * kBM + quad * 32, nt, ks, nbuf);
+        else
+          epi_store_f32<BN>(p, taddr, row, nt, ks);
       } else if constexpr (EPI == kEpiSwiGLU) {
         epi_swiglu<BN>(p, taddr, row, nt);
       } else {
@@ -332,6 +397,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    // bulk stores read shared memory until they complete: finish before exit
+    if (lane == 0 && nbuf > 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -340,6 +408,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return nullptr;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return encode;
+}
+
+// [k_splits][M][N] fp32 output viewed as a 3D tensor (N innermost, row pitch
+// ld_out, slice pitch split_stride) with 32 x 32 x 1 boxes and the 128-byte
+// swizzle.  False when the layout does not allow bulk tensor stores (the
+// kernel then stores from registers).
+bool make_tmap_out_f32(CUtensorMap* map, const GemmParams& p) {
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode || !p.out_f32 || p.N <= 0 || p.M <= 0) return false;
+  const uint64_t slice = p.k_splits > 1 ? p.split_stride : static_cast<uint64_t>(p.M) * p.ld_out;
+  if ((reinterpret_cast<uintptr_t>(p.out_f32) & 15) != 0 || (p.ld_out * 4ull) % 16 != 0 ||
+      (slice * 4ull) % 16 != 0 || p.ld_out < p.N || slice < static_cast<uint64_t>(p.M) * p.ld_out)
+    return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.N), static_cast<cuuint64_t>(p.M),
+                        static_cast<cuuint64_t>(p.k_splits)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.ld_out) * 4, slice * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.out_f32, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 template <int BN, int HD, int EPI>
@@ -361,7 +470,12 @@ cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   const int total = m_tiles * n_tiles * p.k_splits;
   const int grid = total < num_sms ? total : num_sms;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
+  GemmParams q = p;
+  CUtensorMap tmC;
+  memset(&tmC, 0, sizeof(tmC));
+  q.c_tma = 0;
+  if constexpr (EPI == kEpiStoreF32) q.c_tma = make_tmap_out_f32(&tmC, p) ? 1 : 0;
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, tmC, q);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@ struct GemmParams {
   float* out_f32 = nullptr;
   int ld_out = 0;
   size_t split_stride = 0;   // elements between K-split slices
+  int c_tma = 0;             // set by the launcher: output written by bulk tensor stores
   // kEpiSwiGLU: tile of BN columns = [BN/2 gate cols | BN/2 up cols]
   __nv_bfloat16* out_act = nullptr;
   int ld_act = 0;
