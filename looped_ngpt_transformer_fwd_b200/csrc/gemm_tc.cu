@@ -41,8 +41,16 @@ struct GemmCfg {
   static constexpr int kOutBufBytes = 32 * 32 * 4;
   static constexpr int kOutStageBytes = 4 * 2 * kOutBufBytes;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + kBarBytes + 1024;
+  static constexpr int kSqkBytes = 512;   // s_qk (head_dim <= 128 floats) for the QKVG epilogue
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + kOutStageBytes + kBarBytes + kSqkBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
+
+// Output tensor maps of one launch: fp32 output ([0]), or q / k / v for the
+// QKVG epilogue, or the activations ([0]) for SwiGLU.
+struct OutMaps {
+  CUtensorMap m[3];
 };
 
 // Bulk tensor store of one staged box (shared -> global, no multicast) and
@@ -53,6 +61,14 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
       "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
@@ -124,6 +140,56 @@ __device__ __forceinline__ void epi_store_f32_tma(const GemmParams& p, const CUt
   }
 }
 
+// Stage this lane's row of a 32-row x 64-column bf16 box (32 packed words,
+// 128-byte swizzle) and store the box at (x, y) through `map`.  The warp's two
+// staging buffers alternate; `nbuf` counts the boxes.
+__device__ __forceinline__ void store_box_bf16(const CUtensorMap* map, uint8_t* stage, int lane,
+                                               uint32_t& nbuf, const uint32_t (&w)[32], int x,
+                                               int y) {
+  uint8_t* buf = stage + (nbuf & 1u) * (32 * 32 * 4);
+  if (lane == 0) bulk_wait_read_1();          // the store that last read `buf` is done
+  __syncwarp();
+  uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 128);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    rowp[j ^ (lane & 7)] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, buf, x, y);
+    bulk_commit();
+  }
+  ++nbuf;
+}
+
+// SwiGLU activations in 64-column boxes through bulk tensor stores (rows past
+// M are clipped by the tensor map).
+template <int BN>
+__device__ __forceinline__ void epi_swiglu_tma(const GemmParams& p, const CUtensorMap* map,
+                                               uint32_t taddr, uint8_t* stage, int lane, int row0,
+                                               int nt, uint32_t& nbuf) {
+  constexpr int H = BN / 2;
+  static_assert(H % 64 == 0, "activation boxes are 64 columns wide");
+#pragma unroll 1
+  for (int c = 0; c < H; c += 64) {
+    uint32_t w[32];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float g[32], u[32];
+      tmem_ld32(taddr + c + 32 * half, g);
+      tmem_ld32(taddr + H + c + 32 * half, u);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float g0 = p.gate_scale * g[2 * i], g1 = p.gate_scale * g[2 * i + 1];
+        const float a0 = g0 * sigmoidf_(g0) * u[2 * i];
+        const float a1 = g1 * sigmoidf_(g1) * u[2 * i + 1];
+        w[16 * half + i] = pack_bf16x2(a0, a1);
+      }
+    }
+    store_box_bf16(map, stage, lane, nbuf, w, nt * H + c, row0);
+  }
+}
+
 template <int BN>
 __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, int row, int nt) {
   constexpr int H = BN / 2;
@@ -151,11 +217,19 @@ __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, 
 }
 
 // One head-sized column group (HD columns starting at global column col0).
+// q and k heads get RoPE, the per-head L2 norm and the scale s_qk (`sqk`, in
+// shared memory); v heads are stored as computed; gate logits go through the
+// sigmoid.  With bulk stores (p.c_tma) the warp stages 64-column boxes of q,
+// k or v and every lane takes part, rows past M included (the maps clip them).
 template <int HD>
-__device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t taddr, int row,
+__device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float* sqk,
+                                               const OutMaps* om, uint8_t* stage, int lane,
+                                               int row0, uint32_t& nbuf, uint32_t taddr, int row,
                                                int col0) {
   const int hq = p.n_q_heads, hkv = p.n_kv_heads;
   const int q_end = hq * HD, k_end = q_end + hkv * HD, v_end = k_end + hkv * HD;
+  const bool tma = p.c_tma != 0;
+  const bool row_ok = row < p.M;
   float x[HD];
 #pragma unroll
   for (int c = 0; c < HD; c += 32) {
@@ -164,9 +238,9 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t tad
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[c + i] = t[i];
   }
-  if (row >= p.M) return;
   if (col0 >= v_end) {
-    // attention output gate logits, one per query head
+    // attention output gate logits, one per query head (col0 is warp-uniform)
+    if (!row_ok) return;
     float* g = p.gate_out + static_cast<size_t>(row) * hq;
 #pragma unroll
     for (int i = 0; i < HD; ++i) {
@@ -175,11 +249,14 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t tad
     }
     return;
   }
-  __nv_bfloat16* dst;
+  if (!tma && !row_ok) return;
+  int which, head;
   if (col0 < k_end) {
     // RoPE (pairs i, i + HD/2) with this row's (cos, sin) table, then the
-    // per-head L2 norm and the learned per-dimension scale s_qk.
-    const float4* rt = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(row) * (HD / 2));
+    // per-head L2 norm and the learned per-dimension scale s_qk.  Rows past M
+    // read the last valid row's table (their results are clipped).
+    const int trow = row_ok ? row : p.M - 1;
+    const float4* rt = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(trow) * (HD / 2));
 #pragma unroll
     for (int i = 0; i < HD / 2; i += 2) {
       const float4 cs = rt[i / 2];   // cos_i, sin_i, cos_{i+1}, sin_{i+1}
@@ -195,20 +272,31 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, uint32_t tad
     for (int i = 0; i < HD; ++i) ss = fmaf(x[i], x[i], ss);
     const float inv = rsqrtf(fmaxf(ss, p.norm_eps));
 #pragma unroll
-    for (int i = 0; i < HD; ++i) x[i] *= inv * p.s_qk[i];
-    dst = (col0 < q_end)
-              ? p.q_out + (static_cast<size_t>(row) * hq + col0 / HD) * HD
-              : p.k_out + (static_cast<size_t>(row) * hkv + (col0 - q_end) / HD) * HD;
+    for (int i = 0; i < HD; ++i) x[i] *= inv * sqk[i];
+    which = col0 < q_end ? 0 : 1;
+    head = col0 < q_end ? col0 / HD : (col0 - q_end) / HD;
   } else {
-    dst = p.v_out + (static_cast<size_t>(row) * hkv + (col0 - k_end) / HD) * HD;
+    which = 2;
+    head = (col0 - k_end) / HD;
   }
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  if (tma) {
 #pragma unroll
-  for (int i = 0; i < HD / 8; ++i) {
+    for (int half = 0; half < HD / 64; ++half) {
+      uint32_t wb[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) wb[i] = pack_bf16x2(x[64 * half + 2 * i], x[64 * half + 2 * i + 1]);
+      store_box_bf16(&om->m[which], stage, lane, nbuf, wb, head * HD + 64 * half, row0);
+    }
+    return;
+  }
+  const int nh = which == 0 ? hq : hkv;
+  __nv_bfloat16* base = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out);
+  uint4* d4 = reinterpret_cast<uint4*>(base + (static_cast<size_t>(row) * nh + head) * HD);
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i)
     d4[i] = make_uint4(pack_bf16x2(x[8 * i], x[8 * i + 1]), pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
                        pack_bf16x2(x[8 * i + 4], x[8 * i + 5]),
                        pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
-  }
 }
 
 // A wait used only while cleaning up after an abort: short, ignores the flag.
@@ -222,7 +310,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 template <int BN, int HD, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                   const __grid_constant__ OutMaps om, const GemmParams p) {
   using C = GemmCfg<BN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -238,6 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = bars + 2 * S + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sqk = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (p.M + kBM - 1) / kBM;
@@ -267,6 +356,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
+  }
+  if constexpr (EPI == kEpiQKVG) {
+    if (threadIdx.x < HD) sqk[threadIdx.x] = p.s_qk[threadIdx.x];
   }
   tc_fence_before();
   __syncthreads();
@@ -383,14 +475,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       if constexpr (EPI == kEpiStoreF32) {
         if (p.c_tma)
-          epi_store_f32_tma<BN>(p, &tmC, taddr, my_stage, lane, mt * kBM + quad * 32, nt, ks, nbuf);
+          epi_store_f32_tma<BN>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt, ks, nbuf);
         else
           epi_store_f32<BN>(p, taddr, row, nt, ks);
       } else if constexpr (EPI == kEpiSwiGLU) {
-        epi_swiglu<BN>(p, taddr, row, nt);
+        if (p.c_tma)
+          epi_swiglu_tma<BN>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt, nbuf);
+        else
+          epi_swiglu<BN>(p, taddr, row, nt);
       } else {
 #pragma unroll 1
-        for (int g = 0; g < BN / HD; ++g) epi_qkvg_group<HD>(p, taddr + g * HD, row, nt * BN + g * HD);
+        for (int g = 0; g < BN / HD; ++g)
+          epi_qkvg_group<HD>(p, sqk, &om, my_stage, lane, mt * kBM + quad * 32, nbuf,
+                             taddr + g * HD, row, nt * BN + g * HD);
       }
       tc_fence_before();
       // one arrival per warp: many arrivals on one mbarrier are serialised
@@ -451,6 +548,21 @@ bool make_tmap_out_f32(CUtensorMap* map, const GemmParams& p) {
          CUDA_SUCCESS;
 }
 
+// [M][cols] bf16 output (row pitch ld elements) with 64 x 32 boxes and the
+// 128-byte swizzle; false when the layout does not allow bulk tensor stores.
+bool make_tmap_out_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld) {
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode || !base || rows <= 0 || cols <= 0 || cols % 64 != 0 || ld < cols) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (ld * 2ull) % 16 != 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int HD, int EPI>
 cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int num_sms, cudaStream_t s) {
@@ -471,11 +583,18 @@ cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   const int grid = total < num_sms ? total : num_sms;
   if (grid <= 0) return cudaSuccess;
   GemmParams q = p;
-  CUtensorMap tmC;
-  memset(&tmC, 0, sizeof(tmC));
+  OutMaps om;
+  memset(&om, 0, sizeof(om));
   q.c_tma = 0;
-  if constexpr (EPI == kEpiStoreF32) q.c_tma = make_tmap_out_f32(&tmC, p) ? 1 : 0;
-  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, tmC, q);
+  if constexpr (EPI == kEpiStoreF32) q.c_tma = make_tmap_out_f32(&om.m[0], p) ? 1 : 0;
+  if constexpr (EPI == kEpiSwiGLU)
+    q.c_tma = make_tmap_out_bf16(&om.m[0], p.out_act, p.M, p.N / 2, p.ld_act) ? 1 : 0;
+  if constexpr (EPI == kEpiQKVG)
+    q.c_tma = (make_tmap_out_bf16(&om.m[0], p.q_out, p.M, p.n_q_heads * HD, p.n_q_heads * HD) &&
+               make_tmap_out_bf16(&om.m[1], p.k_out, p.M, p.n_kv_heads * HD, p.n_kv_heads * HD) &&
+               make_tmap_out_bf16(&om.m[2], p.v_out, p.M, p.n_kv_heads * HD, p.n_kv_heads * HD))
+                  ? 1 : 0;
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, om, q);
   return cudaGetLastError();
 }
 
