@@ -49,9 +49,9 @@ WORKLOADS = {
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
 # one ncu capture, valid only while the kernel source is unchanged since.
 PROFILED = {
-    "gateup": {"traffic": 138453248 + 58353152,
+    "gateup": {"traffic": 138491136 + 54726144,
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
-                          "cdcf0126741e700b4780d8fe1bf042b1a0b9dfa8"),
+                          "f027590254f0c4cca999fbfb1fcf970c600ec6a3"),
                "profile": "profiles/gemm_tc_4b_prefill_full.md"},
     # decode attention: measured (read + write) / algorithmic bytes, applied to
     # the step's total KV bytes
