@@ -26,7 +26,7 @@
 // a free S buffer) never holds back MMAs of the other, and with three S
 // buffers S runs up to two key tiles ahead of P V.
 // Sixteen softmax warps (row quadrant x key quarter) turn S into P =
-// exp2(...) in place (mask, exp2 on the MUFU and FMA pipes, row sums) and
+// exp2(...) in place (mask, exp2 on the MUFU unit, row sums) and
 // finally write gate * O / l.  Every wait is bounded.
 #include <math.h>
 
@@ -100,22 +100,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x for -126 < x <= 0 on the FMA pipe, to share the exponential work with the
-// MUFU unit: Cody-Waite style reduction x = n + f with n = round(x) (the
-// 1.5 * 2^23 shifter), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients were fitted here to minimise the relative error on that
-// interval (max 7.5e-5, far below the bf16 rounding of P); 2^n added to the
-// exponent field.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float shifter = 12582912.0f;
-  const float t = x + shifter;
-  const float f = x - (t - shifter);
-  float p = fmaf(0.05517113f, f, 0.24261008f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.9999281f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -479,10 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 32; c += 4) {
         float e[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float x = fmaf(sv[c + u], scale, -moff);
-          e[u] = (u == 3) ? ex2_poly(x) : ex2(x);    // a quarter on the FMA pipe
-        }
+        for (int u = 0; u < 4; ++u) e[u] = ex2(fmaf(sv[c + u], scale, -moff));
         if (need_mask) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {

@@ -15,7 +15,7 @@ namespace dory {
 
 namespace {
 
-constexpr int kRowMaxChunks = 4;   // float4 chunks per thread
+constexpr int kRowMaxChunks = 3;   // float4 chunks per thread (256 threads for d = 3072)
 
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
