@@ -141,7 +141,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Work item k of this CTA: query tiles sorted longest first (the causal or
-// windowed key range grows with the query tile), dealt out round by round in
+// windowed key range grows with the query tile), dealt out one pass at a time in
 // alternating direction ("snake"), so every CTA gets a similar total.
 struct Item {
   int qblk, head, m0, rows, q_lo, q_hi, key_lo, kt_begin, n_tiles;
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // gate * O / l of item number kk to the output.  Every softmax thread
     // calls it at the same point of its loop, failed or not; all get the same
-    // verdict (true = carry on).
+    // result (true = carry on).
     auto epilogue = [&](const Item& it, int kk, float l, float gate_v, bool good) -> bool {
       const bool done = __all_sync(0xFFFFFFFFu, good) &&
                         __all_sync(0xFFFFFFFFu,
