@@ -175,6 +175,27 @@ DORY_API int dory_decode_step(dory_model* m, dory_kv* kv, int batch,
                      const void* h_in, void* h_out, int k,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* One decode step in which each sequence has its own loop count: row i runs
+ * d_k[i] recurrent loops (the loop count as a per-request dial: "NVIDIA
+ * Nemotron Labs Dory 1.0 4B: a looped (latent-recurrent) LLM with elastic
+ * inference compute", Why it matters here; prompts routed to different loop
+ * depths: "Dory1.0-4B: A Looped Normalized-GPT", Key Contributions).  Row i's
+ * result equals dory_decode_step of that row alone with k = d_k[i].
+ *   d_k    int32 device array [batch], each value in 1..k_hi (caller-owned,
+ *          read by the kernels, so a captured step replays across steps);
+ *   k_hi   the largest d_k[i]: the step runs k_hi loops and a row whose
+ *          count is below the current loop is left unchanged and writes no
+ *          cache entry.  It is checked like k of dory_decode_step
+ *          (DORY_ERR_K_RANGE, DORY_ERR_K_EXCEEDS_KMAX); a d_k[i] outside
+ *          1..k_hi leaves row i's recurrent loops undone and is reported as
+ *          DORY_ERR_DEVICE_BOUNDS by dory_device_status.
+ * Other arguments as for dory_decode_step.  Under per-loop caching each
+ * sequence's earlier tokens must have been written with the same count. */
+DORY_API int dory_decode_step_mixed(dory_model* m, dory_kv* kv, int batch,
+                     const int32_t* d_seq, const int32_t* d_pos, const int32_t* d_k, int k_hi,
+                     int max_pos_hint, const void* h_in, void* h_out,
+                     void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read and clear the model's device status word:
  * DORY_OK, DORY_ERR_DEVICE_TIMEOUT or DORY_ERR_DEVICE_BOUNDS. */
 DORY_API int dory_device_status(dory_model* m, void* stream);

@@ -27,7 +27,8 @@ STATUS = {
 # every entry point declared in include/dory.h
 EXPORTS = (
     "dory_weight_bytes", "dory_create", "dory_kv_bytes", "dory_kv_alloc", "dory_kv_layout",
-    "dory_workspace_bytes", "dory_prefill", "dory_decode_step", "dory_device_status",
+    "dory_workspace_bytes", "dory_prefill", "dory_decode_step", "dory_decode_step_mixed",
+    "dory_device_status",
     "dory_last_call_stats", "dory_error_string", "dory_kv_free", "dory_destroy",
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
     "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
@@ -87,6 +88,7 @@ def lib():
             "dory_workspace_bytes": (SZ, [P, I]),
             "dory_prefill": (I, [P, P, I, I, I, P, P, I, P, SZ, P]),
             "dory_decode_step": (I, [P, P, I, P, P, I, P, P, I, P, SZ, P]),
+            "dory_decode_step_mixed": (I, [P, P, I, P, P, P, I, I, P, P, P, SZ, P]),
             "dory_device_status": (I, [P, P]),
             "dory_last_call_stats": (I, [P, P, P]),
             "dory_error_string": (ctypes.c_char_p, [I]),
@@ -174,6 +176,13 @@ def dory_decode_step(model, kv, batch, d_seq, d_pos, max_pos_hint, h_in, h_out, 
                      stream):
     return check(lib().dory_decode_step(model, kv, batch, d_seq, d_pos, max_pos_hint, h_in, h_out,
                                         k, ws, ws_bytes, stream), "dory_decode_step")
+
+
+def dory_decode_step_mixed(model, kv, batch, d_seq, d_pos, d_k, k_hi, max_pos_hint, h_in, h_out,
+                           ws, ws_bytes, stream):
+    return check(lib().dory_decode_step_mixed(model, kv, batch, d_seq, d_pos, d_k, k_hi,
+                                              max_pos_hint, h_in, h_out, ws, ws_bytes, stream),
+                 "dory_decode_step_mixed")
 
 
 def dory_device_status(model, stream):

@@ -71,10 +71,11 @@ struct GraphKey {
   const void *src, *dst, *ws;
   uint64_t kv;              // unique id of the KV cache (handles may be recycled)
   const void *dseq, *dpos;
+  const void* dk;           // per-row loop counts (mixed-k decode), else null
   bool operator<(const GraphKey& o) const {
-    return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos) <
+    return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos, dk) <
            std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.prof, o.src, o.dst, o.ws, o.kv,
-                    o.dseq, o.dpos);
+                    o.dseq, o.dpos, o.dk);
   }
 };
 
@@ -281,7 +282,8 @@ struct CallCtx {
   int seq, pos0;         // prefill
   const int32_t *dseq, *dpos;
   int max_pos;
-  int k;
+  int k;                 // loops run (the largest per-row count when dk is set)
+  const int32_t* dk = nullptr;   // decode: per-row loop counts, or null
   cudaStream_t s;
 };
 
@@ -386,7 +388,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   if (c.decode) {
     {
       Launch L(m, c.s, DORY_KK_KVCOMMIT);
-      DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s));
+      DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s,
+                                W.recurrent ? c.dk : nullptr, loop));
     }
     DecodeAttnParams a;
     a.q = c.w.q; a.gate = c.w.gate; a.out = c.w.o; a.kv = view;
@@ -450,6 +453,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   RowUpdateParams r;
   r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = go.k_splits; r.split_stride = go.split_stride;
   r.h = h; r.hb = hb; r.alpha = W.alpha_attn; r.norm_eps = m->cfg.norm_eps;
+  r.row_k = W.recurrent ? c.dk : nullptr; r.loop = loop; r.k_hi = c.k; r.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_ROW);
     DORY_TRY(launch_row_update(r, c.s));
@@ -461,7 +465,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
 // `reinject`: after the update, x <- Norm(x + e); `save_e`: store the update
 // result as e first; `out`: also write the result as bf16 there.
 cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool save_e,
-                         bool reinject, __nv_bfloat16* out) {
+                         bool reinject, __nv_bfloat16* out, int loop = 1) {
   dory_model* m = c.m;
   const BlockW& W = m->blocks[b];
   CUtensorMap tmA;
@@ -510,6 +514,7 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   r.e_save = save_e ? c.w.e32 : nullptr;
   r.e = reinject ? c.w.e32 : nullptr;
   r.out = out;
+  r.row_k = W.recurrent ? c.dk : nullptr; r.loop = loop; r.k_hi = c.k; r.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_ROW);
     DORY_TRY(launch_row_update(r, c.s));
@@ -555,7 +560,8 @@ cudaError_t enqueue_stack(CallCtx& c, const __nv_bfloat16* src, __nv_bfloat16* d
       const bool commit = !last_loop || j == c.k;
       DORY_TRY(attention_sublayer(c, b, j, c.w.h32, c.w.hb, commit));
       const bool reinject = (b == n_in + n_rec - 1) && j < c.k;
-      DORY_TRY(mlp_sublayer(c, b, c.w.h32, c.w.hb, false, reinject, nullptr));
+      // with per-row loop counts the row kernels refine both decisions per row
+      DORY_TRY(mlp_sublayer(c, b, c.w.h32, c.w.hb, false, reinject, nullptr, j));
     }
   }
   for (int b = n_in + n_rec; b < nb; ++b) {
@@ -854,7 +860,8 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv->uid, nullptr, nullptr};
+  GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv->uid, nullptr, nullptr,
+               nullptr};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -863,9 +870,13 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   return DORY_OK;
 }
 
-int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq,
-                     const int32_t* d_pos, int max_pos_hint, const void* h_in, void* h_out, int k,
-                     void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+// One decode step; d_k (device, per row) null means every row runs k loops,
+// else row r runs d_k[r] loops (1..k) and k is the largest of them.
+int decode_step_impl(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq,
+                     const int32_t* d_pos, const int32_t* d_k, int max_pos_hint, const void* h_in,
+                     void* h_out, int k, void* ws, size_t ws_bytes, void* stream) {
   if (!m || !kv || kv->m != m || !d_seq || !d_pos || !h_in || !h_out || !ws || batch <= 0)
     return DORY_ERR_INVALID_ARG;
   if (batch > kMaxDecodeRows) return DORY_ERR_INVALID_ARG;
@@ -880,18 +891,37 @@ int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq
   CallCtx c;
   c.m = m; c.kv = kv; c.w = ws_bind(m, ws, batch); c.n = batch; c.decode = true;
   c.seq = 0; c.pos0 = 0; c.dseq = d_seq; c.dpos = d_pos; c.max_pos = max_pos_hint;
-  c.k = k; c.s = s;
+  c.k = k; c.dk = d_k; c.s = s;
   const size_t bytes = size_t(batch) * m->d * 2;
   const __nv_bfloat16* src = in_dev ? static_cast<const __nv_bfloat16*>(h_in) : c.w.st_in;
   __nv_bfloat16* dst = out_dev ? static_cast<__nv_bfloat16*>(h_out) : c.w.st_out;
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
-  GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv->uid, d_seq, d_pos};
+  GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv->uid, d_seq, d_pos,
+               d_k};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return DORY_ERR_CUDA;
   return DORY_OK;
+}
+
+}  // namespace
+
+int dory_decode_step(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq,
+                     const int32_t* d_pos, int max_pos_hint, const void* h_in, void* h_out, int k,
+                     void* ws, size_t ws_bytes, void* stream) {
+  return decode_step_impl(m, kv, batch, d_seq, d_pos, nullptr, max_pos_hint, h_in, h_out, k, ws,
+                          ws_bytes, stream);
+}
+
+int dory_decode_step_mixed(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq,
+                           const int32_t* d_pos, const int32_t* d_k, int k_hi, int max_pos_hint,
+                           const void* h_in, void* h_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (!d_k || !is_device_ptr(d_k)) return DORY_ERR_INVALID_ARG;
+  return decode_step_impl(m, kv, batch, d_seq, d_pos, d_k, max_pos_hint, h_in, h_out, k_hi, ws,
+                          ws_bytes, stream);
 }
 
 int dory_device_status(dory_model* m, void* stream) {

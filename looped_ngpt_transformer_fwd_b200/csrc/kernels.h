@@ -92,6 +92,14 @@ struct RowUpdateParams {
   float* e_save = nullptr;
   const float* e = nullptr;
   __nv_bfloat16* out = nullptr;  // optional final output [rows, d] bf16
+  // per-row loop counts (one decode step with a different k per sequence):
+  // in recurrent loop `loop`, rows with row_k[r] < loop are left unchanged
+  // and the re-injection applies only while loop < row_k[r].  A count
+  // outside 1..k_hi leaves the row unchanged and sets kStatusBounds.  Null:
+  // every row runs every loop.
+  const int32_t* row_k = nullptr;
+  int loop = 0, k_hi = 0;
+  uint32_t* status = nullptr;
 };
 cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s);
 
@@ -116,10 +124,13 @@ struct KvLayerView {
 // Copy fresh K/V rows [rows, Hkv, hd] into cache slots.  Row r goes to
 // sequence seq (or d_seq[r]) at position pos0 + r (or d_pos[r]); rows below
 // `first_row` are skipped.
+// row_k / loop: as in RowUpdateParams (rows whose loop count is below `loop`
+// write nothing); null commits every row.
 cudaError_t launch_kv_commit(const KvLayerView& kv, const __nv_bfloat16* k_new,
                              const __nv_bfloat16* v_new, int rows, int first_row, int seq,
                              int pos0, const int32_t* d_seq, const int32_t* d_pos,
-                             uint32_t* status, cudaStream_t s);
+                             uint32_t* status, cudaStream_t s, const int32_t* row_k = nullptr,
+                             int loop = 0);
 
 // ----------------------------------------------------------------- attention
 struct PrefillAttnParams {

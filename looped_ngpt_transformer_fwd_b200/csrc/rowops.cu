@@ -36,6 +36,16 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
 __global__ void row_update_kernel(const RowUpdateParams p) {
   __shared__ float red[32];
   const int r = blockIdx.x;
+  // one CTA per row: these exits are uniform across the block
+  if (p.row_k) {
+    const int kr = p.row_k[r];
+    if (kr < 1 || kr > p.k_hi) {
+      if (threadIdx.x == 0 && p.loop == 1) report_status(p.status, kStatusBounds);
+      return;
+    }
+    if (p.loop > kr) return;        // this row's loops are done
+  }
+  const bool reinject = p.e != nullptr && (!p.row_k || p.loop < p.row_k[r]);
   const int nch = p.d >> 2;
   const size_t row_off = static_cast<size_t>(r) * p.d;
   float4 y[kRowMaxChunks], h[kRowMaxChunks];
@@ -76,15 +86,15 @@ __global__ void row_update_kernel(const RowUpdateParams p) {
     if (c < nch) {
       h[j].x *= inv_h; h[j].y *= inv_h; h[j].z *= inv_h; h[j].w *= inv_h;
       if (p.e_save) reinterpret_cast<float4*>(p.e_save + row_off)[c] = h[j];
-      if (p.e) {
+      if (reinject) {
         const float4 e = reinterpret_cast<const float4*>(p.e + row_off)[c];
         h[j].x += e.x; h[j].y += e.y; h[j].z += e.z; h[j].w += e.w;
         ss += dot4(h[j], h[j]);
       }
     }
   }
-  if (p.e) {
-    // block_sum is reached by every thread (p.e is uniform)
+  if (reinject) {
+    // block_sum is reached by every thread (reinject is uniform)
     const float inv_x = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
 #pragma unroll
     for (int j = 0; j < kRowMaxChunks; ++j) {
@@ -123,12 +133,14 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16*
 __global__ void kv_commit_kernel(const KvLayerView kv, const __nv_bfloat16* __restrict__ k_new,
                                  const __nv_bfloat16* __restrict__ v_new, int rows, int first_row,
                                  int seq, int pos0, const int32_t* __restrict__ d_seq,
-                                 const int32_t* __restrict__ d_pos, uint32_t* status) {
+                                 const int32_t* __restrict__ d_pos, uint32_t* status,
+                                 const int32_t* __restrict__ row_k, int loop) {
   const int per_row = kv.n_kv * (kv.hd / 8);
   const size_t id = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   const size_t total = static_cast<size_t>(rows - first_row) * per_row;
   if (id >= total) return;
   const int r = first_row + static_cast<int>(id / per_row);
+  if (row_k && loop > row_k[r]) return;   // this row's loops are done
   const int rem = static_cast<int>(id % per_row);
   const int head = rem / (kv.hd / 8);
   const int c8 = rem % (kv.hd / 8);
@@ -276,11 +288,11 @@ cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, c
 cudaError_t launch_kv_commit(const KvLayerView& kv, const __nv_bfloat16* k_new,
                              const __nv_bfloat16* v_new, int rows, int first_row, int seq,
                              int pos0, const int32_t* d_seq, const int32_t* d_pos,
-                             uint32_t* status, cudaStream_t s) {
+                             uint32_t* status, cudaStream_t s, const int32_t* row_k, int loop) {
   if (first_row >= rows) return cudaSuccess;
   const size_t total = static_cast<size_t>(rows - first_row) * kv.n_kv * (kv.hd / 8);
   kv_commit_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
-      kv, k_new, v_new, rows, first_row, seq, pos0, d_seq, d_pos, status);
+      kv, k_new, v_new, rows, first_row, seq, pos0, d_seq, d_pos, status, row_k, loop);
   return cudaGetLastError();
 }
 

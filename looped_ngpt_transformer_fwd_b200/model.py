@@ -131,6 +131,18 @@ class DoryModel:
                            _ptr(h_in), _ptr(h_out), k, _ptr(ws), ws.numel(), _stream(stream))
         return h_out
 
+    def decode_mixed(self, kv, h_in, d_seq, d_pos, d_k, max_pos, k_hi, h_out=None, stream=None):
+        """One decode step with a loop count per row; d_seq / d_pos / d_k: int32
+        device tensors [batch], k_hi = the largest count."""
+        n = h_in.shape[0]
+        if h_out is None:
+            h_out = torch.empty_like(h_in)
+        ws = self.workspace(n)
+        B.dory_decode_step_mixed(self.handle, kv.handle, n, _ptr(d_seq), _ptr(d_pos), _ptr(d_k),
+                                 k_hi, max_pos, _ptr(h_in), _ptr(h_out), _ptr(ws), ws.numel(),
+                                 _stream(stream))
+        return h_out
+
     def attention_sublayer(self, kv, layer, h, loop=1, seq=0, pos0=0, stream=None):
         """In place on h: [n, d] float32 device tensor."""
         ws = self.workspace(h.shape[0])
