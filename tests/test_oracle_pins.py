@@ -190,18 +190,45 @@ def test_prefix_rows_are_causal():
         np.testing.assert_allclose(full[:33], pre, rtol=0, atol=1e-12)
 
 
-def test_decode_after_prefill_equals_longer_prefill():
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_decode_after_prefill_equals_longer_prefill(k):
     """A decode step is a one-token call: under per-loop caching, prefill(T) then one
-    decode step gives the last row of prefill(T + 1)."""
+    decode step gives the last row of prefill(T + 1), for any loop count."""
     cfg = tiny()
     prov = random_float_weights(cfg, 15)
     h = unit_rows(cfg, 16, 51)
-    ref, _, _ = _run(cfg, prov, h, 2, mode="per_loop", k_max=2)
-    cache = KVCache(cfg, "per_loop", k_max=2)
+    ref, _, _ = _run(cfg, prov, h, k, mode="per_loop", k_max=3)
+    cache = KVCache(cfg, "per_loop", k_max=3)
     orc = Oracle(cfg, prov)
-    orc.forward(h[:50], 0, 2, cache)
-    step = orc.decode(h[50:51], [0], [50], 2, cache)
+    orc.forward(h[:50], 0, k, cache)
+    step = orc.decode(h[50:51], [0], [50], k, cache)
     np.testing.assert_allclose(step[0], ref[50], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_decode_rows_are_independent(mode):
+    """Each row of a decode step attends only to its own sequence's cache: a batched
+    step equals every row decoded alone.  (So a step may give each row its own loop
+    count: the loop count is a per-request dial, [P5] Why it matters here.)"""
+    cfg = tiny()
+    prov = random_float_weights(cfg, 21)
+    lens = [7, 30, 12]
+    hs = [unit_rows(cfg, 30 + s, lens[s] + 1) for s in range(3)]
+    runs = []
+    for _ in range(2):
+        cache = KVCache(cfg, mode, k_max=2)
+        orc = Oracle(cfg, prov)
+        for s in range(3):
+            orc.forward(hs[s][:lens[s]], 0, 2, cache, seq=s)
+        runs.append((orc, cache))
+    rows = np.stack([hs[s][lens[s]] for s in range(3)])
+    orc, cache = runs[0]
+    batched = orc.decode(rows, [0, 1, 2], lens, 2, cache)
+    orc, cache = runs[1]
+    single = np.stack([orc.decode(rows[s:s + 1], [s], [lens[s]], 2, cache)[0] for s in range(3)])
+    np.testing.assert_allclose(batched, single, rtol=0, atol=1e-12)
+    # and the rows really differ (a step that ignored its sequence would not)
+    assert np.abs(batched[0] - batched[1]).max() > 1e-3
 
 
 def test_unwritten_reads_raise():
