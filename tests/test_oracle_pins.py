@@ -54,6 +54,21 @@ def test_depth_and_pattern_match_golden():
         assert orc.sublayer_apps // 2 * 1 == 16 + 20 * k   # blocks = 16 + 20k
 
 
+@pytest.mark.parametrize("k", [6, 8])
+def test_depth_formula_holds_at_extrapolated_loop_counts(k):
+    """[P1] Main Findings: base scores are reported at k = 6 and 8, loop counts never
+    trained on (inference-depth extrapolation).  The stack is the same at any k:
+    32 + 40k sublayer applications ([P1] Key Contributions 1's closed form) and
+    16 + 20k block passes, with the recurrent weights read k times."""
+    g = json.load(open(GOLDEN))
+    cfg = shaped_like_4b()
+    prov = random_float_weights(cfg, 1)
+    _, orc, _ = _run(cfg, prov, unit_rows(cfg, 5, 1), k, k_max=k)
+    apps = g["depth_formula"]["constant"] + g["depth_formula"]["per_loop"] * k
+    assert orc.sublayer_apps == apps == layer_applications(cfg, k)
+    assert orc.sublayer_apps // 2 == 16 + 20 * k
+
+
 def test_recurrent_weights_are_shared_across_loops():
     """[P5] Key ideas / [P4] looping at inference: the same weights serve every k —
     the set of weight blocks read is the 36 physical blocks for every k."""
