@@ -95,3 +95,21 @@ def test_decode_kv_bytes_of_the_4b_workload():
     got = bench.decode_kv_bytes(cfg, 64, 32768, 2)
     assert got == 64 * 4096 * (14 * 32769 + 42 * 4096)
     assert abs(got / 165.4e9 - 1) < 5e-3
+
+
+def test_profiled_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch):
+    import hashlib
+    src = tmp_path / "kernel.cu"
+    src.write_text("// version 1\n")
+    sha = hashlib.sha1(src.read_bytes()).hexdigest()
+    monkeypatch.setattr(bench, "PROFILED", {
+        "k": {"traffic": 123, "source": (str(src), sha)},
+        "r": {"ratio": 1.5, "source": (str(src), sha)},
+    })
+    assert bench.profiled_traffic("k") == 123
+    assert bench.profiled_traffic("r", work=10) == 15.0
+    assert bench.profiled_traffic("r") is None
+    assert bench.profiled_traffic("unknown") is None
+    src.write_text("// version 2\n")
+    assert bench.profiled_traffic("k") is None
+    assert bench.profiled_traffic("r", work=10) is None
