@@ -127,84 +127,6 @@ def test_decode_batch_of_sequences_matches_oracle(tiny):
         assert_parity(to_np(out), ref, what=f"batched decode step {step}")
 
 
-@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
-def test_mixed_k_decode_matches_oracle(tiny, mode):
-    """One decode step with its own loop count per sequence: each row equals that
-    sequence decoded alone with its k (rows in another order than sequences)."""
-    cfg, prov, model = tiny
-    ks = [1, 3, 2, 3]
-    k_hi = max(ks)
-    kv = model.kv_cache(mode, 4, 128, k_max=k_hi)
-    ocache = oracle_cache(cfg, mode, k_max=k_hi)
-    orc = oracle(cfg, prov)
-    lens = [5, 33, 70, 2]
-    xs = [inputs(cfg, 40 + s, lens[s] + 2) for s in range(4)]
-    for s, L in enumerate(lens):
-        model.prefill(kv, xs[s][0][:L], ks[s], seq=s, pos0=0)
-        orc.forward(xs[s][1][:L], 0, ks[s], ocache, seq=s)
-    order = [2, 0, 3, 1]
-    for step in range(2):
-        rows_t = torch.cat([xs[s][0][lens[s] + step:lens[s] + step + 1] for s in order])
-        d_seq = torch.tensor(order, dtype=torch.int32, device="cuda")
-        d_pos = torch.tensor([lens[s] + step for s in order], dtype=torch.int32, device="cuda")
-        d_k = torch.tensor([ks[s] for s in order], dtype=torch.int32, device="cuda")
-        out = to_np(model.decode_mixed(kv, rows_t, d_seq, d_pos, d_k, 127, k_hi))
-        torch.cuda.synchronize()
-        for i, s in enumerate(order):
-            p = lens[s] + step
-            ref = orc.decode(xs[s][1][p:p + 1], [s], [p], ks[s], ocache)
-            assert_parity(out[i:i + 1], ref, what=f"mixed-k decode step {step} seq {s} k={ks[s]} {mode}")
-    assert model.device_status() == 0
-
-
-def test_mixed_k_decode_with_equal_counts_is_the_plain_step(tiny):
-    """Every row with the same count: bit for bit the plain decode step."""
-    cfg, prov, model = tiny
-    k = 2
-    caches = [model.kv_cache("last_loop", 3, 64, k_max=k) for _ in range(2)]
-    lens = [7, 20, 41]
-    xs = [inputs(cfg, 60 + s, lens[s] + 1)[0] for s in range(3)]
-    for kv in caches:
-        for s, L in enumerate(lens):
-            model.prefill(kv, xs[s][:L], k, seq=s, pos0=0)
-    rows = torch.cat([xs[s][lens[s]:lens[s] + 1] for s in range(3)])
-    d_seq = torch.arange(3, dtype=torch.int32, device="cuda")
-    d_pos = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    d_k = torch.full((3,), k, dtype=torch.int32, device="cuda")
-    plain = model.decode(caches[0], rows, d_seq, d_pos, 63, k)
-    mixed = model.decode_mixed(caches[1], rows, d_seq, d_pos, d_k, 63, k)
-    torch.cuda.synchronize()
-    assert torch.equal(plain.view(torch.int16), mixed.view(torch.int16))
-    assert model.device_status() == 0
-
-
-def test_mixed_k_decode_rejects_bad_counts(tiny):
-    """Host-checked k_hi errors, and a device count outside 1..k_hi reported as a
-    bounds error (the row's recurrent loops are skipped, nothing faults)."""
-    from looped_ngpt_transformer_fwd_b200.binding import DoryError
-    cfg, prov, model = tiny
-    kv = model.kv_cache("per_loop", 2, 32, k_max=2)
-    x, _ = inputs(cfg, 70, 4)
-    for s in range(2):
-        model.prefill(kv, x[2 * s:2 * s + 1], 2, seq=s, pos0=0)
-    rows = x[1:3]
-    d_seq = torch.arange(2, dtype=torch.int32, device="cuda")
-    d_pos = torch.ones(2, dtype=torch.int32, device="cuda")
-    with pytest.raises(DoryError) as e:
-        model.decode_mixed(kv, rows, d_seq, d_pos, torch.full((2,), 2, dtype=torch.int32,
-                                                               device="cuda"), 31, 3)
-    assert e.value.status == -4          # k_hi above the per-loop cache's k_max
-    with pytest.raises(DoryError) as e:
-        model.decode_mixed(kv, rows, d_seq, d_pos, torch.full((2,), 1, dtype=torch.int32,
-                                                               device="cuda"), 31, 0)
-    assert e.value.status == -3          # k_hi out of range
-    bad = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
-    model.decode_mixed(kv, rows, d_seq, d_pos, bad, 31, 2)
-    torch.cuda.synchronize()
-    assert model.device_status() == -11
-    assert model.device_status() == 0    # the status word was cleared
-
-
 def test_window_mask_is_exact():
     """W = 4: an off-by-one in the sliding window or causal mask moves a fifth of the
     softmax mass and fails the bar."""
@@ -432,3 +354,82 @@ def test_recycled_cache_handles_do_not_reuse_stale_graphs(tiny):
         kv.free()
         del kv
         gc.collect()
+
+
+# ------------------------------------------------------- loop count per sequence
+@pytest.mark.parametrize("mode", ["last_loop", "per_loop"])
+def test_mixed_k_decode_matches_oracle(tiny, mode):
+    """One decode step with its own loop count per sequence: each row equals that
+    sequence decoded alone with its k (rows in another order than sequences)."""
+    cfg, prov, model = tiny
+    ks = [1, 3, 2, 3]
+    k_hi = max(ks)
+    kv = model.kv_cache(mode, 4, 128, k_max=k_hi)
+    ocache = oracle_cache(cfg, mode, k_max=k_hi)
+    orc = oracle(cfg, prov)
+    lens = [5, 33, 70, 2]
+    xs = [inputs(cfg, 40 + s, lens[s] + 2) for s in range(4)]
+    for s, L in enumerate(lens):
+        model.prefill(kv, xs[s][0][:L], ks[s], seq=s, pos0=0)
+        orc.forward(xs[s][1][:L], 0, ks[s], ocache, seq=s)
+    order = [2, 0, 3, 1]
+    for step in range(2):
+        rows_t = torch.cat([xs[s][0][lens[s] + step:lens[s] + step + 1] for s in order])
+        d_seq = torch.tensor(order, dtype=torch.int32, device="cuda")
+        d_pos = torch.tensor([lens[s] + step for s in order], dtype=torch.int32, device="cuda")
+        d_k = torch.tensor([ks[s] for s in order], dtype=torch.int32, device="cuda")
+        out = to_np(model.decode_mixed(kv, rows_t, d_seq, d_pos, d_k, 127, k_hi))
+        torch.cuda.synchronize()
+        for i, s in enumerate(order):
+            p = lens[s] + step
+            ref = orc.decode(xs[s][1][p:p + 1], [s], [p], ks[s], ocache)
+            assert_parity(out[i:i + 1], ref, what=f"mixed-k decode step {step} seq {s} k={ks[s]} {mode}")
+    assert model.device_status() == 0
+
+
+def test_mixed_k_decode_with_equal_counts_is_the_plain_step(tiny):
+    """Every row with the same count: bit for bit the plain decode step."""
+    cfg, prov, model = tiny
+    k = 2
+    caches = [model.kv_cache("last_loop", 3, 64, k_max=k) for _ in range(2)]
+    lens = [7, 20, 41]
+    xs = [inputs(cfg, 60 + s, lens[s] + 1)[0] for s in range(3)]
+    for kv in caches:
+        for s, L in enumerate(lens):
+            model.prefill(kv, xs[s][:L], k, seq=s, pos0=0)
+    rows = torch.cat([xs[s][lens[s]:lens[s] + 1] for s in range(3)])
+    d_seq = torch.arange(3, dtype=torch.int32, device="cuda")
+    d_pos = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    d_k = torch.full((3,), k, dtype=torch.int32, device="cuda")
+    plain = model.decode(caches[0], rows, d_seq, d_pos, 63, k)
+    mixed = model.decode_mixed(caches[1], rows, d_seq, d_pos, d_k, 63, k)
+    torch.cuda.synchronize()
+    assert torch.equal(plain.view(torch.int16), mixed.view(torch.int16))
+    assert model.device_status() == 0
+
+
+def test_mixed_k_decode_rejects_bad_counts(tiny):
+    """Host-checked k_hi errors, and a device count outside 1..k_hi reported as a
+    bounds error (the row's recurrent loops are skipped, nothing faults)."""
+    from looped_ngpt_transformer_fwd_b200.binding import DoryError
+    cfg, prov, model = tiny
+    kv = model.kv_cache("per_loop", 2, 32, k_max=2)
+    x, _ = inputs(cfg, 70, 4)
+    for s in range(2):
+        model.prefill(kv, x[2 * s:2 * s + 1], 2, seq=s, pos0=0)
+    rows = x[1:3]
+    d_seq = torch.arange(2, dtype=torch.int32, device="cuda")
+    d_pos = torch.ones(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(DoryError) as e:
+        model.decode_mixed(kv, rows, d_seq, d_pos, torch.full((2,), 2, dtype=torch.int32,
+                                                               device="cuda"), 31, 3)
+    assert e.value.status == -4          # k_hi above the per-loop cache's k_max
+    with pytest.raises(DoryError) as e:
+        model.decode_mixed(kv, rows, d_seq, d_pos, torch.full((2,), 1, dtype=torch.int32,
+                                                               device="cuda"), 31, 0)
+    assert e.value.status == -3          # k_hi out of range
+    bad = torch.tensor([2, 0], dtype=torch.int32, device="cuda")
+    model.decode_mixed(kv, rows, d_seq, d_pos, bad, 31, 2)
+    torch.cuda.synchronize()
+    assert model.device_status() == -11
+    assert model.device_status() == 0    # the status word was cleared
