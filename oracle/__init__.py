@@ -7,7 +7,9 @@ binding) never imports it and fails loudly when its extension is missing.
 
 The oracle is a plain, slow, obviously-correct NumPy implementation in float64
 (weights and inputs are the bf16 values of the shared synthetic generators,
-held exactly in float64).  It shares no code with the GPU path.
+held exactly in float64).  It shares no code with the GPU path.  `quant`
+holds the block-scaled weight formats of the quantised checkpoints (MXFP8,
+NVFP4): codecs, block quantisation, dequantisation.
 """
 
 from .ngpt_oracle import (  # noqa: F401

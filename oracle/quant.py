@@ -1,0 +1,152 @@
+"""Block-scaled weight formats of the quantised checkpoints (oracle side).
+
+TEST INFRASTRUCTURE ONLY, like the rest of `oracle/`: only `tests/`,
+`__graft_entry__.smoke()` and the CPU legs of `bench.py` may use it.
+
+"Dory1.0-4B: A Looped Normalized-GPT" (ai.info AI summary), Key Contributions
+item 4: the model is released as BF16, MXFP8 and NVFP4 checkpoints (Main
+Findings: MXFP8 by post-training quantisation, NVFP4 after
+quantisation-aware distillation).  The pages give no bit layout; the plainest
+reading is the public definition of each format:
+
+* MXFP8: blocks of 32 consecutive values along the reduction (K) axis share a
+  power-of-two scale stored as E8M0 (code e means 2^(e - 127)); elements are
+  FP8 E4M3 (exponent bias 7, 3 mantissa bits, subnormals, no infinities,
+  largest finite 448).  The block's scale exponent is floor(log2(amax)) - 8,
+  8 being the largest E4M3 exponent; elements round to nearest (ties to even)
+  and saturate at 448.
+* NVFP4: blocks of 16 share an E4M3 scale and the whole tensor one fp32 scale
+  g = amax / (6 * 448); elements are FP4 E2M1 (exponent bias 1, 1 mantissa
+  bit, largest 6).  Block scale s = E4M3(amax_block / (6 g)); elements
+  E2M1(x / (s g)), nearest even, saturating at 6.
+
+Dequantisation multiplies back; a quantised GEMM is C = A @ W_hat^T with W_hat
+the dequantised weights, in float64.  Rounding here is done at the bit level
+(exponent, then a round-half-even on the grid of that binade); the tests check
+it against an exhaustive nearest-value search and, for E4M3, against
+PyTorch's own float8 conversion.
+"""
+
+import numpy as np
+
+# (exponent bias, mantissa bits, largest finite value) of the element formats
+E4M3 = (7, 3, 448.0)
+E2M1 = (1, 1, 6.0)
+
+
+def round_to_format(x, fmt):
+    """Nearest value of the format (ties to the even grid point), saturating at
+    the largest finite value; keeps the sign (and -0)."""
+    bias, mbits, vmax = fmt
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    emin = 1 - bias                                  # exponent of the smallest normal
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, emin)                          # subnormals share emin's grid
+    ulp = np.exp2(e - mbits)
+    q = np.rint(a / ulp) * ulp                       # np.rint: half to even
+    q = np.minimum(q, vmax)
+    return np.copysign(q, x)
+
+
+def decode(codes, fmt):
+    """Values of element codes (sign bit at 1 << (exponent + mantissa bits));
+    for E4M3 the all-ones magnitude is NaN."""
+    bias, mbits, _ = fmt
+    ebits = 4 if fmt == E4M3 else 2
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where((c >> (ebits + mbits)) & 1, -1.0, 1.0)
+    field = (c >> mbits) & ((1 << ebits) - 1)
+    mant = c & ((1 << mbits) - 1)
+    sub = mant * np.exp2(1 - bias - mbits)
+    nrm = (1.0 + mant / (1 << mbits)) * np.exp2(field - bias)
+    v = sign * np.where(field == 0, sub, nrm)
+    if fmt == E4M3:
+        v = np.where((field == 15) & (mant == 7), np.nan, v)
+    return v
+
+
+def encode(x, fmt):
+    """Codes of values already on the format's grid (see round_to_format)."""
+    bias, mbits, _ = fmt
+    ebits = 4 if fmt == E4M3 else 2
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    neg = np.signbit(x).astype(np.int64)
+    emin = 1 - bias
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    normal = a >= np.exp2(emin)
+    field = np.where(normal, e + bias, 0).astype(np.int64)
+    mant = np.where(normal, (a / np.exp2(e) - 1.0) * (1 << mbits),
+                    a / np.exp2(emin - mbits))
+    mant = np.rint(mant).astype(np.int64)
+    return (neg << (ebits + mbits)) | (field << mbits) | mant
+
+
+def e8m0_value(codes):
+    """E8M0 scale codes -> 2^(e - 127) (code 255 is NaN)."""
+    c = np.asarray(codes, dtype=np.int64)
+    return np.where(c == 255, np.nan, np.exp2(c - 127.0))
+
+
+# ----------------------------------------------------------------- MXFP8
+
+MX_BLOCK = 32
+
+
+def mxfp8_quantize(w):
+    """w [N, K] (K a multiple of 32) -> (element codes [N, K] uint8 E4M3,
+    scale codes [N, K/32] uint8 E8M0)."""
+    w = np.asarray(w, dtype=np.float64)
+    n, k = w.shape
+    assert k % MX_BLOCK == 0
+    blocks = w.reshape(n, k // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    with np.errstate(divide="ignore"):
+        sexp = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127)
+    sexp = np.clip(sexp, -127, 127)
+    q = round_to_format(blocks / np.exp2(sexp)[:, :, None], E4M3)
+    return (encode(q, E4M3).astype(np.uint8).reshape(n, k),
+            (sexp + 127).astype(np.uint8))
+
+
+def mxfp8_dequantize(codes, scales):
+    n, k = codes.shape
+    v = decode(codes, E4M3).reshape(n, k // MX_BLOCK, MX_BLOCK)
+    return (v * e8m0_value(scales)[:, :, None]).reshape(n, k)
+
+
+# ----------------------------------------------------------------- NVFP4
+
+NV_BLOCK = 16
+
+
+def nvfp4_quantize(w):
+    """w [N, K] (K a multiple of 16) -> (element codes [N, K] uint8 holding
+    E2M1 codes in the low nibble, block scale codes [N, K/16] uint8 E4M3,
+    tensor scale g as float32)."""
+    w = np.asarray(w, dtype=np.float64)
+    n, k = w.shape
+    assert k % NV_BLOCK == 0
+    amax = np.abs(w).max()
+    g = np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+    blocks = w.reshape(n, k // NV_BLOCK, NV_BLOCK)
+    bmax = np.abs(blocks).max(axis=2)
+    s = round_to_format(bmax / (6.0 * float(g)), E4M3)
+    denom = (s * float(g))[:, :, None]
+    q = np.where(denom > 0, round_to_format(blocks / np.where(denom > 0, denom, 1.0), E2M1), 0.0)
+    return (encode(q, E2M1).astype(np.uint8).reshape(n, k),
+            encode(s, E4M3).astype(np.uint8), g)
+
+
+def nvfp4_dequantize(codes, scales, g):
+    n, k = codes.shape
+    v = decode(codes, E2M1).reshape(n, k // NV_BLOCK, NV_BLOCK)
+    return (v * decode(scales, E4M3)[:, :, None] * float(g)).reshape(n, k)
+
+
+def quantized_gemm(a, w_hat):
+    """C = A W_hat^T in float64 (W_hat: dequantised [N, K])."""
+    return np.asarray(a, dtype=np.float64) @ np.asarray(w_hat, dtype=np.float64).T

@@ -1,0 +1,187 @@
+"""Pins of the oracle's block-scaled weight formats (oracle/quant.py).
+
+The element and scale codecs are checked against PyTorch's own float8 types
+(a library routine) and against exhaustive nearest-value searches; the block
+formats against invariants that a dropped term, a wrong exponent or a
+transposed block would break.  The formats are those of the released MXFP8 /
+NVFP4 checkpoints ("Dory1.0-4B: A Looped Normalized-GPT", Key Contributions
+item 4), read as the public format definitions.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import quant as Q
+
+
+def _nearest_even(x, fmt):
+    """Exhaustive search: the closest finite value of the format; on a tie the
+    one with the even code; beyond the largest value, the largest value."""
+    ebits = 4 if fmt == Q.E4M3 else 2
+    codes = np.arange(1 << (ebits + fmt[1]))         # the non-negative codes
+    vals = Q.decode(codes, fmt)
+    ok = np.isfinite(vals)
+    codes, vals = codes[ok], vals[ok]
+    out = []
+    for v in np.asarray(x, dtype=np.float64):
+        a = min(abs(v), fmt[2])
+        d = np.abs(vals - a)
+        best = np.flatnonzero(d == d.min())
+        if len(best) > 1:
+            best = [c for c in best if codes[c] % 2 == 0]
+        out.append(np.copysign(vals[best[0]], v))
+    return np.array(out)
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = Q.decode(codes, Q.E4M3)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin])
+    assert np.nanmax(got) == 448.0 and np.nanmin(np.abs(got[got != 0])) == 2.0 ** -9
+
+
+def test_e4m3_rounding_matches_torch_in_range():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.uniform(-460, 460, 4000),
+        rng.standard_normal(2000) * 1e-2,
+        np.exp2(rng.uniform(-12, 8.8, 2000)) * rng.choice([-1, 1], 2000),
+        # exact ties go to the even code: 1 + 1/16 -> 1, 1 + 3/16 -> 1.25; in the
+        # subnormal range (step 2^-9) 2^-10 -> 0 and 3 * 2^-10 -> 2^-8
+        [1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 0.0, -0.0, 448.0, 460.0],
+    ])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = Q.round_to_format(x.astype(np.float32).astype(np.float64), Q.E4M3)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [Q.E4M3, Q.E2M1], ids=["e4m3", "e2m1"])
+def test_rounding_matches_exhaustive_search(fmt):
+    rng = np.random.default_rng(1)
+    vmax = fmt[2]
+    x = np.concatenate([rng.uniform(-1.2 * vmax, 1.2 * vmax, 3000),
+                        np.exp2(rng.uniform(-12, np.log2(vmax) + 0.5, 3000)),
+                        Q.decode(np.arange(1 << (5 if fmt == Q.E2M1 else 8)), fmt)])
+    x = x[np.isfinite(x)]
+    # midpoints between consecutive representable values are exact ties
+    vals = np.unique(np.abs(x[np.isin(x, Q.decode(np.arange(128 if fmt == Q.E4M3 else 8), fmt))]))
+    x = np.concatenate([x, (vals[1:] + vals[:-1]) / 2])
+    assert np.array_equal(Q.round_to_format(x, fmt), _nearest_even(x, fmt))
+
+
+@pytest.mark.parametrize("fmt,n", [(Q.E4M3, 256), (Q.E2M1, 16)], ids=["e4m3", "e2m1"])
+def test_encode_inverts_decode(fmt, n):
+    codes = np.arange(n)
+    vals = Q.decode(codes, fmt)
+    fin = np.isfinite(vals)
+    assert np.array_equal(Q.encode(vals[fin], fmt), codes[fin])
+
+
+def test_e2m1_value_set():
+    # 1 sign, 2 exponent (bias 1), 1 mantissa bit: eight magnitudes, largest 6,
+    # smallest positive 0.5 (subnormal), all exactly representable in E4M3
+    mags = Q.decode(np.arange(8), Q.E2M1)
+    assert len(set(mags)) == 8 and mags.max() == 6.0 and mags[mags > 0].min() == 0.5
+    assert np.array_equal(Q.round_to_format(mags, Q.E4M3), mags)
+    assert np.array_equal(Q.decode(np.arange(8, 16), Q.E2M1), -mags)
+
+
+def test_e8m0_decode_matches_torch():
+    codes = np.arange(255, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    assert np.array_equal(Q.e8m0_value(codes), ref)
+
+
+def _weights(n=12, k=128, seed=3):
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((n, k)) * 0.02
+    w[0, :32] = 0.0                                  # an all-zero block
+    w[1, 32:64] *= 1e-6                              # a tiny block
+    return w
+
+
+def test_mxfp8_block_scale_and_error_bound():
+    w = _weights()
+    codes, scales = Q.mxfp8_quantize(w)
+    assert codes.shape == w.shape and scales.shape == (12, 4)
+    x = Q.e8m0_value(scales)
+    blocks = w.reshape(12, 4, 32)
+    amax = np.abs(blocks).max(axis=2)
+    nz = amax > 0
+    # the block's largest magnitude lands in [256, 512) in scale units
+    assert np.all((amax[nz] / x[nz] >= 256) & (amax[nz] / x[nz] < 512))
+    w_hat = Q.mxfp8_dequantize(codes, scales).reshape(12, 4, 32)
+    scaled = np.abs(blocks) / x[:, :, None]
+    err = np.abs(blocks - w_hat)
+    normal = (scaled >= 2.0 ** -6) & (scaled <= 448)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(blocks[normal]) * (1 + 1e-12))
+    sat = scaled > 448
+    assert np.allclose(err[sat], (scaled[sat] - 448) * np.broadcast_to(x[:, :, None], sat.shape)[sat])
+    assert np.all(w_hat[0, 0] == 0)
+
+
+def test_mxfp8_power_of_two_scaling_only_moves_the_scales():
+    w = _weights(seed=4)
+    c1, s1 = Q.mxfp8_quantize(w)
+    c2, s2 = Q.mxfp8_quantize(w * 2.0 ** 5)
+    assert np.array_equal(c1, c2)
+    nz = np.abs(w.reshape(12, 4, 32)).max(axis=2) > 0
+    assert np.array_equal(s2.astype(int)[nz], s1.astype(int)[nz] + 5)
+
+
+def test_mxfp8_round_trip_of_values_on_the_grid():
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 0x78, size=(4, 64)).astype(np.uint8)   # magnitudes below 256
+    codes[:, ::32] = 0x78 | 0x80 * (rng.integers(0, 2, (4, 2)))   # one of 256 per block
+    codes[:, 1::2] |= 0x80                                         # negative odd columns
+    scales = rng.integers(100, 130, size=(4, 2)).astype(np.uint8)
+    w = Q.mxfp8_dequantize(codes, scales)
+    c2, s2 = Q.mxfp8_quantize(w)
+    assert np.array_equal(s2, scales)
+    assert np.array_equal(Q.decode(c2, Q.E4M3), Q.decode(codes, Q.E4M3))
+
+
+def test_nvfp4_elements_are_nearest_and_scales_consistent():
+    w = _weights(k=64, seed=6)
+    codes, scales, g = Q.nvfp4_quantize(w)
+    assert codes.max() < 16 and scales.shape == (12, 4) and g.dtype == np.float32
+    s = Q.decode(scales, Q.E4M3)
+    assert np.all(np.isfinite(s)) and s.max() <= 448
+    blocks = w.reshape(12, 4, 16)
+    denom = s * float(g)
+    for i in range(12):
+        for j in range(4):
+            if denom[i, j] == 0:
+                assert np.all(codes.reshape(12, 4, 16)[i, j] == 0)
+                continue
+            want = _nearest_even(blocks[i, j] / denom[i, j], Q.E2M1)
+            got = Q.decode(codes.reshape(12, 4, 16)[i, j], Q.E2M1)
+            assert np.array_equal(np.abs(got), np.abs(want))
+    # the block scale is the E4M3 value nearest to amax_block / (6 g)
+    bmax = np.abs(blocks).max(axis=2)
+    assert np.array_equal(s.ravel(), _nearest_even((bmax / (6 * float(g))).ravel(), Q.E4M3))
+
+
+def test_nvfp4_power_of_two_scaling_only_moves_the_tensor_scale():
+    w = _weights(k=64, seed=7)
+    c1, s1, g1 = Q.nvfp4_quantize(w)
+    c2, s2, g2 = Q.nvfp4_quantize(w * 2.0 ** -3)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    assert float(g2) == float(g1) * 2.0 ** -3
+    d1 = Q.nvfp4_dequantize(c1, s1, g1)
+    assert np.array_equal(Q.nvfp4_dequantize(c2, s2, g2), d1 * 2.0 ** -3)
+
+
+def test_quantized_gemm_uses_the_dequantised_weights():
+    rng = np.random.default_rng(8)
+    a = rng.standard_normal((5, 64))
+    codes, scales = Q.mxfp8_quantize(_weights(n=7, k=64, seed=9))
+    w_hat = Q.mxfp8_dequantize(codes, scales)
+    c = Q.quantized_gemm(a, w_hat)
+    brute = np.array([[sum(a[i, t] * w_hat[j, t] for t in range(64)) for j in range(7)]
+                      for i in range(5)])
+    assert np.allclose(c, brute, rtol=1e-12, atol=1e-15)
