@@ -150,3 +150,34 @@ def nvfp4_dequantize(codes, scales, g):
 def quantized_gemm(a, w_hat):
     """C = A W_hat^T in float64 (W_hat: dequantised [N, K])."""
     return np.asarray(a, dtype=np.float64) @ np.asarray(w_hat, dtype=np.float64).T
+
+
+# ------------------------------------------------------ whole-model weights
+
+MATRIX_NAMES = ("wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down")
+
+
+def dequantized_provider(provider, fmt):
+    """Wrap a weight provider (block -> dict) so that every matrix [out, in] is
+    replaced by its quantise -> dequantise version in `fmt` ("mxfp8" or
+    "nvfp4"), blocks running along `in` (the GEMM reduction axis); the vectors
+    (alpha, s_qk) are left as they are."""
+    from synthetic.bf16 import bf16_bits_to_f32
+    memo = {}
+
+    def provide(b):
+        if b not in memo:
+            w = dict(provider(b))
+            for n in MATRIX_NAMES:
+                m = w[n]
+                m = bf16_bits_to_f32(m).astype(np.float64) if m.dtype == np.uint16 else \
+                    np.asarray(m, dtype=np.float64)
+                if fmt == "mxfp8":
+                    w[n] = mxfp8_dequantize(*mxfp8_quantize(m))
+                elif fmt == "nvfp4":
+                    w[n] = nvfp4_dequantize(*nvfp4_quantize(m))
+                else:
+                    raise ValueError(fmt)
+            memo[b] = w
+        return memo[b]
+    return provide

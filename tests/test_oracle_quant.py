@@ -185,3 +185,28 @@ def test_quantized_gemm_uses_the_dequantised_weights():
     brute = np.array([[sum(a[i, t] * w_hat[j, t] for t in range(64)) for j in range(7)]
                       for i in range(5)])
     assert np.allclose(c, brute, rtol=1e-12, atol=1e-15)
+
+
+def test_quantised_stacks_track_the_bf16_stack():
+    """[P1] Main Findings: MXFP8 weights (post-training quantisation) score roughly
+    on par with BF16, NVFP4 needed distillation to close its gap.  The tiny stack
+    (k = 2) with dequantised weights stays close to the bf16 one, MXFP8 (3
+    mantissa bits) closer than NVFP4 (1 bit); a wrong scale exponent or block
+    axis would not."""
+    from oracle import Oracle, KVCache, weights_from_generator
+    from oracle.quant import dequantized_provider
+    from synthetic import load_config, hidden_in
+    from synthetic.bf16 import bf16_bits_to_f32
+    cfg = load_config("tiny")
+    prov = weights_from_generator(cfg, 11)
+    h = bf16_bits_to_f32(hidden_in(cfg, 12, 48)).astype(np.float64)
+    ref = Oracle(cfg, prov).forward(h, 0, 2, KVCache(cfg, "last_loop", k_max=2))
+    err = {}
+    for fmt, min_cos in (("mxfp8", 0.9995), ("nvfp4", 0.995)):
+        out = Oracle(cfg, dequantized_provider(prov, fmt)).forward(
+            h, 0, 2, KVCache(cfg, "last_loop", k_max=2))
+        cos = (out * ref).sum(1) / np.linalg.norm(out, axis=1) / np.linalg.norm(ref, axis=1)
+        assert cos.min() > min_cos, (fmt, cos.min())
+        assert np.allclose(np.linalg.norm(out, axis=1), 1.0, atol=1e-9)
+        err[fmt] = np.abs(out - ref).max()
+    assert 0 < err["mxfp8"] < err["nvfp4"] / 2
