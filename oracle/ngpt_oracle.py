@@ -159,8 +159,9 @@ class KVCache:
 
     Entries hold k-hat (post-RoPE, post-norm, post-s_qk) and v.  Positions a
     sequence had before the oracle saw it may come from `prefill`, a callable
-    (slot_id, seq, lo, hi) -> (K, V) float arrays [hi-lo, n_kv, hd]; any other
-    read of a position never written raises KeyError.
+    (slot_id, seq, lo, hi) -> (K, V) float arrays [hi-lo, n_kv, hd], held in
+    float32 (the filled contents are bf16 values); any other read of a position
+    never written raises KeyError.
 
     Slot ids: block * 16 + loop slot, where the loop slot is (loop - 1) for a
     recurrent block under per-loop caching and 0 otherwise ([P5] Key ideas:

@@ -523,3 +523,158 @@ def test_generator_weights_are_bf16_and_unit_rows():
         m = bf16_bits_to_f32(w[name]).astype(np.float64)
         assert np.abs(np.linalg.norm(m, axis=1) - 1).max() < 1e-2
     assert np.all(w["alpha_attn"] == np.float32(0.05)) and np.all(w["s_qk"] == 1)
+
+
+# ---------------------------------------------------------------- pre-filled caches
+
+def _prefill_values(cfg):
+    """Deterministic K/V contents per (slot, seq, position), independent of how a
+    range is requested (so a range read equals the same positions read one by one).
+    float32 values: the cache holds filled entries in float32, as the GPU caches'
+    bf16 contents are."""
+    hkv, hd = cfg["n_kv_heads"], cfg["head_dim"]
+
+    def pre(slot, seq, lo, hi):
+        ks, vs = [], []
+        for p in range(lo, hi):
+            r = np.random.default_rng([slot, seq, p, 99])
+            ks.append(r.standard_normal((hkv, hd)).astype(np.float32))
+            vs.append(r.standard_normal((hkv, hd)).astype(np.float32))
+        shape = (0, hkv, hd)
+        return (np.stack(ks) if ks else np.zeros(shape)), (np.stack(vs) if vs else np.zeros(shape))
+    return pre
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_prefilled_cache_equals_explicit_writes(mode):
+    """The decode workloads start from caches whose earlier positions come from a
+    fill callback instead of earlier calls.  A cache filled that way must read back
+    exactly like a cache into which the same values were written explicitly: the
+    last W positions of a sliding-window layer, every position of a full layer, in
+    every loop slot, and a position rewritten after the fill returns the new value
+    ([P4] How does looping work at inference time?: each cache keeps a layer's
+    keys/values; SWA layers keep the last W positions)."""
+    cfg = tiny()                      # W = 32, blocks alternate SWA / full
+    W, k = cfg["window"], 2
+    lens = {0: 70, 1: 40}             # seq 0 beyond the window, seq 1 partly
+    pre = _prefill_values(cfg)
+    filled = KVCache(cfg, mode, k_max=k, prefill=pre, prefilled_len=lens)
+    written = KVCache(cfg, mode, k_max=k)
+    for slot in written.slot_ids():
+        b, loop = slot // 16, slot % 16 + 1
+        for seq, n in lens.items():
+            lo = 0 if is_full_layer(cfg, b) else max(0, n - W)
+            K, V = pre(slot, seq, lo, n)
+            written.write(b, loop, seq, lo, K, V)
+    assert is_full_layer(cfg, 1) and not is_full_layer(cfg, 2)
+    loops = (1, 2) if mode == "per_loop" else (1,)
+    for b in (0, 1, 2, 3):            # input SWA, input full, recurrent SWA, recurrent full
+        for loop in (loops if block_role(cfg, b) == "recurrent" else (1,)):
+            for seq, n in lens.items():
+                ranges = ([(0, n), (5, n - 3), (n - 1, n)] if is_full_layer(cfg, b)
+                          else [(max(0, n - W), n), (max(0, n - W) + 4, n - 2)])
+                for lo, hi in ranges:
+                    ka, va = filled.read(b, loop, seq, lo, hi)
+                    kb, vb = written.read(b, loop, seq, lo, hi)
+                    assert np.array_equal(ka, kb) and np.array_equal(va, vb), (b, loop, seq, lo)
+    # a continued call (both modes write and read within the call) and decode steps
+    prov = random_float_weights(cfg, 40)
+    h = unit_rows(cfg, 41, 9)
+    outs = []
+    for cache in (filled, written):
+        orc = Oracle(cfg, prov)
+        o1 = orc.forward(h[:6], lens[0], k, cache, seq=0)
+        o2 = orc.decode(h[6:8], [0, 1], [lens[0] + 6, lens[1]], k, cache)
+        outs.append(np.concatenate([o1, o2]))
+    assert np.array_equal(outs[0], outs[1])
+    # a position inside the filled range rewritten afterwards reads back the new value
+    newk = np.full((1, cfg["n_kv_heads"], cfg["head_dim"]), 0.25)
+    newv = np.full_like(newk, -0.5)
+    for cache in (filled, written):
+        cache.write(2, 1, 1, lens[1] - 3, newk, newv)
+        cache.write(1, 1, 1, 7, newk, newv)
+    for b, lo, hi in ((2, lens[1] - W + 8, lens[1]), (1, 0, lens[1])):
+        ka, va = filled.read(b, 1, 1, lo, hi)
+        kb, vb = written.read(b, 1, 1, lo, hi)
+        assert np.array_equal(ka, kb) and np.array_equal(va, vb)
+    ka, va = filled.read(2, 1, 1, lens[1] - 3, lens[1] - 2)
+    assert np.all(ka == 0.25) and np.all(va == -0.5)
+    # negative control: a fill that ignores the sequence index reads differently
+    wrong = KVCache(cfg, mode, k_max=k, prefill=lambda s, q, lo, hi: pre(s, 0, lo, hi),
+                    prefilled_len=lens)
+    kw, _ = wrong.read(1, 1, 1, 0, lens[1])
+    kb, _ = written.read(1, 1, 1, 0, lens[1])
+    assert not np.array_equal(kw[:7], kb[:7])
+
+
+# ---------------------------------------------------------------- output gate
+
+def _gate_inputs(cfg, w_dir, n, seed):
+    """Rows h = Norm(w_dir + noise) with h . w_dir >= 0.5 for every row."""
+    rng = np.random.default_rng(seed)
+    h = l2norm(w_dir[None, :] + 0.25 * rng.standard_normal((n, cfg["d_model"]))
+               / np.sqrt(cfg["d_model"]))
+    assert (h @ w_dir).min() > 0.5
+    return h
+
+
+def test_gate_equal_across_heads_is_removed_by_the_output_norm():
+    """[P1] Methodology: the sigmoid output gates multiply each head's output, and the
+    concatenated gated output is L2-normalised before the output projection.  When
+    every head of a token gets the same gate value, the gate is a per-token uniform
+    scale that the norm removes: the sublayer equals the one with W_g = 0 (all gates
+    1/2).  A gate read for the wrong token would break this."""
+    cfg = tiny()
+    base = random_float_weights(cfg, 42)
+    w_dir = l2norm(np.random.default_rng(43).standard_normal(cfg["d_model"]))
+    same = modified(base, lambda b, w: w.__setitem__("wg", np.tile(3.0 * w_dir, (cfg["n_q_heads"], 1))))
+    zero = modified(base, lambda b, w: w["wg"].fill(0.0))
+    h = unit_rows(cfg, 44, 40)
+    for layer in (0, 1):
+        a = Oracle(cfg, same).attention_sublayer(layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+        z = Oracle(cfg, zero).attention_sublayer(layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+        np.testing.assert_allclose(a, z, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("head", [0, 1, 2, 3])
+def test_one_hot_gate_selects_that_head(head):
+    """[P1] Methodology: head j's output is scaled by sigmoid(h . W_g[j]).  With
+    W_g[j] = +c u and every other row -c u, on inputs with h . u >= 1/2 and c = 400,
+    head j's gate is 1 and the others are below e^-200: the sublayer keeps head j's
+    attention output alone.  Because the output norm and the nGPT update see only
+    the direction of y = Norm(o) W_o^T, that equals the W_g = 0 sublayer whose W_o
+    keeps only head j's columns.  A gate applied to the wrong head, or sigmoid(-x),
+    fails it."""
+    cfg = tiny()
+    hq, hd = cfg["n_q_heads"], cfg["head_dim"]
+    base = random_float_weights(cfg, 45)
+    u = l2norm(np.random.default_rng(46).standard_normal(cfg["d_model"]))
+
+    def one_hot(b, w):
+        g = np.tile(-400.0 * u, (hq, 1))
+        g[head] = 400.0 * u
+        w["wg"] = g
+
+    def only_head(b, w):
+        w["wg"].fill(0.0)
+        keep = np.zeros(hq * hd)
+        keep[head * hd:(head + 1) * hd] = 1.0
+        w["wo"] = w["wo"] * keep[None, :]
+    h = _gate_inputs(cfg, u, 24, 47)
+    for layer in (0, 1):
+        a = Oracle(cfg, modified(base, one_hot)).attention_sublayer(
+            layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+        b = Oracle(cfg, modified(base, only_head)).attention_sublayer(
+            layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+        # and the choice of head matters
+        other = (head + 1) % hq
+
+        def only_other(bb, w, other=other):
+            w["wg"].fill(0.0)
+            keep = np.zeros(hq * hd)
+            keep[other * hd:(other + 1) * hd] = 1.0
+            w["wo"] = w["wo"] * keep[None, :]
+        c = Oracle(cfg, modified(base, only_other)).attention_sublayer(
+            layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+        assert np.abs(a - c).max() > 1e-4
