@@ -256,6 +256,44 @@ DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
 DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
 
 /* ---------------------------------------------------------------------
+ * Mask and failure-path diagnostics.
+ * --------------------------------------------------------------------- */
+
+/* Mask probe.  The attention of a looped nGPT block is causal, and a
+ * sliding-window layer sees only the last `window` keys up to and including
+ * the query ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
+ * English: interleaved sliding-window and full-attention layers).  While a
+ * probe is set, every attention launch of global block `layer` in later calls
+ * (dory_prefill, dory_decode_step(_mixed), dory_attention_sublayer) first
+ * resets and then fills, per (row, query head), the record
+ *   {first key position given a nonzero softmax weight, last such position,
+ *    number of such keys, sum of their positions mod 2^32}
+ * in d_probe: int32 [max_rows][n_q_heads][4], device, caller-owned, 16-byte
+ * aligned.  Rows are the call's tokens (prefill) or batch rows (decode).  A
+ * recurrent block's record holds its last loop's launch (every loop uses the
+ * same mask).  A call with more rows than max_rows fails with DORY_ERR_CUDA.
+ * Calls captured while a probe is set use separate CUDA graphs with the
+ * recording kernels; d_probe = NULL switches the probe off (layer and
+ * max_rows are then ignored). */
+DORY_API int dory_debug_mask_probe(dory_model* m, int layer, int32_t* d_probe, int max_rows);
+
+/* Attention kernels launched by the most recent call, by kind:
+ * counts[0] tensor-core (tcgen05) prefill attention, counts[1] mma.sync
+ * prefill attention (head_dim 64, or a pos0 / window that is not a multiple
+ * of 128), counts[2] TMA-fed decode attention, counts[3] cp.async decode
+ * attention (head_dim 64, or a window that is not a multiple of 64). */
+DORY_API int dory_debug_attention_paths(const dory_model* m, int32_t counts[4]);
+
+/* Failure-path test aid (no counterpart on the pages).  Every wait inside the
+ * library's kernels gives up after a bounded time and records a timeout in the
+ * model's device status word instead of hanging the GPU.  This launches one
+ * small kernel whose only wait is on a barrier that nothing ever completes,
+ * with a limit of `limit_us` microseconds (1 .. 1000000); no copy or MMA is in
+ * flight.  After it, dory_device_status returns DORY_ERR_DEVICE_TIMEOUT once
+ * (and clears the word). */
+DORY_API int dory_debug_wait_timeout(dory_model* m, uint32_t limit_us, void* stream);
+
+/* ---------------------------------------------------------------------
  * Allocation-free variant (no counterpart in the paper: a deployment aid).
  *
  * Some callers cannot allocate device memory at all: code running where

@@ -32,7 +32,10 @@ EXPORTS = (
     "dory_last_call_stats", "dory_error_string", "dory_kv_free", "dory_destroy",
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
     "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
+    "dory_debug_mask_probe", "dory_debug_attention_paths", "dory_debug_wait_timeout",
 )
+
+ATTENTION_PATHS = ("prefill_tc", "prefill_mma", "decode_tma", "decode_cp")
 
 # size of the library's built-in scratch array (DORY_NOALLOC_SCRATCH_BYTES)
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -100,6 +103,9 @@ def lib():
             "dory_profile_enable": (I, [P, I]),
             "dory_profile_read": (I, [P, I, P, P]),
             "dory_mlp_sublayer_noalloc": (I, [P, I, I, P, P]),
+            "dory_debug_mask_probe": (I, [P, I, P, I]),
+            "dory_debug_attention_paths": (I, [P, P]),
+            "dory_debug_wait_timeout": (I, [P, ctypes.c_uint32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -237,6 +243,22 @@ def dory_profile_read(model, kind):
     check(lib().dory_profile_read(model, kind, ctypes.byref(ms), ctypes.byref(n)),
           "dory_profile_read")
     return ms.value, n.value
+
+
+def dory_debug_mask_probe(model, layer, probe_ptr, max_rows):
+    return check(lib().dory_debug_mask_probe(model, layer, probe_ptr, max_rows),
+                 "dory_debug_mask_probe")
+
+
+def dory_debug_attention_paths(model):
+    """{kind: launches} of the attention kernels of the most recent call."""
+    counts = (ctypes.c_int32 * 4)()
+    check(lib().dory_debug_attention_paths(model, counts), "dory_debug_attention_paths")
+    return dict(zip(ATTENTION_PATHS, list(counts)))
+
+
+def dory_debug_wait_timeout(model, limit_us, stream):
+    return check(lib().dory_debug_wait_timeout(model, limit_us, stream), "dory_debug_wait_timeout")
 
 
 def dory_kv_free(kv):

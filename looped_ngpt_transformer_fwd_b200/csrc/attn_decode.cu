@@ -61,7 +61,8 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>((r * CH + (c ^ (r & 7))) * 16);
 }
 
-template <int HD>
+// kProbe: also record the keys the softmax included (mask probe, diagnostics)
+template <int HD, bool kProbe>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAttnParams p) {
   constexpr int CH = HD / 8;
   constexpr int KSTEPS = HD / 16;
@@ -130,6 +131,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAt
 #pragma unroll
   for (int j = 0; j < ONT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;   // row g only (rows g+8 are padding)
+  ProbeAcc pacc;
+  probe_reset(pacc);
 
   for (int t = 0; t < n_tiles; ++t) {
     const int nxt = t + kDecStages - 1;
@@ -161,6 +164,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAt
         const float v = kp < k_end ? s[j][e] * p.scale_log2 : -INFINITY;
         s[j][e] = v;
         mx = fmaxf(mx, v);
+        if constexpr (kProbe) {
+          if (v != -INFINITY) probe_add(pacc, kp);
+        }
       }
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
@@ -191,6 +197,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeAt
     __syncthreads();
   }
   cp_async_wait<0>();
+  if constexpr (kProbe) {
+    if (g < group)
+      probe_flush(p.probe + (static_cast<size_t>(b) * p.n_q_heads + kvh * group + g) * 4, pacc);
+  }
 
   // merge the 4 warps: shared scratch reuses the pipeline buffers
   __syncthreads();
@@ -253,15 +263,16 @@ __global__ void __launch_bounds__(HD) decode_combine_kernel(const DecodeAttnPara
 template <int HD>
 cudaError_t launch_decode_impl(const DecodeAttnParams& p, cudaStream_t s) {
   const int smem = kDecStages * 2 * kDecTile * HD * 2;
-  auto kern = decode_attn_kernel<HD>;
-  static uint32_t attr_done = 0;
+  auto kern = p.probe ? decode_attn_kernel<HD, true> : decode_attn_kernel<HD, false>;
+  static uint32_t attr_done[2] = {0, 0};   // per instantiation, one bit per device < 32
+  uint32_t& done = attr_done[p.probe ? 1 : 0];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 32 || !(attr_done & (1u << dev))) {
+  if (dev >= 32 || !(done & (1u << dev))) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    if (dev < 32) attr_done |= 1u << dev;
+    if (dev < 32) done |= 1u << dev;
   }
   const int n_splits = decode_attention_splits(p.max_pos, p.window, p.split_keys);
   dim3 grid(n_splits, p.kv.n_kv, p.batch);

@@ -64,6 +64,8 @@ __device__ __forceinline__ uint32_t kv_off(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// kProbe: also record the keys given a nonzero weight (mask probe, diagnostics)
+template <bool kProbe>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_attn_tma_kernel(const __grid_constant__ CUtensorMap tmCache, const DecodeAttnParams p,
                            int split_tiles, float m_log2) {
@@ -137,12 +139,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       if (!ok) {
-        for (int s = 0; s < kStages; ++s) {
-          if (!(issued & (1u << s))) continue;
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[s], (parity_bits >> s) & 1u))
-            if (globaltimer_ns() - t0 > 200000000ull) break;
-        }
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s)) drain_wait(&full[s], (parity_bits >> s) & 1u);
       }
     }
   } else {
@@ -162,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int key0 = warp * 16;
     int stage = 0;
     uint32_t phase = 0;
+    ProbeAcc pacc;
+    probe_reset(pacc);
     for (int j = 0; j < n_tiles; ++j) {
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, abort_flag, p.status)))
         break;
@@ -202,6 +202,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           const bool ok = kp >= lo && kp <= pos;
           pv[n][e] = ok ? ex2(fmaf(s[n][e], p.scale_log2, -m_log2)) : 0.f;
           l += pv[n][e];
+          if constexpr (kProbe) {
+            if (pv[n][e] > 0.f) probe_add(pacc, kp);
+          }
         }
       }
       const uint32_t pb0 = pack_bf16x2(pv[0][0], pv[0][1]);
@@ -222,6 +225,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         stage = 0;
         phase ^= 1u;
       }
+    }
+    if constexpr (kProbe) {
+      if (g < group)
+        probe_flush(p.probe + (static_cast<size_t>(b) * p.n_q_heads + kvh * group + g) * 4, pacc);
     }
   }
 
@@ -288,15 +295,21 @@ cudaError_t launch_decode_attention_tma(const DecodeAttnParams& p, float m_log2,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 32 || !(attr_done & (1u << dev))) {
-    e = cudaFuncSetAttribute(decode_attn_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
+    e = cudaFuncSetAttribute(decode_attn_tma_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_attn_tma_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev < 32) attr_done |= 1u << dev;
   }
   int split_tiles = 0;
   const int n_splits = decode_attention_tma_splits(p.max_pos, p.window, &split_tiles);
   dim3 grid(n_splits, p.kv.n_kv, p.batch);
-  decode_attn_tma_kernel<<<grid, kThreads, kSmemBytes, s>>>(tc, p, split_tiles, m_log2);
+  if (p.probe)
+    decode_attn_tma_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tc, p, split_tiles, m_log2);
+  else
+    decode_attn_tma_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tc, p, split_tiles, m_log2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_combine(p, n_splits, s);

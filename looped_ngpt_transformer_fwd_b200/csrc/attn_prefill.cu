@@ -68,7 +68,8 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>((r * CH + (c ^ (r & 7))) * 16);
 }
 
-template <int HD>
+// kProbe: also record the keys the softmax included (mask probe, diagnostics)
+template <int HD, bool kProbe>
 __global__ void __launch_bounds__(kAttnThreads, 2) prefill_attn_kernel(const PrefillAttnParams p) {
   constexpr int CH = HD / 8;               // 16-byte chunks per row
   constexpr int KSTEPS = HD / 16;          // mma k-steps over the head dimension
@@ -137,6 +138,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) prefill_attn_kernel(const Pre
   const int g = lane >> 2, t4 = lane & 3;
   const int qrow0 = warp * 16 + g;                 // this thread's rows: qrow0, qrow0 + 8
   const int qpos[2] = {q_lo + qrow0, q_lo + qrow0 + 8};
+  ProbeAcc pacc[2];
+  probe_reset(pacc[0]);
+  probe_reset(pacc[1]);
 
   for (int kt = kt_begin; kt <= kt_end; ++kt) {
     const int buf = (kt - kt_begin) & 1;
@@ -192,6 +196,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) prefill_attn_kernel(const Pre
         }
         s[j][e] = v;
         mx[e >> 1] = fmaxf(mx[e >> 1], v);
+        if constexpr (kProbe) {
+          if (v != -INFINITY) probe_add(pacc[e >> 1], kt * kAttnBN + j * 8 + t4 * 2 + (e & 1));
+        }
       }
     }
     float corr[2];
@@ -251,6 +258,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) prefill_attn_kernel(const Pre
     const int r = qrow0 + h * 8;
     if (r >= rows) continue;
     const int t = m0 + r;
+    if constexpr (kProbe)
+      probe_flush(p.probe + (static_cast<size_t>(t) * p.n_q_heads + head) * 4, pacc[h]);
     const float scale = p.gate[static_cast<size_t>(t) * p.n_q_heads + head] / l_run[h];
     __nv_bfloat16* dst = p.out + (static_cast<size_t>(t) * p.n_q_heads + head) * HD;
 #pragma unroll
@@ -264,15 +273,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2) prefill_attn_kernel(const Pre
 template <int HD>
 cudaError_t launch_prefill_impl(const PrefillAttnParams& p, cudaStream_t s) {
   const int smem = (kAttnBM + 4 * kAttnBN) * HD * 2;
-  auto kern = prefill_attn_kernel<HD>;
-  static uint32_t attr_done = 0;
+  auto kern = p.probe ? prefill_attn_kernel<HD, true> : prefill_attn_kernel<HD, false>;
+  static uint32_t attr_done[2] = {0, 0};   // per instantiation, one bit per device < 32
+  uint32_t& done = attr_done[p.probe ? 1 : 0];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 32 || !(attr_done & (1u << dev))) {
+  if (dev >= 32 || !(done & (1u << dev))) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    if (dev < 32) attr_done |= 1u << dev;
+    if (dev < 32) done |= 1u << dev;
   }
   dim3 grid((p.n + kAttnBM - 1) / kAttnBM, p.n_q_heads);
   kern<<<grid, kAttnThreads, smem, s>>>(p);

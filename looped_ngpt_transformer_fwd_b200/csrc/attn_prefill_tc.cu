@@ -133,12 +133,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) return;
-  }
-}
 
 // Work item k of this CTA: query tiles sorted longest first (the causal or
 // windowed key range grows with the query tile), dealt out one pass at a time in
@@ -165,6 +159,8 @@ __device__ __forceinline__ bool get_item(const PrefillAttnTcParams& p, int k, It
   return true;
 }
 
+// kProbe: also record the keys given a nonzero weight (mask probe, diagnostics)
+template <bool kProbe>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmKnew,
@@ -442,6 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int window = p.window;
     float* lsum = reinterpret_cast<float*>(smem + kOffL);
     int g = 0;                                     // key tiles of earlier items
+    ProbeAcc pacc;                                 // mask probe of the current item
+    probe_reset(pacc);
 
     // S -> P for key tile i of item `it`, adding to the row sum l; false when
     // a wait gave up (warp-uniform: TMEM loads and stores are warp-collective)
@@ -473,6 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         l += (e[0] + e[1]) + (e[2] + e[3]);
+        if constexpr (kProbe) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (e[u] > 0.f) probe_add(pacc, kp0 + c + u);
+        }
         packed[c / 2] = pack_bf16x2(e[0], e[1]);
         packed[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
       }
@@ -539,6 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       for (int i = 1; ok && i < it.n_tiles; ++i) ok = softmax_tile(it, i, l);
+      if constexpr (kProbe) {
+        if (r < it.rows)
+          probe_flush(p.probe + (static_cast<size_t>(it.m0 + r) * p.n_q_heads + it.head) * 4, pacc);
+        probe_reset(pacc);
+      }
       g += it.n_tiles;
       prev = it;
       l_prev = l;
@@ -607,8 +615,11 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 32 || !(attr_done & (1u << dev))) {
-    e = cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev < 32) attr_done |= 1u << dev;
   }
@@ -619,7 +630,10 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
   dim3 grid(items < dev_sms ? items : dev_sms);
   PrefillAttnTcParams pq = p;
   pq.q = q;
-  prefill_attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, pq);
+  if (p.probe)
+    prefill_attn_tc_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, pq);
+  else
+    prefill_attn_tc_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, pq);
   return cudaGetLastError();
 }
 

@@ -74,23 +74,71 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) when `abort_flag` becomes nonzero or after kWaitLimitNs; in the
-// latter case it sets `*abort_flag` and reports kStatusTimeout.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint32_t* status) {
+// false) when `abort_flag` becomes nonzero or after `limit_ns`; in the latter
+// case it sets `*abort_flag` and reports kStatusTimeout.
+__device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort_flag, uint32_t* status,
+                                                     uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         if (abort_flag) *abort_flag = 1;
         report_status(status, kStatusTimeout);
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, uint32_t* status) {
+  return mbar_wait_bounded_ns(bar, parity, abort_flag, status, kWaitLimitNs);
+}
+
+// Cleanup wait after an abort: lets a bulk copy or a tcgen05 commit that this
+// thread issued complete before the CTA exits (shared memory and TMEM must
+// outlive them).  Such an operation depends on no other CTA or thread, so the
+// wait ends by itself; the limit only guards against a broken device.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// mask probe (diagnostics): per (row, query head) the first and the last key
+// position an attention kernel gave a nonzero weight, how many keys it
+// included and the sum of their positions (mod 2^32).  Each thread collects
+// its share in registers and merges it into the record with atomics; the
+// record starts as {INT_MAX, -1, 0, 0}.
+// ---------------------------------------------------------------------------
+struct ProbeAcc {
+  int first, last, count;
+  uint32_t sum;
+};
+__device__ __forceinline__ void probe_reset(ProbeAcc& a) {
+  a.first = 0x7FFFFFFF;
+  a.last = -1;
+  a.count = 0;
+  a.sum = 0u;
+}
+__device__ __forceinline__ void probe_add(ProbeAcc& a, int kp) {
+  a.first = min(a.first, kp);
+  a.last = max(a.last, kp);
+  a.count += 1;
+  a.sum += static_cast<uint32_t>(kp);
+}
+__device__ __forceinline__ void probe_flush(int32_t* rec, const ProbeAcc& a) {
+  if (a.count == 0) return;
+  atomicMin(rec, a.first);
+  atomicMax(rec + 1, a.last);
+  atomicAdd(rec + 2, a.count);
+  atomicAdd(reinterpret_cast<unsigned int*>(rec + 3), a.sum);
 }
 
 // ---------------------------------------------------------------------------

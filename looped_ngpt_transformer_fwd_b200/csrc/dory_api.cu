@@ -72,12 +72,18 @@ struct GraphKey {
   uint64_t kv;              // unique id of the KV cache (handles may be recycled)
   const void *dseq, *dpos;
   const void* dk;           // per-row loop counts (mixed-k decode), else null
+  const void* probe;        // mask-probe records (diagnostics), else null
+  int probe_layer;
   bool operator<(const GraphKey& o) const {
-    return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos, dk) <
+    return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos, dk, probe,
+                    probe_layer) <
            std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.prof, o.src, o.dst, o.ws, o.kv,
-                    o.dseq, o.dpos, o.dk);
+                    o.dseq, o.dpos, o.dk, o.probe, o.probe_layer);
   }
 };
+
+// attention kernels launched by one call, by kind (see dory_debug_attention_paths)
+enum { kPathPrefillTc = 0, kPathPrefillMma = 1, kPathDecodeTma = 2, kPathDecodeCp = 3, kPaths = 4 };
 
 // events around one kernel launch of an instrumented graph
 struct Mark {
@@ -88,6 +94,7 @@ struct Mark {
 struct GraphEntry {
   cudaGraphExec_t exec = nullptr;
   int launches = 0, sublayers = 0;
+  int paths[kPaths] = {0, 0, 0, 0};
   uint64_t last_use = 0;
   std::vector<Mark> marks;
 };
@@ -118,8 +125,13 @@ struct dory_model {
   std::map<GraphKey, GraphEntry> graphs;
   uint64_t tick = 0;
   int last_launches = 0, last_sublayers = 0;
+  int last_paths[kPaths] = {0, 0, 0, 0};
   // counters of the call being enqueued
   int cur_launches = 0, cur_sublayers = 0;
+  int cur_paths[kPaths] = {0, 0, 0, 0};
+  // mask probe (diagnostics): records of attention launches of block probe_layer
+  int32_t* probe = nullptr;
+  int probe_layer = -1, probe_rows = 0;
   // per-kernel timing
   bool profile = false;
   std::vector<Mark>* cur_marks = nullptr;      // marks of the graph being captured
@@ -385,6 +397,12 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   const KvLayerView view = kv_view(c.kv, b, loop);
   const int window = W.full ? 0 : m->cfg.window;
   const float scale_log2 = m->cfg.softmax_scale * 1.4426950408889634f;
+  int32_t* probe = (m->probe && b == m->probe_layer) ? m->probe : nullptr;
+  if (probe) {
+    if (c.n > m->probe_rows) return cudaErrorInvalidValue;
+    Launch L(m, c.s, DORY_KK_ATTN);
+    DORY_TRY(launch_probe_init(probe, size_t(c.n) * m->hq, c.s));
+  }
   if (c.decode) {
     {
       Launch L(m, c.s, DORY_KK_KVCOMMIT);
@@ -402,13 +420,17 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     a.scale_log2 = scale_log2;
     a.part_acc = c.w.dacc; a.part_ml = c.w.dml;
     a.status = m->status;
+    a.probe = probe;
     {
       Launch L(m, c.s, DORY_KK_ATTN);
       ++m->cur_launches;   // split-KV kernel + combine kernel
-      if (decode_attention_tma_supported(m->hd, window, m->hq / m->hkv) && 2.f * W.m_log2 < 120.f)
+      if (decode_attention_tma_supported(m->hd, window, m->hq / m->hkv) && 2.f * W.m_log2 < 120.f) {
+        ++m->cur_paths[kPathDecodeTma];
         DORY_TRY(launch_decode_attention_tma(a, W.m_log2, c.s));
-      else
+      } else {
+        ++m->cur_paths[kPathDecodeCp];
         DORY_TRY(launch_decode_attention(a, c.s));
+      }
     }
   } else {
     if (prefill_attention_tc_supported(m->hd, c.pos0, window, W.m_log2)) {
@@ -417,6 +439,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
       a.n_q_heads = m->hq; a.n_kv = m->hkv; a.cap = view.cap; a.window = window;
       a.last_pos = c.pos0 + c.n - 1; a.scale_log2 = scale_log2; a.m_log2 = W.m_log2;
       a.status = m->status;
+      a.probe = probe;
+      ++m->cur_paths[kPathPrefillTc];
       Launch L(m, c.s, DORY_KK_ATTN);
       DORY_TRY(launch_prefill_attention_tc(a, c.w.q, c.w.kf, c.w.vf, view, c.s));
     } else {
@@ -424,6 +448,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
       a.q = c.w.q; a.k_new = c.w.kf; a.v_new = c.w.vf; a.gate = c.w.gate; a.out = c.w.o;
       a.kv = view; a.seq = c.seq; a.pos0 = c.pos0; a.n = c.n; a.n_q_heads = m->hq;
       a.window = window; a.scale_log2 = scale_log2; a.status = m->status;
+      a.probe = probe;
+      ++m->cur_paths[kPathPrefillMma];
       Launch L(m, c.s, DORY_KK_ATTN);
       DORY_TRY(launch_prefill_attention(a, c.s));
     }
@@ -586,6 +612,7 @@ int run_graph(dory_model* m, const GraphKey& key, CallCtx& c, const __nv_bfloat1
     }
     m->cur_launches = 0;
     m->cur_sublayers = 0;
+    for (int i = 0; i < kPaths; ++i) m->cur_paths[i] = 0;
     GraphEntry ent;
     m->cur_marks = key.prof ? &ent.marks : nullptr;
     c.s = m->cap_stream;
@@ -609,12 +636,14 @@ int run_graph(dory_model* m, const GraphKey& key, CallCtx& c, const __nv_bfloat1
     }
     ent.launches = m->cur_launches;
     ent.sublayers = m->cur_sublayers;
+    for (int i = 0; i < kPaths; ++i) ent.paths[i] = m->cur_paths[i];
     it = m->graphs.emplace(key, ent).first;
   }
   it->second.last_use = ++m->tick;
   if (cudaGraphLaunch(it->second.exec, stream) != cudaSuccess) return DORY_ERR_CUDA;
   m->last_launches = it->second.launches;
   m->last_sublayers = it->second.sublayers;
+  for (int i = 0; i < kPaths; ++i) m->last_paths[i] = it->second.paths[i];
   if (key.prof) m->last_marks = &it->second.marks;
   return DORY_OK;
 }
@@ -861,7 +890,7 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
   GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv->uid, nullptr, nullptr,
-               nullptr};
+               nullptr, m->probe, m->probe ? m->probe_layer : -1};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -898,7 +927,7 @@ int decode_step_impl(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
   GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv->uid, d_seq, d_pos,
-               d_k};
+               d_k, m->probe, m->probe ? m->probe_layer : -1};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -1010,10 +1039,12 @@ int dory_attention_sublayer(dory_model* m, dory_kv* kv, int layer, int loop, int
   c.seq = seq; c.pos0 = pos0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = pos0 + n_rows - 1;
   c.k = 1; c.s = static_cast<cudaStream_t>(stream);
   m->cur_launches = m->cur_sublayers = 0;
+  for (int i = 0; i < kPaths; ++i) m->cur_paths[i] = 0;
   if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
   if (enqueue_rope_tables(c) != cudaSuccess) return DORY_ERR_CUDA;
   if (attention_sublayer(c, layer, kv->loops[layer] > 1 ? loop : 1, h, c.w.hb, true) != cudaSuccess)
     return DORY_ERR_CUDA;
+  for (int i = 0; i < kPaths; ++i) m->last_paths[i] = m->cur_paths[i];
   return DORY_OK;
 }
 
@@ -1029,6 +1060,36 @@ int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h, void* ws, 
   m->cur_launches = m->cur_sublayers = 0;
   if (launch_f32_to_bf16(h, c.w.hb, size_t(n_rows) * m->d, c.s) != cudaSuccess) return DORY_ERR_CUDA;
   if (mlp_sublayer(c, layer, h, c.w.hb, false, false, nullptr) != cudaSuccess) return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_debug_mask_probe(dory_model* m, int layer, int32_t* d_probe, int max_rows) {
+  if (!m) return DORY_ERR_INVALID_ARG;
+  if (!d_probe) {
+    m->probe = nullptr;
+    m->probe_layer = -1;
+    m->probe_rows = 0;
+    return DORY_OK;
+  }
+  if (layer < 0 || layer >= m->nb || max_rows <= 0) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(d_probe, 16)) return DORY_ERR_MISALIGNED;
+  m->probe = d_probe;
+  m->probe_layer = layer;
+  m->probe_rows = max_rows;
+  return DORY_OK;
+}
+
+int dory_debug_attention_paths(const dory_model* m, int32_t* counts) {
+  if (!m || !counts) return DORY_ERR_INVALID_ARG;
+  for (int i = 0; i < kPaths; ++i) counts[i] = m->last_paths[i];
+  return DORY_OK;
+}
+
+int dory_debug_wait_timeout(dory_model* m, uint32_t limit_us, void* stream) {
+  if (!m || limit_us == 0 || limit_us > 1000000u) return DORY_ERR_INVALID_ARG;
+  if (launch_wait_timeout(m->status, uint64_t(limit_us) * 1000ull, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return DORY_ERR_CUDA;
   return DORY_OK;
 }
 

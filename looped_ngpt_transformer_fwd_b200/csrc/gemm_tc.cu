@@ -299,13 +299,6 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
                        pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
 }
 
-// A wait used only while cleaning up after an abort: short, ignores the flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) return;   // 0.2 s
-  }
-}
 
 template <int BN, int HD, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)

@@ -145,6 +145,7 @@ struct PrefillAttnParams {
   int window = 0;                       // 0 = full attention
   float scale_log2 = 0.f;               // softmax_scale * log2(e)
   uint32_t* status = nullptr;
+  int32_t* probe = nullptr;             // mask probe records [n, Hq, 4], or null
 };
 cudaError_t launch_prefill_attention(const PrefillAttnParams& p, cudaStream_t s);
 
@@ -161,6 +162,7 @@ struct PrefillAttnTcParams {
   int last_pos = 0;                     // pos0 + n - 1
   float scale_log2 = 0.f, m_log2 = 0.f;
   uint32_t* status = nullptr;
+  int32_t* probe = nullptr;             // mask probe records [n, Hq, 4], or null
 };
 bool prefill_attention_tc_supported(int head_dim, int pos0, int window, float m_log2);
 cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv_bfloat16* q,
@@ -181,6 +183,7 @@ struct DecodeAttnParams {
   float* part_acc = nullptr;            // [B, Hq, n_splits, hd]
   float* part_ml = nullptr;             // [B, Hq, n_splits, 2]
   uint32_t* status = nullptr;
+  int32_t* probe = nullptr;             // mask probe records [B, Hq, 4], or null
 };
 int decode_attention_splits(int max_pos, int window, int split_keys);
 cudaError_t launch_decode_attention(const DecodeAttnParams& p, cudaStream_t s);
@@ -190,5 +193,12 @@ cudaError_t launch_decode_combine(const DecodeAttnParams& p, int n_splits, cudaS
 bool decode_attention_tma_supported(int head_dim, int window, int group);
 int decode_attention_tma_splits(int max_pos, int window, int* split_tiles);
 cudaError_t launch_decode_attention_tma(const DecodeAttnParams& p, float m_log2, cudaStream_t s);
+
+// ----------------------------------------------------------------- diagnostics
+// Set `n_records` mask-probe records to {INT_MAX, -1, 0, 0}.
+cudaError_t launch_probe_init(int32_t* probe, size_t n_records, cudaStream_t s);
+// One kernel whose single thread waits on an mbarrier that nothing arrives at,
+// giving up after `limit_ns` with kStatusTimeout in *status.
+cudaError_t launch_wait_timeout(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 }  // namespace dory

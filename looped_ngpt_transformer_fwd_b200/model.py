@@ -161,6 +161,26 @@ class DoryModel:
         B.dory_mlp_sublayer_noalloc(self.handle, layer, h.shape[0], _ptr(h), _stream(stream))
         return h
 
+    def mask_probe(self, layer, max_rows):
+        """Start recording the attention mask of global block `layer`; returns the
+        int32 device tensor [max_rows, n_q_heads, 4] the kernels fill (see
+        dory_debug_mask_probe).  mask_probe_off() stops it."""
+        rec = torch.empty(max_rows, self.cfg["n_q_heads"], 4, dtype=torch.int32,
+                          device=self.device)
+        B.dory_debug_mask_probe(self.handle, layer, _ptr(rec), max_rows)
+        self._probe = rec
+        return rec
+
+    def mask_probe_off(self):
+        B.dory_debug_mask_probe(self.handle, 0, None, 0)
+        self._probe = None
+
+    def attention_paths(self):
+        return B.dory_debug_attention_paths(self.handle)
+
+    def wait_timeout(self, limit_us, stream=None):
+        B.dory_debug_wait_timeout(self.handle, limit_us, _stream(stream))
+
     def device_status(self, stream=None):
         return B.dory_device_status(self.handle, _stream(stream))
 

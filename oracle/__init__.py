@@ -14,5 +14,5 @@ NVFP4): codecs, block quantisation, dequantisation.
 
 from .ngpt_oracle import (  # noqa: F401
     Oracle, KVCache, l2norm, rope, is_full_layer, block_role, kv_cache_bytes,
-    layer_applications, weights_from_generator,
+    layer_applications, weights_from_generator, mask_allows,
 )

@@ -75,6 +75,20 @@ def rope(x, positions, base):
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
+def mask_allows(q_pos, k_pos, window=None):
+    """Whether the key at position k_pos is visible to the query at q_pos: causal
+    (k_pos <= q_pos) and, in a sliding-window layer, among the last `window`
+    positions up to and including the query's own ([P1] Methodology in Plain
+    English: sliding-window and full-attention layers; the window holds
+    exactly W keys).  Works elementwise on arrays; window None = full layer."""
+    q_pos = np.asarray(q_pos)
+    k_pos = np.asarray(k_pos)
+    ok = k_pos <= q_pos
+    if window is not None:
+        ok = ok & (q_pos - k_pos < window)
+    return ok
+
+
 def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-x))
 
@@ -316,9 +330,7 @@ class Oracle:
             i1 = min(n, i0 + self.q_block)
             qp = positions[i0:i1]
             s = cfg["softmax_scale"] * np.einsum("ihd,jhd->hij", q[i0:i1], Kq)
-            allowed = kpos[None, :] <= qp[:, None]
-            if win is not None:
-                allowed &= (qp[:, None] - kpos[None, :]) < win
+            allowed = mask_allows(qp[:, None], kpos[None, :], win)
             s = np.where(allowed[None, :, :], s, -np.inf)
             s = s - s.max(axis=-1, keepdims=True)
             p = np.exp(s)

@@ -14,13 +14,13 @@ TOL_ABS = 3e-2
 TOL_COS = 0.999
 
 
-def build(cfg_name="tiny", seed=0, variant="random", **over):
+def build(cfg_name="tiny", seed=0, variant="random", allow_extrapolated_k=False, **over):
     from looped_ngpt_transformer_fwd_b200 import build as libbuild
     from looped_ngpt_transformer_fwd_b200.model import DoryModel
     libbuild.build()
     cfg = load_config(cfg_name, **over)
     prov = weights_from_generator(cfg, seed, variant)
-    model = DoryModel(cfg, prov)
+    model = DoryModel(cfg, prov, allow_extrapolated_k=allow_extrapolated_k)
     return cfg, prov, model
 
 

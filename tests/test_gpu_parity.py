@@ -62,15 +62,15 @@ def test_attention_sublayer_matches_oracle(tiny, layer):
 
 # ------------------------------------------------------------------ whole stack
 @pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
-@pytest.mark.parametrize("k", [1, 2, 3])
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
 def test_prefill_matches_oracle(tiny, mode, k):
     cfg, prov, model = tiny
     x, h = inputs(cfg, 13, 128)
-    kv = model.kv_cache(mode, 1, 256, k_max=3)
+    kv = model.kv_cache(mode, 1, 256, k_max=4)
     out = model.prefill(kv, x, k)
     torch.cuda.synchronize()
     assert model.device_status() == 0
-    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=3))
+    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=4))
     assert_parity(to_np(out), ref, what=f"prefill {mode} k={k}")
     launches, sub = model.last_call_stats()
     assert sub == 2 * (cfg["n_in_blocks"] + k * cfg["n_rec_blocks"] + cfg["n_out_blocks"])
@@ -78,13 +78,14 @@ def test_prefill_matches_oracle(tiny, mode, k):
 
 
 @pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
-def test_chunked_prefill_then_decode_matches_oracle(tiny, mode):
-    """Chunks that straddle the 32-slot SWA ring several times, then decode steps."""
+@pytest.mark.parametrize("k", [2, 4])
+def test_chunked_prefill_then_decode_matches_oracle(tiny, mode, k):
+    """Chunks that straddle the 32-slot SWA ring several times, then decode steps
+    (per-loop caching at k = 4 reads and writes all four loop slots)."""
     cfg, prov, model = tiny
-    k = 2
     x, h = inputs(cfg, 14, 110)
-    kv = model.kv_cache(mode, 3, 160, k_max=2)
-    ocache = oracle_cache(cfg, mode, k_max=2)
+    kv = model.kv_cache(mode, 3, 160, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
     orc = oracle(cfg, prov)
     seq = 2
     for a, b in ((0, 45), (45, 46), (46, 100)):
@@ -260,26 +261,28 @@ def hd128():
 
 
 @pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
-def test_hd128_prefill_matches_oracle(hd128, mode):
+@pytest.mark.parametrize("k", [2, 4])
+def test_hd128_prefill_matches_oracle(hd128, mode, k):
     cfg, prov, model = hd128
     x, h = inputs(cfg, 51, 300)
-    kv = model.kv_cache(mode, 1, 400, k_max=2)
-    out = model.prefill(kv, x, 2)
+    kv = model.kv_cache(mode, 1, 400, k_max=k)
+    out = model.prefill(kv, x, k)
     torch.cuda.synchronize()
     assert model.device_status() == 0
-    ref = oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, mode, k_max=2))
-    assert_parity(to_np(out), ref, what=f"hd128 prefill {mode}")
+    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=k))
+    assert_parity(to_np(out), ref, what=f"hd128 prefill {mode} k={k}")
+    assert model.attention_paths()["prefill_tc"] > 0
 
 
 @pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
-def test_hd128_chunked_prefill_and_decode(hd128, mode):
+@pytest.mark.parametrize("k", [2, 4])
+def test_hd128_chunked_prefill_and_decode(hd128, mode, k):
     """Chunks at multiples of 128 (tensor-core attention reading cached tiles and
     ring slots), unaligned chunks (mma.sync kernel), then decode steps."""
     cfg, prov, model = hd128
-    k = 2
     x, h = inputs(cfg, 52, 420)
-    kv = model.kv_cache(mode, 2, 480, k_max=2)
-    ocache = oracle_cache(cfg, mode, k_max=2)
+    kv = model.kv_cache(mode, 2, 480, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
     orc = oracle(cfg, prov)
     seq = 1
     for a, b in ((0, 128), (128, 256), (256, 384), (384, 405), (405, 416)):
@@ -362,7 +365,7 @@ def test_mixed_k_decode_matches_oracle(tiny, mode):
     """One decode step with its own loop count per sequence: each row equals that
     sequence decoded alone with its k (rows in another order than sequences)."""
     cfg, prov, model = tiny
-    ks = [1, 3, 2, 3]
+    ks = [1, 4, 2, 3]
     k_hi = max(ks)
     kv = model.kv_cache(mode, 4, 128, k_max=k_hi)
     ocache = oracle_cache(cfg, mode, k_max=k_hi)
@@ -433,3 +436,149 @@ def test_mixed_k_decode_rejects_bad_counts(tiny):
     torch.cuda.synchronize()
     assert model.device_status() == -11
     assert model.device_status() == 0    # the status word was cleared
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_hd128_chunks_twice_the_window(hd128, mode):
+    """Chunks of 2W (W = 128) at chunk-aligned starts, as the long-context prefill
+    runs 8192-token chunks over a 4096-slot ring: every chunk overwrites the whole
+    ring and reads the previous chunk's last W keys from it."""
+    cfg, prov, model = hd128
+    k = 4
+    x, h = inputs(cfg, 54, 1024 + 2)
+    kv = model.kv_cache(mode, 1, 1100, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
+    orc = oracle(cfg, prov)
+    for a in range(0, 1024, 256):
+        out = model.prefill(kv, x[a:a + 256], k, pos0=a)
+        torch.cuda.synchronize()
+        paths = model.attention_paths()
+        assert paths["prefill_mma"] == 0
+        assert paths["prefill_tc"] == cfg["n_in_blocks"] + k * cfg["n_rec_blocks"] + cfg["n_out_blocks"]
+        ref = orc.forward(h[a:a + 256], a, k, ocache)
+        assert_parity(to_np(out), ref, what=f"2W chunk at {a} {mode}")
+    for p in (1024, 1025):
+        d = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pp = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d, pp, 1099, k)
+        ref = orc.decode(h[p:p + 1], [0], [p], k, ocache)
+        assert_parity(to_np(out), ref, what=f"decode {p} after 2W chunks {mode}")
+    assert model.device_status() == 0
+
+
+# ------------------------------------------------------- GQA group of 3 (the 4B grouping)
+# 6 query heads over 2 KV heads of 128: three query heads per KV head, as in the
+# 24/8 4B shape, at sizes the oracle runs in seconds (many query tiles, so the
+# late, full-window tiles of the tensor-core kernel are compared too).
+G3 = dict(d_model=768, n_q_heads=6, n_kv_heads=2, head_dim=128, d_ff=1024, window=128,
+          softmax_scale=float(np.sqrt(128.0)))
+
+
+@pytest.fixture(scope="module")
+def g3():
+    return build("tiny", seed=9, variant="random", **G3)
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+@pytest.mark.parametrize("k", [1, 4])
+def test_gqa3_prefill_matches_oracle(g3, mode, k):
+    cfg, prov, model = g3
+    x, h = inputs(cfg, 55, 640)
+    kv = model.kv_cache(mode, 1, 700, k_max=k)
+    out = model.prefill(kv, x, k)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    assert model.attention_paths()["prefill_tc"] > 0
+    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=k))
+    assert_parity(to_np(out), ref, what=f"GQA-3 prefill {mode} k={k}")
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_gqa3_chunks_and_decode_batch(g3, mode):
+    cfg, prov, model = g3
+    k = 2
+    kv = model.kv_cache(mode, 3, 700, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
+    orc = oracle(cfg, prov)
+    lens = [384, 300, 513]
+    xs = [inputs(cfg, 56 + s, lens[s] + 2) for s in range(3)]
+    for s, L in enumerate(lens):
+        cut = 256 if L > 256 else L
+        for a, b in ((0, cut), (cut, L)):
+            if b > a:
+                out = model.prefill(kv, xs[s][0][a:b], k, seq=s, pos0=a)
+                ref = orc.forward(xs[s][1][a:b], a, k, ocache, seq=s)
+                assert_parity(to_np(out), ref, what=f"GQA-3 seq {s} chunk {a}:{b} {mode}")
+    for step in range(2):
+        rows_t = torch.cat([xs[s][0][lens[s] + step:lens[s] + step + 1] for s in range(3)])
+        rows_h = np.concatenate([xs[s][1][lens[s] + step:lens[s] + step + 1] for s in range(3)])
+        d_seq = torch.arange(3, dtype=torch.int32, device="cuda")
+        d_pos = torch.tensor([L + step for L in lens], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, rows_t, d_seq, d_pos, 699, k)
+        torch.cuda.synchronize()
+        assert model.attention_paths()["decode_tma"] > 0
+        ref = orc.decode(rows_h, [0, 1, 2], [L + step for L in lens], k, ocache)
+        assert_parity(to_np(out), ref, what=f"GQA-3 decode step {step} {mode}")
+    assert model.device_status() == 0
+
+
+# ------------------------------------------------------- extrapolated loop counts
+@pytest.fixture(scope="module")
+def tiny_extrap():
+    return build("tiny", seed=10, variant="random", allow_extrapolated_k=True)
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+@pytest.mark.parametrize("k", [6, 8])
+def test_extrapolated_k_prefill_and_decode(tiny_extrap, mode, k):
+    """Loop counts beyond the trained 1..4 ("Dory1.0-4B: A Looped Normalized-GPT",
+    Main Findings: base scores at k = 6 and 8), accepted with allow_extrapolated_k:
+    the same stack with more passes of the shared block."""
+    cfg, prov, model = tiny_extrap
+    x, h = inputs(cfg, 57, 82)
+    kv = model.kv_cache(mode, 1, 96, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
+    orc = oracle(cfg, prov)
+    out = model.prefill(kv, x[:80], k)
+    torch.cuda.synchronize()
+    assert_parity(to_np(out), orc.forward(h[:80], 0, k, ocache), what=f"k={k} prefill {mode}")
+    _, sub = model.last_call_stats()
+    assert sub == 2 * (cfg["n_in_blocks"] + k * cfg["n_rec_blocks"] + cfg["n_out_blocks"])
+    for p in (80, 81):
+        d = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pp = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d, pp, 95, k)
+        ref = orc.decode(h[p:p + 1], [0], [p], k, ocache)
+        assert_parity(to_np(out), ref, what=f"k={k} decode {p} {mode}")
+    assert model.device_status() == 0
+
+
+def test_extrapolated_k_needs_the_flag(tiny):
+    from looped_ngpt_transformer_fwd_b200.binding import DoryError
+    cfg, prov, model = tiny
+    x, _ = inputs(cfg, 58, 8)
+    kv = model.kv_cache("last_loop", 1, 16, k_max=1)
+    with pytest.raises(DoryError) as e:
+        model.prefill(kv, x, 6)
+    assert e.value.status == -3
+
+
+# ------------------------------------------------------- failure path: bounded waits
+def test_bounded_wait_timeout_is_reported_and_the_model_stays_usable(tiny):
+    """A kernel's wait that runs out records a timeout in the device status word
+    instead of hanging the GPU.  The test kernel waits on a barrier nothing
+    completes, with a 5 ms limit; the status reads DORY_ERR_DEVICE_TIMEOUT once,
+    and the next prefill still matches the oracle."""
+    cfg, prov, model = tiny
+    assert model.device_status() == 0
+    model.wait_timeout(5000)
+    torch.cuda.synchronize()
+    assert model.device_status() == -9
+    assert model.device_status() == 0
+    x, h = inputs(cfg, 59, 64)
+    kv = model.kv_cache("last_loop", 1, 64, k_max=2)
+    out = model.prefill(kv, x, 2)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, "last_loop", k_max=2))
+    assert_parity(to_np(out), ref, what="prefill after a timeout")

@@ -678,3 +678,18 @@ def test_one_hot_gate_selects_that_head(head):
         c = Oracle(cfg, modified(base, only_other)).attention_sublayer(
             layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
         assert np.abs(a - c).max() > 1e-4
+
+
+def test_mask_rule_closed_forms():
+    """[P1] Methodology: causal attention, sliding-window layers see the last W
+    positions including the query's own.  Visible keys of query q: [max(0, q-W+1), q]
+    (W keys once q >= W - 1) for a window, [0, q] for a full layer."""
+    from oracle import mask_allows
+    for W in (1, 2, 4, 7):
+        for q in range(12):
+            vis = [j for j in range(20) if mask_allows(q, j, W)]
+            assert vis == list(range(max(0, q - W + 1), q + 1))
+            assert len(vis) == min(q + 1, W)
+    assert [j for j in range(20) if mask_allows(9, j)] == list(range(10))
+    grid = mask_allows(np.arange(6)[:, None], np.arange(6)[None, :], 2)
+    assert np.array_equal(grid, np.tril(np.ones((6, 6), bool)) & ~np.tril(np.ones((6, 6), bool), -2))
