@@ -51,14 +51,12 @@ WORKLOADS = {
 PROFILED = {
     "gateup": {"traffic": 138491136 + 54726144,
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
-                          "f027590254f0c4cca999fbfb1fcf970c600ec6a3"),
-               "profile": "profiles/gemm_tc_4b_prefill_full.md"},
+                          "f027590254f0c4cca999fbfb1fcf970c600ec6a3")},
     # decode attention: measured (read + write) / algorithmic bytes, applied to
     # the step's total KV bytes
     "attn": {"ratio": (1075908000 + 8675840) / 1073758208,
              "source": ("looped_ngpt_transformer_fwd_b200/csrc/attn_decode_tma.cu",
-                        "364d8cd720bac77c12c3080afcf6ee162dea4681"),
-             "profile": "profiles/attn_decode_tma_b8_ctx32768_full.md"},
+                        "364d8cd720bac77c12c3080afcf6ee162dea4681")},
 }
 
 
@@ -218,19 +216,35 @@ def fill_decode_cache(model, kv, cfg, seed, ctx, mode, k_max, batch):
     torch.cuda.synchronize()
 
 
-def run_ours(args, wl, rank, world, device_index):
+def weight_provider(cfg, seed):
+    """Seeded synthetic 4B-class weights (block -> dict), each block drawn once."""
+    from synthetic import block_weights
+    memo = {}
+
+    def provide(b):
+        if b not in memo:
+            memo[b] = block_weights(cfg, seed, b)
+        return memo[b]
+    return provide
+
+
+def run_ours(args, wl, rank, world, device_index, model=None, prov=None, steps=None,
+             warmup=None):
+    """Time one workload; `model` / `prov` reuse an existing model (same weights)."""
     import torch
     from looped_ngpt_transformer_fwd_b200 import build as libbuild
     from looped_ngpt_transformer_fwd_b200.model import DoryModel
-    from oracle import weights_from_generator
     from synthetic import load_config, hidden_in
 
+    steps = steps or args.steps
+    warmup = warmup or args.warmup
     libbuild.build()
     torch.cuda.set_device(device_index)
     cfg = load_config("dory4b", **block_override(args))
     seed = wl["seed"] + 1000 * rank
-    prov = weights_from_generator(cfg, wl["seed"], cache_blocks=True)
-    model = DoryModel(cfg, prov, device=f"cuda:{device_index}")
+    if model is None:
+        prov = weight_provider(cfg, wl["seed"])
+        model = DoryModel(cfg, prov, device=f"cuda:{device_index}")
     k, mode = wl["k"], wl["mode"]
     stream = torch.cuda.current_stream()
     res = {}
@@ -297,7 +311,7 @@ def run_ours(args, wl, rank, world, device_index):
         extra = {"tokens_per_step": T, "chunk": C, "k": k, "kv_mode": mode}
 
     # warm-up (captures graphs)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     status = model.device_status()
@@ -312,12 +326,12 @@ def run_ours(args, wl, rank, world, device_index):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(device_index) as clk:
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
     ms = reduce_max(ms, world)
     clocks = clk.summary()
 
@@ -329,11 +343,11 @@ def run_ours(args, wl, rank, world, device_index):
         torch.cuda.synchronize()
         barrier(world)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world)
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / steps, world)
         e2e = {"value": units_per_step * world / e2e_ms * 1e3,
                "unit": "tokens/s", "h2d_bytes_per_step": e2e_bytes[0],
                "d2h_bytes_per_step": e2e_bytes[1]}
@@ -354,7 +368,7 @@ def run_ours(args, wl, rank, world, device_index):
                 tot[kk][0] += t
                 tot[kk][1] += n
     else:
-        reps = max(1, min(args.steps, 5))
+        reps = max(1, min(steps, 5))
         for _ in range(reps):
             step()
             torch.cuda.synchronize()
@@ -472,6 +486,49 @@ def oracle_sample(wl, prov=None, n_blocks=4):
                                 f"0-{n_blocks - 1}, time scaled x{apps}/{n_blocks} to the k={k} stack")
 
 
+# ----------------------------------------------------------------- roofline
+DATASHEET = {"tensor": 2250.0, "hbm": 8000.0}    # dense bf16 TFLOP/s, HBM3e GB/s (context only)
+
+
+def roofline(res, wl, peaks, peak_src):
+    """Roofline of the dominant kernel: algorithmic work of its launches in one
+    step over their summed device time (events around every launch)."""
+    dom_name, dom_work, bound, dom_ms, dom_n = res["dom"]
+    if bound == "tensor":
+        achieved = dom_work / (dom_ms / 1e3) / 1e12 if dom_ms > 0 else None
+        if wl["kind"] != "prefill_chunked" and dom_ms > 0:
+            achieved = dom_work / (dom_ms / dom_n / 1e3) / 1e12   # dom_work is per launch
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        unit, key = "TFLOP/s", "bf16_tflops_sustained"
+        per_launch = dom_work if wl["kind"] != "prefill_chunked" else dom_work / max(dom_n, 1)
+        traffic = profiled_traffic(dom_name)
+    else:
+        achieved = dom_work / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
+        peak = peaks["hbm_gbs"]
+        unit, key = "GB/s", "hbm_gbs"
+        per_launch = dom_work / max(dom_n, 1)
+        traffic = profiled_traffic(dom_name, per_launch)
+    return {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": (achieved / peak) if achieved else None,
+            "peak_source": f"{peak_src} ({key})",
+            "frac_of_datasheet": (achieved / DATASHEET[bound]) if achieved else None,
+            "traffic": traffic, "work_per_launch": per_launch, "launches_per_step": dom_n,
+            "device_ms_per_step": dom_ms}
+
+
+def footprint_check(cfg, wl):
+    """The last-loop cache of the workload's shape is the same size for every k
+    and equals the one-loop (per-loop, k_max = 1) size."""
+    from looped_ngpt_transformer_fwd_b200 import binding as B
+    c = B.make_config(cfg)
+    B_, ctx = wl["batch"], wl["ctx"] + 64
+    one = B.dory_kv_bytes(c, "per_loop", B_, ctx, 1)
+    return all(B.dory_kv_bytes(c, "last_loop", B_, ctx, k) == one for k in (1, 2, 3, 4))
+
+
+DEFAULT_EXTRAS = ["prefill_k1", "decode_k2", "decode_k4_last", "decode_k4_per"]
+
+
 # ----------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -485,6 +542,10 @@ def main():
                     help="profiling aid: IN,REC,OUT block counts (same kernel shapes, smaller model)")
     ap.add_argument("--batch", type=int, default=None,
                     help="profiling aid: decode batch override (same per-sequence work)")
+    ap.add_argument("--extra-workloads", default="auto",
+                    help="comma-separated workloads reported under 'workloads' in the same line; "
+                         "'auto' = the k = 1 prefill and the three decode workloads when the "
+                         "headline workload runs on one GPU; 'none' = off")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -526,21 +587,41 @@ def main():
 
     res = run_ours(args, wl, rank, world, local)
     peaks, peak_src = load_peaks()
-    dom_name, dom_work, bound, dom_ms, dom_n = res["dom"]
-    if bound == "tensor":
-        achieved = dom_work / (dom_ms / dom_n / 1e3) / 1e12 if dom_ms > 0 else None
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        unit = "TFLOP/s"
-        if wl["kind"] == "prefill_chunked":
-            achieved = dom_work / (dom_ms / 1e3) / 1e12   # all chunks' attention FLOPs / time
-    else:
-        achieved = dom_work / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
+    roof = roofline(res, wl, peaks, peak_src)
     cpu = None
     if rank == 0 and not args.no_cpu_baseline and not args.blocks and not args.batch:
         v, u, sample = oracle_sample(wl, res["prov"])
         cpu = {"value": v, "unit": u, "cores": blas_threads(), "kind": "oracle", "sample": sample}
+
+    # the other workloads of the metric (k = 1 prefill, decode at k = 2 and 4 in both
+    # cache modes) on the same model, fewer steps each, at N = 1
+    extras = {}
+    names = [] if args.extra_workloads in ("", "none") else (
+        DEFAULT_EXTRAS if args.extra_workloads == "auto" else args.extra_workloads.split(","))
+    if args.extra_workloads == "auto" and (world > 1 or args.workload != "prefill_k2"
+                                           or args.blocks or args.batch):
+        names = []
+    for name in names:
+        xwl = dict(WORKLOADS[name])
+        xsteps = min(args.steps, 10)
+        r = run_ours(args, xwl, rank, world, local, model=res["model"], prov=res["prov"],
+                     steps=xsteps, warmup=args.warmup)
+        entry = {"tokens_per_s": r["units"] * world / r["ms"] * 1e3, "ms_per_step": r["ms"],
+                 "steps": xsteps, "warmup": args.warmup, "workload": r["workload"],
+                 "e2e_tokens_per_s": r["e2e"]["value"] if r["e2e"] else None,
+                 "roofline": roofline(r, xwl, peaks, peak_src),
+                 "kernel_ms_per_step": {kk: round(v[0], 4) for kk, v in r["kernel_ms"].items()},
+                 "gpu_launches": r["launches"] * xsteps, "clocks": r["clocks"],
+                 "weights_seed": WORKLOADS[args.workload]["seed"]}
+        entry.update({kk: vv for kk, vv in r["extra"].items() if kk not in ("k", "kv_mode")})
+        entry["k"], entry["kv_mode"] = xwl["k"], xwl["mode"]
+        if xwl["kind"] == "decode":
+            entry["last_loop_footprint_equals_k1"] = footprint_check(r["cfg"], xwl)
+        extras[name] = entry
+        del r
+        import torch
+        torch.cuda.empty_cache()
+
     if rank == 0:
         value = res["units"] * world / res["ms"] * 1e3   # res["ms"] is already the max over ranks
         line = {
@@ -553,20 +634,17 @@ def main():
                             "parallelism": f"replicas x{world}",
                             "l2": "per-step working set (7.9 GB of weights) exceeds the 126 MB L2"},
                            **res["extra"]),
-            "roofline": {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
-                         "unit": unit, "frac": (achieved / peak) if achieved else None,
-                         "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
-                         "traffic": (profiled_traffic(dom_name, dom_work) if bound == "hbm"
-                                     else profiled_traffic(dom_name)),
-                         "work_per_step": dom_work, "launches_per_step": dom_n,
-                         "device_ms_per_step": dom_ms},
+            "roofline": roof,
             "kernel_ms_per_step": {kk: round(v[0], 4) for kk, v in res["kernel_ms"].items()},
+            "kernel_ms_source": "CUDA events around every kernel of one instrumented replay of the step",
             "cpu_baseline": cpu,
             "e2e": res["e2e"],
             "gpu_launches": res["launches"] * args.steps,
             "clocks": res["clocks"],
             "sublayer_updates_per_call": res["sublayers"],
         }
+        if extras:
+            line["workloads"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
