@@ -114,6 +114,7 @@ void destroy_entry(GraphEntry& g) {
 struct dory_model {
   dory_config cfg;
   int d, hq, hkv, hd, ff, d_attn, n_qkvg, nb;
+  int ld_qkvg;   // row pitch (floats) of the decode QKVG partial products: n_qkvg rounded up to 32
   int device = 0, num_sms = 148;
   uint8_t* wbuf = nullptr;
   size_t wbytes = 0;
@@ -231,7 +232,7 @@ WsLayout ws_layout(const dory_model* m, int T) {
   L.rope_swa = take(size_t(T) * (m->hd / 2) * 8);
   L.rope_full = take(size_t(T) * (m->hd / 2) * 8);
   // K-split partial products of the decode QKVG and gate/up projections
-  L.part = take(size_t(dec_rows) * kMaxKSplits * std::max<size_t>(m->n_qkvg, 2 * ff) * 4);
+  L.part = take(size_t(dec_rows) * kMaxKSplits * std::max<size_t>(m->ld_qkvg, 2 * ff) * 4);
   L.total = o;
   return L;
 }
@@ -365,14 +366,16 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
     g.epi = kEpiStoreF32;
     g.k_splits = pick_k_splits(m, c.n, m->n_qkvg, 128, m->d);
-    g.out_f32 = c.w.part; g.ld_out = m->n_qkvg; g.split_stride = size_t(c.n) * m->n_qkvg;
+    // rows of the partial products start on 128-byte boundaries whatever the
+    // number of gate columns (vector and bulk stores need 16-byte alignment)
+    g.out_f32 = c.w.part; g.ld_out = m->ld_qkvg; g.split_stride = size_t(c.n) * m->ld_qkvg;
     g.status = m->status;
     {
       Launch L(m, c.s, DORY_KK_QKVG);
       DORY_TRY(launch_gemm(tmA, W.tm_qkvg[0], g, 128, m->hd, m->num_sms, c.s));
     }
     QkvgPostParams pp;
-    pp.part = c.w.part; pp.splits = g.k_splits; pp.split_stride = g.split_stride;
+    pp.part = c.w.part; pp.splits = g.k_splits; pp.split_stride = g.split_stride; pp.ld = m->ld_qkvg;
     pp.rows = c.n; pp.n_q_heads = m->hq; pp.n_kv_heads = m->hkv; pp.hd = m->hd;
     pp.s_qk = W.s_qk; pp.rope = rope; pp.norm_eps = m->cfg.norm_eps;
     pp.q_out = c.w.q; pp.k_out = c.w.kf; pp.v_out = c.w.vf; pp.gate_out = c.w.gate;
@@ -717,6 +720,7 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
   m->d = cfg->d_model; m->hq = cfg->n_q_heads; m->hkv = cfg->n_kv_heads; m->hd = cfg->head_dim;
   m->ff = cfg->d_ff; m->d_attn = m->hq * m->hd;
   m->n_qkvg = m->d_attn + 2 * m->hkv * m->hd + m->hq;
+  m->ld_qkvg = (m->n_qkvg + 31) / 32 * 32;
   m->nb = n_blocks(cfg);
   m->device = dev;
   m->num_sms = prop.multiProcessorCount;

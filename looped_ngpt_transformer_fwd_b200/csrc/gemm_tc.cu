@@ -84,12 +84,14 @@ __device__ __forceinline__ void bulk_wait_all() {
 
 // --------------------------------------------------------------- epilogues
 __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32], int valid) {
-  if (valid >= 32) {
+  // vector stores only where the row start allows them (any row pitch works)
+  if (valid >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
     float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
     for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   } else {
-    for (int i = 0; i < valid; ++i) dst[i] = v[i];
+    const int n = valid < 32 ? valid : 32;
+    for (int i = 0; i < n; ++i) dst[i] = v[i];
   }
 }
 

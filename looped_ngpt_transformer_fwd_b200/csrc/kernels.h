@@ -63,6 +63,7 @@ struct QkvgPostParams {
   const float* part = nullptr;
   int splits = 1;
   size_t split_stride = 0;   // elements
+  int ld = 0;                // row pitch of `part` (elements, >= the QKVG column count)
   int rows = 0, n_q_heads = 0, n_kv_heads = 0, hd = 0;
   const float* s_qk = nullptr;
   const float2* rope = nullptr;

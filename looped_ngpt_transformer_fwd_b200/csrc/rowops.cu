@@ -179,8 +179,7 @@ __global__ void qkvg_post_kernel(const QkvgPostParams p) {
   __shared__ float red[32];
   const int r = blockIdx.x, g = blockIdx.y, i = threadIdx.x;
   const int hd = p.hd, half = hd / 2;
-  const int n_qkvg = (p.n_q_heads + 2 * p.n_kv_heads) * hd + p.n_q_heads;
-  const float* row = p.part + static_cast<size_t>(r) * n_qkvg;
+  const float* row = p.part + static_cast<size_t>(r) * p.ld;
   const int n_heads = p.n_q_heads + 2 * p.n_kv_heads;
   if (g == n_heads) {
     // gate logits
