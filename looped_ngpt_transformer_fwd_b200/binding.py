@@ -33,6 +33,7 @@ EXPORTS = (
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
     "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
     "dory_debug_mask_probe", "dory_debug_attention_paths", "dory_debug_wait_timeout",
+    "dory_debug_fused_update",
 )
 
 ATTENTION_PATHS = ("prefill_tc", "prefill_mma", "decode_tma", "decode_cp")
@@ -106,6 +107,7 @@ def lib():
             "dory_debug_mask_probe": (I, [P, I, P, I]),
             "dory_debug_attention_paths": (I, [P, P]),
             "dory_debug_wait_timeout": (I, [P, ctypes.c_uint32, P]),
+            "dory_debug_fused_update": (I, [P, I]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -259,6 +261,12 @@ def dory_debug_attention_paths(model):
 
 def dory_debug_wait_timeout(model, limit_us, stream):
     return check(lib().dory_debug_wait_timeout(model, limit_us, stream), "dory_debug_wait_timeout")
+
+
+def dory_debug_fused_update(model, enable):
+    """Fused projection + nGPT update on (default) or off; returns the status
+    (DORY_ERR_BAD_CONFIG when the model's d_model has no fused kernel)."""
+    return lib().dory_debug_fused_update(model, 1 if enable else 0)
 
 
 def dory_kv_free(kv):

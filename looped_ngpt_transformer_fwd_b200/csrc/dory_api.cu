@@ -64,6 +64,8 @@ struct BlockW {
   float m_log2 = 0.f;   // static softmax maximum: softmax_scale * log2(e) * max s_qk^2
   // B-operand tensor maps, box rows 128 and 256
   CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
+  // W_o / W_down for the fused projection + nGPT update (box rows = one MMA's N)
+  CUtensorMap tm_o_n, tm_d_n;
 };
 
 struct GraphKey {
@@ -74,11 +76,12 @@ struct GraphKey {
   const void* dk;           // per-row loop counts (mixed-k decode), else null
   const void* probe;        // mask-probe records (diagnostics), else null
   int probe_layer;
+  int fused;                // nGPT update fused into the prefill projections
   bool operator<(const GraphKey& o) const {
     return std::tie(phase, k, n, seq, pos0, max_pos, prof, src, dst, ws, kv, dseq, dpos, dk, probe,
-                    probe_layer) <
+                    probe_layer, fused) <
            std::tie(o.phase, o.k, o.n, o.seq, o.pos0, o.max_pos, o.prof, o.src, o.dst, o.ws, o.kv,
-                    o.dseq, o.dpos, o.dk, o.probe, o.probe_layer);
+                    o.dseq, o.dpos, o.dk, o.probe, o.probe_layer, o.fused);
   }
 };
 
@@ -115,6 +118,10 @@ struct dory_model {
   dory_config cfg;
   int d, hq, hkv, hd, ff, d_attn, n_qkvg, nb;
   int ld_qkvg;   // row pitch (floats) of the decode QKVG partial products: n_qkvg rounded up to 32
+  // fused projection + nGPT update (prefill): columns per CTA (0 = not
+  // available for this d_model), CTAs per cluster, and whether it is used
+  int ngpt_bnc = 0, ngpt_cluster = 0;
+  bool fused_update = true;
   int device = 0, num_sms = 148;
   uint8_t* wbuf = nullptr;
   size_t wbytes = 0;
@@ -352,6 +359,13 @@ int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
   return (kb + per - 1) / per;
 }
 
+// Prefill projections with the nGPT update in their epilogue (a cluster of
+// CTAs covers each row); decode keeps K-split GEMMs and the row kernel, which
+// spread its few rows' weight stream over all SMs.
+bool use_fused(const CallCtx& c) {
+  return !c.decode && !c.dk && c.m->fused_update && c.m->ngpt_bnc > 0;
+}
+
 cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloat16* hb,
                                bool commit_after) {
   dory_model* m = c.m;
@@ -467,6 +481,18 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   // output projection, then the nGPT update of the stream
   CUtensorMap tmO;
   if (!make_tmap_bf16(&tmO, c.w.o, c.n, m->d_attn, 128)) return cudaErrorInvalidValue;
+  if (use_fused(c)) {
+    NgptGemmParams f;
+    f.M = c.n; f.N = m->d; f.K = m->d_attn; f.cluster = m->ngpt_cluster;
+    f.h = h; f.hb = hb; f.alpha = W.alpha_attn; f.norm_eps = m->cfg.norm_eps;
+    f.status = m->status;
+    {
+      Launch L(m, c.s, DORY_KK_OPROJ);
+      DORY_TRY(launch_gemm_ngpt(tmO, W.tm_o_n, f, c.s));
+    }
+    ++c.m->cur_sublayers;
+    return cudaSuccess;
+  }
   const int bn_o = c.decode ? 128 : 256;
   GemmParams go;
   go.M = c.n; go.N = m->d; go.K = m->d_attn;
@@ -525,6 +551,21 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
 
   CUtensorMap tmAct;
   if (!make_tmap_bf16(&tmAct, c.w.a, c.n, m->ff, 128)) return cudaErrorInvalidValue;
+  if (use_fused(c)) {
+    NgptGemmParams f;
+    f.M = c.n; f.N = m->d; f.K = m->ff; f.cluster = m->ngpt_cluster;
+    f.h = h; f.hb = hb; f.alpha = W.alpha_mlp; f.norm_eps = m->cfg.norm_eps;
+    f.e_save = save_e ? c.w.e32 : nullptr;
+    f.e = reinject ? c.w.e32 : nullptr;
+    f.out = out;
+    f.status = m->status;
+    {
+      Launch L(m, c.s, DORY_KK_DOWN);
+      DORY_TRY(launch_gemm_ngpt(tmAct, W.tm_d_n, f, c.s));
+    }
+    ++c.m->cur_sublayers;
+    return cudaSuccess;
+  }
   const int bn_d = c.decode ? 128 : 256;
   GemmParams gd;
   gd.M = c.n; gd.N = m->d; gd.K = m->ff;
@@ -721,6 +762,8 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
   m->ff = cfg->d_ff; m->d_attn = m->hq * m->hd;
   m->n_qkvg = m->d_attn + 2 * m->hkv * m->hd + m->hq;
   m->ld_qkvg = (m->n_qkvg + 31) / 32 * 32;
+  m->ngpt_bnc = ngpt_gemm_cols_per_cta(m->d);
+  m->ngpt_cluster = m->ngpt_bnc ? m->d / m->ngpt_bnc : 0;
   m->nb = n_blocks(cfg);
   m->device = dev;
   m->num_sms = prop.multiProcessorCount;
@@ -785,6 +828,11 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
     }
     ok &= make_tmap_bf16(&W.tm_gu[0], W.wgu, 2 * F, d, 128);
     ok &= make_tmap_bf16(&W.tm_gu[1], W.wgu, 2 * F, d, 256);
+    if (m->ngpt_bnc) {
+      const uint32_t box = m->ngpt_bnc > 256 ? m->ngpt_bnc / 2 : m->ngpt_bnc;
+      ok &= make_tmap_bf16(&W.tm_o_n, W.wo, d, da, box);
+      ok &= make_tmap_bf16(&W.tm_d_n, W.wd, d, F, box);
+    }
     if (!ok) return DORY_ERR_CUDA;
   }
   // static softmax maxima from the packed s_qk vectors (one-time host read)
@@ -894,7 +942,7 @@ int dory_prefill(dory_model* m, dory_kv* kv, int seq, int pos0, int n_tokens, co
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
   GraphKey key{0, k, n_tokens, seq, pos0, 0, m->profile ? 1 : 0, src, dst, ws, kv->uid, nullptr, nullptr,
-               nullptr, m->probe, m->probe ? m->probe_layer : -1};
+               nullptr, m->probe, m->probe ? m->probe_layer : -1, m->fused_update ? 1 : 0};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -931,7 +979,7 @@ int decode_step_impl(dory_model* m, dory_kv* kv, int batch, const int32_t* d_seq
   if (!in_dev && cudaMemcpyAsync(c.w.st_in, h_in, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return DORY_ERR_CUDA;
   GraphKey key{1, k, batch, 0, 0, max_pos_hint, m->profile ? 1 : 0, src, dst, ws, kv->uid, d_seq, d_pos,
-               d_k, m->probe, m->probe ? m->probe_layer : -1};
+               d_k, m->probe, m->probe ? m->probe_layer : -1, m->fused_update ? 1 : 0};
   st = run_graph(m, key, c, src, dst, s);
   if (st != DORY_OK) return st;
   if (!out_dev && cudaMemcpyAsync(h_out, c.w.st_out, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -1081,6 +1129,12 @@ int dory_debug_mask_probe(dory_model* m, int layer, int32_t* d_probe, int max_ro
   m->probe_layer = layer;
   m->probe_rows = max_rows;
   return DORY_OK;
+}
+
+int dory_debug_fused_update(dory_model* m, int enable) {
+  if (!m) return DORY_ERR_INVALID_ARG;
+  m->fused_update = enable != 0;
+  return m->ngpt_bnc > 0 ? DORY_OK : DORY_ERR_BAD_CONFIG;
 }
 
 int dory_debug_attention_paths(const dory_model* m, int32_t* counts) {

@@ -1,0 +1,490 @@
+// Output / down projection with the nGPT hypersphere update fused into the
+// epilogue (prefill):
+//   y = A W^T   (A = the attention output o or the SwiGLU activations a,
+//                W = W_o or W_down; their L2 norms before the projection are
+//                dropped, Norm(c y) = Norm(y) for c > 0)
+//   h <- Norm(h + alpha * (Norm(y) - h))            ("Dory1.0-4B: A Looped
+//   Normalized-GPT", Methodology in Plain English: nGPT residual update)
+// optionally followed by saving the result as the input block's output e and by
+// the re-injection x <- Norm(x + e) before a pass of the recurrent block (same
+// page, Methodology).
+//
+// Both norms are over a whole row of d_model columns, more than one CTA's
+// accumulator holds, so a thread-block cluster of CS CTAs covers the row: CTA
+// rank q owns columns [q*BNC, (q+1)*BNC) of a 128-row band, its fp32
+// accumulator in TMEM (one TMEM lane per row).  Every row norm the update needs
+// is a sum over the row of per-column terms:
+//   ||y||^2                = D  = sum y^2
+//   ||h + a(u - h)||^2     = P1 + 2 P2 / ||y|| + P3 / ||y||^2   (u = y / ||y||)
+//        with P1 = sum ((1-a) h)^2, P2 = sum (1-a) h a y, P3 = sum (a y)^2
+//   ||h_new + e||^2        = |h'|^2 / ||h'||^2 + 2 (Q1 + Q2 / ||y||) / ||h'|| + Q3
+//        with Q1 = sum (1-a) h e, Q2 = sum a y e, Q3 = sum e^2
+// so each CTA reduces its columns' partials per row (one thread = one row),
+// pushes them to every CTA of the cluster through distributed shared memory
+// (st.async with mbarrier transaction counts, no cluster-wide barrier inside
+// the loop), sums the CS partials in rank order (deterministic), and finishes
+// its columns: h (fp32, in place), the bf16 copy for the next GEMM, and the
+// optional e / output rows.
+//
+// Warp roles (192 threads): warp 0 TMA producer (also prefetches this tile's
+// h and e rows into L2), warp 1 TMEM owner and MMA issuer, warps 2..5
+// epilogue.  Persistent clusters walk the row bands.  Every wait is bounded;
+// on expiry the kernel records kStatusTimeout and winds down.
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dory {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kPartials = 8;     // D, P1, P2, P3, Q1, Q2, Q3, (pad) per row
+
+template <int BNC>
+struct NgptCfg {
+  static constexpr int kHalfN = BNC > 256 ? BNC / 2 : BNC;   // N of one MMA / TMA box rows
+  static constexpr int kMmas = BNC / kHalfN;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BNC * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kRecvBytes = 8 * kBM * kPartials * 4;  // up to 8 CTAs x 128 rows
+  static constexpr int kBarOff = kStages * kStageBytes + kRecvBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr uint32_t kTmemCols = BNC <= 128 ? 128 : (BNC <= 256 ? 256 : 512);
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+  static_assert(kHalfN % 16 == 0 && kHalfN <= 256, "MMA N");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// the same shared-memory offset in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// 16 bytes into a peer's shared memory, counted on the peer's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float a, float b, float c, float d,
+                                            uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(raddr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
+      "r"(__float_as_uint(d)), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t rbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait on a barrier completed by other CTAs of the cluster
+__device__ __forceinline__ bool cluster_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort_flag, uint32_t* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 63u) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (abort_flag) *abort_flag = 1;
+        report_status(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void load32(const float* p, float (&v)[32]) {
+  const float4* p4 = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = p4[i];
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+}
+
+template <int BNC>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_ngpt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const NgptGemmParams p) {
+  using C = NgptCfg<BNC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  float* recv = reinterpret_cast<float*>(smem + kStages * C::kStageBytes);   // [CS][128][8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;                    // [kStages]
+  uint64_t* empty = bars + kStages;         // [kStages]
+  uint64_t* tfull = bars + 2 * kStages;     // accumulator ready
+  uint64_t* tempty = tfull + 1;             // accumulator read out (4 epilogue warps)
+  uint64_t* recv_full = tempty + 1;         // all CS CTAs' partials of this tile arrived
+  uint64_t* peers_free = recv_full + 1;     // every CTA has read the previous tile's partials
+  uint64_t* drain = peers_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int CS = p.cluster;
+  const uint32_t rank = cluster_rank();
+  const int cluster_id = blockIdx.x / CS;
+  const int n_clusters = gridDim.x / CS;
+  const int bands = (p.M + kBM - 1) / kBM;
+  const int kb_total = p.K / kBK;
+  const int col0 = static_cast<int>(rank) * BNC;   // this CTA's first column
+  const uint32_t recv_tx = static_cast<uint32_t>(CS) * kBM * kPartials * 4;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 4);
+    mbar_init(recv_full, 1);
+    mbar_init(peers_free, 4 * CS);   // one arrival per epilogue warp of every CTA
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  // every CTA's barriers are initialised before any peer signals them
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      // the epilogue reads each tile's h (and e) columns: bring them towards L2
+      // during the main loop, a few rows per k-block
+      const int rows_per_kb = (kBM + kb_total - 1) / kb_total;
+      for (int band = cluster_id; band < bands && ok; band += n_clusters) {
+        const int r_end = min(p.M, (band + 1) * kBM);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          for (int r = band * kBM + kb * rows_per_kb;
+               r < min(r_end, band * kBM + (kb + 1) * rows_per_kb); ++r) {
+            prefetch_l2(p.h + static_cast<size_t>(r) * p.N + col0, BNC * 4);
+            if (p.e) prefetch_l2(p.e + static_cast<size_t>(r) * p.N + col0, BNC * 4);
+          }
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = tiles + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * kBK, band * kBM);
+#pragma unroll
+          for (int h = 0; h < C::kMmas; ++h)
+            tma_load_2d(a_dst + C::kABytes + h * C::kHalfN * 128, &tmB, &full[stage], kb * kBK,
+                        col0 + h * C::kHalfN);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) drain_wait(&full[s], (issued_parity >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, C::kHalfN);
+      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(tiles));
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(tiles + C::kABytes));
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true, issued = false;
+      for (int band = cluster_id; band < bands && ok; band += n_clusters, ++it) {
+        if (!mbar_wait_bounded(tempty, (it & 1) ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t soff = static_cast<uint64_t>((stage * C::kStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+            for (int h = 0; h < C::kMmas; ++h)
+              umma_bf16(tmem_base + h * C::kHalfN, a_desc0 + soff + ((kk * 32) >> 4),
+                        b_desc0 + soff + ((h * C::kHalfN * 128 + kk * 32) >> 4), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(tfull);
+      }
+      if (!ok && issued) {
+        umma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else {
+    // ---------------------------------------------------- epilogue warps
+    const int quad = warp & 3;
+    const int lrow = quad * 32 + lane;                        // row within the band
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const bool reinject = p.e != nullptr;
+    int it = 0;
+    for (int band = cluster_id; band < bands; band += n_clusters, ++it) {
+      const int row = band * kBM + lrow;
+      const bool row_ok = row < p.M;
+      const size_t roff = static_cast<size_t>(row_ok ? row : 0) * p.N + col0;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull, it & 1, abort_flag, p.status))) break;
+      tc_fence_after();
+      // pass 1: this CTA's columns' share of every row sum
+      float D = 0.f, P1 = 0.f, P2 = 0.f, P3 = 0.f, Q1 = 0.f, Q2 = 0.f, Q3 = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BNC; c += 32) {
+        float y[32], h[32], a[32];
+        tmem_ld32(taddr + c, y);
+        load32(p.alpha + col0 + c, a);
+        if (row_ok) {
+          load32(p.h + roff + c, h);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float hk = (1.f - a[i]) * h[i], ay = a[i] * y[i];
+          D = fmaf(y[i], y[i], D);
+          P1 = fmaf(hk, hk, P1);
+          P2 = fmaf(hk, ay, P2);
+          P3 = fmaf(ay, ay, P3);
+        }
+        if (reinject) {
+          float e[32];
+          if (row_ok) {
+            load32(p.e + roff + c, e);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) e[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            Q1 = fmaf((1.f - a[i]) * h[i], e[i], Q1);
+            Q2 = fmaf(a[i] * y[i], e[i], Q2);
+            Q3 = fmaf(e[i], e[i], Q3);
+          }
+        }
+      }
+      // push the partials to every CTA of the cluster (slot `rank`), once all of
+      // them have read the previous tile's
+      const bool free_ok = cluster_wait_bounded(peers_free, (it & 1) ^ 1u, abort_flag, p.status);
+      if (!__all_sync(0xFFFFFFFFu, free_ok)) break;
+      if (warp == 2 && lane == 0) mbar_arrive_expect_tx(recv_full, recv_tx);
+      {
+        const uint32_t slot = smem_u32(recv + (static_cast<size_t>(rank) * kBM + lrow) * kPartials);
+        const uint32_t bar = smem_u32(recv_full);
+        for (int q = 0; q < CS; ++q) {
+          const uint32_t ra = peer_addr(slot, q), rb = peer_addr(bar, q);
+          st_async_v4(ra, D, P1, P2, P3, rb);
+          st_async_v4(ra + 16, Q1, Q2, Q3, 0.f, rb);
+        }
+      }
+      if (!__all_sync(0xFFFFFFFFu, cluster_wait_bounded(recv_full, it & 1, abort_flag, p.status)))
+        break;
+      // the row sums, added in rank order (the same result in every CTA)
+      D = P1 = P2 = P3 = Q1 = Q2 = Q3 = 0.f;
+      for (int q = 0; q < CS; ++q) {
+        const float4 u = *reinterpret_cast<const float4*>(recv + (static_cast<size_t>(q) * kBM + lrow) * kPartials);
+        const float4 v = *reinterpret_cast<const float4*>(recv + (static_cast<size_t>(q) * kBM + lrow) * kPartials + 4);
+        D += u.x; P1 += u.y; P2 += u.z; P3 += u.w;
+        Q1 += v.x; Q2 += v.y; Q3 += v.z;
+      }
+      __syncwarp();
+      // this CTA's receive slots may take the next tile's partials
+      if (lane == 0)
+        for (int q = 0; q < CS; ++q) remote_arrive(peer_addr(smem_u32(peers_free), q));
+      const float inv_y = rsqrtf(fmaxf(D, p.norm_eps));
+      const float hp2 = P1 + 2.f * P2 * inv_y + P3 * inv_y * inv_y;      // ||h'||^2
+      const float inv_hp = rsqrtf(fmaxf(hp2, p.norm_eps));
+      float inv_x = 1.f;
+      if (reinject) {
+        const float x2 = hp2 * inv_hp * inv_hp + 2.f * (Q1 + Q2 * inv_y) * inv_hp + Q3;
+        inv_x = rsqrtf(fmaxf(x2, p.norm_eps));
+      }
+      // pass 2: h_new = Norm(h + alpha (y / ||y|| - h)) [-> e] [-> Norm(h_new + e)]
+#pragma unroll 1
+      for (int c = 0; c < BNC; c += 32) {
+        float y[32], h[32], a[32];
+        tmem_ld32(taddr + c, y);
+        if (!row_ok) continue;                     // TMEM loads above stay warp-wide
+        load32(p.alpha + col0 + c, a);
+        load32(p.h + roff + c, h);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[i] = (h[i] + a[i] * (y[i] * inv_y - h[i])) * inv_hp;
+        if (p.e_save) {
+          float4* d4 = reinterpret_cast<float4*>(p.e_save + roff + c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d4[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        }
+        if (reinject) {
+          float e[32];
+          load32(p.e + roff + c, e);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = (h[i] + e[i]) * inv_x;
+        }
+        float4* h4 = reinterpret_cast<float4*>(p.h + roff + c);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h4[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        uint4 b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          b[i] = make_uint4(pack_bf16x2(h[8 * i], h[8 * i + 1]), pack_bf16x2(h[8 * i + 2], h[8 * i + 3]),
+                            pack_bf16x2(h[8 * i + 4], h[8 * i + 5]), pack_bf16x2(h[8 * i + 6], h[8 * i + 7]));
+        if (p.hb) {
+          uint4* d = reinterpret_cast<uint4*>(p.hb + roff + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d[i] = b[i];
+        }
+        if (p.out) {
+          uint4* d = reinterpret_cast<uint4*>(p.out + roff + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d[i] = b[i];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);
+    }
+  }
+
+  // no CTA leaves while a peer may still write into its shared memory
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int BNC>
+struct ClusterOcc {
+  int clusters[32] = {0};   // per device ordinal: co-resident clusters (0 = not queried)
+};
+
+template <int BNC>
+cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const NgptGemmParams& p,
+                        cudaStream_t s) {
+  using C = NgptCfg<BNC>;
+  auto kern = gemm_ngpt_kernel<BNC>;
+  static ClusterOcc<BNC> occ;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 32) return cudaErrorInvalidDevice;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (occ.clusters[dev] == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    cfg.gridDim = dim3(p.cluster);
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    occ.clusters[dev] = n;
+  }
+  const int bands = (p.M + kBM - 1) / kBM;
+  const int n_clusters = bands < occ.clusters[dev] ? bands : occ.clusters[dev];
+  if (n_clusters <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(n_clusters * p.cluster);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p);
+}
+
+}  // namespace
+
+int ngpt_gemm_cols_per_cta(int d_model) {
+  // 384 columns per CTA first (d_model 3072 = 8 x 384), then 256 and 128; a
+  // cluster of at most 8 CTAs (the portable limit) covers the row
+  const int options[3] = {384, 256, 128};
+  for (int bnc : options)
+    if (d_model % bnc == 0 && d_model / bnc <= 8) return bnc;
+  return 0;
+}
+
+cudaError_t launch_gemm_ngpt(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const NgptGemmParams& p, cudaStream_t s) {
+  if (p.K % kBK != 0 || p.K <= 0 || p.M <= 0) return cudaErrorInvalidValue;
+  const int bnc = ngpt_gemm_cols_per_cta(p.N);
+  if (bnc == 0 || p.cluster != p.N / bnc) return cudaErrorInvalidValue;
+  switch (bnc) {
+    case 384: return launch_impl<384>(tmA, tmB, p, s);
+    case 256: return launch_impl<256>(tmA, tmB, p, s);
+    case 128: return launch_impl<128>(tmA, tmB, p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dory

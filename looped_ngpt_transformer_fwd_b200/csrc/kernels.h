@@ -50,6 +50,26 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int BN, int head_dim, int num_sms, cudaStream_t s);
 
+// Output / down projection with the nGPT update fused into the epilogue
+// (prefill): a cluster of `cluster` CTAs covers the N = d_model columns of a
+// 128-row band; h is updated in place (see gemm_ngpt.cu).
+struct NgptGemmParams {
+  int M = 0, N = 0, K = 0;
+  int cluster = 0;                   // N / ngpt_gemm_cols_per_cta(N)
+  float* h = nullptr;                // [M, N] fp32 stream, updated in place
+  __nv_bfloat16* hb = nullptr;       // [M, N] bf16 copy for the next GEMM (may be null)
+  const float* alpha = nullptr;      // [N]
+  float* e_save = nullptr;           // optional: the update result is saved here
+  const float* e = nullptr;          // optional: then x <- Norm(x + e)
+  __nv_bfloat16* out = nullptr;      // optional final output [M, N] bf16
+  float norm_eps = 1e-20f;
+  uint32_t* status = nullptr;
+};
+// Columns per CTA of the fused kernel for this d_model (0: not supported).
+int ngpt_gemm_cols_per_cta(int d_model);
+cudaError_t launch_gemm_ngpt(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const NgptGemmParams& p, cudaStream_t s);
+
 // RoPE (cos, sin) table [rows][hd/2] for row r at position pos0 + r (or
 // d_pos[r]): angle = pos * inv_freq[i] in float64, reduced mod 2*pi, then
 // sincosf.

@@ -175,6 +175,10 @@ class DoryModel:
         B.dory_debug_mask_probe(self.handle, 0, None, 0)
         self._probe = None
 
+    def fused_update(self, enable=True):
+        """True when the prefill projections apply the nGPT update in their epilogue."""
+        return B.dory_debug_fused_update(self.handle, enable) == 0 and enable
+
     def attention_paths(self):
         return B.dory_debug_attention_paths(self.handle)
 

@@ -77,3 +77,35 @@ def test_4b_decode_b64_ctx32768_sampled_sequence(big):
     assert_parity(to_np(out[s:s + 1]), ref, what="4B decode sampled sequence")
     del kv
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_4b_shape_stack_matches_oracle_at_every_row(mode):
+    """The 4B block shapes (d_model 3072, 24 / 8 heads of 128, MLP 9216, window
+    4096) with one input, one recurrent and one output block, k = 2, on 300
+    tokens: every row against the oracle.  The fused projections run with an
+    8-CTA cluster per row and a ragged last band (300 = 2 x 128 + 44)."""
+    from looped_ngpt_transformer_fwd_b200 import build as libbuild
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from oracle import weights_from_generator
+    from synthetic import load_config
+    libbuild.build()
+    cfg = load_config("dory4b", n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1, full_period=2)
+    prov = weights_from_generator(cfg, 11, "random")
+    model = DoryModel(cfg, prov)
+    k = 2
+    x, h = inputs(cfg, 43, 302)
+    kv = model.kv_cache(mode, 1, 400, k_max=k)
+    ocache = oracle_cache(cfg, mode, k_max=k)
+    orc = oracle(cfg, prov)
+    out = model.prefill(kv, x[:300], k)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    assert_parity(to_np(out), orc.forward(h[:300], 0, k, ocache), what=f"4B-shape prefill {mode}")
+    for p in (300, 301):
+        d = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pp = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d, pp, 399, k)
+        ref = orc.decode(h[p:p + 1], [0], [p], k, ocache)
+        assert_parity(to_np(out), ref, what=f"4B-shape decode {p} {mode}")
+    model.close()

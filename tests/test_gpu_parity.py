@@ -582,3 +582,37 @@ def test_bounded_wait_timeout_is_reported_and_the_model_stays_usable(tiny):
     assert model.device_status() == 0
     ref = oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, "last_loop", k_max=2))
     assert_parity(to_np(out), ref, what="prefill after a timeout")
+
+
+# ------------------------------------------------------- fused projection + nGPT update
+@pytest.mark.parametrize("mode", ["per_loop", "last_loop"])
+def test_fused_update_matches_unfused_path_and_oracle(hd128, mode):
+    """The output / down projections with the nGPT update (and the re-injection)
+    in their epilogue, a 2-CTA cluster per row at d_model 512, against the
+    unfused path (projection, then the row kernel) and against the oracle."""
+    cfg, prov, model = hd128
+    k = 3
+    x, h = inputs(cfg, 61, 300)
+    outs = []
+    for fused in (True, False):
+        assert model.fused_update(fused) == fused
+        kv = model.kv_cache(mode, 1, 320, k_max=k)
+        outs.append(to_np(model.prefill(kv, x, k)))
+        torch.cuda.synchronize()
+    model.fused_update(True)
+    ref = oracle(cfg, prov).forward(h, 0, k, oracle_cache(cfg, mode, k_max=k))
+    assert_parity(outs[0], ref, what=f"fused {mode}")
+    assert_parity(outs[1], ref, what=f"unfused {mode}")
+    assert_parity(outs[0], outs[1], tol_abs=2e-2, tol_cos=0.9995, what="fused vs unfused")
+    assert model.device_status() == 0
+
+
+def test_fused_update_is_deterministic(g3):
+    """Row sums are added in a fixed order: two runs give the same bits."""
+    cfg, prov, model = g3
+    x, _ = inputs(cfg, 62, 400)
+    kv = model.kv_cache("last_loop", 1, 400, k_max=2)
+    a = model.prefill(kv, x, 2).clone()
+    b = model.prefill(kv, x, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
