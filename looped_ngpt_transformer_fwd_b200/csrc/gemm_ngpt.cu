@@ -479,10 +479,14 @@ cudaError_t launch_gemm_ngpt(const CUtensorMap& tmA, const CUtensorMap& tmB,
   if (p.K % kBK != 0 || p.K <= 0 || p.M <= 0) return cudaErrorInvalidValue;
   const int bnc = ngpt_gemm_cols_per_cta(p.N);
   if (bnc == 0 || p.cluster != p.N / bnc) return cudaErrorInvalidValue;
+  NgptGemmParams q = p;
+  // Re-injecting the row just saved as e gives Norm(2 h_new) = h_new (h_new has
+  // unit norm): the first pass would otherwise read e before it is written.
+  if (q.e && q.e == q.e_save) q.e = nullptr;
   switch (bnc) {
-    case 384: return launch_impl<384>(tmA, tmB, p, s);
-    case 256: return launch_impl<256>(tmA, tmB, p, s);
-    case 128: return launch_impl<128>(tmA, tmB, p, s);
+    case 384: return launch_impl<384>(tmA, tmB, q, s);
+    case 256: return launch_impl<256>(tmA, tmB, q, s);
+    case 128: return launch_impl<128>(tmA, tmB, q, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -597,6 +597,8 @@ def test_fused_update_matches_unfused_path_and_oracle(hd128, mode):
     for fused in (True, False):
         assert model.fused_update(fused) == fused
         kv = model.kv_cache(mode, 1, 320, k_max=k)
+        # every workspace byte is written before it is read: fill it with junk first
+        model.workspace(300).fill_(0x3F)
         outs.append(to_np(model.prefill(kv, x, k)))
         torch.cuda.synchronize()
     model.fused_update(True)
@@ -612,6 +614,7 @@ def test_fused_update_is_deterministic(g3):
     cfg, prov, model = g3
     x, _ = inputs(cfg, 62, 400)
     kv = model.kv_cache("last_loop", 1, 400, k_max=2)
+    model.workspace(400).fill_(0x3F)
     a = model.prefill(kv, x, 2).clone()
     b = model.prefill(kv, x, 2)
     torch.cuda.synchronize()
