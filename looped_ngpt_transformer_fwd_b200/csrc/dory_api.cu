@@ -119,9 +119,12 @@ struct dory_model {
   int d, hq, hkv, hd, ff, d_attn, n_qkvg, nb;
   int ld_qkvg;   // row pitch (floats) of the decode QKVG partial products: n_qkvg rounded up to 32
   // fused projection + nGPT update (prefill): columns per CTA (0 = not
-  // available for this d_model), CTAs per cluster, and whether it is used
+  // available for this d_model), CTAs per cluster, and whether it is used.
+  // Off by default: with an 8-CTA cluster per 3072-column row only 15 clusters
+  // (120 of 148 SMs) are co-resident, and a 4096-token projection then takes
+  // three waves; the unfused projection + row kernel measured faster.
   int ngpt_bnc = 0, ngpt_cluster = 0;
-  bool fused_update = true;
+  bool fused_update = false;
   int device = 0, num_sms = 148;
   uint8_t* wbuf = nullptr;
   size_t wbytes = 0;

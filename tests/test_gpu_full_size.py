@@ -83,8 +83,8 @@ def test_4b_decode_b64_ctx32768_sampled_sequence(big):
 def test_4b_shape_stack_matches_oracle_at_every_row(mode):
     """The 4B block shapes (d_model 3072, 24 / 8 heads of 128, MLP 9216, window
     4096) with one input, one recurrent and one output block, k = 2, on 300
-    tokens: every row against the oracle.  The fused projections run with an
-    8-CTA cluster per row and a ragged last band (300 = 2 x 128 + 44)."""
+    tokens: every row against the oracle, with the fused projections on (an
+    8-CTA cluster per row and a ragged last band, 300 = 2 x 128 + 44)."""
     from looped_ngpt_transformer_fwd_b200 import build as libbuild
     from looped_ngpt_transformer_fwd_b200.model import DoryModel
     from oracle import weights_from_generator
@@ -93,6 +93,7 @@ def test_4b_shape_stack_matches_oracle_at_every_row(mode):
     cfg = load_config("dory4b", n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1, full_period=2)
     prov = weights_from_generator(cfg, 11, "random")
     model = DoryModel(cfg, prov)
+    assert model.fused_update(True)        # the 8-CTA cluster path at the 4B shape
     k = 2
     x, h = inputs(cfg, 43, 302)
     kv = model.kv_cache(mode, 1, 400, k_max=k)
