@@ -269,11 +269,14 @@ class Oracle:
     alpha_mlp [d]; s_qk [hd]).
     """
 
-    def __init__(self, cfg, weights, dtype=np.float64, on_state=None):
+    def __init__(self, cfg, weights, dtype=np.float64, on_state=None, act_quant=None):
         self.cfg = cfg
         self.weights = weights
         self.dt = dtype
         self.on_state = on_state          # optional hook(h) after every sublayer
+        # optional x -> Q(x) applied to every projection's input (quantised
+        # checkpoints: MXFP8 activations, see oracle.quant.mxfp8_fake_quant)
+        self.act_quant = act_quant
         self.sublayer_apps = 0
         self.q_block = 128                # queries per softmax batch (memory only)
 
@@ -281,6 +284,9 @@ class Oracle:
     def _w(self, b, names):
         raw = self.weights(b)
         return {name: _as_float(raw[name], self.dt) for name in names}
+
+    def _act(self, x):
+        return x if self.act_quant is None else self.act_quant(x)
 
     def _norm(self, x, axis=-1):
         return l2norm(x, self.cfg["norm_eps"], axis)
@@ -309,10 +315,11 @@ class Oracle:
         base = cfg["rope_base_full"] if full else cfg["rope_base_swa"]
         positions = pos0 + np.arange(n)
 
-        q = (h @ W["wq"].T).reshape(n, hq, hd)
-        k = (h @ W["wk"].T).reshape(n, hkv, hd)
-        v = (h @ W["wv"].T).reshape(n, hkv, hd)
-        gate = sigmoid(h @ W["wg"].T)                                # [n, hq]
+        hx = self._act(h)                                            # projection input
+        q = (hx @ W["wq"].T).reshape(n, hq, hd)
+        k = (hx @ W["wk"].T).reshape(n, hkv, hd)
+        v = (hx @ W["wv"].T).reshape(n, hkv, hd)
+        gate = sigmoid(hx @ W["wg"].T)                               # [n, hq]
         q = W["s_qk"] * self._norm(rope(q, positions, base))
         k = W["s_qk"] * self._norm(rope(k, positions, base))
 
@@ -338,15 +345,16 @@ class Oracle:
             o[i0:i1] = np.einsum("hij,jhd->ihd", p, Vq)
         o = o * gate[:, :, None]
         o_hat = self._norm(o.reshape(n, hq * hd))
-        y = o_hat @ W["wo"].T
+        y = self._act(o_hat) @ W["wo"].T
         return self._ngpt_update(h, y, W["alpha_attn"])
 
     def mlp_sublayer(self, b, h):
         """SwiGLU sublayer with L2-normalised activations before the down-projection
         ([P1] Methodology in Plain English)."""
         W = self._w(b, ("w_gate", "w_up", "w_down", "alpha_mlp"))
-        a = silu(self.cfg["gate_scale"] * (h @ W["w_gate"].T)) * (h @ W["w_up"].T)
-        y = self._norm(a) @ W["w_down"].T
+        hx = self._act(h)
+        a = silu(self.cfg["gate_scale"] * (hx @ W["w_gate"].T)) * (hx @ W["w_up"].T)
+        y = self._act(self._norm(a)) @ W["w_down"].T
         return self._ngpt_update(h, y, W["alpha_mlp"])
 
     def block(self, b, h, pos0, seq, loop, cache):

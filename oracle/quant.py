@@ -21,7 +21,11 @@ reading is the public definition of each format:
   E2M1(x / (s g)), nearest even, saturating at 6.
 
 Dequantisation multiplies back; a quantised GEMM is C = A @ W_hat^T with W_hat
-the dequantised weights, in float64.  Rounding here is done at the bit level
+the dequantised weights, in float64.  Serving an MXFP8 checkpoint ("standard
+post-training quantisation", same page, Methodology in Plain English) is read
+as the public MX recipe: the weights are stored in MXFP8 and every projection's
+input is quantised to MXFP8 along K as well (mxfp8_gemm), so both operands of
+the block-scaled product are E4M3 with E8M0 block scales.  Rounding here is done at the bit level
 (exponent, then a round-half-even on the grid of that binade); the tests check
 it against an exhaustive nearest-value search and, for E4M3, against
 PyTorch's own float8 conversion.
@@ -145,6 +149,22 @@ def nvfp4_dequantize(codes, scales, g):
     n, k = codes.shape
     v = decode(codes, E2M1).reshape(n, k // NV_BLOCK, NV_BLOCK)
     return (v * decode(scales, E4M3)[:, :, None] * float(g)).reshape(n, k)
+
+
+def mxfp8_fake_quant(x):
+    """x [..., K] (K a multiple of 32) -> the values an MXFP8 encoding of x holds:
+    blocks of 32 consecutive values along the last axis get their E8M0 scale and
+    E4M3 elements (mxfp8_quantize), then are decoded back."""
+    x = np.asarray(x, dtype=np.float64)
+    flat = x.reshape(-1, x.shape[-1])
+    return mxfp8_dequantize(*mxfp8_quantize(flat)).reshape(x.shape)
+
+
+def mxfp8_gemm(a, w):
+    """Both operands in MXFP8 along the reduction axis K, products summed in
+    float64: C = Q(A) Q(W)^T, Q = mxfp8_fake_quant.  This is what a block-scaled
+    MMA computes on an MXFP8 weight and an activation quantised on the fly."""
+    return mxfp8_fake_quant(a) @ mxfp8_fake_quant(w).T
 
 
 def quantized_gemm(a, w_hat):

@@ -210,3 +210,55 @@ def test_quantised_stacks_track_the_bf16_stack():
         assert np.allclose(np.linalg.norm(out, axis=1), 1.0, atol=1e-9)
         err[fmt] = np.abs(out - ref).max()
     assert 0 < err["mxfp8"] < err["nvfp4"] / 2
+
+
+def test_fake_quant_equals_quantise_then_dequantise_per_row():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((3, 5, 96)) * np.exp2(rng.integers(-6, 6, (3, 5, 1)))
+    fq = Q.mxfp8_fake_quant(x)
+    for i in range(3):
+        for j in range(5):
+            c, s = Q.mxfp8_quantize(x[i, j][None, :])
+            assert np.array_equal(fq[i, j], Q.mxfp8_dequantize(c, s)[0])
+    assert np.array_equal(Q.mxfp8_fake_quant(fq), fq)          # idempotent on the grid
+
+
+def test_mxfp8_gemm_brute_force():
+    """Both operands quantised along K, then an exact product: a brute-force sum
+    over decoded codes times their two block scales."""
+    rng = np.random.default_rng(14)
+    a = rng.standard_normal((4, 64))
+    w = rng.standard_normal((6, 64)) * 0.03
+    ca, sa = Q.mxfp8_quantize(a)
+    cw, sw = Q.mxfp8_quantize(w)
+    va, vw = Q.decode(ca, Q.E4M3), Q.decode(cw, Q.E4M3)
+    brute = np.array([[sum(va[i, t] * 2.0 ** (int(sa[i, t // 32]) - 127) *
+                           vw[j, t] * 2.0 ** (int(sw[j, t // 32]) - 127) for t in range(64))
+                       for j in range(6)] for i in range(4)])
+    assert np.allclose(Q.mxfp8_gemm(a, w), brute, rtol=1e-13, atol=1e-15)
+    # relative error of the quantised product stays within a few e4m3 half-ulps
+    exact = a @ w.T
+    assert np.abs(Q.mxfp8_gemm(a, w) - exact).max() < 0.1 * np.abs(exact).max()
+
+
+def test_activation_quantised_stack():
+    """The oracle with MXFP8 weights and MXFP8 projection inputs (the MX serving
+    recipe) stays on the sphere and close to the bf16 stack, closer than NVFP4
+    weights alone; quantising the inputs changes the result (the hook is live)."""
+    from oracle import Oracle, KVCache, weights_from_generator
+    from oracle.quant import dequantized_provider, mxfp8_fake_quant
+    from synthetic import load_config, hidden_in
+    from synthetic.bf16 import bf16_bits_to_f32
+    cfg = load_config("tiny")
+    prov = weights_from_generator(cfg, 11)
+    h = bf16_bits_to_f32(hidden_in(cfg, 12, 48)).astype(np.float64)
+    run = lambda p, aq=None: Oracle(cfg, p, act_quant=aq).forward(
+        h, 0, 2, KVCache(cfg, "last_loop", k_max=2))
+    ref = run(prov)
+    w8 = dequantized_provider(prov, "mxfp8")
+    wonly = run(w8)
+    both = run(w8, mxfp8_fake_quant)
+    cos = (both * ref).sum(1) / np.linalg.norm(both, axis=1) / np.linalg.norm(ref, axis=1)
+    assert cos.min() > 0.999
+    assert np.allclose(np.linalg.norm(both, axis=1), 1.0, atol=1e-9)
+    assert np.abs(both - wonly).max() > 1e-5
