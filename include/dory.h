@@ -67,6 +67,11 @@ typedef enum dory_status {
   DORY_ERR_SCRATCH_LIMIT = -12    /* rows exceed the library's built-in scratch    */
 } dory_status;
 
+typedef enum dory_weight_format {
+  DORY_WEIGHTS_BF16 = 0,  /* bf16 weights, bf16 projection inputs                   */
+  DORY_WEIGHTS_MXFP8 = 1  /* MXFP8 weights and projection inputs (see dory_config)  */
+} dory_weight_format;
+
 typedef enum dory_kv_mode {
   DORY_KV_PER_LOOP = 0,   /* recurrent layers keep one cache per loop (k_max of them) */
   DORY_KV_LAST_LOOP = 1   /* one cache per layer; each loop overwrites the last        */
@@ -95,6 +100,18 @@ typedef struct dory_config {
   float gate_scale;         /* SwiGLU: SiLU(gate_scale * h Wg^T) * (h Wu^T) */
   float norm_eps;           /* Norm(x) = x / sqrt(max(sum x^2, norm_eps))  */
   int32_t allow_extrapolated_k; /* nonzero: accept k up to 8               */
+  /* DORY_WEIGHTS_BF16, or DORY_WEIGHTS_MXFP8: the released MXFP8 checkpoint
+   * format ("Dory1.0-4B: A Looped Normalized-GPT", Key Contributions item 4;
+   * Methodology in Plain English: MXFP8 by standard post-training
+   * quantisation), served as both operands of every projection in MXFP8:
+   * blocks of 32 values along the reduction axis share an E8M0 scale
+   * 2^(floor(log2 amax) - 8) and hold E4M3 elements (nearest, ties to even,
+   * saturating at 448).  dory_create quantises the bf16 source matrices (which
+   * must then be device pointers, 16-byte aligned); every projection input is
+   * quantised on the fly (the attention output and the SwiGLU activations
+   * after their L2 norm), and the products run on the block-scaled tensor
+   * cores (tcgen05.mma kind::mxf8f6f4). */
+  int32_t weight_format;
 } dory_config;
 
 /* Source tensors of one block, row-major [out, in] bf16 matrices (as
@@ -255,6 +272,25 @@ DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
  * all row-major device buffers, K a multiple of 64, N a multiple of 128. */
 DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
 
+/* MXFP8 quantisation along K of bf16 rows src [rows, K] (device, K a multiple
+ * of 128): E4M3 codes [rows, K] bytes into `codes`, E8M0 scale codes into
+ * `scales` (dory_mxfp8_scale_bytes) in 512-byte chunks, one per 128 rows x
+ * 128 K: chunk (kc, rb) at (kc * ceil(rows/128) + rb) * 512, the scale of row
+ * rb*128 + 32*j + i and K block q (0..3) of the chunk at byte i*16 + j*4 + q;
+ * padding rows of the last chunk hold code 127.  Same rule as weight_format
+ * DORY_WEIGHTS_MXFP8. */
+DORY_API int dory_quant_mxfp8(const void* src, int rows, int K, void* codes, void* scales,
+                              void* stream);
+DORY_API size_t dory_mxfp8_scale_bytes(int rows, int K);
+
+/* The block-scaled (MXFP8 x MXFP8) tensor-core GEMM alone: quantises A [M,K]
+ * and B [N,K] (bf16, device) into `ws` (dory_gemm_mxfp8_workspace_bytes, 256-byte
+ * aligned) and writes C = Q(A) Q(B)^T in fp32, split over K into k_splits
+ * slices C[s][M][N] (1..8) whose sum is the product.  K a multiple of 128. */
+DORY_API size_t dory_gemm_mxfp8_workspace_bytes(int M, int N, int K);
+DORY_API int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K,
+                             int k_splits, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------
  * Mask and failure-path diagnostics.
  * --------------------------------------------------------------------- */
@@ -337,6 +373,7 @@ DORY_API int dory_debug_wait_timeout(dory_model* m, uint32_t limit_us, void* str
 
 DORY_API int dory_mlp_sublayer_noalloc(dory_model* m, int layer, int n_rows, float* h,
                                        void* stream);
+/* (Models with weight_format DORY_WEIGHTS_MXFP8 return DORY_ERR_BAD_CONFIG.) */
 
 #ifdef __cplusplus
 }

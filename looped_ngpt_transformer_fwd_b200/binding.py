@@ -33,8 +33,11 @@ EXPORTS = (
     "dory_attention_sublayer", "dory_mlp_sublayer", "dory_gemm_bf16",
     "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
     "dory_debug_mask_probe", "dory_debug_attention_paths", "dory_debug_wait_timeout",
-    "dory_debug_fused_update",
+    "dory_debug_fused_update", "dory_quant_mxfp8", "dory_mxfp8_scale_bytes",
+    "dory_gemm_mxfp8_workspace_bytes", "dory_gemm_mxfp8",
 )
+
+WEIGHT_FORMATS = {"bf16": 0, "mxfp8": 1}
 
 ATTENTION_PATHS = ("prefill_tc", "prefill_mma", "decode_tma", "decode_cp")
 
@@ -60,6 +63,7 @@ class DoryConfig(ctypes.Structure):
         ("rope_base_swa", ctypes.c_double), ("rope_base_full", ctypes.c_double),
         ("softmax_scale", ctypes.c_float), ("gate_scale", ctypes.c_float),
         ("norm_eps", ctypes.c_float), ("allow_extrapolated_k", ctypes.c_int32),
+        ("weight_format", ctypes.c_int32),
     ]
 
 
@@ -108,6 +112,10 @@ def lib():
             "dory_debug_attention_paths": (I, [P, P]),
             "dory_debug_wait_timeout": (I, [P, ctypes.c_uint32, P]),
             "dory_debug_fused_update": (I, [P, I]),
+            "dory_quant_mxfp8": (I, [P, I, I, P, P, P]),
+            "dory_mxfp8_scale_bytes": (SZ, [I, I]),
+            "dory_gemm_mxfp8_workspace_bytes": (SZ, [I, I, I]),
+            "dory_gemm_mxfp8": (I, [P, P, P, I, I, I, I, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -130,14 +138,14 @@ def check(status, where):
     return status
 
 
-def make_config(cfg, allow_extrapolated_k=False):
+def make_config(cfg, allow_extrapolated_k=False, weight_format="bf16"):
     """dory_config from a config dict (configs/*.json)."""
     return DoryConfig(
         cfg["d_model"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"], cfg["d_ff"],
         cfg["n_in_blocks"], cfg["n_rec_blocks"], cfg["n_out_blocks"], cfg["window"],
         cfg["full_period"], float(cfg["rope_base_swa"]), float(cfg["rope_base_full"]),
         float(cfg["softmax_scale"]), float(cfg["gate_scale"]), float(cfg["norm_eps"]),
-        1 if allow_extrapolated_k else 0)
+        1 if allow_extrapolated_k else 0, WEIGHT_FORMATS.get(weight_format, weight_format))
 
 
 # ----------------------------------------------------------------- thin wrappers
@@ -267,6 +275,23 @@ def dory_debug_fused_update(model, enable):
     """Fused projection + nGPT update on (default) or off; returns the status
     (DORY_ERR_BAD_CONFIG when the model's d_model has no fused kernel)."""
     return lib().dory_debug_fused_update(model, 1 if enable else 0)
+
+
+def dory_quant_mxfp8(src, rows, K, codes, scales, stream):
+    return check(lib().dory_quant_mxfp8(src, rows, K, codes, scales, stream), "dory_quant_mxfp8")
+
+
+def dory_mxfp8_scale_bytes(rows, K):
+    return lib().dory_mxfp8_scale_bytes(rows, K)
+
+
+def dory_gemm_mxfp8_workspace_bytes(M, N, K):
+    return lib().dory_gemm_mxfp8_workspace_bytes(M, N, K)
+
+
+def dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream):
+    return check(lib().dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream),
+                 "dory_gemm_mxfp8")
 
 
 def dory_kv_free(kv):

@@ -66,6 +66,11 @@ struct BlockW {
   CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
   // W_o / W_down for the fused projection + nGPT update (box rows = one MMA's N)
   CUtensorMap tm_o_n, tm_d_n;
+  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks, tensor
+  // maps with 128-row boxes; gate / up rows interleaved in groups of 64
+  uint8_t *q8 = nullptr, *o8 = nullptr, *gu8 = nullptr, *d8 = nullptr;
+  uint8_t *qsf = nullptr, *osf = nullptr, *gusf = nullptr, *dsf = nullptr;
+  CUtensorMap tm8_qkvg, tm8_o, tm8_gu, tm8_d;
 };
 
 struct GraphKey {
@@ -125,6 +130,7 @@ struct dory_model {
   // three waves; the unfused projection + row kernel measured faster.
   int ngpt_bnc = 0, ngpt_cluster = 0;
   bool fused_update = false;
+  bool mx = false;   // MXFP8 weights and projection inputs
   int device = 0, num_sms = 148;
   uint8_t* wbuf = nullptr;
   size_t wbytes = 0;
@@ -184,6 +190,8 @@ int validate_config(const dory_config* c) {
   if (c->window < 1 || c->full_period < 1) return DORY_ERR_BAD_CONFIG;
   if (!(c->rope_base_swa > 1.0) || !(c->rope_base_full > 1.0)) return DORY_ERR_BAD_CONFIG;
   if (!(c->softmax_scale > 0.f) || !(c->norm_eps > 0.f)) return DORY_ERR_BAD_CONFIG;
+  if (c->weight_format != DORY_WEIGHTS_BF16 && c->weight_format != DORY_WEIGHTS_MXFP8)
+    return DORY_ERR_BAD_CONFIG;
   return DORY_OK;
 }
 
@@ -191,6 +199,9 @@ struct WeightLayout {
   size_t header = 0;                 // status word + RoPE tables
   size_t per_block = 0;
   size_t off_qkvg = 0, off_o = 0, off_gu = 0, off_d = 0, off_aa = 0, off_am = 0, off_sqk = 0;
+  // MXFP8: codes and scale chunks of the four matrices
+  size_t off_q8 = 0, off_qsf = 0, off_o8 = 0, off_osf = 0, off_gu8 = 0, off_gusf = 0, off_d8 = 0,
+         off_dsf = 0;
   size_t total = 0;
 };
 
@@ -200,10 +211,21 @@ WeightLayout weight_layout(const dory_config* c) {
   const size_t nq = da + 2 * size_t(c->n_kv_heads) * hd + c->n_q_heads;
   L.header = align_up(64) + 2 * align_up(hd / 2 * sizeof(double));
   size_t o = 0;
-  L.off_qkvg = o; o = align_up(o + nq * d * 2);
-  L.off_o = o;    o = align_up(o + d * da * 2);
-  L.off_gu = o;   o = align_up(o + 2 * ff * d * 2);
-  L.off_d = o;    o = align_up(o + d * ff * 2);
+  if (c->weight_format == DORY_WEIGHTS_MXFP8) {
+    L.off_q8 = o;   o = align_up(o + nq * d);
+    L.off_qsf = o;  o = align_up(o + mxfp8_scale_bytes(int(nq), int(d)));
+    L.off_o8 = o;   o = align_up(o + d * da);
+    L.off_osf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(da)));
+    L.off_gu8 = o;  o = align_up(o + 2 * ff * d);
+    L.off_gusf = o; o = align_up(o + mxfp8_scale_bytes(int(2 * ff), int(d)));
+    L.off_d8 = o;   o = align_up(o + d * ff);
+    L.off_dsf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(ff)));
+  } else {
+    L.off_qkvg = o; o = align_up(o + nq * d * 2);
+    L.off_o = o;    o = align_up(o + d * da * 2);
+    L.off_gu = o;   o = align_up(o + 2 * ff * d * 2);
+    L.off_d = o;    o = align_up(o + d * ff * 2);
+  }
   L.off_aa = o;   o = align_up(o + d * 4);
   L.off_am = o;   o = align_up(o + d * 4);
   L.off_sqk = o;  o = align_up(o + hd * 4);
@@ -214,7 +236,7 @@ WeightLayout weight_layout(const dory_config* c) {
 
 struct WsLayout {
   size_t h32, e32, hb, st_in, st_out, q, kf, vf, gate, o, y, a, dacc, dml, rope_swa, rope_full,
-      part, total;
+      part, x8, xsf, total;
   int y_rows;
 };
 
@@ -243,6 +265,10 @@ WsLayout ws_layout(const dory_model* m, int T) {
   L.rope_full = take(size_t(T) * (m->hd / 2) * 8);
   // K-split partial products of the decode QKVG and gate/up projections
   L.part = take(size_t(dec_rows) * kMaxKSplits * std::max<size_t>(m->ld_qkvg, 2 * ff) * 4);
+  // MXFP8 mode: the current projection's input as E4M3 codes and scale chunks
+  const int kmax = std::max(m->d, std::max(m->d_attn, m->ff));
+  L.x8 = m->mx ? take(size_t(T) * kmax) : o;
+  L.xsf = m->mx ? take(mxfp8_scale_bytes(T, kmax)) : o;
   L.total = o;
   return L;
 }
@@ -251,6 +277,7 @@ struct Ws {
   float *h32, *e32, *y, *gate, *dacc, *dml, *part;
   __nv_bfloat16 *hb, *st_in, *st_out, *q, *kf, *vf, *o, *a;
   float2 *rope_swa, *rope_full;
+  uint8_t *x8, *xsf;
 };
 
 Ws ws_bind(const dory_model* m, void* base, int T) {
@@ -274,6 +301,8 @@ Ws ws_bind(const dory_model* m, void* base, int T) {
   w.rope_swa = reinterpret_cast<float2*>(b + L.rope_swa);
   w.rope_full = reinterpret_cast<float2*>(b + L.rope_full);
   w.part = reinterpret_cast<float*>(b + L.part);
+  w.x8 = b + L.x8;
+  w.xsf = b + L.xsf;
   return w;
 }
 
@@ -354,19 +383,55 @@ struct Launch {
 int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   if (tiles >= m->num_sms / 2) return 1;
+  const int kstep = m->mx ? 128 : 64;   // K per pipeline stage
   int s = std::max(1, m->num_sms / tiles);
   s = std::min(s, kMaxKSplits);
-  s = std::min(s, std::max(1, (K / 64) / 4));
+  s = std::min(s, std::max(1, (K / kstep) / 4));
   // the kernel gives each split ceil(kb / s) k-blocks: drop splits left empty
-  const int kb = K / 64, per = (kb + s - 1) / s;
+  const int kb = K / kstep, per = (kb + s - 1) / s;
   return (kb + per - 1) / per;
+}
+
+// The A operand of a projection over this call's rows: the bf16 rows, or in
+// MXFP8 mode their E4M3 codes and scales (from the fp32 stream `f32`, or from
+// bf16 rows scaled to unit L2 norm first when `normalize`; the norms before
+// the output and down projections are applied here, where quantisation makes
+// them matter).  Sets the tensor map and the MXFP8 fields of g.
+cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const __nv_bfloat16* rows,
+                             const float* f32, int K, bool normalize) {
+  dory_model* m = c.m;
+  if (!m->mx) {
+    if (!make_tmap_bf16(tm, rows, c.n, K, 128)) return cudaErrorInvalidValue;
+    return cudaSuccess;
+  }
+  {
+    Launch L(m, c.s, DORY_KK_ROW);
+    if (f32) {
+      DORY_TRY(launch_quant_mxfp8_f32(f32, c.n, K, 0, m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
+    } else {
+      const __nv_bfloat16* seg[1] = {rows};
+      DORY_TRY(launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, c.n, K, normalize ? 1 : 0,
+                                       m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
+    }
+  }
+  if (!make_tmap_u8(tm, c.w.x8, c.n, K, 128)) return cudaErrorInvalidValue;
+  g.mx = 1;
+  g.sfa = c.w.xsf;
+  g.sfa_blocks = (c.n + 127) / 128;
+  return cudaSuccess;
+}
+
+// B operand (weights) of the MXFP8 GEMMs: scale chunks and their row blocks
+void mx_weights(GemmParams& g, const uint8_t* sf, int n_rows) {
+  g.sfb = sf;
+  g.sfb_blocks = (n_rows + 127) / 128;
 }
 
 // Prefill projections with the nGPT update in their epilogue (a cluster of
 // CTAs covers each row); decode keeps K-split GEMMs and the row kernel, which
 // spread its few rows' weight stream over all SMs.
 bool use_fused(const CallCtx& c) {
-  return !c.decode && !c.dk && c.m->fused_update && c.m->ngpt_bnc > 0;
+  return !c.decode && !c.dk && !c.m->mx && c.m->fused_update && c.m->ngpt_bnc > 0;
 }
 
 cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloat16* hb,
@@ -374,12 +439,13 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   dory_model* m = c.m;
   const BlockW& W = m->blocks[b];
   CUtensorMap tmA;
-  if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
+  GemmParams g;
+  DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
+  if (m->mx) mx_weights(g, W.qsf, m->n_qkvg);
   const float2* rope = W.full ? c.w.rope_full : c.w.rope_swa;
   if (c.decode) {
     // few rows: spread the weight stream over the SMs with K splits, then a
     // row kernel applies RoPE / QK-norm / gates to the summed partials
-    GemmParams g;
     g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
     g.epi = kEpiStoreF32;
     g.k_splits = pick_k_splits(m, c.n, m->n_qkvg, 128, m->d);
@@ -389,7 +455,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.status = m->status;
     {
       Launch L(m, c.s, DORY_KK_QKVG);
-      DORY_TRY(launch_gemm(tmA, W.tm_qkvg[0], g, 128, m->hd, m->num_sms, c.s));
+      DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_qkvg : W.tm_qkvg[0], g, 128, m->hd, m->num_sms, c.s));
     }
     QkvgPostParams pp;
     pp.part = c.w.part; pp.splits = g.k_splits; pp.split_stride = g.split_stride; pp.ld = m->ld_qkvg;
@@ -401,7 +467,6 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
       DORY_TRY(launch_qkvg_post(pp, c.s));
     }
   } else {
-    GemmParams g;
     g.M = c.n; g.N = m->n_qkvg; g.K = m->d;
     g.epi = kEpiQKVG;
     g.q_out = c.w.q; g.k_out = c.w.kf; g.v_out = c.w.vf; g.gate_out = c.w.gate;
@@ -411,7 +476,10 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.norm_eps = m->cfg.norm_eps;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_QKVG);
-    DORY_TRY(launch_gemm(tmA, W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
+    if (m->mx)
+      DORY_TRY(launch_gemm(tmA, W.tm8_qkvg, g, 128, m->hd, m->num_sms, c.s));
+    else
+      DORY_TRY(launch_gemm(tmA, W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   const KvLayerView view = kv_view(c.kv, b, loop);
@@ -483,7 +551,9 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
 
   // output projection, then the nGPT update of the stream
   CUtensorMap tmO;
-  if (!make_tmap_bf16(&tmO, c.w.o, c.n, m->d_attn, 128)) return cudaErrorInvalidValue;
+  GemmParams go;
+  DORY_TRY(projection_input(c, &tmO, go, c.w.o, nullptr, m->d_attn, true));
+  if (m->mx) mx_weights(go, W.osf, m->d);
   if (use_fused(c)) {
     NgptGemmParams f;
     f.M = c.n; f.N = m->d; f.K = m->d_attn; f.cluster = m->ngpt_cluster;
@@ -496,8 +566,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     ++c.m->cur_sublayers;
     return cudaSuccess;
   }
-  const int bn_o = c.decode ? 128 : 256;
-  GemmParams go;
+  const int bn_o = (c.decode || m->mx) ? 128 : 256;
   go.M = c.n; go.N = m->d; go.K = m->d_attn;
   go.epi = kEpiStoreF32;
   go.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_o, m->d_attn) : 1;
@@ -505,7 +574,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   go.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_OPROJ);
-    DORY_TRY(launch_gemm(tmO, W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_gemm(tmO, m->mx ? W.tm8_o : W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms,
+                         c.s));
   }
 
   RowUpdateParams r;
@@ -527,9 +597,12 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   dory_model* m = c.m;
   const BlockW& W = m->blocks[b];
   CUtensorMap tmA;
-  if (!make_tmap_bf16(&tmA, hb, c.n, m->d, 128)) return cudaErrorInvalidValue;
+  GemmParams g;
+  DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
+  if (m->mx) mx_weights(g, W.gusf, 2 * m->ff);
+  // gate and up rows alternate in groups of half a GEMM tile
+  const int gu_group = m->mx ? 64 : 128;
   if (c.decode) {
-    GemmParams g;
     g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
     g.epi = kEpiStoreF32;
     g.k_splits = pick_k_splits(m, c.n, 2 * m->ff, 128, m->d);
@@ -537,23 +610,27 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
     g.status = m->status;
     {
       Launch L(m, c.s, DORY_KK_GATEUP);
-      DORY_TRY(launch_gemm(tmA, W.tm_gu[0], g, 128, m->hd, m->num_sms, c.s));
+      DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_gu : W.tm_gu[0], g, 128, m->hd, m->num_sms, c.s));
     }
     Launch L(m, c.s, DORY_KK_GATEUP);
     DORY_TRY(launch_swiglu_post(c.w.part, g.k_splits, g.split_stride, c.n, m->ff,
-                                m->cfg.gate_scale, c.w.a, c.s));
+                                m->cfg.gate_scale, gu_group, c.w.a, c.s));
   } else {
-    GemmParams g;
     g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
     g.epi = kEpiSwiGLU;
     g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_GATEUP);
-    DORY_TRY(launch_gemm(tmA, W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
+    if (m->mx)
+      DORY_TRY(launch_gemm(tmA, W.tm8_gu, g, 128, m->hd, m->num_sms, c.s));
+    else
+      DORY_TRY(launch_gemm(tmA, W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   CUtensorMap tmAct;
-  if (!make_tmap_bf16(&tmAct, c.w.a, c.n, m->ff, 128)) return cudaErrorInvalidValue;
+  GemmParams gd;
+  DORY_TRY(projection_input(c, &tmAct, gd, c.w.a, nullptr, m->ff, true));
+  if (m->mx) mx_weights(gd, W.dsf, m->d);
   if (use_fused(c)) {
     NgptGemmParams f;
     f.M = c.n; f.N = m->d; f.K = m->ff; f.cluster = m->ngpt_cluster;
@@ -569,8 +646,7 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
     ++c.m->cur_sublayers;
     return cudaSuccess;
   }
-  const int bn_d = c.decode ? 128 : 256;
-  GemmParams gd;
+  const int bn_d = (c.decode || m->mx) ? 128 : 256;
   gd.M = c.n; gd.N = m->d; gd.K = m->ff;
   gd.epi = kEpiStoreF32;
   gd.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_d, m->ff) : 1;
@@ -578,7 +654,8 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   gd.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_DOWN);
-    DORY_TRY(launch_gemm(tmAct, W.tm_d[bn_d == 256], gd, bn_d, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_gemm(tmAct, m->mx ? W.tm8_d : W.tm_d[bn_d == 256], gd, bn_d, m->hd,
+                         m->num_sms, c.s));
   }
 
   RowUpdateParams r;
@@ -756,6 +833,12 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
     if (!s.wq || !s.wk || !s.wv || !s.wg || !s.wo || !s.w_gate || !s.w_up || !s.w_down ||
         !s.alpha_attn || !s.alpha_mlp || !s.s_qk)
       return DORY_ERR_INVALID_ARG;
+    // MXFP8 weights are quantised by a kernel that reads the bf16 matrices
+    if (cfg->weight_format == DORY_WEIGHTS_MXFP8) {
+      const void* mats[8] = {s.wq, s.wk, s.wv, s.wg, s.wo, s.w_gate, s.w_up, s.w_down};
+      for (const void* p : mats)
+        if (!is_device_ptr(p) || !is_aligned(p, 16)) return DORY_ERR_INVALID_ARG;
+    }
   }
 
   std::unique_ptr<dory_model> m(new (std::nothrow) dory_model());
@@ -765,6 +848,7 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
   m->ff = cfg->d_ff; m->d_attn = m->hq * m->hd;
   m->n_qkvg = m->d_attn + 2 * m->hkv * m->hd + m->hq;
   m->ld_qkvg = (m->n_qkvg + 31) / 32 * 32;
+  m->mx = cfg->weight_format == DORY_WEIGHTS_MXFP8;
   m->ngpt_bnc = ngpt_gemm_cols_per_cta(m->d);
   m->ngpt_cluster = m->ngpt_bnc ? m->d / m->ngpt_bnc : 0;
   m->nb = n_blocks(cfg);
@@ -803,39 +887,69 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
     const dory_block_src& S = src[b];
     const size_t kvr = size_t(m->hkv) * hd;
     cudaError_t e = cudaSuccess;
-    uint8_t* q = reinterpret_cast<uint8_t*>(W.wqkvg);
-    e = e ? e : cudaMemcpyAsync(q, S.wq, da * d * 2, cudaMemcpyDefault, s);
-    e = e ? e : cudaMemcpyAsync(q + da * d * 2, S.wk, kvr * d * 2, cudaMemcpyDefault, s);
-    e = e ? e : cudaMemcpyAsync(q + (da + kvr) * d * 2, S.wv, kvr * d * 2, cudaMemcpyDefault, s);
-    e = e ? e : cudaMemcpyAsync(q + (da + 2 * kvr) * d * 2, S.wg, size_t(m->hq) * d * 2, cudaMemcpyDefault, s);
-    e = e ? e : cudaMemcpyAsync(W.wo, S.wo, d * da * 2, cudaMemcpyDefault, s);
-    // gate/up interleaved in groups of 128 rows (the SwiGLU epilogue's tile halves)
-    for (size_t t = 0; t < F / 128 && e == cudaSuccess; ++t) {
-      uint8_t* g = reinterpret_cast<uint8_t*>(W.wgu) + (2 * t) * 128 * d * 2;
-      e = cudaMemcpyAsync(g, reinterpret_cast<const uint8_t*>(S.w_gate) + t * 128 * d * 2,
-                          128 * d * 2, cudaMemcpyDefault, s);
-      e = e ? e : cudaMemcpyAsync(g + 128 * d * 2, reinterpret_cast<const uint8_t*>(S.w_up) + t * 128 * d * 2,
-                                  128 * d * 2, cudaMemcpyDefault, s);
+    bool ok = true;
+    if (m->mx) {
+      // MXFP8 weights quantised on the device from the bf16 sources (rows
+      // quantised independently along K: the q | k | v | gate rows of the
+      // fused projection keep their own scales; gate / up rows interleaved in
+      // groups of 64, half a 128-column tile)
+      W.q8 = base + L.off_q8;   W.qsf = base + L.off_qsf;
+      W.o8 = base + L.off_o8;   W.osf = base + L.off_osf;
+      W.gu8 = base + L.off_gu8; W.gusf = base + L.off_gusf;
+      W.d8 = base + L.off_d8;   W.dsf = base + L.off_dsf;
+      const __nv_bfloat16* qs[4] = {reinterpret_cast<const __nv_bfloat16*>(S.wq),
+                                    reinterpret_cast<const __nv_bfloat16*>(S.wk),
+                                    reinterpret_cast<const __nv_bfloat16*>(S.wv),
+                                    reinterpret_cast<const __nv_bfloat16*>(S.wg)};
+      const int qrows[4] = {0, int(da), int(da + kvr), int(da + 2 * kvr)};
+      const __nv_bfloat16* os[1] = {reinterpret_cast<const __nv_bfloat16*>(S.wo)};
+      const __nv_bfloat16* gs[2] = {reinterpret_cast<const __nv_bfloat16*>(S.w_gate),
+                                    reinterpret_cast<const __nv_bfloat16*>(S.w_up)};
+      const __nv_bfloat16* ds[1] = {reinterpret_cast<const __nv_bfloat16*>(S.w_down)};
+      const float eps = cfg->norm_eps;
+      e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, int(d), 0, eps, W.q8, W.qsf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), int(da), 0, eps, W.o8, W.osf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 64, int(2 * F), int(d), 0, eps, W.gu8,
+                                          W.gusf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), int(F), 0, eps, W.d8, W.dsf, s);
+      ok &= make_tmap_u8(&W.tm8_qkvg, W.q8, m->n_qkvg, d, 128);
+      ok &= make_tmap_u8(&W.tm8_o, W.o8, d, da, 128);
+      ok &= make_tmap_u8(&W.tm8_gu, W.gu8, 2 * F, d, 128);
+      ok &= make_tmap_u8(&W.tm8_d, W.d8, d, F, 128);
+    } else {
+      uint8_t* q = reinterpret_cast<uint8_t*>(W.wqkvg);
+      e = e ? e : cudaMemcpyAsync(q, S.wq, da * d * 2, cudaMemcpyDefault, s);
+      e = e ? e : cudaMemcpyAsync(q + da * d * 2, S.wk, kvr * d * 2, cudaMemcpyDefault, s);
+      e = e ? e : cudaMemcpyAsync(q + (da + kvr) * d * 2, S.wv, kvr * d * 2, cudaMemcpyDefault, s);
+      e = e ? e : cudaMemcpyAsync(q + (da + 2 * kvr) * d * 2, S.wg, size_t(m->hq) * d * 2, cudaMemcpyDefault, s);
+      e = e ? e : cudaMemcpyAsync(W.wo, S.wo, d * da * 2, cudaMemcpyDefault, s);
+      // gate/up interleaved in groups of 128 rows (the SwiGLU epilogue's tile halves)
+      for (size_t t = 0; t < F / 128 && e == cudaSuccess; ++t) {
+        uint8_t* g = reinterpret_cast<uint8_t*>(W.wgu) + (2 * t) * 128 * d * 2;
+        e = cudaMemcpyAsync(g, reinterpret_cast<const uint8_t*>(S.w_gate) + t * 128 * d * 2,
+                            128 * d * 2, cudaMemcpyDefault, s);
+        e = e ? e : cudaMemcpyAsync(g + 128 * d * 2, reinterpret_cast<const uint8_t*>(S.w_up) + t * 128 * d * 2,
+                                    128 * d * 2, cudaMemcpyDefault, s);
+      }
+      e = e ? e : cudaMemcpyAsync(W.wd, S.w_down, d * F * 2, cudaMemcpyDefault, s);
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t box = i ? 256 : 128;
+        ok &= make_tmap_bf16(&W.tm_qkvg[i], W.wqkvg, m->n_qkvg, d, box);
+        ok &= make_tmap_bf16(&W.tm_o[i], W.wo, d, da, box);
+        ok &= make_tmap_bf16(&W.tm_d[i], W.wd, d, F, box);
+      }
+      ok &= make_tmap_bf16(&W.tm_gu[0], W.wgu, 2 * F, d, 128);
+      ok &= make_tmap_bf16(&W.tm_gu[1], W.wgu, 2 * F, d, 256);
+      if (m->ngpt_bnc) {
+        const uint32_t box = m->ngpt_bnc > 256 ? m->ngpt_bnc / 2 : m->ngpt_bnc;
+        ok &= make_tmap_bf16(&W.tm_o_n, W.wo, d, da, box);
+        ok &= make_tmap_bf16(&W.tm_d_n, W.wd, d, F, box);
+      }
     }
-    e = e ? e : cudaMemcpyAsync(W.wd, S.w_down, d * F * 2, cudaMemcpyDefault, s);
     e = e ? e : cudaMemcpyAsync(W.alpha_attn, S.alpha_attn, d * 4, cudaMemcpyDefault, s);
     e = e ? e : cudaMemcpyAsync(W.alpha_mlp, S.alpha_mlp, d * 4, cudaMemcpyDefault, s);
     e = e ? e : cudaMemcpyAsync(W.s_qk, S.s_qk, hd * 4, cudaMemcpyDefault, s);
     if (e != cudaSuccess) return DORY_ERR_CUDA;
-    bool ok = true;
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t box = i ? 256 : 128;
-      ok &= make_tmap_bf16(&W.tm_qkvg[i], W.wqkvg, m->n_qkvg, d, box);
-      ok &= make_tmap_bf16(&W.tm_o[i], W.wo, d, da, box);
-      ok &= make_tmap_bf16(&W.tm_d[i], W.wd, d, F, box);
-    }
-    ok &= make_tmap_bf16(&W.tm_gu[0], W.wgu, 2 * F, d, 128);
-    ok &= make_tmap_bf16(&W.tm_gu[1], W.wgu, 2 * F, d, 256);
-    if (m->ngpt_bnc) {
-      const uint32_t box = m->ngpt_bnc > 256 ? m->ngpt_bnc / 2 : m->ngpt_bnc;
-      ok &= make_tmap_bf16(&W.tm_o_n, W.wo, d, da, box);
-      ok &= make_tmap_bf16(&W.tm_d_n, W.wd, d, F, box);
-    }
     if (!ok) return DORY_ERR_CUDA;
   }
   // static softmax maxima from the packed s_qk vectors (one-time host read)
@@ -1154,6 +1268,60 @@ int dory_debug_wait_timeout(dory_model* m, uint32_t limit_us, void* stream) {
   return DORY_OK;
 }
 
+int dory_quant_mxfp8(const void* src, int rows, int K, void* codes, void* scales, void* stream) {
+  if (!src || !codes || !scales || rows <= 0 || K <= 0 || K % 128) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(src, 16) || !is_aligned(codes, 16)) return DORY_ERR_MISALIGNED;
+  const __nv_bfloat16* seg[1] = {static_cast<const __nv_bfloat16*>(src)};
+  if (launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, rows, K, 0, 1e-20f, static_cast<uint8_t*>(codes),
+                              static_cast<uint8_t*>(scales),
+                              static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+size_t dory_mxfp8_scale_bytes(int rows, int K) {
+  if (rows <= 0 || K <= 0 || K % 128) return 0;
+  return mxfp8_scale_bytes(rows, K);
+}
+
+size_t dory_gemm_mxfp8_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
+  return align_up(size_t(M) * K) + align_up(mxfp8_scale_bytes(M, K)) + align_up(size_t(N) * K) +
+         align_up(mxfp8_scale_bytes(N, K));
+}
+
+int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K, int k_splits,
+                    void* ws, size_t ws_bytes, void* stream) {
+  if (!A || !B || !C || !ws || M <= 0 || N <= 0 || K <= 0 || K % 128 || k_splits < 1 ||
+      k_splits > kMaxKSplits)
+    return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16) || !is_aligned(ws))
+    return DORY_ERR_MISALIGNED;
+  if (ws_bytes < dory_gemm_mxfp8_workspace_bytes(M, N, K)) return DORY_ERR_BUFFER_TOO_SMALL;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* a8 = static_cast<uint8_t*>(ws);
+  uint8_t* asf = a8 + align_up(size_t(M) * K);
+  uint8_t* b8 = asf + align_up(mxfp8_scale_bytes(M, K));
+  uint8_t* bsf = b8 + align_up(size_t(N) * K);
+  const __nv_bfloat16* sa[1] = {static_cast<const __nv_bfloat16*>(A)};
+  const __nv_bfloat16* sb[1] = {static_cast<const __nv_bfloat16*>(B)};
+  if (launch_quant_mxfp8_bf16(sa, nullptr, 1, 0, M, K, 0, 1e-20f, a8, asf, s) != cudaSuccess ||
+      launch_quant_mxfp8_bf16(sb, nullptr, 1, 0, N, K, 0, 1e-20f, b8, bsf, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, a8, M, K, 128) || !make_tmap_u8(&tb, b8, N, K, 128)) return DORY_ERR_CUDA;
+  GemmParams p;
+  p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  p.k_splits = k_splits; p.split_stride = size_t(M) * N;
+  p.mx = 1; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128; p.sfb_blocks = (N + 127) / 128;
+  if (launch_gemm(ta, tb, p, 128, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
 int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream) {
   if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || K % 64 || N % 128) return DORY_ERR_INVALID_ARG;
   if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return DORY_ERR_MISALIGNED;
@@ -1205,6 +1373,7 @@ void* noalloc_scratch(int dev) {
 extern "C" int dory_mlp_sublayer_noalloc(dory_model* m, int layer, int n_rows, float* h,
                                          void* stream) {
   if (!m || !h || n_rows <= 0 || layer < 0 || layer >= m->nb) return DORY_ERR_INVALID_ARG;
+  if (m->mx) return DORY_ERR_BAD_CONFIG;   // the built-in scratch has no room for MXFP8 operands
   if (!is_aligned(h, 16)) return DORY_ERR_MISALIGNED;
   const size_t hb_bytes = align_up(size_t(n_rows) * m->d * 2);
   const size_t a_bytes = align_up(size_t(n_rows) * m->ff * 2);

@@ -29,13 +29,24 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kGemmThreads = 192;
 
-template <int BN>
+// MX = false: bf16 operands, 64 K per stage.  MX = true: MXFP8 operands (E4M3
+// codes, one E8M0 scale per 32 along K), 128 K per stage (the same 128 bytes
+// per row), the stage's scale chunks staged in shared memory after the tiles
+// and copied to TMEM for the block-scaled MMA.
+template <int BN, bool MX = false>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kStages = MX ? 5 : ((BN == 256) ? 4 : 6);
+  static constexpr int kKStep = MX ? 128 : kBK;              // K elements per stage
+  static constexpr int kABytes = kBM * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kSfaBytes = MX ? 512 : 0;             // 128 rows x 4 scales
+  static constexpr int kSfbBytes = MX ? 512 * (BN / 128) : 0;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  // accumulators (2 x BN columns), then per stage the A and B scale columns
+  static constexpr int kSfCols = 4 + 4 * (BN / 128);
+  static constexpr int kTmemCols = MX ? 512 : 2 * BN;
+  static_assert(!MX || 2 * BN + kStages * kSfCols <= 512, "TMEM columns");
+  static_assert(kStageBytes % 1024 == 0, "stages keep the tiles 1024-byte aligned");
   // fp32 output staging for bulk tensor stores: 4 epilogue warps x 2 buffers
   // of 32 rows x 32 columns
   static constexpr int kOutBufBytes = 32 * 32 * 4;
@@ -80,6 +91,54 @@ __device__ __forceinline__ void bulk_wait_read_1() {
 }
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// ------------------------------------------------------- MXFP8 (block-scaled) MMA
+// Plain bulk copy global -> shared, counted on an mbarrier (16-byte multiples).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Shared-memory descriptor of one 512-byte scale chunk read by tcgen05.cp as
+// 32 rows of 16 bytes: no swizzle, 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;    // leading byte offset (one core matrix wide)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;    // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1u) << 46;           // descriptor version
+  return d;                                       // layout type 0: no swizzle
+}
+// 32 TMEM lanes x 128 bits from shared memory, repeated in all four 32-lane groups
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4 with block scaling: E4M3
+// A and B (K-major), E8M0 scales, fp32 accumulation, scale byte `sf` of each
+// 32-bit scale column for both operands.
+__host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N, int sf) {
+  return (static_cast<uint32_t>(sf) << 4)          // B scale factor id
+         | (0u << 7) | (0u << 10)                  // A, B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
+         | (1u << 23)                              // scale format: E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)   // M / 16
+         | (static_cast<uint32_t>(sf) << 29);      // A scale factor id
+}
+__device__ __forceinline__ void umma_mxf8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
 }
 
 // --------------------------------------------------------------- epilogues
@@ -302,11 +361,11 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
 }
 
 
-template <int BN, int HD, int EPI>
+template <int BN, int HD, int EPI, bool MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ OutMaps om, const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, MX>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -326,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (p.M + kBM - 1) / kBM;
   const int n_tiles = (p.N + BN - 1) / BN;
-  const int kb_total = p.K / kBK;
+  const int kb_total = p.K / C::kKStep;
   const int kb_per_split = (kb_total + p.k_splits - 1) / p.k_splits;
   const int total = m_tiles * n_tiles * p.k_splits;
 
@@ -381,8 +440,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* a_dst = tiles + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * kBK, mt * kBM);
-          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * kBK, nt * BN);
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKStep, mt * kBM);
+          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKStep, nt * BN);
+          if constexpr (MX) {
+            // this K step's scale chunks: one for A's 128 rows, BN/128 for B's
+            bulk_load(a_dst + C::kABytes + C::kBBytes,
+                      p.sfa + (static_cast<size_t>(kb) * p.sfa_blocks + mt) * 512, C::kSfaBytes,
+                      &full[stage]);
+            bulk_load(a_dst + C::kABytes + C::kBBytes + C::kSfaBytes,
+                      p.sfb + (static_cast<size_t>(kb) * p.sfb_blocks + nt * (BN / 128)) * 512,
+                      C::kSfbBytes, &full[stage]);
+          }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -430,10 +498,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint64_t soff = static_cast<uint64_t>((stage * C::kStageBytes) >> 4);
           const uint64_t a_desc = a_desc0 + soff, b_desc = b_desc0 + soff;
+          if constexpr (MX) {
+            // scales to TMEM (this stage's own columns: the MMAs that read
+            // them last time completed before the stage was refilled), then
+            // four K = 32 block-scaled MMAs, MMA kk reading scale byte kk
+            const uint32_t sf_col = tmem_base + 2 * BN + stage * C::kSfCols;
+            const uint32_t sf_smem = smem_u32(tiles + stage * C::kStageBytes + C::kABytes + C::kBBytes);
+            tmem_cp_32x128b_x4(sf_col, sf_desc(sf_smem));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            umma_bf16(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4), idesc,
-                      (kb > kb0 || kk > 0) ? 1u : 0u);
+            for (int j = 0; j < BN / 128; ++j)
+              tmem_cp_32x128b_x4(sf_col + 4 + 4 * j, sf_desc(sf_smem + C::kSfaBytes + 512 * j));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_mxf8(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4),
+                        umma_idesc_mxf8(kBM, BN, kk), sf_col, sf_col + 4,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              umma_bf16(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4), idesc,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+            }
           }
           issued = true;
           umma_commit(&empty[stage]);
@@ -558,11 +643,11 @@ bool make_tmap_out_bf16(CUtensorMap* map, const void* base, int rows, int cols, 
                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int HD, int EPI>
+template <int BN, int HD, int EPI, bool MX = false>
 cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int num_sms, cudaStream_t s) {
-  using C = GemmCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, HD, EPI>;
+  using C = GemmCfg<BN, MX>;
+  auto kern = gemm_tc_kernel<BN, HD, EPI, MX>;
   static uint32_t attr_done = 0;   // one bit per device ordinal < 32
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -623,13 +708,42 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode || cols % 16 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int BN, int head_dim, int num_sms, cudaStream_t s) {
-  if (p.K % kBK != 0 || p.K <= 0 || p.k_splits < 1) return cudaErrorInvalidValue;
+  const int kstep = p.mx ? 128 : kBK;
+  if (p.K % kstep != 0 || p.K <= 0 || p.k_splits < 1) return cudaErrorInvalidValue;
   {
     // every K split must own at least one k-block
-    const int kb = p.K / kBK, per = (kb + p.k_splits - 1) / p.k_splits;
+    const int kb = p.K / kstep, per = (kb + p.k_splits - 1) / p.k_splits;
     if ((p.k_splits - 1) * per >= kb) return cudaErrorInvalidValue;
+  }
+  if (p.mx) {
+    // block-scaled MXFP8 operands: 128-column tiles (accumulators and scale
+    // columns share TMEM)
+    if (BN != 128 || !p.sfa || !p.sfb) return cudaErrorInvalidValue;
+    switch (p.epi) {
+      case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32, true>(tmA, tmB, p, num_sms, s);
+      case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU, true>(tmA, tmB, p, num_sms, s);
+      case kEpiQKVG:
+        if (p.k_splits != 1) return cudaErrorInvalidValue;
+        if (head_dim == 128) return launch_impl<128, 128, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
+        if (head_dim == 64) return launch_impl<128, 64, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
+        return cudaErrorInvalidValue;
+    }
+    return cudaErrorInvalidValue;
   }
   if (BN == 256) {
     switch (p.epi) {

@@ -38,7 +38,32 @@ struct GemmParams {
   const float2* rope = nullptr;      // [M][hd/2] (cos, sin) of each row's angles, this layer's base
   float norm_eps = 1e-20f;
   uint32_t* status = nullptr;
+  // MXFP8 operands (mx != 0): A and B tensor maps are over E4M3 codes
+  // (make_tmap_u8) and sfa / sfb hold their E8M0 scales in the chunked layout
+  // of quant.cu with sfa_blocks = ceil(M / 128), sfb_blocks = ceil(N / 128)
+  int mx = 0;
+  const uint8_t* sfa = nullptr;
+  const uint8_t* sfb = nullptr;
+  int sfa_blocks = 0, sfb_blocks = 0;
 };
+
+// Encode a 2D tensor map for a row-major uint8 matrix [rows, cols] (MXFP8
+// codes) with a (128 x box_rows) box and the 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows);
+
+// MXFP8 quantisation along K (see quant.cu): codes [rows, K] and scales in
+// 512-byte chunks of (128 rows, 128 K).  `normalize` first scales every row to
+// unit L2 norm.  bf16 sources come in up to 4 row segments (rows
+// [seg_rows[i], seg_rows[i+1]) from segs[i], seg_rows[0] = 0), or with
+// group > 0 as two matrices whose rows alternate in groups of `group`.
+size_t mxfp8_scale_bytes(int rows, int K);
+cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
+                                    int n_seg, int group, int rows, int K, int normalize,
+                                    float norm_eps, uint8_t* codes, uint8_t* scales,
+                                    cudaStream_t s);
+cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normalize, float norm_eps,
+                                   uint8_t* codes, uint8_t* scales, cudaStream_t s);
 
 // Encode a 2D tensor map for a row-major bf16 matrix [rows, cols] with a
 // (64 x box_rows) box and the 128-byte swizzle.  Returns false on failure.
@@ -94,9 +119,10 @@ struct QkvgPostParams {
 cudaError_t launch_qkvg_post(const QkvgPostParams& p, cudaStream_t s);
 
 // K-split gate/up post-processing (decode): columns are the interleaved
-// weight rows (128 gate, 128 up, ...); a = SiLU(gate_scale * g) * u.
+// weight rows (`group` gate, `group` up, ...); a = SiLU(gate_scale * g) * u.
 cudaError_t launch_swiglu_post(const float* part, int splits, size_t split_stride, int rows,
-                               int d_ff, float gate_scale, __nv_bfloat16* out, cudaStream_t s);
+                               int d_ff, float gate_scale, int group, __nv_bfloat16* out,
+                               cudaStream_t s);
 
 // ----------------------------------------------------------------- rows
 struct RowUpdateParams {

@@ -1,0 +1,158 @@
+// MXFP8 quantisation of GEMM operands (the released MXFP8 checkpoint format,
+// "Dory1.0-4B: A Looped Normalized-GPT", Key Contributions item 4, served with
+// both operands of every projection in MXFP8): blocks of 32 consecutive values
+// along K share an E8M0 scale 2^(floor(log2 amax) - 8); each value becomes the
+// E4M3 code nearest to x / scale (ties to even, saturating at 448).
+//
+// Output layout, chosen for the block-scaled tensor-core GEMM:
+//   codes  [rows, K] bytes, row-major (a TMA box of 128 rows x 128 bytes is one
+//          K step of the GEMM);
+//   scales in 512-byte chunks, one per (128 rows, 128 K): chunk (kc, rb) at
+//          ((kc * row_blocks) + rb) * 512, and inside it the scale of row
+//          r = rb*128 + 32*j + i and K block q (0..3) at byte i*16 + j*4 + q.
+//          tcgen05.cp of a chunk (32 rows of 16 bytes, copied to every group of
+//          32 TMEM lanes) puts the scales of row r in column r / 32 of lane
+//          r % 32, byte q: the layout the block-scaled MMA reads.
+// Rows past `rows` (up to the next multiple of 128) get scale code 127 (1.0)
+// so that the MMA never multiplies the zero-filled padding by a NaN scale.
+#include <cuda_fp8.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dory {
+
+namespace {
+
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }
+
+// Where output row r comes from: rows [seg_row[i], seg_row[i+1]) are rows of
+// seg[i]; with `group` > 0 the rows instead alternate in groups of `group`
+// between seg[0] and seg[1] (gate and up projections of one SwiGLU tile).
+template <typename T>
+struct QuantSrc {
+  const T* seg[4];
+  int seg_row[5];
+  int n_seg;
+  int group;
+};
+
+template <typename T>
+__device__ __forceinline__ const T* source_row(const QuantSrc<T>& q, int r, int K) {
+  if (q.group > 0) {
+    const int t = r / (2 * q.group), i = r % (2 * q.group);
+    return (i < q.group ? q.seg[0] : q.seg[1]) +
+           static_cast<size_t>(t * q.group + (i < q.group ? i : i - q.group)) * K;
+  }
+  int i = 0;
+  while (i + 1 < q.n_seg && r >= q.seg_row[i + 1]) ++i;
+  return q.seg[i] + static_cast<size_t>(r - q.seg_row[i]) * K;
+}
+
+// One CTA per (padded) row, one thread per block of 32 values.
+template <typename T>
+__global__ void quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int K, int row_blocks,
+                                   int normalize, float norm_eps, uint8_t* __restrict__ codes,
+                                   uint8_t* __restrict__ scales) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const int q32 = threadIdx.x;                 // block of 32 along K
+  const int nblk = K / 32;
+  const bool live = r < rows && q32 < nblk;
+  const T* row = r < rows ? source_row(src, r, K) : nullptr;
+  float v[32];
+  float amax = 0.f, ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = live ? load_elem(row, static_cast<size_t>(q32) * 32 + i) : 0.f;
+    amax = fmaxf(amax, fabsf(v[i]));
+    ss = fmaf(v[i], v[i], ss);
+  }
+  if (normalize) {
+    // the row's L2 norm first (uniform branch: every thread of the CTA reaches it)
+    ss = warp_sum(ss);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    const int nw = (blockDim.x + 31) >> 5;
+    for (int i = 0; i < nw; ++i) tot += red[i];
+    const float inv = rsqrtf(fmaxf(tot, norm_eps));
+    amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[i] *= inv;
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+  }
+  if (q32 >= nblk) return;
+  int sexp = -127;
+  if (amax > 0.f) sexp = min(127, max(-127, ilogbf(amax) - 8));
+  const int rb = r / 128, rr = r % 128, kc = q32 / 4;
+  scales[(static_cast<size_t>(kc) * row_blocks + rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (q32 % 4)] =
+      static_cast<uint8_t>(r < rows ? sexp + 127 : 127);
+  if (r >= rows) return;
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(ldexpf(v[4 * i], -sexp), ldexpf(v[4 * i + 1], -sexp)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(ldexpf(v[4 * i + 2], -sexp), ldexpf(v[4 * i + 3], -sexp)), __NV_SATFINITE, __NV_E4M3);
+    w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(r) * K + static_cast<size_t>(q32) * 32);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+template <typename T>
+cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int K, int normalize, float norm_eps,
+                         uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (K % 128 != 0 || K / 32 > 1024) return cudaErrorInvalidValue;
+  const int row_blocks = (rows + 127) / 128;
+  const int threads = ((K / 32 + 31) / 32) * 32;
+  quant_mxfp8_kernel<T><<<row_blocks * 128, threads, 0, s>>>(src, rows, K, row_blocks, normalize,
+                                                              norm_eps, codes, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t mxfp8_scale_bytes(int rows, int K) {
+  return static_cast<size_t>((rows + 127) / 128) * (K / 128) * 512;
+}
+
+cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
+                                    int n_seg, int group, int rows, int K, int normalize,
+                                    float norm_eps, uint8_t* codes, uint8_t* scales,
+                                    cudaStream_t s) {
+  if (n_seg < 1 || n_seg > 4 || (group > 0 && n_seg != 2)) return cudaErrorInvalidValue;
+  QuantSrc<__nv_bfloat16> q;
+  memset(&q, 0, sizeof(q));
+  for (int i = 0; i < n_seg; ++i) {
+    q.seg[i] = segs[i];
+    q.seg_row[i] = seg_rows ? seg_rows[i] : 0;
+  }
+  q.seg_row[n_seg] = rows;
+  q.n_seg = n_seg;
+  q.group = group;
+  return launch_quant(q, rows, K, normalize, norm_eps, codes, scales, s);
+}
+
+cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normalize, float norm_eps,
+                                   uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+  QuantSrc<float> q;
+  memset(&q, 0, sizeof(q));
+  q.seg[0] = src;
+  q.seg_row[1] = rows;
+  q.n_seg = 1;
+  return launch_quant(q, rows, K, normalize, norm_eps, codes, scales, s);
+}
+
+}  // namespace dory

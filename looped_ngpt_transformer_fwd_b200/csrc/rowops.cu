@@ -216,17 +216,17 @@ __global__ void qkvg_post_kernel(const QkvgPostParams p) {
 }
 
 __global__ void swiglu_post_kernel(const float* __restrict__ part, int splits, size_t split_stride,
-                                   int rows, int d_ff, float gate_scale,
+                                   int rows, int d_ff, float gate_scale, int group,
                                    __nv_bfloat16* __restrict__ out) {
   const size_t id = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   if (id >= static_cast<size_t>(rows) * d_ff) return;
   const int r = static_cast<int>(id / d_ff), c = static_cast<int>(id % d_ff);
-  const size_t gcol = static_cast<size_t>(c / 128) * 256 + (c % 128);
+  const size_t gcol = static_cast<size_t>(c / group) * 2 * group + (c % group);
   const float* row = part + static_cast<size_t>(r) * 2 * d_ff;
   float g = 0.f, u = 0.f;
   for (int s = 0; s < splits; ++s) {
     g += row[s * split_stride + gcol];
-    u += row[s * split_stride + gcol + 128];
+    u += row[s * split_stride + gcol + group];
   }
   g *= gate_scale;
   out[id] = __float2bfloat16_rn(g * sigmoidf_(g) * u);
@@ -250,11 +250,13 @@ cudaError_t launch_qkvg_post(const QkvgPostParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_swiglu_post(const float* part, int splits, size_t split_stride, int rows,
-                               int d_ff, float gate_scale, __nv_bfloat16* out, cudaStream_t s) {
+                               int d_ff, float gate_scale, int group, __nv_bfloat16* out,
+                               cudaStream_t s) {
   const size_t n = static_cast<size_t>(rows) * d_ff;
   if (n == 0) return cudaSuccess;
+  if (group <= 0 || d_ff % group != 0) return cudaErrorInvalidValue;
   swiglu_post_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-      part, splits, split_stride, rows, d_ff, gate_scale, out);
+      part, splits, split_stride, rows, d_ff, gate_scale, group, out);
   return cudaGetLastError();
 }
 

@@ -68,10 +68,12 @@ class DoryModel:
     matrices as uint16 arrays [out, in], float32 vectors).
     """
 
-    def __init__(self, cfg, weights, device="cuda:0", allow_extrapolated_k=False, stream=None):
+    def __init__(self, cfg, weights, device="cuda:0", allow_extrapolated_k=False, stream=None,
+                 weight_format="bf16"):
         self.cfg = cfg
         self.device = torch.device(device)
-        self.cfg_struct = B.make_config(cfg, allow_extrapolated_k)
+        self.weight_format = weight_format
+        self.cfg_struct = B.make_config(cfg, allow_extrapolated_k, weight_format)
         nb = cfg["n_in_blocks"] + cfg["n_rec_blocks"] + cfg["n_out_blocks"]
         self.n_blocks = nb
         self.wbytes = B.dory_weight_bytes(self.cfg_struct)
@@ -208,6 +210,27 @@ class DoryModel:
             self.close()
         except Exception:
             pass
+
+
+def quant_mxfp8(x, stream=None):
+    """MXFP8 codes [rows, K] (uint8) and the chunked E8M0 scale bytes of bf16 rows x."""
+    rows, K = x.shape
+    codes = torch.empty(rows, K, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(B.dory_mxfp8_scale_bytes(rows, K), dtype=torch.uint8, device=x.device)
+    B.dory_quant_mxfp8(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(stream))
+    return codes, scales
+
+
+def gemm_mxfp8(A, Bm, k_splits=1, stream=None):
+    """Q(A) Q(Bm)^T through the block-scaled GEMM (bf16 in, MXFP8 operands, fp32
+    out) as its K slices [k_splits, M, N]; the product is their sum."""
+    M, K = A.shape
+    N = Bm.shape[0]
+    ws = torch.empty(B.dory_gemm_mxfp8_workspace_bytes(M, N, K), dtype=torch.uint8, device=A.device)
+    C = torch.empty(k_splits, M, N, dtype=torch.float32, device=A.device)
+    B.dory_gemm_mxfp8(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, k_splits, _ptr(ws), ws.numel(),
+                      _stream(stream))
+    return C
 
 
 def gemm_bf16(A, Bm, stream=None):
