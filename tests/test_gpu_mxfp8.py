@@ -40,7 +40,7 @@ def _unchunk(scales, rows, K):
     """Scale codes [rows, K/32] from the chunked layout (dory_quant_mxfp8)."""
     rb = (rows + 127) // 128
     ch = scales.reshape(K // 128, rb, 32, 4, 4)        # kc, rb, i, j, q
-    s = ch.permute(1, 3, 2, 0, 4).reshape(rb * 128, K // 32)   # row = rb*128 + 32 j + i
+    s = ch.transpose(1, 3, 2, 0, 4).reshape(rb * 128, K // 32)   # row = rb*128 + 32 j + i
     return s[:rows], s[rows:]
 
 
