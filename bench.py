@@ -44,6 +44,11 @@ WORKLOADS = {
     "decode_k4_per": dict(kind="decode", batch=8, ctx=131072, k=4, mode="per_loop", seed=3),
     "prefill_long": dict(kind="prefill_chunked", tokens=262144, chunk=8192, k=4, mode="last_loop",
                          seed=4),
+    # the released MXFP8 checkpoint format: MXFP8 weights and projection inputs
+    "prefill_k2_mxfp8": dict(kind="prefill", tokens=4096, k=2, mode="last_loop", seed=1,
+                             fmt="mxfp8"),
+    "decode_k2_mxfp8": dict(kind="decode", batch=64, ctx=32768, k=2, mode="last_loop", seed=2,
+                            fmt="mxfp8"),
 }
 
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
@@ -244,7 +249,8 @@ def run_ours(args, wl, rank, world, device_index, model=None, prov=None, steps=N
     seed = wl["seed"] + 1000 * rank
     if model is None:
         prov = weight_provider(cfg, wl["seed"])
-        model = DoryModel(cfg, prov, device=f"cuda:{device_index}")
+        model = DoryModel(cfg, prov, device=f"cuda:{device_index}",
+                          weight_format=wl.get("fmt", "bf16"))
     k, mode = wl["k"], wl["mode"]
     stream = torch.cuda.current_stream()
     res = {}
@@ -488,6 +494,7 @@ def oracle_sample(wl, prov=None, n_blocks=4):
 
 # ----------------------------------------------------------------- roofline
 DATASHEET = {"tensor": 2250.0, "hbm": 8000.0}    # dense bf16 TFLOP/s, HBM3e GB/s (context only)
+DATASHEET_FP8 = 4500.0
 
 
 def roofline(res, wl, peaks, peak_src):
@@ -500,6 +507,9 @@ def roofline(res, wl, peaks, peak_src):
             achieved = dom_work / (dom_ms / dom_n / 1e3) / 1e12   # dom_work is per launch
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit, key = "TFLOP/s", "bf16_tflops_sustained"
+        if wl.get("fmt") == "mxfp8":
+            # fp8 contraction: the bf16 figure times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+            peak, key = 2.0 * peak, "bf16_tflops_sustained x 2 (fp8)"
         per_launch = dom_work if wl["kind"] != "prefill_chunked" else dom_work / max(dom_n, 1)
         traffic = profiled_traffic(dom_name)
     else:
@@ -511,7 +521,8 @@ def roofline(res, wl, peaks, peak_src):
     return {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": (achieved / peak) if achieved else None,
             "peak_source": f"{peak_src} ({key})",
-            "frac_of_datasheet": (achieved / DATASHEET[bound]) if achieved else None,
+            "frac_of_datasheet": (achieved / (DATASHEET_FP8 if (bound == "tensor" and wl.get("fmt") == "mxfp8")
+                                              else DATASHEET[bound])) if achieved else None,
             "traffic": traffic, "work_per_launch": per_launch, "launches_per_step": dom_n,
             "device_ms_per_step": dom_ms}
 
@@ -526,7 +537,8 @@ def footprint_check(cfg, wl):
     return all(B.dory_kv_bytes(c, "last_loop", B_, ctx, k) == one for k in (1, 2, 3, 4))
 
 
-DEFAULT_EXTRAS = ["prefill_k1", "decode_k2", "decode_k4_last", "decode_k4_per"]
+DEFAULT_EXTRAS = ["prefill_k1", "decode_k2", "decode_k4_last", "decode_k4_per",
+                  "prefill_k2_mxfp8", "decode_k2_mxfp8"]
 
 
 # ----------------------------------------------------------------- main
@@ -596,6 +608,7 @@ def main():
     # the other workloads of the metric (k = 1 prefill, decode at k = 2 and 4 in both
     # cache modes) on the same model, fewer steps each, at N = 1
     extras = {}
+    models = {res["model"].weight_format: res["model"]}
     names = [] if args.extra_workloads in ("", "none") else (
         DEFAULT_EXTRAS if args.extra_workloads == "auto" else args.extra_workloads.split(","))
     if args.extra_workloads == "auto" and (world > 1 or args.workload != "prefill_k2"
@@ -604,7 +617,12 @@ def main():
     for name in names:
         xwl = dict(WORKLOADS[name])
         xsteps = min(args.steps, 10)
-        r = run_ours(args, xwl, rank, world, local, model=res["model"], prov=res["prov"],
+        fmt = xwl.get("fmt", "bf16")
+        if fmt not in models:
+            from looped_ngpt_transformer_fwd_b200.model import DoryModel
+            models[fmt] = DoryModel(res["cfg"], res["prov"], device=f"cuda:{local}",
+                                    weight_format=fmt)
+        r = run_ours(args, xwl, rank, world, local, model=models[fmt], prov=res["prov"],
                      steps=xsteps, warmup=args.warmup)
         entry = {"tokens_per_s": r["units"] * world / r["ms"] * 1e3, "ms_per_step": r["ms"],
                  "steps": xsteps, "warmup": args.warmup, "workload": r["workload"],
@@ -612,7 +630,9 @@ def main():
                  "roofline": roofline(r, xwl, peaks, peak_src),
                  "kernel_ms_per_step": {kk: round(v[0], 4) for kk, v in r["kernel_ms"].items()},
                  "gpu_launches": r["launches"] * xsteps, "clocks": r["clocks"],
-                 "weights_seed": WORKLOADS[args.workload]["seed"]}
+                 "weights_seed": WORKLOADS[args.workload]["seed"],
+                 "dtype": "mxfp8 (E4M3 x E4M3, E8M0 block scales, fp32 accumulation)"
+                 if fmt == "mxfp8" else "bf16"}
         entry.update({kk: vv for kk, vv in r["extra"].items() if kk not in ("k", "kv_mode")})
         entry["k"], entry["kv_mode"] = xwl["k"], xwl["mode"]
         if xwl["kind"] == "decode":
