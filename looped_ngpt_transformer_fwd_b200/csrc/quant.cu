@@ -25,11 +25,6 @@ namespace dory {
 
 namespace {
 
-__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, size_t i) {
-  return __bfloat162float(p[i]);
-}
-__device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }
-
 // Where output row r comes from: rows [seg_row[i], seg_row[i+1]) are rows of
 // seg[i]; with `group` > 0 the rows instead alternate in groups of `group`
 // between seg[0] and seg[1] (gate and up projections of one SwiGLU tile).
@@ -53,72 +48,90 @@ __device__ __forceinline__ const T* source_row(const QuantSrc<T>& q, int r, int 
   return q.seg[i] + static_cast<size_t>(r - q.seg_row[i]) * K;
 }
 
-// One CTA per (padded) row, one thread per block of 32 values.
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+}
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+  const float4 u = *reinterpret_cast<const float4*>(p);
+  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+}
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantMaxIter = 9;     // K up to 9 x 1024
+
+// One CTA per (padded) row.  Thread t holds 4 consecutive values of each 1024
+// of the row (coalesced loads and stores), so the 8 threads t..t+7 (t a
+// multiple of 8) hold one block of 32: its amax is a 3-step shuffle.
 template <typename T>
-__global__ void quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int K, int row_blocks,
-                                   int normalize, float norm_eps, uint8_t* __restrict__ codes,
-                                   uint8_t* __restrict__ scales) {
-  __shared__ float red[32];
+__global__ void __launch_bounds__(kQuantThreads)
+    quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int K, int row_blocks, int normalize,
+                       float norm_eps, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  __shared__ float red[kQuantThreads / 32];
   const int r = blockIdx.x;
-  const int q32 = threadIdx.x;                 // block of 32 along K
-  const int nblk = K / 32;
-  const bool live = r < rows && q32 < nblk;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int iters = K / 1024 + ((K % 1024) ? 1 : 0);
   const T* row = r < rows ? source_row(src, r, K) : nullptr;
-  float v[32];
-  float amax = 0.f, ss = 0.f;
+  float v[kQuantMaxIter][4];
+  float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    v[i] = live ? load_elem(row, static_cast<size_t>(q32) * 32 + i) : 0.f;
-    amax = fmaxf(amax, fabsf(v[i]));
-    ss = fmaf(v[i], v[i], ss);
+  for (int it = 0; it < kQuantMaxIter; ++it) {
+    const int k0 = it * 1024 + tid * 4;
+    if (it < iters && row && k0 < K) {
+      load4(row + k0, v[it]);
+    } else {
+      v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ss = fmaf(v[it][u], v[it][u], ss);
   }
   if (normalize) {
     // the row's L2 norm first (uniform branch: every thread of the CTA reaches it)
     ss = warp_sum(ss);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (l == 0) red[w] = ss;
+    if (lane == 0) red[tid >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
-    const int nw = (blockDim.x + 31) >> 5;
-    for (int i = 0; i < nw; ++i) tot += red[i];
+#pragma unroll
+    for (int i = 0; i < kQuantThreads / 32; ++i) tot += red[i];
     const float inv = rsqrtf(fmaxf(tot, norm_eps));
-    amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      v[i] *= inv;
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
+    for (int it = 0; it < kQuantMaxIter; ++it)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[it][u] *= inv;
   }
-  if (q32 >= nblk) return;
-  int sexp = -127;
-  if (amax > 0.f) sexp = min(127, max(-127, ilogbf(amax) - 8));
-  const int rb = r / 128, rr = r % 128, kc = q32 / 4;
-  scales[(static_cast<size_t>(kc) * row_blocks + rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (q32 % 4)] =
-      static_cast<uint8_t>(r < rows ? sexp + 127 : 127);
-  if (r >= rows) return;
-  uint32_t w[8];
+  const int rb = r / 128, rr = r % 128;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int it = 0; it < kQuantMaxIter; ++it) {
+    if (it >= iters) break;                      // uniform
+    const int k0 = it * 1024 + tid * 4;
+    float amax = fmaxf(fmaxf(fabsf(v[it][0]), fabsf(v[it][1])), fmaxf(fabsf(v[it][2]), fabsf(v[it][3])));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (k0 >= K) continue;                       // whole groups of 8 (K % 32 == 0)
+    int sexp = -127;
+    if (amax > 0.f) sexp = min(127, max(-127, ilogbf(amax) - 8));
+    const int q32 = k0 / 32;
+    if ((tid & 7) == 0)
+      scales[(static_cast<size_t>(q32 / 4) * row_blocks + rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 +
+             (q32 % 4)] = static_cast<uint8_t>(r < rows ? sexp + 127 : 127);
+    if (r >= rows) continue;
     const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[4 * i], -sexp), ldexpf(v[4 * i + 1], -sexp)), __NV_SATFINITE, __NV_E4M3);
+        make_float2(ldexpf(v[it][0], -sexp), ldexpf(v[it][1], -sexp)), __NV_SATFINITE, __NV_E4M3);
     const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[4 * i + 2], -sexp), ldexpf(v[4 * i + 3], -sexp)), __NV_SATFINITE, __NV_E4M3);
-    w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        make_float2(ldexpf(v[it][2], -sexp), ldexpf(v[it][3], -sexp)), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * K + k0) =
+        static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
   }
-  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(r) * K + static_cast<size_t>(q32) * 32);
-  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 template <typename T>
 cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int K, int normalize, float norm_eps,
                          uint8_t* codes, uint8_t* scales, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  if (K % 128 != 0 || K / 32 > 1024) return cudaErrorInvalidValue;
+  if (K % 128 != 0 || K > kQuantMaxIter * 1024) return cudaErrorInvalidValue;
   const int row_blocks = (rows + 127) / 128;
-  const int threads = ((K / 32 + 31) / 32) * 32;
-  quant_mxfp8_kernel<T><<<row_blocks * 128, threads, 0, s>>>(src, rows, K, row_blocks, normalize,
-                                                              norm_eps, codes, scales);
+  quant_mxfp8_kernel<T><<<row_blocks * 128, kQuantThreads, 0, s>>>(src, rows, K, row_blocks,
+                                                                    normalize, norm_eps, codes, scales);
   return cudaGetLastError();
 }
 
