@@ -57,68 +57,56 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
   v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
 }
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantMaxIter = 9;     // K up to 9 x 1024
+constexpr int kQuantWarps = 8;      // rows per CTA (one warp per row)
 
-// One CTA per (padded) row.  Thread t holds 4 consecutive values of each 1024
-// of the row (coalesced loads and stores), so the 8 threads t..t+7 (t a
-// multiple of 8) hold one block of 32: its amax is a 3-step shuffle.
+// One warp per (padded) row.  Lane l holds values 4l..4l+3 of each 128 of the
+// row (coalesced loads and stores); the 8 lanes of a group of 8 hold one block
+// of 32, whose amax is a 3-step shuffle.  With `normalize` a first pass over
+// the row sums the squares (no block-wide barrier: the warp owns the row) and
+// the second pass re-reads the row from cache.
 template <typename T>
-__global__ void __launch_bounds__(kQuantThreads)
-    quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int K, int row_blocks, int normalize,
-                       float norm_eps, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  __shared__ float red[kQuantThreads / 32];
-  const int r = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int iters = K / 1024 + ((K % 1024) ? 1 : 0);
+__global__ void __launch_bounds__(32 * kQuantWarps)
+    quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
+                       int normalize, float norm_eps, uint8_t* __restrict__ codes,
+                       uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (r >= rows_pad) return;                      // warp-uniform
   const T* row = r < rows ? source_row(src, r, K) : nullptr;
-  float v[kQuantMaxIter][4];
-  float ss = 0.f;
-#pragma unroll
-  for (int it = 0; it < kQuantMaxIter; ++it) {
-    const int k0 = it * 1024 + tid * 4;
-    if (it < iters && row && k0 < K) {
-      load4(row + k0, v[it]);
-    } else {
-      v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.f;
+  float inv = 1.f;
+  if (normalize && row) {
+    float ss = 0.f;
+    for (int k0 = lane * 4; k0 < K; k0 += 128) {
+      float v[4];
+      load4(row + k0, v);
+      ss = fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], fmaf(v[3], v[3], ss))));
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) ss = fmaf(v[it][u], v[it][u], ss);
-  }
-  if (normalize) {
-    // the row's L2 norm first (uniform branch: every thread of the CTA reaches it)
-    ss = warp_sum(ss);
-    if (lane == 0) red[tid >> 5] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int i = 0; i < kQuantThreads / 32; ++i) tot += red[i];
-    const float inv = rsqrtf(fmaxf(tot, norm_eps));
-#pragma unroll
-    for (int it = 0; it < kQuantMaxIter; ++it)
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[it][u] *= inv;
+    inv = rsqrtf(fmaxf(warp_sum(ss), norm_eps));
   }
   const int rb = r / 128, rr = r % 128;
+  // K is a multiple of 128: every lane of the warp is inside the row each step
+  for (int base = 0; base < K; base += 128) {
+    const int k0 = base + lane * 4;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (row) {
+      load4(row + k0, v);
 #pragma unroll
-  for (int it = 0; it < kQuantMaxIter; ++it) {
-    if (it >= iters) break;                      // uniform
-    const int k0 = it * 1024 + tid * 4;
-    float amax = fmaxf(fmaxf(fabsf(v[it][0]), fabsf(v[it][1])), fmaxf(fabsf(v[it][2]), fabsf(v[it][3])));
+      for (int u = 0; u < 4; ++u) v[u] *= inv;
+    }
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    if (k0 >= K) continue;                       // whole groups of 8 (K % 32 == 0)
     int sexp = -127;
     if (amax > 0.f) sexp = min(127, max(-127, ilogbf(amax) - 8));
     const int q32 = k0 / 32;
-    if ((tid & 7) == 0)
+    if ((lane & 7) == 0)
       scales[(static_cast<size_t>(q32 / 4) * row_blocks + rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 +
-             (q32 % 4)] = static_cast<uint8_t>(r < rows ? sexp + 127 : 127);
-    if (r >= rows) continue;
+             (q32 % 4)] = static_cast<uint8_t>(row ? sexp + 127 : 127);
+    if (!row) continue;
     const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[it][0], -sexp), ldexpf(v[it][1], -sexp)), __NV_SATFINITE, __NV_E4M3);
+        make_float2(ldexpf(v[0], -sexp), ldexpf(v[1], -sexp)), __NV_SATFINITE, __NV_E4M3);
     const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[it][2], -sexp), ldexpf(v[it][3], -sexp)), __NV_SATFINITE, __NV_E4M3);
+        make_float2(ldexpf(v[2], -sexp), ldexpf(v[3], -sexp)), __NV_SATFINITE, __NV_E4M3);
     *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * K + k0) =
         static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
   }
@@ -128,10 +116,11 @@ template <typename T>
 cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int K, int normalize, float norm_eps,
                          uint8_t* codes, uint8_t* scales, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  if (K % 128 != 0 || K > kQuantMaxIter * 1024) return cudaErrorInvalidValue;
+  if (K % 128 != 0) return cudaErrorInvalidValue;
   const int row_blocks = (rows + 127) / 128;
-  quant_mxfp8_kernel<T><<<row_blocks * 128, kQuantThreads, 0, s>>>(src, rows, K, row_blocks,
-                                                                    normalize, norm_eps, codes, scales);
+  const int rows_pad = row_blocks * 128;
+  quant_mxfp8_kernel<T><<<(rows_pad + kQuantWarps - 1) / kQuantWarps, 32 * kQuantWarps, 0, s>>>(
+      src, rows, rows_pad, K, row_blocks, normalize, norm_eps, codes, scales);
   return cudaGetLastError();
 }
 
