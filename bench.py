@@ -251,6 +251,8 @@ def run_ours(args, wl, rank, world, device_index, model=None, prov=None, steps=N
         prov = weight_provider(cfg, wl["seed"])
         model = DoryModel(cfg, prov, device=f"cuda:{device_index}",
                           weight_format=wl.get("fmt", "bf16"))
+        if args.fused_update:
+            model.fused_update(True)
     k, mode = wl["k"], wl["mode"]
     stream = torch.cuda.current_stream()
     res = {}
@@ -554,6 +556,8 @@ def main():
                     help="profiling aid: IN,REC,OUT block counts (same kernel shapes, smaller model)")
     ap.add_argument("--batch", type=int, default=None,
                     help="profiling aid: decode batch override (same per-sequence work)")
+    ap.add_argument("--fused-update", action="store_true",
+                    help="profiling aid: prefill projections with the nGPT update in their epilogue")
     ap.add_argument("--extra-workloads", default="auto",
                     help="comma-separated workloads reported under 'workloads' in the same line; "
                          "'auto' = the k = 1 prefill and the three decode workloads when the "
