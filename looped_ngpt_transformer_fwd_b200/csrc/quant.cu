@@ -58,12 +58,26 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
 }
 
 constexpr int kQuantWarps = 8;      // rows per CTA (one warp per row)
+constexpr int kQuantUnroll = 8;     // 128-value steps whose loads are in flight together
+
+// Block scale exponent floor(log2 amax) - 8 from the float's exponent field
+// (a subnormal amax gives -135, clamped like any value below 2^-119 to -127),
+// and the exact power of two 2^-sexp that maps the block into E4M3 range.
+__device__ __forceinline__ int block_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  const int e = ((__float_as_int(amax) >> 23) & 0xFF) - 127;
+  return min(127, max(-127, e - 8));
+}
+__device__ __forceinline__ float pow2_neg(int sexp) {   // sexp in [-127, 119]: a normal float
+  return __int_as_float((127 - sexp) << 23);
+}
 
 // One warp per (padded) row.  Lane l holds values 4l..4l+3 of each 128 of the
 // row (coalesced loads and stores); the 8 lanes of a group of 8 hold one block
-// of 32, whose amax is a 3-step shuffle.  With `normalize` a first pass over
-// the row sums the squares (no block-wide barrier: the warp owns the row) and
-// the second pass re-reads the row from cache.
+// of 32, whose amax is a 3-step shuffle.  Loads go out kQuantUnroll steps at a
+// time.  With `normalize` a first pass over the row sums the squares (no
+// block-wide barrier: the warp owns the row) and the second pass re-reads the
+// row from cache.
 template <typename T>
 __global__ void __launch_bounds__(32 * kQuantWarps)
     quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
@@ -76,39 +90,52 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   float inv = 1.f;
   if (normalize && row) {
     float ss = 0.f;
-    for (int k0 = lane * 4; k0 < K; k0 += 128) {
-      float v[4];
-      load4(row + k0, v);
-      ss = fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], fmaf(v[3], v[3], ss))));
+    for (int base = 0; base < K; base += 128 * kQuantUnroll) {
+      float v[kQuantUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int k0 = base + u * 128 + lane * 4;
+        if (k0 < K) load4(row + k0, v[u]);
+        else v[u][0] = v[u][1] = v[u][2] = v[u][3] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u)
+        ss = fmaf(v[u][0], v[u][0], fmaf(v[u][1], v[u][1], fmaf(v[u][2], v[u][2], fmaf(v[u][3], v[u][3], ss))));
     }
     inv = rsqrtf(fmaxf(warp_sum(ss), norm_eps));
   }
   const int rb = r / 128, rr = r % 128;
-  // K is a multiple of 128: every lane of the warp is inside the row each step
-  for (int base = 0; base < K; base += 128) {
-    const int k0 = base + lane * 4;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (row) {
-      load4(row + k0, v);
+  uint8_t* srow = scales + static_cast<size_t>(rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4;
+  for (int base = 0; base < K; base += 128 * kQuantUnroll) {
+    float v[kQuantUnroll][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] *= inv;
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int k0 = base + u * 128 + lane * 4;
+      if (row && k0 < K) load4(row + k0, v[u]);
+      else v[u][0] = v[u][1] = v[u][2] = v[u][3] = 0.f;
     }
-    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    int sexp = -127;
-    if (amax > 0.f) sexp = min(127, max(-127, ilogbf(amax) - 8));
-    const int q32 = k0 / 32;
-    if ((lane & 7) == 0)
-      scales[(static_cast<size_t>(q32 / 4) * row_blocks + rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 +
-             (q32 % 4)] = static_cast<uint8_t>(row ? sexp + 127 : 127);
-    if (!row) continue;
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[0], -sexp), ldexpf(v[1], -sexp)), __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(ldexpf(v[2], -sexp), ldexpf(v[3], -sexp)), __NV_SATFINITE, __NV_E4M3);
-    *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * K + k0) =
-        static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      if (base + u * 128 >= K) break;             // warp-uniform (K is a multiple of 128)
+      const int k0 = base + u * 128 + lane * 4;
+      float amax = fmaxf(fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), fmaxf(fabsf(v[u][2]), fabsf(v[u][3])));
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      // the normalised values' amax (a uniform positive scale commutes with max)
+      const int sexp = block_exponent(amax * inv);
+      const int q32 = k0 / 32;
+      if ((lane & 7) == 0)
+        srow[static_cast<size_t>(q32 / 4) * row_blocks * 512 + (q32 % 4)] =
+            static_cast<uint8_t>(row ? sexp + 127 : 127);
+      if (!row) continue;
+      const float f = inv * pow2_neg(sexp);
+      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[u][0] * f, v[u][1] * f), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[u][2] * f, v[u][3] * f), __NV_SATFINITE, __NV_E4M3);
+      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * K + k0) =
+          static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
   }
 }
 
