@@ -66,11 +66,12 @@ struct BlockW {
   CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
   // W_o / W_down for the fused projection + nGPT update (box rows = one MMA's N)
   CUtensorMap tm_o_n, tm_d_n;
-  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks, tensor
-  // maps with 128-row boxes; gate / up rows interleaved in groups of 64
+  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks; gate /
+  // up rows interleaved in groups of 128 as in the bf16 layout
   uint8_t *q8 = nullptr, *o8 = nullptr, *gu8 = nullptr, *d8 = nullptr;
   uint8_t *qsf = nullptr, *osf = nullptr, *gusf = nullptr, *dsf = nullptr;
-  CUtensorMap tm8_qkvg, tm8_o, tm8_gu, tm8_d;
+  CUtensorMap tm8_qkvg, tm8_o, tm8_gu, tm8_d;                  // 128-row boxes (decode)
+  CUtensorMap tm8_qkvg_256, tm8_o_256, tm8_gu_256, tm8_d_256;  // 256-row boxes (prefill)
 };
 
 struct GraphKey {
@@ -476,10 +477,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.norm_eps = m->cfg.norm_eps;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_QKVG);
-    if (m->mx)
-      DORY_TRY(launch_gemm(tmA, W.tm8_qkvg, g, 128, m->hd, m->num_sms, c.s));
-    else
-      DORY_TRY(launch_gemm(tmA, W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_qkvg_256 : W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   const KvLayerView view = kv_view(c.kv, b, loop);
@@ -566,7 +564,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     ++c.m->cur_sublayers;
     return cudaSuccess;
   }
-  const int bn_o = (c.decode || m->mx) ? 128 : 256;
+  const int bn_o = c.decode ? 128 : 256;
   go.M = c.n; go.N = m->d; go.K = m->d_attn;
   go.epi = kEpiStoreF32;
   go.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_o, m->d_attn) : 1;
@@ -574,8 +572,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   go.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_OPROJ);
-    DORY_TRY(launch_gemm(tmO, m->mx ? W.tm8_o : W.tm_o[bn_o == 256], go, bn_o, m->hd, m->num_sms,
-                         c.s));
+    const CUtensorMap& tb = m->mx ? (bn_o == 256 ? W.tm8_o_256 : W.tm8_o) : W.tm_o[bn_o == 256];
+    DORY_TRY(launch_gemm(tmO, tb, go, bn_o, m->hd, m->num_sms, c.s));
   }
 
   RowUpdateParams r;
@@ -600,8 +598,8 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   GemmParams g;
   DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
   if (m->mx) mx_weights(g, W.gusf, 2 * m->ff);
-  // gate and up rows alternate in groups of half a GEMM tile
-  const int gu_group = m->mx ? 64 : 128;
+  // gate and up rows alternate in groups of 128 (half a 256-column GEMM tile)
+  const int gu_group = 128;
   if (c.decode) {
     g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
     g.epi = kEpiStoreF32;
@@ -621,10 +619,7 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
     g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_GATEUP);
-    if (m->mx)
-      DORY_TRY(launch_gemm(tmA, W.tm8_gu, g, 128, m->hd, m->num_sms, c.s));
-    else
-      DORY_TRY(launch_gemm(tmA, W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
+    DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_gu_256 : W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   CUtensorMap tmAct;
@@ -646,7 +641,7 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
     ++c.m->cur_sublayers;
     return cudaSuccess;
   }
-  const int bn_d = (c.decode || m->mx) ? 128 : 256;
+  const int bn_d = c.decode ? 128 : 256;
   gd.M = c.n; gd.N = m->d; gd.K = m->ff;
   gd.epi = kEpiStoreF32;
   gd.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_d, m->ff) : 1;
@@ -654,8 +649,8 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   gd.status = m->status;
   {
     Launch L(m, c.s, DORY_KK_DOWN);
-    DORY_TRY(launch_gemm(tmAct, m->mx ? W.tm8_d : W.tm_d[bn_d == 256], gd, bn_d, m->hd,
-                         m->num_sms, c.s));
+    const CUtensorMap& tb = m->mx ? (bn_d == 256 ? W.tm8_d_256 : W.tm8_d) : W.tm_d[bn_d == 256];
+    DORY_TRY(launch_gemm(tmAct, tb, gd, bn_d, m->hd, m->num_sms, c.s));
   }
 
   RowUpdateParams r;
@@ -892,7 +887,7 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
       // MXFP8 weights quantised on the device from the bf16 sources (rows
       // quantised independently along K: the q | k | v | gate rows of the
       // fused projection keep their own scales; gate / up rows interleaved in
-      // groups of 64, half a 128-column tile)
+      // groups of 128, half a 256-column tile)
       W.q8 = base + L.off_q8;   W.qsf = base + L.off_qsf;
       W.o8 = base + L.off_o8;   W.osf = base + L.off_osf;
       W.gu8 = base + L.off_gu8; W.gusf = base + L.off_gusf;
@@ -909,13 +904,17 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
       const float eps = cfg->norm_eps;
       e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, int(d), 0, eps, W.q8, W.qsf, s);
       e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), int(da), 0, eps, W.o8, W.osf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 64, int(2 * F), int(d), 0, eps, W.gu8,
+      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 128, int(2 * F), int(d), 0, eps, W.gu8,
                                           W.gusf, s);
       e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), int(F), 0, eps, W.d8, W.dsf, s);
       ok &= make_tmap_u8(&W.tm8_qkvg, W.q8, m->n_qkvg, d, 128);
       ok &= make_tmap_u8(&W.tm8_o, W.o8, d, da, 128);
       ok &= make_tmap_u8(&W.tm8_gu, W.gu8, 2 * F, d, 128);
       ok &= make_tmap_u8(&W.tm8_d, W.d8, d, F, 128);
+      ok &= make_tmap_u8(&W.tm8_qkvg_256, W.q8, m->n_qkvg, d, 256);
+      ok &= make_tmap_u8(&W.tm8_o_256, W.o8, d, da, 256);
+      ok &= make_tmap_u8(&W.tm8_gu_256, W.gu8, 2 * F, d, 256);
+      ok &= make_tmap_u8(&W.tm8_d_256, W.d8, d, F, 256);
     } else {
       uint8_t* q = reinterpret_cast<uint8_t*>(W.wqkvg);
       e = e ? e : cudaMemcpyAsync(q, S.wq, da * d * 2, cudaMemcpyDefault, s);
@@ -1312,13 +1311,15 @@ int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K,
   if (launch_quant_mxfp8_bf16(sa, nullptr, 1, 0, M, K, 0, 1e-20f, a8, asf, s) != cudaSuccess ||
       launch_quant_mxfp8_bf16(sb, nullptr, 1, 0, N, K, 0, 1e-20f, b8, bsf, s) != cudaSuccess)
     return DORY_ERR_CUDA;
+  // 256-column tiles (one accumulator) when N allows, else 128 (two)
+  const int BN = (N % 256 == 0) ? 256 : 128;
   CUtensorMap ta, tb;
-  if (!make_tmap_u8(&ta, a8, M, K, 128) || !make_tmap_u8(&tb, b8, N, K, 128)) return DORY_ERR_CUDA;
+  if (!make_tmap_u8(&ta, a8, M, K, 128) || !make_tmap_u8(&tb, b8, N, K, BN)) return DORY_ERR_CUDA;
   GemmParams p;
   p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
   p.k_splits = k_splits; p.split_stride = size_t(M) * N;
   p.mx = 1; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128; p.sfb_blocks = (N + 127) / 128;
-  if (launch_gemm(ta, tb, p, 128, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
+  if (launch_gemm(ta, tb, p, BN, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
   return DORY_OK;
 }
 

@@ -35,17 +35,20 @@ constexpr int kGemmThreads = 192;
 // and copied to TMEM for the block-scaled MMA.
 template <int BN, bool MX = false>
 struct GemmCfg {
-  static constexpr int kStages = MX ? 5 : ((BN == 256) ? 4 : 6);
+  static constexpr int kStages = MX ? (BN == 256 ? 3 : 5) : ((BN == 256) ? 4 : 6);
   static constexpr int kKStep = MX ? 128 : kBK;              // K elements per stage
   static constexpr int kABytes = kBM * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = MX ? 512 : 0;             // 128 rows x 4 scales
   static constexpr int kSfbBytes = MX ? 512 * (BN / 128) : 0;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  // accumulators (2 x BN columns), then per stage the A and B scale columns
+  static constexpr int kStageBytes = (kABytes + kBBytes + kSfaBytes + kSfbBytes + 1023) / 1024 * 1024;
+  // accumulators (kAccBufs x BN columns), then per stage the A and B scale
+  // columns; a 256-column MXFP8 tile keeps a single accumulator so that the
+  // scale columns fit next to it
+  static constexpr int kAccBufs = (MX && BN == 256) ? 1 : 2;
   static constexpr int kSfCols = 4 + 4 * (BN / 128);
   static constexpr int kTmemCols = MX ? 512 : 2 * BN;
-  static_assert(!MX || 2 * BN + kStages * kSfCols <= 512, "TMEM columns");
+  static_assert(!MX || kAccBufs * BN + kStages * kSfCols <= 512, "TMEM columns");
   static_assert(kStageBytes % 1024 == 0, "stages keep the tiles 1024-byte aligned");
   // fp32 output staging for bulk tensor stores: 4 epilogue warps x 2 buffers
   // of 32 rows x 32 columns
@@ -482,8 +485,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int ks = rest / n_tiles;
         const int kb0 = ks * kb_per_split;
         const int kb1 = min(kb_total, kb0 + kb_per_split);
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int acc = it % C::kAccBufs;
+        const uint32_t aph = (it / C::kAccBufs) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) {
           ok = false;
           break;
@@ -502,7 +505,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // scales to TMEM (this stage's own columns: the MMAs that read
             // them last time completed before the stage was refilled), then
             // four K = 32 block-scaled MMAs, MMA kk reading scale byte kk
-            const uint32_t sf_col = tmem_base + 2 * BN + stage * C::kSfCols;
+            const uint32_t sf_col = tmem_base + C::kAccBufs * BN + stage * C::kSfCols;
             const uint32_t sf_smem = smem_u32(tiles + stage * C::kStageBytes + C::kABytes + C::kBBytes);
             tmem_cp_32x128b_x4(sf_col, sf_desc(sf_smem));
 #pragma unroll
@@ -546,8 +549,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int rest = t / m_tiles;
       const int nt = rest % n_tiles;
       const int ks = rest / n_tiles;
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      const int acc = it % C::kAccBufs;
+      const uint32_t aph = (it / C::kAccBufs) & 1;
       // warp-uniform: the TMEM loads below are warp-collective
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status))) break;
       tc_fence_after();
@@ -731,9 +734,21 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
     if ((p.k_splits - 1) * per >= kb) return cudaErrorInvalidValue;
   }
   if (p.mx) {
-    // block-scaled MXFP8 operands: 128-column tiles (accumulators and scale
-    // columns share TMEM)
-    if (BN != 128 || !p.sfa || !p.sfb) return cudaErrorInvalidValue;
+    // block-scaled MXFP8 operands (accumulators and scale columns share TMEM)
+    if (!p.sfa || !p.sfb) return cudaErrorInvalidValue;
+    if (BN == 256) {
+      switch (p.epi) {
+        case kEpiStoreF32: return launch_impl<256, 128, kEpiStoreF32, true>(tmA, tmB, p, num_sms, s);
+        case kEpiSwiGLU: return launch_impl<256, 128, kEpiSwiGLU, true>(tmA, tmB, p, num_sms, s);
+        case kEpiQKVG:
+          if (p.k_splits != 1) return cudaErrorInvalidValue;
+          if (head_dim == 128) return launch_impl<256, 128, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
+          if (head_dim == 64) return launch_impl<256, 64, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
+          return cudaErrorInvalidValue;
+      }
+      return cudaErrorInvalidValue;
+    }
+    if (BN != 128) return cudaErrorInvalidValue;
     switch (p.epi) {
       case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32, true>(tmA, tmB, p, num_sms, s);
       case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU, true>(tmA, tmB, p, num_sms, s);

@@ -60,7 +60,9 @@ def test_quantiser_codes_and_scales_are_bit_exact(M, K):
 
 
 @pytest.mark.parametrize("M,N,K,splits", [(300, 512, 384, 1), (64, 384, 3072, 4), (1, 128, 128, 1),
-                                          (129, 1286, 256, 1), (1000, 768, 1024, 2)])
+                                          (129, 1286, 256, 1), (1000, 768, 1024, 2),
+                                          (700, 1024, 3072, 1), (64, 2048, 1024, 3)])
+# (N a multiple of 256: 256-column tiles with one accumulator; else 128-column tiles)
 def test_block_scaled_gemm_matches_decoded_product(M, N, K, splits):
     from looped_ngpt_transformer_fwd_b200 import build as libbuild
     from looped_ngpt_transformer_fwd_b200.model import gemm_mxfp8
