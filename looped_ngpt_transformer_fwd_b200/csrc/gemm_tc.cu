@@ -41,7 +41,11 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = MX ? 512 : 0;             // 128 rows x 4 scales
   static constexpr int kSfbBytes = MX ? 512 * (BN / 128) : 0;
-  static constexpr int kStageBytes = (kABytes + kBBytes + kSfaBytes + kSfbBytes + 1023) / 1024 * 1024;
+  // bytes the TMA and bulk copies of one stage deliver (the mbarrier's
+  // transaction count), and the stage's footprint, padded to keep every
+  // stage's tiles 1024-byte aligned
+  static constexpr int kLoadBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStageBytes = (kLoadBytes + 1023) / 1024 * 1024;
   // accumulators (kAccBufs x BN columns), then per stage the A and B scale
   // columns; a 256-column MXFP8 tile keeps a single accumulator so that the
   // scale columns fit next to it
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           uint8_t* a_dst = tiles + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], C::kLoadBytes);
           tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKStep, mt * kBM);
           tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKStep, nt * BN);
           if constexpr (MX) {
