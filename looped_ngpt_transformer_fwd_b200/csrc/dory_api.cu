@@ -214,13 +214,14 @@ WeightLayout weight_layout(const dory_config* c) {
   size_t o = 0;
   if (c->weight_format == DORY_WEIGHTS_MXFP8) {
     L.off_q8 = o;   o = align_up(o + nq * d);
-    L.off_qsf = o;  o = align_up(o + mxfp8_scale_bytes(int(nq), int(d)));
+    // weight scale chunks cover whole 256-row tiles
+    L.off_qsf = o;  o = align_up(o + mxfp8_scale_bytes(int(nq), int(d), 256));
     L.off_o8 = o;   o = align_up(o + d * da);
-    L.off_osf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(da)));
+    L.off_osf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(da), 256));
     L.off_gu8 = o;  o = align_up(o + 2 * ff * d);
-    L.off_gusf = o; o = align_up(o + mxfp8_scale_bytes(int(2 * ff), int(d)));
+    L.off_gusf = o; o = align_up(o + mxfp8_scale_bytes(int(2 * ff), int(d), 256));
     L.off_d8 = o;   o = align_up(o + d * ff);
-    L.off_dsf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(ff)));
+    L.off_dsf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(ff), 256));
   } else {
     L.off_qkvg = o; o = align_up(o + nq * d * 2);
     L.off_o = o;    o = align_up(o + d * da * 2);
@@ -411,7 +412,7 @@ cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const _
       DORY_TRY(launch_quant_mxfp8_f32(f32, c.n, K, 0, m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
     } else {
       const __nv_bfloat16* seg[1] = {rows};
-      DORY_TRY(launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, c.n, K, normalize ? 1 : 0,
+      DORY_TRY(launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, c.n, 128, K, normalize ? 1 : 0,
                                        m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
     }
   }
@@ -423,9 +424,10 @@ cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const _
 }
 
 // B operand (weights) of the MXFP8 GEMMs: scale chunks and their row blocks
+// (weights' chunks cover whole 256-row tiles)
 void mx_weights(GemmParams& g, const uint8_t* sf, int n_rows) {
   g.sfb = sf;
-  g.sfb_blocks = (n_rows + 127) / 128;
+  g.sfb_blocks = (n_rows + 255) / 256 * 2;
 }
 
 // Prefill projections with the nGPT update in their epilogue (a cluster of
@@ -902,11 +904,14 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
                                     reinterpret_cast<const __nv_bfloat16*>(S.w_up)};
       const __nv_bfloat16* ds[1] = {reinterpret_cast<const __nv_bfloat16*>(S.w_down)};
       const float eps = cfg->norm_eps;
-      e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, int(d), 0, eps, W.q8, W.qsf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), int(da), 0, eps, W.o8, W.osf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 128, int(2 * F), int(d), 0, eps, W.gu8,
-                                          W.gusf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), int(F), 0, eps, W.d8, W.dsf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, 256, int(d), 0, eps, W.q8,
+                                          W.qsf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), 256, int(da), 0, eps, W.o8,
+                                          W.osf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 128, int(2 * F), 256, int(d), 0, eps,
+                                          W.gu8, W.gusf, s);
+      e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), 256, int(F), 0, eps, W.d8,
+                                          W.dsf, s);
       ok &= make_tmap_u8(&W.tm8_qkvg, W.q8, m->n_qkvg, d, 128);
       ok &= make_tmap_u8(&W.tm8_o, W.o8, d, da, 128);
       ok &= make_tmap_u8(&W.tm8_gu, W.gu8, 2 * F, d, 128);
@@ -1271,7 +1276,7 @@ int dory_quant_mxfp8(const void* src, int rows, int K, void* codes, void* scales
   if (!src || !codes || !scales || rows <= 0 || K <= 0 || K % 128) return DORY_ERR_INVALID_ARG;
   if (!is_aligned(src, 16) || !is_aligned(codes, 16)) return DORY_ERR_MISALIGNED;
   const __nv_bfloat16* seg[1] = {static_cast<const __nv_bfloat16*>(src)};
-  if (launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, rows, K, 0, 1e-20f, static_cast<uint8_t*>(codes),
+  if (launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, rows, 128, K, 0, 1e-20f, static_cast<uint8_t*>(codes),
                               static_cast<uint8_t*>(scales),
                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DORY_ERR_CUDA;
@@ -1286,7 +1291,7 @@ size_t dory_mxfp8_scale_bytes(int rows, int K) {
 size_t dory_gemm_mxfp8_workspace_bytes(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
   return align_up(size_t(M) * K) + align_up(mxfp8_scale_bytes(M, K)) + align_up(size_t(N) * K) +
-         align_up(mxfp8_scale_bytes(N, K));
+         align_up(mxfp8_scale_bytes(N, K, 256));
 }
 
 int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K, int k_splits,
@@ -1308,17 +1313,19 @@ int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K,
   uint8_t* bsf = b8 + align_up(size_t(N) * K);
   const __nv_bfloat16* sa[1] = {static_cast<const __nv_bfloat16*>(A)};
   const __nv_bfloat16* sb[1] = {static_cast<const __nv_bfloat16*>(B)};
-  if (launch_quant_mxfp8_bf16(sa, nullptr, 1, 0, M, K, 0, 1e-20f, a8, asf, s) != cudaSuccess ||
-      launch_quant_mxfp8_bf16(sb, nullptr, 1, 0, N, K, 0, 1e-20f, b8, bsf, s) != cudaSuccess)
-    return DORY_ERR_CUDA;
-  // 256-column tiles (one accumulator) when N allows, else 128 (two)
+  // 256-column tiles (one accumulator) when N allows, else 128 (two); B's
+  // scale chunks cover whole tiles
   const int BN = (N % 256 == 0) ? 256 : 128;
+  if (launch_quant_mxfp8_bf16(sa, nullptr, 1, 0, M, 128, K, 0, 1e-20f, a8, asf, s) != cudaSuccess ||
+      launch_quant_mxfp8_bf16(sb, nullptr, 1, 0, N, BN, K, 0, 1e-20f, b8, bsf, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
   CUtensorMap ta, tb;
   if (!make_tmap_u8(&ta, a8, M, K, 128) || !make_tmap_u8(&tb, b8, N, K, BN)) return DORY_ERR_CUDA;
   GemmParams p;
   p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
   p.k_splits = k_splits; p.split_stride = size_t(M) * N;
-  p.mx = 1; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128; p.sfb_blocks = (N + 127) / 128;
+  p.mx = 1; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128;
+  p.sfb_blocks = (N + BN - 1) / BN * (BN / 128);
   if (launch_gemm(ta, tb, p, BN, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
   return DORY_OK;
 }

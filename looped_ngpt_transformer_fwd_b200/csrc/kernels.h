@@ -57,10 +57,12 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 // unit L2 norm.  bf16 sources come in up to 4 row segments (rows
 // [seg_rows[i], seg_rows[i+1]) from segs[i], seg_rows[0] = 0), or with
 // group > 0 as two matrices whose rows alternate in groups of `group`.
-size_t mxfp8_scale_bytes(int rows, int K);
+// Scale chunks cover the rows rounded up to `row_align` (128, or 256 for
+// weights read as 256-row tiles); the padding rows get scale code 127.
+size_t mxfp8_scale_bytes(int rows, int K, int row_align = 128);
 cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
-                                    int n_seg, int group, int rows, int K, int normalize,
-                                    float norm_eps, uint8_t* codes, uint8_t* scales,
+                                    int n_seg, int group, int rows, int row_align, int K,
+                                    int normalize, float norm_eps, uint8_t* codes, uint8_t* scales,
                                     cudaStream_t s);
 cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normalize, float norm_eps,
                                    uint8_t* codes, uint8_t* scales, cudaStream_t s);

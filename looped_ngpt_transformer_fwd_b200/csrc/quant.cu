@@ -13,8 +13,9 @@
 //          tcgen05.cp of a chunk (32 rows of 16 bytes, copied to every group of
 //          32 TMEM lanes) puts the scales of row r in column r / 32 of lane
 //          r % 32, byte q: the layout the block-scaled MMA reads.
-// Rows past `rows` (up to the next multiple of 128) get scale code 127 (1.0)
-// so that the MMA never multiplies the zero-filled padding by a NaN scale.
+// Rows past `rows` (up to the next multiple of 128, or of 256 for weights read
+// as 256-row tiles) get scale code 127 (1.0), so the MMA never multiplies the
+// zero-filled padding by an undefined scale.
 #include <cuda_fp8.h>
 #include <string.h>
 
@@ -140,12 +141,12 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
 }
 
 template <typename T>
-cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int K, int normalize, float norm_eps,
-                         uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K, int normalize,
+                         float norm_eps, uint8_t* codes, uint8_t* scales, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  if (K % 128 != 0) return cudaErrorInvalidValue;
-  const int row_blocks = (rows + 127) / 128;
-  const int rows_pad = row_blocks * 128;
+  if (K % 128 != 0 || (row_align != 128 && row_align != 256)) return cudaErrorInvalidValue;
+  const int rows_pad = (rows + row_align - 1) / row_align * row_align;
+  const int row_blocks = rows_pad / 128;
   quant_mxfp8_kernel<T><<<(rows_pad + kQuantWarps - 1) / kQuantWarps, 32 * kQuantWarps, 0, s>>>(
       src, rows, rows_pad, K, row_blocks, normalize, norm_eps, codes, scales);
   return cudaGetLastError();
@@ -153,13 +154,13 @@ cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int K, int normalize,
 
 }  // namespace
 
-size_t mxfp8_scale_bytes(int rows, int K) {
-  return static_cast<size_t>((rows + 127) / 128) * (K / 128) * 512;
+size_t mxfp8_scale_bytes(int rows, int K, int row_align) {
+  return static_cast<size_t>((rows + row_align - 1) / row_align * (row_align / 128)) * (K / 128) * 512;
 }
 
 cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
-                                    int n_seg, int group, int rows, int K, int normalize,
-                                    float norm_eps, uint8_t* codes, uint8_t* scales,
+                                    int n_seg, int group, int rows, int row_align, int K,
+                                    int normalize, float norm_eps, uint8_t* codes, uint8_t* scales,
                                     cudaStream_t s) {
   if (n_seg < 1 || n_seg > 4 || (group > 0 && n_seg != 2)) return cudaErrorInvalidValue;
   QuantSrc<__nv_bfloat16> q;
@@ -171,7 +172,7 @@ cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int*
   q.seg_row[n_seg] = rows;
   q.n_seg = n_seg;
   q.group = group;
-  return launch_quant(q, rows, K, normalize, norm_eps, codes, scales, s);
+  return launch_quant(q, rows, row_align, K, normalize, norm_eps, codes, scales, s);
 }
 
 cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normalize, float norm_eps,
@@ -181,7 +182,7 @@ cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normal
   q.seg[0] = src;
   q.seg_row[1] = rows;
   q.n_seg = 1;
-  return launch_quant(q, rows, K, normalize, norm_eps, codes, scales, s);
+  return launch_quant(q, rows, 128, K, normalize, norm_eps, codes, scales, s);
 }
 
 }  // namespace dory
