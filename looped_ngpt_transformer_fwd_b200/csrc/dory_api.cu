@@ -66,8 +66,8 @@ struct BlockW {
   CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
   // W_o / W_down for the fused projection + nGPT update (box rows = one MMA's N)
   CUtensorMap tm_o_n, tm_d_n;
-  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks; gate /
-  // up rows interleaved in groups of 128 as in the bf16 layout
+  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks (whole
+  // 256-row tiles); gate / up rows interleaved in groups of 64
   uint8_t *q8 = nullptr, *o8 = nullptr, *gu8 = nullptr, *d8 = nullptr;
   uint8_t *qsf = nullptr, *osf = nullptr, *gusf = nullptr, *dsf = nullptr;
   CUtensorMap tm8_qkvg, tm8_o, tm8_gu, tm8_d;                  // 128-row boxes (decode)
@@ -479,7 +479,12 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.norm_eps = m->cfg.norm_eps;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_QKVG);
-    DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_qkvg_256 : W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
+    // MXFP8: 128-column tiles keep two accumulators, so the QKVG epilogue
+    // overlaps the next tile's MMAs
+    if (m->mx)
+      DORY_TRY(launch_gemm(tmA, W.tm8_qkvg, g, 128, m->hd, m->num_sms, c.s));
+    else
+      DORY_TRY(launch_gemm(tmA, W.tm_qkvg[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   const KvLayerView view = kv_view(c.kv, b, loop);
@@ -600,8 +605,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   GemmParams g;
   DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
   if (m->mx) mx_weights(g, W.gusf, 2 * m->ff);
-  // gate and up rows alternate in groups of 128 (half a 256-column GEMM tile)
-  const int gu_group = 128;
+  // gate and up rows alternate in groups of half a GEMM tile: 128 (bf16,
+  // 256-column tiles), 64 (MXFP8, 128-column tiles with two accumulators, so
+  // the SwiGLU epilogue overlaps the next tile's MMAs)
+  const int gu_group = m->mx ? 64 : 128;
   if (c.decode) {
     g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
     g.epi = kEpiStoreF32;
@@ -621,7 +628,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
     g.out_act = c.w.a; g.ld_act = m->ff; g.gate_scale = m->cfg.gate_scale;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_GATEUP);
-    DORY_TRY(launch_gemm(tmA, m->mx ? W.tm8_gu_256 : W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
+    if (m->mx)
+      DORY_TRY(launch_gemm(tmA, W.tm8_gu, g, 128, m->hd, m->num_sms, c.s));
+    else
+      DORY_TRY(launch_gemm(tmA, W.tm_gu[1], g, 256, m->hd, m->num_sms, c.s));
   }
 
   CUtensorMap tmAct;
@@ -889,7 +899,7 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
       // MXFP8 weights quantised on the device from the bf16 sources (rows
       // quantised independently along K: the q | k | v | gate rows of the
       // fused projection keep their own scales; gate / up rows interleaved in
-      // groups of 128, half a 256-column tile)
+      // groups of 64, half a 128-column tile)
       W.q8 = base + L.off_q8;   W.qsf = base + L.off_qsf;
       W.o8 = base + L.off_o8;   W.osf = base + L.off_osf;
       W.gu8 = base + L.off_gu8; W.gusf = base + L.off_gusf;
@@ -908,7 +918,7 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
                                           W.qsf, s);
       e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), 256, int(da), 0, eps, W.o8,
                                           W.osf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 128, int(2 * F), 256, int(d), 0, eps,
+      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 64, int(2 * F), 256, int(d), 0, eps,
                                           W.gu8, W.gusf, s);
       e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), 256, int(F), 0, eps, W.d8,
                                           W.dsf, s);
