@@ -230,6 +230,50 @@ DORY_API void dory_kv_free(dory_kv* kv);
 DORY_API void dory_destroy(dory_model* m);
 
 /* ---------------------------------------------------------------------
+ * Tokens in and out.  The pages describe the stack between its first and
+ * last hidden states only ("Dory1.0-4B: A Looped Normalized-GPT", Overview:
+ * no vocabulary, no head); these follow the nGPT backbone the model card
+ * cites ("NVIDIA Nemotron Labs Dory 1.0 4B ...", Key ideas: every vector on
+ * the unit sphere).  The vocabulary size is the caller's (a multiple of 256).
+ * --------------------------------------------------------------------- */
+typedef struct dory_vocab dory_vocab;
+
+/* Bytes of the device buffer dory_vocab_create packs the tables into (0 for
+ * invalid arguments). */
+DORY_API size_t dory_vocab_bytes(const dory_config* cfg, int vocab);
+
+/* Input table emb_in [vocab, d_model] and output table emb_out [vocab,
+ * d_model] (bf16 bit patterns, rows expected unit-norm), per-token logit scale
+ * s_z [vocab] (fp32); host or device pointers, copied into `buf` (device,
+ * caller-owned, >= dory_vocab_bytes, 256-byte aligned) on `stream`. */
+DORY_API int dory_vocab_create(dory_model* m, int vocab, const uint16_t* emb_in,
+                               const uint16_t* emb_out, const float* logit_scale, void* buf,
+                               size_t bytes, void* stream, dory_vocab** out);
+
+/* h_out [n, d_model] bf16 (device) = Norm(emb_in[d_tokens[i]]): the unit-norm
+ * input rows of dory_prefill / dory_decode_step.  d_tokens: int32 device.  A
+ * token outside 0..vocab-1 gives a zero row and DORY_ERR_DEVICE_BOUNDS from
+ * dory_device_status. */
+DORY_API int dory_embed(dory_vocab* v, const int32_t* d_tokens, int n, void* h_out, void* stream);
+
+/* logits [n, vocab] fp32 (device) = s_z[v] * (emb_out[v] . h[i]) for rows h
+ * [n, d_model] bf16 (device), on the tensor-core GEMM. */
+DORY_API int dory_lm_head(dory_vocab* v, const void* h, int n, float* logits, void* stream);
+
+/* One token per row of logits [n, vocab] into d_tokens [n] (int32 device).
+ * temperature 0: argmax (the lowest index among equal maxima).  temperature
+ * > 0: the Gumbel-max draw argmax_v logits[v] / T - log(-log U_v), which
+ * samples softmax(logits / T), with U_v = (H(H(H(seed) ^ d_steps[i]) ^ v) +
+ * 0.5) / 2^32, H the lowbias32 hash (xorshift 16, * 0x7feb352d, xorshift 15,
+ * * 0x846ca68b, xorshift 16), evaluated in double precision; d_steps [n]
+ * (int32 device) is each row's step counter, so a draw is a pure function of
+ * (seed, step, row's logits). */
+DORY_API int dory_sample(dory_vocab* v, const float* logits, int n, float temperature,
+                         uint32_t seed, const int32_t* d_steps, int32_t* d_tokens, void* stream);
+
+DORY_API void dory_vocab_free(dory_vocab* v);
+
+/* ---------------------------------------------------------------------
  * Per-kernel timing (diagnostics).  While enabled, calls whose CUDA graph is
  * captured afterwards record a CUDA event before and after every kernel they
  * launch (graphs captured without it are kept separately and stay

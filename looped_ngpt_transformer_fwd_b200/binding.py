@@ -35,6 +35,8 @@ EXPORTS = (
     "dory_debug_mask_probe", "dory_debug_attention_paths", "dory_debug_wait_timeout",
     "dory_debug_fused_update", "dory_quant_mxfp8", "dory_mxfp8_scale_bytes",
     "dory_gemm_mxfp8_workspace_bytes", "dory_gemm_mxfp8",
+    "dory_vocab_bytes", "dory_vocab_create", "dory_embed", "dory_lm_head", "dory_sample",
+    "dory_vocab_free",
 )
 
 WEIGHT_FORMATS = {"bf16": 0, "mxfp8": 1}
@@ -116,6 +118,12 @@ def lib():
             "dory_mxfp8_scale_bytes": (SZ, [I, I]),
             "dory_gemm_mxfp8_workspace_bytes": (SZ, [I, I, I]),
             "dory_gemm_mxfp8": (I, [P, P, P, I, I, I, I, P, SZ, P]),
+            "dory_vocab_bytes": (SZ, [P, I]),
+            "dory_vocab_create": (I, [P, I, P, P, P, P, SZ, P, P]),
+            "dory_embed": (I, [P, P, I, P, P]),
+            "dory_lm_head": (I, [P, P, I, P, P]),
+            "dory_sample": (I, [P, P, I, ctypes.c_float, ctypes.c_uint32, P, P, P]),
+            "dory_vocab_free": (None, [P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -292,6 +300,34 @@ def dory_gemm_mxfp8_workspace_bytes(M, N, K):
 def dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream):
     return check(lib().dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream),
                  "dory_gemm_mxfp8")
+
+
+def dory_vocab_bytes(cfg_struct, vocab):
+    return lib().dory_vocab_bytes(ctypes.byref(cfg_struct), vocab)
+
+
+def dory_vocab_create(model, vocab, emb_in, emb_out, scale, buf, nbytes, stream):
+    out = ctypes.c_void_p()
+    check(lib().dory_vocab_create(model, vocab, emb_in, emb_out, scale, buf, nbytes, stream,
+                                  ctypes.byref(out)), "dory_vocab_create")
+    return out.value
+
+
+def dory_embed(vocab, tokens, n, h_out, stream):
+    return check(lib().dory_embed(vocab, tokens, n, h_out, stream), "dory_embed")
+
+
+def dory_lm_head(vocab, h, n, logits, stream):
+    return check(lib().dory_lm_head(vocab, h, n, logits, stream), "dory_lm_head")
+
+
+def dory_sample(vocab, logits, n, temperature, seed, steps, tokens, stream):
+    return check(lib().dory_sample(vocab, logits, n, temperature, seed, steps, tokens, stream),
+                 "dory_sample")
+
+
+def dory_vocab_free(vocab):
+    lib().dory_vocab_free(vocab)
 
 
 def dory_kv_free(kv):

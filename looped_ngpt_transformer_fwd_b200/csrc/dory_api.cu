@@ -1359,6 +1359,105 @@ int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, 
 
 }  // extern "C"
 
+// ================================================================ vocabulary
+struct dory_vocab {
+  dory_model* m = nullptr;
+  int vocab = 0;
+  __nv_bfloat16* emb_in = nullptr;
+  __nv_bfloat16* emb_out = nullptr;
+  float* scale = nullptr;
+  CUtensorMap tm_out;   // emb_out as the B operand, 256-row boxes
+};
+
+namespace {
+struct VocabLayout {
+  size_t in, out, scale, total;
+};
+VocabLayout vocab_layout(const dory_config* c, int vocab) {
+  VocabLayout L;
+  size_t o = 0;
+  L.in = o;    o = align_up(o + size_t(vocab) * c->d_model * 2);
+  L.out = o;   o = align_up(o + size_t(vocab) * c->d_model * 2);
+  L.scale = o; o = align_up(o + size_t(vocab) * 4);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+extern "C" {
+
+size_t dory_vocab_bytes(const dory_config* cfg, int vocab) {
+  if (validate_config(cfg) != DORY_OK || vocab <= 0 || vocab % 256) return 0;
+  return vocab_layout(cfg, vocab).total;
+}
+
+int dory_vocab_create(dory_model* m, int vocab, const uint16_t* emb_in, const uint16_t* emb_out,
+                      const float* logit_scale, void* buf, size_t bytes, void* stream,
+                      dory_vocab** out) {
+  if (!m || !emb_in || !emb_out || !logit_scale || !buf || !out || vocab <= 0 || vocab % 256)
+    return DORY_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!is_aligned(buf)) return DORY_ERR_MISALIGNED;
+  const VocabLayout L = vocab_layout(&m->cfg, vocab);
+  if (bytes < L.total) return DORY_ERR_BUFFER_TOO_SMALL;
+  std::unique_ptr<dory_vocab> v(new (std::nothrow) dory_vocab());
+  if (!v) return DORY_ERR_INVALID_ARG;
+  uint8_t* b = static_cast<uint8_t*>(buf);
+  v->m = m;
+  v->vocab = vocab;
+  v->emb_in = reinterpret_cast<__nv_bfloat16*>(b + L.in);
+  v->emb_out = reinterpret_cast<__nv_bfloat16*>(b + L.out);
+  v->scale = reinterpret_cast<float*>(b + L.scale);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tb = size_t(vocab) * m->d * 2;
+  if (cudaMemcpyAsync(v->emb_in, emb_in, tb, cudaMemcpyDefault, s) != cudaSuccess ||
+      cudaMemcpyAsync(v->emb_out, emb_out, tb, cudaMemcpyDefault, s) != cudaSuccess ||
+      cudaMemcpyAsync(v->scale, logit_scale, size_t(vocab) * 4, cudaMemcpyDefault, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  if (!make_tmap_bf16(&v->tm_out, v->emb_out, vocab, m->d, 256)) return DORY_ERR_CUDA;
+  *out = v.release();
+  return DORY_OK;
+}
+
+int dory_embed(dory_vocab* v, const int32_t* d_tokens, int n, void* h_out, void* stream) {
+  if (!v || !v->m || !d_tokens || !h_out || n <= 0) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(h_out, 16)) return DORY_ERR_MISALIGNED;
+  if (launch_embed(v->emb_in, v->vocab, v->m->d, d_tokens, n, static_cast<__nv_bfloat16*>(h_out),
+                   v->m->status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_lm_head(dory_vocab* v, const void* h, int n, float* logits, void* stream) {
+  if (!v || !v->m || !h || !logits || n <= 0) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(h, 16) || !is_aligned(logits, 16)) return DORY_ERR_MISALIGNED;
+  dory_model* m = v->m;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap ta;
+  if (!make_tmap_bf16(&ta, h, n, m->d, 128)) return DORY_ERR_CUDA;
+  GemmParams p;
+  p.M = n; p.N = v->vocab; p.K = m->d; p.epi = kEpiStoreF32; p.out_f32 = logits;
+  p.ld_out = v->vocab; p.status = m->status;
+  if (launch_gemm(ta, v->tm_out, p, 256, m->hd, m->num_sms, s) != cudaSuccess ||
+      launch_scale_columns(logits, v->scale, n, v->vocab, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_sample(dory_vocab* v, const float* logits, int n, float temperature, uint32_t seed,
+                const int32_t* d_steps, int32_t* d_tokens, void* stream) {
+  if (!v || !logits || !d_tokens || n <= 0 || !(temperature >= 0.f)) return DORY_ERR_INVALID_ARG;
+  if (temperature > 0.f && !d_steps) return DORY_ERR_INVALID_ARG;
+  if (launch_sample(logits, n, v->vocab, temperature, seed, d_steps, d_tokens,
+                    static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+void dory_vocab_free(dory_vocab* v) { delete v; }
+
+}  // extern "C"
+
 // ========================================================== allocation-free MLP
 // Scratch of dory_mlp_sublayer_noalloc, part of the library image: no call
 // ever allocates it.  Host code must not hand the symbol itself to a kernel;

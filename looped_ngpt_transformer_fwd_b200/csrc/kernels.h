@@ -243,6 +243,17 @@ bool decode_attention_tma_supported(int head_dim, int window, int group);
 int decode_attention_tma_splits(int max_pos, int window, int* split_tiles);
 cudaError_t launch_decode_attention_tma(const DecodeAttnParams& p, float m_log2, cudaStream_t s);
 
+// ----------------------------------------------------------------- vocabulary
+// Embedding rows Norm(table[token]) as bf16 [n, d] (a token outside 0..vocab-1
+// gives a zero row and kStatusBounds); logits z[r][v] *= scale[v]; one token
+// per row of logits [n, vocab] (greedy at temperature 0, else Gumbel-max from
+// the counter hash of (seed, steps[r], v)).
+cudaError_t launch_embed(const __nv_bfloat16* table, int vocab, int d, const int32_t* tokens,
+                         int n, __nv_bfloat16* out, uint32_t* status, cudaStream_t s);
+cudaError_t launch_scale_columns(float* z, const float* scale, int rows, int cols, cudaStream_t s);
+cudaError_t launch_sample(const float* logits, int n, int vocab, float temperature, uint32_t seed,
+                          const int32_t* steps, int32_t* tokens, cudaStream_t s);
+
 // ----------------------------------------------------------------- diagnostics
 // Set `n_records` mask-probe records to {INT_MAX, -1, 0, 0}.
 cudaError_t launch_probe_init(int32_t* probe, size_t n_records, cudaStream_t s);

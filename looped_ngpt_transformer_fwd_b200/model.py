@@ -61,6 +61,56 @@ class KVCache:
             pass
 
 
+class Vocab:
+    """Embedding and output tables bound to a model (dory_vocab_create)."""
+
+    def __init__(self, model, tables):
+        self.model = model
+        self.size = int(tables["logit_scale"].shape[0])
+        self.nbytes = B.dory_vocab_bytes(model.cfg_struct, self.size)
+        if self.nbytes == 0:
+            raise ValueError("vocabulary size must be a positive multiple of 256")
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=model.device)
+        staged = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16
+                                      else np.ascontiguousarray(v)).to(model.device)
+                  for k, v in tables.items()}
+        self.handle = B.dory_vocab_create(model.handle, self.size, _ptr(staged["emb_in"]),
+                                          _ptr(staged["emb_out"]), _ptr(staged["logit_scale"]),
+                                          _ptr(self.buf), self.nbytes, _stream(None))
+        torch.cuda.synchronize(model.device)
+
+    def embed(self, tokens, stream=None):
+        """int32 device tokens [n] -> unit-norm bf16 rows [n, d]."""
+        out = torch.empty(tokens.shape[0], self.model.cfg["d_model"], dtype=torch.bfloat16,
+                          device=self.model.device)
+        B.dory_embed(self.handle, _ptr(tokens), tokens.shape[0], _ptr(out), _stream(stream))
+        return out
+
+    def logits(self, h, stream=None):
+        """bf16 device rows [n, d] -> fp32 logits [n, V]."""
+        z = torch.empty(h.shape[0], self.size, dtype=torch.float32, device=self.model.device)
+        B.dory_lm_head(self.handle, _ptr(h), h.shape[0], _ptr(z), _stream(stream))
+        return z
+
+    def sample(self, z, temperature=0.0, seed=0, steps=None, stream=None):
+        """One int32 token per row of z (greedy at temperature 0)."""
+        tok = torch.empty(z.shape[0], dtype=torch.int32, device=self.model.device)
+        B.dory_sample(self.handle, _ptr(z), z.shape[0], float(temperature), int(seed),
+                      _ptr(steps) if steps is not None else None, _ptr(tok), _stream(stream))
+        return tok
+
+    def free(self):
+        if getattr(self, "handle", None):
+            B.dory_vocab_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
 class DoryModel:
     """Packed weights on the device plus a library handle.
 
@@ -104,6 +154,10 @@ class DoryModel:
     # ---------------------------------------------------------------- buffers
     def kv_cache(self, mode, max_seqs, max_ctx, k_max=1):
         return KVCache(self, mode, max_seqs, max_ctx, k_max)
+
+    def vocab(self, tables):
+        """Bind embedding / output tables (dict: emb_in, emb_out, logit_scale)."""
+        return Vocab(self, tables)
 
     def workspace(self, max_tokens):
         if self._ws is None or self._ws_tokens < max_tokens:

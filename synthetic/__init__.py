@@ -10,4 +10,4 @@ counter-based hash on the GPU for the multi-GB decode caches.
 
 from .config import load_config, CONFIG_DIR  # noqa: F401
 from .bf16 import f32_to_bf16_bits, bf16_bits_to_f32, round_bf16  # noqa: F401
-from .weights import block_weights, hidden_in  # noqa: F401
+from .weights import block_weights, hidden_in, vocab_weights  # noqa: F401

@@ -28,6 +28,7 @@ _TENSOR_IDS = {
     "wq": 1, "wk": 2, "wv": 3, "wg": 4, "wo": 5,
     "w_gate": 6, "w_up": 7, "w_down": 8,
     "alpha_attn": 9, "alpha_mlp": 10, "s_qk": 11,
+    "emb_in": 12, "emb_out": 13, "logit_scale": 14,
 }
 MATRICES = ("wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down")
 VECTORS = ("alpha_attn", "alpha_mlp", "s_qk")
@@ -118,3 +119,16 @@ def hidden_in(cfg, seed, n, row0=0):
     allrows = np.concatenate(parts, axis=0)
     off = row0 - c0 * _ROW_CHUNK
     return np.ascontiguousarray(allrows[off:off + n])
+
+
+def vocab_weights(cfg, seed, vocab=None):
+    """Token embedding tables around the stack (the vocabulary size is not on the
+    pages: `vocab_size` of the config): emb_in, emb_out [V, d] as bf16 bits with
+    N(0, weight_std) rows scaled to unit norm (as the block matrices), and
+    logit_scale [V] float32 drawn U(10, 20)."""
+    V = int(vocab or cfg["vocab_size"])
+    d = cfg["d_model"]
+    out = {name: _matrix(seed, 0xE0, name, (V, d), cfg["weight_std"])
+           for name in ("emb_in", "emb_out")}
+    out["logit_scale"] = _rng(seed, 0xE0, _TENSOR_IDS["logit_scale"]).uniform(10.0, 20.0, V).astype(np.float32)
+    return out
