@@ -33,16 +33,12 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
-// The three row norms of the update come from one pass of per-element terms
-// (u = y / ||y||, a = alpha):
-//   ||y||^2              = D  = sum y^2
-//   ||h + a (u - h)||^2  = P1 + 2 P2 / ||y|| + P3 / ||y||^2,
-//        P1 = sum ((1-a) h)^2, P2 = sum (1-a) h a y, P3 = sum (a y)^2
-//   ||h_new + e||^2      = ||h'||^2 / ||h'||^2 + 2 (Q1 + Q2 / ||y||) / ||h'|| + Q3,
-//        Q1 = sum (1-a) h e, Q2 = sum a y e, Q3 = sum e^2
-// so the CTA needs a single block reduction (of 4 or 7 sums) per row.
+// Three block reductions per row (||y||, ||h'||, ||h_new + e||), with y and h
+// held in registers between them.  A variant that derives all three norms from
+// one pass of seven per-row sums (one barrier) measured slower on B200: it
+// needs more live registers, which cost more occupancy than the barriers do.
 __global__ void row_update_kernel(const RowUpdateParams p) {
-  __shared__ float red[32][8];
+  __shared__ float red[32];
   const int r = blockIdx.x;
   // one CTA per row: these exits are uniform across the block
   if (p.row_k) {
@@ -53,86 +49,73 @@ __global__ void row_update_kernel(const RowUpdateParams p) {
     }
     if (p.loop > kr) return;        // this row's loops are done
   }
-  const bool reinject = p.e != nullptr && (!p.row_k || p.loop < p.row_k[r]);
-  // re-injecting the row just saved as e gives Norm(2 h_new) = h_new
-  const bool use_e = reinject && p.e != p.e_save;
+  // re-injecting the row just saved as e would give Norm(2 h_new) = h_new
+  const bool reinject =
+      p.e != nullptr && p.e != p.e_save && (!p.row_k || p.loop < p.row_k[r]);
   const int nch = p.d >> 2;
   const size_t row_off = static_cast<size_t>(r) * p.d;
-  float4 y[kRowMaxChunks], h[kRowMaxChunks], a[kRowMaxChunks], e[kRowMaxChunks];
-  float sums[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // D, P1, P2, P3, Q1, Q2, Q3
+  float4 y[kRowMaxChunks], h[kRowMaxChunks];
+  float ss = 0.f;
 #pragma unroll
   for (int j = 0; j < kRowMaxChunks; ++j) {
     const int c = threadIdx.x + j * blockDim.x;
     y[j] = make_float4(0.f, 0.f, 0.f, 0.f);
     h[j] = y[j];
-    a[j] = y[j];
-    e[j] = y[j];
     if (c < nch) {
       for (int s = 0; s < p.splits; ++s) {
         const float4 t = reinterpret_cast<const float4*>(p.y + s * p.split_stride + row_off)[c];
         y[j].x += t.x; y[j].y += t.y; y[j].z += t.z; y[j].w += t.w;
       }
       h[j] = reinterpret_cast<const float4*>(p.h + row_off)[c];
-      a[j] = reinterpret_cast<const float4*>(p.alpha)[c];
-      if (use_e) e[j] = reinterpret_cast<const float4*>(p.e + row_off)[c];
-    }
-    const float yv[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
-    const float hv[4] = {h[j].x, h[j].y, h[j].z, h[j].w};
-    const float av[4] = {a[j].x, a[j].y, a[j].z, a[j].w};
-    const float ev[4] = {e[j].x, e[j].y, e[j].z, e[j].w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float hk = (1.f - av[u]) * hv[u], ay = av[u] * yv[u];
-      sums[0] = fmaf(yv[u], yv[u], sums[0]);
-      sums[1] = fmaf(hk, hk, sums[1]);
-      sums[2] = fmaf(hk, ay, sums[2]);
-      sums[3] = fmaf(ay, ay, sums[3]);
-      sums[4] = fmaf(hk, ev[u], sums[4]);
-      sums[5] = fmaf(ay, ev[u], sums[5]);
-      sums[6] = fmaf(ev[u], ev[u], sums[6]);
+      ss += dot4(y[j], y[j]);
     }
   }
-  // one block reduction of the 7 sums (warp shuffles, one barrier)
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int nw = (blockDim.x + 31) >> 5;
+  const float inv_y = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+  ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < 7; ++i) {
-    const float v = warp_sum(sums[i]);
-    if (l == 0) red[w][i] = v;
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    if (c < nch) {
+      const float4 a = reinterpret_cast<const float4*>(p.alpha)[c];
+      h[j].x += a.x * (y[j].x * inv_y - h[j].x);
+      h[j].y += a.y * (y[j].y * inv_y - h[j].y);
+      h[j].z += a.z * (y[j].z * inv_y - h[j].z);
+      h[j].w += a.w * (y[j].w * inv_y - h[j].w);
+      ss += dot4(h[j], h[j]);
+    }
   }
-  __syncthreads();
+  const float inv_h = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+  ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < 7; ++i) {
-    float t = 0.f;
-    for (int k = 0; k < nw; ++k) t += red[k][i];
-    sums[i] = t;
+  for (int j = 0; j < kRowMaxChunks; ++j) {
+    const int c = threadIdx.x + j * blockDim.x;
+    if (c < nch) {
+      h[j].x *= inv_h; h[j].y *= inv_h; h[j].z *= inv_h; h[j].w *= inv_h;
+      if (p.e_save) reinterpret_cast<float4*>(p.e_save + row_off)[c] = h[j];
+      if (reinject) {
+        const float4 e = reinterpret_cast<const float4*>(p.e + row_off)[c];
+        h[j].x += e.x; h[j].y += e.y; h[j].z += e.z; h[j].w += e.w;
+        ss += dot4(h[j], h[j]);
+      }
+    }
   }
-  const float inv_y = rsqrtf(fmaxf(sums[0], p.norm_eps));
-  const float hp2 = sums[1] + 2.f * sums[2] * inv_y + sums[3] * inv_y * inv_y;   // ||h'||^2
-  const float inv_h = rsqrtf(fmaxf(hp2, p.norm_eps));
-  float inv_x = 1.f;
-  if (use_e) {
-    const float x2 = hp2 * inv_h * inv_h + 2.f * (sums[4] + sums[5] * inv_y) * inv_h + sums[6];
-    inv_x = rsqrtf(fmaxf(x2, p.norm_eps));
+  if (reinject) {
+    // block_sum is reached by every thread (reinject is uniform)
+    const float inv_x = rsqrtf(fmaxf(block_sum(ss, red), p.norm_eps));
+#pragma unroll
+    for (int j = 0; j < kRowMaxChunks; ++j) {
+      h[j].x *= inv_x; h[j].y *= inv_x; h[j].z *= inv_x; h[j].w *= inv_x;
+    }
   }
 #pragma unroll
   for (int j = 0; j < kRowMaxChunks; ++j) {
     const int c = threadIdx.x + j * blockDim.x;
-    if (c >= nch) continue;
-    float4 o;
-    o.x = (h[j].x + a[j].x * (y[j].x * inv_y - h[j].x)) * inv_h;
-    o.y = (h[j].y + a[j].y * (y[j].y * inv_y - h[j].y)) * inv_h;
-    o.z = (h[j].z + a[j].z * (y[j].z * inv_y - h[j].z)) * inv_h;
-    o.w = (h[j].w + a[j].w * (y[j].w * inv_y - h[j].w)) * inv_h;
-    if (p.e_save) reinterpret_cast<float4*>(p.e_save + row_off)[c] = o;
-    if (use_e) {
-      o.x = (o.x + e[j].x) * inv_x; o.y = (o.y + e[j].y) * inv_x;
-      o.z = (o.z + e[j].z) * inv_x; o.w = (o.w + e[j].w) * inv_x;
+    if (c < nch) {
+      reinterpret_cast<float4*>(p.h + row_off)[c] = h[j];
+      const uint2 b = make_uint2(pack_bf16x2(h[j].x, h[j].y), pack_bf16x2(h[j].z, h[j].w));
+      if (p.hb) reinterpret_cast<uint2*>(p.hb + row_off)[c] = b;
+      if (p.out) reinterpret_cast<uint2*>(p.out + row_off)[c] = b;
     }
-    reinterpret_cast<float4*>(p.h + row_off)[c] = o;
-    const uint2 b = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
-    if (p.hb) reinterpret_cast<uint2*>(p.hb + row_off)[c] = b;
-    if (p.out) reinterpret_cast<uint2*>(p.out + row_off)[c] = b;
   }
 }
 
