@@ -18,7 +18,17 @@ reading is the public definition of each format:
 * NVFP4: blocks of 16 share an E4M3 scale and the whole tensor one fp32 scale
   g = amax / (6 * 448); elements are FP4 E2M1 (exponent bias 1, 1 mantissa
   bit, largest 6).  Block scale s = E4M3(amax_block / (6 g)); elements
-  E2M1(x / (s g)), nearest even, saturating at 6.
+  E2M1(x / (s g)), nearest even, saturating at 6.  "The whole tensor" is read
+  as the weight one projection GEMM reads: the matrices the forward pass
+  multiplies with the same input in one product (q, k, v and the output-gate
+  rows; the SwiGLU gate and up rows) share one g, the maximum over the group
+  (NVFP4_GROUPS), as the released NVFP4 format does for fused projections.
+  Serving is read like MXFP8's: both operands of every projection in NVFP4.
+  A projection input's tensor scale is fixed at g = 1 / (6 * 448): its rows
+  are unit vectors (the stream, and the attention output and SwiGLU
+  activations after their norm), so no element exceeds 1 and every block
+  scale stays within E4M3's range (NVFP4_ACT_G); a static input scale is what
+  the format's checkpoints carry for activations.
 
 Dequantisation multiplies back; a quantised GEMM is C = A @ W_hat^T with W_hat
 the dequantised weights, in float64.  Serving an MXFP8 checkpoint ("standard
@@ -127,15 +137,25 @@ def mxfp8_dequantize(codes, scales):
 NV_BLOCK = 16
 
 
-def nvfp4_quantize(w):
+NVFP4_ACT_G = np.float32(1.0 / (6.0 * 448.0))
+NVFP4_GROUPS = (("wq", "wk", "wv", "wg"), ("wo",), ("w_gate", "w_up"), ("w_down",))
+
+
+def nvfp4_tensor_scale(*mats):
+    """g = amax / (6 * 448) over all elements of the matrices (the quotient in
+    float64, then rounded to float32); 1 when every element is zero."""
+    amax = max(float(np.abs(np.asarray(m, dtype=np.float64)).max()) for m in mats)
+    return np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+
+
+def nvfp4_quantize(w, g=None):
     """w [N, K] (K a multiple of 16) -> (element codes [N, K] uint8 holding
     E2M1 codes in the low nibble, block scale codes [N, K/16] uint8 E4M3,
-    tensor scale g as float32)."""
+    tensor scale g as float32).  g None: the tensor's own (nvfp4_tensor_scale)."""
     w = np.asarray(w, dtype=np.float64)
     n, k = w.shape
     assert k % NV_BLOCK == 0
-    amax = np.abs(w).max()
-    g = np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+    g = nvfp4_tensor_scale(w) if g is None else np.float32(g)
     blocks = w.reshape(n, k // NV_BLOCK, NV_BLOCK)
     bmax = np.abs(blocks).max(axis=2)
     s = round_to_format(bmax / (6.0 * float(g)), E4M3)
@@ -149,6 +169,20 @@ def nvfp4_dequantize(codes, scales, g):
     n, k = codes.shape
     v = decode(codes, E2M1).reshape(n, k // NV_BLOCK, NV_BLOCK)
     return (v * decode(scales, E4M3)[:, :, None] * float(g)).reshape(n, k)
+
+
+def nvfp4_fake_quant(x, g=NVFP4_ACT_G):
+    """x [..., K] (K a multiple of 16) -> the values an NVFP4 encoding of x
+    under tensor scale g holds (blocks of 16 along the last axis)."""
+    x = np.asarray(x, dtype=np.float64)
+    flat = x.reshape(-1, x.shape[-1])
+    return nvfp4_dequantize(*nvfp4_quantize(flat, g)).reshape(x.shape)
+
+
+def nvfp4_gemm(a, w, g_a=NVFP4_ACT_G, g_w=None):
+    """Both operands in NVFP4 along K, products summed in float64:
+    C = Q(A; g_a) Q(W; g_w)^T (g_w None: W's own tensor scale)."""
+    return nvfp4_fake_quant(a, g_a) @ nvfp4_dequantize(*nvfp4_quantize(w, g_w)).T
 
 
 def mxfp8_fake_quant(x):
@@ -181,23 +215,29 @@ def dequantized_provider(provider, fmt):
     """Wrap a weight provider (block -> dict) so that every matrix [out, in] is
     replaced by its quantise -> dequantise version in `fmt` ("mxfp8" or
     "nvfp4"), blocks running along `in` (the GEMM reduction axis); the vectors
-    (alpha, s_qk) are left as they are."""
+    (alpha, s_qk) are left as they are.  NVFP4 matrices of one NVFP4_GROUPS
+    entry share the group's tensor scale."""
     from synthetic.bf16 import bf16_bits_to_f32
+    if fmt not in ("mxfp8", "nvfp4"):
+        raise ValueError(fmt)
     memo = {}
 
     def provide(b):
         if b not in memo:
             w = dict(provider(b))
+            mats = {}
             for n in MATRIX_NAMES:
                 m = w[n]
-                m = bf16_bits_to_f32(m).astype(np.float64) if m.dtype == np.uint16 else \
+                mats[n] = bf16_bits_to_f32(m).astype(np.float64) if m.dtype == np.uint16 else \
                     np.asarray(m, dtype=np.float64)
-                if fmt == "mxfp8":
-                    w[n] = mxfp8_dequantize(*mxfp8_quantize(m))
-                elif fmt == "nvfp4":
-                    w[n] = nvfp4_dequantize(*nvfp4_quantize(m))
-                else:
-                    raise ValueError(fmt)
+            if fmt == "mxfp8":
+                for n in MATRIX_NAMES:
+                    w[n] = mxfp8_dequantize(*mxfp8_quantize(mats[n]))
+            else:
+                for group in NVFP4_GROUPS:
+                    g = nvfp4_tensor_scale(*(mats[n] for n in group))
+                    for n in group:
+                        w[n] = nvfp4_dequantize(*nvfp4_quantize(mats[n], g))
             memo[b] = w
         return memo[b]
     return provide

@@ -262,3 +262,118 @@ def test_activation_quantised_stack():
     assert cos.min() > 0.999
     assert np.allclose(np.linalg.norm(both, axis=1), 1.0, atol=1e-9)
     assert np.abs(both - wonly).max() > 1e-5
+
+
+def _nvfp4_brute(x, g):
+    """NVFP4 values of x [K] (K a multiple of 16) under tensor scale g by
+    exhaustive search: each block's scale is the nearest E4M3 value to
+    amax / (6 g), each element the nearest E2M1 value to x / (s g), times s g."""
+    out = []
+    for blk in np.asarray(x, dtype=np.float64).reshape(-1, 16):
+        s = _nearest_even([np.abs(blk).max() / (6.0 * float(g))], Q.E4M3)[0]
+        unit = s * float(g)
+        if unit == 0:
+            out.append(np.zeros(16))
+            continue
+        out.append(_nearest_even(blk / unit, Q.E2M1) * unit)
+    return np.concatenate(out)
+
+
+def test_nvfp4_given_tensor_scale_matches_brute_force():
+    """With the tensor scale given (as for the projection inputs), every block
+    scale and element is the exhaustive nearest value; unit-norm rows under
+    NVFP4_ACT_G = 1 / (6 * 448) never need a block scale above 448."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((3, 64))
+    x[1] *= np.exp2(rng.integers(-8, 0, 64))          # mixed magnitudes, tiny blocks
+    x[2, :16] = 0.0                                   # an all-zero block
+    x /= np.linalg.norm(x, axis=1, keepdims=True)
+    codes, scales, g = Q.nvfp4_quantize(x, Q.NVFP4_ACT_G)
+    assert g == Q.NVFP4_ACT_G
+    assert Q.decode(scales, Q.E4M3).max() <= 448
+    got = Q.nvfp4_dequantize(codes, scales, g)
+    for i in range(3):
+        assert np.array_equal(got[i], _nvfp4_brute(x[i], g))
+    assert np.array_equal(Q.nvfp4_fake_quant(x), got)
+    assert np.all(codes[2, :16] == 0) and np.all(scales[2, 0] == 0)
+
+
+def test_nvfp4_exact_ties_round_to_even():
+    """Values exactly halfway between two E2M1 grid points (t s g with t a
+    midpoint, all exact in float64) go to the even code: 0.25 -> 0, 0.75 -> 1,
+    1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4 (times s g)."""
+    g = np.float32(2.0 ** -12)
+    s = 1.5
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    want = np.array([0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0])
+    blk = np.concatenate([[6.0], mids, -mids, [0.0]]) * s * float(g)   # amax / (6 g) = s exactly
+    codes, scales, _ = Q.nvfp4_quantize(blk[None, :], g)
+    assert Q.decode(scales, Q.E4M3)[0, 0] == s
+    vals = Q.decode(codes, Q.E2M1)[0]
+    assert np.array_equal(vals[1:8], want) and np.array_equal(vals[8:15], -want)
+    assert vals[0] == 6.0
+
+
+def test_nvfp4_group_shares_the_largest_tensor_scale():
+    """Matrices of one GEMM share one g: the block holding the group's largest
+    value gets scale 448, and no block of a matrix whose values are at most half
+    the group's maximum comes near it (with a per-matrix g every matrix would
+    have a 448 block)."""
+    from oracle.quant import dequantized_provider, NVFP4_GROUPS
+    rng = np.random.default_rng(22)
+    names = [n for grp in NVFP4_GROUPS for n in grp]
+    base = {n: rng.standard_normal((32, 64)) for n in names}
+    for n, top_val in (("wq", 0.02), ("wg", 0.018), ("wk", 0.01), ("wv", 0.005)):
+        base[n] *= top_val / np.abs(base[n]).max()      # the group's maxima: 1, 0.9, 0.5, 0.25
+    prov = lambda b: base
+    deq = dequantized_provider(prov, "nvfp4")(0)
+    g = Q.nvfp4_tensor_scale(base["wq"], base["wk"], base["wv"], base["wg"])
+    assert g == Q.nvfp4_tensor_scale(np.concatenate([base[n] for n in ("wq", "wk", "wv", "wg")]))
+    for n in ("wq", "wk", "wv", "wg"):
+        c, sc, _ = Q.nvfp4_quantize(base[n], g)
+        assert np.array_equal(deq[n], Q.nvfp4_dequantize(c, sc, g))
+    assert Q.decode(Q.nvfp4_quantize(base["wq"], g)[1], Q.E4M3).max() == 448
+    assert Q.decode(Q.nvfp4_quantize(base["wg"], g)[1], Q.E4M3).max() < 448
+    for n in ("wk", "wv"):
+        assert Q.decode(Q.nvfp4_quantize(base[n], g)[1], Q.E4M3).max() <= 240
+
+
+def test_nvfp4_gemm_brute_force():
+    """Both operands quantised along K under their tensor scales, then an exact
+    product: a brute-force sum over decoded codes times block and tensor
+    scales."""
+    rng = np.random.default_rng(23)
+    a = rng.standard_normal((3, 32))
+    a /= np.linalg.norm(a, axis=1, keepdims=True)
+    w = rng.standard_normal((4, 32)) * 0.05
+    ca, sa, ga = Q.nvfp4_quantize(a, Q.NVFP4_ACT_G)
+    cw, sw, gw = Q.nvfp4_quantize(w)
+    va, vw = Q.decode(ca, Q.E2M1), Q.decode(cw, Q.E2M1)
+    fa, fw = Q.decode(sa, Q.E4M3), Q.decode(sw, Q.E4M3)
+    brute = np.array([[sum(va[i, t] * fa[i, t // 16] * float(ga) * vw[j, t] * fw[j, t // 16] *
+                           float(gw) for t in range(32)) for j in range(4)] for i in range(3)])
+    assert np.allclose(Q.nvfp4_gemm(a, w), brute, rtol=1e-13, atol=1e-16)
+    exact = a @ w.T
+    assert np.abs(Q.nvfp4_gemm(a, w) - exact).max() < 0.3 * np.abs(exact).max()
+
+
+def test_nvfp4_activation_quantised_stack():
+    """NVFP4 weights and NVFP4 projection inputs: the tiny stack stays on the
+    sphere and near the bf16 stack, further from it than with MXFP8 (1 mantissa
+    bit against 3)."""
+    from oracle import Oracle, KVCache, weights_from_generator
+    from oracle.quant import dequantized_provider, mxfp8_fake_quant, nvfp4_fake_quant
+    from synthetic import load_config, hidden_in
+    from synthetic.bf16 import bf16_bits_to_f32
+    cfg = load_config("tiny")
+    prov = weights_from_generator(cfg, 11)
+    h = bf16_bits_to_f32(hidden_in(cfg, 12, 48)).astype(np.float64)
+    run = lambda p, aq=None: Oracle(cfg, p, act_quant=aq).forward(
+        h, 0, 2, KVCache(cfg, "last_loop", k_max=2))
+    ref = run(prov)
+    nv = run(dequantized_provider(prov, "nvfp4"), nvfp4_fake_quant)
+    mx = run(dequantized_provider(prov, "mxfp8"), mxfp8_fake_quant)
+    cos = lambda u: ((u * ref).sum(1) / np.linalg.norm(u, axis=1) / np.linalg.norm(ref, axis=1)).min()
+    assert cos(nv) > 0.98
+    assert np.allclose(np.linalg.norm(nv, axis=1), 1.0, atol=1e-9)
+    assert cos(mx) > cos(nv)
