@@ -14,6 +14,9 @@ SWA:full 3:1 with window 4096, bf16 weights and activations):
   decode_k2    64 sequences x 32768 cached positions, last-loop cache, k = 2
   decode_k4_last / decode_k4_per   32 / 8 sequences x 131072 positions, k = 4
   prefill_long 262144 tokens in 8192-token chunks, k = 4, last-loop cache
+  prefill_k2_mxfp8 / decode_k2_mxfp8, prefill_k2_nvfp4 / decode_k2_nvfp4
+               the prefill_k2 / decode_k2 shapes with MXFP8 or NVFP4 weights and
+               projection inputs (block-scaled tensor-core GEMMs)
 
 N > 1 runs N independent replicas (one per GPU, no collective on the data
 path; the harness only uses a barrier and a max-reduction of the timings).
@@ -49,6 +52,11 @@ WORKLOADS = {
                              fmt="mxfp8"),
     "decode_k2_mxfp8": dict(kind="decode", batch=64, ctx=32768, k=2, mode="last_loop", seed=2,
                             fmt="mxfp8"),
+    # the released NVFP4 checkpoint format: NVFP4 weights and projection inputs
+    "prefill_k2_nvfp4": dict(kind="prefill", tokens=4096, k=2, mode="last_loop", seed=1,
+                             fmt="nvfp4"),
+    "decode_k2_nvfp4": dict(kind="decode", batch=64, ctx=32768, k=2, mode="last_loop", seed=2,
+                            fmt="nvfp4"),
 }
 
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
@@ -496,7 +504,9 @@ def oracle_sample(wl, prov=None, n_blocks=4):
 
 # ----------------------------------------------------------------- roofline
 DATASHEET = {"tensor": 2250.0, "hbm": 8000.0}    # dense bf16 TFLOP/s, HBM3e GB/s (context only)
-DATASHEET_FP8 = 4500.0
+DATASHEET_LOWP = {"mxfp8": 4500.0, "nvfp4": 9000.0}   # dense fp8 / fp4 TFLOP/s (context only)
+# nominal ratio of a low-precision contraction's peak to bf16's (4.5 / 2.25, 9 / 2.25)
+LOWP_RATIO = {"mxfp8": 2.0, "nvfp4": 4.0}
 
 
 def roofline(res, wl, peaks, peak_src):
@@ -509,9 +519,10 @@ def roofline(res, wl, peaks, peak_src):
             achieved = dom_work / (dom_ms / dom_n / 1e3) / 1e12   # dom_work is per launch
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit, key = "TFLOP/s", "bf16_tflops_sustained"
-        if wl.get("fmt") == "mxfp8":
-            # fp8 contraction: the bf16 figure times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-            peak, key = 2.0 * peak, "bf16_tflops_sustained x 2 (fp8)"
+        fmt = wl.get("fmt")
+        if fmt in LOWP_RATIO:
+            # fp8 / fp4 contraction: the bf16 figure times the nominal ratio of the peaks
+            peak, key = LOWP_RATIO[fmt] * peak, f"bf16_tflops_sustained x {LOWP_RATIO[fmt]:g} ({fmt})"
         per_launch = dom_work if wl["kind"] != "prefill_chunked" else dom_work / max(dom_n, 1)
         traffic = profiled_traffic(dom_name)
     else:
@@ -523,7 +534,8 @@ def roofline(res, wl, peaks, peak_src):
     return {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": (achieved / peak) if achieved else None,
             "peak_source": f"{peak_src} ({key})",
-            "frac_of_datasheet": (achieved / (DATASHEET_FP8 if (bound == "tensor" and wl.get("fmt") == "mxfp8")
+            "frac_of_datasheet": (achieved / (DATASHEET_LOWP[wl["fmt"]]
+                                              if (bound == "tensor" and wl.get("fmt") in DATASHEET_LOWP)
                                               else DATASHEET[bound])) if achieved else None,
             "traffic": traffic, "work_per_launch": per_launch, "launches_per_step": dom_n,
             "device_ms_per_step": dom_ms}
@@ -540,7 +552,11 @@ def footprint_check(cfg, wl):
 
 
 DEFAULT_EXTRAS = ["prefill_k1", "decode_k2", "decode_k4_last", "decode_k4_per",
-                  "prefill_k2_mxfp8", "decode_k2_mxfp8"]
+                  "prefill_k2_mxfp8", "decode_k2_mxfp8", "prefill_k2_nvfp4", "decode_k2_nvfp4"]
+DTYPES = {"bf16": "bf16",
+          "mxfp8": "mxfp8 (E4M3 x E4M3, E8M0 block scales, fp32 accumulation)",
+          "nvfp4": "nvfp4 (E2M1 x E2M1, E4M3 block scales of 16, fp32 tensor scales, "
+                   "fp32 accumulation)"}
 
 
 # ----------------------------------------------------------------- main
@@ -635,8 +651,7 @@ def main():
                  "kernel_ms_per_step": {kk: round(v[0], 4) for kk, v in r["kernel_ms"].items()},
                  "gpu_launches": r["launches"] * xsteps, "clocks": r["clocks"],
                  "weights_seed": WORKLOADS[args.workload]["seed"],
-                 "dtype": "mxfp8 (E4M3 x E4M3, E8M0 block scales, fp32 accumulation)"
-                 if fmt == "mxfp8" else "bf16"}
+                 "dtype": DTYPES[fmt]}
         entry.update({kk: vv for kk, vv in r["extra"].items() if kk not in ("k", "kv_mode")})
         entry["k"], entry["kv_mode"] = xwl["k"], xwl["mode"]
         if xwl["kind"] == "decode":
@@ -652,7 +667,7 @@ def main():
             "metric": f"{'prefill' if 'prefill' in wl['kind'] else 'decode'} tokens/s",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPES[wl.get("fmt", "bf16")],
             "data": "synthetic (seeded unit-norm inputs, seeded random 4B-class weights)",
             "config": dict({"workload": res["workload"] + (f" blocks={args.blocks}" if args.blocks else ""),
                             "parallelism": f"replicas x{world}",

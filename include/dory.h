@@ -69,7 +69,8 @@ typedef enum dory_status {
 
 typedef enum dory_weight_format {
   DORY_WEIGHTS_BF16 = 0,  /* bf16 weights, bf16 projection inputs                   */
-  DORY_WEIGHTS_MXFP8 = 1  /* MXFP8 weights and projection inputs (see dory_config)  */
+  DORY_WEIGHTS_MXFP8 = 1, /* MXFP8 weights and projection inputs (see dory_config)  */
+  DORY_WEIGHTS_NVFP4 = 2  /* NVFP4 weights and projection inputs (see dory_config)  */
 } dory_weight_format;
 
 typedef enum dory_kv_mode {
@@ -110,7 +111,19 @@ typedef struct dory_config {
    * must then be device pointers, 16-byte aligned); every projection input is
    * quantised on the fly (the attention output and the SwiGLU activations
    * after their L2 norm), and the products run on the block-scaled tensor
-   * cores (tcgen05.mma kind::mxf8f6f4). */
+   * cores (tcgen05.mma kind::mxf8f6f4).
+   * DORY_WEIGHTS_NVFP4: the released NVFP4 checkpoint format (same page, Key
+   * Contributions item 4; Main Findings: NVFP4 after quantisation-aware
+   * distillation), served as both operands of every projection in NVFP4:
+   * blocks of 16 values along the reduction axis share an E4M3 scale
+   * E4M3(amax_block / (6 g)) and hold E2M1 elements (nearest, ties to even,
+   * saturating at 6) under a per-tensor fp32 scale g.  The weights' g is
+   * amax / (6 * 448) over the matrices one GEMM reads together (q, k, v and
+   * the gate rows; gate and up; W_o; W_down), computed by dory_create; every
+   * projection input takes g = 1 / (6 * 448), since its rows are unit vectors
+   * (no element above 1).  Products run on tcgen05.mma kind::mxf4nvf4 with the
+   * two tensor scales applied in the epilogue.  Needs d_model and d_ff
+   * multiples of 256; sources as for MXFP8. */
   int32_t weight_format;
 } dory_config;
 
@@ -335,6 +348,31 @@ DORY_API size_t dory_gemm_mxfp8_workspace_bytes(int M, int N, int K);
 DORY_API int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K,
                              int k_splits, void* ws, size_t ws_bytes, void* stream);
 
+/* NVFP4 quantisation along K of bf16 rows src [rows, K] (device, K a multiple
+ * of 256) under the tensor scale g: g > 0 as given, else g = amax / (6 * 448)
+ * of src computed on the device and written to d_g (a device float, also used
+ * as scratch).  Packed E2M1 codes [rows, K / 2] bytes into `codes` (element 2i
+ * in the low nibble of byte i), E4M3 block scale codes into `scales`
+ * (dory_nvfp4_scale_bytes) in 2048-byte chunks, one per 128 rows x 256 K:
+ * chunk (kc, rb) at (kc * ceil(rows/128) + rb) * 2048, the scale of row
+ * rb*128 + 32*j + i and 16-block b (0..15) of the chunk at byte
+ * (b / 4) * 512 + i*16 + j*4 + b % 4; padding rows of the last chunk hold
+ * 0x38 (1.0).  Same rule as weight_format DORY_WEIGHTS_NVFP4. */
+DORY_API int dory_quant_nvfp4(const void* src, int rows, int K, float g, float* d_g, void* codes,
+                              void* scales, void* stream);
+DORY_API size_t dory_nvfp4_scale_bytes(int rows, int K);
+
+/* The block-scaled (NVFP4 x NVFP4) tensor-core GEMM alone: quantises A [M,K]
+ * under tensor scale g_a and B [N,K] under g_b (bf16, device; both scales
+ * > 0) into `ws` (dory_gemm_nvfp4_workspace_bytes, 256-byte aligned) and
+ * writes C = Q(A) Q(B)^T in fp32 (the product of the two tensor scales
+ * applied to the accumulators), split over K into k_splits slices C[s][M][N]
+ * (1..8) whose sum is the product.  K a multiple of 256. */
+DORY_API size_t dory_gemm_nvfp4_workspace_bytes(int M, int N, int K);
+DORY_API int dory_gemm_nvfp4(const void* A, const void* B, float* C, int M, int N, int K,
+                             float g_a, float g_b, int k_splits, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* ---------------------------------------------------------------------
  * Mask and failure-path diagnostics.
  * --------------------------------------------------------------------- */
@@ -417,7 +455,7 @@ DORY_API int dory_debug_wait_timeout(dory_model* m, uint32_t limit_us, void* str
 
 DORY_API int dory_mlp_sublayer_noalloc(dory_model* m, int layer, int n_rows, float* h,
                                        void* stream);
-/* (Models with weight_format DORY_WEIGHTS_MXFP8 return DORY_ERR_BAD_CONFIG.) */
+/* (Models with block-scaled weights, MXFP8 or NVFP4, return DORY_ERR_BAD_CONFIG.) */
 
 #ifdef __cplusplus
 }

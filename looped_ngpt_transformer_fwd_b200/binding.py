@@ -34,12 +34,13 @@ EXPORTS = (
     "dory_profile_enable", "dory_profile_read", "dory_mlp_sublayer_noalloc",
     "dory_debug_mask_probe", "dory_debug_attention_paths", "dory_debug_wait_timeout",
     "dory_debug_fused_update", "dory_quant_mxfp8", "dory_mxfp8_scale_bytes",
-    "dory_gemm_mxfp8_workspace_bytes", "dory_gemm_mxfp8",
+    "dory_gemm_mxfp8_workspace_bytes", "dory_gemm_mxfp8", "dory_quant_nvfp4",
+    "dory_nvfp4_scale_bytes", "dory_gemm_nvfp4_workspace_bytes", "dory_gemm_nvfp4",
     "dory_vocab_bytes", "dory_vocab_create", "dory_embed", "dory_lm_head", "dory_sample",
     "dory_vocab_free",
 )
 
-WEIGHT_FORMATS = {"bf16": 0, "mxfp8": 1}
+WEIGHT_FORMATS = {"bf16": 0, "mxfp8": 1, "nvfp4": 2}
 
 ATTENTION_PATHS = ("prefill_tc", "prefill_mma", "decode_tma", "decode_cp")
 
@@ -118,6 +119,10 @@ def lib():
             "dory_mxfp8_scale_bytes": (SZ, [I, I]),
             "dory_gemm_mxfp8_workspace_bytes": (SZ, [I, I, I]),
             "dory_gemm_mxfp8": (I, [P, P, P, I, I, I, I, P, SZ, P]),
+            "dory_quant_nvfp4": (I, [P, I, I, ctypes.c_float, P, P, P, P]),
+            "dory_nvfp4_scale_bytes": (SZ, [I, I]),
+            "dory_gemm_nvfp4_workspace_bytes": (SZ, [I, I, I]),
+            "dory_gemm_nvfp4": (I, [P, P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, SZ, P]),
             "dory_vocab_bytes": (SZ, [P, I]),
             "dory_vocab_create": (I, [P, I, P, P, P, P, SZ, P, P]),
             "dory_embed": (I, [P, P, I, P, P]),
@@ -300,6 +305,24 @@ def dory_gemm_mxfp8_workspace_bytes(M, N, K):
 def dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream):
     return check(lib().dory_gemm_mxfp8(A, B, C, M, N, K, k_splits, ws, ws_bytes, stream),
                  "dory_gemm_mxfp8")
+
+
+def dory_quant_nvfp4(src, rows, K, g, d_g, codes, scales, stream):
+    return check(lib().dory_quant_nvfp4(src, rows, K, g, d_g, codes, scales, stream),
+                 "dory_quant_nvfp4")
+
+
+def dory_nvfp4_scale_bytes(rows, K):
+    return lib().dory_nvfp4_scale_bytes(rows, K)
+
+
+def dory_gemm_nvfp4_workspace_bytes(M, N, K):
+    return lib().dory_gemm_nvfp4_workspace_bytes(M, N, K)
+
+
+def dory_gemm_nvfp4(A, B, C, M, N, K, g_a, g_b, k_splits, ws, ws_bytes, stream):
+    return check(lib().dory_gemm_nvfp4(A, B, C, M, N, K, g_a, g_b, k_splits, ws, ws_bytes, stream),
+                 "dory_gemm_nvfp4")
 
 
 def dory_vocab_bytes(cfg_struct, vocab):

@@ -66,13 +66,25 @@ struct BlockW {
   CUtensorMap tm_qkvg[2], tm_o[2], tm_gu[2], tm_d[2];
   // W_o / W_down for the fused projection + nGPT update (box rows = one MMA's N)
   CUtensorMap tm_o_n, tm_d_n;
-  // MXFP8 weights (weight_format 1): E4M3 codes, E8M0 scale chunks (whole
-  // 256-row tiles); gate / up rows interleaved in groups of 64
+  // Block-scaled weights (weight_format MXFP8: E4M3 codes, E8M0 scale chunks;
+  // NVFP4: packed E2M1 codes, E4M3 scale chunks), scale chunks covering whole
+  // 256-row tiles; gate / up rows interleaved in groups of 64
   uint8_t *q8 = nullptr, *o8 = nullptr, *gu8 = nullptr, *d8 = nullptr;
   uint8_t *qsf = nullptr, *osf = nullptr, *gusf = nullptr, *dsf = nullptr;
   CUtensorMap tm8_qkvg, tm8_o, tm8_gu, tm8_d;                  // 128-row boxes (decode)
   CUtensorMap tm8_qkvg_256, tm8_o_256, tm8_gu_256, tm8_d_256;  // 256-row boxes (prefill)
+  // NVFP4 tensor scales of the four projections' weights (one per GEMM: the
+  // q | k | v | gate rows share one, as do the gate and up rows), on the
+  // device (tscale) and copied to the host once they are computed
+  float* tscale = nullptr;
+  float g_qkvg = 1.f, g_o = 1.f, g_gu = 1.f, g_d = 1.f;
 };
+
+// Tensor scale of every NVFP4 projection input: the rows are unit vectors
+// (the stream h, and the attention output and SwiGLU activations after their
+// L2 norm), so no element exceeds 1 and g = 1 / (6 * 448) keeps every block
+// scale amax / (6 g) <= 448 within E4M3's range.
+constexpr float kNvfp4ActScale = static_cast<float>(1.0 / 2688.0);
 
 struct GraphKey {
   int phase, k, n, seq, pos0, max_pos, prof;
@@ -131,7 +143,7 @@ struct dory_model {
   // three waves; the unfused projection + row kernel measured faster.
   int ngpt_bnc = 0, ngpt_cluster = 0;
   bool fused_update = false;
-  bool mx = false;   // MXFP8 weights and projection inputs
+  int mx = kOperandsBf16;   // block-scaled weights and projection inputs (MXFP8 or NVFP4)
   int device = 0, num_sms = 148;
   uint8_t* wbuf = nullptr;
   size_t wbytes = 0;
@@ -191,7 +203,11 @@ int validate_config(const dory_config* c) {
   if (c->window < 1 || c->full_period < 1) return DORY_ERR_BAD_CONFIG;
   if (!(c->rope_base_swa > 1.0) || !(c->rope_base_full > 1.0)) return DORY_ERR_BAD_CONFIG;
   if (!(c->softmax_scale > 0.f) || !(c->norm_eps > 0.f)) return DORY_ERR_BAD_CONFIG;
-  if (c->weight_format != DORY_WEIGHTS_BF16 && c->weight_format != DORY_WEIGHTS_MXFP8)
+  if (c->weight_format != DORY_WEIGHTS_BF16 && c->weight_format != DORY_WEIGHTS_MXFP8 &&
+      c->weight_format != DORY_WEIGHTS_NVFP4)
+    return DORY_ERR_BAD_CONFIG;
+  // NVFP4 GEMMs take K in steps of 256
+  if (c->weight_format == DORY_WEIGHTS_NVFP4 && (c->d_model % 256 || c->d_ff % 256))
     return DORY_ERR_BAD_CONFIG;
   return DORY_OK;
 }
@@ -200,9 +216,10 @@ struct WeightLayout {
   size_t header = 0;                 // status word + RoPE tables
   size_t per_block = 0;
   size_t off_qkvg = 0, off_o = 0, off_gu = 0, off_d = 0, off_aa = 0, off_am = 0, off_sqk = 0;
-  // MXFP8: codes and scale chunks of the four matrices
+  // MXFP8 / NVFP4: codes and scale chunks of the four matrices; NVFP4 tensor
+  // scales (4 floats) and an amax scratch word
   size_t off_q8 = 0, off_qsf = 0, off_o8 = 0, off_osf = 0, off_gu8 = 0, off_gusf = 0, off_d8 = 0,
-         off_dsf = 0;
+         off_dsf = 0, off_ts = 0;
   size_t total = 0;
 };
 
@@ -222,6 +239,16 @@ WeightLayout weight_layout(const dory_config* c) {
     L.off_gusf = o; o = align_up(o + mxfp8_scale_bytes(int(2 * ff), int(d), 256));
     L.off_d8 = o;   o = align_up(o + d * ff);
     L.off_dsf = o;  o = align_up(o + mxfp8_scale_bytes(int(d), int(ff), 256));
+  } else if (c->weight_format == DORY_WEIGHTS_NVFP4) {
+    L.off_q8 = o;   o = align_up(o + nq * d / 2);
+    L.off_qsf = o;  o = align_up(o + nvfp4_scale_bytes(int(nq), int(d), 256));
+    L.off_o8 = o;   o = align_up(o + d * da / 2);
+    L.off_osf = o;  o = align_up(o + nvfp4_scale_bytes(int(d), int(da), 256));
+    L.off_gu8 = o;  o = align_up(o + 2 * ff * d / 2);
+    L.off_gusf = o; o = align_up(o + nvfp4_scale_bytes(int(2 * ff), int(d), 256));
+    L.off_d8 = o;   o = align_up(o + d * ff / 2);
+    L.off_dsf = o;  o = align_up(o + nvfp4_scale_bytes(int(d), int(ff), 256));
+    L.off_ts = o;   o = align_up(o + 8 * sizeof(float));
   } else {
     L.off_qkvg = o; o = align_up(o + nq * d * 2);
     L.off_o = o;    o = align_up(o + d * da * 2);
@@ -267,10 +294,13 @@ WsLayout ws_layout(const dory_model* m, int T) {
   L.rope_full = take(size_t(T) * (m->hd / 2) * 8);
   // K-split partial products of the decode QKVG and gate/up projections
   L.part = take(size_t(dec_rows) * kMaxKSplits * std::max<size_t>(m->ld_qkvg, 2 * ff) * 4);
-  // MXFP8 mode: the current projection's input as E4M3 codes and scale chunks
+  // block-scaled modes: the current projection's input as codes and scale
+  // chunks
   const int kmax = std::max(m->d, std::max(m->d_attn, m->ff));
   L.x8 = m->mx ? take(size_t(T) * kmax) : o;
-  L.xsf = m->mx ? take(mxfp8_scale_bytes(T, kmax)) : o;
+  L.xsf = m->mx ? take(m->mx == kOperandsNvfp4 ? nvfp4_scale_bytes(T, kmax)
+                                                : mxfp8_scale_bytes(T, kmax))
+                : o;
   L.total = o;
   return L;
 }
@@ -385,7 +415,7 @@ struct Launch {
 int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   if (tiles >= m->num_sms / 2) return 1;
-  const int kstep = m->mx ? 128 : 64;   // K per pipeline stage
+  const int kstep = m->mx == kOperandsNvfp4 ? 256 : (m->mx ? 128 : 64);   // K per pipeline stage
   int s = std::max(1, m->num_sms / tiles);
   s = std::min(s, kMaxKSplits);
   s = std::min(s, std::max(1, (K / kstep) / 4));
@@ -395,10 +425,11 @@ int pick_k_splits(const dory_model* m, int M, int N, int BN, int K) {
 }
 
 // The A operand of a projection over this call's rows: the bf16 rows, or in
-// MXFP8 mode their E4M3 codes and scales (from the fp32 stream `f32`, or from
-// bf16 rows scaled to unit L2 norm first when `normalize`; the norms before
-// the output and down projections are applied here, where quantisation makes
-// them matter).  Sets the tensor map and the MXFP8 fields of g.
+// the block-scaled modes their MXFP8 / NVFP4 codes and scales (from the fp32
+// stream `f32`, or from bf16 rows scaled to unit L2 norm first when
+// `normalize`; the norms before the output and down projections are applied
+// here, where quantisation makes them matter).  Sets the tensor map and the
+// block-scaled fields of g (NVFP4: alpha starts as the inputs' tensor scale).
 cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const __nv_bfloat16* rows,
                              const float* f32, int K, bool normalize) {
   dory_model* m = c.m;
@@ -406,28 +437,41 @@ cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const _
     if (!make_tmap_bf16(tm, rows, c.n, K, 128)) return cudaErrorInvalidValue;
     return cudaSuccess;
   }
+  const bool nv = m->mx == kOperandsNvfp4;
   {
     Launch L(m, c.s, DORY_KK_ROW);
-    if (f32) {
-      DORY_TRY(launch_quant_mxfp8_f32(f32, c.n, K, 0, m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
+    const float eps = m->cfg.norm_eps;
+    const int nrm = normalize ? 1 : 0;
+    const __nv_bfloat16* seg[1] = {rows};
+    if (nv && f32) {
+      DORY_TRY(launch_quant_nvfp4_f32(f32, c.n, K, 0, eps, nullptr, kNvfp4ActScale, c.w.x8,
+                                      c.w.xsf, c.s));
+    } else if (nv) {
+      DORY_TRY(launch_quant_nvfp4_bf16(seg, nullptr, 1, 0, c.n, 128, K, nrm, eps, nullptr,
+                                       kNvfp4ActScale, c.w.x8, c.w.xsf, c.s));
+    } else if (f32) {
+      DORY_TRY(launch_quant_mxfp8_f32(f32, c.n, K, 0, eps, c.w.x8, c.w.xsf, c.s));
     } else {
-      const __nv_bfloat16* seg[1] = {rows};
-      DORY_TRY(launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, c.n, 128, K, normalize ? 1 : 0,
-                                       m->cfg.norm_eps, c.w.x8, c.w.xsf, c.s));
+      DORY_TRY(launch_quant_mxfp8_bf16(seg, nullptr, 1, 0, c.n, 128, K, nrm, eps, c.w.x8, c.w.xsf,
+                                       c.s));
     }
   }
-  if (!make_tmap_u8(tm, c.w.x8, c.n, K, 128)) return cudaErrorInvalidValue;
-  g.mx = 1;
+  // NVFP4 rows hold K / 2 bytes (two codes per byte)
+  if (!make_tmap_u8(tm, c.w.x8, c.n, nv ? K / 2 : K, 128)) return cudaErrorInvalidValue;
+  g.mx = m->mx;
   g.sfa = c.w.xsf;
   g.sfa_blocks = (c.n + 127) / 128;
+  g.alpha = nv ? kNvfp4ActScale : 1.f;
   return cudaSuccess;
 }
 
-// B operand (weights) of the MXFP8 GEMMs: scale chunks and their row blocks
-// (weights' chunks cover whole 256-row tiles)
-void mx_weights(GemmParams& g, const uint8_t* sf, int n_rows) {
+// B operand (weights) of the block-scaled GEMMs: scale chunks and their row
+// blocks (weights' chunks cover whole 256-row tiles), and for NVFP4 the
+// weights' tensor scale g_w into alpha
+void mx_weights(GemmParams& g, const uint8_t* sf, int n_rows, float g_w) {
   g.sfb = sf;
   g.sfb_blocks = (n_rows + 255) / 256 * 2;
+  if (g.mx == kOperandsNvfp4) g.alpha *= g_w;
 }
 
 // Prefill projections with the nGPT update in their epilogue (a cluster of
@@ -444,7 +488,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   CUtensorMap tmA;
   GemmParams g;
   DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
-  if (m->mx) mx_weights(g, W.qsf, m->n_qkvg);
+  if (m->mx) mx_weights(g, W.qsf, m->n_qkvg, W.g_qkvg);
   const float2* rope = W.full ? c.w.rope_full : c.w.rope_swa;
   if (c.decode) {
     // few rows: spread the weight stream over the SMs with K splits, then a
@@ -479,8 +523,8 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     g.norm_eps = m->cfg.norm_eps;
     g.status = m->status;
     Launch L(m, c.s, DORY_KK_QKVG);
-    // MXFP8: 128-column tiles keep two accumulators, so the QKVG epilogue
-    // overlaps the next tile's MMAs
+    // block-scaled: 128-column tiles keep two accumulators, so the QKVG
+    // epilogue overlaps the next tile's MMAs
     if (m->mx)
       DORY_TRY(launch_gemm(tmA, W.tm8_qkvg, g, 128, m->hd, m->num_sms, c.s));
     else
@@ -558,7 +602,7 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   CUtensorMap tmO;
   GemmParams go;
   DORY_TRY(projection_input(c, &tmO, go, c.w.o, nullptr, m->d_attn, true));
-  if (m->mx) mx_weights(go, W.osf, m->d);
+  if (m->mx) mx_weights(go, W.osf, m->d, W.g_o);
   if (use_fused(c)) {
     NgptGemmParams f;
     f.M = c.n; f.N = m->d; f.K = m->d_attn; f.cluster = m->ngpt_cluster;
@@ -604,10 +648,10 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   CUtensorMap tmA;
   GemmParams g;
   DORY_TRY(projection_input(c, &tmA, g, hb, h, m->d, false));
-  if (m->mx) mx_weights(g, W.gusf, 2 * m->ff);
+  if (m->mx) mx_weights(g, W.gusf, 2 * m->ff, W.g_gu);
   // gate and up rows alternate in groups of half a GEMM tile: 128 (bf16,
-  // 256-column tiles), 64 (MXFP8, 128-column tiles with two accumulators, so
-  // the SwiGLU epilogue overlaps the next tile's MMAs)
+  // 256-column tiles), 64 (block-scaled, 128-column tiles with two
+  // accumulators, so the SwiGLU epilogue overlaps the next tile's MMAs)
   const int gu_group = m->mx ? 64 : 128;
   if (c.decode) {
     g.M = c.n; g.N = 2 * m->ff; g.K = m->d;
@@ -637,7 +681,7 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   CUtensorMap tmAct;
   GemmParams gd;
   DORY_TRY(projection_input(c, &tmAct, gd, c.w.a, nullptr, m->ff, true));
-  if (m->mx) mx_weights(gd, W.dsf, m->d);
+  if (m->mx) mx_weights(gd, W.dsf, m->d, W.g_d);
   if (use_fused(c)) {
     NgptGemmParams f;
     f.M = c.n; f.N = m->d; f.K = m->ff; f.cluster = m->ngpt_cluster;
@@ -840,8 +884,8 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
     if (!s.wq || !s.wk || !s.wv || !s.wg || !s.wo || !s.w_gate || !s.w_up || !s.w_down ||
         !s.alpha_attn || !s.alpha_mlp || !s.s_qk)
       return DORY_ERR_INVALID_ARG;
-    // MXFP8 weights are quantised by a kernel that reads the bf16 matrices
-    if (cfg->weight_format == DORY_WEIGHTS_MXFP8) {
+    // MXFP8 / NVFP4 weights are quantised by kernels that read the bf16 matrices
+    if (cfg->weight_format != DORY_WEIGHTS_BF16) {
       const void* mats[8] = {s.wq, s.wk, s.wv, s.wg, s.wo, s.w_gate, s.w_up, s.w_down};
       for (const void* p : mats)
         if (!is_device_ptr(p) || !is_aligned(p, 16)) return DORY_ERR_INVALID_ARG;
@@ -855,7 +899,9 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
   m->ff = cfg->d_ff; m->d_attn = m->hq * m->hd;
   m->n_qkvg = m->d_attn + 2 * m->hkv * m->hd + m->hq;
   m->ld_qkvg = (m->n_qkvg + 31) / 32 * 32;
-  m->mx = cfg->weight_format == DORY_WEIGHTS_MXFP8;
+  m->mx = cfg->weight_format == DORY_WEIGHTS_MXFP8   ? kOperandsMxfp8
+          : cfg->weight_format == DORY_WEIGHTS_NVFP4 ? kOperandsNvfp4
+                                                     : kOperandsBf16;
   m->ngpt_bnc = ngpt_gemm_cols_per_cta(m->d);
   m->ngpt_cluster = m->ngpt_bnc ? m->d / m->ngpt_bnc : 0;
   m->nb = n_blocks(cfg);
@@ -914,22 +960,47 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
                                     reinterpret_cast<const __nv_bfloat16*>(S.w_up)};
       const __nv_bfloat16* ds[1] = {reinterpret_cast<const __nv_bfloat16*>(S.w_down)};
       const float eps = cfg->norm_eps;
-      e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, 256, int(d), 0, eps, W.q8,
-                                          W.qsf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), 256, int(da), 0, eps, W.o8,
-                                          W.osf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 64, int(2 * F), 256, int(d), 0, eps,
-                                          W.gu8, W.gusf, s);
-      e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), 256, int(F), 0, eps, W.d8,
-                                          W.dsf, s);
-      ok &= make_tmap_u8(&W.tm8_qkvg, W.q8, m->n_qkvg, d, 128);
-      ok &= make_tmap_u8(&W.tm8_o, W.o8, d, da, 128);
-      ok &= make_tmap_u8(&W.tm8_gu, W.gu8, 2 * F, d, 128);
-      ok &= make_tmap_u8(&W.tm8_d, W.d8, d, F, 128);
-      ok &= make_tmap_u8(&W.tm8_qkvg_256, W.q8, m->n_qkvg, d, 256);
-      ok &= make_tmap_u8(&W.tm8_o_256, W.o8, d, da, 256);
-      ok &= make_tmap_u8(&W.tm8_gu_256, W.gu8, 2 * F, d, 256);
-      ok &= make_tmap_u8(&W.tm8_d_256, W.d8, d, F, 256);
+      if (m->mx == kOperandsNvfp4) {
+        // one tensor scale per GEMM's weights: q | k | v | gate together,
+        // gate and up together (g = amax / (6 * 448) over the group)
+        W.tscale = reinterpret_cast<float*>(base + L.off_ts);
+        uint32_t* amax = reinterpret_cast<uint32_t*>(W.tscale + 4);
+        const size_t qcounts[4] = {da * d, kvr * d, kvr * d, size_t(m->hq) * d};
+        const size_t ocount[1] = {d * da}, gcounts[2] = {F * d, F * d}, dcount[1] = {d * F};
+        e = e ? e : launch_nvfp4_tensor_scale(qs, qcounts, 4, amax, W.tscale + 0, s);
+        e = e ? e : launch_nvfp4_tensor_scale(os, ocount, 1, amax, W.tscale + 1, s);
+        e = e ? e : launch_nvfp4_tensor_scale(gs, gcounts, 2, amax, W.tscale + 2, s);
+        e = e ? e : launch_nvfp4_tensor_scale(ds, dcount, 1, amax, W.tscale + 3, s);
+        e = e ? e : launch_quant_nvfp4_bf16(qs, qrows, 4, 0, m->n_qkvg, 256, int(d), 0, eps,
+                                            W.tscale + 0, 0.f, W.q8, W.qsf, s);
+        e = e ? e : launch_quant_nvfp4_bf16(os, nullptr, 1, 0, int(d), 256, int(da), 0, eps,
+                                            W.tscale + 1, 0.f, W.o8, W.osf, s);
+        e = e ? e : launch_quant_nvfp4_bf16(gs, nullptr, 2, 64, int(2 * F), 256, int(d), 0, eps,
+                                            W.tscale + 2, 0.f, W.gu8, W.gusf, s);
+        e = e ? e : launch_quant_nvfp4_bf16(ds, nullptr, 1, 0, int(d), 256, int(F), 0, eps,
+                                            W.tscale + 3, 0.f, W.d8, W.dsf, s);
+      } else {
+        e = e ? e : launch_quant_mxfp8_bf16(qs, qrows, 4, 0, m->n_qkvg, 256, int(d), 0, eps, W.q8,
+                                            W.qsf, s);
+        e = e ? e : launch_quant_mxfp8_bf16(os, nullptr, 1, 0, int(d), 256, int(da), 0, eps, W.o8,
+                                            W.osf, s);
+        e = e ? e : launch_quant_mxfp8_bf16(gs, nullptr, 2, 64, int(2 * F), 256, int(d), 0, eps,
+                                            W.gu8, W.gusf, s);
+        e = e ? e : launch_quant_mxfp8_bf16(ds, nullptr, 1, 0, int(d), 256, int(F), 0, eps, W.d8,
+                                            W.dsf, s);
+      }
+      // tensor maps over the code bytes (NVFP4: K / 2 per row)
+      const size_t kd = m->mx == kOperandsNvfp4 ? d / 2 : d;
+      const size_t kda = m->mx == kOperandsNvfp4 ? da / 2 : da;
+      const size_t kF = m->mx == kOperandsNvfp4 ? F / 2 : F;
+      ok &= make_tmap_u8(&W.tm8_qkvg, W.q8, m->n_qkvg, kd, 128);
+      ok &= make_tmap_u8(&W.tm8_o, W.o8, d, kda, 128);
+      ok &= make_tmap_u8(&W.tm8_gu, W.gu8, 2 * F, kd, 128);
+      ok &= make_tmap_u8(&W.tm8_d, W.d8, d, kF, 128);
+      ok &= make_tmap_u8(&W.tm8_qkvg_256, W.q8, m->n_qkvg, kd, 256);
+      ok &= make_tmap_u8(&W.tm8_o_256, W.o8, d, kda, 256);
+      ok &= make_tmap_u8(&W.tm8_gu_256, W.gu8, 2 * F, kd, 256);
+      ok &= make_tmap_u8(&W.tm8_d_256, W.d8, d, kF, 256);
     } else {
       uint8_t* q = reinterpret_cast<uint8_t*>(W.wqkvg);
       e = e ? e : cudaMemcpyAsync(q, S.wq, da * d * 2, cudaMemcpyDefault, s);
@@ -966,18 +1037,30 @@ int dory_create(const dory_config* cfg, void* weight_buf, size_t weight_bytes,
     if (e != cudaSuccess) return DORY_ERR_CUDA;
     if (!ok) return DORY_ERR_CUDA;
   }
-  // static softmax maxima from the packed s_qk vectors (one-time host read)
+  // static softmax maxima from the packed s_qk vectors, and the NVFP4 weight
+  // tensor scales (one-time host read: the GEMM epilogues take them as
+  // launch parameters)
   {
-    std::vector<float> sq(size_t(m->nb) * hd);
-    for (int b = 0; b < m->nb; ++b)
+    std::vector<float> sq(size_t(m->nb) * hd), ts(size_t(m->nb) * 4, 1.f);
+    for (int b = 0; b < m->nb; ++b) {
       if (cudaMemcpyAsync(sq.data() + size_t(b) * hd, m->blocks[b].s_qk, hd * 4,
                           cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return DORY_ERR_CUDA;
+      if (m->blocks[b].tscale &&
+          cudaMemcpyAsync(ts.data() + size_t(b) * 4, m->blocks[b].tscale, 4 * sizeof(float),
+                          cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return DORY_ERR_CUDA;
+    }
     if (cudaStreamSynchronize(s) != cudaSuccess) return DORY_ERR_CUDA;
     for (int b = 0; b < m->nb; ++b) {
       float mx = 0.f;
       for (size_t i = 0; i < hd; ++i) mx = std::max(mx, sq[size_t(b) * hd + i] * sq[size_t(b) * hd + i]);
-      m->blocks[b].m_log2 = cfg->softmax_scale * 1.4426950408889634f * mx;
+      BlockW& W = m->blocks[b];
+      W.m_log2 = cfg->softmax_scale * 1.4426950408889634f * mx;
+      W.g_qkvg = ts[size_t(b) * 4 + 0];
+      W.g_o = ts[size_t(b) * 4 + 1];
+      W.g_gu = ts[size_t(b) * 4 + 2];
+      W.g_d = ts[size_t(b) * 4 + 3];
     }
   }
   if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
@@ -1334,8 +1417,78 @@ int dory_gemm_mxfp8(const void* A, const void* B, float* C, int M, int N, int K,
   GemmParams p;
   p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
   p.k_splits = k_splits; p.split_stride = size_t(M) * N;
-  p.mx = 1; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128;
+  p.mx = kOperandsMxfp8; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128;
   p.sfb_blocks = (N + BN - 1) / BN * (BN / 128);
+  if (launch_gemm(ta, tb, p, BN, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+int dory_quant_nvfp4(const void* src, int rows, int K, float g, float* d_g, void* codes,
+                     void* scales, void* stream) {
+  if (!src || !codes || !scales || rows <= 0 || K <= 0 || K % 256) return DORY_ERR_INVALID_ARG;
+  if (!(g > 0.f) && !d_g) return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(src, 16) || !is_aligned(codes, 16)) return DORY_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* seg[1] = {static_cast<const __nv_bfloat16*>(src)};
+  if (!(g > 0.f)) {
+    // the tensor scale from the data: amax / (6 * 448), computed into d_g
+    const size_t count[1] = {size_t(rows) * K};
+    if (launch_nvfp4_tensor_scale(seg, count, 1, reinterpret_cast<uint32_t*>(d_g), d_g, s) !=
+        cudaSuccess)
+      return DORY_ERR_CUDA;
+  }
+  if (launch_quant_nvfp4_bf16(seg, nullptr, 1, 0, rows, 128, K, 0, 1e-20f, g > 0.f ? nullptr : d_g,
+                              g, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                              s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
+size_t dory_nvfp4_scale_bytes(int rows, int K) {
+  if (rows <= 0 || K <= 0 || K % 256) return 0;
+  return nvfp4_scale_bytes(rows, K);
+}
+
+size_t dory_gemm_nvfp4_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 256) return 0;
+  return align_up(size_t(M) * K / 2) + align_up(nvfp4_scale_bytes(M, K)) +
+         align_up(size_t(N) * K / 2) + align_up(nvfp4_scale_bytes(N, K, 256));
+}
+
+int dory_gemm_nvfp4(const void* A, const void* B, float* C, int M, int N, int K, float g_a,
+                    float g_b, int k_splits, void* ws, size_t ws_bytes, void* stream) {
+  if (!A || !B || !C || !ws || M <= 0 || N <= 0 || K <= 0 || K % 256 || k_splits < 1 ||
+      k_splits > kMaxKSplits || !(g_a > 0.f) || !(g_b > 0.f))
+    return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16) || !is_aligned(ws))
+    return DORY_ERR_MISALIGNED;
+  if (ws_bytes < dory_gemm_nvfp4_workspace_bytes(M, N, K)) return DORY_ERR_BUFFER_TOO_SMALL;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* a4 = static_cast<uint8_t*>(ws);
+  uint8_t* asf = a4 + align_up(size_t(M) * K / 2);
+  uint8_t* b4 = asf + align_up(nvfp4_scale_bytes(M, K));
+  uint8_t* bsf = b4 + align_up(size_t(N) * K / 2);
+  const __nv_bfloat16* sa[1] = {static_cast<const __nv_bfloat16*>(A)};
+  const __nv_bfloat16* sb[1] = {static_cast<const __nv_bfloat16*>(B)};
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  if (launch_quant_nvfp4_bf16(sa, nullptr, 1, 0, M, 128, K, 0, 1e-20f, nullptr, g_a, a4, asf, s) !=
+          cudaSuccess ||
+      launch_quant_nvfp4_bf16(sb, nullptr, 1, 0, N, BN, K, 0, 1e-20f, nullptr, g_b, b4, bsf, s) !=
+          cudaSuccess)
+    return DORY_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, a4, M, K / 2, 128) || !make_tmap_u8(&tb, b4, N, K / 2, BN))
+    return DORY_ERR_CUDA;
+  GemmParams p;
+  p.M = M; p.N = N; p.K = K; p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  p.k_splits = k_splits; p.split_stride = size_t(M) * N;
+  p.mx = kOperandsNvfp4; p.sfa = asf; p.sfb = bsf; p.sfa_blocks = (M + 127) / 128;
+  p.sfb_blocks = (N + BN - 1) / BN * (BN / 128);
+  p.alpha = g_a * g_b;
   if (launch_gemm(ta, tb, p, BN, 128, sms, s) != cudaSuccess) return DORY_ERR_CUDA;
   return DORY_OK;
 }

@@ -29,28 +29,37 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kGemmThreads = 192;
 
-// MX = false: bf16 operands, 64 K per stage.  MX = true: MXFP8 operands (E4M3
-// codes, one E8M0 scale per 32 along K), 128 K per stage (the same 128 bytes
-// per row), the stage's scale chunks staged in shared memory after the tiles
-// and copied to TMEM for the block-scaled MMA.
-template <int BN, bool MX = false>
+// MX = kOperandsBf16: bf16 operands, 64 K per stage.  kOperandsMxfp8: E4M3
+// codes with one E8M0 scale per 32 along K, 128 K per stage (the same 128
+// bytes per row).  kOperandsNvfp4: packed E2M1 codes with one E4M3 scale per
+// 16 along K, 256 K per stage (again 128 bytes per row).  The block-scaled
+// forms stage the step's scale chunks in shared memory after the tiles and
+// copy them to TMEM for the MMAs.
+template <int BN, int MX = kOperandsBf16>
 struct GemmCfg {
+  static constexpr bool kNv = MX == kOperandsNvfp4;
   static constexpr int kStages = MX ? (BN == 256 ? 3 : 5) : ((BN == 256) ? 4 : 6);
-  static constexpr int kKStep = MX ? 128 : kBK;              // K elements per stage
+  static constexpr int kKStep = kNv ? 256 : (MX ? 128 : kBK);   // K elements per stage
+  // the stage's step of the tensor maps' x coordinate, in map elements (bf16
+  // values, or bytes of codes: 128 per row and stage in both block-scaled forms)
+  static constexpr int kKCoord = MX ? 128 : kBK;
   static constexpr int kABytes = kBM * 128;
   static constexpr int kBBytes = BN * 128;
-  static constexpr int kSfaBytes = MX ? 512 : 0;             // 128 rows x 4 scales
-  static constexpr int kSfbBytes = MX ? 512 * (BN / 128) : 0;
+  // scale bytes per 128 rows and stage: 128 x 4 (MXFP8), 128 x 16 (NVFP4)
+  static constexpr int kSfChunk = kNv ? 2048 : (MX ? 512 : 0);
+  static constexpr int kSfaBytes = kSfChunk;
+  static constexpr int kSfbBytes = kSfChunk * (BN / 128);
   // bytes the TMA and bulk copies of one stage deliver (the mbarrier's
   // transaction count), and the stage's footprint, padded to keep every
   // stage's tiles 1024-byte aligned
   static constexpr int kLoadBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStageBytes = (kLoadBytes + 1023) / 1024 * 1024;
   // accumulators (kAccBufs x BN columns), then per stage the A and B scale
-  // columns; a 256-column MXFP8 tile keeps a single accumulator so that the
-  // scale columns fit next to it
+  // columns (MXFP8: one 32-bit word per row holds the stage's four scales;
+  // NVFP4: one word per row and 64-K MMA); a 256-column block-scaled tile
+  // keeps a single accumulator so that the scale columns fit next to it
   static constexpr int kAccBufs = (MX && BN == 256) ? 1 : 2;
-  static constexpr int kSfCols = 4 + 4 * (BN / 128);
+  static constexpr int kSfCols = (kNv ? 16 : 4) * (1 + BN / 128);
   static constexpr int kTmemCols = MX ? 512 : 2 * BN;
   static_assert(!MX || kAccBufs * BN + kStages * kSfCols <= 512, "TMEM columns");
   static_assert(kStageBytes % 1024 == 0, "stages keep the tiles 1024-byte aligned");
@@ -148,7 +157,38 @@ __device__ __forceinline__ void umma_mxf8(uint32_t tmem_d, uint64_t adesc, uint6
       : "memory");
 }
 
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4 with block scaling:
+// E2M1 A and B (K-major, packed two per byte), UE4M3 scales, one per 16 along
+// K (scale_vec::4X: the four scales of a 64-K step fill a 32-bit word, so the
+// scale factor ids stay 0), fp32 accumulation.
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10)                    // A, B format: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
+         | (0u << 23)                              // scale format: UE4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
+}
+__device__ __forceinline__ void umma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
 // --------------------------------------------------------------- epilogues
+// Accumulators times the tensor-scale product alpha (NVFP4 operands only).
+template <bool kAlpha, int N>
+__device__ __forceinline__ void apply_alpha(float (&v)[N], float alpha) {
+  if constexpr (kAlpha) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] *= alpha;
+  }
+}
+
 __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32], int valid) {
   // vector stores only where the row start allows them (any row pitch works)
   if (valid >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
@@ -161,7 +201,7 @@ __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32]
   }
 }
 
-template <int BN>
+template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t taddr, int row, int nt,
                                               int ks) {
   float* out = p.out_f32 + static_cast<size_t>(ks) * p.split_stride;
@@ -170,6 +210,7 @@ __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t tadd
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld32(taddr + c, v);
+    apply_alpha<kAlpha>(v, p.alpha);
     const int col = nt * BN + c;
     if (row_ok && col < p.N)
       store_f32_chunk(out + static_cast<size_t>(row) * p.ld_out + col, v, p.N - col);
@@ -181,7 +222,7 @@ __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t tadd
 // at chunk j ^ (r % 8), conflict-free) and one lane stores the box; the tensor
 // map [splits][M][N] clips rows past M and columns past N.  Two buffers per
 // warp alternate so staging overlaps the previous store.
-template <int BN>
+template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_store_f32_tma(const GemmParams& p, const CUtensorMap* tmC,
                                                   uint32_t taddr, uint8_t* stage, int lane,
                                                   int row0, int nt, int ks, uint32_t& nbuf) {
@@ -189,6 +230,7 @@ __device__ __forceinline__ void epi_store_f32_tma(const GemmParams& p, const CUt
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld32(taddr + c, v);
+    apply_alpha<kAlpha>(v, p.alpha);
     const int col = nt * BN + c;
     if (col >= p.N) continue;                   // warp-uniform
     uint8_t* buf = stage + (nbuf & 1u) * (32 * 32 * 4);
@@ -232,7 +274,7 @@ __device__ __forceinline__ void store_box_bf16(const CUtensorMap* map, uint8_t* 
 
 // SwiGLU activations in 64-column boxes through bulk tensor stores (rows past
 // M are clipped by the tensor map).
-template <int BN>
+template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_swiglu_tma(const GemmParams& p, const CUtensorMap* map,
                                                uint32_t taddr, uint8_t* stage, int lane, int row0,
                                                int nt, uint32_t& nbuf) {
@@ -246,6 +288,8 @@ __device__ __forceinline__ void epi_swiglu_tma(const GemmParams& p, const CUtens
       float g[32], u[32];
       tmem_ld32(taddr + c + 32 * half, g);
       tmem_ld32(taddr + H + c + 32 * half, u);
+      apply_alpha<kAlpha>(g, p.alpha);
+      apply_alpha<kAlpha>(u, p.alpha);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float g0 = p.gate_scale * g[2 * i], g1 = p.gate_scale * g[2 * i + 1];
@@ -258,7 +302,7 @@ __device__ __forceinline__ void epi_swiglu_tma(const GemmParams& p, const CUtens
   }
 }
 
-template <int BN>
+template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, int row, int nt) {
   constexpr int H = BN / 2;
   const bool row_ok = row < p.M;
@@ -269,6 +313,8 @@ __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, 
     tmem_ld32(taddr + c, g);
     tmem_ld32(taddr + H + c, u);
     if (!row_ok) continue;
+    apply_alpha<kAlpha>(g, p.alpha);
+    apply_alpha<kAlpha>(u, p.alpha);
     uint32_t packed[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -289,7 +335,7 @@ __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, 
 // shared memory); v heads are stored as computed; gate logits go through the
 // sigmoid.  With bulk stores (p.c_tma) the warp stages 64-column boxes of q,
 // k or v and every lane takes part, rows past M included (the maps clip them).
-template <int HD>
+template <int HD, bool kAlpha>
 __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float* sqk,
                                                const OutMaps* om, uint8_t* stage, int lane,
                                                int row0, uint32_t& nbuf, uint32_t taddr, int row,
@@ -303,6 +349,7 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
   for (int c = 0; c < HD; c += 32) {
     float t[32];
     tmem_ld32(taddr + c, t);
+    apply_alpha<kAlpha>(t, p.alpha);
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[c + i] = t[i];
   }
@@ -368,7 +415,7 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
 }
 
 
-template <int BN, int HD, int EPI, bool MX>
+template <int BN, int HD, int EPI, int MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ OutMaps om, const GemmParams p) {
@@ -447,15 +494,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* a_dst = tiles + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kLoadBytes);
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKStep, mt * kBM);
-          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKStep, nt * BN);
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKCoord, mt * kBM);
+          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKCoord, nt * BN);
           if constexpr (MX) {
             // this K step's scale chunks: one for A's 128 rows, BN/128 for B's
             bulk_load(a_dst + C::kABytes + C::kBBytes,
-                      p.sfa + (static_cast<size_t>(kb) * p.sfa_blocks + mt) * 512, C::kSfaBytes,
-                      &full[stage]);
+                      p.sfa + (static_cast<size_t>(kb) * p.sfa_blocks + mt) * C::kSfChunk,
+                      C::kSfaBytes, &full[stage]);
             bulk_load(a_dst + C::kABytes + C::kBBytes + C::kSfaBytes,
-                      p.sfb + (static_cast<size_t>(kb) * p.sfb_blocks + nt * (BN / 128)) * 512,
+                      p.sfb + (static_cast<size_t>(kb) * p.sfb_blocks + nt * (BN / 128)) * C::kSfChunk,
                       C::kSfbBytes, &full[stage]);
           }
           issued_mask |= 1u << stage;
@@ -505,7 +552,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint64_t soff = static_cast<uint64_t>((stage * C::kStageBytes) >> 4);
           const uint64_t a_desc = a_desc0 + soff, b_desc = b_desc0 + soff;
-          if constexpr (MX) {
+          if constexpr (C::kNv) {
+            // scales to TMEM (this stage's own columns, as for MXFP8): the
+            // 512-byte piece kk of each chunk holds 64-K step kk's scales, one
+            // 32-bit word per row; A's go to columns 4kk.., B's (BN / 32
+            // columns per step) after them; then four K = 64 MMAs
+            const uint32_t sf_col = tmem_base + C::kAccBufs * BN + stage * C::kSfCols;
+            const uint32_t sfb_col = sf_col + 16;
+            const uint32_t sf_smem = smem_u32(tiles + stage * C::kStageBytes + C::kABytes + C::kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              tmem_cp_32x128b_x4(sf_col + 4 * kk, sf_desc(sf_smem + 512 * kk));
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tmem_cp_32x128b_x4(sfb_col + kk * (BN / 32) + 4 * j,
+                                   sf_desc(sf_smem + C::kSfaBytes + 2048 * j + 512 * kk));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_nvf4(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4),
+                        umma_idesc_nvf4(kBM, BN), sf_col + 4 * kk, sfb_col + kk * (BN / 32),
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+          } else if constexpr (MX) {
             // scales to TMEM (this stage's own columns: the MMAs that read
             // them last time completed before the stage was refilled), then
             // four K = 32 block-scaled MMAs, MMA kk reading scale byte kk
@@ -560,20 +628,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int row = mt * kBM + quad * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      constexpr bool kAlpha = C::kNv;
       if constexpr (EPI == kEpiStoreF32) {
         if (p.c_tma)
-          epi_store_f32_tma<BN>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt, ks, nbuf);
+          epi_store_f32_tma<BN, kAlpha>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32,
+                                        nt, ks, nbuf);
         else
-          epi_store_f32<BN>(p, taddr, row, nt, ks);
+          epi_store_f32<BN, kAlpha>(p, taddr, row, nt, ks);
       } else if constexpr (EPI == kEpiSwiGLU) {
         if (p.c_tma)
-          epi_swiglu_tma<BN>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt, nbuf);
+          epi_swiglu_tma<BN, kAlpha>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt,
+                                     nbuf);
         else
-          epi_swiglu<BN>(p, taddr, row, nt);
+          epi_swiglu<BN, kAlpha>(p, taddr, row, nt);
       } else {
 #pragma unroll 1
         for (int g = 0; g < BN / HD; ++g)
-          epi_qkvg_group<HD>(p, sqk, &om, my_stage, lane, mt * kBM + quad * 32, nbuf,
+          epi_qkvg_group<HD, kAlpha>(p, sqk, &om, my_stage, lane, mt * kBM + quad * 32, nbuf,
                              taddr + g * HD, row, nt * BN + g * HD);
       }
       tc_fence_before();
@@ -650,7 +721,7 @@ bool make_tmap_out_bf16(CUtensorMap* map, const void* base, int rows, int cols, 
                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int HD, int EPI, bool MX = false>
+template <int BN, int HD, int EPI, int MX = kOperandsBf16>
 cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int num_sms, cudaStream_t s) {
   using C = GemmCfg<BN, MX>;
@@ -728,64 +799,56 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+
+template <int MX>
+cudaError_t dispatch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                          int BN, int head_dim, int num_sms, cudaStream_t s) {
+  if (BN == 256) {
+    switch (p.epi) {
+      case kEpiStoreF32: return launch_impl<256, 128, kEpiStoreF32, MX>(tmA, tmB, p, num_sms, s);
+      case kEpiSwiGLU: return launch_impl<256, 128, kEpiSwiGLU, MX>(tmA, tmB, p, num_sms, s);
+      case kEpiQKVG:
+        if (p.k_splits != 1) return cudaErrorInvalidValue;
+        if (head_dim == 128) return launch_impl<256, 128, kEpiQKVG, MX>(tmA, tmB, p, num_sms, s);
+        if (head_dim == 64) return launch_impl<256, 64, kEpiQKVG, MX>(tmA, tmB, p, num_sms, s);
+        return cudaErrorInvalidValue;
+    }
+  } else if (BN == 128) {
+    switch (p.epi) {
+      case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32, MX>(tmA, tmB, p, num_sms, s);
+      case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU, MX>(tmA, tmB, p, num_sms, s);
+      case kEpiQKVG:
+        if (p.k_splits != 1) return cudaErrorInvalidValue;
+        if (head_dim == 128) return launch_impl<128, 128, kEpiQKVG, MX>(tmA, tmB, p, num_sms, s);
+        if (head_dim == 64) return launch_impl<128, 64, kEpiQKVG, MX>(tmA, tmB, p, num_sms, s);
+        return cudaErrorInvalidValue;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                         int BN, int head_dim, int num_sms, cudaStream_t s) {
-  const int kstep = p.mx ? 128 : kBK;
+  if (p.mx != kOperandsBf16 && p.mx != kOperandsMxfp8 && p.mx != kOperandsNvfp4)
+    return cudaErrorInvalidValue;
+  const int kstep = p.mx == kOperandsNvfp4 ? 256 : (p.mx ? 128 : kBK);
   if (p.K % kstep != 0 || p.K <= 0 || p.k_splits < 1) return cudaErrorInvalidValue;
   {
     // every K split must own at least one k-block
     const int kb = p.K / kstep, per = (kb + p.k_splits - 1) / p.k_splits;
     if ((p.k_splits - 1) * per >= kb) return cudaErrorInvalidValue;
   }
-  if (p.mx) {
-    // block-scaled MXFP8 operands (accumulators and scale columns share TMEM)
-    if (!p.sfa || !p.sfb) return cudaErrorInvalidValue;
-    if (BN == 256) {
-      switch (p.epi) {
-        case kEpiStoreF32: return launch_impl<256, 128, kEpiStoreF32, true>(tmA, tmB, p, num_sms, s);
-        case kEpiSwiGLU: return launch_impl<256, 128, kEpiSwiGLU, true>(tmA, tmB, p, num_sms, s);
-        case kEpiQKVG:
-          if (p.k_splits != 1) return cudaErrorInvalidValue;
-          if (head_dim == 128) return launch_impl<256, 128, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
-          if (head_dim == 64) return launch_impl<256, 64, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
-          return cudaErrorInvalidValue;
-      }
-      return cudaErrorInvalidValue;
-    }
-    if (BN != 128) return cudaErrorInvalidValue;
-    switch (p.epi) {
-      case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32, true>(tmA, tmB, p, num_sms, s);
-      case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU, true>(tmA, tmB, p, num_sms, s);
-      case kEpiQKVG:
-        if (p.k_splits != 1) return cudaErrorInvalidValue;
-        if (head_dim == 128) return launch_impl<128, 128, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
-        if (head_dim == 64) return launch_impl<128, 64, kEpiQKVG, true>(tmA, tmB, p, num_sms, s);
-        return cudaErrorInvalidValue;
-    }
-    return cudaErrorInvalidValue;
+  // block-scaled operands need their scales (accumulators and scale columns
+  // share TMEM)
+  if (p.mx && (!p.sfa || !p.sfb)) return cudaErrorInvalidValue;
+  switch (p.mx) {
+    case kOperandsMxfp8: return dispatch_gemm<kOperandsMxfp8>(tmA, tmB, p, BN, head_dim, num_sms, s);
+    case kOperandsNvfp4: return dispatch_gemm<kOperandsNvfp4>(tmA, tmB, p, BN, head_dim, num_sms, s);
+    default: return dispatch_gemm<kOperandsBf16>(tmA, tmB, p, BN, head_dim, num_sms, s);
   }
-  if (BN == 256) {
-    switch (p.epi) {
-      case kEpiStoreF32: return launch_impl<256, 128, kEpiStoreF32>(tmA, tmB, p, num_sms, s);
-      case kEpiSwiGLU: return launch_impl<256, 128, kEpiSwiGLU>(tmA, tmB, p, num_sms, s);
-      case kEpiQKVG:
-        if (p.k_splits != 1) return cudaErrorInvalidValue;
-        if (head_dim == 128) return launch_impl<256, 128, kEpiQKVG>(tmA, tmB, p, num_sms, s);
-        if (head_dim == 64) return launch_impl<256, 64, kEpiQKVG>(tmA, tmB, p, num_sms, s);
-        return cudaErrorInvalidValue;
-    }
-  } else if (BN == 128) {
-    switch (p.epi) {
-      case kEpiStoreF32: return launch_impl<128, 128, kEpiStoreF32>(tmA, tmB, p, num_sms, s);
-      case kEpiSwiGLU: return launch_impl<128, 128, kEpiSwiGLU>(tmA, tmB, p, num_sms, s);
-      case kEpiQKVG:
-        if (p.k_splits != 1) return cudaErrorInvalidValue;
-        if (head_dim == 128) return launch_impl<128, 128, kEpiQKVG>(tmA, tmB, p, num_sms, s);
-        if (head_dim == 64) return launch_impl<128, 64, kEpiQKVG>(tmA, tmB, p, num_sms, s);
-        return cudaErrorInvalidValue;
-    }
-  }
-  return cudaErrorInvalidValue;
 }
 
 }  // namespace dory

@@ -38,14 +38,22 @@ struct GemmParams {
   const float2* rope = nullptr;      // [M][hd/2] (cos, sin) of each row's angles, this layer's base
   float norm_eps = 1e-20f;
   uint32_t* status = nullptr;
-  // MXFP8 operands (mx != 0): A and B tensor maps are over E4M3 codes
-  // (make_tmap_u8) and sfa / sfb hold their E8M0 scales in the chunked layout
-  // of quant.cu with sfa_blocks = ceil(M / 128), sfb_blocks = ceil(N / 128)
+  // Block-scaled operands: mx = kOperandsMxfp8 (A and B tensor maps over E4M3
+  // codes, make_tmap_u8; sfa / sfb their E8M0 scales in 512-byte chunks per
+  // (128 rows, 128 K)) or kOperandsNvfp4 (maps over packed E2M1 codes, K / 2
+  // bytes per row; sfa / sfb their E4M3 scales in 2048-byte chunks per (128
+  // rows, 256 K)), with sfa_blocks = ceil(M / 128), sfb_blocks = 128-row
+  // blocks of B's scale layout
   int mx = 0;
   const uint8_t* sfa = nullptr;
   const uint8_t* sfb = nullptr;
   int sfa_blocks = 0, sfb_blocks = 0;
+  // every accumulator is multiplied by alpha before the epilogue uses it (the
+  // product of the two NVFP4 tensor scales; 1 otherwise)
+  float alpha = 1.f;
 };
+
+enum { kOperandsBf16 = 0, kOperandsMxfp8 = 1, kOperandsNvfp4 = 2 };
 
 // Encode a 2D tensor map for a row-major uint8 matrix [rows, cols] (MXFP8
 // codes) with a (128 x box_rows) box and the 128-byte swizzle.
@@ -66,6 +74,25 @@ cudaError_t launch_quant_mxfp8_bf16(const __nv_bfloat16* const* segs, const int*
                                     cudaStream_t s);
 cudaError_t launch_quant_mxfp8_f32(const float* src, int rows, int K, int normalize, float norm_eps,
                                    uint8_t* codes, uint8_t* scales, cudaStream_t s);
+
+// NVFP4 quantisation along K (see quant.cu): packed E2M1 codes [rows, K / 2]
+// (element 2i in the low nibble of byte i), E4M3 block scales (blocks of 16)
+// in 2048-byte chunks of (128 rows, 256 K), given the fp32 tensor scale g
+// (`d_g` on the device when not null, else `g`).  Sources and padding as for
+// MXFP8 (padding rows get scale 1.0); K must be a multiple of 256.
+size_t nvfp4_scale_bytes(int rows, int K, int row_align = 128);
+cudaError_t launch_quant_nvfp4_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
+                                    int n_seg, int group, int rows, int row_align, int K,
+                                    int normalize, float norm_eps, const float* d_g, float g,
+                                    uint8_t* codes, uint8_t* scales, cudaStream_t s);
+cudaError_t launch_quant_nvfp4_f32(const float* src, int rows, int K, int normalize, float norm_eps,
+                                   const float* d_g, float g, uint8_t* codes, uint8_t* scales,
+                                   cudaStream_t s);
+// The NVFP4 tensor scale of a group of bf16 matrices quantised with one scale:
+// g = amax / (6 * 448) over all their elements (1 when all are zero), written
+// to d_g.  d_amax is a 4-byte scratch word.
+cudaError_t launch_nvfp4_tensor_scale(const __nv_bfloat16* const* mats, const size_t* counts, int n,
+                                      uint32_t* d_amax, float* d_g, cudaStream_t s);
 
 // Encode a 2D tensor map for a row-major bf16 matrix [rows, cols] with a
 // (64 x box_rows) box and the 128-byte swizzle.  Returns false on failure.

@@ -16,8 +16,25 @@
 // Rows past `rows` (up to the next multiple of 128, or of 256 for weights read
 // as 256-row tiles) get scale code 127 (1.0), so the MMA never multiplies the
 // zero-filled padding by an undefined scale.
+//
+// NVFP4 (same page, the NVFP4 release): blocks of 16 consecutive values along
+// K share an E4M3 scale s = E4M3(amax_block / (6 g)) under a per-tensor fp32
+// scale g; each value becomes the E2M1 code nearest to x / (s g) (ties to
+// even, saturating at 6).  Both decisions are taken in float64 on exact
+// quantities: the scale from a correctly rounded quotient (no E4M3 tie lies
+// within its rounding error), the element by comparing |x| with the seven
+// midpoints of the E2M1 grid times s g, all exact in float64, so the codes are
+// those of the exact rational rounding.  Codes are packed two per byte
+// (element 2i in the low nibble); scales go in 2048-byte chunks, one per (128
+// rows, 256 K): chunk (kc, rb) at ((kc * row_blocks) + rb) * 2048, and inside
+// it the scale of row r = rb*128 + 32*j + i and 16-block b (0..15) at byte
+// (b / 4) * 512 + i*16 + j*4 + b % 4, i.e. four 512-byte pieces, one per
+// 64-K MMA, each laid out like an MXFP8 chunk with the four bytes of a word
+// being the word's four 16-blocks.
 #include <cuda_fp8.h>
 #include <string.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -152,7 +169,205 @@ cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ NVFP4
+
+// E4M3 value nearest to v >= 0 (ties to even, saturating at 448) and its code.
+__device__ __forceinline__ uint32_t e4m3_round(double v, double& val) {
+  if (!(v > 0.0)) { val = 0.0; return 0u; }
+  if (v >= 448.0) { val = 448.0; return 0x7Eu; }
+  int ex;
+  frexp(v, &ex);                                   // v = f 2^ex, f in [0.5, 1)
+  const int e = max(ex - 1, -6);                   // binade; subnormals share 2^-6's grid
+  const double ulp = ldexp(1.0, e - 3);
+  const double n = rint(v / ulp);                  // exact scaling, then half-even
+  val = n * ulp;
+  if (val == 0.0) return 0u;
+  int ex2;
+  frexp(val, &ex2);
+  const int e2 = ex2 - 1;
+  if (e2 < -6) return static_cast<uint32_t>(val * 512.0);        // subnormal: mantissa only
+  const uint32_t mant = static_cast<uint32_t>((ldexp(val, -e2) - 1.0) * 8.0);
+  return (static_cast<uint32_t>(e2 + 7) << 3) | mant;
+}
+
+// E2M1 code of x for the block's unit T = s g: the magnitude code counts the
+// grid midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (times T) that |x| passes,
+// a midpoint going to the even neighbour (0, 1, 1, 2, 2, 4, 4).
+__device__ __forceinline__ uint32_t e2m1_code(float x, double T) {
+  const double a = fabs(static_cast<double>(x));
+  const uint32_t m = (a > 0.25 * T) + (a >= 0.75 * T) + (a > 1.25 * T) + (a >= 1.75 * T) +
+                     (a > 2.5 * T) + (a >= 3.5 * T) + (a > 5.0 * T);
+  return m | (signbit(x) ? 8u : 0u);
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int kNvUnroll = 4;   // 256-value steps whose loads are in flight together
+
+// One warp per (padded) row.  Lane l holds values 8l..8l+7 of each 256 of the
+// row; lanes 2b and 2b+1 share 16-block b (amax by one shuffle).
+template <typename T>
+__global__ void __launch_bounds__(32 * kQuantWarps)
+    quant_nvfp4_kernel(const QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
+                       int normalize, float norm_eps, const float* __restrict__ d_g, float g_host,
+                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (r >= rows_pad) return;                      // warp-uniform
+  const T* row = r < rows ? source_row(src, r, K) : nullptr;
+  const double g = static_cast<double>(d_g ? *d_g : g_host);
+  const double six_g = 6.0 * g;                   // exact: g has 24 significant bits
+  float inv = 1.f;
+  if (normalize && row) {
+    float ss = 0.f;
+    for (int base = 0; base < K; base += 256 * kNvUnroll) {
+      float v[kNvUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kNvUnroll; ++u) {
+        const int k0 = base + u * 256 + lane * 8;
+        if (k0 < K) load8(row + k0, v[u]);
+        else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kNvUnroll; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(v[u][i], v[u][i], ss);
+    }
+    inv = rsqrtf(fmaxf(warp_sum(ss), norm_eps));
+  }
+  const int rb = r / 128, rr = r % 128;
+  uint8_t* srow = scales + static_cast<size_t>(rb) * 2048 + (rr % 32) * 16 + (rr / 32) * 4;
+  for (int base = 0; base < K; base += 256 * kNvUnroll) {
+    float v[kNvUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int k0 = base + u * 256 + lane * 8;
+      if (row && k0 < K) load8(row + k0, v[u]);
+      else
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      if (base + u * 256 >= K) break;             // warp-uniform (K is a multiple of 256)
+      const int k0 = base + u * 256 + lane * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[u][i] *= inv;
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      double sval;
+      const uint32_t scode = e4m3_round(static_cast<double>(amax) / six_g, sval);
+      const int b = (k0 % 256) / 16;              // 16-block within the 256
+      if ((lane & 1) == 0)
+        srow[static_cast<size_t>(k0 / 256) * row_blocks * 2048 + (b / 4) * 512 + (b % 4)] =
+            static_cast<uint8_t>(row ? scode : 0x38u);
+      if (!row) continue;
+      uint32_t word = 0;
+      if (sval > 0.0) {
+        const double unit = sval * g;             // exact: 4 x 24 significant bits
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= e2m1_code(v[u][i], unit) << (4 * i);
+      }
+      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * (K / 2) + k0 / 2) = word;
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_quant_nv(const QuantSrc<T>& src, int rows, int row_align, int K, int normalize,
+                            float norm_eps, const float* d_g, float g, uint8_t* codes,
+                            uint8_t* scales, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (K % 256 != 0 || (row_align != 128 && row_align != 256)) return cudaErrorInvalidValue;
+  if (!d_g && !(g > 0.f)) return cudaErrorInvalidValue;
+  const int rows_pad = (rows + row_align - 1) / row_align * row_align;
+  const int row_blocks = rows_pad / 128;
+  quant_nvfp4_kernel<T><<<(rows_pad + kQuantWarps - 1) / kQuantWarps, 32 * kQuantWarps, 0, s>>>(
+      src, rows, rows_pad, K, row_blocks, normalize, norm_eps, d_g, g, codes, scales);
+  return cudaGetLastError();
+}
+
+// amax of |x| over n bf16 values, as the bits of a non-negative float (their
+// order as unsigned integers is the order of the values)
+__global__ void amax_bf16_kernel(const __nv_bfloat16* __restrict__ x, size_t n,
+                                 uint32_t* __restrict__ amax) {
+  float m = 0.f;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    m = fmaxf(m, fabsf(__bfloat162float(x[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax, __float_as_uint(m));
+}
+
+// g = amax / (6 * 448): the quotient rounded to float64, then to fp32
+__global__ void tensor_scale_kernel(const uint32_t* amax, float* g) {
+  const float a = __uint_as_float(*amax);
+  *g = a > 0.f ? static_cast<float>(static_cast<double>(a) / 2688.0) : 1.f;
+}
+
 }  // namespace
+
+size_t nvfp4_scale_bytes(int rows, int K, int row_align) {
+  return static_cast<size_t>((rows + row_align - 1) / row_align * (row_align / 128)) * (K / 256) *
+         2048;
+}
+
+cudaError_t launch_quant_nvfp4_bf16(const __nv_bfloat16* const* segs, const int* seg_rows,
+                                    int n_seg, int group, int rows, int row_align, int K,
+                                    int normalize, float norm_eps, const float* d_g, float g,
+                                    uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+  if (n_seg < 1 || n_seg > 4 || (group > 0 && n_seg != 2)) return cudaErrorInvalidValue;
+  QuantSrc<__nv_bfloat16> q;
+  memset(&q, 0, sizeof(q));
+  for (int i = 0; i < n_seg; ++i) {
+    q.seg[i] = segs[i];
+    q.seg_row[i] = seg_rows ? seg_rows[i] : 0;
+  }
+  q.seg_row[n_seg] = rows;
+  q.n_seg = n_seg;
+  q.group = group;
+  return launch_quant_nv(q, rows, row_align, K, normalize, norm_eps, d_g, g, codes, scales, s);
+}
+
+cudaError_t launch_quant_nvfp4_f32(const float* src, int rows, int K, int normalize, float norm_eps,
+                                   const float* d_g, float g, uint8_t* codes, uint8_t* scales,
+                                   cudaStream_t s) {
+  QuantSrc<float> q;
+  memset(&q, 0, sizeof(q));
+  q.seg[0] = src;
+  q.seg_row[1] = rows;
+  q.n_seg = 1;
+  return launch_quant_nv(q, rows, 128, K, normalize, norm_eps, d_g, g, codes, scales, s);
+}
+
+cudaError_t launch_nvfp4_tensor_scale(const __nv_bfloat16* const* mats, const size_t* counts, int n,
+                                      uint32_t* d_amax, float* d_g, cudaStream_t s) {
+  if (n < 1 || !d_amax || !d_g) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(d_amax, 0, sizeof(uint32_t), s);
+  for (int i = 0; i < n && e == cudaSuccess; ++i) {
+    if (counts[i] == 0) continue;
+    const size_t blocks = std::min<size_t>((counts[i] + 255) / 256, 4096);
+    amax_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(mats[i], counts[i], d_amax);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return e;
+  tensor_scale_kernel<<<1, 1, 0, s>>>(d_amax, d_g);
+  return cudaGetLastError();
+}
 
 size_t mxfp8_scale_bytes(int rows, int K, int row_align) {
   return static_cast<size_t>((rows + row_align - 1) / row_align * (row_align / 128)) * (K / 128) * 512;

@@ -287,6 +287,32 @@ def gemm_mxfp8(A, Bm, k_splits=1, stream=None):
     return C
 
 
+def quant_nvfp4(x, g=None, stream=None):
+    """NVFP4 packed codes [rows, K/2] (uint8), the chunked E4M3 scale bytes and
+    the tensor scale (a 1-element fp32 device tensor) of bf16 rows x; g None
+    takes the tensor scale from the data (amax / (6 * 448))."""
+    rows, K = x.shape
+    codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(B.dory_nvfp4_scale_bytes(rows, K), dtype=torch.uint8, device=x.device)
+    d_g = torch.full((1,), float(g) if g is not None else 0.0, dtype=torch.float32,
+                     device=x.device)
+    B.dory_quant_nvfp4(_ptr(x), rows, K, float(g) if g is not None else 0.0, _ptr(d_g),
+                       _ptr(codes), _ptr(scales), _stream(stream))
+    return codes, scales, d_g
+
+
+def gemm_nvfp4(A, Bm, g_a, g_b, k_splits=1, stream=None):
+    """Q(A) Q(Bm)^T through the NVFP4 block-scaled GEMM (bf16 in, tensor scales
+    g_a and g_b, fp32 out) as its K slices [k_splits, M, N]."""
+    M, K = A.shape
+    N = Bm.shape[0]
+    ws = torch.empty(B.dory_gemm_nvfp4_workspace_bytes(M, N, K), dtype=torch.uint8, device=A.device)
+    C = torch.empty(k_splits, M, N, dtype=torch.float32, device=A.device)
+    B.dory_gemm_nvfp4(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, float(g_a), float(g_b), k_splits,
+                      _ptr(ws), ws.numel(), _stream(stream))
+    return C
+
+
 def gemm_bf16(A, Bm, stream=None):
     """C = A @ Bm^T through the library's tcgen05 GEMM (bf16 in, fp32 out)."""
     M, K = A.shape
