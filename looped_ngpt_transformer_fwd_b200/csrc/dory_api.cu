@@ -369,6 +369,9 @@ struct CallCtx {
   int k;                 // loops run (the largest per-row count when dk is set)
   const int32_t* dk = nullptr;   // decode: per-row loop counts, or null
   cudaStream_t s;
+  // block-scaled modes: the last row update already wrote the stream's codes
+  // and scales into the projection-input buffer (w.x8 / w.xsf)
+  bool h_quantized = false;
 };
 
 #define DORY_TRY(expr)                         \
@@ -438,7 +441,9 @@ cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const _
     return cudaSuccess;
   }
   const bool nv = m->mx == kOperandsNvfp4;
-  {
+  const bool ready = f32 && c.h_quantized;   // the row kernel quantised the stream already
+  c.h_quantized = false;                     // any other input overwrites the buffer
+  if (!ready) {
     Launch L(m, c.s, DORY_KK_ROW);
     const float eps = m->cfg.norm_eps;
     const int nrm = normalize ? 1 : 0;
@@ -463,6 +468,19 @@ cudaError_t projection_input(CallCtx& c, CUtensorMap* tm, GemmParams& g, const _
   g.sfa_blocks = (c.n + 127) / 128;
   g.alpha = nv ? kNvfp4ActScale : 1.f;
   return cudaSuccess;
+}
+
+// Let a row update quantise its result for the next projection (the stream
+// is the input of the QKVG and gate / up projections), sparing a pass of the
+// stand-alone quantiser.  Not with per-row loop counts: rows whose loops are
+// done are skipped and would keep stale codes.
+void fuse_stream_quant(CallCtx& c, RowUpdateParams& r) {
+  if (!c.m->mx || c.dk) return;
+  r.q_fmt = c.m->mx;
+  r.q_codes = c.w.x8;
+  r.q_scales = c.w.xsf;
+  r.q_row_blocks = (c.n + 127) / 128;
+  r.q_g = kNvfp4ActScale;
 }
 
 // B operand (weights) of the block-scaled GEMMs: scale chunks and their row
@@ -631,10 +649,12 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
   r.rows = c.n; r.d = m->d; r.y = c.w.y; r.splits = go.k_splits; r.split_stride = go.split_stride;
   r.h = h; r.hb = hb; r.alpha = W.alpha_attn; r.norm_eps = m->cfg.norm_eps;
   r.row_k = W.recurrent ? c.dk : nullptr; r.loop = loop; r.k_hi = c.k; r.status = m->status;
+  fuse_stream_quant(c, r);
   {
     Launch L(m, c.s, DORY_KK_ROW);
     DORY_TRY(launch_row_update(r, c.s));
   }
+  c.h_quantized = r.q_fmt != 0;
   ++c.m->cur_sublayers;
   return cudaSuccess;
 }
@@ -716,10 +736,12 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   r.e = reinject ? c.w.e32 : nullptr;
   r.out = out;
   r.row_k = W.recurrent ? c.dk : nullptr; r.loop = loop; r.k_hi = c.k; r.status = m->status;
+  fuse_stream_quant(c, r);
   {
     Launch L(m, c.s, DORY_KK_ROW);
     DORY_TRY(launch_row_update(r, c.s));
   }
+  c.h_quantized = r.q_fmt != 0;
   ++c.m->cur_sublayers;
   return cudaSuccess;
 }

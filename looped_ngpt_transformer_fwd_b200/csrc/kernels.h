@@ -176,6 +176,18 @@ struct RowUpdateParams {
   const int32_t* row_k = nullptr;
   int loop = 0, k_hi = 0;
   uint32_t* status = nullptr;
+  // optional: the final rows quantised for the next projection, exactly as
+  // launch_quant_mxfp8_f32 / launch_quant_nvfp4_f32 would (q_fmt
+  // kOperandsMxfp8 or kOperandsNvfp4; codes [rows, d] or [rows, d / 2], scale
+  // chunks over q_row_blocks = ceil(rows / 128) row blocks, NVFP4 tensor scale
+  // q_g).  The scales of the padding rows of the last block are left as they
+  // are: they only reach accumulator rows that are never stored.  Not with
+  // row_k (skipped rows would keep stale codes).
+  int q_fmt = 0;
+  uint8_t* q_codes = nullptr;
+  uint8_t* q_scales = nullptr;
+  int q_row_blocks = 0;
+  float q_g = 0.f;
 };
 cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s);
 

@@ -20,11 +20,10 @@
 // NVFP4 (same page, the NVFP4 release): blocks of 16 consecutive values along
 // K share an E4M3 scale s = E4M3(amax_block / (6 g)) under a per-tensor fp32
 // scale g; each value becomes the E2M1 code nearest to x / (s g) (ties to
-// even, saturating at 6).  Both decisions are taken in float64 on exact
-// quantities: the scale from a correctly rounded quotient (no E4M3 tie lies
-// within its rounding error), the element by comparing |x| with the seven
-// midpoints of the E2M1 grid times s g, all exact in float64, so the codes are
-// those of the exact rational rounding.  Codes are packed two per byte
+// even, saturating at 6).  Both decisions are exact (blockscale.cuh): the
+// scale from a quotient rounded once to float64, the element by the exact sign
+// of |x| minus each E2M1 midpoint times s g, so the codes are those of the
+// exact rational rounding.  Codes are packed two per byte
 // (element 2i in the low nibble); scales go in 2048-byte chunks, one per (128
 // rows, 256 K): chunk (kc, rb) at ((kc * row_blocks) + rb) * 2048, and inside
 // it the scale of row r = rb*128 + 32*j + i and 16-block b (0..15) at byte
@@ -36,6 +35,7 @@
 
 #include <algorithm>
 
+#include "blockscale.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -78,17 +78,6 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
 constexpr int kQuantWarps = 8;      // rows per CTA (one warp per row)
 constexpr int kQuantUnroll = 8;     // 128-value steps whose loads are in flight together
 
-// Block scale exponent floor(log2 amax) - 8 from the float's exponent field
-// (a subnormal amax gives -135, clamped like any value below 2^-119 to -127),
-// and the exact power of two 2^-sexp that maps the block into E4M3 range.
-__device__ __forceinline__ int block_exponent(float amax) {
-  if (!(amax > 0.f)) return -127;
-  const int e = ((__float_as_int(amax) >> 23) & 0xFF) - 127;
-  return min(127, max(-127, e - 8));
-}
-__device__ __forceinline__ float pow2_neg(int sexp) {   // sexp in [-127, 119]: a normal float
-  return __int_as_float((127 - sexp) << 23);
-}
 
 // One warp per (padded) row.  Lane l holds values 4l..4l+3 of each 128 of the
 // row (coalesced loads and stores); the 8 lanes of a group of 8 hold one block
@@ -140,19 +129,15 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
       // the normalised values' amax (a uniform positive scale commutes with max)
-      const int sexp = block_exponent(amax * inv);
+      const int sexp = mx_block_exponent(amax * inv);
       const int q32 = k0 / 32;
       if ((lane & 7) == 0)
         srow[static_cast<size_t>(q32 / 4) * row_blocks * 512 + (q32 % 4)] =
             static_cast<uint8_t>(row ? sexp + 127 : 127);
       if (!row) continue;
-      const float f = inv * pow2_neg(sexp);
-      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-          make_float2(v[u][0] * f, v[u][1] * f), __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(v[u][2] * f, v[u][3] * f), __NV_SATFINITE, __NV_E4M3);
+      const float f = inv * mx_pow2_neg(sexp);
       *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * K + k0) =
-          static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+          mx_codes4(v[u][0], v[u][1], v[u][2], v[u][3], f);
     }
   }
 }
@@ -170,35 +155,6 @@ cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K,
 }
 
 // ------------------------------------------------------------------ NVFP4
-
-// E4M3 value nearest to v >= 0 (ties to even, saturating at 448) and its code.
-__device__ __forceinline__ uint32_t e4m3_round(double v, double& val) {
-  if (!(v > 0.0)) { val = 0.0; return 0u; }
-  if (v >= 448.0) { val = 448.0; return 0x7Eu; }
-  int ex;
-  frexp(v, &ex);                                   // v = f 2^ex, f in [0.5, 1)
-  const int e = max(ex - 1, -6);                   // binade; subnormals share 2^-6's grid
-  const double ulp = ldexp(1.0, e - 3);
-  const double n = rint(v / ulp);                  // exact scaling, then half-even
-  val = n * ulp;
-  if (val == 0.0) return 0u;
-  int ex2;
-  frexp(val, &ex2);
-  const int e2 = ex2 - 1;
-  if (e2 < -6) return static_cast<uint32_t>(val * 512.0);        // subnormal: mantissa only
-  const uint32_t mant = static_cast<uint32_t>((ldexp(val, -e2) - 1.0) * 8.0);
-  return (static_cast<uint32_t>(e2 + 7) << 3) | mant;
-}
-
-// E2M1 code of x for the block's unit T = s g: the magnitude code counts the
-// grid midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (times T) that |x| passes,
-// a midpoint going to the even neighbour (0, 1, 1, 2, 2, 4, 4).
-__device__ __forceinline__ uint32_t e2m1_code(float x, double T) {
-  const double a = fabs(static_cast<double>(x));
-  const uint32_t m = (a > 0.25 * T) + (a >= 0.75 * T) + (a > 1.25 * T) + (a >= 1.75 * T) +
-                     (a > 2.5 * T) + (a >= 3.5 * T) + (a > 5.0 * T);
-  return m | (signbit(x) ? 8u : 0u);
-}
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
   const uint4 u = *reinterpret_cast<const uint4*>(p);
@@ -224,8 +180,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
   if (r >= rows_pad) return;                      // warp-uniform
   const T* row = r < rows ? source_row(src, r, K) : nullptr;
-  const double g = static_cast<double>(d_g ? *d_g : g_host);
-  const double six_g = 6.0 * g;                   // exact: g has 24 significant bits
+  const float g = d_g ? *d_g : g_host;
   float inv = 1.f;
   if (normalize && row) {
     float ss = 0.f;
@@ -268,18 +223,17 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
       amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      double sval;
-      const uint32_t scode = e4m3_round(static_cast<double>(amax) / six_g, sval);
+      const NvScale sc = nv_block_scale(amax, g);
       const int b = (k0 % 256) / 16;              // 16-block within the 256
       if ((lane & 1) == 0)
         srow[static_cast<size_t>(k0 / 256) * row_blocks * 2048 + (b / 4) * 512 + (b % 4)] =
-            static_cast<uint8_t>(row ? scode : 0x38u);
+            static_cast<uint8_t>(row ? sc.code : 0x38u);
       if (!row) continue;
       uint32_t word = 0;
-      if (sval > 0.0) {
-        const double unit = sval * g;             // exact: 4 x 24 significant bits
+      if (sc.s > 0.f) {
+        const NvThresholds th = nv_thresholds(sc.s);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= e2m1_code(v[u][i], unit) << (4 * i);
+        for (int i = 0; i < 8; ++i) word |= nv_code(v[u][i], th, g) << (4 * i);
       }
       *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * (K / 2) + k0 / 2) = word;
     }

@@ -8,6 +8,7 @@
 //   - input staging (bf16 -> fp32 stream + bf16 GEMM operand);
 //   - KV-cache commits of fresh keys/values into their slots (ring slots
 //     pos % window for sliding-window layers, pos for full layers).
+#include "blockscale.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,6 +32,46 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 
 __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+}
+
+// Quantise float4 chunk c (values 4c..4c+3) of row r for the next projection.
+// The chunks of one scale block sit in consecutive lanes of one warp (4 for
+// an NVFP4 block of 16, 8 for an MXFP8 block of 32), and every lane of the
+// warp holds a valid chunk or none does, so the block amax is a few shuffles.
+__device__ __forceinline__ void quant_chunk(const RowUpdateParams& p, int r, int c,
+                                            const float4& v) {
+  const int rb = r / 128, rr = r % 128;
+  float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  if (p.q_fmt == kOperandsNvfp4) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    const NvScale sc = nv_block_scale(amax, p.q_g);
+    uint32_t word = 0;
+    if (sc.s > 0.f) {
+      const NvThresholds th = nv_thresholds(sc.s);
+      word = nv_code(v.x, th, p.q_g) | (nv_code(v.y, th, p.q_g) << 4) |
+             (nv_code(v.z, th, p.q_g) << 8) | (nv_code(v.w, th, p.q_g) << 12);
+    }
+    reinterpret_cast<uint16_t*>(p.q_codes + static_cast<size_t>(r) * (p.d / 2))[c] =
+        static_cast<uint16_t>(word);
+    if ((c & 3) == 0) {
+      const int b16 = c / 4, kc = b16 / 16, b = b16 % 16;
+      p.q_scales[(static_cast<size_t>(kc) * p.q_row_blocks + rb) * 2048 + (b / 4) * 512 +
+                 (rr % 32) * 16 + (rr / 32) * 4 + (b % 4)] = static_cast<uint8_t>(sc.code);
+    }
+  } else {
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const int sexp = mx_block_exponent(amax);
+    reinterpret_cast<uint32_t*>(p.q_codes + static_cast<size_t>(r) * p.d)[c] =
+        mx_codes4(v.x, v.y, v.z, v.w, mx_pow2_neg(sexp));
+    if ((c & 7) == 0) {
+      const int q32 = c / 8;
+      p.q_scales[static_cast<size_t>(rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4 +
+                 static_cast<size_t>(q32 / 4) * p.q_row_blocks * 512 + (q32 % 4)] =
+          static_cast<uint8_t>(sexp + 127);
+    }
+  }
 }
 
 // Three block reductions per row (||y||, ||h'||, ||h_new + e||), with y and h
@@ -115,6 +156,7 @@ __global__ void row_update_kernel(const RowUpdateParams p) {
       const uint2 b = make_uint2(pack_bf16x2(h[j].x, h[j].y), pack_bf16x2(h[j].z, h[j].w));
       if (p.hb) reinterpret_cast<uint2*>(p.hb + row_off)[c] = b;
       if (p.out) reinterpret_cast<uint2*>(p.out + row_off)[c] = b;
+      if (p.q_fmt) quant_chunk(p, r, c, h[j]);   // warp-uniform (c < nch is)
     }
   }
 }
@@ -268,6 +310,10 @@ cudaError_t launch_swiglu_post(const float* part, int splits, size_t split_strid
 
 cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s) {
   if (p.d % 4 != 0 || p.rows < 0) return cudaErrorInvalidValue;
+  if (p.q_fmt && (p.row_k || !p.q_codes || !p.q_scales || p.d % 128 != 0 ||
+                  (p.q_fmt == kOperandsNvfp4 && (p.d % 256 != 0 || !(p.q_g > 0.f))) ||
+                  p.q_row_blocks < (p.rows + 127) / 128))
+    return cudaErrorInvalidValue;
   if (p.rows == 0) return cudaSuccess;
   int threads = (p.d / 4 + kRowMaxChunks - 1) / kRowMaxChunks;
   threads = ((threads + 31) / 32) * 32;
