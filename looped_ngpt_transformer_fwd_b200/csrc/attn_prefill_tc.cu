@@ -15,11 +15,16 @@
 // online-softmax kernel.
 //
 // Persistent: one CTA per SM works through (128-query tile, head) items dealt
-// longest first in snake order; 128-key K/V tiles.  Warp 0 issues TMA loads:
-// Q tiles into two slots (the next item's Q lands while this one runs), K
-// tiles through a 2-slot ring and V tiles through a 3-slot ring (from the
-// layer's cache for positions below pos0, from this call's fresh K/V
-// otherwise).  Warp 1 owns TMEM and issues S = Q K^T (N = 128 keys) into one of
+// longest first in snake order; 128-key K/V tiles aligned to absolute
+// positions.  Warp 0 loads: Q tiles into two slots (the next item's Q lands
+// while this one runs), K tiles through a 2-slot ring and V tiles through a
+// 3-slot ring, by TMA from the layer's cache for positions below pos0 and
+// from this call's fresh K/V otherwise.  A key tile that no single box
+// covers -- one holding both cached and fresh keys (pos0 not a multiple of
+// 128), or a cached tile that runs past the end of a sliding-window ring
+// (window not a multiple of 128, or below 128) -- is gathered row by row by
+// the whole warp with cp.async into the same swizzled layout, positions that
+// do not exist (below 0, at or past pos0 + n) as zeros.  Warp 1 owns TMEM and issues S = Q K^T (N = 128 keys) into one of
 // three 128-column buffers; warp 18 issues O += P V with the A operand (P)
 // read from TMEM, where the softmax warps wrote it over S.  Two issuing
 // threads keep the two dependency chains apart: a wait in one (for P, or for
@@ -69,6 +74,47 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Key tile [kp0, kp0 + 128) of KV head kvh (K, or V when `v`) gathered into a
+// ring slot by the 32 lanes of the calling warp, in the layout a TMA box of 64
+// dims x 128 rows with the 128-byte swizzle writes: two 64-dim sub-tiles,
+// 16-byte chunk c of row r at chunk c ^ (r % 8) of the row's 128 bytes.
+// Positions below pos0 come from the cache (ring slot pos % cap), the others
+// from this call's rows; positions below 0 or at or past pos0 + n are zeros
+// (they are masked, and a zero V row adds nothing to P V).  On return the
+// slot's bytes are visible to the tensor cores (async proxy).
+__device__ void gather_kv_tile(uint8_t* dst, const PrefillAttnTcParams& p, int kvh, int kp0,
+                               bool v, int lane) {
+  const __nv_bfloat16* fresh = v ? p.v_new : p.k_new;
+  const size_t plane =
+      static_cast<size_t>(p.seq * 2 * p.n_kv + (v ? p.n_kv : 0) + kvh) * static_cast<size_t>(p.cap);
+  for (int idx = lane; idx < kKT * 16; idx += 32) {
+    const int r = idx >> 4, c = idx & 15;
+    const int pos = kp0 + r;
+    uint8_t* d = dst + (c >> 3) * kSub + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    const __nv_bfloat16* src = nullptr;
+    if (pos >= 0 && pos < p.pos0)
+      src = p.cache + (plane + static_cast<size_t>(pos % p.cap)) * kHD + c * 8;
+    else if (pos >= p.pos0 && pos - p.pos0 < p.n)
+      src = fresh + (static_cast<size_t>(pos - p.pos0) * p.n_kv + kvh) * kHD + c * 8;
+    if (src)
+      cp_async16(d, src);
+    else
+      *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_wait_all();
+  fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+  __syncwarp();
 }
 
 // Descriptor of the MN-major B operand (V, dims contiguous): SW128 atoms of
@@ -235,86 +281,112 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------- TMA producer
-      bool ok = true;
-      int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0;
-      // parity of the last copy into each slot, for draining after an error
-      uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
-      uint32_t q_issued = 0, q_par = 0;
-      Item it;
-      for (int k = 0; ok && get_item(p, k, it); ++k) {
-        const int kvh = it.head / group_size;
-        // Q slot k % 2 is free once every S MMA of item k - 2 has completed
-        const int qs = k & 1;
-        const uint32_t qph = (k >> 1) & 1u;
-        if (!mbar_wait_bounded(&q_empty[qs], qph ^ 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
+    // --------------------------------------------------------- loads (warp 0)
+    // Lane 0 waits on the rings and issues the TMA copies; the whole warp
+    // gathers the tiles no box covers.  Wait results are broadcast from lane 0,
+    // so the warp stays converged.
+    bool ok = true;
+    int ks = 0, vs = 0;
+    uint32_t kph = 0, vph = 0;
+    // parity of the last TMA copy into each slot, for draining after an error
+    uint32_t k_issued = 0, v_issued = 0, k_par = 0, v_par = 0;
+    uint32_t q_issued = 0, q_par = 0;
+    Item it;
+    auto lane0_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      bool w = true;
+      if (lane == 0) w = mbar_wait_bounded(bar, parity, abort_flag, p.status);
+      return __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
+    };
+    for (int k = 0; ok && get_item(p, k, it); ++k) {
+      const int kvh = it.head / group_size;
+      // Q slot k % 2 is free once every S MMA of item k - 2 has completed
+      const int qs = k & 1;
+      const uint32_t qph = (k >> 1) & 1u;
+      if (!lane0_wait(&q_empty[qs], qph ^ 1u)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
         uint8_t* qd = smem + kOffQ + qs * kSlotBytes;
         mbar_arrive_expect_tx(&q_full[qs], kSlotBytes);
         tma_load_3d(qd, &tmQ, &q_full[qs], 0, it.head, it.m0);
         tma_load_3d(qd + kSub, &tmQ, &q_full[qs], 64, it.head, it.m0);
-        q_issued |= 1u << qs;
-        q_par = (q_par & ~(1u << qs)) | (qph << qs);
-        for (int j = 0; j < it.n_tiles; ++j) {
-          const int kp0 = (it.kt_begin + j) * kKT;
-          // cached positions: slot rows of this sequence's K and V planes
-          const bool cached = kp0 < p.pos0;
-          const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + (cached ? kp0 % p.cap : 0);
-          const int vrow = krow + p.n_kv * p.cap;
-          const int t0 = kp0 - p.pos0;
-          if (!mbar_wait_bounded(&k_empty[ks], kph ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* kd = smem + kOffK + ks * kSlotBytes;
-          mbar_arrive_expect_tx(&k_full[ks], kSlotBytes);
-          if (cached) {
-            tma_load_2d(kd, &tmCache, &k_full[ks], 0, krow);
-            tma_load_2d(kd + kSub, &tmCache, &k_full[ks], 64, krow);
-          } else {
-            tma_load_3d(kd, &tmKnew, &k_full[ks], 0, kvh, t0);
-            tma_load_3d(kd + kSub, &tmKnew, &k_full[ks], 64, kvh, t0);
+      }
+      q_issued |= 1u << qs;
+      q_par = (q_par & ~(1u << qs)) | (qph << qs);
+      for (int j = 0; j < it.n_tiles; ++j) {
+        const int kp0 = (it.kt_begin + j) * kKT;
+        // wholly cached tiles: slot rows of this sequence's K and V planes
+        const bool cached = kp0 + kKT <= p.pos0;
+        const int slot = cached ? kp0 % p.cap : 0;
+        const bool gather = (kp0 < p.pos0 && !cached) || (cached && slot + kKT > p.cap);
+        const int krow = (p.seq * 2 * p.n_kv + kvh) * p.cap + slot;
+        const int vrow = krow + p.n_kv * p.cap;
+        const int t0 = kp0 - p.pos0;
+        if (!lane0_wait(&k_empty[ks], kph ^ 1u)) {
+          ok = false;
+          break;
+        }
+        uint8_t* kd = smem + kOffK + ks * kSlotBytes;
+        if (gather) {
+          gather_kv_tile(kd, p, kvh, kp0, false, lane);
+          if (lane == 0) mbar_arrive(&k_full[ks]);
+          k_issued &= ~(1u << ks);   // nothing in flight
+        } else {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&k_full[ks], kSlotBytes);
+            if (cached) {
+              tma_load_2d(kd, &tmCache, &k_full[ks], 0, krow);
+              tma_load_2d(kd + kSub, &tmCache, &k_full[ks], 64, krow);
+            } else {
+              tma_load_3d(kd, &tmKnew, &k_full[ks], 0, kvh, t0);
+              tma_load_3d(kd + kSub, &tmKnew, &k_full[ks], 64, kvh, t0);
+            }
           }
           k_issued |= 1u << ks;
           k_par = (k_par & ~(1u << ks)) | (kph << ks);
-          if (++ks == kKSlots) {
-            ks = 0;
-            kph ^= 1u;
-          }
-          if (!mbar_wait_bounded(&v_empty[vs], vph ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* vd = smem + kOffV + vs * kSlotBytes;
-          mbar_arrive_expect_tx(&v_full[vs], kSlotBytes);
-          if (cached) {
-            tma_load_2d(vd, &tmCache, &v_full[vs], 0, vrow);
-            tma_load_2d(vd + kSub, &tmCache, &v_full[vs], 64, vrow);
-          } else {
-            tma_load_3d(vd, &tmVnew, &v_full[vs], 0, kvh, t0);
-            tma_load_3d(vd + kSub, &tmVnew, &v_full[vs], 64, kvh, t0);
+        }
+        if (++ks == kKSlots) {
+          ks = 0;
+          kph ^= 1u;
+        }
+        if (!lane0_wait(&v_empty[vs], vph ^ 1u)) {
+          ok = false;
+          break;
+        }
+        uint8_t* vd = smem + kOffV + vs * kSlotBytes;
+        if (gather) {
+          gather_kv_tile(vd, p, kvh, kp0, true, lane);
+          if (lane == 0) mbar_arrive(&v_full[vs]);
+          v_issued &= ~(1u << vs);
+        } else {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&v_full[vs], kSlotBytes);
+            if (cached) {
+              tma_load_2d(vd, &tmCache, &v_full[vs], 0, vrow);
+              tma_load_2d(vd + kSub, &tmCache, &v_full[vs], 64, vrow);
+            } else {
+              tma_load_3d(vd, &tmVnew, &v_full[vs], 0, kvh, t0);
+              tma_load_3d(vd + kSub, &tmVnew, &v_full[vs], 64, kvh, t0);
+            }
           }
           v_issued |= 1u << vs;
           v_par = (v_par & ~(1u << vs)) | (vph << vs);
-          if (++vs == kVSlots) {
-            vs = 0;
-            vph ^= 1u;
-          }
+        }
+        if (++vs == kVSlots) {
+          vs = 0;
+          vph ^= 1u;
         }
       }
-      if (!ok) {
-        // let the copies already in flight land before the CTA exits
-        for (int s = 0; s < kQSlots; ++s)
-          if (q_issued & (1u << s)) drain_wait(&q_full[s], (q_par >> s) & 1u);
-        for (int s = 0; s < kKSlots; ++s)
-          if (k_issued & (1u << s)) drain_wait(&k_full[s], (k_par >> s) & 1u);
-        for (int s = 0; s < kVSlots; ++s)
-          if (v_issued & (1u << s)) drain_wait(&v_full[s], (v_par >> s) & 1u);
-      }
+    }
+    if (!ok && lane == 0) {
+      // let the copies already in flight land before the CTA exits
+      for (int s = 0; s < kQSlots; ++s)
+        if (q_issued & (1u << s)) drain_wait(&q_full[s], (q_par >> s) & 1u);
+      for (int s = 0; s < kKSlots; ++s)
+        if (k_issued & (1u << s)) drain_wait(&k_full[s], (k_par >> s) & 1u);
+      for (int s = 0; s < kVSlots; ++s)
+        if (v_issued & (1u << s)) drain_wait(&v_full[s], (v_par >> s) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -594,9 +666,9 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, 
 }  // namespace
 
 bool prefill_attention_tc_supported(int head_dim, int pos0, int window, float m_log2) {
-  if (head_dim != kHD || pos0 % kKT != 0) return false;
-  if (window > 0 && window % kKT != 0) return false;
-  return 2.f * m_log2 < 120.f;
+  (void)pos0;     // any chunk start: tiles across pos0 are gathered
+  (void)window;   // any window: ring tiles across the ring's end are gathered
+  return head_dim == kHD && 2.f * m_log2 < 120.f;
 }
 
 cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv_bfloat16* q,
@@ -630,6 +702,13 @@ cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv
   dim3 grid(items < dev_sms ? items : dev_sms);
   PrefillAttnTcParams pq = p;
   pq.q = q;
+  pq.k_new = k_new;
+  pq.v_new = v_new;
+  pq.cache = kv.k_base;
+  // gathered rows are 16-byte copies
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
+       reinterpret_cast<uintptr_t>(kv.k_base)) & 15)
+    return cudaErrorInvalidValue;
   if (p.probe)
     prefill_attn_tc_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, pq);
   else

@@ -251,6 +251,12 @@ struct PrefillAttnTcParams {
   float scale_log2 = 0.f, m_log2 = 0.f;
   uint32_t* status = nullptr;
   int32_t* probe = nullptr;             // mask probe records [n, Hq, 4], or null
+  // set by the launcher: this call's K / V [n, Hkv, hd] and the layer's cache
+  // (K plane of (seq, head) at rows (seq * 2 * Hkv + head) * cap, V planes
+  // after the Hkv K planes), read directly for key tiles gathered row by row
+  const __nv_bfloat16* k_new = nullptr;
+  const __nv_bfloat16* v_new = nullptr;
+  const __nv_bfloat16* cache = nullptr;
 };
 bool prefill_attention_tc_supported(int head_dim, int pos0, int window, float m_log2);
 cudaError_t launch_prefill_attention_tc(const PrefillAttnTcParams& p, const __nv_bfloat16* q,

@@ -7,8 +7,9 @@ those records bit for bit with the set of visible keys that the oracle's mask
 rule gives (causal; a sliding-window layer sees the last W positions including
 the query's own: "Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
 English), for every attention kernel of the library:
-  * tcgen05 prefill attention (head_dim 128, pos0 and window multiples of 128),
-  * mma.sync prefill attention (head_dim 64, or unaligned pos0 / window),
+  * tcgen05 prefill attention (head_dim 128, any chunk start and window:
+    key tiles across the chunk start or a ring's end are gathered row by row),
+  * mma.sync prefill attention (head_dim 64),
   * TMA-fed decode attention (head_dim 128, window a multiple of 64),
   * cp.async decode attention (head_dim 64, or another window),
 at windows 1, 4, 100, 128 and 4096, aligned and unaligned chunk starts, and
@@ -73,8 +74,7 @@ def expected_paths(cfg, a, decode):
         if decode:
             kinds.add("decode_tma" if hd == 128 and (full or W % 64 == 0) else "decode_cp")
         else:
-            kinds.add("prefill_tc" if hd == 128 and a % 128 == 0 and (full or W % 128 == 0)
-                      else "prefill_mma")
+            kinds.add("prefill_tc" if hd == 128 else "prefill_mma")
     return kinds
 
 
@@ -112,9 +112,9 @@ def scenario(model, cfg, chunks, decode_positions, max_ctx, layers=(0, 1)):
 
 @pytest.mark.parametrize("window", [128, 4096])
 def test_masks_head_dim_128_tensor_core_paths(window):
-    """Aligned chunks run the tcgen05 prefill kernel, decode the TMA kernel; with
-    W = 128 the later chunks read a wrapped ring; an unaligned chunk runs the
-    mma.sync kernel."""
+    """Every chunk runs the tcgen05 prefill kernel (the unaligned ones gather the
+    key tile across their start), decode the TMA kernel; with W = 128 the later
+    chunks read a wrapped ring."""
     cfg, _, model = build("tiny", seed=3, variant="random", window=window, **SMALL128)
     if window == 128:
         chunks, dec, ctx = [(0, 384), (384, 640), (640, 661), (661, 700)], [700, 701, 765], 800
@@ -127,11 +127,12 @@ def test_masks_head_dim_128_tensor_core_paths(window):
 
 @pytest.mark.parametrize("window", [1, 4, 100])
 def test_masks_head_dim_128_other_windows(window):
-    """Windows that are not a multiple of 128 (prefill: mma.sync kernel) nor of 64
-    (decode: cp.async kernel); the full layers keep the tensor-core paths."""
+    """Windows that are not a multiple of 128 nor of 64: prefill stays on the
+    tcgen05 kernel (ring tiles that run past the ring's end are gathered), decode
+    runs the cp.async kernel; the full layers keep the TMA decode path."""
     cfg, _, model = build("tiny", seed=4, variant="random", window=window, **SMALL128)
     seen = scenario(model, cfg, [(0, 256), (256, 300), (300, 512)], [512, 513], 600)
-    assert seen == {"prefill_tc", "prefill_mma", "decode_tma", "decode_cp"}
+    assert seen == {"prefill_tc", "decode_tma", "decode_cp"}
     model.close()
 
 

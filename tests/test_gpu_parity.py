@@ -249,8 +249,9 @@ def test_kernel_profiling_counts_every_launch(tiny):
 
 # ------------------------------------------------------------------ head_dim 128
 # (d 512, 4/2 heads of 128, window 128): prefill attention runs on the tcgen05
-# kernel whenever pos0 and the window are multiples of 128, else on the
-# mma.sync kernel; both must match the oracle.
+# kernel at any chunk start and window (key tiles across the chunk start or a
+# ring's end gathered row by row), on the mma.sync online-softmax kernel when
+# the static softmax maximum would underflow; both must match the oracle.
 HD128 = dict(d_model=512, n_q_heads=4, n_kv_heads=2, head_dim=128, d_ff=1024, window=128,
              softmax_scale=float(np.sqrt(128.0)))
 
@@ -278,7 +279,8 @@ def test_hd128_prefill_matches_oracle(hd128, mode, k):
 @pytest.mark.parametrize("k", [2, 4])
 def test_hd128_chunked_prefill_and_decode(hd128, mode, k):
     """Chunks at multiples of 128 (tensor-core attention reading cached tiles and
-    ring slots), unaligned chunks (mma.sync kernel), then decode steps."""
+    ring slots), unaligned chunks (the same kernel, gathering the key tile that
+    holds both cached and fresh keys), then decode steps."""
     cfg, prov, model = hd128
     x, h = inputs(cfg, 52, 420)
     kv = model.kv_cache(mode, 2, 480, k_max=k)
@@ -288,6 +290,8 @@ def test_hd128_chunked_prefill_and_decode(hd128, mode, k):
     for a, b in ((0, 128), (128, 256), (256, 384), (384, 405), (405, 416)):
         out = model.prefill(kv, x[a:b], k, seq=seq, pos0=a)
         torch.cuda.synchronize()
+        paths = model.attention_paths()
+        assert paths["prefill_tc"] > 0 and paths["prefill_mma"] == 0, (a, paths)
         ref = orc.forward(h[a:b], a, k, ocache, seq=seq)
         assert_parity(to_np(out), ref, what=f"hd128 chunk {a}:{b} {mode}")
     for p in range(416, 420):
@@ -297,6 +301,81 @@ def test_hd128_chunked_prefill_and_decode(hd128, mode, k):
         ref = orc.decode(h[p:p + 1], [seq], [p], k, ocache)
         assert_parity(to_np(out), ref, what=f"hd128 decode {p} {mode}")
     assert model.device_status() == 0
+
+
+def _alpha_one_model(cfg, seed, sqk=None):
+    """A model and its weight provider with alpha_attn = 1 (and optionally every
+    s_qk entry set to `sqk`), in the generator's storage format."""
+    from tests.oracle_util import modified
+    from oracle import weights_from_generator
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from synthetic import f32_to_bf16_bits
+    base = weights_from_generator(cfg, seed, "random")
+
+    def change(b, w):
+        w["alpha_attn"][:] = 1.0
+        if sqk is not None:
+            w["s_qk"][:] = sqk
+    prov = modified(base, change)
+
+    def as_generator_format(b):
+        w = prov(b)
+        return {k_: (v.astype(np.float32) if k_ in ("alpha_attn", "alpha_mlp", "s_qk")
+                     else f32_to_bf16_bits(v.astype(np.float32))) for k_, v in w.items()}
+    return DoryModel(cfg, as_generator_format), as_generator_format
+
+
+@pytest.mark.parametrize("window", [100, 128])
+def test_hd128_unaligned_chunks_alpha_one_on_tensor_cores(window):
+    """Chunks starting off the 128-key tile grid, and a window that is not a
+    multiple of 128 (ring tiles that run past the ring's end), on the tcgen05
+    kernel with alpha = 1: the attention output is compared almost undiluted,
+    so a wrong row in a gathered key tile would show."""
+    from synthetic import load_config
+    cfg = load_config("tiny", **dict(HD128, window=window))
+    model, prov = _alpha_one_model(cfg, 9)
+    _, h = inputs(cfg, 54, 460)
+    kv = model.kv_cache("last_loop", 1, 512)
+    ocache = oracle_cache(cfg, "last_loop")
+    orc = oracle(cfg, prov)
+    for layer in (0, 1):                        # SWA, full
+        for pos0, n in ((0, 200), (200, 57), (257, 130), (387, 73)):
+            ht = torch.from_numpy(h[pos0:pos0 + n].astype(np.float32)).cuda()
+            model.attention_sublayer(kv, layer, ht, loop=1, seq=0, pos0=pos0)
+            torch.cuda.synchronize()
+            paths = model.attention_paths()
+            assert paths["prefill_tc"] > 0 and paths["prefill_mma"] == 0, paths
+            ref = orc.attention_sublayer(layer, h[pos0:pos0 + n], pos0, 0, 1, ocache)
+            assert_parity(to_np(ht), ref, tol_abs=1e-2, tol_cos=0.99995,
+                          what=f"alpha=1 W={window} layer {layer} @{pos0}")
+    assert model.device_status() == 0
+    model.close()
+
+
+def test_hd128_large_sqk_runs_the_online_softmax_kernel():
+    """s_qk = 3 everywhere bounds the logits by softmax_scale * 9 ~ 102, too wide
+    for the static softmax maximum (2 B log2(e) > 120), so prefill attention runs
+    the mma.sync online-softmax kernel, aligned and unaligned chunks alike.  At
+    logits near 100 the bf16 rounding of q and k (2^-9 relative) moves an
+    exponent by up to ~0.2, so this case's bar is cos >= 0.999."""
+    from synthetic import load_config
+    cfg = load_config("tiny", **HD128)
+    model, prov = _alpha_one_model(cfg, 10, sqk=3.0)
+    _, h = inputs(cfg, 55, 300)
+    kv = model.kv_cache("last_loop", 1, 320)
+    ocache = oracle_cache(cfg, "last_loop")
+    orc = oracle(cfg, prov)
+    for pos0, n in ((0, 128), (128, 77), (205, 95)):
+        ht = torch.from_numpy(h[pos0:pos0 + n].astype(np.float32)).cuda()
+        model.attention_sublayer(kv, 1, ht, loop=1, seq=0, pos0=pos0)
+        torch.cuda.synchronize()
+        paths = model.attention_paths()
+        assert paths["prefill_mma"] > 0 and paths["prefill_tc"] == 0, paths
+        ref = orc.attention_sublayer(1, h[pos0:pos0 + n], pos0, 0, 1, ocache)
+        assert_parity(to_np(ht), ref, tol_abs=2e-2, tol_cos=0.999,
+                      what=f"online softmax @{pos0}")
+    assert model.device_status() == 0
+    model.close()
 
 
 @pytest.mark.parametrize("layer", [0, 1])      # SWA (W = 128), full
