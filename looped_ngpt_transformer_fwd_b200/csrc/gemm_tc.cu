@@ -330,11 +330,37 @@ __device__ __forceinline__ void epi_swiglu(const GemmParams& p, uint32_t taddr, 
   }
 }
 
+// 32 fp32 values per lane to TMEM columns taddr..taddr+31 (this warp's lanes),
+// then wait until they are written.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
+      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
+      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
+      "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // One head-sized column group (HD columns starting at global column col0).
 // q and k heads get RoPE, the per-head L2 norm and the scale s_qk (`sqk`, in
 // shared memory); v heads are stored as computed; gate logits go through the
-// sigmoid.  With bulk stores (p.c_tma) the warp stages 64-column boxes of q,
-// k or v and every lane takes part, rows past M included (the maps clip them).
+// sigmoid.  q / k take two passes over the accumulator columns, which this
+// warp owns until it releases the buffer: the first rotates 32 pairs (i,
+// i + HD/2) at a time, adds their squares and writes them back, the second
+// scales by s_qk / ||.|| and stores, so no more than 64 values are live.  The
+// RoPE table is pair-major ([HD/2][M]): for one pair the 32 lanes (32
+// consecutive rows) read 256 contiguous bytes.  With bulk stores (p.c_tma) the
+// warp stages 64-column boxes of q, k or v and every lane takes part, rows past
+// M included (the maps clip them).  TMEM accesses are warp-collective: every
+// lane runs them, whatever its row.
 template <int HD, bool kAlpha>
 __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float* sqk,
                                                const OutMaps* om, uint8_t* stage, int lane,
@@ -344,76 +370,87 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
   const int q_end = hq * HD, k_end = q_end + hkv * HD, v_end = k_end + hkv * HD;
   const bool tma = p.c_tma != 0;
   const bool row_ok = row < p.M;
-  float x[HD];
-#pragma unroll
-  for (int c = 0; c < HD; c += 32) {
-    float t[32];
-    tmem_ld32(taddr + c, t);
-    apply_alpha<kAlpha>(t, p.alpha);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[c + i] = t[i];
-  }
   if (col0 >= v_end) {
     // attention output gate logits, one per query head (col0 is warp-uniform)
-    if (!row_ok) return;
     float* g = p.gate_out + static_cast<size_t>(row) * hq;
+#pragma unroll 1
+    for (int c = 0; c < HD && col0 - v_end + c < hq; c += 32) {
+      float t[32];
+      tmem_ld32(taddr + c, t);
+      apply_alpha<kAlpha>(t, p.alpha);
+      if (!row_ok) continue;
 #pragma unroll
-    for (int i = 0; i < HD; ++i) {
-      const int j = col0 - v_end + i;
-      if (j < hq) g[j] = sigmoidf_(x[i]);
+      for (int i = 0; i < 32; ++i) {
+        const int j = col0 - v_end + c + i;
+        if (j < hq) g[j] = sigmoidf_(t[i]);
+      }
     }
     return;
   }
-  if (!tma && !row_ok) return;
   int which, head;
-  if (col0 < k_end) {
-    // RoPE (pairs i, i + HD/2) with this row's (cos, sin) table, then the
-    // per-head L2 norm and the learned per-dimension scale s_qk.  Rows past M
-    // read the last valid row's table (their results are clipped).
+  float inv = 1.f;
+  const bool qk = col0 < k_end;
+  if (qk) {
+    // rows past M read the last valid row's angles (their results are clipped)
     const int trow = row_ok ? row : p.M - 1;
-    const float4* rt = reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(trow) * (HD / 2));
-#pragma unroll
-    for (int i = 0; i < HD / 2; i += 2) {
-      const float4 cs = rt[i / 2];   // cos_i, sin_i, cos_{i+1}, sin_{i+1}
-      const float a0 = x[i], b0 = x[i + HD / 2];
-      const float a1 = x[i + 1], b1 = x[i + 1 + HD / 2];
-      x[i] = a0 * cs.x - b0 * cs.y;
-      x[i + HD / 2] = b0 * cs.x + a0 * cs.y;
-      x[i + 1] = a1 * cs.z - b1 * cs.w;
-      x[i + 1 + HD / 2] = b1 * cs.z + a1 * cs.w;
-    }
     float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < HD / 2; c += 32) {
+      float a[32], b[32];
+      tmem_ld32(taddr + c, a);
+      tmem_ld32(taddr + c + HD / 2, b);
+      apply_alpha<kAlpha>(a, p.alpha);
+      apply_alpha<kAlpha>(b, p.alpha);
+      const float2* rt = p.rope + static_cast<size_t>(c) * p.M + trow;
 #pragma unroll
-    for (int i = 0; i < HD; ++i) ss = fmaf(x[i], x[i], ss);
-    const float inv = rsqrtf(fmaxf(ss, p.norm_eps));
-#pragma unroll
-    for (int i = 0; i < HD; ++i) x[i] *= inv * sqk[i];
+      for (int u = 0; u < 32; ++u) {
+        const float2 cs = rt[static_cast<size_t>(u) * p.M];   // cos_i, sin_i of pair c + u
+        const float a2 = a[u] * cs.x - b[u] * cs.y;
+        const float b2 = b[u] * cs.x + a[u] * cs.y;
+        ss = fmaf(a2, a2, fmaf(b2, b2, ss));
+        a[u] = a2;
+        b[u] = b2;
+      }
+      tmem_st32(taddr + c, a);
+      tmem_st32(taddr + c + HD / 2, b);
+    }
+    tmem_wait_st();
+    inv = rsqrtf(fmaxf(ss, p.norm_eps));
     which = col0 < q_end ? 0 : 1;
     head = col0 < q_end ? col0 / HD : (col0 - q_end) / HD;
   } else {
     which = 2;
     head = (col0 - k_end) / HD;
   }
-  if (tma) {
-#pragma unroll
-    for (int half = 0; half < HD / 64; ++half) {
-      uint32_t wb[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) wb[i] = pack_bf16x2(x[64 * half + 2 * i], x[64 * half + 2 * i + 1]);
-      store_box_bf16(&om->m[which], stage, lane, nbuf, wb, head * HD + 64 * half, row0);
-    }
-    return;
-  }
   const int nh = which == 0 ? hq : hkv;
   __nv_bfloat16* base = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out);
-  uint4* d4 = reinterpret_cast<uint4*>(base + (static_cast<size_t>(row) * nh + head) * HD);
+#pragma unroll 1
+  for (int half = 0; half < HD / 64; ++half) {
+    uint32_t wb[32];
 #pragma unroll
-  for (int i = 0; i < HD / 8; ++i)
-    d4[i] = make_uint4(pack_bf16x2(x[8 * i], x[8 * i + 1]), pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
-                       pack_bf16x2(x[8 * i + 4], x[8 * i + 5]),
-                       pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
+    for (int cc = 0; cc < 64; cc += 32) {
+      float t[32];
+      tmem_ld32(taddr + 64 * half + cc, t);
+      if (qk) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) t[u] *= inv * sqk[64 * half + cc + u];
+      } else {
+        apply_alpha<kAlpha>(t, p.alpha);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) wb[cc / 2 + u] = pack_bf16x2(t[2 * u], t[2 * u + 1]);
+    }
+    if (tma) {
+      store_box_bf16(&om->m[which], stage, lane, nbuf, wb, head * HD + 64 * half, row0);
+    } else if (row_ok) {
+      uint4* d4 = reinterpret_cast<uint4*>(base + (static_cast<size_t>(row) * nh + head) * HD +
+                                           64 * half);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        d4[i] = make_uint4(wb[4 * i], wb[4 * i + 1], wb[4 * i + 2], wb[4 * i + 3]);
+    }
+  }
 }
-
 
 template <int BN, int HD, int EPI, int MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)

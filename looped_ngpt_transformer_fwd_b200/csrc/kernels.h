@@ -35,7 +35,7 @@ struct GemmParams {
   float* gate_out = nullptr;        // [M, Hq]
   int n_q_heads = 0, n_kv_heads = 0;
   const float* s_qk = nullptr;       // [hd]
-  const float2* rope = nullptr;      // [M][hd/2] (cos, sin) of each row's angles, this layer's base
+  const float2* rope = nullptr;      // [hd/2][M] (cos, sin) of each row's angles (pair-major), this layer's base
   float norm_eps = 1e-20f;
   uint32_t* status = nullptr;
   // Block-scaled operands: mx = kOperandsMxfp8 (A and B tensor maps over E4M3
@@ -124,7 +124,7 @@ int ngpt_gemm_cols_per_cta(int d_model);
 cudaError_t launch_gemm_ngpt(const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const NgptGemmParams& p, cudaStream_t s);
 
-// RoPE (cos, sin) table [rows][hd/2] for row r at position pos0 + r (or
+// RoPE (cos, sin) table, pair-major [hd/2][rows], for row r at position pos0 + r (or
 // d_pos[r]): angle = pos * inv_freq[i] in float64, reduced mod 2*pi, then
 // sincosf.
 cudaError_t launch_rope_table(const double* inv_freq, int hd, int rows, int pos0,

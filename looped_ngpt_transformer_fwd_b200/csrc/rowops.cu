@@ -210,9 +210,10 @@ constexpr double kTwoPi = 6.283185307179586476925286766559;
 __global__ void rope_table_kernel(const double* __restrict__ inv_freq, int half, int rows,
                                   int pos0, const int32_t* __restrict__ d_pos,
                                   float2* __restrict__ out) {
+  // pair-major: entry (pair i, row r) at i * rows + r
   const int id = blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= rows * half) return;
-  const int r = id / half, i = id % half;
+  const int i = id / rows, r = id % rows;
   const int pos = d_pos ? d_pos[r] : pos0 + r;
   const double ang = static_cast<double>(pos) * inv_freq[i];
   const double turns = rint(ang * (1.0 / kTwoPi));
@@ -245,7 +246,7 @@ __global__ void qkvg_post_kernel(const QkvgPostParams p) {
   }
   const bool is_v = g >= p.n_q_heads + p.n_kv_heads;
   if (!is_v) {
-    const float2 cs = p.rope[static_cast<size_t>(r) * half + i];
+    const float2 cs = p.rope[static_cast<size_t>(i) * p.rows + r];
     const float a2 = a * cs.x - b * cs.y;
     const float b2 = b * cs.x + a * cs.y;
     const float inv = rsqrtf(fmaxf(block_sum(a2 * a2 + b2 * b2, red), p.norm_eps));
