@@ -723,6 +723,8 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   gd.k_splits = c.decode ? pick_k_splits(m, c.n, m->d, bn_d, m->ff) : 1;
   gd.out_f32 = c.w.y; gd.ld_out = m->d; gd.split_stride = size_t(c.n) * m->d;
   gd.status = m->status;
+  // the activations (rows x d_ff) outweigh W_down (d x d_ff) once rows > d
+  gd.raster_n = c.n > m->d ? 1 : 0;
   {
     Launch L(m, c.s, DORY_KK_DOWN);
     const CUtensorMap& tb = m->mx ? (bn_d == 256 ? W.tm8_d_256 : W.tm8_d) : W.tm_d[bn_d == 256];

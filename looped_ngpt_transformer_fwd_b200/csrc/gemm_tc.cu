@@ -452,6 +452,29 @@ __device__ __forceinline__ void epi_qkvg_group(const GemmParams& p, const float*
   }
 }
 
+// Tile t of the persistent loop: K split outermost; inside it the M tiles
+// vary fastest (raster_n = 0: the B panel stays while the A panels stream,
+// for a small A) or the N tiles do (raster_n = 1: a wave covers few A panels
+// and every B panel, which stay in L2 together when A is the larger operand).
+struct TileCoord {
+  int mt, nt, ks;
+};
+__device__ __forceinline__ TileCoord tile_coord(int t, int m_tiles, int n_tiles, int raster_n) {
+  TileCoord c;
+  if (raster_n) {
+    c.nt = t % n_tiles;
+    const int rest = t / n_tiles;
+    c.mt = rest % m_tiles;
+    c.ks = rest / m_tiles;
+  } else {
+    c.mt = t % m_tiles;
+    const int rest = t / m_tiles;
+    c.nt = rest % n_tiles;
+    c.ks = rest / n_tiles;
+  }
+  return c;
+}
+
 template <int BN, int HD, int EPI, int MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -518,10 +541,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const int mt = t % m_tiles;
-        const int rest = t / m_tiles;
-        const int nt = rest % n_tiles;
-        const int ks = rest / n_tiles;
+        const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+        const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
         const int kb0 = ks * kb_per_split;
         const int kb1 = min(kb_total, kb0 + kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -569,8 +590,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const int rest = t / m_tiles;
-        const int ks = rest / n_tiles;
+        const int ks = tile_coord(t, m_tiles, n_tiles, p.raster_n).ks;
         const int kb0 = ks * kb_per_split;
         const int kb1 = min(kb_total, kb0 + kb_per_split);
         const int acc = it % C::kAccBufs;
@@ -654,10 +674,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t nbuf = 0;                 // staged boxes so far (buffer rotation)
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const int mt = t % m_tiles;
-      const int rest = t / m_tiles;
-      const int nt = rest % n_tiles;
-      const int ks = rest / n_tiles;
+      const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+      const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
       const int acc = it % C::kAccBufs;
       const uint32_t aph = (it / C::kAccBufs) & 1;
       // warp-uniform: the TMEM loads below are warp-collective

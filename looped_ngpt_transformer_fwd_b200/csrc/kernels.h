@@ -51,6 +51,9 @@ struct GemmParams {
   // every accumulator is multiplied by alpha before the epilogue uses it (the
   // product of the two NVFP4 tensor scales; 1 otherwise)
   float alpha = 1.f;
+  // order of the persistent tile loop: 0 = M tiles fastest, 1 = N tiles
+  // fastest (keeps a wave's A panels and all of B in L2 when A is larger)
+  int raster_n = 0;
 };
 
 enum { kOperandsBf16 = 0, kOperandsMxfp8 = 1, kOperandsNvfp4 = 2 };
