@@ -1,0 +1,79 @@
+"""Pins of the oracle's MLP-sublayer backward (oracle/backward.py).
+
+Truncated back-propagation of depth one trains only the final recurrent
+invocation ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
+English); its sublayers' gradients are derivatives of the forward.  Pinned
+against things other than the chain rule it writes out:
+  * central finite differences of L = <dh_out, h_out> in every input and
+    parameter (float64, step 1e-6);
+  * the forward it differentiates is the oracle's MLP sublayer;
+  * an output gradient along h_out changes nothing (h_out is a unit vector, so
+    L cannot move with its length): every gradient vanishes;
+  * gate_scale enters SiLU's argument (a different gate_scale changes dWg).
+"""
+
+import numpy as np
+import pytest
+
+from oracle import Oracle, weights_from_generator
+from oracle.backward import mlp_sublayer_backward, mlp_sublayer_forward
+from synthetic import load_config, hidden_in
+from synthetic.bf16 import bf16_bits_to_f32
+
+
+def _setup(seed=3, rows=5, **over):
+    cfg = load_config("tiny", **over)
+    prov = weights_from_generator(cfg, seed, "random")
+    raw = prov(1)
+    W = {k: (bf16_bits_to_f32(v).astype(np.float64) if v.dtype == np.uint16
+             else np.asarray(v, dtype=np.float64)) for k, v in raw.items()}
+    h = bf16_bits_to_f32(hidden_in(cfg, seed + 1, rows)).astype(np.float64)
+    rng = np.random.default_rng(seed + 2)
+    dh_out = rng.standard_normal(h.shape)
+    return cfg, prov, W, h, dh_out
+
+
+def _loss(cfg, W, h, dh_out):
+    return float((mlp_sublayer_forward(cfg, W, h)["h_out"] * dh_out).sum())
+
+
+def test_forward_is_the_oracle_mlp_sublayer():
+    cfg, prov, W, h, _ = _setup()
+    ref = Oracle(cfg, prov).mlp_sublayer(1, h)
+    assert np.allclose(mlp_sublayer_forward(cfg, W, h)["h_out"], ref, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("name", ["h", "w_gate", "w_up", "w_down", "alpha_mlp"])
+def test_gradients_match_central_differences(name):
+    cfg, _, W, h, dh_out = _setup(d_model=128, n_q_heads=2, d_ff=256)
+    g = mlp_sublayer_backward(cfg, W, h, dh_out)
+    grad = {"h": g["dh"], "w_gate": g["d_w_gate"], "w_up": g["d_w_up"], "w_down": g["d_w_down"],
+            "alpha_mlp": g["d_alpha"]}[name]
+    rng = np.random.default_rng(7)
+    eps = 1e-6
+    target = h if name == "h" else W[name]
+    idx = [tuple(rng.integers(0, n) for n in target.shape) for _ in range(12)]
+    for ix in idx:
+        old = target[ix]
+        target[ix] = old + eps
+        lp = _loss(cfg, W, h, dh_out)
+        target[ix] = old - eps
+        lm = _loss(cfg, W, h, dh_out)
+        target[ix] = old
+        fd = (lp - lm) / (2 * eps)
+        assert abs(fd - grad[ix]) <= 1e-6 * max(1.0, abs(fd)), (name, ix, fd, grad[ix])
+
+
+def test_gradient_along_the_output_vanishes():
+    cfg, _, W, h, _ = _setup()
+    h_out = mlp_sublayer_forward(cfg, W, h)["h_out"]
+    g = mlp_sublayer_backward(cfg, W, h, 3.0 * h_out)
+    for k in ("dh", "d_w_gate", "d_w_up", "d_w_down", "d_alpha"):
+        assert np.abs(g[k]).max() < 1e-12, k
+
+
+def test_gate_scale_reaches_the_gate_gradient():
+    cfg, _, W, h, dh_out = _setup()
+    g1 = mlp_sublayer_backward(cfg, W, h, dh_out)["d_w_gate"]
+    g2 = mlp_sublayer_backward(dict(cfg, gate_scale=2.0), W, h, dh_out)["d_w_gate"]
+    assert np.abs(g1 - g2).max() > 1e-3 * np.abs(g1).max()
