@@ -329,6 +329,33 @@ DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
  * all row-major device buffers, K a multiple of 64, N a multiple of 128. */
 DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
 
+/* The same GEMM with operands read transposed (MN-major): A is stored row-major
+ * as [M][K] (a_mn = 0) or [K][M] (a_mn = 1), B as [N][K] (b_mn = 0) or [K][N]
+ * (b_mn = 1); C[M,N] = A B^T in fp32.  Any K (rounded up inside, the tail read
+ * as zeros); N a multiple of 128; the contiguous dimension of each operand a
+ * multiple of 8 (16-byte rows).  The backward's dgrad (dX = dY W) and wgrad
+ * (dW = dY^T X) products. */
+DORY_API int dory_gemm_bf16_mn(const void* A, const void* B, float* C, int M, int N, int K,
+                               int a_mn, int b_mn, void* stream);
+
+/* Backward of one MLP sublayer, the building block of the training step that
+ * truncated depth-one back-propagation runs over the final recurrent
+ * invocation ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
+ * English).  Given the sublayer's input h_in [n_rows, d_model] and dL/dh_out
+ * [n_rows, d_model] (fp32, device), recomputes the forward with the inference
+ * path's bf16 operands and writes dL/dh_in [n_rows, d_model], dL/dW_gate and
+ * dL/dW_up [d_ff, d_model], dL/dW_down [d_model, d_ff] (fp32, row-major like
+ * the source matrices) and dL/dalpha_mlp [d_model] (fp32, summed over the
+ * rows, deterministic).  All outputs are overwritten.  `ws`:
+ * dory_mlp_backward_workspace_bytes(m, n_rows), 256-byte aligned; other
+ * buffers 16-byte aligned.  bf16 weight format only (DORY_ERR_BAD_CONFIG
+ * otherwise). */
+DORY_API size_t dory_mlp_backward_workspace_bytes(const dory_model* m, int n_rows);
+DORY_API int dory_mlp_sublayer_backward(dory_model* m, int layer, int n_rows, const float* h_in,
+                                        const float* dh_out, float* dh_in, float* d_w_gate,
+                                        float* d_w_up, float* d_w_down, float* d_alpha, void* ws,
+                                        size_t ws_bytes, void* stream);
+
 /* MXFP8 quantisation along K of bf16 rows src [rows, K] (device, K a multiple
  * of 128): E4M3 codes [rows, K] bytes into `codes`, E8M0 scale codes into
  * `scales` (dory_mxfp8_scale_bytes) in 512-byte chunks, one per 128 rows x

@@ -117,19 +117,6 @@ __device__ void gather_kv_tile(uint8_t* dst, const PrefillAttnTcParams& p, int k
   __syncwarp();
 }
 
-// Descriptor of the MN-major B operand (V, dims contiguous): SW128 atoms of
-// 64 dims x 8 keys; LBO = distance between the two 64-dim sub-tiles, SBO =
-// 1024 B between groups of 8 keys.
-__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint32_t lbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
-  return d;
-}
-
 // tcgen05.mma with the A operand in TMEM (K-major rows = TMEM lanes, two bf16
 // per 32-bit column) and B from shared memory.
 __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,

@@ -195,6 +195,20 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// Descriptor of an MN-major operand (MN contiguous in memory: V in P V, or a
+// matrix read transposed): 128-byte swizzle atoms of 64 MN elements x 8 K
+// rows; LBO = distance between consecutive 64-element MN sub-tiles, SBO =
+// 1024 B between groups of 8 K rows; a 16-K step advances 16 rows (2048 B).
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint32_t lbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B (both
 // K-major), fp32 accumulation, shape M x N.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {

@@ -1353,6 +1353,133 @@ int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h, void* ws, 
   return DORY_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of the MLP-sublayer backward for R rows.
+struct BwdLayout {
+  size_t hb, gu, a, y, dy, da, dgu, dg, du, dhx, part, total;
+  int grid;
+};
+
+BwdLayout bwd_layout(const dory_model* m, int R) {
+  BwdLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  const size_t r = size_t(R), d = m->d, ff = m->ff;
+  L.grid = mlp_bwd_row_grid(R, m->num_sms);
+  L.hb = take(r * d * 2);          // bf16 copy of h (both GEMMs' operand)
+  L.gu = take(r * 2 * ff * 4);     // [g | u] products, packed like W_gu
+  L.a = take(r * ff * 2);          // SwiGLU activations (bf16)
+  L.y = take(r * d * 4);           // down projection
+  L.dy = take(r * d * 2);          // dL/dy (bf16 operand)
+  L.da = take(r * ff * 4);         // dL/da
+  L.dgu = take(r * 2 * ff * 2);    // dL/d[g | u], packed (dgrad operand)
+  L.dg = take(r * ff * 2);         // dL/dg, dL/du (wgrad operands)
+  L.du = take(r * ff * 2);
+  L.dhx = take(r * d * 4);         // dL/dh through the gate / up projection
+  L.part = take(size_t(L.grid) * d * 4);
+  L.total = o;
+  return L;
+}
+
+// C[M, N] (fp32, row pitch N) = op(A) op(B)^T on the tcgen05 GEMM; A is
+// stored [M][K] or, with a_mn, [K][M]; B [N][K] or, with b_mn, [K][N].  K is
+// rounded up to the 64-element step: the maps' K extent is K, so the tail
+// reads zeros.
+cudaError_t gemm_f32(const dory_model* m, const void* A, int a_mn, const void* B, int b_mn,
+                     float* C, int M, int N, int K, cudaStream_t s) {
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap ta, tb;
+  const bool ok = (a_mn ? make_tmap_bf16_mn(&ta, A, K, M) : make_tmap_bf16(&ta, A, M, K, 128)) &&
+                  (b_mn ? make_tmap_bf16_mn(&tb, B, K, N) : make_tmap_bf16(&tb, B, N, K, BN));
+  if (!ok) return cudaErrorInvalidValue;
+  GemmParams p;
+  p.M = M; p.N = N; p.K = (K + 63) / 64 * 64;
+  p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  p.a_mn = a_mn; p.b_mn = b_mn;
+  p.status = m->status;
+  return launch_gemm(ta, tb, p, BN, 128, m->num_sms, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dory_mlp_backward_workspace_bytes(const dory_model* m, int n_rows) {
+  if (!m || n_rows <= 0) return 0;
+  return bwd_layout(m, n_rows).total;
+}
+
+int dory_mlp_sublayer_backward(dory_model* m, int layer, int n_rows, const float* h_in,
+                               const float* dh_out, float* dh_in, float* d_w_gate, float* d_w_up,
+                               float* d_w_down, float* d_alpha, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (!m || !h_in || !dh_out || !dh_in || !d_w_gate || !d_w_up || !d_w_down || !d_alpha || !ws ||
+      n_rows <= 0 || layer < 0 || layer >= m->nb)
+    return DORY_ERR_INVALID_ARG;
+  if (m->mx) return DORY_ERR_BAD_CONFIG;   // bf16 weights only
+  const void* ptrs[8] = {h_in, dh_out, dh_in, d_w_gate, d_w_up, d_w_down, d_alpha, nullptr};
+  for (int i = 0; i < 7; ++i)
+    if (!is_aligned(ptrs[i], 16)) return DORY_ERR_MISALIGNED;
+  if (!is_aligned(ws)) return DORY_ERR_MISALIGNED;
+  const BwdLayout L = bwd_layout(m, n_rows);
+  if (ws_bytes < L.total) return DORY_ERR_BUFFER_TOO_SMALL;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(b + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  const BlockW& W = m->blocks[layer];
+  const int R = n_rows, d = m->d, ff = m->ff;
+  const float eps = m->cfg.norm_eps, gs = m->cfg.gate_scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  // forward again (the same bf16 operands as the inference path)
+  e = e ? e : launch_f32_to_bf16(h_in, bf(L.hb), size_t(R) * d, s);
+  e = e ? e : gemm_f32(m, bf(L.hb), 0, W.wgu, 0, f32(L.gu), R, 2 * ff, d, s);
+  e = e ? e : launch_swiglu_post(f32(L.gu), 1, size_t(R) * 2 * ff, R, ff, gs, 128, bf(L.a), s);
+  e = e ? e : gemm_f32(m, bf(L.a), 0, W.wd, 0, f32(L.y), R, d, ff, s);
+  // the nGPT update's backward: dh (direct part), dL/dy, dalpha partials
+  e = e ? e : launch_mlp_bwd_row(f32(L.y), h_in, W.alpha_mlp, dh_out, R, d, eps, dh_in, bf(L.dy),
+                                 f32(L.part), L.grid, s);
+  // down projection: da = dy W_d (W_d [d][ff] read MN-major), dW_d = dy^T a
+  e = e ? e : gemm_f32(m, bf(L.dy), 0, W.wd, 1, f32(L.da), R, ff, d, s);
+  e = e ? e : gemm_f32(m, bf(L.dy), 1, bf(L.a), 1, d_w_down, d, ff, R, s);
+  // SwiGLU, then the gate / up projection: dh += d[g | u] W_gu, dW_g = dg^T h_b, dW_u = du^T h_b
+  e = e ? e : launch_swiglu_bwd(f32(L.gu), f32(L.da), R, ff, 128, gs, bf(L.dgu), bf(L.dg),
+                                bf(L.du), s);
+  e = e ? e : gemm_f32(m, bf(L.dgu), 0, W.wgu, 1, f32(L.dhx), R, d, 2 * ff, s);
+  e = e ? e : gemm_f32(m, bf(L.dg), 1, bf(L.hb), 1, d_w_gate, ff, d, R, s);
+  e = e ? e : gemm_f32(m, bf(L.du), 1, bf(L.hb), 1, d_w_up, ff, d, R, s);
+  e = e ? e : launch_add_inplace(dh_in, f32(L.dhx), size_t(R) * d, s);
+  e = e ? e : launch_colsum(f32(L.part), L.grid, d, d_alpha, s);
+  return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
+}
+
+int dory_gemm_bf16_mn(const void* A, const void* B, float* C, int M, int N, int K, int a_mn,
+                      int b_mn, void* stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || N % 128) return DORY_ERR_INVALID_ARG;
+  if ((a_mn && M % 8) || (b_mn && N % 8) || (!a_mn && K % 8) || (!b_mn && K % 8))
+    return DORY_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return DORY_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap ta, tb;
+  const bool ok = (a_mn ? make_tmap_bf16_mn(&ta, A, K, M) : make_tmap_bf16(&ta, A, M, K, 128)) &&
+                  (b_mn ? make_tmap_bf16_mn(&tb, B, K, N) : make_tmap_bf16(&tb, B, N, K, BN));
+  if (!ok) return DORY_ERR_CUDA;
+  GemmParams p;
+  p.M = M; p.N = N; p.K = (K + 63) / 64 * 64;
+  p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  p.a_mn = a_mn ? 1 : 0; p.b_mn = b_mn ? 1 : 0;
+  if (launch_gemm(ta, tb, p, BN, 128, sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
+}
+
 int dory_debug_mask_probe(dory_model* m, int layer, int32_t* d_probe, int max_rows) {
   if (!m) return DORY_ERR_INVALID_ARG;
   if (!d_probe) {

@@ -552,8 +552,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* a_dst = tiles + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kLoadBytes);
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKCoord, mt * kBM);
-          tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKCoord, nt * BN);
+          if (MX == kOperandsBf16 && p.a_mn) {
+            // [K][M] source: 64-element M sub-tiles of 64 K rows (8 KB each)
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d(a_dst + j * 8192, &tmA, &full[stage], mt * kBM + 64 * j, kb * kBK);
+          } else {
+            tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKCoord, mt * kBM);
+          }
+          if (MX == kOperandsBf16 && p.b_mn) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(a_dst + C::kABytes + j * 8192, &tmB, &full[stage], nt * BN + 64 * j,
+                          kb * kBK);
+          } else {
+            tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKCoord, nt * BN);
+          }
           if constexpr (MX) {
             // this K step's scale chunks: one for A's 128 rows, BN/128 for B's
             bulk_load(a_dst + C::kABytes + C::kBBytes,
@@ -580,10 +594,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      // MN-major operands (bf16 only): transpose bits 15 (A) and 16 (B), the
+      // MN-major swizzled layout (64-element sub-tiles 8 KB apart), and a
+      // 16-K step of 16 rows (2048 B) instead of 32 bytes within a row
+      const bool a_mn = MX == kOperandsBf16 && p.a_mn, b_mn = MX == kOperandsBf16 && p.b_mn;
+      const uint32_t idesc = umma_idesc_bf16(kBM, BN) | (a_mn ? 1u << 15 : 0u) |
+                             (b_mn ? 1u << 16 : 0u);
       // descriptors built once; a stage or k-step adds (byte offset >> 4)
-      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(tiles));
-      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(tiles + C::kABytes));
+      const uint64_t a_desc0 = a_mn ? umma_desc_sw128_mn(smem_u32(tiles), 8192)
+                                    : umma_desc_sw128(smem_u32(tiles));
+      const uint64_t b_desc0 = b_mn ? umma_desc_sw128_mn(smem_u32(tiles + C::kABytes), 8192)
+                                    : umma_desc_sw128(smem_u32(tiles + C::kABytes));
+      const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -648,8 +670,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              umma_bf16(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4), idesc,
-                        (kb > kb0 || kk > 0) ? 1u : 0u);
+              umma_bf16(d_tmem, a_desc + ((kk * a_step) >> 4), b_desc + ((kk * b_step) >> 4),
+                        idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
             }
           }
           issued = true;
@@ -841,6 +863,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols) {
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode || (mn_cols * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0)
+    return false;
+  cuuint64_t dims[2] = {mn_cols, k_rows};
+  cuuint64_t strides[1] = {mn_cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows) {
   EncodeTiledFn encode = encode_tiled();
@@ -897,8 +933,9 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
     if ((p.k_splits - 1) * per >= kb) return cudaErrorInvalidValue;
   }
   // block-scaled operands need their scales (accumulators and scale columns
-  // share TMEM)
+  // share TMEM); MN-major operands are bf16 only
   if (p.mx && (!p.sfa || !p.sfb)) return cudaErrorInvalidValue;
+  if (p.mx && (p.a_mn || p.b_mn)) return cudaErrorInvalidValue;
   switch (p.mx) {
     case kOperandsMxfp8: return dispatch_gemm<kOperandsMxfp8>(tmA, tmB, p, BN, head_dim, num_sms, s);
     case kOperandsNvfp4: return dispatch_gemm<kOperandsNvfp4>(tmA, tmB, p, BN, head_dim, num_sms, s);

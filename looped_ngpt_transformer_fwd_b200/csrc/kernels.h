@@ -54,7 +54,30 @@ struct GemmParams {
   // order of the persistent tile loop: 0 = M tiles fastest, 1 = N tiles
   // fastest (keeps a wave's A panels and all of B in L2 when A is larger)
   int raster_n = 0;
+  // bf16 operands stored MN-major: A as [K][M] (a_mn) and / or B as [K][N]
+  // (b_mn) row-major, their tensor maps from make_tmap_bf16_mn; the MMAs read
+  // them transposed (the backward's dgrad and wgrad products)
+  int a_mn = 0, b_mn = 0;
 };
+
+// MLP-sublayer backward pieces (backward.cu): the nGPT update's backward
+// (rows spread over `grid` CTAs, each writing its dalpha partial row), the
+// column sum of those partials, the SwiGLU backward (packed and separate
+// gradient layouts) and an in-place add.
+int mlp_bwd_row_grid(int rows, int num_sms);
+cudaError_t launch_mlp_bwd_row(const float* y, const float* h, const float* alpha,
+                               const float* dh_out, int rows, int d, float norm_eps, float* dh,
+                               __nv_bfloat16* dy_b, float* dalpha_part, int grid, cudaStream_t s);
+cudaError_t launch_colsum(const float* part, int groups, int d, float* out, cudaStream_t s);
+cudaError_t launch_swiglu_bwd(const float* gu, const float* da, int rows, int ff, int group,
+                              float gate_scale, __nv_bfloat16* dgu_packed, __nv_bfloat16* dg_sep,
+                              __nv_bfloat16* du_sep, cudaStream_t s);
+cudaError_t launch_add_inplace(float* x, const float* y, size_t n, cudaStream_t s);
+
+// Tensor map of a row-major bf16 matrix [k_rows, mn_cols] read as an MN-major
+// GEMM operand: 64 x 64 boxes (64 MN elements = 128 bytes, 64 K rows) with
+// the 128-byte swizzle.
+bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols);
 
 enum { kOperandsBf16 = 0, kOperandsMxfp8 = 1, kOperandsNvfp4 = 2 };
 

@@ -212,6 +212,23 @@ class DoryModel:
                             _stream(stream))
         return h
 
+    def mlp_sublayer_backward(self, layer, h, dh_out, stream=None):
+        """Gradients of one MLP sublayer given its input h and dL/dh_out (fp32
+        [n, d] device tensors): dict of dh, d_w_gate, d_w_up, d_w_down, d_alpha."""
+        n, d = h.shape
+        ff = self.cfg["d_ff"]
+        ws = torch.empty(B.dory_mlp_backward_workspace_bytes(self.handle, n), dtype=torch.uint8,
+                         device=self.device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        out = dict(dh=torch.empty(n, d, **f32), d_w_gate=torch.empty(ff, d, **f32),
+                   d_w_up=torch.empty(ff, d, **f32), d_w_down=torch.empty(d, ff, **f32),
+                   d_alpha=torch.empty(d, **f32))
+        B.dory_mlp_sublayer_backward(self.handle, layer, n, _ptr(h), _ptr(dh_out), _ptr(out["dh"]),
+                                     _ptr(out["d_w_gate"]), _ptr(out["d_w_up"]),
+                                     _ptr(out["d_w_down"]), _ptr(out["d_alpha"]), _ptr(ws),
+                                     ws.numel(), _stream(stream))
+        return out
+
     def mlp_sublayer_noalloc(self, layer, h, stream=None):
         """As mlp_sublayer, but the library supplies the scratch (no workspace)."""
         B.dory_mlp_sublayer_noalloc(self.handle, layer, h.shape[0], _ptr(h), _stream(stream))
@@ -310,6 +327,14 @@ def gemm_nvfp4(A, Bm, g_a, g_b, k_splits=1, stream=None):
     C = torch.empty(k_splits, M, N, dtype=torch.float32, device=A.device)
     B.dory_gemm_nvfp4(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, float(g_a), float(g_b), k_splits,
                       _ptr(ws), ws.numel(), _stream(stream))
+    return C
+
+
+def gemm_bf16_mn(A, Bm, M, N, K, a_mn, b_mn, stream=None):
+    """C[M, N] = op(A) op(Bm)^T through the tcgen05 GEMM with operands read
+    MN-major where asked (A stored [K, M] when a_mn, Bm stored [K, N] when b_mn)."""
+    C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    B.dory_gemm_bf16_mn(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, int(a_mn), int(b_mn), _stream(stream))
     return C
 
 

@@ -1,0 +1,117 @@
+"""Backward of the MLP sublayer on the GPU against the float64 oracle.
+
+Truncated depth-one back-propagation trains only the final recurrent
+invocation ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
+English); dory_mlp_sublayer_backward is its MLP-sublayer step.  Checked:
+  * the tcgen05 GEMM with operands read MN-major (the dgrad and wgrad
+    products) against float64 matmuls, every transposed layout, ragged sizes;
+  * every gradient (dh, dW_gate, dW_up, dW_down, dalpha) against
+    oracle/backward.py on the tiny, head_dim-128 and 4B shapes;
+  * an output gradient along h_out gives (nearly) zero gradients on the GPU
+    too: the closed form the oracle is pinned by.
+Bar (the forward is recomputed with the inference path's bf16 operands:
+h, the SwiGLU activations and dL/dy are rounded to bf16, 2^-9 relative, before
+their products): per gradient tensor, relative Frobenius error <= 2e-2 and
+cosine (flattened) >= 0.9998.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.backward import mlp_sublayer_backward
+from tests.gpu_util import build, inputs, to_np
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO, MIN_COS = 2e-2, 0.9998
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(304, 384, 512), (3072, 1024, 200), (256, 256, 4096),
+                                   (136, 1280, 1000)])
+def test_gemm_with_transposed_operands(a_mn, b_mn, M, N, K):
+    from looped_ngpt_transformer_fwd_b200 import build as libbuild
+    from looped_ngpt_transformer_fwd_b200.model import gemm_bf16_mn
+    libbuild.build()
+    if (not a_mn or not b_mn) and K % 8:
+        pytest.skip("a K-major operand needs 16-byte rows")
+    g = torch.Generator(device="cuda").manual_seed(M + N + K)
+    A = torch.randn(K, M, device="cuda", generator=g) if a_mn else torch.randn(M, K, device="cuda", generator=g)
+    Bm = torch.randn(K, N, device="cuda", generator=g) if b_mn else torch.randn(N, K, device="cuda", generator=g)
+    A, Bm = A.to(torch.bfloat16), Bm.to(torch.bfloat16)
+    C = gemm_bf16_mn(A, Bm, M, N, K, a_mn, b_mn)
+    torch.cuda.synchronize()
+    An = A.double().cpu().numpy()
+    Bn = Bm.double().cpu().numpy()
+    ref = (An.T if a_mn else An) @ (Bn if b_mn else Bn.T)
+    err = np.abs(C.double().cpu().numpy() - ref).max()
+    assert err <= 1e-4 * np.abs(ref).max(), err
+
+
+def _weights(prov, layer):
+    from synthetic.bf16 import bf16_bits_to_f32
+    raw = prov(layer)
+    return {k: (bf16_bits_to_f32(v).astype(np.float64) if v.dtype == np.uint16
+                else np.asarray(v, dtype=np.float64)) for k, v in raw.items()}
+
+
+def _check(got, want, what):
+    g, w = to_np(got).ravel(), np.asarray(want, np.float64).ravel()
+    rel = np.linalg.norm(g - w) / np.linalg.norm(w)
+    cos = float(g @ w / (np.linalg.norm(g) * np.linalg.norm(w)))
+    assert rel <= REL_FRO and cos >= MIN_COS, f"{what}: rel {rel:.3e} cos {cos:.6f}"
+    return rel, cos
+
+
+def _run(cfg_name, seed, rows, layer, **over):
+    cfg, prov, model = build(cfg_name, seed=seed, **over)
+    _, h = inputs(cfg, seed + 1, rows)
+    rng = np.random.default_rng(seed + 2)
+    dh_out = rng.standard_normal(h.shape) * 0.1
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    gt = torch.from_numpy(dh_out.astype(np.float32)).cuda()
+    out = model.mlp_sublayer_backward(layer, ht, gt)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = mlp_sublayer_backward(cfg, _weights(prov, layer), h, dh_out)
+    res = {}
+    for k, rk in (("dh", "dh"), ("d_w_gate", "d_w_gate"), ("d_w_up", "d_w_up"),
+                  ("d_w_down", "d_w_down"), ("d_alpha", "d_alpha")):
+        res[k] = _check(out[k], ref[rk], f"{cfg_name} {k}")
+    model.close()
+    return res
+
+
+@pytest.mark.parametrize("rows,layer", [(200, 3), (64, 0), (1, 1)])
+def test_mlp_backward_tiny(rows, layer):
+    _run("tiny", 41, rows, layer)
+
+
+def test_mlp_backward_head_dim_128_shapes():
+    _run("tiny", 42, 300, 2, d_model=768, n_q_heads=6, n_kv_heads=2, head_dim=128, d_ff=1024,
+         softmax_scale=float(np.sqrt(128.0)))
+
+
+def test_mlp_backward_4b_shapes():
+    """d_model 3072, d_ff 9216 (one block of each kind), 256 rows."""
+    _run("dory4b", 43, 256, 1, n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1)
+
+
+def test_gradient_along_the_output_vanishes_on_the_gpu():
+    """dL/dh_out = 3 h_out: the output is a unit vector, so every gradient is
+    zero up to the bf16 rounding of the recomputed forward."""
+    cfg, prov, model = build("tiny", seed=44)
+    _, h = inputs(cfg, 45, 128)
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    h_out = ht.clone()
+    model.mlp_sublayer(2, h_out)
+    rng = np.random.default_rng(46)
+    ref_scale = model.mlp_sublayer_backward(
+        2, ht, torch.from_numpy((rng.standard_normal(h.shape) * 0.1).astype(np.float32)).cuda())
+    along = model.mlp_sublayer_backward(2, ht, 3.0 * h_out)
+    torch.cuda.synchronize()
+    for k in ("dh", "d_w_gate", "d_w_up", "d_w_down"):
+        typical = ref_scale[k].abs().max().item()
+        assert along[k].abs().max().item() < 0.05 * typical, k
+    model.close()
