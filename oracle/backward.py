@@ -1,4 +1,4 @@
-"""Backward pass of the MLP sublayer (oracle side).
+"""Backward pass of the MLP and attention sublayers (oracle side).
 
 TEST INFRASTRUCTURE ONLY, like the rest of `oracle/`: only `tests/`,
 `__graft_entry__.smoke()` and the CPU legs of `bench.py` may use it.
@@ -19,13 +19,19 @@ Every norm step x -> x / |x| has the derivative
     dx = (dx_hat - x_hat * <x_hat, dx_hat>) / |x|,
 and SiLU(x) = x sigma(x) has SiLU'(x) = sigma(x) (1 + x (1 - sigma(x))).
 Given dL/dh_out it returns dL/dh, dL/dWg, dL/dWu, dL/dWd and dL/dalpha
-(summed over the rows).  Pinned by central finite differences and by the
-closed form of an output gradient along h_out (tests/test_oracle_backward.py).
+(summed over the rows).  The attention sublayer of a training sequence
+(positions 0..n-1, every key one of the sequence's own) is written out the same
+way: projections, RoPE (an orthogonal rotation: its backward is the rotation
+by the opposite angle), the per-head norm times s_qk, masked softmax attention
+(dS = P * (dP - rowsum(P * dP))), the per-head sigmoid gate, the norm of the
+gated output and the nGPT update.  Pinned by central finite differences and by
+the closed form of an output gradient along h_out
+(tests/test_oracle_backward.py).
 """
 
 import numpy as np
 
-from .ngpt_oracle import sigmoid
+from .ngpt_oracle import is_full_layer, mask_allows, rope, sigmoid
 
 
 def _norm_backward(x_hat, x_len, dx_hat):
@@ -87,3 +93,93 @@ def mlp_sublayer_backward(cfg, W, h, dh_out):
     return dict(dh=dh, d_w_gate=d_w_gate, d_w_up=d_w_up, d_w_down=d_w_down, d_alpha=d_alpha,
                 h_out=f["h_out"])
 
+
+
+def _rows_norm(x, eps):
+    return np.sqrt(np.maximum((x * x).sum(axis=-1, keepdims=True), eps))
+
+
+def attention_sublayer_forward(cfg, W, h, b):
+    """Block b's attention sublayer on a training sequence h [n, d] at positions
+    0..n-1 (keys: the sequence's own), with every intermediate the backward
+    needs.  The same computation as the oracle's attention sublayer."""
+    eps = cfg["norm_eps"]
+    n, d = h.shape
+    hq, hkv, hd = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    full = is_full_layer(cfg, b)
+    base = cfg["rope_base_full"] if full else cfg["rope_base_swa"]
+    pos = np.arange(n)
+    rq = rope((h @ W["wq"].T).reshape(n, hq, hd), pos, base)
+    rk = rope((h @ W["wk"].T).reshape(n, hkv, hd), pos, base)
+    v = (h @ W["wv"].T).reshape(n, hkv, hd)
+    gate = sigmoid(h @ W["wg"].T)                                     # [n, hq]
+    lq, lk = _rows_norm(rq, eps), _rows_norm(rk, eps)
+    uq, uk = rq / lq, rk / lk
+    q, k = W["s_qk"] * uq, W["s_qk"] * uk
+    group = hq // hkv
+    Kq, Vq = np.repeat(k, group, axis=1), np.repeat(v, group, axis=1)
+    allowed = mask_allows(pos[:, None], pos[None, :], None if full else cfg["window"])
+    s = cfg["softmax_scale"] * np.einsum("ihd,jhd->hij", q, Kq)
+    s = np.where(allowed[None], s, -np.inf)
+    s = s - s.max(axis=-1, keepdims=True)
+    P = np.exp(s)
+    P /= P.sum(axis=-1, keepdims=True)
+    O = np.einsum("hij,jhd->ihd", P, Vq)                             # before the gate
+    o = (O * gate[:, :, None]).reshape(n, hq * hd)
+    o_len = _rows_norm(o, eps)
+    o_hat = o / o_len
+    y = o_hat @ W["wo"].T
+    y_len = _rows_norm(y, eps)
+    y_hat = y / y_len
+    z = h + W["alpha_attn"][None, :] * (y_hat - h)
+    z_len = _rows_norm(z, eps)
+    return dict(base=base, pos=pos, lq=lq, lk=lk, uq=uq, uk=uk, q=q, Kq=Kq, Vq=Vq, gate=gate,
+                P=P, O=O, o_hat=o_hat, o_len=o_len, y_hat=y_hat, y_len=y_len, z_len=z_len,
+                h_out=z / z_len)
+
+
+def attention_sublayer_backward(cfg, W, h, dh_out, b):
+    """dL/d(inputs and parameters) of block b's attention sublayer on a training
+    sequence, given dL/dh_out.  W: wq, wk, wv [*, d], wg [hq, d], wo [d, hq*hd],
+    alpha_attn [d], s_qk [hd] as float64.  Returns dh, d_wq, d_wk, d_wv, d_wg,
+    d_wo, d_alpha, d_s_qk and h_out."""
+    h = np.asarray(h, dtype=np.float64)
+    dh_out = np.asarray(dh_out, dtype=np.float64)
+    n, d = h.shape
+    hq, hkv, hd = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    group = hq // hkv
+    f = attention_sublayer_forward(cfg, W, h, b)
+    alpha = W["alpha_attn"][None, :]
+    # nGPT update and output projection
+    dz = _norm_backward(f["h_out"], f["z_len"], dh_out)
+    d_alpha = (dz * (f["y_hat"] - h)).sum(axis=0)
+    dh = dz * (1.0 - alpha)
+    dy = _norm_backward(f["y_hat"], f["y_len"], dz * alpha)
+    d_wo = dy.T @ f["o_hat"]
+    do = _norm_backward(f["o_hat"], f["o_len"], dy @ W["wo"]).reshape(n, hq, hd)
+    # gate: o = O * gate, gate = sigmoid(h Wg^T)
+    dgate = (do * f["O"]).sum(axis=-1)
+    dgl = dgate * f["gate"] * (1.0 - f["gate"])
+    dO = do * f["gate"][:, :, None]
+    # softmax attention (masked entries have P = 0 and get no gradient)
+    P = f["P"]
+    dP = np.einsum("ihd,jhd->hij", dO, f["Vq"])
+    dVq = np.einsum("hij,ihd->jhd", P, dO)
+    dS = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+    scale = cfg["softmax_scale"]
+    dq = scale * np.einsum("hij,jhd->ihd", dS, f["Kq"])
+    dKq = scale * np.einsum("hij,ihd->jhd", dS, f["q"])
+    dk = dKq.reshape(n, hkv, group, hd).sum(axis=2)
+    dv = dVq.reshape(n, hkv, group, hd).sum(axis=2)
+    # q = s_qk * rq / |rq| (per head), rq = RoPE(q_raw); likewise k
+    s_qk = W["s_qk"]
+    d_s_qk = (dq * f["uq"]).sum(axis=(0, 1)) + (dk * f["uk"]).sum(axis=(0, 1))
+    drq = (s_qk * dq - f["uq"] * (f["uq"] * s_qk * dq).sum(axis=-1, keepdims=True)) / f["lq"]
+    drk = (s_qk * dk - f["uk"] * (f["uk"] * s_qk * dk).sum(axis=-1, keepdims=True)) / f["lk"]
+    dq_raw = rope(drq, -f["pos"], f["base"]).reshape(n, hq * hd)     # the inverse rotation
+    dk_raw = rope(drk, -f["pos"], f["base"]).reshape(n, hkv * hd)
+    dv_raw = dv.reshape(n, hkv * hd)
+    d_wq, d_wk, d_wv, d_wg = dq_raw.T @ h, dk_raw.T @ h, dv_raw.T @ h, dgl.T @ h
+    dh = dh + dq_raw @ W["wq"] + dk_raw @ W["wk"] + dv_raw @ W["wv"] + dgl @ W["wg"]
+    return dict(dh=dh, d_wq=d_wq, d_wk=d_wk, d_wv=d_wv, d_wg=d_wg, d_wo=d_wo, d_alpha=d_alpha,
+                d_s_qk=d_s_qk, h_out=f["h_out"])

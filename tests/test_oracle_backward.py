@@ -77,3 +77,59 @@ def test_gate_scale_reaches_the_gate_gradient():
     g1 = mlp_sublayer_backward(cfg, W, h, dh_out)["d_w_gate"]
     g2 = mlp_sublayer_backward(dict(cfg, gate_scale=2.0), W, h, dh_out)["d_w_gate"]
     assert np.abs(g1 - g2).max() > 1e-3 * np.abs(g1).max()
+
+
+# ------------------------------------------------------------------ attention
+
+def _att_setup(seed=11, rows=9, layer=1, **over):
+    over = dict(dict(d_model=64, n_q_heads=4, n_kv_heads=2, head_dim=16, d_ff=128, window=4), **over)
+    cfg = load_config("tiny", **over)
+    prov = weights_from_generator(cfg, seed, "random")
+    raw = prov(layer)
+    W = {k: (bf16_bits_to_f32(v).astype(np.float64) if v.dtype == np.uint16
+             else np.asarray(v, dtype=np.float64)) for k, v in raw.items()}
+    h = bf16_bits_to_f32(hidden_in(cfg, seed + 1, rows)).astype(np.float64)
+    dh_out = np.random.default_rng(seed + 2).standard_normal(h.shape)
+    return cfg, prov, W, h, dh_out
+
+
+@pytest.mark.parametrize("layer", [0, 1])   # sliding window (W = 4), full
+def test_attention_forward_is_the_oracle_sublayer(layer):
+    from oracle import KVCache
+    from oracle.backward import attention_sublayer_forward
+    cfg, prov, W, h, _ = _att_setup(layer=layer)
+    ref = Oracle(cfg, prov).attention_sublayer(layer, h, 0, 0, 1, KVCache(cfg, "last_loop"))
+    assert np.allclose(attention_sublayer_forward(cfg, W, h, layer)["h_out"], ref, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+@pytest.mark.parametrize("name", ["h", "wq", "wk", "wv", "wg", "wo", "alpha_attn", "s_qk"])
+def test_attention_gradients_match_central_differences(layer, name):
+    from oracle.backward import attention_sublayer_backward, attention_sublayer_forward
+    cfg, _, W, h, dh_out = _att_setup(layer=layer)
+    g = attention_sublayer_backward(cfg, W, h, dh_out, layer)
+    key = {"h": "dh", "alpha_attn": "d_alpha", "s_qk": "d_s_qk"}.get(name, "d_" + name)
+    grad = g[key]
+    target = h if name == "h" else W[name]
+    loss = lambda: float((attention_sublayer_forward(cfg, W, h, layer)["h_out"] * dh_out).sum())
+    rng = np.random.default_rng(13)
+    eps = 1e-6
+    for _ in range(10):
+        ix = tuple(rng.integers(0, n) for n in target.shape)
+        old = target[ix]
+        target[ix] = old + eps
+        lp = loss()
+        target[ix] = old - eps
+        lm = loss()
+        target[ix] = old
+        fd = (lp - lm) / (2 * eps)
+        assert abs(fd - grad[ix]) <= 1e-6 * max(1.0, abs(fd)), (name, ix, fd, grad[ix])
+
+
+def test_attention_gradient_along_the_output_vanishes():
+    from oracle.backward import attention_sublayer_backward, attention_sublayer_forward
+    cfg, _, W, h, _ = _att_setup()
+    h_out = attention_sublayer_forward(cfg, W, h, 1)["h_out"]
+    g = attention_sublayer_backward(cfg, W, h, -2.0 * h_out, 1)
+    for k in ("dh", "d_wq", "d_wk", "d_wv", "d_wg", "d_wo", "d_alpha", "d_s_qk"):
+        assert np.abs(g[k]).max() < 1e-12, k
