@@ -351,6 +351,27 @@ DORY_API int dory_gemm_bf16_mn(const void* A, const void* B, float* C, int M, in
  * buffers 16-byte aligned.  bf16 weight format only (DORY_ERR_BAD_CONFIG
  * otherwise). */
 DORY_API size_t dory_mlp_backward_workspace_bytes(const dory_model* m, int n_rows);
+
+/* Backward of one attention sublayer on a training sequence: rows are the
+ * positions 0..n_rows-1 of one sequence and every key is one of its own (no KV
+ * cache is read or written).  Same page and section as the MLP sublayer's
+ * backward.  Given h_in and dL/dh_out [n_rows, d_model] (fp32, device),
+ * recomputes the forward (bf16 projection operands; the softmax with each
+ * row's exact maximum) and writes dL/dh_in [n_rows, d_model], dL/dW_q
+ * [n_q_heads*head_dim, d_model], dL/dW_k and dL/dW_v [n_kv_heads*head_dim,
+ * d_model], dL/dW_gate [n_q_heads, d_model], dL/dW_o [d_model,
+ * n_q_heads*head_dim], dL/dalpha_attn [d_model] and dL/ds_qk [head_dim]
+ * (fp32; the last two summed deterministically).  Attention runs per KV head
+ * on the tensor cores with the score matrix of the group's stacked queries
+ * held in the workspace, so the workspace
+ * (dory_attention_backward_workspace_bytes) grows with n_rows squared.  bf16
+ * weight format only (DORY_ERR_BAD_CONFIG otherwise). */
+DORY_API size_t dory_attention_backward_workspace_bytes(const dory_model* m, int n_rows);
+DORY_API int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows,
+                                              const float* h_in, const float* dh_out, float* dh_in,
+                                              float* d_wq, float* d_wk, float* d_wv, float* d_wg,
+                                              float* d_wo, float* d_alpha, float* d_s_qk, void* ws,
+                                              size_t ws_bytes, void* stream);
 DORY_API int dory_mlp_sublayer_backward(dory_model* m, int layer, int n_rows, const float* h_in,
                                         const float* dh_out, float* dh_in, float* d_w_gate,
                                         float* d_w_up, float* d_w_down, float* d_alpha, void* ws,

@@ -37,6 +37,7 @@ EXPORTS = (
     "dory_gemm_mxfp8_workspace_bytes", "dory_gemm_mxfp8", "dory_quant_nvfp4",
     "dory_nvfp4_scale_bytes", "dory_gemm_nvfp4_workspace_bytes", "dory_gemm_nvfp4",
     "dory_gemm_bf16_mn", "dory_mlp_backward_workspace_bytes", "dory_mlp_sublayer_backward",
+    "dory_attention_backward_workspace_bytes", "dory_attention_sublayer_backward",
     "dory_vocab_bytes", "dory_vocab_create", "dory_embed", "dory_lm_head", "dory_sample",
     "dory_vocab_free",
 )
@@ -127,6 +128,8 @@ def lib():
             "dory_gemm_bf16_mn": (I, [P, P, P, I, I, I, I, I, P]),
             "dory_mlp_backward_workspace_bytes": (SZ, [P, I]),
             "dory_mlp_sublayer_backward": (I, [P, I, I, P, P, P, P, P, P, P, P, SZ, P]),
+            "dory_attention_backward_workspace_bytes": (SZ, [P, I]),
+            "dory_attention_sublayer_backward": (I, [P, I, I] + [P] * 11 + [SZ, P]),
             "dory_vocab_bytes": (SZ, [P, I]),
             "dory_vocab_create": (I, [P, I, P, P, P, P, SZ, P, P]),
             "dory_embed": (I, [P, P, I, P, P]),
@@ -324,6 +327,18 @@ def dory_mlp_sublayer_backward(m, layer, n_rows, h_in, dh_out, dh_in, d_w_gate, 
     return check(lib().dory_mlp_sublayer_backward(m, layer, n_rows, h_in, dh_out, dh_in, d_w_gate,
                                                   d_w_up, d_w_down, d_alpha, ws, ws_bytes, stream),
                  "dory_mlp_sublayer_backward")
+
+
+def dory_attention_backward_workspace_bytes(m, n_rows):
+    return lib().dory_attention_backward_workspace_bytes(m, n_rows)
+
+
+def dory_attention_sublayer_backward(m, layer, n_rows, h_in, dh_out, dh_in, d_wq, d_wk, d_wv, d_wg,
+                                     d_wo, d_alpha, d_s_qk, ws, ws_bytes, stream):
+    return check(lib().dory_attention_sublayer_backward(m, layer, n_rows, h_in, dh_out, dh_in, d_wq,
+                                                        d_wk, d_wv, d_wg, d_wo, d_alpha, d_s_qk,
+                                                        ws, ws_bytes, stream),
+                 "dory_attention_sublayer_backward")
 
 
 def dory_quant_nvfp4(src, rows, K, g, d_g, codes, scales, stream):

@@ -1384,23 +1384,77 @@ BwdLayout bwd_layout(const dory_model* m, int R) {
   return L;
 }
 
-// C[M, N] (fp32, row pitch N) = op(A) op(B)^T on the tcgen05 GEMM; A is
-// stored [M][K] or, with a_mn, [K][M]; B [N][K] or, with b_mn, [K][N].  K is
-// rounded up to the 64-element step: the maps' K extent is K, so the tail
+// C[M, N] (fp32, row pitch ld_out, 0 = N) = op(A) op(B)^T on the tcgen05
+// GEMM; A is stored [M][K] or, with a_mn, [K][M]; B [N][K] or, with b_mn,
+// [K][N]; lda / ldb: their row pitches in elements (0 = the row length).  K
+// is rounded up to the 64-element step: the maps' K extent is K, so the tail
 // reads zeros.
 cudaError_t gemm_f32(const dory_model* m, const void* A, int a_mn, const void* B, int b_mn,
-                     float* C, int M, int N, int K, cudaStream_t s) {
+                     float* C, int M, int N, int K, cudaStream_t s, int ld_out = 0, int lda = 0,
+                     int ldb = 0) {
   const int BN = (N % 256 == 0) ? 256 : 128;
   CUtensorMap ta, tb;
-  const bool ok = (a_mn ? make_tmap_bf16_mn(&ta, A, K, M) : make_tmap_bf16(&ta, A, M, K, 128)) &&
-                  (b_mn ? make_tmap_bf16_mn(&tb, B, K, N) : make_tmap_bf16(&tb, B, N, K, BN));
+  const bool ok =
+      (a_mn ? make_tmap_bf16_mn(&ta, A, K, M, lda) : make_tmap_bf16_ld(&ta, A, M, K, lda ? lda : K, 128)) &&
+      (b_mn ? make_tmap_bf16_mn(&tb, B, K, N, ldb) : make_tmap_bf16_ld(&tb, B, N, K, ldb ? ldb : K, BN));
   if (!ok) return cudaErrorInvalidValue;
   GemmParams p;
   p.M = M; p.N = N; p.K = (K + 63) / 64 * 64;
-  p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = N;
+  p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = ld_out > 0 ? ld_out : N;
   p.a_mn = a_mn; p.b_mn = b_mn;
   p.status = m->status;
   return launch_gemm(ta, tb, p, BN, 128, m->num_sms, s);
+}
+
+// Scratch of the attention-sublayer backward for a T-row training sequence.
+struct AttnBwdLayout {
+  size_t hb, raw, qh, kh, vb, gate, rope, qs, ks, vs, S, P, Os, o, y, dy, part, dout, dOs, dS, dV,
+      dQ, dK, dq_hat, dk_hat, dv, d_raw, dhx, dW, ds_part, total;
+  int Tp, grid_row, grid_qk;
+};
+
+AttnBwdLayout attn_bwd_layout(const dory_model* m, int T) {
+  AttnBwdLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  const size_t t = size_t(T), d = m->d, hq = m->hq, hkv = m->hkv, hd = m->hd, G = hq / hkv;
+  const size_t da = hq * hd, ldq = m->ld_qkvg;
+  L.Tp = (T + 7) / 8 * 8;
+  const size_t tp = size_t(L.Tp);
+  L.grid_row = mlp_bwd_row_grid(T, m->num_sms);
+  L.grid_qk = qk_bwd_grid(m->num_sms);
+  L.hb = take(t * d * 2);
+  L.raw = take(t * ldq * 4);               // q | k | v | gate logits before the epilogue
+  L.qh = take(t * hq * hd * 2);
+  L.kh = take(t * hkv * hd * 2);
+  L.vb = take(t * hkv * hd * 2);
+  L.gate = take(t * hq * 4);
+  L.rope = take(t * (hd / 2) * 8);
+  L.qs = take(hkv * G * t * hd * 2);       // per KV head: its group's queries stacked
+  L.ks = take(hkv * t * hd * 2);
+  L.vs = take(hkv * t * hd * 2);
+  L.S = take(G * t * tp * 4);              // S, then dP (one KV head at a time)
+  L.P = take(hkv * G * t * tp * 2);        // P of every KV head
+  L.Os = take(hkv * G * t * hd * 4);       // P V before the gate
+  L.o = take(t * da * 2);
+  L.y = take(t * d * 4);
+  L.dy = take(t * d * 2);
+  L.part = take(size_t(L.grid_row) * d * 4);
+  L.dout = take(t * da * 4);
+  L.dOs = take(hkv * G * t * hd * 2);
+  L.dS = take(G * t * tp * 2);
+  L.dV = take(t * hd * 4);
+  L.dQ = take(G * t * hd * 4);
+  L.dK = take(t * hd * 4);
+  L.dq_hat = take(t * hq * hd * 4);
+  L.dk_hat = take(t * hkv * hd * 4);
+  L.dv = take(t * hkv * hd * 4);
+  L.d_raw = take(t * ldq * 2);
+  L.dhx = take(t * d * 4);
+  L.dW = take(size_t(m->n_qkvg) * d * 4);
+  L.ds_part = take(size_t(L.grid_qk) * hd * 4);
+  L.total = o;
+  return L;
 }
 
 }  // namespace
@@ -1453,6 +1507,112 @@ int dory_mlp_sublayer_backward(dory_model* m, int layer, int n_rows, const float
   e = e ? e : gemm_f32(m, bf(L.du), 1, bf(L.hb), 1, d_w_up, ff, d, R, s);
   e = e ? e : launch_add_inplace(dh_in, f32(L.dhx), size_t(R) * d, s);
   e = e ? e : launch_colsum(f32(L.part), L.grid, d, d_alpha, s);
+  return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
+}
+
+size_t dory_attention_backward_workspace_bytes(const dory_model* m, int n_rows) {
+  if (!m || n_rows <= 0) return 0;
+  return attn_bwd_layout(m, n_rows).total;
+}
+
+int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows, const float* h_in,
+                                     const float* dh_out, float* dh_in, float* d_wq, float* d_wk,
+                                     float* d_wv, float* d_wg, float* d_wo, float* d_alpha,
+                                     float* d_s_qk, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !h_in || !dh_out || !dh_in || !d_wq || !d_wk || !d_wv || !d_wg || !d_wo || !d_alpha ||
+      !d_s_qk || !ws || n_rows <= 0 || layer < 0 || layer >= m->nb)
+    return DORY_ERR_INVALID_ARG;
+  if (m->mx) return DORY_ERR_BAD_CONFIG;   // bf16 weights only
+  const void* ptrs[10] = {h_in, dh_out, dh_in, d_wq, d_wk, d_wv, d_wg, d_wo, d_alpha, d_s_qk};
+  for (const void* q : ptrs)
+    if (!is_aligned(q, 16)) return DORY_ERR_MISALIGNED;
+  if (!is_aligned(ws)) return DORY_ERR_MISALIGNED;
+  const AttnBwdLayout L = attn_bwd_layout(m, n_rows);
+  if (ws_bytes < L.total) return DORY_ERR_BUFFER_TOO_SMALL;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(b + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  const BlockW& W = m->blocks[layer];
+  const int T = n_rows, Tp = L.Tp, d = m->d, hq = m->hq, hkv = m->hkv, hd = m->hd;
+  const int G = hq / hkv, da = hq * hd, nq = m->n_qkvg, ldq = m->ld_qkvg;
+  const int window = W.full ? 0 : m->cfg.window;
+  const float eps = m->cfg.norm_eps, scale = m->cfg.softmax_scale;
+  const size_t head_q = size_t(G) * T * hd, head_kv = size_t(T) * hd, head_p = size_t(G) * T * Tp;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float2* rope = reinterpret_cast<float2*>(b + L.rope);
+  cudaError_t e = cudaSuccess;
+
+  // ---- forward again: projections, q_hat / k_hat / v / gates, attention, y
+  e = e ? e : launch_f32_to_bf16(h_in, bf(L.hb), size_t(T) * d, s);
+  e = e ? e : launch_rope_table(W.full ? m->inv_freq_full : m->inv_freq_swa, hd, T, 0, nullptr,
+                                rope, s);
+  e = e ? e : gemm_f32(m, bf(L.hb), 0, W.wqkvg, 0, f32(L.raw), T, nq, d, s, ldq);
+  if (e == cudaSuccess) {
+    QkvgPostParams pp;
+    pp.part = f32(L.raw); pp.splits = 1; pp.split_stride = size_t(T) * ldq; pp.ld = ldq;
+    pp.rows = T; pp.n_q_heads = hq; pp.n_kv_heads = hkv; pp.hd = hd;
+    pp.s_qk = W.s_qk; pp.rope = rope; pp.norm_eps = eps;
+    pp.q_out = bf(L.qh); pp.k_out = bf(L.kh); pp.v_out = bf(L.vb); pp.gate_out = f32(L.gate);
+    e = launch_qkvg_post(pp, s);
+  }
+  for (int h = 0; h < hkv && e == cudaSuccess; ++h) {
+    __nv_bfloat16* qs = bf(L.qs) + h * head_q;
+    __nv_bfloat16* ks = bf(L.ks) + h * head_kv;
+    __nv_bfloat16* vs = bf(L.vs) + h * head_kv;
+    __nv_bfloat16* P = bf(L.P) + h * head_p;
+    e = e ? e : launch_gather_heads(bf(L.qh), T, hq, h * G, G, hd, qs, s);
+    e = e ? e : launch_gather_heads(bf(L.kh), T, hkv, h, 1, hd, ks, s);
+    e = e ? e : launch_gather_heads(bf(L.vb), T, hkv, h, 1, hd, vs, s);
+    e = e ? e : gemm_f32(m, qs, 0, ks, 0, f32(L.S), G * T, T, hd, s, Tp);          // S = Q_s K^T
+    e = e ? e : launch_softmax_rows(f32(L.S), G * T, T, Tp, window, scale, P, s);
+    e = e ? e : gemm_f32(m, P, 0, vs, 1, f32(L.Os) + h * head_q, G * T, hd, T, s, 0, Tp);   // P V
+  }
+  e = e ? e : launch_gated_output(f32(L.Os), f32(L.gate), T, hq, G, hd, bf(L.o), s);
+  e = e ? e : gemm_f32(m, bf(L.o), 0, W.wo, 0, f32(L.y), T, d, da, s);
+
+  // ---- backward: nGPT update, output projection, gates
+  e = e ? e : launch_mlp_bwd_row(f32(L.y), h_in, W.alpha_attn, dh_out, T, d, eps, dh_in, bf(L.dy),
+                                 f32(L.part), L.grid_row, s);
+  e = e ? e : gemm_f32(m, bf(L.dy), 0, W.wo, 1, f32(L.dout), T, da, d, s);       // do = dy W_o
+  e = e ? e : gemm_f32(m, bf(L.dy), 1, bf(L.o), 1, d_wo, d, da, T, s);          // dW_o = dy^T o
+  e = e ? e : cudaMemsetAsync(b + L.d_raw, 0, size_t(T) * ldq * 2, s);
+  e = e ? e : launch_gate_bwd(f32(L.dout), f32(L.Os), f32(L.gate), T, hq, G, hd, bf(L.dOs),
+                              bf(L.d_raw), ldq, da + 2 * hkv * hd, s);
+  // ---- attention, one KV head at a time
+  for (int h = 0; h < hkv && e == cudaSuccess; ++h) {
+    const __nv_bfloat16* qs = bf(L.qs) + h * head_q;
+    const __nv_bfloat16* ks = bf(L.ks) + h * head_kv;
+    const __nv_bfloat16* vs = bf(L.vs) + h * head_kv;
+    const __nv_bfloat16* P = bf(L.P) + h * head_p;
+    const __nv_bfloat16* dOs = bf(L.dOs) + h * head_q;
+    e = e ? e : gemm_f32(m, dOs, 0, vs, 0, f32(L.S), G * T, T, hd, s, Tp);        // dP = dO V^T
+    e = e ? e : launch_softmax_bwd_rows(P, f32(L.S), G * T, Tp, scale, bf(L.dS), s);
+    e = e ? e : gemm_f32(m, P, 1, dOs, 1, f32(L.dV), T, hd, G * T, s, 0, Tp);       // dV = P^T dO
+    e = e ? e : gemm_f32(m, bf(L.dS), 0, ks, 1, f32(L.dQ), G * T, hd, T, s, 0, Tp);  // dQ = dS K
+    e = e ? e : gemm_f32(m, bf(L.dS), 1, qs, 1, f32(L.dK), T, hd, G * T, s, 0, Tp);  // dK = dS^T Q
+    e = e ? e : launch_scatter_heads(f32(L.dQ), T, G, hd, hq, h * G, f32(L.dq_hat), s);
+    e = e ? e : launch_scatter_heads(f32(L.dK), T, 1, hd, hkv, h, f32(L.dk_hat), s);
+    e = e ? e : launch_scatter_heads(f32(L.dV), T, 1, hd, hkv, h, f32(L.dv), s);
+  }
+  // ---- QK norm and RoPE, then the projection's dgrad and wgrad
+  e = e ? e : launch_v_grad(f32(L.dv), T, hkv, hd, bf(L.d_raw), ldq, da + hkv * hd, s);
+  e = e ? e : launch_qk_bwd(f32(L.raw), ldq, f32(L.dq_hat), f32(L.dk_hat), W.s_qk, rope, T, hq,
+                            hkv, hd, eps, bf(L.d_raw), ldq, f32(L.ds_part), L.grid_qk, s);
+  e = e ? e : gemm_f32(m, bf(L.d_raw), 0, W.wqkvg, 1, f32(L.dhx), T, d, nq, s, 0, ldq);
+  e = e ? e : launch_add_inplace(dh_in, f32(L.dhx), size_t(T) * d, s);
+  e = e ? e : gemm_f32(m, bf(L.d_raw), 1, bf(L.hb), 1, f32(L.dW), nq, d, T, s, 0, ldq);
+  if (e == cudaSuccess) {
+    const size_t row = size_t(d) * 4;
+    const size_t kvr = size_t(hkv) * hd;
+    const uint8_t* dW = b + L.dW;
+    e = cudaMemcpyAsync(d_wq, dW, size_t(da) * row, cudaMemcpyDeviceToDevice, s);
+    e = e ? e : cudaMemcpyAsync(d_wk, dW + size_t(da) * row, kvr * row, cudaMemcpyDeviceToDevice, s);
+    e = e ? e : cudaMemcpyAsync(d_wv, dW + (da + kvr) * row, kvr * row, cudaMemcpyDeviceToDevice, s);
+    e = e ? e : cudaMemcpyAsync(d_wg, dW + (da + 2 * kvr) * row, size_t(hq) * row,
+                                cudaMemcpyDeviceToDevice, s);
+  }
+  e = e ? e : launch_colsum(f32(L.part), L.grid_row, d, d_alpha, s);
+  e = e ? e : launch_colsum(f32(L.ds_part), L.grid_qk, hd, d_s_qk, s);
   return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
 

@@ -835,6 +835,21 @@ cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
 
 }  // namespace
 
+bool make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint64_t ld, uint32_t box_rows) {
+  EncodeTiledFn encode = encode_tiled();
+  if (!encode || (ld * 2) % 16 != 0 || ld < cols || (reinterpret_cast<uintptr_t>(base) & 15) != 0)
+    return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows) {
   using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -863,12 +878,14 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols) {
+bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols,
+                       uint64_t ld) {
   EncodeTiledFn encode = encode_tiled();
-  if (!encode || (mn_cols * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0)
+  if (ld == 0) ld = mn_cols;
+  if (!encode || (ld * 2) % 16 != 0 || ld < mn_cols || (reinterpret_cast<uintptr_t>(base) & 15) != 0)
     return false;
   cuuint64_t dims[2] = {mn_cols, k_rows};
-  cuuint64_t strides[1] = {mn_cols * 2};
+  cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {64, 64};
   cuuint32_t estr[2] = {1, 1};
   return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,

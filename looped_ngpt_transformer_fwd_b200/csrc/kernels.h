@@ -74,10 +74,36 @@ cudaError_t launch_swiglu_bwd(const float* gu, const float* da, int rows, int ff
                               __nv_bfloat16* du_sep, cudaStream_t s);
 cudaError_t launch_add_inplace(float* x, const float* y, size_t n, cudaStream_t s);
 
-// Tensor map of a row-major bf16 matrix [k_rows, mn_cols] read as an MN-major
-// GEMM operand: 64 x 64 boxes (64 MN elements = 128 bytes, 64 K rows) with
-// the 128-byte swizzle.
-bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols);
+// Attention-sublayer backward pieces (attn_backward.cu), see that file.
+cudaError_t launch_gather_heads(const __nv_bfloat16* src, int T, int src_heads, int head0, int G,
+                                int hd, __nv_bfloat16* dst, cudaStream_t s);
+cudaError_t launch_softmax_rows(const float* S, int rows, int T, int ld, int window, float scale,
+                                __nv_bfloat16* P, cudaStream_t s);
+cudaError_t launch_softmax_bwd_rows(const __nv_bfloat16* P, const float* dP, int rows, int ld,
+                                    float scale, __nv_bfloat16* dS, cudaStream_t s);
+cudaError_t launch_gated_output(const float* Os, const float* gate, int T, int hq, int G, int hd,
+                                __nv_bfloat16* o, cudaStream_t s);
+cudaError_t launch_gate_bwd(const float* dout, const float* Os, const float* gate, int T, int hq,
+                            int G, int hd, __nv_bfloat16* dOs, __nv_bfloat16* d_raw, int ld_raw,
+                            int gate_col0, cudaStream_t s);
+cudaError_t launch_scatter_heads(const float* src, int T, int G, int hd, int dst_heads, int head0,
+                                 float* dst, cudaStream_t s);
+int qk_bwd_grid(int num_sms);
+cudaError_t launch_qk_bwd(const float* raw, int ld_raw_f, const float* dq_hat, const float* dk_hat,
+                          const float* s_qk, const float2* rope, int T, int hq, int hkv, int hd,
+                          float norm_eps, __nv_bfloat16* d_raw, int ld_raw, float* ds_part,
+                          int grid, cudaStream_t s);
+cudaError_t launch_v_grad(const float* dv, int T, int hkv, int hd, __nv_bfloat16* d_raw, int ld_raw,
+                          int col0, cudaStream_t s);
+
+// Tensor map of a row-major bf16 matrix [k_rows, mn_cols] (row pitch ld
+// elements, 0 = mn_cols) read as an MN-major GEMM operand: 64 x 64 boxes (64
+// MN elements = 128 bytes, 64 K rows) with the 128-byte swizzle.
+bool make_tmap_bf16_mn(CUtensorMap* map, const void* base, uint64_t k_rows, uint64_t mn_cols,
+                       uint64_t ld = 0);
+// make_tmap_bf16 with a row pitch of ld elements (>= cols)
+bool make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint64_t ld, uint32_t box_rows);
 
 enum { kOperandsBf16 = 0, kOperandsMxfp8 = 1, kOperandsNvfp4 = 2 };
 

@@ -212,6 +212,26 @@ class DoryModel:
                             _stream(stream))
         return h
 
+    def attention_sublayer_backward(self, layer, h, dh_out, stream=None):
+        """Gradients of one attention sublayer on a training sequence (rows =
+        positions 0..n-1) given its input h and dL/dh_out (fp32 [n, d] device
+        tensors): dict of dh, d_wq, d_wk, d_wv, d_wg, d_wo, d_alpha, d_s_qk."""
+        n, d = h.shape
+        c = self.cfg
+        hq, hkv, hd = c["n_q_heads"], c["n_kv_heads"], c["head_dim"]
+        ws = torch.empty(B.dory_attention_backward_workspace_bytes(self.handle, n),
+                         dtype=torch.uint8, device=self.device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        out = dict(dh=torch.empty(n, d, **f32), d_wq=torch.empty(hq * hd, d, **f32),
+                   d_wk=torch.empty(hkv * hd, d, **f32), d_wv=torch.empty(hkv * hd, d, **f32),
+                   d_wg=torch.empty(hq, d, **f32), d_wo=torch.empty(d, hq * hd, **f32),
+                   d_alpha=torch.empty(d, **f32), d_s_qk=torch.empty(hd, **f32))
+        B.dory_attention_sublayer_backward(
+            self.handle, layer, n, _ptr(h), _ptr(dh_out), _ptr(out["dh"]), _ptr(out["d_wq"]),
+            _ptr(out["d_wk"]), _ptr(out["d_wv"]), _ptr(out["d_wg"]), _ptr(out["d_wo"]),
+            _ptr(out["d_alpha"]), _ptr(out["d_s_qk"]), _ptr(ws), ws.numel(), _stream(stream))
+        return out
+
     def mlp_sublayer_backward(self, layer, h, dh_out, stream=None):
         """Gradients of one MLP sublayer given its input h and dL/dh_out (fp32
         [n, d] device tensors): dict of dh, d_w_gate, d_w_up, d_w_down, d_alpha."""

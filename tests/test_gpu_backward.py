@@ -115,3 +115,55 @@ def test_gradient_along_the_output_vanishes_on_the_gpu():
         typical = ref_scale[k].abs().max().item()
         assert along[k].abs().max().item() < 0.05 * typical, k
     model.close()
+
+
+# ------------------------------------------------------------------ attention
+
+def _run_attention(cfg_name, seed, rows, layer, **over):
+    from oracle.backward import attention_sublayer_backward
+    cfg, prov, model = build(cfg_name, seed=seed, **over)
+    _, h = inputs(cfg, seed + 1, rows)
+    dh_out = np.random.default_rng(seed + 2).standard_normal(h.shape) * 0.1
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    gt = torch.from_numpy(dh_out.astype(np.float32)).cuda()
+    out = model.attention_sublayer_backward(layer, ht, gt)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = attention_sublayer_backward(cfg, _weights(prov, layer), h, dh_out, layer)
+    for k in ("dh", "d_wq", "d_wk", "d_wv", "d_wg", "d_wo", "d_alpha", "d_s_qk"):
+        _check(out[k], ref[k], f"{cfg_name} layer {layer} {k}")
+    model.close()
+
+
+@pytest.mark.parametrize("layer", [0, 1])        # sliding window (W = 32), full
+@pytest.mark.parametrize("rows", [100, 7])
+def test_attention_backward_tiny(layer, rows):
+    _run_attention("tiny", 51, rows, layer)
+
+
+@pytest.mark.parametrize("layer", [0, 1])        # W = 128, full; GQA group 3
+def test_attention_backward_head_dim_128(layer):
+    _run_attention("tiny", 52, 300, layer, d_model=768, n_q_heads=6, n_kv_heads=2, head_dim=128,
+                   d_ff=1024, window=128, softmax_scale=float(np.sqrt(128.0)))
+
+
+def test_attention_backward_4b_shapes():
+    """d_model 3072, 24 / 8 heads of 128, window 4096 (full causal at 256 rows)."""
+    _run_attention("dory4b", 53, 256, 1, n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1)
+
+
+def test_attention_gradient_along_the_output_vanishes_on_the_gpu():
+    cfg, prov, model = build("tiny", seed=54)
+    _, h = inputs(cfg, 55, 64)
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    kv = model.kv_cache("last_loop", 1, 64)
+    h_out = ht.clone()
+    model.attention_sublayer(kv, 1, h_out, loop=1, seq=0, pos0=0)
+    rng = np.random.default_rng(56)
+    typical = model.attention_sublayer_backward(
+        1, ht, torch.from_numpy((rng.standard_normal(h.shape) * 0.1).astype(np.float32)).cuda())
+    along = model.attention_sublayer_backward(1, ht, -2.0 * h_out)
+    torch.cuda.synchronize()
+    for k in ("dh", "d_wq", "d_wk", "d_wv", "d_wg", "d_wo"):
+        assert along[k].abs().max().item() < 0.05 * typical[k].abs().max().item(), k
+    model.close()
