@@ -183,3 +183,85 @@ def attention_sublayer_backward(cfg, W, h, dh_out, b):
     dh = dh + dq_raw @ W["wq"] + dk_raw @ W["wk"] + dv_raw @ W["wv"] + dgl @ W["wg"]
     return dict(dh=dh, d_wq=d_wq, d_wk=d_wk, d_wv=d_wv, d_wg=d_wg, d_wo=d_wo, d_alpha=d_alpha,
                 d_s_qk=d_s_qk, h_out=f["h_out"])
+
+
+# --------------------------------------------------------------- the stack
+
+TENSORS = ("wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down", "alpha_attn", "alpha_mlp",
+           "s_qk")
+
+
+def _block_weights(provider, b):
+    from synthetic.bf16 import bf16_bits_to_f32
+    raw = provider(b)
+    return {k: (bf16_bits_to_f32(v).astype(np.float64) if v.dtype == np.uint16
+                else np.asarray(v, dtype=np.float64)) for k, v in raw.items()}
+
+
+def _block_forward(cfg, W, h, b):
+    h = attention_sublayer_forward(cfg, W, h, b)["h_out"]
+    return mlp_sublayer_forward(cfg, W, h)["h_out"]
+
+
+def trained_part_forward(cfg, provider, x_k):
+    """The part of the stack that depth-one truncated back-propagation trains:
+    the final recurrent invocation on its input x_k, then the output block.
+    Returns the output and the input of every sublayer on the way."""
+    n_in, n_rec, n_out = cfg["n_in_blocks"], cfg["n_rec_blocks"], cfg["n_out_blocks"]
+    h = np.asarray(x_k, dtype=np.float64)
+    saved = []
+    for b in range(n_in, n_in + n_rec + n_out):
+        W = _block_weights(provider, b)
+        saved.append(("att", b, h))
+        h = attention_sublayer_forward(cfg, W, h, b)["h_out"]
+        saved.append(("mlp", b, h))
+        h = mlp_sublayer_forward(cfg, W, h)["h_out"]
+    return h, saved
+
+
+def last_loop_input(cfg, provider, h_in, k):
+    """x_k, the input of the final recurrent invocation of a training sequence
+    (positions 0..n-1): e = InputBlock(h_in), x_1 = e, x_{j+1} =
+    Norm(RecurrentBlock(x_j) + e) ("Dory1.0-4B: A Looped Normalized-GPT",
+    Methodology in Plain English: the input block's output is re-injected
+    before every pass)."""
+    n_in, n_rec = cfg["n_in_blocks"], cfg["n_rec_blocks"]
+    h = np.asarray(h_in, dtype=np.float64)
+    for b in range(n_in):
+        h = _block_forward(cfg, _block_weights(provider, b), h, b)
+    e = h
+    x = e
+    for _ in range(k - 1):
+        y = x
+        for b in range(n_in, n_in + n_rec):
+            y = _block_forward(cfg, _block_weights(provider, b), y, b)
+        s = y + e
+        x = s / np.sqrt(np.maximum((s * s).sum(axis=1, keepdims=True), cfg["norm_eps"]))
+    return x
+
+
+def last_loop_backward(cfg, provider, h_in, dh_out, k):
+    """Depth-one truncated back-propagation through a training sequence's stack
+    ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain English: only
+    the final recurrent invocation is trained): the loops before the last are
+    run forward only, their output x_k is a constant, and dL/dh_out flows back
+    through the output block and the final recurrent invocation.  Returns
+    h_out, dx (dL/dx_k) and per trained block b a dict of gradients named like
+    TENSORS."""
+    x_k = last_loop_input(cfg, provider, h_in, k)
+    h_out, saved = trained_part_forward(cfg, provider, x_k)
+    dh = np.asarray(dh_out, dtype=np.float64)
+    grads = {}
+    for kind, b, h in reversed(saved):
+        W = _block_weights(provider, b)
+        gb = grads.setdefault(b, {})
+        if kind == "mlp":
+            g = mlp_sublayer_backward(cfg, W, h, dh)
+            gb.update(w_gate=g["d_w_gate"], w_up=g["d_w_up"], w_down=g["d_w_down"],
+                      alpha_mlp=g["d_alpha"])
+        else:
+            g = attention_sublayer_backward(cfg, W, h, dh, b)
+            gb.update(wq=g["d_wq"], wk=g["d_wk"], wv=g["d_wv"], wg=g["d_wg"], wo=g["d_wo"],
+                      alpha_attn=g["d_alpha"], s_qk=g["d_s_qk"])
+        dh = g["dh"]
+    return dict(h_out=h_out, dx=dh, x_k=x_k, grads=grads)

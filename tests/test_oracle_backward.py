@@ -133,3 +133,63 @@ def test_attention_gradient_along_the_output_vanishes():
     g = attention_sublayer_backward(cfg, W, h, -2.0 * h_out, 1)
     for k in ("dh", "d_wq", "d_wk", "d_wv", "d_wg", "d_wo", "d_alpha", "d_s_qk"):
         assert np.abs(g[k]).max() < 1e-12, k
+
+
+# ------------------------------------------------------------------ the stack
+
+def _stack_setup(seed=21, rows=10):
+    cfg = load_config("tiny", d_model=64, n_q_heads=4, n_kv_heads=2, head_dim=16, d_ff=128,
+                      window=4, n_in_blocks=1, n_rec_blocks=2, n_out_blocks=1)
+    prov = weights_from_generator(cfg, seed, "random")
+    h = bf16_bits_to_f32(hidden_in(cfg, seed + 1, rows)).astype(np.float64)
+    dh_out = np.random.default_rng(seed + 2).standard_normal(h.shape)
+    return cfg, prov, h, dh_out
+
+
+def test_stack_forward_is_the_oracle_stack():
+    from oracle import KVCache
+    from oracle.backward import last_loop_backward
+    cfg, prov, h, dh_out = _stack_setup()
+    got = last_loop_backward(cfg, prov, h, dh_out, 3)["h_out"]
+    ref = Oracle(cfg, prov).forward(h, 0, 3, KVCache(cfg, "last_loop", k_max=3))
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_last_loop_gradients_match_truncated_differences():
+    """Finite differences of L = <dh_out, output> with the final invocation's
+    input x_k held fixed (the truncation): for x_k itself and for a parameter
+    of every trained block (the shared recurrent weights change only the final
+    invocation here)."""
+    from oracle.backward import last_loop_backward, trained_part_forward
+    cfg, prov, h, dh_out = _stack_setup()
+    res = last_loop_backward(cfg, prov, h, dh_out, 2)
+    x_k = res["x_k"]
+    rng = np.random.default_rng(9)
+    eps = 1e-6
+
+    def loss(p, xk):
+        return float((trained_part_forward(cfg, p, xk)[0] * dh_out).sum())
+    for _ in range(6):
+        ix = tuple(rng.integers(0, n) for n in x_k.shape)
+        xp, xm = x_k.copy(), x_k.copy()
+        xp[ix] += eps
+        xm[ix] -= eps
+        fd = (loss(prov, xp) - loss(prov, xm)) / (2 * eps)
+        assert abs(fd - res["dx"][ix]) <= 1e-6 * max(1.0, abs(fd))
+    for b in res["grads"]:
+        for name in ("wq", "w_down", "alpha_attn", "s_qk"):
+            base = prov(b)[name]
+            ix = tuple(rng.integers(0, n) for n in base.shape)
+
+            def bumped(delta):
+                def p(bb):
+                    w = dict(prov(bb))
+                    if bb == b:
+                        arr = (bf16_bits_to_f32(w[name]).astype(np.float64) if w[name].dtype == np.uint16
+                               else np.asarray(w[name], dtype=np.float64)).copy()
+                        arr[ix] += delta
+                        w[name] = arr
+                    return w
+                return p
+            fd = (loss(bumped(eps), x_k) - loss(bumped(-eps), x_k)) / (2 * eps)
+            assert abs(fd - res["grads"][b][name][ix]) <= 1e-6 * max(1.0, abs(fd)), (b, name)
