@@ -366,6 +366,29 @@ DORY_API size_t dory_mlp_backward_workspace_bytes(const dory_model* m, int n_row
  * held in the workspace, so the workspace
  * (dory_attention_backward_workspace_bytes) grows with n_rows squared.  bf16
  * weight format only (DORY_ERR_BAD_CONFIG otherwise). */
+/* Depth-one truncated back-propagation through the stack for one training
+ * sequence ("Dory1.0-4B: A Looped Normalized-GPT", Methodology in Plain
+ * English: only the final recurrent invocation is trained).  h_in [n_rows,
+ * d_model] (fp32, device; the sequence's positions 0..n_rows-1) runs forward
+ * as a prefill into `kv` (sequence 0, max_ctx >= n_rows): the input block,
+ * k - 1 loops of the recurrent block with re-injection, the final loop and the
+ * output block; the loops before the last are not differentiated, so their
+ * output x_k is a constant.  dL/dh_out [n_rows, d_model] then flows back
+ * through the output block and the final recurrent invocation.  Writes the
+ * output (h_out, optional), dL/dx_k [n_rows, d_model] (dx) and into `grads`
+ * the fp32 gradients of every trained block -- the n_rec_blocks recurrent
+ * blocks then the n_out_blocks output blocks, each as W_q, W_k, W_v, W_gate,
+ * W_o, W_mlp_gate, W_up, W_down (the shapes of dory_block_src), alpha_attn,
+ * alpha_mlp, s_qk, each tensor 256-byte aligned at the offset
+ * dory_last_loop_grad_layout reports (offsets[i * 11 + t] for trained block
+ * i, tensor t; it returns the total bytes).  bf16 weight format only. */
+DORY_API size_t dory_last_loop_grad_layout(const dory_model* m, size_t* offsets);
+DORY_API size_t dory_last_loop_backward_workspace_bytes(const dory_model* m, int n_rows);
+DORY_API int dory_last_loop_backward(dory_model* m, dory_kv* kv, int n_rows, const float* h_in,
+                                     const float* dh_out, int k, float* h_out, float* dx,
+                                     void* grads, size_t grad_bytes, void* ws, size_t ws_bytes,
+                                     void* stream);
+
 DORY_API size_t dory_attention_backward_workspace_bytes(const dory_model* m, int n_rows);
 DORY_API int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows,
                                               const float* h_in, const float* dh_out, float* dh_in,

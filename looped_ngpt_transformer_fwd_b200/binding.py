@@ -38,6 +38,8 @@ EXPORTS = (
     "dory_nvfp4_scale_bytes", "dory_gemm_nvfp4_workspace_bytes", "dory_gemm_nvfp4",
     "dory_gemm_bf16_mn", "dory_mlp_backward_workspace_bytes", "dory_mlp_sublayer_backward",
     "dory_attention_backward_workspace_bytes", "dory_attention_sublayer_backward",
+    "dory_last_loop_grad_layout", "dory_last_loop_backward_workspace_bytes",
+    "dory_last_loop_backward",
     "dory_vocab_bytes", "dory_vocab_create", "dory_embed", "dory_lm_head", "dory_sample",
     "dory_vocab_free",
 )
@@ -129,6 +131,9 @@ def lib():
             "dory_mlp_backward_workspace_bytes": (SZ, [P, I]),
             "dory_mlp_sublayer_backward": (I, [P, I, I, P, P, P, P, P, P, P, P, SZ, P]),
             "dory_attention_backward_workspace_bytes": (SZ, [P, I]),
+            "dory_last_loop_grad_layout": (SZ, [P, P]),
+            "dory_last_loop_backward_workspace_bytes": (SZ, [P, I]),
+            "dory_last_loop_backward": (I, [P, P, I, P, P, I, P, P, P, SZ, P, SZ, P]),
             "dory_attention_sublayer_backward": (I, [P, I, I] + [P] * 11 + [SZ, P]),
             "dory_vocab_bytes": (SZ, [P, I]),
             "dory_vocab_create": (I, [P, I, P, P, P, P, SZ, P, P]),
@@ -339,6 +344,29 @@ def dory_attention_sublayer_backward(m, layer, n_rows, h_in, dh_out, dh_in, d_wq
                                                         d_wk, d_wv, d_wg, d_wo, d_alpha, d_s_qk,
                                                         ws, ws_bytes, stream),
                  "dory_attention_sublayer_backward")
+
+
+GRAD_TENSORS = ("wq", "wk", "wv", "wg", "wo", "w_gate", "w_up", "w_down", "alpha_attn",
+                "alpha_mlp", "s_qk")
+
+
+def dory_last_loop_grad_layout(m, n_trained):
+    """(total bytes, [n_trained][11] byte offsets) of the gradient buffer."""
+    offs = (ctypes.c_size_t * (n_trained * len(GRAD_TENSORS)))()
+    total = lib().dory_last_loop_grad_layout(m, offs)
+    return total, [[offs[i * len(GRAD_TENSORS) + t] for t in range(len(GRAD_TENSORS))]
+                   for i in range(n_trained)]
+
+
+def dory_last_loop_backward_workspace_bytes(m, n_rows):
+    return lib().dory_last_loop_backward_workspace_bytes(m, n_rows)
+
+
+def dory_last_loop_backward(m, kv, n_rows, h_in, dh_out, k, h_out, dx, grads, grad_bytes, ws,
+                            ws_bytes, stream):
+    return check(lib().dory_last_loop_backward(m, kv, n_rows, h_in, dh_out, k, h_out, dx, grads,
+                                               grad_bytes, ws, ws_bytes, stream),
+                 "dory_last_loop_backward")
 
 
 def dory_quant_nvfp4(src, rows, K, g, d_g, codes, scales, stream):

@@ -169,6 +169,9 @@ struct dory_model {
   std::set<dory_kv*> caches;                   // live KV caches bound to this model
 };
 
+// tensors of one trained block's gradients, in the order of dory_last_loop_grad_layout
+constexpr int kGradTensors = 11;
+
 struct dory_kv {
   dory_model* m = nullptr;
   uint64_t uid = 0;
@@ -1614,6 +1617,127 @@ int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows, const
   e = e ? e : launch_colsum(f32(L.part), L.grid_row, d, d_alpha, s);
   e = e ? e : launch_colsum(f32(L.ds_part), L.grid_qk, hd, d_s_qk, s);
   return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
+}
+
+size_t dory_last_loop_grad_layout(const dory_model* m, size_t* offsets) {
+  if (!m) return 0;
+  const size_t d = m->d, hd = m->hd, da = size_t(m->hq) * hd, kvr = size_t(m->hkv) * hd,
+               ff = m->ff;
+  const size_t sizes[kGradTensors] = {da * d, kvr * d, kvr * d, size_t(m->hq) * d, d * da,
+                                      ff * d, ff * d, d * ff, d, d, hd};
+  const int trained = m->cfg.n_rec_blocks + m->cfg.n_out_blocks;
+  size_t o = 0;
+  for (int i = 0; i < trained; ++i)
+    for (int t = 0; t < kGradTensors; ++t) {
+      if (offsets) offsets[i * kGradTensors + t] = o;
+      o = align_up(o + sizes[t] * 4);
+    }
+  return o;
+}
+
+size_t dory_last_loop_backward_workspace_bytes(const dory_model* m, int n_rows) {
+  if (!m || n_rows <= 0) return 0;
+  const size_t act = align_up(size_t(n_rows) * m->d * 4);
+  const int saved = 2 * (m->cfg.n_rec_blocks + m->cfg.n_out_blocks);
+  return align_up(ws_layout(m, n_rows).total) + (saved + 2) * act +
+         std::max(bwd_layout(m, n_rows).total, attn_bwd_layout(m, n_rows).total);
+}
+
+int dory_last_loop_backward(dory_model* m, dory_kv* kv, int n_rows, const float* h_in,
+                            const float* dh_out, int k, float* h_out, float* dx, void* grads,
+                            size_t grad_bytes, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !kv || kv->m != m || !h_in || !dh_out || !dx || !grads || !ws || n_rows <= 0)
+    return DORY_ERR_INVALID_ARG;
+  if (m->mx) return DORY_ERR_BAD_CONFIG;   // bf16 weights only
+  if (k < 1 || k > (m->cfg.allow_extrapolated_k ? 8 : 4)) return DORY_ERR_K_RANGE;
+  if (kv->mode == DORY_KV_PER_LOOP && k > kv->k_max) return DORY_ERR_K_EXCEEDS_KMAX;
+  if (n_rows > kv->max_ctx) return DORY_ERR_CTX_OVERFLOW;
+  if (!is_aligned(h_in, 16) || !is_aligned(dh_out, 16) || !is_aligned(dx, 16) ||
+      (h_out && !is_aligned(h_out, 16)) || !is_aligned(grads) || !is_aligned(ws))
+    return DORY_ERR_MISALIGNED;
+  if (grad_bytes < dory_last_loop_grad_layout(m, nullptr) ||
+      ws_bytes < dory_last_loop_backward_workspace_bytes(m, n_rows))
+    return DORY_ERR_BUFFER_TOO_SMALL;
+  const int T = n_rows, n_in = m->cfg.n_in_blocks, n_rec = m->cfg.n_rec_blocks, nb = m->nb;
+  const size_t act = align_up(size_t(T) * m->d * 4);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  uint8_t* saved = b + align_up(ws_layout(m, T).total);
+  const int n_saved = 2 * (nb - n_in);
+  float* A = reinterpret_cast<float*>(saved + size_t(n_saved) * act);
+  float* Bf = reinterpret_cast<float*>(saved + size_t(n_saved + 1) * act);
+  uint8_t* sub = saved + size_t(n_saved + 2) * act;
+  const size_t sub_bytes = ws_bytes - size_t(sub - b);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto save = [&](int i, const float* h) {
+    return cudaMemcpyAsync(saved + size_t(i) * act, h, size_t(T) * m->d * 4,
+                           cudaMemcpyDeviceToDevice, s);
+  };
+
+  // ---- forward: the stack as a prefill of the sequence at position 0, the
+  // inputs of the final recurrent invocation's and the output block's
+  // sublayers saved
+  CallCtx c;
+  c.m = m; c.kv = kv; c.w = ws_bind(m, b, T); c.n = T; c.decode = false;
+  c.seq = 0; c.pos0 = 0; c.dseq = nullptr; c.dpos = nullptr; c.max_pos = T - 1; c.k = k;
+  c.s = s;
+  m->cur_launches = m->cur_sublayers = 0;
+  for (int i = 0; i < kPaths; ++i) m->cur_paths[i] = 0;
+  cudaError_t e = cudaMemcpyAsync(c.w.h32, h_in, size_t(T) * m->d * 4, cudaMemcpyDeviceToDevice, s);
+  e = e ? e : launch_f32_to_bf16(c.w.h32, c.w.hb, size_t(T) * m->d, s);
+  e = e ? e : enqueue_rope_tables(c);
+  const bool last_loop = kv->mode == DORY_KV_LAST_LOOP;
+  for (int blk = 0; blk < n_in && e == cudaSuccess; ++blk) {
+    const bool last = blk == n_in - 1;
+    e = attention_sublayer(c, blk, 1, c.w.h32, c.w.hb, true);
+    e = e ? e : mlp_sublayer(c, blk, c.w.h32, c.w.hb, last, last, nullptr);
+  }
+  int si = 0;
+  for (int j = 1; j <= k && e == cudaSuccess; ++j) {
+    for (int blk = n_in; blk < n_in + n_rec && e == cudaSuccess; ++blk) {
+      const bool commit = !last_loop || j == k;
+      if (j == k) e = save(si++, c.w.h32);
+      e = e ? e : attention_sublayer(c, blk, j, c.w.h32, c.w.hb, commit);
+      if (j == k) e = e ? e : save(si++, c.w.h32);
+      const bool reinject = (blk == n_in + n_rec - 1) && j < k;
+      e = e ? e : mlp_sublayer(c, blk, c.w.h32, c.w.hb, false, reinject, nullptr, j);
+    }
+  }
+  for (int blk = n_in + n_rec; blk < nb && e == cudaSuccess; ++blk) {
+    e = save(si++, c.w.h32);
+    e = e ? e : attention_sublayer(c, blk, 1, c.w.h32, c.w.hb, true);
+    e = e ? e : save(si++, c.w.h32);
+    e = e ? e : mlp_sublayer(c, blk, c.w.h32, c.w.hb, false, false, nullptr);
+  }
+  if (e == cudaSuccess && h_out)
+    e = cudaMemcpyAsync(h_out, c.w.h32, size_t(T) * m->d * 4, cudaMemcpyDeviceToDevice, s);
+  e = e ? e : cudaMemcpyAsync(A, dh_out, size_t(T) * m->d * 4, cudaMemcpyDeviceToDevice, s);
+  for (int i = 0; i < kPaths; ++i) m->last_paths[i] = m->cur_paths[i];
+  if (e != cudaSuccess) return DORY_ERR_CUDA;
+
+  // ---- backward through the output block, then the final recurrent invocation
+  size_t off[kGradTensors * 64];
+  const int trained = nb - n_in;
+  if (trained > 64) return DORY_ERR_BAD_CONFIG;
+  dory_last_loop_grad_layout(m, off);
+  uint8_t* g = static_cast<uint8_t*>(grads);
+  auto gp = [&](int blk, int t) { return reinterpret_cast<float*>(g + off[(blk - n_in) * kGradTensors + t]); };
+  for (int i = n_saved - 1; i >= 0; --i) {
+    const int blk = n_in + i / 2;
+    const float* hin = reinterpret_cast<const float*>(saved + size_t(i) * act);
+    int st;
+    if (i % 2 == 1)
+      st = dory_mlp_sublayer_backward(m, blk, T, hin, A, Bf, gp(blk, 5), gp(blk, 6), gp(blk, 7),
+                                      gp(blk, 9), sub, sub_bytes, stream);
+    else
+      st = dory_attention_sublayer_backward(m, blk, T, hin, A, Bf, gp(blk, 0), gp(blk, 1),
+                                            gp(blk, 2), gp(blk, 3), gp(blk, 4), gp(blk, 8),
+                                            gp(blk, 10), sub, sub_bytes, stream);
+    if (st != DORY_OK) return st;
+    std::swap(A, Bf);
+  }
+  if (cudaMemcpyAsync(dx, A, size_t(T) * m->d * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  return DORY_OK;
 }
 
 int dory_gemm_bf16_mn(const void* A, const void* B, float* C, int M, int N, int K, int a_mn,

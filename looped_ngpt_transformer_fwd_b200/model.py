@@ -212,6 +212,38 @@ class DoryModel:
                             _stream(stream))
         return h
 
+    def last_loop_backward(self, kv, h, dh_out, k, stream=None):
+        """Depth-one truncated back-propagation of one training sequence (rows of
+        h = positions 0..n-1, fp32 [n, d] device tensors): returns h_out, dx
+        (dL/dx_k) and grads[b][name] for every trained block b (recurrent, then
+        output blocks; names as binding.GRAD_TENSORS, shapes of the weights)."""
+        n, d = h.shape
+        c = self.cfg
+        hq, hkv, hd, ff = c["n_q_heads"], c["n_kv_heads"], c["head_dim"], c["d_ff"]
+        n_in = c["n_in_blocks"]
+        trained = list(range(n_in, self.n_blocks))
+        total, offs = B.dory_last_loop_grad_layout(self.handle, len(trained))
+        gbuf = torch.empty(total, dtype=torch.uint8, device=self.device)
+        ws = torch.empty(B.dory_last_loop_backward_workspace_bytes(self.handle, n),
+                         dtype=torch.uint8, device=self.device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        h_out = torch.empty(n, d, **f32)
+        dx = torch.empty(n, d, **f32)
+        B.dory_last_loop_backward(self.handle, kv.handle, n, _ptr(h), _ptr(dh_out), k, _ptr(h_out),
+                                  _ptr(dx), _ptr(gbuf), gbuf.numel(), _ptr(ws), ws.numel(),
+                                  _stream(stream))
+        shapes = dict(wq=(hq * hd, d), wk=(hkv * hd, d), wv=(hkv * hd, d), wg=(hq, d),
+                      wo=(d, hq * hd), w_gate=(ff, d), w_up=(ff, d), w_down=(d, ff),
+                      alpha_attn=(d,), alpha_mlp=(d,), s_qk=(hd,))
+        grads = {}
+        for i, b in enumerate(trained):
+            grads[b] = {}
+            for t, name in enumerate(B.GRAD_TENSORS):
+                nel = int(np.prod(shapes[name]))
+                grads[b][name] = gbuf[offs[i][t]:offs[i][t] + 4 * nel].view(torch.float32).view(
+                    *shapes[name])
+        return dict(h_out=h_out, dx=dx, grads=grads, buffer=gbuf)
+
     def attention_sublayer_backward(self, layer, h, dh_out, stream=None):
         """Gradients of one attention sublayer on a training sequence (rows =
         positions 0..n-1) given its input h and dL/dh_out (fp32 [n, d] device

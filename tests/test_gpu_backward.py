@@ -167,3 +167,40 @@ def test_attention_gradient_along_the_output_vanishes_on_the_gpu():
     for k in ("dh", "d_wq", "d_wk", "d_wv", "d_wg", "d_wo"):
         assert along[k].abs().max().item() < 0.05 * typical[k].abs().max().item(), k
     model.close()
+
+
+# ------------------------------------------------------------------ the stack
+
+# Bar for the whole truncated backward: the rounding of every sublayer's
+# recomputed forward and backward operands to bf16 adds up along the chain
+# (12 sublayers for the tiny stack), so it could exceed one sublayer's error;
+# measured it stays at the sublayer level (worst tensor 8.3e-3 relative,
+# cosine 0.99997; dL/dx_k 1.4e-3), and the chain keeps the sublayer bar.
+CHAIN_REL, CHAIN_COS = REL_FRO, MIN_COS
+
+
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_last_loop_backward_matches_the_oracle(k):
+    from oracle.backward import last_loop_backward
+    from tests.gpu_util import assert_parity
+    cfg, prov, model = build("tiny", seed=61)
+    _, h = inputs(cfg, 62, 64)
+    dh_out = np.random.default_rng(63).standard_normal(h.shape) * 0.1
+    kv = model.kv_cache("last_loop", 1, 64)
+    res = model.last_loop_backward(kv, torch.from_numpy(h.astype(np.float32)).cuda(),
+                                   torch.from_numpy(dh_out.astype(np.float32)).cuda(), k)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    ref = last_loop_backward(cfg, prov, h, dh_out, k)
+    assert_parity(to_np(res["h_out"]), ref["h_out"], what=f"training forward k={k}")
+    worst = (0.0, 1.0)
+    for b, gb in ref["grads"].items():
+        for name, want in gb.items():
+            g, w = to_np(res["grads"][b][name]).ravel(), np.asarray(want).ravel()
+            rel = np.linalg.norm(g - w) / np.linalg.norm(w)
+            cos = float(g @ w / (np.linalg.norm(g) * np.linalg.norm(w)))
+            worst = (max(worst[0], rel), min(worst[1], cos))
+            assert rel <= CHAIN_REL and cos >= CHAIN_COS, f"block {b} {name}: rel {rel:.3e} cos {cos:.6f}"
+    g, w = to_np(res["dx"]).ravel(), ref["dx"].ravel()
+    assert np.linalg.norm(g - w) / np.linalg.norm(w) <= CHAIN_REL
+    model.close()
