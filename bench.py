@@ -17,6 +17,8 @@ SWA:full 3:1 with window 4096, bf16 weights and activations):
   prefill_k2_mxfp8 / decode_k2_mxfp8, prefill_k2_nvfp4 / decode_k2_nvfp4
                the prefill_k2 / decode_k2 shapes with MXFP8 or NVFP4 weights and
                projection inputs (block-scaled tensor-core GEMMs)
+  train_k2     (extra only) one training step of depth-one truncated
+               back-propagation, 1 x 4096 tokens, k = 2
 
 N > 1 runs N independent replicas (one per GPU, no collective on the data
 path; the harness only uses a barrier and a max-reduction of the timings).
@@ -57,6 +59,10 @@ WORKLOADS = {
                              fmt="nvfp4"),
     "decode_k2_nvfp4": dict(kind="decode", batch=64, ctx=32768, k=2, mode="last_loop", seed=2,
                             fmt="nvfp4"),
+    # one training step of depth-one truncated back-propagation: the stack's
+    # forward, then the backward through the output block and the final
+    # recurrent invocation (an extra workload only)
+    "train_k2": dict(kind="train", tokens=4096, k=2, mode="last_loop", seed=1),
 }
 
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
@@ -130,6 +136,20 @@ def prefill_flops(cfg, T, k, pos0=0):
     per_pair = 4 * cfg["head_dim"] * cfg["n_q_heads"]
     blocks = stack_blocks(cfg, k)
     return sum(block_gemm_flops(cfg) * T + per_pair * attn_pairs(cfg, b, T, pos0) for b in blocks)
+
+
+def train_flops(cfg, T, k):
+    """Algorithmic FLOPs of one truncated training step on a T-token sequence:
+    the forward of the whole stack, then for every trained block (the final
+    recurrent invocation and the output block) its GEMMs three times (the
+    recomputed forward, dgrad and wgrad) and its attention three times (the
+    recomputed S and P V; dP, dV, dQ and dK), unmasked pairs only."""
+    n_in = cfg["n_in_blocks"]
+    nb = n_in + cfg["n_rec_blocks"] + cfg["n_out_blocks"]
+    per_pair = 4 * cfg["head_dim"] * cfg["n_q_heads"]
+    bwd = sum(3 * block_gemm_flops(cfg) * T + 3 * per_pair * attn_pairs(cfg, b, T)
+              for b in range(n_in, nb))
+    return prefill_flops(cfg, T, k) + bwd
 
 
 def decode_kv_bytes(cfg, B, pos, k):
@@ -404,6 +424,53 @@ def run_ours(args, wl, rank, world, device_index, model=None, prov=None, steps=N
     return res
 
 
+def run_train(args, wl, model, device_index, steps, warmup, peaks, peak_src):
+    """Time the truncated training step (dory_last_loop_backward) on the 4B
+    shapes; the roofline is the whole step's algorithmic FLOPs over its device
+    time against the sustained bf16 figure."""
+    import torch
+    from synthetic import hidden_in
+    from synthetic.bf16 import bf16_bits_to_f32
+    cfg = model.cfg
+    T, k = wl["tokens"], wl["k"]
+    h = torch.from_numpy(bf16_bits_to_f32(hidden_in(cfg, wl["seed"], T)).astype(np.float32)).cuda()
+    g = torch.Generator(device="cuda").manual_seed(wl["seed"])
+    dh = torch.randn(T, cfg["d_model"], device="cuda", generator=g) * 0.1
+    kv = model.kv_cache(wl["mode"], 1, T, k_max=k)
+    stream = torch.cuda.current_stream()
+    out = None
+    for _ in range(warmup):
+        out = model.last_loop_backward(kv, h, dh, k)
+    torch.cuda.synchronize()
+    if model.device_status() != 0:
+        raise RuntimeError("device status after the training warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_index) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            out = model.last_loop_backward(kv, h, dh, k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    flops = train_flops(cfg, T, k)
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    roof = {"bound": "tensor", "kernel": "whole step (stack forward + truncated backward)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{peak_src} (bf16_tflops_sustained)",
+            "frac_of_datasheet": achieved / DATASHEET["tensor"], "traffic": None,
+            "work_per_launch": flops, "launches_per_step": 1, "device_ms_per_step": ms}
+    grad_bytes = int(out["buffer"].numel())
+    del out, kv, h, dh
+    return {"tokens_per_s": T / ms * 1e3, "ms_per_step": ms, "steps": steps, "warmup": warmup,
+            "workload": f"dory4b training step 1x{T} k={k}: stack forward + depth-one truncated "
+                        "backward (final recurrent invocation and output block)",
+            "e2e_tokens_per_s": None, "roofline": roof, "clocks": clk.summary(),
+            "flops_per_step": flops, "tokens_per_step": T, "gradient_bytes": grad_bytes,
+            "dtype": "bf16 operands, fp32 accumulation and gradients", "k": k,
+            "kv_mode": wl["mode"]}
+
+
 def block_override(args):
     if not args.blocks:
         return {}
@@ -552,7 +619,8 @@ def footprint_check(cfg, wl):
 
 
 DEFAULT_EXTRAS = ["prefill_k1", "decode_k2", "decode_k4_last", "decode_k4_per",
-                  "prefill_k2_mxfp8", "decode_k2_mxfp8", "prefill_k2_nvfp4", "decode_k2_nvfp4"]
+                  "prefill_k2_mxfp8", "decode_k2_mxfp8", "prefill_k2_nvfp4", "decode_k2_nvfp4",
+                  "train_k2"]
 DTYPES = {"bf16": "bf16",
           "mxfp8": "mxfp8 (E4M3 x E4M3, E8M0 block scales, fp32 accumulation)",
           "nvfp4": "nvfp4 (E2M1 x E2M1, E4M3 block scales of 16, fp32 tensor scales, "
@@ -565,7 +633,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill_k2", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="prefill_k2",
+                    choices=sorted(n for n, w in WORKLOADS.items() if w["kind"] != "train"))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--blocks", default=None,
@@ -638,6 +707,12 @@ def main():
         xwl = dict(WORKLOADS[name])
         xsteps = min(args.steps, 10)
         fmt = xwl.get("fmt", "bf16")
+        if xwl["kind"] == "train":
+            import torch
+            extras[name] = run_train(args, xwl, res["model"], local, min(xsteps, 5), args.warmup,
+                                     peaks, peak_src)
+            torch.cuda.empty_cache()
+            continue
         if fmt not in models:
             from looped_ngpt_transformer_fwd_b200.model import DoryModel
             models[fmt] = DoryModel(res["cfg"], res["prov"], device=f"cuda:{local}",
