@@ -40,9 +40,37 @@ __global__ void gather_heads_kernel(const __nv_bfloat16* __restrict__ src, int T
       reinterpret_cast<const uint4*>(src + (static_cast<size_t>(t) * src_heads + head0 + g) * hd)[c];
 }
 
+// Eight consecutive fp32 values and eight bf16 values (16-byte accesses; row
+// pitches are multiples of 8 elements).
+__device__ __forceinline__ void ld8f(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ld8h(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ void st8h(__nv_bfloat16* p, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
+  v = is_max ? warp_max_f(v) : warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = is_max ? -INFINITY : 0.f;
+  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w)
+    r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();   // red is reused by the next reduction
+  return r;
+}
+
 // One CTA per row r of S [rows, ld] (row r is query t = r % T): P = masked
 // softmax(scale S) over keys j in [lo(t), t] (lo = max(0, t - W + 1) for a
-// window W, else 0), bf16, zeros elsewhere up to ld.
+// window W, else 0), bf16, zeros elsewhere up to ld.  Eight keys per access.
 __global__ void softmax_rows_kernel(const float* __restrict__ S, int T, int ld, int window,
                                     float scale, __nv_bfloat16* __restrict__ P) {
   __shared__ float red[32];
@@ -51,45 +79,70 @@ __global__ void softmax_rows_kernel(const float* __restrict__ S, int T, int ld, 
   const int lo = window > 0 ? max(0, t - window + 1) : 0;
   const float* s = S + static_cast<size_t>(r) * ld;
   __nv_bfloat16* p = P + static_cast<size_t>(r) * ld;
+  const int c0 = lo / 8, c1 = t / 8;   // chunks holding visible keys
   float m = -INFINITY;
-  for (int j = lo + threadIdx.x; j <= t; j += blockDim.x) m = fmaxf(m, s[j]);
-  m = warp_max_f(m);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  float mm = -INFINITY;
-  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w) mm = fmaxf(mm, red[w]);
-  __syncthreads();
+  for (int c = c0 + threadIdx.x; c <= c1; c += blockDim.x) {
+    float v[8];
+    ld8f(s + 8 * c, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (8 * c + u >= lo && 8 * c + u <= t) m = fmaxf(m, v[u]);
+  }
+  m = block_reduce(m, red, true);
   float l = 0.f;
-  for (int j = lo + threadIdx.x; j <= t; j += blockDim.x) l += __expf(scale * (s[j] - mm));
-  l = warp_sum(l);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = l;
-  __syncthreads();
-  float ll = 0.f;
-  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w) ll += red[w];
-  const float inv = 1.f / ll;
-  for (int j = threadIdx.x; j < ld; j += blockDim.x) {
-    const float v = (j >= lo && j <= t) ? __expf(scale * (s[j] - mm)) * inv : 0.f;
-    p[j] = __float2bfloat16_rn(v);
+  for (int c = c0 + threadIdx.x; c <= c1; c += blockDim.x) {
+    float v[8];
+    ld8f(s + 8 * c, v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (8 * c + u >= lo && 8 * c + u <= t) l += __expf(scale * (v[u] - m));
+  }
+  const float inv = 1.f / block_reduce(l, red, false);
+  for (int c = threadIdx.x; c < ld / 8; c += blockDim.x) {
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c >= c0 && c <= c1) {
+      float x[8];
+      ld8f(s + 8 * c, x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = (8 * c + u >= lo && 8 * c + u <= t) ? __expf(scale * (x[u] - m)) * inv : 0.f;
+    }
+    st8h(p + 8 * c, v);
   }
 }
 
-// dS = scale * P * (dP - D), D = sum_j P dP over the row (one CTA per row)
+// dS = scale * P * (dP - D), D = sum_j P dP over the row's visible keys (one
+// CTA per row, query t = row % T); entries outside [lo(t), t] are zero and
+// their dP is not read (the dP GEMM skips tiles above the diagonal).
 __global__ void softmax_bwd_rows_kernel(const __nv_bfloat16* __restrict__ P,
-                                        const float* __restrict__ dP, int ld, float scale,
-                                        __nv_bfloat16* __restrict__ dS) {
+                                        const float* __restrict__ dP, int T, int ld, int window,
+                                        float scale, __nv_bfloat16* __restrict__ dS) {
   __shared__ float red[32];
   const size_t off = static_cast<size_t>(blockIdx.x) * ld;
+  const int t = blockIdx.x % T;
+  const int lo = window > 0 ? max(0, t - window + 1) : 0;
+  const int c0 = lo / 8, c1 = t / 8;
   float acc = 0.f;
-  for (int j = threadIdx.x; j < ld; j += blockDim.x)
-    acc += __bfloat162float(P[off + j]) * dP[off + j];
-  acc = warp_sum(acc);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
-  __syncthreads();
-  float D = 0.f;
-  for (int w = 0; w < static_cast<int>((blockDim.x + 31) >> 5); ++w) D += red[w];
-  for (int j = threadIdx.x; j < ld; j += blockDim.x) {
-    const float pj = __bfloat162float(P[off + j]);
-    dS[off + j] = __float2bfloat16_rn(scale * pj * (dP[off + j] - D));
+  for (int c = c0 + threadIdx.x; c <= c1; c += blockDim.x) {
+    float pv[8], dv[8];
+    ld8h(P + off + 8 * c, pv);
+    ld8f(dP + off + 8 * c, dv);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (8 * c + u >= lo && 8 * c + u <= t) acc += pv[u] * dv[u];
+  }
+  const float D = block_reduce(acc, red, false);
+  for (int c = threadIdx.x; c < ld / 8; c += blockDim.x) {
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c >= c0 && c <= c1) {
+      float pv[8], dv[8];
+      ld8h(P + off + 8 * c, pv);
+      ld8f(dP + off + 8 * c, dv);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = (8 * c + u >= lo && 8 * c + u <= t) ? scale * pv[u] * (dv[u] - D) : 0.f;
+    }
+    st8h(dS + off + 8 * c, v);
   }
 }
 
@@ -259,14 +312,17 @@ cudaError_t launch_gather_heads(const __nv_bfloat16* src, int T, int src_heads, 
 cudaError_t launch_softmax_rows(const float* S, int rows, int T, int ld, int window, float scale,
                                 __nv_bfloat16* P, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  if (ld % 8) return cudaErrorInvalidValue;
   softmax_rows_kernel<<<rows, 256, 0, s>>>(S, T, ld, window, scale, P);
   return cudaGetLastError();
 }
 
-cudaError_t launch_softmax_bwd_rows(const __nv_bfloat16* P, const float* dP, int rows, int ld,
-                                    float scale, __nv_bfloat16* dS, cudaStream_t s) {
+cudaError_t launch_softmax_bwd_rows(const __nv_bfloat16* P, const float* dP, int rows, int T,
+                                    int ld, int window, float scale, __nv_bfloat16* dS,
+                                    cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  softmax_bwd_rows_kernel<<<rows, 256, 0, s>>>(P, dP, ld, scale, dS);
+  if (ld % 8) return cudaErrorInvalidValue;
+  softmax_bwd_rows_kernel<<<rows, 256, 0, s>>>(P, dP, T, ld, window, scale, dS);
   return cudaGetLastError();
 }
 

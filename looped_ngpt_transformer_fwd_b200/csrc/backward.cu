@@ -134,14 +134,25 @@ __global__ void mlp_bwd_row_kernel(const float* __restrict__ y, const float* __r
   }
 }
 
-// out[c] = sum over g of part[g][c], in g order (deterministic)
+// out[c] = sum over g of part[g][c]: 32 columns per CTA, 8 row lanes each
+// summing every 8th group in order, then the 8 partial sums in lane order (a
+// fixed order: deterministic)
 __global__ void colsum_kernel(const float* __restrict__ part, int groups, int d,
                               float* __restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d) return;
+  __shared__ float sm[8][33];
+  const int cx = threadIdx.x & 31, gy = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + cx;
   float s = 0.f;
-  for (int g = 0; g < groups; ++g) s += part[static_cast<size_t>(g) * d + c];
-  out[c] = s;
+  if (c < d)
+    for (int g = gy; g < groups; g += 8) s += part[static_cast<size_t>(g) * d + c];
+  sm[gy][cx] = s;
+  __syncthreads();
+  if (gy == 0 && c < d) {
+    float t = 0.f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) t += sm[y][cx];
+    out[c] = t;
+  }
 }
 
 // SwiGLU backward over [rows, ff]: g, u from the fp32 products laid out like
@@ -208,7 +219,7 @@ cudaError_t launch_mlp_bwd_row(const float* y, const float* h, const float* alph
 
 cudaError_t launch_colsum(const float* part, int groups, int d, float* out, cudaStream_t s) {
   if (d <= 0) return cudaSuccess;
-  colsum_kernel<<<(d + 255) / 256, 256, 0, s>>>(part, groups, d, out);
+  colsum_kernel<<<(d + 31) / 32, 256, 0, s>>>(part, groups, d, out);
   return cudaGetLastError();
 }
 

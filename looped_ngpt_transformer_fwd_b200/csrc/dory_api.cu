@@ -152,6 +152,11 @@ struct dory_model {
   double* inv_freq_full = nullptr;
   std::vector<BlockW> blocks;
   cudaStream_t cap_stream = nullptr;
+  // the attention backward runs its KV heads concurrently on these (created on
+  // first use, forked from and joined to the caller's stream by events)
+  std::vector<cudaStream_t> aux_streams;
+  std::vector<cudaEvent_t> aux_events;
+  cudaEvent_t fork_event = nullptr;
   std::map<GraphKey, GraphEntry> graphs;
   uint64_t tick = 0;
   int last_launches = 0, last_sublayers = 0;
@@ -1316,6 +1321,9 @@ void dory_destroy(dory_model* m) {
   for (auto& g : m->graphs) destroy_entry(g.second);
   for (dory_kv* kv : m->caches) kv->m = nullptr;   // caches outliving the model stay freeable
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  for (cudaStream_t x : m->aux_streams) cudaStreamDestroy(x);
+  for (cudaEvent_t x : m->aux_events) cudaEventDestroy(x);
+  if (m->fork_event) cudaEventDestroy(m->fork_event);
   delete m;
 }
 
@@ -1394,7 +1402,7 @@ BwdLayout bwd_layout(const dory_model* m, int R) {
 // reads zeros.
 cudaError_t gemm_f32(const dory_model* m, const void* A, int a_mn, const void* B, int b_mn,
                      float* C, int M, int N, int K, cudaStream_t s, int ld_out = 0, int lda = 0,
-                     int ldb = 0) {
+                     int ldb = 0, int causal = kCausalNone, int causal_T = 0) {
   const int BN = (N % 256 == 0) ? 256 : 128;
   CUtensorMap ta, tb;
   const bool ok =
@@ -1405,6 +1413,7 @@ cudaError_t gemm_f32(const dory_model* m, const void* A, int a_mn, const void* B
   p.M = M; p.N = N; p.K = (K + 63) / 64 * 64;
   p.epi = kEpiStoreF32; p.out_f32 = C; p.ld_out = ld_out > 0 ? ld_out : N;
   p.a_mn = a_mn; p.b_mn = b_mn;
+  p.causal = causal; p.causal_T = causal_T;
   p.status = m->status;
   return launch_gemm(ta, tb, p, BN, 128, m->num_sms, s);
 }
@@ -1436,7 +1445,7 @@ AttnBwdLayout attn_bwd_layout(const dory_model* m, int T) {
   L.qs = take(hkv * G * t * hd * 2);       // per KV head: its group's queries stacked
   L.ks = take(hkv * t * hd * 2);
   L.vs = take(hkv * t * hd * 2);
-  L.S = take(G * t * tp * 4);              // S, then dP (one KV head at a time)
+  L.S = take(hkv * G * t * tp * 4);        // per KV head: S, then dP
   L.P = take(hkv * G * t * tp * 2);        // P of every KV head
   L.Os = take(hkv * G * t * hd * 4);       // P V before the gate
   L.o = take(t * da * 2);
@@ -1445,10 +1454,10 @@ AttnBwdLayout attn_bwd_layout(const dory_model* m, int T) {
   L.part = take(size_t(L.grid_row) * d * 4);
   L.dout = take(t * da * 4);
   L.dOs = take(hkv * G * t * hd * 2);
-  L.dS = take(G * t * tp * 2);
-  L.dV = take(t * hd * 4);
-  L.dQ = take(G * t * hd * 4);
-  L.dK = take(t * hd * 4);
+  L.dS = take(hkv * G * t * tp * 2);
+  L.dV = take(hkv * t * hd * 4);
+  L.dQ = take(hkv * G * t * hd * 4);
+  L.dK = take(hkv * t * hd * 4);
   L.dq_hat = take(t * hq * hd * 4);
   L.dk_hat = take(t * hkv * hd * 4);
   L.dv = take(t * hkv * hd * 4);
@@ -1513,6 +1522,49 @@ int dory_mlp_sublayer_backward(dory_model* m, int layer, int n_rows, const float
   return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// n auxiliary streams of the model (created on first use)
+bool aux_streams(dory_model* m, int n) {
+  if (!m->fork_event && cudaEventCreateWithFlags(&m->fork_event, cudaEventDisableTiming) != cudaSuccess)
+    return false;
+  while (static_cast<int>(m->aux_streams.size()) < n) {
+    cudaStream_t x;
+    cudaEvent_t ev;
+    if (cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(x);
+      return false;
+    }
+    m->aux_streams.push_back(x);
+    m->aux_events.push_back(ev);
+  }
+  return true;
+}
+
+// Work recorded on `s` so far happens before what is enqueued next on the
+// first n auxiliary streams, and what those hold happens before what is
+// enqueued next on `s`.
+cudaError_t fork_streams(dory_model* m, int n, cudaStream_t s) {
+  cudaError_t e = cudaEventRecord(m->fork_event, s);
+  for (int i = 0; i < n && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(m->aux_streams[i], m->fork_event, 0);
+  return e;
+}
+cudaError_t join_streams(dory_model* m, int n, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < n && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(m->aux_events[i], m->aux_streams[i]);
+    e = e ? e : cudaStreamWaitEvent(s, m->aux_events[i], 0);
+  }
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t dory_attention_backward_workspace_bytes(const dory_model* m, int n_rows) {
   if (!m || n_rows <= 0) return 0;
   return attn_bwd_layout(m, n_rows).total;
@@ -1558,18 +1610,25 @@ int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows, const
     pp.q_out = bf(L.qh); pp.k_out = bf(L.kh); pp.v_out = bf(L.vb); pp.gate_out = f32(L.gate);
     e = launch_qkvg_post(pp, s);
   }
+  // the KV heads run concurrently, one auxiliary stream each
+  if (!aux_streams(m, hkv)) return DORY_ERR_CUDA;
+  e = e ? e : fork_streams(m, hkv, s);
   for (int h = 0; h < hkv && e == cudaSuccess; ++h) {
+    cudaStream_t hs = m->aux_streams[h];
     __nv_bfloat16* qs = bf(L.qs) + h * head_q;
     __nv_bfloat16* ks = bf(L.ks) + h * head_kv;
     __nv_bfloat16* vs = bf(L.vs) + h * head_kv;
     __nv_bfloat16* P = bf(L.P) + h * head_p;
-    e = e ? e : launch_gather_heads(bf(L.qh), T, hq, h * G, G, hd, qs, s);
-    e = e ? e : launch_gather_heads(bf(L.kh), T, hkv, h, 1, hd, ks, s);
-    e = e ? e : launch_gather_heads(bf(L.vb), T, hkv, h, 1, hd, vs, s);
-    e = e ? e : gemm_f32(m, qs, 0, ks, 0, f32(L.S), G * T, T, hd, s, Tp);          // S = Q_s K^T
-    e = e ? e : launch_softmax_rows(f32(L.S), G * T, T, Tp, window, scale, P, s);
-    e = e ? e : gemm_f32(m, P, 0, vs, 1, f32(L.Os) + h * head_q, G * T, hd, T, s, 0, Tp);   // P V
+    float* S = f32(L.S) + h * head_p;
+    e = e ? e : launch_gather_heads(bf(L.qh), T, hq, h * G, G, hd, qs, hs);
+    e = e ? e : launch_gather_heads(bf(L.kh), T, hkv, h, 1, hd, ks, hs);
+    e = e ? e : launch_gather_heads(bf(L.vb), T, hkv, h, 1, hd, vs, hs);
+    e = e ? e : gemm_f32(m, qs, 0, ks, 0, S, G * T, T, hd, hs, Tp, 0, 0, kCausalTiles, T);
+    e = e ? e : launch_softmax_rows(S, G * T, T, Tp, window, scale, P, hs);
+    e = e ? e : gemm_f32(m, P, 0, vs, 1, f32(L.Os) + h * head_q, G * T, hd, T, hs, 0, Tp, 0,
+                         kCausalKeysK, T);                                          // P V
   }
+  e = e ? e : join_streams(m, hkv, s);
   e = e ? e : launch_gated_output(f32(L.Os), f32(L.gate), T, hq, G, hd, bf(L.o), s);
   e = e ? e : gemm_f32(m, bf(L.o), 0, W.wo, 0, f32(L.y), T, d, da, s);
 
@@ -1581,22 +1640,35 @@ int dory_attention_sublayer_backward(dory_model* m, int layer, int n_rows, const
   e = e ? e : cudaMemsetAsync(b + L.d_raw, 0, size_t(T) * ldq * 2, s);
   e = e ? e : launch_gate_bwd(f32(L.dout), f32(L.Os), f32(L.gate), T, hq, G, hd, bf(L.dOs),
                               bf(L.d_raw), ldq, da + 2 * hkv * hd, s);
-  // ---- attention, one KV head at a time
+  // ---- attention, the KV heads concurrently (each writes its own rows of
+  // dq_hat / dk_hat / dv)
+  e = e ? e : fork_streams(m, hkv, s);
   for (int h = 0; h < hkv && e == cudaSuccess; ++h) {
+    cudaStream_t hs = m->aux_streams[h];
     const __nv_bfloat16* qs = bf(L.qs) + h * head_q;
     const __nv_bfloat16* ks = bf(L.ks) + h * head_kv;
     const __nv_bfloat16* vs = bf(L.vs) + h * head_kv;
     const __nv_bfloat16* P = bf(L.P) + h * head_p;
     const __nv_bfloat16* dOs = bf(L.dOs) + h * head_q;
-    e = e ? e : gemm_f32(m, dOs, 0, vs, 0, f32(L.S), G * T, T, hd, s, Tp);        // dP = dO V^T
-    e = e ? e : launch_softmax_bwd_rows(P, f32(L.S), G * T, Tp, scale, bf(L.dS), s);
-    e = e ? e : gemm_f32(m, P, 1, dOs, 1, f32(L.dV), T, hd, G * T, s, 0, Tp);       // dV = P^T dO
-    e = e ? e : gemm_f32(m, bf(L.dS), 0, ks, 1, f32(L.dQ), G * T, hd, T, s, 0, Tp);  // dQ = dS K
-    e = e ? e : gemm_f32(m, bf(L.dS), 1, qs, 1, f32(L.dK), T, hd, G * T, s, 0, Tp);  // dK = dS^T Q
-    e = e ? e : launch_scatter_heads(f32(L.dQ), T, G, hd, hq, h * G, f32(L.dq_hat), s);
-    e = e ? e : launch_scatter_heads(f32(L.dK), T, 1, hd, hkv, h, f32(L.dk_hat), s);
-    e = e ? e : launch_scatter_heads(f32(L.dV), T, 1, hd, hkv, h, f32(L.dv), s);
+    float* dP = f32(L.S) + h * head_p;
+    __nv_bfloat16* dS = bf(L.dS) + h * head_p;
+    float* dV = f32(L.dV) + h * head_kv;
+    float* dQ = f32(L.dQ) + h * head_q;
+    float* dK = f32(L.dK) + h * head_kv;
+    e = e ? e : gemm_f32(m, dOs, 0, vs, 0, dP, G * T, T, hd, hs, Tp, 0, 0, kCausalTiles,
+                         T);                                                        // dP = dO V^T
+    e = e ? e : launch_softmax_bwd_rows(P, dP, G * T, T, Tp, window, scale, dS, hs);
+    e = e ? e : gemm_f32(m, P, 1, dOs, 1, dV, T, hd, G * T, hs, 0, Tp, 0, kCausalRowsK,
+                         T);                                                        // dV = P^T dO
+    e = e ? e : gemm_f32(m, dS, 0, ks, 1, dQ, G * T, hd, T, hs, 0, Tp, 0, kCausalKeysK,
+                         T);                                                        // dQ = dS K
+    e = e ? e : gemm_f32(m, dS, 1, qs, 1, dK, T, hd, G * T, hs, 0, Tp, 0, kCausalRowsK,
+                         T);                                                        // dK = dS^T Q
+    e = e ? e : launch_scatter_heads(dQ, T, G, hd, hq, h * G, f32(L.dq_hat), hs);
+    e = e ? e : launch_scatter_heads(dK, T, 1, hd, hkv, h, f32(L.dk_hat), hs);
+    e = e ? e : launch_scatter_heads(dV, T, 1, hd, hkv, h, f32(L.dv), hs);
   }
+  e = e ? e : join_streams(m, hkv, s);
   // ---- QK norm and RoPE, then the projection's dgrad and wgrad
   e = e ? e : launch_v_grad(f32(L.dv), T, hkv, hd, bf(L.d_raw), ldq, da + hkv * hd, s);
   e = e ? e : launch_qk_bwd(f32(L.raw), ldq, f32(L.dq_hat), f32(L.dk_hat), W.s_qk, rope, T, hq,

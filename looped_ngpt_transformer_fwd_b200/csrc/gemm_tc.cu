@@ -475,6 +475,22 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int m_tiles, int n_tiles,
   return c;
 }
 
+// Causal skipping (GemmParams.causal): the largest query position among
+// stacked rows [r0, r0 + rows) (T - 1 when they wrap into the next head).
+__device__ __forceinline__ int stack_tmax(int r0, int rows, int T) {
+  const int t0 = r0 % T;
+  return t0 + rows - 1 >= T ? T - 1 : t0 + rows - 1;
+}
+__device__ __forceinline__ bool tile_live(const GemmParams& p, int mt, int nt, int bn) {
+  return p.causal != kCausalTiles || nt * bn <= stack_tmax(mt * kBM, kBM, p.causal_T);
+}
+__device__ __forceinline__ int kb_limit(const GemmParams& p, int mt, int kb1) {
+  return p.causal == kCausalKeysK ? min(kb1, stack_tmax(mt * kBM, kBM, p.causal_T) / kBK + 1) : kb1;
+}
+__device__ __forceinline__ bool kb_live(const GemmParams& p, int mt, int kb) {
+  return p.causal != kCausalRowsK || stack_tmax(kb * kBK, kBK, p.causal_T) >= mt * kBM;
+}
+
 template <int BN, int HD, int EPI, int MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -543,9 +559,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
         const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
+        if (!tile_live(p, mt, nt, BN)) continue;   // the same decision in every role
         const int kb0 = ks * kb_per_split;
-        const int kb1 = min(kb_total, kb0 + kb_per_split);
+        const int kb1 = kb_limit(p, mt, min(kb_total, kb0 + kb_per_split));
         for (int kb = kb0; kb < kb1; ++kb) {
+          if (!kb_live(p, mt, kb)) continue;
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
@@ -611,10 +629,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       bool issued = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const int ks = tile_coord(t, m_tiles, n_tiles, p.raster_n).ks;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+        const int mt = tc.mt, ks = tc.ks;
+        if (!tile_live(p, mt, tc.nt, BN)) continue;
         const int kb0 = ks * kb_per_split;
-        const int kb1 = min(kb_total, kb0 + kb_per_split);
+        const int kb1 = kb_limit(p, mt, min(kb_total, kb0 + kb_per_split));
         const int acc = it % C::kAccBufs;
         const uint32_t aph = (it / C::kAccBufs) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) {
@@ -623,7 +643,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        bool first = true;                 // the tile's first live K block overwrites
         for (int kb = kb0; kb < kb1; ++kb) {
+          if (!kb_live(p, mt, kb)) continue;
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status)) {
             ok = false;
             break;
@@ -651,7 +673,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int kk = 0; kk < 4; ++kk)
               umma_nvf4(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4),
                         umma_idesc_nvf4(kBM, BN), sf_col + 4 * kk, sfb_col + kk * (BN / 32),
-                        (kb > kb0 || kk > 0) ? 1u : 0u);
+                        (!first || kk > 0) ? 1u : 0u);
           } else if constexpr (MX) {
             // scales to TMEM (this stage's own columns: the MMAs that read
             // them last time completed before the stage was refilled), then
@@ -666,15 +688,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int kk = 0; kk < 4; ++kk)
               umma_mxf8(d_tmem, a_desc + ((kk * 32) >> 4), b_desc + ((kk * 32) >> 4),
                         umma_idesc_mxf8(kBM, BN, kk), sf_col, sf_col + 4,
-                        (kb > kb0 || kk > 0) ? 1u : 0u);
+                        (!first || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               umma_bf16(d_tmem, a_desc + ((kk * a_step) >> 4), b_desc + ((kk * b_step) >> 4),
-                        idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        idesc, (!first || kk > 0) ? 1u : 0u);
             }
           }
           issued = true;
+          first = false;
           umma_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
@@ -683,6 +706,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
+        ++it;
       }
       if (!ok && issued) {
         umma_commit(drain);
@@ -695,9 +719,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* my_stage = out_stage + (warp - 2) * 2 * C::kOutBufBytes;
     uint32_t nbuf = 0;                 // staged boxes so far (buffer rotation)
     int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
       const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
+      if (!tile_live(p, mt, nt, BN)) continue;
       const int acc = it % C::kAccBufs;
       const uint32_t aph = (it / C::kAccBufs) & 1;
       // warp-uniform: the TMEM loads below are warp-collective
@@ -728,6 +753,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // one arrival per warp: many arrivals on one mbarrier are serialised
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      ++it;
     }
     // bulk stores read shared memory until they complete: finish before exit
     if (lane == 0 && nbuf > 0) bulk_wait_all();
@@ -953,6 +979,8 @@ cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   // share TMEM); MN-major operands are bf16 only
   if (p.mx && (!p.sfa || !p.sfb)) return cudaErrorInvalidValue;
   if (p.mx && (p.a_mn || p.b_mn)) return cudaErrorInvalidValue;
+  // causal skipping: bf16 and whole-K tiles only
+  if (p.causal && (p.mx || p.k_splits != 1 || p.causal_T <= 0)) return cudaErrorInvalidValue;
   switch (p.mx) {
     case kOperandsMxfp8: return dispatch_gemm<kOperandsMxfp8>(tmA, tmB, p, BN, head_dim, num_sms, s);
     case kOperandsNvfp4: return dispatch_gemm<kOperandsNvfp4>(tmA, tmB, p, BN, head_dim, num_sms, s);

@@ -58,6 +58,17 @@ struct GemmParams {
   // (b_mn) row-major, their tensor maps from make_tmap_bf16_mn; the MMAs read
   // them transposed (the backward's dgrad and wgrad products)
   int a_mn = 0, b_mn = 0;
+  // causal structure of the attention backward's products (bf16 only): rows
+  // r = g * causal_T + t stack the query heads of a KV head's group, keys are
+  // positions j; query t sees keys j <= t (kCausal* below)
+  int causal = 0, causal_T = 0;
+};
+
+enum {
+  kCausalNone = 0,
+  kCausalTiles = 1,   // C[r][j]: tiles whose keys all follow every query of the tile are skipped (never written)
+  kCausalKeysK = 2,   // K runs over keys: a tile's K loop ends after the last key its queries see
+  kCausalRowsK = 3    // K runs over stacked rows, output rows are keys: K blocks whose queries all precede the tile's keys are skipped
 };
 
 // MLP-sublayer backward pieces (backward.cu): the nGPT update's backward
@@ -79,8 +90,9 @@ cudaError_t launch_gather_heads(const __nv_bfloat16* src, int T, int src_heads, 
                                 int hd, __nv_bfloat16* dst, cudaStream_t s);
 cudaError_t launch_softmax_rows(const float* S, int rows, int T, int ld, int window, float scale,
                                 __nv_bfloat16* P, cudaStream_t s);
-cudaError_t launch_softmax_bwd_rows(const __nv_bfloat16* P, const float* dP, int rows, int ld,
-                                    float scale, __nv_bfloat16* dS, cudaStream_t s);
+cudaError_t launch_softmax_bwd_rows(const __nv_bfloat16* P, const float* dP, int rows, int T,
+                                    int ld, int window, float scale, __nv_bfloat16* dS,
+                                    cudaStream_t s);
 cudaError_t launch_gated_output(const float* Os, const float* gate, int T, int hq, int G, int hd,
                                 __nv_bfloat16* o, cudaStream_t s);
 cudaError_t launch_gate_bwd(const float* dout, const float* Os, const float* gate, int T, int hq,
