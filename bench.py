@@ -68,14 +68,14 @@ WORKLOADS = {
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
 # one ncu capture, valid only while the kernel source is unchanged since.
 PROFILED = {
-    "gateup": {"traffic": 138692864 + 54441216,
+    "gateup": {"traffic": 138715136 + 58497024,
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
-                          "6c28c8229b5b4f7261ab8f2c3bc8754ca72a8492")},
-    # decode attention: measured (read + write) / algorithmic bytes, applied to
-    # the step's total KV bytes
-    "attn": {"ratio": (1075908000 + 8675840) / 1073758208,
+                          "192005c0b8fe343c8273df3ce0b755a10f3a1243")},
+    # decode attention: measured (read + write) / algorithmic bytes of the
+    # full-layer launch, applied to the step's total KV bytes
+    "attn": {"ratio": (1075915520 + 5085440) / 1073758208,
              "source": ("looped_ngpt_transformer_fwd_b200/csrc/attn_decode_tma.cu",
-                        "364d8cd720bac77c12c3080afcf6ee162dea4681")},
+                        "ae876dbfaa034702e200369ffd5e61e734159c4b")},
 }
 
 
