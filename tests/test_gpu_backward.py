@@ -204,3 +204,51 @@ def test_last_loop_backward_matches_the_oracle(k):
     g, w = to_np(res["dx"]).ravel(), ref["dx"].ravel()
     assert np.linalg.norm(g - w) / np.linalg.norm(w) <= CHAIN_REL
     model.close()
+
+
+# ------------------------------------------------------------------ contracts
+
+def test_backward_is_deterministic():
+    """Two identical calls give bit-identical gradients: the dalpha and ds_qk
+    sums run in a fixed order, and the concurrent KV heads write disjoint
+    rows."""
+    cfg, prov, model = build("tiny", seed=71, d_model=768, n_q_heads=6, n_kv_heads=2, head_dim=128,
+                             d_ff=1024, window=128, softmax_scale=float(np.sqrt(128.0)))
+    _, h = inputs(cfg, 72, 300)
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    gt = torch.from_numpy((np.random.default_rng(73).standard_normal(h.shape) * 0.1)
+                          .astype(np.float32)).cuda()
+    a1 = model.attention_sublayer_backward(0, ht, gt)
+    a2 = model.attention_sublayer_backward(0, ht, gt)
+    m1 = model.mlp_sublayer_backward(1, ht, gt)
+    m2 = model.mlp_sublayer_backward(1, ht, gt)
+    torch.cuda.synchronize()
+    for k in a1:
+        assert torch.equal(a1[k], a2[k]), k
+    for k in m1:
+        assert torch.equal(m1[k], m2[k]), k
+    model.close()
+
+
+def test_backward_refuses_what_it_does_not_cover():
+    """Block-scaled weights have no backward (BAD_CONFIG), and a per-loop cache
+    with fewer loop slots than k is refused (K_EXCEEDS_KMAX)."""
+    from looped_ngpt_transformer_fwd_b200.binding import DoryError
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from oracle import weights_from_generator
+    from synthetic import load_config
+    cfg = load_config("tiny")
+    prov = weights_from_generator(cfg, 74, "random")
+    mx = DoryModel(cfg, prov, weight_format="mxfp8")
+    _, h = inputs(cfg, 75, 32)
+    ht = torch.from_numpy(h.astype(np.float32)).cuda()
+    with pytest.raises(DoryError, match="BAD_CONFIG"):
+        mx.mlp_sublayer_backward(1, ht, ht.clone())
+    with pytest.raises(DoryError, match="BAD_CONFIG"):
+        mx.attention_sublayer_backward(1, ht, ht.clone())
+    mx.close()
+    model = DoryModel(cfg, prov)
+    kv = model.kv_cache("per_loop", 1, 32, k_max=1)
+    with pytest.raises(DoryError, match="K_EXCEEDS_KMAX"):
+        model.last_loop_backward(kv, ht, ht.clone(), 2)
+    model.close()
