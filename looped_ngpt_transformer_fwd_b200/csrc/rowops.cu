@@ -75,10 +75,12 @@ __device__ __forceinline__ void quant_chunk(const RowUpdateParams& p, int r, int
 }
 
 // Three block reductions per row (||y||, ||h'||, ||h_new + e||), with y and h
-// held in registers between them.  A variant that derives all three norms from
-// one pass of seven per-row sums (one barrier) measured slower on B200: it
-// needs more live registers, which cost more occupancy than the barriers do.
-__global__ void row_update_kernel(const RowUpdateParams p) {
+// held in registers between them.  The kernel is bound by how many rows are in
+// flight per SM: variants that need more live registers (all three norms from
+// one pass of seven row sums, or two rows per CTA) measured slower on B200,
+// and capping the registers at 40 (six resident CTAs instead of four, a
+// 12-byte spill) measured 10 % faster than the uncapped 52.
+__global__ void __launch_bounds__(256, 6) row_update_kernel(const RowUpdateParams p) {
   __shared__ float red[32];
   const int r = blockIdx.x;
   // one CTA per row: these exits are uniform across the block
