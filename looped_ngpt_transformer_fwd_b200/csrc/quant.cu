@@ -87,7 +87,7 @@ constexpr int kQuantUnroll = 8;     // 128-value steps whose loads are in flight
 // row from cache.
 template <typename T>
 __global__ void __launch_bounds__(32 * kQuantWarps)
-    quant_mxfp8_kernel(const QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
+    quant_mxfp8_kernel(const __grid_constant__ QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
                        int normalize, float norm_eps, uint8_t* __restrict__ codes,
                        uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
@@ -173,7 +173,7 @@ constexpr int kNvUnroll = 4;   // 256-value steps whose loads are in flight toge
 // row; lanes 2b and 2b+1 share 16-block b (amax by one shuffle).
 template <typename T>
 __global__ void __launch_bounds__(32 * kQuantWarps)
-    quant_nvfp4_kernel(const QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
+    quant_nvfp4_kernel(const __grid_constant__ QuantSrc<T> src, int rows, int rows_pad, int K, int row_blocks,
                        int normalize, float norm_eps, const float* __restrict__ d_g, float g_host,
                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
