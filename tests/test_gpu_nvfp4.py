@@ -240,3 +240,41 @@ def test_nvfp4_tracks_the_bf16_model(tiny_nv):
     bf = Oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, "last_loop", k_max=2))
     nv = _nv_oracle(cfg, prov).forward(h, 0, 2, oracle_cache(cfg, "last_loop", k_max=2))
     assert np.abs(out - nv).max() < np.abs(out - bf).max()
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
+def test_mixed_k_decode_block_scaled(fmt):
+    """A decode step with its own loop count per sequence on block-scaled
+    weights: rows whose loops are done are skipped by the row kernel, so the
+    stream's codes come from the stand-alone quantiser; each row equals that
+    sequence decoded alone with its k by the oracle of the same format."""
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from oracle import weights_from_generator
+    from synthetic import load_config
+    _lib()
+    cfg = load_config("tiny")
+    prov = weights_from_generator(cfg, 33, "random")
+    model = DoryModel(cfg, prov, weight_format=fmt)
+    orc = Oracle(cfg, Q.dequantized_provider(prov, fmt),
+                 act_quant=Q.nvfp4_fake_quant if fmt == "nvfp4" else Q.mxfp8_fake_quant)
+    ks = [1, 3, 2]
+    k_hi = max(ks)
+    kv = model.kv_cache("last_loop", 3, 96, k_max=k_hi)
+    ocache = oracle_cache(cfg, "last_loop", k_max=k_hi)
+    lens = [9, 40, 3]
+    xs = [inputs(cfg, 80 + s, lens[s] + 1) for s in range(3)]
+    for s, L in enumerate(lens):
+        model.prefill(kv, xs[s][0][:L], ks[s], seq=s, pos0=0)
+        orc.forward(xs[s][1][:L], 0, ks[s], ocache, seq=s)
+    order = [1, 2, 0]
+    rows_t = torch.cat([xs[s][0][lens[s]:lens[s] + 1] for s in order])
+    d_seq = torch.tensor(order, dtype=torch.int32, device="cuda")
+    d_pos = torch.tensor([lens[s] for s in order], dtype=torch.int32, device="cuda")
+    d_k = torch.tensor([ks[s] for s in order], dtype=torch.int32, device="cuda")
+    out = to_np(model.decode_mixed(kv, rows_t, d_seq, d_pos, d_k, 95, k_hi))
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    for i, s in enumerate(order):
+        ref = orc.decode(xs[s][1][lens[s]:lens[s] + 1], [s], [lens[s]], ks[s], ocache)
+        assert_parity(out[i:i + 1], ref, tol_cos=NV_TOL_COS, what=f"{fmt} mixed-k seq {s} k={ks[s]}")
+    model.close()
