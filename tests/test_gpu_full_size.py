@@ -110,3 +110,39 @@ def test_4b_shape_stack_matches_oracle_at_every_row(mode):
         ref = orc.decode(h[p:p + 1], [0], [p], k, ocache)
         assert_parity(to_np(out), ref, what=f"4B-shape decode {p} {mode}")
     model.close()
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "nvfp4"])
+def test_4b_shape_block_scaled_stack_matches_oracle(fmt):
+    """The 4B block shapes (d_model 3072, 24 / 8 heads of 128, MLP 9216) with one
+    input, one recurrent and one output block, k = 2, MXFP8 or NVFP4 weights and
+    projection inputs, 300 tokens then two decode steps: every row against the
+    oracle of the same format (NVFP4 at its stack bar, cosine 0.998)."""
+    from looped_ngpt_transformer_fwd_b200 import build as libbuild
+    from looped_ngpt_transformer_fwd_b200.model import DoryModel
+    from oracle import Oracle, weights_from_generator
+    from oracle import quant as Q
+    from synthetic import load_config
+    libbuild.build()
+    cfg = load_config("dory4b", n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1, full_period=2)
+    prov = weights_from_generator(cfg, 12, "random")
+    model = DoryModel(cfg, prov, weight_format=fmt)
+    orc = Oracle(cfg, Q.dequantized_provider(prov, fmt),
+                 act_quant=Q.nvfp4_fake_quant if fmt == "nvfp4" else Q.mxfp8_fake_quant)
+    tol_cos = 0.998 if fmt == "nvfp4" else 0.999
+    k = 2
+    x, h = inputs(cfg, 44, 302)
+    kv = model.kv_cache("last_loop", 1, 400, k_max=k)
+    ocache = oracle_cache(cfg, "last_loop", k_max=k)
+    out = model.prefill(kv, x[:300], k)
+    torch.cuda.synchronize()
+    assert model.device_status() == 0
+    assert_parity(to_np(out), orc.forward(h[:300], 0, k, ocache), tol_cos=tol_cos,
+                  what=f"4B-shape {fmt} prefill")
+    for p in (300, 301):
+        d = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pp = torch.tensor([p], dtype=torch.int32, device="cuda")
+        out = model.decode(kv, x[p:p + 1], d, pp, 399, k)
+        ref = orc.decode(h[p:p + 1], [0], [p], k, ocache)
+        assert_parity(to_np(out), ref, tol_cos=tol_cos, what=f"4B-shape {fmt} decode {p}")
+    model.close()
