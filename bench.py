@@ -71,6 +71,10 @@ PROFILED = {
     "gateup": {"traffic": 138715136 + 58497024,
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
                           "192005c0b8fe343c8273df3ce0b755a10f3a1243")},
+    # NVFP4 weights and activations: a different kernel instance, its own capture
+    "gateup:nvfp4": {"traffic": 38998528 + 28373504,
+                     "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
+                                "192005c0b8fe343c8273df3ce0b755a10f3a1243")},
     # decode attention: measured (read + write) / algorithmic bytes of the
     # full-layer launch, applied to the step's total KV bytes
     "attn": {"ratio": (1075915520 + 5085440) / 1073758208,
@@ -79,9 +83,11 @@ PROFILED = {
 }
 
 
-def profiled_traffic(kernel, work=None):
+def profiled_traffic(kernel, work=None, fmt=None):
+    """DRAM bytes of one launch from a committed ncu capture, or None when the
+    kernel's source changed since (or no capture of this weight format exists)."""
     import hashlib
-    ent = PROFILED.get(kernel)
+    ent = PROFILED.get(kernel if fmt in (None, "bf16") else f"{kernel}:{fmt}")
     if not ent:
         return None
     path, sha = ent["source"]
@@ -591,7 +597,7 @@ def roofline(res, wl, peaks, peak_src):
             # fp8 / fp4 contraction: the bf16 figure times the nominal ratio of the peaks
             peak, key = LOWP_RATIO[fmt] * peak, f"bf16_tflops_sustained x {LOWP_RATIO[fmt]:g} ({fmt})"
         per_launch = dom_work if wl["kind"] != "prefill_chunked" else dom_work / max(dom_n, 1)
-        traffic = profiled_traffic(dom_name)
+        traffic = profiled_traffic(dom_name, fmt=fmt)
     else:
         achieved = dom_work / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
         peak = peaks["hbm_gbs"]

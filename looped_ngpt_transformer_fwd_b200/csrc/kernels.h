@@ -252,6 +252,7 @@ struct RowUpdateParams {
   uint8_t* q_scales = nullptr;
   int q_row_blocks = 0;
   float q_g = 0.f;
+  float q_r6 = 0.f;   // 1 / (6 q_g) in fp32: set by launch_row_update
 };
 cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s);
 

@@ -142,6 +142,151 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   }
 }
 
+// ------------------------------------------------------------------ one CTA per row
+//
+// The row kernel of both formats: a CTA quantises one (padded) row, its
+// threads holding the whole row in registers as loaded (chunks of 8 values:
+// chunk c in thread c % blockDim, slot c / blockDim), so the normalising
+// variant reads the row once and sums its squares with one block reduction.
+// Many small CTAs (one per row) keep the last wave short; the warp-per-row
+// kernels remain for rows too long to hold.
+
+template <typename T> struct Chunk8;
+template <> struct Chunk8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    u = *reinterpret_cast<const uint4*>(p);
+  }
+  __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+  __device__ __forceinline__ void get(float (&v)[8]) const {
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+  }
+};
+template <> struct Chunk8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = reinterpret_cast<const float4*>(p)[0];
+    b = reinterpret_cast<const float4*>(p)[1];
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void get(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// chunks of 8 a thread holds: 36 registers of bf16 or 32 of fp32
+template <typename T> constexpr int kRowQuantChunks = sizeof(T) == 2 ? 9 : 4;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+template <int FMT, typename T>
+__global__ void __launch_bounds__(1024)
+    quant_rows_kernel(const __grid_constant__ QuantSrc<T> src, int rows, int K, int row_blocks,
+                      int normalize, float norm_eps, const float* __restrict__ d_g, float g_host,
+                      uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int NC = kRowQuantChunks<T>;
+  __shared__ float red[32];
+  const int r = blockIdx.x;                  // one CTA per row: exits are uniform
+  const int nch = K / 8, t = threadIdx.x, nt = blockDim.x;
+  const T* row = r < rows ? source_row(src, r, K) : nullptr;
+  Chunk8<T> x[NC];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < NC; ++j) {
+    const int c = t + j * nt;
+    if (row && c < nch) x[j].load(row + static_cast<size_t>(c) * 8);
+    else x[j].zero();
+  }
+  float inv = 1.f;
+  if (normalize && row) {                     // uniform
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      float v[8];
+      x[j].get(v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
+    }
+    inv = rsqrtf(fmaxf(block_sum(ss, red), norm_eps));
+  }
+  const int rb = r / 128, rr = r % 128;
+  if constexpr (FMT == kOperandsNvfp4) {
+    const float g = d_g ? *d_g : g_host;
+    const float r6 = nv_scale_factor(g);
+    uint8_t* srow = scales + static_cast<size_t>(rb) * 2048 + (rr % 32) * 16 + (rr / 32) * 4;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int c = t + j * nt;
+      if (j * nt >= nch) break;               // uniform
+      float v[8];
+      x[j].get(v);
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] *= inv;
+        amax = fmaxf(amax, fabsf(v[i]));
+      }
+      // lanes 2b, 2b+1 hold 16-block c / 2 (every lane shuffles: chunks past
+      // the row are zeros and store nothing)
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      if (c >= nch) continue;
+      const NvScale sc = nv_block_scale_fast(amax, g, r6);
+      if ((c & 1) == 0)
+        srow[static_cast<size_t>(c / 32) * row_blocks * 2048 + ((c % 32) / 8) * 512 +
+             ((c % 32) / 2) % 4] = static_cast<uint8_t>(row ? sc.code : 0x38u);
+      if (!row) continue;
+      const uint32_t word = nv_codes8(v, sc, g);
+      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * (K / 2) + c * 4) = word;
+    }
+  } else {
+    uint8_t* srow = scales + static_cast<size_t>(rb) * 512 + (rr % 32) * 16 + (rr / 32) * 4;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int c = t + j * nt;
+      if (j * nt >= nch) break;               // uniform
+      float v[8];
+      x[j].get(v);
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      // lanes 4q..4q+3 hold 32-block c / 4
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      if (c >= nch) continue;
+      // the normalised values' amax (a uniform positive scale commutes with max)
+      const int sexp = mx_block_exponent(amax * inv);
+      const int q32 = c / 4;
+      if ((c & 3) == 0)
+        srow[static_cast<size_t>(q32 / 4) * row_blocks * 512 + (q32 % 4)] =
+            static_cast<uint8_t>(row ? sexp + 127 : 127);
+      if (!row) continue;
+      const float f = inv * mx_pow2_neg(sexp);
+      *reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * K + c * 8) =
+          make_uint2(mx_codes4(v[0], v[1], v[2], v[3], f), mx_codes4(v[4], v[5], v[6], v[7], f));
+    }
+  }
+}
+
+// Threads per row for the CTA-per-row kernel (0: the row is too long to hold):
+// 128 when the rows fill the GPU, else up to one chunk per thread.
+template <typename T>
+int row_quant_threads(int rows_pad, int K) {
+  const int nch = K / 8;
+  int t = rows_pad >= 1024 ? 128 : 1024;
+  t = std::min(t, (nch + 31) / 32 * 32);
+  const int need = (nch + kRowQuantChunks<T> - 1) / kRowQuantChunks<T>;
+  t = std::max(t, (need + 31) / 32 * 32);
+  return t <= 1024 ? t : 0;
+}
+
 template <typename T>
 cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K, int normalize,
                          float norm_eps, uint8_t* codes, uint8_t* scales, cudaStream_t s) {
@@ -149,6 +294,11 @@ cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K,
   if (K % 128 != 0 || (row_align != 128 && row_align != 256)) return cudaErrorInvalidValue;
   const int rows_pad = (rows + row_align - 1) / row_align * row_align;
   const int row_blocks = rows_pad / 128;
+  if (const int nt = row_quant_threads<T>(rows_pad, K)) {
+    quant_rows_kernel<kOperandsMxfp8, T><<<rows_pad, nt, 0, s>>>(
+        src, rows, K, row_blocks, normalize, norm_eps, nullptr, 0.f, codes, scales);
+    return cudaGetLastError();
+  }
   quant_mxfp8_kernel<T><<<(rows_pad + kQuantWarps - 1) / kQuantWarps, 32 * kQuantWarps, 0, s>>>(
       src, rows, rows_pad, K, row_blocks, normalize, norm_eps, codes, scales);
   return cudaGetLastError();
@@ -181,6 +331,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   if (r >= rows_pad) return;                      // warp-uniform
   const T* row = r < rows ? source_row(src, r, K) : nullptr;
   const float g = d_g ? *d_g : g_host;
+  const float r6 = nv_scale_factor(g);
   float inv = 1.f;
   if (normalize && row) {
     float ss = 0.f;
@@ -223,18 +374,13 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
       amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      const NvScale sc = nv_block_scale(amax, g);
+      const NvScale sc = nv_block_scale_fast(amax, g, r6);
       const int b = (k0 % 256) / 16;              // 16-block within the 256
       if ((lane & 1) == 0)
         srow[static_cast<size_t>(k0 / 256) * row_blocks * 2048 + (b / 4) * 512 + (b % 4)] =
             static_cast<uint8_t>(row ? sc.code : 0x38u);
       if (!row) continue;
-      uint32_t word = 0;
-      if (sc.s > 0.f) {
-        const NvThresholds th = nv_thresholds(sc.s);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) word |= nv_code(v[u][i], th, g) << (4 * i);
-      }
+      const uint32_t word = nv_codes8(v[u], sc, g);
       *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(r) * (K / 2) + k0 / 2) = word;
     }
   }
@@ -249,6 +395,11 @@ cudaError_t launch_quant_nv(const QuantSrc<T>& src, int rows, int row_align, int
   if (!d_g && !(g > 0.f)) return cudaErrorInvalidValue;
   const int rows_pad = (rows + row_align - 1) / row_align * row_align;
   const int row_blocks = rows_pad / 128;
+  if (const int nt = row_quant_threads<T>(rows_pad, K)) {
+    quant_rows_kernel<kOperandsNvfp4, T><<<rows_pad, nt, 0, s>>>(
+        src, rows, K, row_blocks, normalize, norm_eps, d_g, g, codes, scales);
+    return cudaGetLastError();
+  }
   quant_nvfp4_kernel<T><<<(rows_pad + kQuantWarps - 1) / kQuantWarps, 32 * kQuantWarps, 0, s>>>(
       src, rows, rows_pad, K, row_blocks, normalize, norm_eps, d_g, g, codes, scales);
   return cudaGetLastError();

@@ -45,13 +45,8 @@ __device__ __forceinline__ void quant_chunk(const RowUpdateParams& p, int r, int
   if (p.q_fmt == kOperandsNvfp4) {
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    const NvScale sc = nv_block_scale(amax, p.q_g);
-    uint32_t word = 0;
-    if (sc.s > 0.f) {
-      const NvThresholds th = nv_thresholds(sc.s);
-      word = nv_code(v.x, th, p.q_g) | (nv_code(v.y, th, p.q_g) << 4) |
-             (nv_code(v.z, th, p.q_g) << 8) | (nv_code(v.w, th, p.q_g) << 12);
-    }
+    const NvScale sc = nv_block_scale_fast(amax, p.q_g, p.q_r6);
+    const uint32_t word = nv_codes4(v.x, v.y, v.z, v.w, sc, p.q_g);
     reinterpret_cast<uint16_t*>(p.q_codes + static_cast<size_t>(r) * (p.d / 2))[c] =
         static_cast<uint16_t>(word);
     if ((c & 3) == 0) {
@@ -322,7 +317,9 @@ cudaError_t launch_row_update(const RowUpdateParams& p, cudaStream_t s) {
   threads = ((threads + 31) / 32) * 32;
   if (threads > 1024) return cudaErrorInvalidValue;
   if (threads < 32) threads = 32;
-  row_update_kernel<<<p.rows, threads, 0, s>>>(p);
+  RowUpdateParams q = p;
+  if (q.q_fmt == kOperandsNvfp4) q.q_r6 = 1.f / (6.f * q.q_g);
+  row_update_kernel<<<p.rows, threads, 0, s>>>(q);
   return cudaGetLastError();
 }
 

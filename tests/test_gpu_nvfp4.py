@@ -119,6 +119,52 @@ def test_quantiser_exact_ties_round_to_even():
     assert np.array_equal(_unchunk(scales.cpu().numpy(), 8, 256)[0], want_s)
 
 
+def test_quantiser_block_scale_ties_saturation_and_subnormals():
+    """Blocks whose quotient amax / (6 g) lies exactly on an E4M3 midpoint
+    (normal and subnormal, one carrying into the next binade), on the
+    saturation point 448 and above it, and just beside such points; each
+    block also holds the E2M1 midpoints of its own decoded scale.  The
+    kernels decide most values from a bracketed fp32 quotient and hand these
+    ones to the exact comparisons: codes and scales equal the oracle's."""
+    from looped_ngpt_transformer_fwd_b200.model import quant_nvfp4
+    _lib()
+    g = 2.0 ** -12
+    qs = [1.0625, 1.9375, 248.0, 432.0, 448.0, 456.0, 464.0, 1024.0,
+          2.0 ** -10, 1.5 * 2.0 ** -9, 15 * 2.0 ** -10, 2.5 * 2.0 ** -9,
+          1.0, 17.0, 0.3125, 96.0]
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    rng = np.random.default_rng(11)
+    rows, K = 24, 512
+    x = np.zeros((rows, K))
+    for r in range(rows):
+        for b in range(K // 16):
+            q = qs[(b + 5 * r) % len(qs)] * (1.0 + 2.0 ** -7 * ((r // 8) - 1))   # on, below, above
+            amax = 6.0 * g * q
+            x[r, 16 * b:16 * b + 16] = rng.uniform(-amax, amax, 16)
+            x[r, 16 * b + rng.integers(16)] = amax * rng.choice([-1.0, 1.0])
+    x = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).float().numpy().astype(np.float64)
+    # E2M1 midpoints of each block's scale (those not above the block's amax)
+    _, s_codes, _ = Q.nvfp4_quantize(x, np.float32(g))
+    s = Q.decode(s_codes, Q.E4M3)
+    for r in range(rows):
+        for b in range(K // 16):
+            blk = x[r, 16 * b:16 * b + 16]
+            amax = np.abs(blk).max()
+            j = int(np.argmax(np.abs(blk)))
+            free = [i for i in range(16) if i != j]
+            for i, m in zip(free, mids):
+                v = m * s[r, b] * g * (-1.0) ** i
+                if 0.0 < abs(v) <= amax:
+                    blk[i] = v
+    xt = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda()
+    assert np.array_equal(xt.float().cpu().numpy(), x)
+    codes, scales, _ = quant_nvfp4(xt, g=g)
+    torch.cuda.synchronize()
+    want_c, want_s, _ = Q.nvfp4_quantize(x, np.float32(g))
+    assert np.array_equal(_unchunk(scales.cpu().numpy(), rows, K)[0], want_s)
+    assert np.array_equal(_unpack(codes.cpu().numpy()), want_c)
+
+
 @pytest.mark.parametrize("M,N,K,splits", [(300, 512, 512, 1), (64, 384, 3072, 4), (1, 128, 256, 1),
                                           (129, 1286, 256, 1), (1000, 768, 1024, 2),
                                           (700, 1024, 3072, 1), (64, 2048, 1536, 3)])
