@@ -287,6 +287,8 @@ def run_ours(args, wl, rank, world, device_index, model=None, prov=None, steps=N
                           weight_format=wl.get("fmt", "bf16"))
         if args.fused_update:
             model.fused_update(True)
+        if args.stream_k:
+            model.stream_k(True)
     k, mode = wl["k"], wl["mode"]
     stream = torch.cuda.current_stream()
     res = {}
@@ -649,6 +651,8 @@ def main():
                     help="profiling aid: decode batch override (same per-sequence work)")
     ap.add_argument("--fused-update", action="store_true",
                     help="profiling aid: prefill projections with the nGPT update in their epilogue")
+    ap.add_argument("--stream-k", action="store_true",
+                    help="profiling aid: stream-K tails in the prefill output / down projections")
     ap.add_argument("--extra-workloads", default="auto",
                     help="comma-separated workloads reported under 'workloads' in the same line; "
                          "'auto' = the k = 1 prefill and the three decode workloads when the "

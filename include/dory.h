@@ -147,7 +147,8 @@ typedef struct dory_model dory_model;
 typedef struct dory_kv dory_kv;
 
 /* Bytes of the device buffer dory_create packs the weights into
- * (weights in the kernels' layout plus a small device status area). */
+ * (weights in the kernels' layout, a small device status area and about
+ * 21 MB of stream-K partial slots for the prefill projections). */
 DORY_API size_t dory_weight_bytes(const dory_config* cfg);
 
 /* Validate `cfg`, check that the current device is sm_100, and pack the
@@ -329,6 +330,28 @@ DORY_API int dory_mlp_sublayer(dory_model* m, int layer, int n_rows, float* h,
  * all row-major device buffers, K a multiple of 64, N a multiple of 128. */
 DORY_API int dory_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
 
+/* The same GEMM with a stream-K tail, the schedule of the prefill output and
+ * down projections.  A persistent grid of one CTA per SM runs whole
+ * 128 x BN tiles (BN = 256 when N is a multiple of 256, else 128); when the
+ * tiles leave a partial last wave, the last one-and-a-fraction waves are cut
+ * into contiguous runs of k blocks of equal length, one per CTA, so every
+ * CTA does the same work.  A tile split between two CTAs is finished by the
+ * one holding its first k blocks, which adds the other's fp32 partial
+ * (passed through `ws`) in a fixed order: results are identical from call to
+ * call, and equal to dory_gemm_bf16's up to fp32 rounding.  `ws` (device,
+ * dory_gemm_bf16_streamk_workspace_bytes(N), 256-byte aligned) must be
+ * zero-filled before its first use; it keeps a launch counter between
+ * calls, so calls sharing one `ws` must not overlap on the GPU.  Every CTA of
+ * the grid must be resident at once: kernels running concurrently on other
+ * streams can delay the partials.  A CTA that waits more than 2 s for one
+ * gives up, stores its tile without it and sets the last 32-bit word of
+ * `ws` nonzero (the output is then wrong; zero the word to clear it).
+ * Grids of more than 160 CTAs run without the tail.  Same argument rules as
+ * dory_gemm_bf16. */
+DORY_API size_t dory_gemm_bf16_streamk_workspace_bytes(int N);
+DORY_API int dory_gemm_bf16_streamk(const void* A, const void* B, float* C, int M, int N, int K,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* The same GEMM with operands read transposed (MN-major): A is stored row-major
  * as [M][K] (a_mn = 0) or [K][M] (a_mn = 1), B as [N][K] (b_mn = 0) or [K][N]
  * (b_mn = 1); C[M,N] = A B^T in fp32.  Any K (rounded up inside, the tail read
@@ -477,6 +500,15 @@ DORY_API int dory_debug_mask_probe(dory_model* m, int layer, int32_t* d_probe, i
  * DORY_ERR_BAD_CONFIG when d_model has no fused kernel (not a multiple of 384,
  * 256 or 128 with at most 8 CTAs per row); such models always run unfused. */
 DORY_API int dory_debug_fused_update(dory_model* m, int enable);
+
+/* Stream-K tails in the prefill output and down projections (the schedule of
+ * dory_gemm_bf16_streamk over the model's own slots).  enable = 1 makes later
+ * prefill calls use them; the default (enable = 0) runs whole tiles only,
+ * measured faster on B200 at the 4B shape under its power cap: with every SM
+ * busy through the last wave the clock drops more than the idle share of that
+ * wave costs.  Returns DORY_ERR_BAD_CONFIG where the device has more SMs than
+ * the model buffer has slots (the tails then stay off). */
+DORY_API int dory_debug_stream_k(dory_model* m, int enable);
 
 /* Attention kernels launched by the most recent call, by kind:
  * counts[0] tensor-core (tcgen05) prefill attention, counts[1] mma.sync

@@ -41,7 +41,8 @@ EXPORTS = (
     "dory_last_loop_grad_layout", "dory_last_loop_backward_workspace_bytes",
     "dory_last_loop_backward",
     "dory_vocab_bytes", "dory_vocab_create", "dory_embed", "dory_lm_head", "dory_sample",
-    "dory_vocab_free",
+    "dory_vocab_free", "dory_gemm_bf16_streamk_workspace_bytes", "dory_gemm_bf16_streamk",
+    "dory_debug_stream_k",
 )
 
 WEIGHT_FORMATS = {"bf16": 0, "mxfp8": 1, "nvfp4": 2}
@@ -112,6 +113,9 @@ def lib():
             "dory_attention_sublayer": (I, [P, P, I, I, I, I, I, P, P, SZ, P]),
             "dory_mlp_sublayer": (I, [P, I, I, P, P, SZ, P]),
             "dory_gemm_bf16": (I, [P, P, P, I, I, I, P]),
+            "dory_gemm_bf16_streamk_workspace_bytes": (SZ, [I]),
+            "dory_gemm_bf16_streamk": (I, [P, P, P, I, I, I, P, SZ, P]),
+            "dory_debug_stream_k": (I, [P, I]),
             "dory_profile_enable": (I, [P, I]),
             "dory_profile_read": (I, [P, I, P, P]),
             "dory_mlp_sublayer_noalloc": (I, [P, I, I, P, P]),
@@ -265,6 +269,21 @@ def noalloc_max_rows(d_model, d_ff):
 
 def dory_gemm_bf16(A, B, C, M, N, K, stream):
     return check(lib().dory_gemm_bf16(A, B, C, M, N, K, stream), "dory_gemm_bf16")
+
+
+def dory_gemm_bf16_streamk_workspace_bytes(N):
+    return lib().dory_gemm_bf16_streamk_workspace_bytes(N)
+
+
+def dory_gemm_bf16_streamk(A, B, C, M, N, K, ws, ws_bytes, stream):
+    return check(lib().dory_gemm_bf16_streamk(A, B, C, M, N, K, ws, ws_bytes, stream),
+                 "dory_gemm_bf16_streamk")
+
+
+def dory_debug_stream_k(model, enable):
+    """Stream-K tails of the prefill projections on or off (default); returns
+    the status (DORY_ERR_BAD_CONFIG when the device has more SMs than slots)."""
+    return lib().dory_debug_stream_k(model, 1 if enable else 0)
 
 
 def dory_profile_enable(model, enable):

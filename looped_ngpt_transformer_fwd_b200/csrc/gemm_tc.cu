@@ -201,15 +201,30 @@ __device__ __forceinline__ void store_f32_chunk(float* dst, const float (&v)[32]
   }
 }
 
+// Accumulators plus the tail's partial (when there is one).
+__device__ __forceinline__ void add_partial(float (&v)[32], const float* part, int c) {
+  if (part) {
+    // from L2 (another SM wrote it)
+    const float4* s4 = reinterpret_cast<const float4*>(part + c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = __ldcg(s4 + i);
+      v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
+    }
+  }
+}
+
+// `part`: this lane's row of a stream-K tail partial to add, or nullptr.
 template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t taddr, int row, int nt,
-                                              int ks) {
+                                              int ks, const float* part) {
   float* out = p.out_f32 + static_cast<size_t>(ks) * p.split_stride;
   const bool row_ok = row < p.M;
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld32(taddr + c, v);
+    add_partial(v, part, c);
     apply_alpha<kAlpha>(v, p.alpha);
     const int col = nt * BN + c;
     if (row_ok && col < p.N)
@@ -225,11 +240,13 @@ __device__ __forceinline__ void epi_store_f32(const GemmParams& p, uint32_t tadd
 template <int BN, bool kAlpha>
 __device__ __forceinline__ void epi_store_f32_tma(const GemmParams& p, const CUtensorMap* tmC,
                                                   uint32_t taddr, uint8_t* stage, int lane,
-                                                  int row0, int nt, int ks, uint32_t& nbuf) {
+                                                  int row0, int nt, int ks, uint32_t& nbuf,
+                                                  const float* part) {
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld32(taddr + c, v);
+    add_partial(v, part, c);
     apply_alpha<kAlpha>(v, p.alpha);
     const int col = nt * BN + c;
     if (col >= p.N) continue;                   // warp-uniform
@@ -491,6 +508,124 @@ __device__ __forceinline__ bool kb_live(const GemmParams& p, int mt, int kb) {
   return p.causal != kCausalRowsK || stack_tmax(kb * kBK, kBK, p.causal_T) >= mt * kBM;
 }
 
+// ------------------------------------------------------------ work units
+// A CTA's work: with the stream-K tail (GemmParams.sk), first its range of
+// the tile-major k blocks of tiles [0, sk_tiles), then whole tiles
+// sk_tiles + c, + grid, ...; otherwise whole tiles c, c + grid, ...  Every
+// role walks the same sequence.
+enum { kUnitWhole = 0, kUnitTail = 1, kUnitHead = 2 };
+struct Unit {
+  int t;          // tile index (tile_coord)
+  int kb0, kb1;   // stream-K: k blocks [kb0, kb1) of the tile; -1: the tile's K split
+  int role;       // kUnitTail: partial to this CTA's slot; kUnitHead: adds the next CTA's slot
+};
+struct Sched {
+  int pos, pos_end;       // stream-K k blocks still to do
+  int t, t_end, t_step;   // whole tiles still to do
+};
+__device__ __forceinline__ Sched sched_init(const GemmParams& p, int total, int kb_total) {
+  Sched s;
+  const int G = gridDim.x, c = blockIdx.x;
+  s.pos = s.pos_end = 0;
+  s.t = c;
+  s.t_step = G;
+  s.t_end = total;
+  if (p.sk) {
+    // launcher: total > G and total % G != 0, so sk_tiles is in (G, 2G) and
+    // every range is longer than a tile: a tile meets at most two ranges
+    const int sk_tiles = total - (total / G - 1) * G;
+    const long long n = static_cast<long long>(sk_tiles) * kb_total;
+    s.pos = static_cast<int>(n * c / G);
+    s.pos_end = static_cast<int>(n * (c + 1) / G);
+    s.t = sk_tiles + c;
+  }
+  return s;
+}
+__device__ __forceinline__ bool sched_next(Sched& s, int kb_total, Unit& u) {
+  if (s.pos < s.pos_end) {
+    u.t = s.pos / kb_total;
+    u.kb0 = s.pos % kb_total;
+    u.kb1 = min(kb_total, u.kb0 + (s.pos_end - s.pos));
+    u.role = u.kb0 > 0 ? kUnitTail : (u.kb1 < kb_total ? kUnitHead : kUnitWhole);
+    s.pos += u.kb1 - u.kb0;
+    return true;
+  }
+  if (s.t < s.t_end) {
+    u.t = s.t;
+    u.kb0 = u.kb1 = -1;
+    u.role = kUnitWhole;
+    s.t += s.t_step;
+    return true;
+  }
+  return false;
+}
+
+// k blocks [kb0, kb1) of a unit: its stream-K range, or its K split's
+// (clipped by causal key skipping)
+__device__ __forceinline__ void unit_kblocks(const GemmParams& p, const Unit& u, int mt, int ks,
+                                             int kb_per_split, int kb_total, int& kb0, int& kb1) {
+  if (u.kb0 >= 0) {
+    kb0 = u.kb0;
+    kb1 = u.kb1;
+    return;
+  }
+  kb0 = ks * kb_per_split;
+  kb1 = kb_limit(p, mt, min(kb_total, kb0 + kb_per_split));
+}
+
+// sk_sync words: [0] launch counter, [1] CTAs done, [2 + 4 c + w] slot c's
+// rows 32w.. published (the counter value + 1 of the launch that wrote them)
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Tail segment: this warp's 32 rows of the partial accumulator to slot
+// `slot` (fp32 [128][BN], one row per lane), then publish them.
+template <int BN>
+__device__ __forceinline__ void epi_sk_tail(const GemmParams& p, uint32_t taddr, int quad,
+                                            int lane, int slot, uint32_t tag) {
+  float* dst = p.sk_ws + (static_cast<size_t>(slot) * kBM + quad * 32 + lane) * BN;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float v[32];
+    tmem_ld32(taddr + c, v);
+    float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) st_release_gpu(p.sk_sync + 2 + 4 * slot + quad, tag);
+}
+
+// Head segment: wait (bounded) until slot `slot` holds this warp's rows of
+// the tile's tail; returns this lane's row of it, or nullptr when the wait
+// gave up (timeout reported; the tile is then stored without it).
+template <int BN>
+__device__ __forceinline__ const float* sk_head_wait(const GemmParams& p, int quad, int lane,
+                                                     int slot, uint32_t tag,
+                                                     volatile int* abort_flag) {
+  const uint32_t* f = p.sk_sync + 2 + 4 * slot + quad;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (__all_sync(0xFFFFFFFFu, ld_acquire_gpu(f) == tag)) break;
+    if ((it & 15u) == 15u) {
+      const bool give_up = (abort_flag && *abort_flag) || globaltimer_ns() - t0 > kWaitLimitNs;
+      if (__any_sync(0xFFFFFFFFu, give_up)) {
+        if (lane == 0) report_status(p.status, kStatusTimeout);
+        return nullptr;
+      }
+    }
+  }
+  return p.sk_ws + (static_cast<size_t>(slot) * kBM + quad * 32 + lane) * BN;
+}
+
+
 template <int BN, int HD, int EPI, int MX>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -556,12 +691,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+      Sched sch = sched_init(p, total, kb_total);
+      Unit u;
+      while (ok && sched_next(sch, kb_total, u)) {
+        const TileCoord tc = tile_coord(u.t, m_tiles, n_tiles, p.raster_n);
         const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
         if (!tile_live(p, mt, nt, BN)) continue;   // the same decision in every role
-        const int kb0 = ks * kb_per_split;
-        const int kb1 = kb_limit(p, mt, min(kb_total, kb0 + kb_per_split));
+        int kb0, kb1;
+        unit_kblocks(p, u, mt, ks, kb_per_split, kb_total, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!kb_live(p, mt, kb)) continue;
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
@@ -629,12 +766,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       bool issued = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+      Sched sch = sched_init(p, total, kb_total);
+      Unit u;
+      while (ok && sched_next(sch, kb_total, u)) {
+        const TileCoord tc = tile_coord(u.t, m_tiles, n_tiles, p.raster_n);
         const int mt = tc.mt, ks = tc.ks;
         if (!tile_live(p, mt, tc.nt, BN)) continue;
-        const int kb0 = ks * kb_per_split;
-        const int kb1 = kb_limit(p, mt, min(kb_total, kb0 + kb_per_split));
+        int kb0, kb1;
+        unit_kblocks(p, u, mt, ks, kb_per_split, kb_total, kb0, kb1);
         const int acc = it % C::kAccBufs;
         const uint32_t aph = (it / C::kAccBufs) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) {
@@ -719,8 +858,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* my_stage = out_stage + (warp - 2) * 2 * C::kOutBufBytes;
     uint32_t nbuf = 0;                 // staged boxes so far (buffer rotation)
     int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const TileCoord tc = tile_coord(t, m_tiles, n_tiles, p.raster_n);
+    // stream-K tag of this launch (the counter only moves after every CTA
+    // of the launch has finished)
+    const uint32_t tag = p.sk ? *reinterpret_cast<volatile uint32_t*>(p.sk_sync) + 1u : 0u;
+    Sched sch = sched_init(p, total, kb_total);
+    Unit u;
+    while (sched_next(sch, kb_total, u)) {
+      const TileCoord tc = tile_coord(u.t, m_tiles, n_tiles, p.raster_n);
       const int mt = tc.mt, nt = tc.nt, ks = tc.ks;
       if (!tile_live(p, mt, nt, BN)) continue;
       const int acc = it % C::kAccBufs;
@@ -732,11 +876,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       constexpr bool kAlpha = C::kNv;
       if constexpr (EPI == kEpiStoreF32) {
-        if (p.c_tma)
-          epi_store_f32_tma<BN, kAlpha>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32,
-                                        nt, ks, nbuf);
-        else
-          epi_store_f32<BN, kAlpha>(p, taddr, row, nt, ks);
+        if (u.role == kUnitTail) {
+          epi_sk_tail<BN>(p, taddr, quad, lane, blockIdx.x, tag);
+        } else {
+          // a head adds the tail that opens the next CTA's range
+          const float* part = u.role == kUnitHead
+                                  ? sk_head_wait<BN>(p, quad, lane, blockIdx.x + 1, tag, abort_flag)
+                                  : nullptr;
+          if (p.c_tma)
+            epi_store_f32_tma<BN, kAlpha>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32,
+                                          nt, ks, nbuf, part);
+          else
+            epi_store_f32<BN, kAlpha>(p, taddr, row, nt, ks, part);
+        }
       } else if constexpr (EPI == kEpiSwiGLU) {
         if (p.c_tma)
           epi_swiglu_tma<BN, kAlpha>(p, &om.m[0], taddr, my_stage, lane, mt * kBM + quad * 32, nt,
@@ -765,6 +917,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if (p.sk && threadIdx.x == 0) {
+    // the last CTA of the launch resets the done count and moves the counter
+    __threadfence();
+    if (atomicAdd(p.sk_sync + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sk_sync + 1, 0u);
+      __threadfence();
+      atomicAdd(p.sk_sync, 1u);
+    }
   }
 }
 
@@ -844,6 +1005,12 @@ cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
   const int grid = total < num_sms ? total : num_sms;
   if (grid <= 0) return cudaSuccess;
   GemmParams q = p;
+  // stream-K only where a partial last wave exists and its slots fit
+  if (q.sk) {
+    const bool usable = EPI == kEpiStoreF32 && q.k_splits == 1 && q.causal == kCausalNone &&
+                        q.sk_ws && q.sk_sync && total > grid && total % grid != 0;
+    if (!usable) q.sk = 0;
+  }
   OutMaps om;
   memset(&om, 0, sizeof(om));
   q.c_tma = 0;
@@ -860,6 +1027,11 @@ cudaError_t launch_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const Ge
 }
 
 }  // namespace
+
+size_t gemm_sk_workspace_bytes(int grid, int BN) {
+  const size_t slots = static_cast<size_t>(grid) * kBM * BN * 4;
+  return (slots + 255) / 256 * 256 + (3 + 4 * static_cast<size_t>(grid)) * 4;
+}
 
 bool make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint64_t ld, uint32_t box_rows) {

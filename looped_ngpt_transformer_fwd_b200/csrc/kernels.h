@@ -62,7 +62,26 @@ struct GemmParams {
   // r = g * causal_T + t stack the query heads of a KV head's group, keys are
   // positions j; query t sees keys j <= t (kCausal* below)
   int causal = 0, causal_T = 0;
+  // stream-K tail (kEpiStoreF32, whole K, no causal skipping): when the
+  // tiles leave a partial last wave, the last one-and-a-fraction waves of
+  // tiles are cut into contiguous k-block ranges of equal length, one per
+  // CTA.  A tile then has at most two segments: the CTA holding its tail
+  // writes an fp32 partial to its slot of sk_ws ([grid][128][BN]) and
+  // publishes it through sk_sync; the CTA holding its head adds it and
+  // stores the tile.  sk_sync ([2 + 4 * grid] words, zero before the first
+  // use) keeps a launch counter, so it must not serve two launches at once.
+  // Every CTA of the grid must be resident at once (one per SM): only for
+  // launches that share the GPU with no concurrent kernel.  The launcher
+  // clears sk where the tiles divide evenly into waves.
+  int sk = 0;
+  float* sk_ws = nullptr;
+  uint32_t* sk_sync = nullptr;
 };
+
+// Bytes of a stream-K workspace for `grid` CTAs and BN-column tiles: the
+// partial slots, then (256-byte aligned) the synchronisation words and a
+// spare status word at the end.
+size_t gemm_sk_workspace_bytes(int grid, int BN);
 
 enum {
   kCausalNone = 0,

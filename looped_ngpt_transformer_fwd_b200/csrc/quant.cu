@@ -20,10 +20,11 @@
 // NVFP4 (same page, the NVFP4 release): blocks of 16 consecutive values along
 // K share an E4M3 scale s = E4M3(amax_block / (6 g)) under a per-tensor fp32
 // scale g; each value becomes the E2M1 code nearest to x / (s g) (ties to
-// even, saturating at 6).  Both decisions are exact (blockscale.cuh): the
-// scale from a quotient rounded once to float64, the element by the exact sign
-// of |x| minus each E2M1 midpoint times s g, so the codes are those of the
-// exact rational rounding.  Codes are packed two per byte
+// even, saturating at 6).  Both decisions are those of the exact rational
+// rounding (blockscale.cuh): taken from the hardware conversions of a tight
+// fp32 bracket of the quotient, and where the bracket straddles a decision
+// point from a float64 quotient (scale) or the exact sign of |x| minus each
+// E2M1 midpoint times s g (element).  Codes are packed two per byte
 // (element 2i in the low nibble); scales go in 2048-byte chunks, one per (128
 // rows, 256 K): chunk (kc, rb) at ((kc * row_blocks) + rb) * 2048, and inside
 // it the scale of row r = rb*128 + 32*j + i and 16-block b (0..15) at byte

@@ -304,6 +304,10 @@ class DoryModel:
         """True when the prefill projections apply the nGPT update in their epilogue."""
         return B.dory_debug_fused_update(self.handle, enable) == 0 and enable
 
+    def stream_k(self, enable=True):
+        """True when the prefill output / down projections use stream-K tails."""
+        return B.dory_debug_stream_k(self.handle, enable) == 0 and enable
+
     def attention_paths(self):
         return B.dory_debug_attention_paths(self.handle)
 
@@ -388,6 +392,21 @@ def gemm_bf16_mn(A, Bm, M, N, K, a_mn, b_mn, stream=None):
     C = torch.empty(M, N, dtype=torch.float32, device=A.device)
     B.dory_gemm_bf16_mn(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, int(a_mn), int(b_mn), _stream(stream))
     return C
+
+
+def gemm_bf16_streamk(A, Bm, ws=None, stream=None):
+    """C = A @ Bm^T through the stream-K schedule; `ws` (uint8, device, zeroed
+    before its first use) may be passed to keep its launch counter across
+    calls.  Returns (C, ws)."""
+    M, K = A.shape
+    N = Bm.shape[0]
+    if ws is None:
+        ws = torch.zeros(B.dory_gemm_bf16_streamk_workspace_bytes(N), dtype=torch.uint8,
+                         device=A.device)
+    C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    B.dory_gemm_bf16_streamk(_ptr(A), _ptr(Bm), _ptr(C), M, N, K, _ptr(ws), ws.numel(),
+                             _stream(stream))
+    return C, ws
 
 
 def gemm_bf16(A, Bm, stream=None):
