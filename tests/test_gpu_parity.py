@@ -33,6 +33,24 @@ def test_gemm_matches_fp64(M, N, K):
 
 
 # ------------------------------------------------------------------ sublayers
+def test_d_model_4096_mlp_sublayer_matches_oracle():
+    """d_model 4096 (32 heads of 128, the widest the library takes): the row
+    update's wide forms -- the pipelined kernel for 200 rows and the
+    512-thread one-row kernel for 100 -- against the oracle."""
+    cfg, prov, model = build("tiny", seed=3, d_model=4096, n_q_heads=32, n_kv_heads=8,
+                             head_dim=128, d_ff=512, n_in_blocks=1, n_rec_blocks=1,
+                             n_out_blocks=1, window=64)
+    for n in (200, 100):
+        _, h = inputs(cfg, 21 + n, n)
+        ht = torch.from_numpy(h.astype(np.float32)).cuda()
+        model.mlp_sublayer(0, ht)
+        torch.cuda.synchronize()
+        assert model.device_status() == 0
+        ref = oracle(cfg, prov).mlp_sublayer(0, h)
+        assert_parity(to_np(ht), ref, tol_abs=5e-3, tol_cos=0.9999, what=f"mlp d4096 rows {n}")
+    model.close()
+
+
 def test_mlp_sublayer_matches_oracle(tiny):
     cfg, prov, model = tiny
     _, h = inputs(cfg, 11, 200)
