@@ -82,11 +82,14 @@ def test_streamk_gemm_rejects_a_short_or_misaligned_workspace():
                                       None) == -7   # DORY_ERR_MISALIGNED
 
 
-def test_4b_shape_prefill_streamk_on_and_off_agree():
+@pytest.mark.parametrize("fmt", ["bf16", "mxfp8", "nvfp4"])
+def test_4b_shape_prefill_streamk_on_and_off_agree(fmt):
     """4B block shapes (1 + 1 + 1 blocks, k = 2) on 4096 tokens: the output and
     down projections have 384 tiles, so their last wave runs as stream-K
-    tails.  With the tails on and off the stack agrees to fp32 rounding
-    (propagated through six nGPT updates), and two calls with the tails on are
+    tails (block-scaled too: the partial is added before the tensor-scale
+    product).  With the tails on and off the stack agrees to fp32 rounding
+    (propagated through six nGPT updates; for the block-scaled formats also
+    through the requantised stream), and two calls with the tails on are
     bit-identical."""
     from looped_ngpt_transformer_fwd_b200.model import DoryModel
     from oracle import weights_from_generator
@@ -94,7 +97,7 @@ def test_4b_shape_prefill_streamk_on_and_off_agree():
     _lib()
     cfg = load_config("dory4b", n_in_blocks=1, n_rec_blocks=1, n_out_blocks=1, full_period=2)
     prov = weights_from_generator(cfg, 13, "random")
-    model = DoryModel(cfg, prov)
+    model = DoryModel(cfg, prov, weight_format=fmt)
     T, k = 4096, 2
     x, _ = inputs(cfg, 47, T)
     outs = []
@@ -106,9 +109,14 @@ def test_4b_shape_prefill_streamk_on_and_off_agree():
         assert model.device_status() == 0
         del kv
     assert torch.equal(outs[0], outs[1])
-    diff = (outs[0] - outs[2]).abs().max().item()
-    assert diff <= 2e-3, diff          # bf16 outputs: a rounding flip is 2^-9 of a unit row value
     cos = torch.nn.functional.cosine_similarity(outs[0], outs[2], dim=1).min().item()
-    assert cos >= 0.99999, cos
+    if fmt == "bf16":
+        diff = (outs[0] - outs[2]).abs().max().item()
+        assert diff <= 2e-3, diff      # bf16 outputs: a rounding flip is 2^-9 of a unit row value
+        assert cos >= 0.99999, cos
+    else:
+        # an fp32 rounding difference can flip an element's code in the next
+        # projection's quantised input (a whole grid step of E4M3 / E2M1)
+        assert cos >= 0.9995, cos
     model.close()
     torch.cuda.empty_cache()
