@@ -68,13 +68,13 @@ WORKLOADS = {
 # DRAM traffic (read + write bytes per launch) of the dominant kernels from
 # one ncu capture, valid only while the kernel source is unchanged since.
 PROFILED = {
-    "gateup": {"traffic": 138501888 + 54807296,
+    "gateup": {"traffic": 138575360 + 55643648,
                "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
-                          "53a43e62a3f2014d62313285d8b5bf5193a778fc")},
+                          "13f70dca9836ca126719cb6bc46bdcb3bb4102ce")},
     # NVFP4 weights and activations: a different kernel instance, its own capture
-    "gateup:nvfp4": {"traffic": 39005184 + 24676096,
+    "gateup:nvfp4": {"traffic": 39038464 + 25788672,
                      "source": ("looped_ngpt_transformer_fwd_b200/csrc/gemm_tc.cu",
-                                "53a43e62a3f2014d62313285d8b5bf5193a778fc")},
+                                "13f70dca9836ca126719cb6bc46bdcb3bb4102ce")},
     # decode attention: measured (read + write) / algorithmic bytes of the
     # full-layer launch, applied to the step's total KV bytes
     "attn": {"ratio": (1075915520 + 5085440) / 1073758208,

@@ -691,6 +691,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
+      const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
       Sched sch = sched_init(p, total, kb_total);
       Unit u;
       while (ok && sched_next(sch, kb_total, u)) {
@@ -712,6 +713,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < kBM / 64; ++j)
               tma_load_2d(a_dst + j * 8192, &tmA, &full[stage], mt * kBM + 64 * j, kb * kBK);
+          } else if (p.l2_hint) {
+            tma_load_2d_hint(a_dst, &tmA, &full[stage], kb * C::kKCoord, mt * kBM, pol_a);
           } else {
             tma_load_2d(a_dst, &tmA, &full[stage], kb * C::kKCoord, mt * kBM);
           }
@@ -720,6 +723,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 0; j < BN / 64; ++j)
               tma_load_2d(a_dst + C::kABytes + j * 8192, &tmB, &full[stage], nt * BN + 64 * j,
                           kb * kBK);
+          } else if (p.l2_hint) {
+            tma_load_2d_hint(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKCoord, nt * BN, pol_b);
           } else {
             tma_load_2d(a_dst + C::kABytes, &tmB, &full[stage], kb * C::kKCoord, nt * BN);
           }

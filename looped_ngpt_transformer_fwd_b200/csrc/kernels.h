@@ -54,6 +54,10 @@ struct GemmParams {
   // order of the persistent tile loop: 0 = M tiles fastest, 1 = N tiles
   // fastest (keeps a wave's A panels and all of B in L2 when A is larger)
   int raster_n = 0;
+  // L2 hints on the K-major operand loads: A evict-first (each A panel is
+  // read by the N tiles of one wave, then never again) and B evict-last (B is
+  // read again by every wave), so B stays in L2 while A streams past
+  int l2_hint = 0;
   // bf16 operands stored MN-major: A as [K][M] (a_mn) and / or B as [K][N]
   // (b_mn) row-major, their tensor maps from make_tmap_bf16_mn; the MMAs read
   // them transposed (the backward's dgrad and wgrad products)
