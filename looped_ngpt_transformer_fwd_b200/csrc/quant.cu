@@ -288,6 +288,116 @@ int row_quant_threads(int rows_pad, int K) {
   return t <= 1024 ? t : 0;
 }
 
+// ------------------------------------------------------------------ NVFP4: a block per thread
+// The NVFP4 quantiser with one CTA per (padded) row and each thread owning
+// whole 16-value blocks (block b = thread + j * blockDim, two adjacent 16-byte
+// loads): the block scale is formed once per block and no shuffles are
+// needed.  A normalising row folds 1 / ||row|| into the bracket factor of
+// the element decisions: x * fl(fl(inv * (1 / (s g))) * (1 -+ 2^-20)) carries
+// one rounding more than without the norm, still inside the 2^-20 margin;
+// the block scale uses fl(amax * inv), which is the largest fl(x * inv)
+// (rounding is monotone), and the exact fallback takes the normalised
+// values fl(x * inv) themselves: the codes are those of quant_rows_kernel.
+template <typename T> constexpr int kNvBlocks = sizeof(T) == 2 ? 5 : 3;   // blocks per thread
+constexpr int kNvBlockThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kNvBlockThreads)
+    quant_nv_blocks_kernel(const __grid_constant__ QuantSrc<T> src, int rows, int K,
+                           int row_blocks, int normalize, float norm_eps,
+                           const float* __restrict__ d_g, float g_host,
+                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int NB = kNvBlocks<T>;
+  __shared__ float red[32];
+  const int r = blockIdx.x;                  // one CTA per row: exits are uniform
+  const int nb = K / 16, t = threadIdx.x, nt = blockDim.x;
+  const T* row = r < rows ? source_row(src, r, K) : nullptr;
+  Chunk8<T> x[NB][2];
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    const int b = t + j * nt;
+    if (row && b < nb) {
+      x[j][0].load(row + static_cast<size_t>(b) * 16);
+      x[j][1].load(row + static_cast<size_t>(b) * 16 + 8);
+    } else {
+      x[j][0].zero();
+      x[j][1].zero();
+    }
+  }
+  float inv = 1.f;
+  if (normalize && row) {                     // uniform
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v[8];
+        x[j][h].get(v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+    inv = rsqrtf(fmaxf(block_sum(ss, red), norm_eps));
+  }
+  const float g = d_g ? *d_g : g_host;
+  const float r6 = nv_scale_factor(g);
+  const int rb = r / 128, rr = r % 128;
+  uint8_t* srow = scales + static_cast<size_t>(rb) * 2048 + (rr % 32) * 16 + (rr / 32) * 4;
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    const int b = t + j * nt;
+    if (b >= nb) break;
+    float v[8], w[8];
+    x[j][0].get(v);
+    x[j][1].get(w);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i]), fabsf(w[i])));
+    const NvScale sc = nv_block_scale_fast(amax * inv, g, r6);
+    srow[static_cast<size_t>(b / 16) * row_blocks * 2048 + ((b % 16) / 4) * 512 + (b % 4)] =
+        static_cast<uint8_t>(row ? sc.code : 0x38u);
+    if (!row) continue;
+    uint32_t c0 = 0u, c1 = 0u;
+    if (sc.s > 0.f) {
+      float rs;
+      bool done = false;
+      if (nv_fast_scale(sc, g, rs)) {
+        const float f = inv * rs;
+        const float flo = f * kNvBracketLo, fhi = f * kNvBracketHi;
+        const uint32_t l0 = e2m1_codes8(v, flo), l1 = e2m1_codes8(w, flo);
+        if (l0 == e2m1_codes8(v, fhi) && l1 == e2m1_codes8(w, fhi)) {
+          c0 = l0;
+          c1 = l1;
+          done = true;
+        }
+      }
+      if (!done) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[i] *= inv;
+          w[i] *= inv;
+        }
+        c0 = nv_codes4_exact(v[0], v[1], v[2], v[3], sc.s, g) |
+             (nv_codes4_exact(v[4], v[5], v[6], v[7], sc.s, g) << 16);
+        c1 = nv_codes4_exact(w[0], w[1], w[2], w[3], sc.s, g) |
+             (nv_codes4_exact(w[4], w[5], w[6], w[7], sc.s, g) << 16);
+      }
+    }
+    *reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * (K / 2) + static_cast<size_t>(b) * 8) =
+        make_uint2(c0, c1);
+  }
+}
+
+// Threads per row for quant_nv_blocks_kernel (0: the row has too many blocks)
+template <typename T>
+int nv_block_threads(int rows_pad, int K) {
+  const int nb = K / 16;
+  int t = rows_pad >= 1024 ? 128 : kNvBlockThreads;
+  t = std::min(t, (nb + 31) / 32 * 32);
+  const int need = (nb + kNvBlocks<T> - 1) / kNvBlocks<T>;
+  t = std::max(t, (need + 31) / 32 * 32);
+  return t <= kNvBlockThreads ? t : 0;
+}
+
 template <typename T>
 cudaError_t launch_quant(const QuantSrc<T>& src, int rows, int row_align, int K, int normalize,
                          float norm_eps, uint8_t* codes, uint8_t* scales, cudaStream_t s) {
@@ -396,6 +506,11 @@ cudaError_t launch_quant_nv(const QuantSrc<T>& src, int rows, int row_align, int
   if (!d_g && !(g > 0.f)) return cudaErrorInvalidValue;
   const int rows_pad = (rows + row_align - 1) / row_align * row_align;
   const int row_blocks = rows_pad / 128;
+  if (const int nt = nv_block_threads<T>(rows_pad, K)) {
+    quant_nv_blocks_kernel<T><<<rows_pad, nt, 0, s>>>(src, rows, K, row_blocks, normalize,
+                                                      norm_eps, d_g, g, codes, scales);
+    return cudaGetLastError();
+  }
   if (const int nt = row_quant_threads<T>(rows_pad, K)) {
     quant_rows_kernel<kOperandsNvfp4, T><<<rows_pad, nt, 0, s>>>(
         src, rows, K, row_blocks, normalize, norm_eps, d_g, g, codes, scales);
