@@ -70,7 +70,10 @@ def _unchunk(scales, rows, K):
     return s[:rows], s[rows:]
 
 
-@pytest.mark.parametrize("M,K", [(300, 512), (1, 256), (128, 3072), (77, 9216)])
+# K up to 20480 (bf16): the block-per-thread kernel; (3, 24576): the
+# CTA-per-row kernel with lane pairs per block; (3, 81920): the warp-per-row one
+@pytest.mark.parametrize("M,K", [(300, 512), (1, 256), (128, 3072), (77, 9216), (3, 24576),
+                                 (3, 81920)])
 def test_quantiser_is_bit_exact_with_the_input_scale(M, K):
     from looped_ngpt_transformer_fwd_b200.model import quant_nvfp4
     _lib()
