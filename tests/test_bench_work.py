@@ -113,3 +113,31 @@ def test_profiled_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, mo
     src.write_text("// version 2\n")
     assert bench.profiled_traffic("k") is None
     assert bench.profiled_traffic("r", work=10) is None
+
+
+def test_profiled_traffic_is_kept_per_weight_format(tmp_path, monkeypatch):
+    """A capture of the bf16 kernel never stands in for the block-scaled one:
+    the lookup is keyed by format, bf16 (or no format) using the plain key."""
+    import hashlib
+    src = tmp_path / "kernel.cu"
+    src.write_text("// v\n")
+    sha = hashlib.sha1(src.read_bytes()).hexdigest()
+    monkeypatch.setattr(bench, "PROFILED", {
+        "k": {"traffic": 100, "source": (str(src), sha)},
+        "k:nvfp4": {"traffic": 40, "source": (str(src), sha)},
+    })
+    assert bench.profiled_traffic("k") == 100
+    assert bench.profiled_traffic("k", fmt="bf16") == 100
+    assert bench.profiled_traffic("k", fmt="nvfp4") == 40
+    assert bench.profiled_traffic("k", fmt="mxfp8") is None
+
+
+def test_committed_traffic_captures_match_the_current_sources():
+    """Every committed capture names the kernel source it was taken on; the
+    ones the bench reports must still match it (else the bench prints null)."""
+    import hashlib
+    import os
+    for name, ent in bench.PROFILED.items():
+        path, sha = ent["source"]
+        with open(os.path.join(bench.ROOT, path), "rb") as f:
+            assert hashlib.sha1(f.read()).hexdigest() == sha, name
