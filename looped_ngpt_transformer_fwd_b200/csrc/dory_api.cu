@@ -561,6 +561,12 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     pp.rows = c.n; pp.n_q_heads = m->hq; pp.n_kv_heads = m->hkv; pp.hd = m->hd;
     pp.s_qk = W.s_qk; pp.rope = rope; pp.norm_eps = m->cfg.norm_eps;
     pp.q_out = c.w.q; pp.k_out = c.w.kf; pp.v_out = c.w.vf; pp.gate_out = c.w.gate;
+    // this step's keys and values go to the cache here (no separate commit)
+    pp.commit = 1;
+    pp.kv = kv_view(c.kv, b, loop);
+    pp.d_seq = c.dseq; pp.d_pos = c.dpos;
+    pp.row_k = W.recurrent ? c.dk : nullptr; pp.loop = loop;
+    pp.status = m->status;
     {
       Launch L(m, c.s, DORY_KK_QKVG);
       DORY_TRY(launch_qkvg_post(pp, c.s));
@@ -593,11 +599,6 @@ cudaError_t attention_sublayer(CallCtx& c, int b, int loop, float* h, __nv_bfloa
     DORY_TRY(launch_probe_init(probe, size_t(c.n) * m->hq, c.s));
   }
   if (c.decode) {
-    {
-      Launch L(m, c.s, DORY_KK_KVCOMMIT);
-      DORY_TRY(launch_kv_commit(view, c.w.kf, c.w.vf, c.n, 0, 0, 0, c.dseq, c.dpos, m->status, c.s,
-                                W.recurrent ? c.dk : nullptr, loop));
-    }
     DecodeAttnParams a;
     a.q = c.w.q; a.gate = c.w.gate; a.out = c.w.o; a.kv = view;
     a.d_seq = c.dseq; a.d_pos = c.dpos;

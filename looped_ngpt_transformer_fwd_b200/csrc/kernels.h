@@ -220,6 +220,15 @@ cudaError_t launch_rope_table(const double* inv_freq, int hd, int rows, int pos0
 // K-split QKVG post-processing (decode): sum the split partial products
 // [splits][rows][n_qkvg], then the same per-head RoPE / L2 norm / s_qk / gate
 // steps as the fused kEpiQKVG epilogue.
+struct KvLayerView {
+  __nv_bfloat16* k_base = nullptr;
+  __nv_bfloat16* v_base = nullptr;
+  size_t seq_stride = 0;   // elements
+  int cap = 0;             // slots per (seq, head)
+  int n_kv = 0, hd = 0;
+  int max_seqs = 0, max_ctx = 0;
+};
+
 struct QkvgPostParams {
   const float* part = nullptr;
   int splits = 1;
@@ -231,6 +240,17 @@ struct QkvgPostParams {
   float norm_eps = 1e-20f;
   __nv_bfloat16 *q_out = nullptr, *k_out = nullptr, *v_out = nullptr;
   float* gate_out = nullptr;
+  // commit = 1: also write each row's k and v into its cache slot (decode:
+  // row r of sequence d_seq[r] at position d_pos[r], slot pos % cap), as a
+  // separate kv_commit would: rows with row_k[r] < loop skipped, positions
+  // or sequences out of range reported (kStatusBounds) and skipped
+  int commit = 0;
+  KvLayerView kv;
+  const int32_t* d_seq = nullptr;
+  const int32_t* d_pos = nullptr;
+  const int32_t* row_k = nullptr;
+  int loop = 0;
+  uint32_t* status = nullptr;
 };
 cudaError_t launch_qkvg_post(const QkvgPostParams& p, cudaStream_t s);
 
@@ -288,14 +308,6 @@ cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, c
 // ----------------------------------------------------------------- KV cache
 // Where one layer's cache lives: sequence s, KV head h, slot t:
 //   K at k_base + s*seq_stride + (h*cap + t)*hd, V at v_base + same (elements)
-struct KvLayerView {
-  __nv_bfloat16* k_base = nullptr;
-  __nv_bfloat16* v_base = nullptr;
-  size_t seq_stride = 0;   // elements
-  int cap = 0;             // slots per (seq, head)
-  int n_kv = 0, hd = 0;
-  int max_seqs = 0, max_ctx = 0;
-};
 
 // Copy fresh K/V rows [rows, Hkv, hd] into cache slots.  Row r goes to
 // sequence seq (or d_seq[r]) at position pos0 + r (or d_pos[r]); rows below

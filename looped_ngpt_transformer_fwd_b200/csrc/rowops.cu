@@ -465,6 +465,19 @@ __global__ void qkvg_post_kernel(const QkvgPostParams p) {
     dst = p.v_out + (static_cast<size_t>(r) * p.n_kv_heads + (g - p.n_q_heads - p.n_kv_heads)) * hd;
   dst[i] = __float2bfloat16_rn(a);
   dst[i + half] = __float2bfloat16_rn(b);
+  if (p.commit && g >= p.n_q_heads && !(p.row_k && p.loop > p.row_k[r])) {
+    // this row's k or v head straight into its cache slot
+    const int sq = p.d_seq[r], pos = p.d_pos[r];
+    if (sq < 0 || sq >= p.kv.max_seqs || pos < 0 || pos >= p.kv.max_ctx) {
+      if (i == 0) report_status(p.status, kStatusBounds);
+    } else {
+      const int head = is_v ? g - p.n_q_heads - p.n_kv_heads : g - p.n_q_heads;
+      __nv_bfloat16* cache = (is_v ? p.kv.v_base : p.kv.k_base) + sq * p.kv.seq_stride +
+                             (static_cast<size_t>(head) * p.kv.cap + pos % p.kv.cap) * hd;
+      cache[i] = __float2bfloat16_rn(a);
+      cache[i + half] = __float2bfloat16_rn(b);
+    }
+  }
 }
 
 __global__ void swiglu_post_kernel(const float* __restrict__ part, int splits, size_t split_stride,
