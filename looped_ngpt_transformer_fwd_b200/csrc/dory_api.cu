@@ -760,7 +760,8 @@ cudaError_t mlp_sublayer(CallCtx& c, int b, float* h, __nv_bfloat16* hb, bool sa
   gd.out_f32 = c.w.y; gd.ld_out = m->d; gd.split_stride = size_t(c.n) * m->d;
   gd.status = m->status;
   // the activations (rows x d_ff) outweigh W_down (d x d_ff) once rows > d:
-  // N tiles fastest, and W_down kept in L2 across the waves
+  // N tiles fastest, and W_down's loads marked evict-last in L2 (every wave
+  // reads all of it again; the hint trims the re-reads a little)
   gd.raster_n = c.n > m->d ? 1 : 0;
   gd.l2_hint = gd.raster_n;
   streamk_tail(c, gd);
